@@ -1,0 +1,32 @@
+"""Plain CPU oracle for the fused low-bit weight dequantize + matmul.
+
+TEST INFRASTRUCTURE ONLY. Nothing in the product package imports, calls or
+links anything here; only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may use it.
+
+What it computes, and where each step comes from:
+
+* ``oracle.int4``   -- group-wise INT4 quantisation (symmetric ``(q-8)*s`` and
+  asymmetric ``(q-zp)*s`` with an int8 zero point), the canonical two-nibbles-
+  per-byte packing (low nibble = even k) and the exact FP32 dequantisation.
+  Sources: "Low Bit Metal Kernels" (INT4 dequant + matmul listing) and
+  "Low Bit ARM kernels" (group-wise scale section).
+* ``oracle.lut3``   -- the 3-bit LUT format: a 3-bit index into an 8-entry E4M3
+  codebook shared by a tile of 8 output channels x 64 K, scaled by one UE8M0
+  exponent per tile; its canonical index bit stream and its exact decode.
+  Source: vLLM PR 62759 write-up (format section; tile and memory budget).
+* ``oracle.matmul`` -- Y = X . W accumulated in FP64, the error scale
+  S = |X| . |W|, and the acceptance test |y - y_ref| <= 4e-3*S + ulp16(|y_ref|).
+
+Everything is plain numpy in FP64 (FP32 where the pages fix a quantity that
+decides an integer code, so that both sides take that decision in the same
+precision). The oracle shares no code with the CUDA path.
+
+Parity status: every function here is pinned by ``tests/test_oracle.py``
+(hand examples in ``tests/golden/``, exact rational brute force, library
+decoders, nearest-level characterisation of the quantiser). Quantisation
+*quality* (MSE, task accuracy) is not modelled: parity unpinned for that,
+and it is out of scope.
+"""
+
+from . import int4, lut3, matmul  # noqa: F401

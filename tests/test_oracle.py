@@ -1,0 +1,327 @@
+"""Pins for the CPU oracle: each test ties it to something other than itself.
+
+Sources of the pins: the hand-derived fixtures under tests/golden (each names
+the page passage it follows), exact rational arithmetic, library decoders
+(ml_dtypes, torch), Python's own IEEE half packing, and a brute-force
+nearest-level characterisation of the quantiser.
+"""
+
+import math
+import struct
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import int4, lut3, matmul
+
+
+# ----------------------------------------------------------------------------- INT4 fixtures
+
+def test_sym_4x4_golden(golden):
+    g = golden("int4_sym_4x4.json")
+    W = np.array(g["W"], dtype=np.float32)
+    q, s = int4.quantize_sym(W, g["group"])
+    assert q.tolist() == g["q"]
+    assert s.astype(np.float64).tolist() == g["scale"]
+    packed = int4.pack_nibbles(q)
+    assert packed.tolist() == g["packed"]
+    assert [[int(h, 16) for h in row] for row in g["packed_hex"]] == g["packed"]
+    deq = int4.dequant(q, s, g["group"])
+    assert deq.tolist() == g["dequant"]
+    Y = matmul.matmul_f64(np.array(g["X"]), deq)
+    assert Y.tolist() == g["Y"]
+
+
+def test_asym_4x2_golden(golden):
+    g = golden("int4_asym_4x2.json")
+    W = np.array(g["W"], dtype=np.float32)
+    q, s, zp = int4.quantize_asym(W, g["group"])
+    assert q.tolist() == g["q"]
+    assert s.astype(np.float64).tolist() == g["scale"]
+    assert zp.tolist() == g["zp"]
+    assert int4.pack_nibbles(q).tolist() == g["packed"]
+    assert [[int(h, 16) for h in row] for row in g["packed_hex"]] == g["packed"]
+    assert int4.dequant(q, s, g["group"], zp).tolist() == g["dequant"]
+
+
+def test_metal_listing_byte_example():
+    """The INT4 listing: low nibble 15 -> (15-8)*s = 7s; high nibble 9 -> (9-8)*s = s,
+    and the low nibble belongs to the even k."""
+    packed = np.array([[0x9F]], dtype=np.uint8)
+    q = int4.unpack_nibbles(packed)
+    assert q[:, 0].tolist() == [15, 9]
+    s = np.array([[0.375]], dtype=np.float16)
+    assert int4.dequant(q, s, 2)[:, 0].tolist() == [7 * 0.375, 0.375]
+
+
+def test_low_nibble_is_even_k():
+    q = np.zeros((4, 1), np.uint8)
+    q[0, 0] = 1
+    q[3, 0] = 2
+    assert int4.pack_nibbles(q)[:, 0].tolist() == [0x01, 0x20]
+
+
+def test_pack_roundtrip_random():
+    rng = np.random.default_rng(7)
+    q = rng.integers(0, 16, size=(64, 24), dtype=np.uint8)
+    assert np.array_equal(int4.unpack_nibbles(int4.pack_nibbles(q)), q)
+    b = rng.integers(0, 256, size=(32, 24), dtype=np.uint8)
+    assert np.array_equal(int4.pack_nibbles(int4.unpack_nibbles(b)), b)
+
+
+# ----------------------------------------------------------------------------- quantiser
+
+def _half_via_struct(x):
+    """Python's own IEEE binary16 packing (round to nearest even)."""
+    return struct.unpack("<e", struct.pack("<e", x))[0]
+
+
+def _f32_div(a, b):
+    """Correctly rounded FP32 quotient via FP64 (53 >= 2*24+2 bits makes this exact)."""
+    return float(np.float32(float(a) / float(b)))
+
+
+@pytest.mark.parametrize("group", [32, 64, 128])
+def test_sym_scale_is_fp16_of_fp32_quotient(group):
+    rng = np.random.default_rng(group)
+    W = (rng.standard_normal((4 * group, 16)) * 0.02).astype(np.float32)
+    _, s = int4.quantize_sym(W, group)
+    for gi in range(4):
+        for n in range(16):
+            amax = max(abs(float(v)) for v in W[gi * group:(gi + 1) * group, n])
+            assert float(s[gi, n]) == _half_via_struct(_f32_div(amax, 7.0))
+
+
+def test_asym_scale_is_fp16_of_fp32_quotient():
+    rng = np.random.default_rng(11)
+    W = (rng.standard_normal((64, 16)) * 0.02).astype(np.float32)
+    _, s, _ = int4.quantize_asym(W, 32)
+    for gi in range(2):
+        for n in range(16):
+            col = W[gi * 32:(gi + 1) * 32, n]
+            span = float(np.float32(float(col.max()) - float(col.min())))
+            assert float(s[gi, n]) == _half_via_struct(_f32_div(span, 15.0))
+
+
+def _not_a_tie(v):
+    return abs(v - math.floor(v) - 0.5) > 1e-4
+
+
+@pytest.mark.parametrize("group", [32, 128])
+def test_sym_codes_are_nearest_levels(group):
+    """Independent characterisation: each code is the level (c-8)*s, c in 0..15,
+    nearest to w (ties excluded), i.e. no other code would reconstruct w better."""
+    rng = np.random.default_rng(100 + group)
+    W = (rng.standard_normal((2 * group, 40)) * 0.02).astype(np.float32)
+    W[3, 5] *= 20.0  # an outlier group
+    q, s = int4.quantize_sym(W, group)
+    levels = np.arange(16) - 8.0
+    checked = 0
+    for k in range(W.shape[0]):
+        for n in range(W.shape[1]):
+            sc = float(s[k // group, n])
+            w = float(W[k, n])
+            if not _not_a_tie(float(np.float32(w) / np.float32(sc))):
+                continue
+            best = int(np.argmin(np.abs(w - levels * sc)))
+            assert q[k, n] == best
+            checked += 1
+    assert checked > 0.99 * W.size
+
+
+def test_asym_codes_are_nearest_levels():
+    rng = np.random.default_rng(5)
+    W = (rng.standard_normal((128, 32)) * 0.02).astype(np.float32)
+    W[:32, 0] = np.abs(W[:32, 0]) + 0.05     # an all-positive group
+    W[32:64, 1] = -np.abs(W[32:64, 1]) - 0.05  # an all-negative group
+    q, s, zp = int4.quantize_asym(W, 32)
+    for gi in range(4):
+        for n in range(32):
+            sc = float(s[gi, n])
+            lo = float(W[gi * 32:(gi + 1) * 32, n].min())
+            t = float(np.float32(-lo) / np.float32(sc))
+            if _not_a_tie(t):
+                assert zp[gi, n] == int(np.clip(round(t), -128, 127))
+            for k in range(gi * 32, (gi + 1) * 32):
+                w = float(W[k, n])
+                if not _not_a_tie(float(np.float32(w) / np.float32(sc))):
+                    continue
+                levels = (np.arange(16) - float(zp[gi, n])) * sc
+                assert q[k, n] == int(np.argmin(np.abs(w - levels)))
+
+
+def test_quantisation_error_within_half_step():
+    rng = np.random.default_rng(9)
+    W = (rng.standard_normal((256, 64)) * 0.02).astype(np.float32)
+    for mode in ("sym", "asym"):
+        q, s, zp = int4.quantize(W, 32, mode)
+        deq = int4.dequant(q, s, 32, zp)
+        step = np.repeat(s.astype(np.float64), 32, axis=0)
+        # the fp16 rounding of the scale can push the extreme code by < 1/14 step
+        assert np.all(np.abs(W - deq) <= 0.5 * step * (1 + 1 / 7) + 1e-12)
+
+
+def test_sym_range_and_extremes():
+    rng = np.random.default_rng(3)
+    W = (rng.standard_normal((128, 64)) * 0.02).astype(np.float32)
+    q, s = int4.quantize_sym(W, 32)
+    assert q.min() >= 1 and q.max() <= 15          # code 0 (-8) is never produced
+    Wg = W.reshape(4, 32, 64)
+    arg = np.abs(Wg).argmax(axis=1)
+    for gi in range(4):
+        for n in range(64):
+            k = gi * 32 + arg[gi, n]
+            assert q[k, n] == (15 if W[k, n] > 0 else 1)
+
+
+def test_degenerate_groups():
+    W = np.zeros((64, 3), np.float32)
+    W[32:, 1] = 0.5          # constant non-zero group: hi == lo
+    W[:32, 2] = 1e-9         # max/7 underflows FP16 to 0
+    q, s = int4.quantize_sym(W, 32)
+    assert float(s[0, 0]) == 0.0 and np.all(q[:32, 0] == 8)
+    assert np.all(int4.dequant(q, s, 32)[:32, 0] == 0.0)
+    assert float(s[0, 2]) == 0.0 and np.all(q[:32, 2] == 8)
+    qa, sa, za = int4.quantize_asym(W, 32)
+    assert float(sa[1, 1]) == 0.0 and za[1, 1] == 0 and np.all(qa[32:, 1] == 0)
+    assert np.all(int4.dequant(qa, sa, 32, za) == 0.0)
+
+
+def test_dequant_is_exact_rational():
+    rng = np.random.default_rng(21)
+    W = (rng.standard_normal((64, 8)) * 0.02).astype(np.float32)
+    q, s, zp = int4.quantize_asym(W, 32)
+    deq = int4.dequant(q, s, 32, zp)
+    for k in range(64):
+        for n in range(8):
+            exact = (int(q[k, n]) - int(zp[k // 32, n])) * Fraction(float(s[k // 32, n]))
+            assert Fraction(float(deq[k, n])) == exact
+
+
+# ----------------------------------------------------------------------------- matmul + tolerance
+
+def test_matmul_matches_exact_rational_brute_force():
+    rng = np.random.default_rng(13)
+    M, K, N = 3, 64, 8
+    X = rng.standard_normal((M, K)).astype(np.float16).astype(np.float64)
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    q, s, zp = int4.quantize_asym(W, 32)
+    deq = int4.dequant(q, s, 32, zp)
+    Y = matmul.matmul_f64(X, deq)
+    S = matmul.abs_scale(X, deq)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(float(X[m, k])) * Fraction(float(deq[k, n])) for k in range(K))
+            assert abs(Fraction(float(Y[m, n])) - exact) <= Fraction(1e-14) * Fraction(float(S[m, n]))
+
+
+def test_ulp16_values():
+    u = matmul.ulp16(np.array([1.0, 1.5, 2.0, 1000.0, 2.0 ** -14, 1e-6, 0.0, -3.0]))
+    assert u.tolist() == [2.0 ** -10, 2.0 ** -10, 2.0 ** -9, 0.5, 2.0 ** -24, 2.0 ** -24, 2.0 ** -24, 2.0 ** -9]
+
+
+def test_tolerance_accepts_fp32_accumulation_and_rejects_mistakes():
+    rng = np.random.default_rng(17)
+    M, K, N = 2, 512, 64
+    X = rng.standard_normal((M, K)).astype(np.float16)
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    q, s = int4.quantize_sym(W, 32)
+    deq = int4.dequant(q, s, 32)
+    Y_ref = matmul.matmul_f64(X, deq)
+    S = matmul.abs_scale(X, deq)
+    # FP32 accumulation, rounded to fp16 output: accepted
+    Y32 = (X.astype(np.float32) @ deq.astype(np.float32)).astype(np.float16)
+    ok, _ = matmul.check(Y32, Y_ref, S)
+    assert ok
+    # nibble order swapped (high nibble taken as the even k): rejected
+    packed = int4.pack_nibbles(q)
+    swapped = np.empty_like(q)
+    swapped[0::2] = packed >> 4
+    swapped[1::2] = packed & 0xF
+    ok, _ = matmul.check(matmul.matmul_f64(X, int4.dequant(swapped, s, 32)), Y_ref, S)
+    assert not ok
+    # scale of the neighbouring group: rejected
+    s_shift = np.roll(s, 1, axis=0)
+    ok, _ = matmul.check(matmul.matmul_f64(X, int4.dequant(q, s_shift, 32)), Y_ref, S)
+    assert not ok
+    # zero point off by one (7 instead of 8): rejected
+    ok, _ = matmul.check(matmul.matmul_f64(X, int4.dequant(q, s, 32, np.full(s.shape, 7, np.int8))), Y_ref, S)
+    assert not ok
+    # a NaN output is never accepted
+    Ybad = Y32.astype(np.float64)
+    Ybad[0, 0] = np.nan
+    assert not matmul.check(Ybad, Y_ref, S)[0]
+
+
+# ----------------------------------------------------------------------------- LUT3
+
+def test_e4m3_table_matches_ml_dtypes_and_torch():
+    import ml_dtypes
+    import torch
+    raw = np.arange(256, dtype=np.uint8)
+    lib = raw.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    tor = torch.from_numpy(raw.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for ref in (lib, tor):
+        nan = np.isnan(ref)
+        assert np.array_equal(nan, np.isnan(lut3.E4M3_TABLE))
+        assert np.array_equal(ref[~nan], lut3.E4M3_TABLE[~nan])
+    assert sorted(np.flatnonzero(np.isnan(lut3.E4M3_TABLE)).tolist()) == [0x7F, 0xFF]
+    assert lut3.e4m3_value(0x7E) == 448.0 and lut3.e4m3_value(0x01) == 2.0 ** -9
+
+
+def test_ue8m0_values():
+    import ml_dtypes
+    raw = np.arange(255, dtype=np.uint8)
+    if hasattr(ml_dtypes, "float8_e8m0fnu"):
+        lib = raw.view(ml_dtypes.float8_e8m0fnu).astype(np.float64)
+        assert [lut3.ue8m0_value(b) for b in range(255)] == lib.tolist()
+    assert [lut3.ue8m0_value(b) for b in (0, 127, 130, 254)] == [2.0 ** -127, 1.0, 8.0, 2.0 ** 127]
+    assert math.isnan(lut3.ue8m0_value(255))
+
+
+def test_lut3_tile_golden(golden):
+    g = golden("lut3_tile_64x8.json")
+    K, N = g["K"], g["N"]
+    idx = ((np.arange(K)[:, None] + np.arange(N)[None, :]) % 8).astype(np.uint8)
+    cb = np.array(g["codebook"], np.uint8).reshape(1, 1, 8)
+    ex = np.array([[g["exponent"]]], np.uint8)
+    assert [lut3.e4m3_value(b) for b in g["codebook"]] == g["codebook_values"]
+    W = lut3.dequant(idx, cb, ex)
+    for k, n, v in g["W_samples"]:
+        assert W[k, n] == v
+    p = lut3.pack_indices(idx)
+    assert p.shape == (1, 1, 8, 24)
+    assert p[0, 0, 0].tolist() == g["stream_ch0"] * 8
+    assert p[0, 0, 1].tolist() == g["stream_ch1"] * 8
+    ones = lut3.pack_indices(np.ones((K, N), np.uint8))
+    assert np.all(ones[0, 0] == np.array(g["stream_all_ones"] * 8, np.uint8))
+    Y = matmul.matmul_f64(np.ones((1, K)), W)
+    assert np.all(Y == g["Y_ones"])
+
+
+def test_lut3_pack_roundtrip_random():
+    rng = np.random.default_rng(31)
+    idx = rng.integers(0, 8, size=(128, 24), dtype=np.uint8)
+    assert np.array_equal(lut3.unpack_indices(lut3.pack_indices(idx)), idx)
+
+
+def test_lut3_sizes_match_the_page():
+    # "about 3.14 bits per weight" and 6144 index bytes per 128N x 128K block
+    assert lut3.algorithmic_bytes(64, 8) * 8 / (64 * 8) == 3.140625
+    assert 128 * 128 * 3 // 8 == lut3.pack_indices(np.zeros((128, 128), np.uint8)).size
+    assert lut3.algorithmic_bytes(4096, 14336) == 23052288
+
+
+def test_lut3_rejects_nan_entries():
+    idx = np.zeros((64, 8), np.uint8)
+    with pytest.raises(ValueError):
+        lut3.dequant(idx, np.full((1, 1, 8), 0x7F, np.uint8), np.array([[127]], np.uint8))
+    with pytest.raises(ValueError):
+        lut3.dequant(idx, np.zeros((1, 1, 8), np.uint8), np.array([[255]], np.uint8))
+
+
+def test_int4_algorithmic_bytes():
+    # bits per weight: 4 + 16/g (sym), 4 + 24/g (asym)
+    assert int4.algorithmic_bytes(4096, 4096, 32, "sym") == 4096 * 4096 * 4.5 / 8
+    assert int4.algorithmic_bytes(4096, 14336, 128, "asym") == 4096 * 14336 * (4 + 24 / 128) / 8
