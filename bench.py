@@ -1,0 +1,568 @@
+#!/usr/bin/env python
+"""Throughput of the fused low-bit dequant + matmul on B200.
+
+Workload of the headline number: one Llama-3-8B-shaped decode step at batch 1,
+the 7 projections (q, k, v, o, gate, up, down) of 32 layers, 224 distinct
+asymmetric INT4 weights (group 32, fp16 scale + int8 zero point), fp16
+activations. A step is the 224 GEMVs, replayed as one CUDA graph. The metric
+is weight-GB/s: bytes of the format (nibbles + scales + zero points) streamed
+per second, against the measured HBM copy bandwidth. The step's weights
+(4.14 GB) are far larger than L2, so no flush is needed between steps.
+
+Secondary numbers (same JSON line, key "secondary"): the single 4096x4096
+GEMV, the K=8192 N=28672 batch sweep, the prefill GEMM and the LUT3 path.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lbq|reference]
+Multi-GPU: one process per GPU under torchrun; each rank runs its own decode
+step (replicas, weak scaling, no collective on the data path); the timing is
+the max over ranks.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode GEMV weight-GB/s & % HBM peak; prefill GEMM TFLOP/s & % tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    return dict(FALLBACK_PEAKS)
+
+
+def int4_bytes(K, N, group, mode):
+    return K * N // 2 + (K // group) * N * (3 if mode == "asym" else 2)
+
+
+def lut3_bytes(K, N):
+    return K * N * 3 // 8 + (K // 64) * (N // 8) * 9
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "power_w_max": max(power),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- distributed
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(world, value):
+    import torch
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def physical_gpu_index(local):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v for v in vis.split(",") if v.strip()]
+        if local < len(ids) and ids[local].strip().isdigit():
+            return int(ids[local])
+    return local
+
+
+# ----------------------------------------------------------------------------- the decode step
+
+class DecodeStep:
+    """224 asym INT4 g32 GEMVs (32 layers x 7 projections), images resident in HBM."""
+
+    def __init__(self, torch, lbq, workloads, device, layers):
+        self.torch = torch
+        self.projs = []
+        self.bytes = 0
+        x_len = sum(K for _ in range(layers) for (_, K, _) in workloads.LLAMA3_8B_PROJ)
+        y_len = sum(N for _ in range(layers) for (_, _, N) in workloads.LLAMA3_8B_PROJ)
+        self.x_all = torch.empty(x_len, dtype=torch.float16, device=device)
+        self.y_all = torch.empty(y_len, dtype=torch.float16, device=device)
+        xo = yo = 0
+        ws_bytes = 0
+        for layer in range(layers):
+            for p, (name, K, N) in enumerate(workloads.LLAMA3_8B_PROJ):
+                seed = workloads.c2_seed(layer, p)
+                W = workloads.weights_device(seed, K, N, device)
+                img = lbq.pack(W, 32, "asym")
+                del W
+                x = self.x_all[xo:xo + K].view(1, K)
+                x.copy_(workloads.activations_device(seed, 1, K, "f16", device))
+                y = self.y_all[yo:yo + N].view(1, N)
+                xo += K
+                yo += N
+                self.projs.append((K, N, img, x, y))
+                self.bytes += int4_bytes(K, N, 32, "asym")
+                ws_bytes = max(ws_bytes, lbq.lbq_workspace_size(0, 1, K, N, 32, 1))
+        self.ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=device)
+        self.lbq = lbq
+        torch.cuda.synchronize()
+
+    def launch_all(self):
+        lbq = self.lbq
+        stream = self.torch.cuda.current_stream().cuda_stream
+        for K, N, img, x, y in self.projs:
+            lbq.lbq_gemv(x.data_ptr(), 0, 1, K, N, 32, 1, img.data_ptr(), y.data_ptr(), 0,
+                         self.ws.data_ptr(), self.ws.numel(), stream)
+
+    def capture(self):
+        torch = self.torch
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.launch_all()  # warm the planner caches outside capture
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        before = self.lbq.lbq_launch_count()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.launch_all()
+        self.launches_per_step = self.lbq.lbq_launch_count() - before
+        torch.cuda.synchronize()
+        return g
+
+
+def time_graph(torch, graph, steps, warmup, world):
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return e0.elapsed_time(e1)
+
+
+def rotating_gemv_ms(torch, lbq, images, X, N, group, mode, ws, reps=5):
+    """Per-launch time of one GEMV shape, cycling through distinct weight copies
+    (their total exceeds L2) inside one CUDA graph."""
+    Y = torch.empty((X.shape[0], N), dtype=X.dtype, device=X.device)
+    xdt = 0 if X.dtype == torch.float16 else 1
+    stream_of = lambda: torch.cuda.current_stream().cuda_stream
+    m = {"sym": 0, "asym": 1}[mode]
+
+    def run():
+        s = stream_of()
+        for img in images:
+            lbq.lbq_gemm(X.data_ptr(), xdt, X.shape[0], X.shape[1], N, group, m, img.data_ptr(), Y.data_ptr(), xdt,
+                         ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0, s)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        run()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / (reps * len(images))
+
+
+def secondary_measurements(torch, lbq, workloads, device, peaks, quick):
+    out = {}
+    hbm = peaks["hbm_gbs"]
+    l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
+    # c1: single 4096x4096 sym g32 GEMV, fp16
+    K, N = 4096, 4096
+    W = workloads.weights_device(0, K, N, device)
+    img0 = lbq.pack(W, 32, "sym")
+    del W
+    copies = max(3, (3 * l2_bytes) // img0.numel() + 1)
+    images = [img0] + [img0.clone() for _ in range(copies - 1)]
+    X = workloads.activations_device(0, 1, K, "f16", device)
+    ms = rotating_gemv_ms(torch, lbq, images, X, N, 32, "sym", lbq.workspace(0, 1, K, N, 32, "sym"))
+    b = int4_bytes(K, N, 32, "sym")
+    out["c1_gemv_4096x4096_sym_g32_m1"] = {"us": ms * 1e3, "GBps": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm,
+                                           "weight_copies": copies}
+    lbq.lbq_debug_force_skinny(1)
+    ms = rotating_gemv_ms(torch, lbq, images, X, N, 32, "sym", lbq.workspace(0, 1, K, N, 32, "sym"))
+    lbq.lbq_debug_force_skinny(0)
+    out["c1_gemv_m1_on_tensor_core_kernel"] = {"us": ms * 1e3, "GBps": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm}
+    del images, img0
+    if quick:
+        return out
+    # c3: K=8192 N=28672 sym g64/g128 with outliers, bf16, M in {1,2,4,8,16}
+    K, N = 8192, 28672
+    W = workloads.weights_device(3, K, N, device, outlier_frac=1e-3, outlier_mult=20.0)
+    for group in (64, 128):
+        img0 = lbq.pack(W, group, "sym")
+        copies = max(2, (3 * l2_bytes) // img0.numel() + 1)
+        images = [img0] + [img0.clone() for _ in range(copies - 1)]
+        b = int4_bytes(K, N, group, "sym")
+        for M in (1, 2, 4, 8, 16):
+            X = workloads.activations_device(3, M, K, "bf16", device)
+            ws = lbq.workspace(0, M, K, N, group, "sym")
+            ms = rotating_gemv_ms(torch, lbq, images, X, N, group, "sym", ws, reps=3)
+            out[f"c3_g{group}_m{M}"] = {"us": ms * 1e3, "GBps": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm}
+            if M == 1:
+                lbq.lbq_debug_force_skinny(1)
+                ws = lbq.workspace(0, M, K, N, group, "sym")
+                ms = rotating_gemv_ms(torch, lbq, images, X, N, group, "sym", ws, reps=3)
+                lbq.lbq_debug_force_skinny(0)
+                out[f"c3_g{group}_m1_on_tensor_core_kernel"] = {"us": ms * 1e3, "GBps": b / ms / 1e6,
+                                                                "frac_hbm": b / ms / 1e6 / hbm}
+        del images, img0
+    del W
+    return out
+
+
+# ----------------------------------------------------------------------------- CPU baseline (oracle)
+
+def oracle_sample(seconds_target, layer=0, max_proj=7):
+    """Time the oracle (dequant + FP64 matmul) on the first projections of one
+    layer of the decode step, host-generated and quantised outside the timer."""
+    import numpy as np
+    import workloads
+    from oracle import int4, matmul
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    done_bytes, spent, names = 0, 0.0, []
+    for p, (name, K, N) in enumerate(workloads.LLAMA3_8B_PROJ[:max_proj]):
+        seed = workloads.c2_seed(layer, p)
+        W = workloads.weights_host(seed, K, N)
+        q, s, z = int4.quantize_asym(W, 32)
+        X = workloads.activations_host(seed, 1, K, "f16")
+        t0 = time.perf_counter()
+        deq = int4.dequant(q, s, 32, z)
+        matmul.matmul_f64(X, deq)
+        spent += time.perf_counter() - t0
+        done_bytes += int4_bytes(K, N, 32, "asym")
+        names.append(name)
+        if spent >= seconds_target:
+            break
+    return {"value": done_bytes / spent / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"layer {layer} projections {'+'.join(names)} of the decode step: exact dequant + FP64 "
+                      f"matmul (numpy), {done_bytes} weight bytes in {spent:.2f} s"}
+
+
+def run_reference(args):
+    """The reference arm: the oracle as it stands, on the host cores, same metric."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1 and rank != 0:
+        return 0
+    import numpy as np
+    import workloads
+    from oracle import int4, matmul
+    projs = list(enumerate(workloads.LLAMA3_8B_PROJ))
+    prepared = []
+    for p, (name, K, N) in projs:
+        seed = workloads.c2_seed(0, p)
+        W = workloads.weights_host(seed, K, N)
+        q, s, z = int4.quantize_asym(W, 32)
+        prepared.append((K, N, q, s, z, workloads.activations_host(seed, 1, K, "f16")))
+    total_bytes, total_s = 0, 0.0
+    for i in range(args.warmup + args.steps):
+        K, N, q, s, z, X = prepared[i % len(prepared)]
+        t0 = time.perf_counter()
+        matmul.matmul_f64(X, int4.dequant(q, s, 32, z))
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            total_bytes += int4_bytes(K, N, 32, "asym")
+            total_s += dt
+    value = total_bytes / total_s / 1e9
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_s / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "Llama-3-8B-shaped decode step (layer 0 projections, one per step), asym INT4 "
+                                   "g32, fp16 X, M=1", "l2": "n/a (host)"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": "one projection of layer 0 per step, cycling q,k,v,o,gate,up,down: exact "
+                                       "dequant + FP64 numpy matmul"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- ncu cases
+
+# name -> (K, N, group, mode, x dtype, M); a "_tc" suffix routes M = 1 through the tensor-core kernel
+PROFILE_CASES = {
+    "c1": (4096, 4096, 32, "sym", "f16", 1),
+    "c2gate": (4096, 14336, 32, "asym", "f16", 1),
+    "c2gate_tc": (4096, 14336, 32, "asym", "f16", 1),
+    "c4m2048": (4096, 14336, 128, "asym", "bf16", 2048),
+    "c2down": (14336, 4096, 32, "asym", "f16", 1),
+    "c2kv": (4096, 1024, 32, "asym", "f16", 1),
+    "c3m1": (8192, 28672, 128, "sym", "bf16", 1),
+    "c3m16": (8192, 28672, 128, "sym", "bf16", 16),
+}
+
+
+def run_profile_case(name):
+    """A handful of launches of one shape, each on a distinct weight copy (the
+    copies total more than L2), for an ncu capture; prints nothing to parse."""
+    import torch
+    import bit_weight_only_pack_b200 as lbq
+    import workloads
+    K, N, group, mode, xdt, M = PROFILE_CASES[name]
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    W = workloads.weights_device(7, K, N, device)
+    img0 = lbq.pack(W, group, mode)
+    del W
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    copies = max(3, (3 * l2) // img0.numel() + 1)
+    images = [img0] + [img0.clone() for _ in range(copies - 1)]
+    X = workloads.activations_device(7, M, K, xdt, device)
+    if name.endswith("_tc"):
+        lbq.lbq_debug_force_skinny(1)
+    ws = lbq.workspace(0, M, K, N, group, mode)
+    for img in images:
+        lbq.gemm(X, img, N, group, mode, ws=ws)
+    torch.cuda.synchronize()
+    lbq.lbq_debug_force_skinny(0)
+    lbq.device_status()
+    print(f"profile case {name}: {copies} launches of K={K} N={N} g={group} {mode} M={M}", flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- main
+
+def traffic_from_profiles(kernel):
+    """DRAM bytes per launch recorded by the last ncu capture of `kernel`, if the
+    kernel source has not changed since (hash recorded beside the figure)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        import hashlib
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+        if not rec:
+            return None
+        src = os.path.join(ROOT, "bit_weight_only_pack_b200", "csrc", rec["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        return rec["dram_bytes_per_launch_full"] if h == rec["source_sha"] else None
+    except Exception:
+        return None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="lbq", choices=["lbq", "reference"])
+    ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--quick", action="store_true", help="skip the longer secondary measurements")
+    ap.add_argument("--no-pdl", action="store_true",
+                    help="launch the decode-step GEMVs without programmatic dependent launch")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", default=None, choices=sorted(PROFILE_CASES),
+                    help="run a small case for ncu (a few launches over weight copies larger than L2) and exit")
+    args = ap.parse_args()
+    if args.profile:
+        return run_profile_case(args.profile)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import bit_weight_only_pack_b200 as lbq
+    import workloads
+
+    world, rank, local = dist_setup(args)
+    device = torch.device("cuda", local)
+    peaks = load_peaks()
+
+    step = DecodeStep(torch, lbq, workloads, device, args.layers)
+    # the step's weights are written once and then only read, so the GEMVs may
+    # overlap their weight streaming with the previous kernel's tail
+    lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 0 if args.no_pdl else 1)
+    graph = step.capture()
+    lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 0)
+    sampler = ClockSampler(physical_gpu_index(local))
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.25)
+    elapsed_ms = time_graph(torch, graph, args.steps, 0, world)
+    clocks = sampler.stop()
+    elapsed_ms = max_over_ranks(world, elapsed_ms)
+    ms_per_step = elapsed_ms / args.steps
+    value = world * step.bytes / (ms_per_step / 1e3) / 1e9
+
+    # end to end: pinned host X in, pinned host Y out, every step
+    x_host = torch.empty_like(step.x_all, device="cpu").pin_memory()
+    x_host.copy_(step.x_all.cpu())
+    y_host = torch.empty_like(step.y_all, device="cpu").pin_memory()
+    x_stage = torch.empty_like(step.x_all)
+    for _ in range(args.warmup):
+        step.x_all.copy_(x_host, non_blocking=True)
+        graph.replay()
+        y_host.copy_(step.y_all, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step.x_all.copy_(x_host, non_blocking=True)
+        graph.replay()
+        y_host.copy_(step.y_all, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(world, e0.elapsed_time(e1)) / args.steps
+    del x_stage
+
+    secondary = None
+    if not args.no_secondary:
+        secondary = secondary_measurements(torch, lbq, workloads, device, peaks, args.quick)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(10.0)
+
+    hbm = peaks["hbm_gbs"]
+    per_gpu = step.bytes / (ms_per_step / 1e3) / 1e9
+    launches = step.launches_per_step
+    traffic = traffic_from_profiles("gemv_m1_kernel")
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16 x int4 -> f32 accumulate", "data": "synthetic",
+        "config": {"workload": "c2: Llama-3-8B-shaped decode step at M=1, 7 projections x %d layers, asymmetric "
+                               "INT4 group 32 (fp16 scale + int8 zp), fp16 X, fp16 Y" % args.layers,
+                   "weight_bytes_per_step": step.bytes, "gemvs_per_step": len(step.projs),
+                   "l2": "inputs larger than L2 (%.2f GB of weights per step vs %d MB L2); no flush"
+                         % (step.bytes / 1e9, torch.cuda.get_device_properties(device).L2_cache_size >> 20),
+                   "timing": "CUDA events around K replays of one CUDA graph holding the step",
+                   "pdl": not args.no_pdl,
+                   "parallelism": "replicas" if world > 1 else "1 GPU"},
+        "frac_hbm": per_gpu / hbm,
+        "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": hbm, "unit": "GB/s", "frac": per_gpu / hbm,
+                     "peak_source": peaks["source"],
+                     "traffic": (traffic * launches if traffic is not None else None),
+                     "traffic_note": "DRAM bytes per step from ncu (sum over the step's launches) when the "
+                                     "kernel source is unchanged since the capture, else null",
+                     "kernel": "gemv_m1_kernel", "algorithmic_bytes_per_step": step.bytes},
+        "clocks": clocks,
+        "e2e": {"value": world * step.bytes / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": step.x_all.numel() * 2, "d2h_bytes_per_step": step.y_all.numel() * 2,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": launches * args.steps,
+        "cpu_baseline": cpu,
+        "secondary": secondary,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,16 @@
+"""bit_weight_only_pack_b200: fused low-bit weight dequantize + matmul on B200.
+
+Y[M, N] = X[M, K] . dequant(Wq)[K, N] for INT4 (group-wise FP16 scales,
+symmetric or asymmetric with an int8 zero point) and 3-bit LUT weights
+(E4M3 codebook per 8 x 64 tile, UE8M0 exponent), as a decode GEMV / skinny
+GEMM and as a tcgen05 prefill GEMM. The work is done by liblbq.so (C ABI in
+include/lbq.h); this package is its thin Python binding.
+"""
+
+from .binding import (  # noqa: F401
+    DTYPES, MODES, LbqError, dequant, device_status, gemm, gemv, lut3_gemm, pack, pack_lut3,
+    unpack_canonical, unpack_lut3_canonical, workspace,
+    lbq_debug_force_splits, lbq_debug_force_skinny, lbq_debug_force_tc, lbq_dequant, lbq_device_status, lbq_gemm, lbq_gemv, lbq_last_error,
+    lbq_launch_count, lbq_lut3_gemm, lbq_pack, lbq_set_option, LBQ_OPT_PDL, lbq_pack_lut3, lbq_packed_size, lbq_unpack_canonical,
+    lbq_unpack_lut3_canonical, lbq_version, lbq_workspace_size,
+)

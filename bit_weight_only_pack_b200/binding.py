@@ -1,0 +1,290 @@
+"""Thin ctypes binding of liblbq.so: the C ABI of include/lbq.h, same names.
+
+Argument marshalling only. Every step of the computation runs in the CUDA
+kernels of liblbq.so; there is no CPU or Python fallback. If the library has
+not been built, importing this module raises.
+
+Two layers:
+* ``lbq_*`` functions mirror the C calls one to one (integers and raw
+  pointers; a non-OK status raises :class:`LbqError`).
+* Small torch helpers (``pack``, ``gemv``, ``gemm``, ...) take CUDA tensors,
+  pass their data pointers and the current stream, and allocate outputs with
+  torch (the library itself never allocates).
+"""
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblbq.so")
+
+LBQ_OK, LBQ_ERR_INVALID_ARG, LBQ_ERR_UNSUPPORTED, LBQ_ERR_CUDA, LBQ_ERR_DEVICE = range(5)
+MODES = {"sym": 0, "asym": 1, "lut3": 2}
+DTYPES = {"f16": 0, "bf16": 1}
+STATUS_NAMES = {0: "LBQ_OK", 1: "LBQ_ERR_INVALID_ARG", 2: "LBQ_ERR_UNSUPPORTED", 3: "LBQ_ERR_CUDA",
+                4: "LBQ_ERR_DEVICE"}
+
+
+class LbqError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python bit_weight_only_pack_b200/build.py` "
+                      "(the CUDA library is required; there is no fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_c_int, _c_size, _vp, _u64 = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_uint64
+
+_SIGS = {
+    "lbq_last_error": ([], ctypes.c_char_p),
+    "lbq_version": ([], _c_int),
+    "lbq_launch_count": ([], _u64),
+    "lbq_packed_size": ([_c_int, _c_int, _c_int, _c_int, ctypes.POINTER(_c_size)], _c_int),
+    "lbq_pack": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _c_size, _vp], _c_int),
+    "lbq_pack_lut3": ([_vp, _vp, _vp, _c_int, _c_int, _vp, _c_size, _vp], _c_int),
+    "lbq_workspace_size": ([_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, ctypes.POINTER(_c_size)], _c_int),
+    "lbq_gemv": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp, _c_size, _vp], _c_int),
+    "lbq_gemm": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp, _c_size, _vp], _c_int),
+    "lbq_lut3_gemm": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp, _c_size, _vp], _c_int),
+    "lbq_unpack_canonical": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp], _c_int),
+    "lbq_unpack_lut3_canonical": ([_vp, _c_int, _c_int, _vp, _vp, _vp, _vp], _c_int),
+    "lbq_dequant": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
+    "lbq_device_status": ([_vp], _c_int),
+    "lbq_set_option": ([_c_int, _c_int], _c_int),
+    "lbq_debug_force_splits": ([_c_int], None),
+    "lbq_debug_force_skinny": ([_c_int], None),
+    "lbq_debug_force_tc": ([_c_int], None),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+
+def exported_symbols():
+    """Names this binding binds (each must be exported by liblbq.so)."""
+    return sorted(_SIGS)
+
+
+def _check(status):
+    if status != LBQ_OK:
+        raise LbqError(status, _lib.lbq_last_error().decode())
+
+
+def lbq_last_error():
+    return _lib.lbq_last_error().decode()
+
+
+def lbq_version():
+    return _lib.lbq_version()
+
+
+def lbq_launch_count():
+    return int(_lib.lbq_launch_count())
+
+
+def lbq_packed_size(K, N, group, mode):
+    out = _c_size(0)
+    _check(_lib.lbq_packed_size(K, N, group, mode, ctypes.byref(out)))
+    return out.value
+
+
+def lbq_workspace_size(op, M, K, N, group, mode):
+    out = _c_size(0)
+    _check(_lib.lbq_workspace_size(op, M, K, N, group, mode, ctypes.byref(out)))
+    return out.value
+
+
+def lbq_pack(W, K, N, group, mode, image, image_bytes, stream):
+    _check(_lib.lbq_pack(W, K, N, group, mode, image, image_bytes, stream))
+
+
+def lbq_pack_lut3(idx, codebooks, exponents, K, N, image, image_bytes, stream):
+    _check(_lib.lbq_pack_lut3(idx, codebooks, exponents, K, N, image, image_bytes, stream))
+
+
+def lbq_gemv(X, x_dtype, M, K, N, group, mode, image, Y, y_dtype, ws, ws_bytes, stream):
+    _check(_lib.lbq_gemv(X, x_dtype, M, K, N, group, mode, image, Y, y_dtype, ws, ws_bytes, stream))
+
+
+def lbq_gemm(X, x_dtype, M, K, N, group, mode, image, Y, y_dtype, ws, ws_bytes, stream):
+    _check(_lib.lbq_gemm(X, x_dtype, M, K, N, group, mode, image, Y, y_dtype, ws, ws_bytes, stream))
+
+
+def lbq_lut3_gemm(X, x_dtype, M, K, N, image, Y, y_dtype, ws, ws_bytes, stream):
+    _check(_lib.lbq_lut3_gemm(X, x_dtype, M, K, N, image, Y, y_dtype, ws, ws_bytes, stream))
+
+
+def lbq_unpack_canonical(image, K, N, group, mode, q_packed, scales, zp, stream):
+    _check(_lib.lbq_unpack_canonical(image, K, N, group, mode, q_packed, scales, zp, stream))
+
+
+def lbq_unpack_lut3_canonical(image, K, N, idx_stream, codebooks, exponents, stream):
+    _check(_lib.lbq_unpack_lut3_canonical(image, K, N, idx_stream, codebooks, exponents, stream))
+
+
+def lbq_dequant(image, K, N, group, mode, W_out, stream):
+    _check(_lib.lbq_dequant(image, K, N, group, mode, W_out, stream))
+
+
+def lbq_device_status(stream):
+    _check(_lib.lbq_device_status(stream))
+
+
+LBQ_OPT_PDL = 1
+
+
+def lbq_set_option(option, value):
+    _check(_lib.lbq_set_option(option, value))
+
+
+def lbq_debug_force_splits(splits):
+    _lib.lbq_debug_force_splits(splits)
+
+
+def lbq_debug_force_tc(on):
+    _lib.lbq_debug_force_tc(1 if on else 0)
+
+
+def lbq_debug_force_skinny(on):
+    _lib.lbq_debug_force_skinny(1 if on else 0)
+
+
+# ----------------------------------------------------------------------------- torch helpers
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream():
+    return _torch().cuda.current_stream().cuda_stream
+
+
+def _mode(mode):
+    return MODES[mode] if isinstance(mode, str) else int(mode)
+
+
+def _dt(t):
+    torch = _torch()
+    if t.dtype == torch.float16:
+        return DTYPES["f16"]
+    if t.dtype == torch.bfloat16:
+        return DTYPES["bf16"]
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def pack(W, group, mode):
+    """Quantise + repack a float32 [K, N] CUDA tensor; returns the uint8 image."""
+    torch = _torch()
+    _need_cuda(W)
+    K, N = W.shape
+    m = _mode(mode)
+    img = torch.empty(lbq_packed_size(K, N, group, m), dtype=torch.uint8, device=W.device)
+    lbq_pack(W.data_ptr(), K, N, group, m, img.data_ptr(), img.numel(), _stream())
+    return img
+
+
+def pack_lut3(idx, codebooks, exponents):
+    """Build a LUT3 image from idx uint8 [K, N], codebooks uint8 [K/64, N/8, 8], exponents uint8 [K/64, N/8]."""
+    torch = _torch()
+    _need_cuda(idx, codebooks, exponents)
+    K, N = idx.shape
+    img = torch.empty(lbq_packed_size(K, N, 0, MODES["lut3"]), dtype=torch.uint8, device=idx.device)
+    lbq_pack_lut3(idx.data_ptr(), codebooks.data_ptr(), exponents.data_ptr(), K, N, img.data_ptr(), img.numel(),
+                  _stream())
+    return img
+
+
+def workspace(op, M, K, N, group, mode, device="cuda"):
+    """A zero-filled workspace of the size the call needs (None when it needs none)."""
+    torch = _torch()
+    n = lbq_workspace_size(op, M, K, N, group, _mode(mode))
+    return torch.zeros(n, dtype=torch.uint8, device=device) if n else None
+
+
+def _out(X, N, y_dtype):
+    torch = _torch()
+    dt = {None: X.dtype, "f16": torch.float16, "bf16": torch.bfloat16}[y_dtype] if not hasattr(y_dtype, "is_floating_point") else y_dtype
+    return torch.empty((X.shape[0], N), dtype=dt, device=X.device)
+
+
+def gemv(X, image, N, group, mode, y_dtype=None, ws=None, Y=None):
+    """Y[M, N] = X[M, K] . dequant(image) for 1 <= M <= 16 (INT4 image)."""
+    _need_cuda(X, image, ws, Y)
+    M, K = X.shape
+    m = _mode(mode)
+    if ws is None:
+        ws = workspace(0, M, K, N, group, m, X.device)
+    Y = _out(X, N, y_dtype) if Y is None else Y
+    lbq_gemv(X.data_ptr(), _dt(X), M, K, N, group, m, image.data_ptr(), Y.data_ptr(), _dt(Y),
+             ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0, _stream())
+    return Y
+
+
+def gemm(X, image, N, group, mode, y_dtype=None, ws=None, Y=None):
+    """Y[M, N] = X[M, K] . dequant(image) for any M (INT4 image)."""
+    _need_cuda(X, image, ws, Y)
+    M, K = X.shape
+    m = _mode(mode)
+    if ws is None:
+        ws = workspace(1, M, K, N, group, m, X.device)
+    Y = _out(X, N, y_dtype) if Y is None else Y
+    lbq_gemm(X.data_ptr(), _dt(X), M, K, N, group, m, image.data_ptr(), Y.data_ptr(), _dt(Y),
+             ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0, _stream())
+    return Y
+
+
+def lut3_gemm(X, image, N, y_dtype=None, ws=None, Y=None):
+    """Y[M, N] = X[M, K] . decode(image) for a LUT3 image, any M."""
+    _need_cuda(X, image, ws, Y)
+    M, K = X.shape
+    if ws is None:
+        ws = workspace(2, M, K, N, 0, MODES["lut3"], X.device)
+    Y = _out(X, N, y_dtype) if Y is None else Y
+    lbq_lut3_gemm(X.data_ptr(), _dt(X), M, K, N, image.data_ptr(), Y.data_ptr(), _dt(Y),
+                  ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0, _stream())
+    return Y
+
+
+def unpack_canonical(image, K, N, group, mode):
+    """(q_packed uint8 [K/2, N], scale fp16 [K/group, N], zp int8 [K/group, N] or None)."""
+    torch = _torch()
+    m = _mode(mode)
+    q = torch.empty((K // 2, N), dtype=torch.uint8, device=image.device)
+    s = torch.empty((K // group, N), dtype=torch.int16, device=image.device)
+    z = torch.empty((K // group, N), dtype=torch.int8, device=image.device) if m == MODES["asym"] else None
+    lbq_unpack_canonical(image.data_ptr(), K, N, group, m, q.data_ptr(), s.data_ptr(),
+                         z.data_ptr() if z is not None else None, _stream())
+    return q, s.view(torch.float16), z
+
+
+def unpack_lut3_canonical(image, K, N):
+    torch = _torch()
+    idx = torch.empty((K // 64, N // 8, 8, 24), dtype=torch.uint8, device=image.device)
+    cb = torch.empty((K // 64, N // 8, 8), dtype=torch.uint8, device=image.device)
+    ex = torch.empty((K // 64, N // 8), dtype=torch.uint8, device=image.device)
+    lbq_unpack_lut3_canonical(image.data_ptr(), K, N, idx.data_ptr(), cb.data_ptr(), ex.data_ptr(), _stream())
+    return idx, cb, ex
+
+
+def dequant(image, K, N, group, mode):
+    """Exact FP32 [K, N] dequantisation of an image (debug / parity)."""
+    torch = _torch()
+    W = torch.empty((K, N), dtype=torch.float32, device=image.device)
+    lbq_dequant(image.data_ptr(), K, N, group, _mode(mode), W.data_ptr(), _stream())
+    return W
+
+
+def device_status():
+    lbq_device_status(_stream())

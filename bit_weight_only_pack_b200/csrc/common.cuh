@@ -1,0 +1,159 @@
+// Shared definitions of the lbq device library: image layout, launch
+// bookkeeping and the small PTX wrappers the kernels use.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "lbq.h"
+
+namespace lbq {
+
+// Device-side error word: kernels OR a code into it; lbq_device_status()
+// reads and clears it.
+__device__ unsigned int g_device_error;
+
+// ----------------------------------------------------------------------------
+// Device image layout
+//
+// [0, 256)           header (ImageHeader, zero padded)
+// INT4 (SYM / ASYM):
+//   Q region         N rows of K/2 bytes. Row n holds column n of the logical
+//                    [K, N] weight, k ascending, in 16-byte chunks of 32 k.
+//                    Chunk c = four little-endian 32-bit words; word w holds
+//                    k = 32c + 8w + i (i = 0..7) with code i in nibble slot
+//                    kSlot[i] (bits 4*slot .. 4*slot+3). The slot order puts
+//                    (k, k+1) pairs in the two 16-bit halves of the same mask,
+//                    so one AND/OR turns two codes into a half2/bf16x2.
+//   S region         FP16 scales, N rows of K/group values (row n = the
+//                    groups of column n), row stride padded to 16 bytes.
+//   Z region (ASYM)  int8 zero points, same shape, row stride padded to 16 bytes.
+// LUT3:
+//   I region         N rows of (K/64)*24 bytes: row n = channel n, 24 bytes
+//                    per 64-k tile, in the kernel order of lut3.cuh.
+//   C region         codebooks, [N/8][K/64][8] E4M3 bytes.
+//   E region         exponents, [N/8][K/64] UE8M0 bytes.
+// Every region starts on a 256-byte boundary.
+// ----------------------------------------------------------------------------
+
+constexpr uint32_t kMagicInt4 = 0x3451424Cu;  // "LBQ4"
+constexpr uint32_t kMagicLut3 = 0x3351424Cu;  // "LBQ3"
+constexpr uint32_t kImageVersion = 1;
+constexpr size_t kHeaderBytes = 256;
+constexpr size_t kRegionAlign = 256;
+
+// nibble slot of the i-th k of an 8-k word: pairs (k0,k1) (k2,k3) (k4,k5) (k6,k7)
+// sit in slots (0,4) (1,5) (2,6) (3,7).
+__host__ __device__ constexpr int slot_of(int i) { return (i >> 1) + ((i & 1) << 2); }
+
+struct ImageHeader {
+  uint32_t magic;
+  uint32_t version;
+  int32_t K, N, group, mode;
+  uint64_t off0, off1, off2;  // INT4: Q, S, Z   LUT3: I, C, E
+  uint64_t total;
+};
+static_assert(sizeof(ImageHeader) <= kHeaderBytes, "header too large");
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Layout {
+  int K, N, group, mode;
+  size_t off0, off1, off2, total;
+  size_t bytes0, bytes1, bytes2;
+  size_t s_stride, z_stride;  // INT4: padded row strides (bytes) of the S and Z regions
+};
+
+inline Layout make_layout(int K, int N, int group, int mode) {
+  Layout L{};
+  L.K = K; L.N = N; L.group = group; L.mode = mode;
+  if (mode == LBQ_MODE_LUT3) {
+    L.bytes0 = (size_t)N * (size_t)(K / 64) * 24;
+    L.bytes1 = (size_t)(N / 8) * (size_t)(K / 64) * 8;
+    L.bytes2 = (size_t)(N / 8) * (size_t)(K / 64);
+  } else {
+    L.s_stride = align_up((size_t)(K / group) * 2, 16);
+    L.z_stride = align_up((size_t)(K / group), 16);
+    L.bytes0 = (size_t)N * (size_t)(K / 2);
+    L.bytes1 = (size_t)N * L.s_stride;
+    L.bytes2 = mode == LBQ_MODE_ASYM ? (size_t)N * L.z_stride : 0;
+  }
+  L.off0 = kHeaderBytes;
+  L.off1 = align_up(L.off0 + L.bytes0, kRegionAlign);
+  L.off2 = align_up(L.off1 + L.bytes1, kRegionAlign);
+  L.total = align_up(L.off2 + L.bytes2, kRegionAlign);
+  return L;
+}
+
+inline ImageHeader make_header(const Layout& L) {
+  ImageHeader h{};
+  h.magic = L.mode == LBQ_MODE_LUT3 ? kMagicLut3 : kMagicInt4;
+  h.version = kImageVersion;
+  h.K = L.K; h.N = L.N; h.group = L.group; h.mode = L.mode;
+  h.off0 = L.off0; h.off1 = L.off1; h.off2 = L.off2; h.total = L.total;
+  return h;
+}
+
+// ----------------------------------------------------------------------------
+// PTX wrappers
+// ----------------------------------------------------------------------------
+
+// 16-byte streaming load through the non-coherent path, no L1 allocation.
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+// (a & b) | c in one LOP3.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// acc += x.lo * w.lo + x.hi * w.hi with FP16 (or BF16) products accumulated in
+// FP32 (mixed-precision FMA; the FP16 x FP16 product is exact in FP32).
+__device__ __forceinline__ float fma2_f16_f32(uint32_t x2, uint32_t w2, float acc) {
+  asm("{\n\t.reg .b16 xl, xh, wl, wh;\n\t"
+      "mov.b32 {xl, xh}, %1;\n\t"
+      "mov.b32 {wl, wh}, %2;\n\t"
+      "fma.rn.f32.f16 %0, xl, wl, %0;\n\t"
+      "fma.rn.f32.f16 %0, xh, wh, %0;\n\t}"
+      : "+f"(acc) : "r"(x2), "r"(w2));
+  return acc;
+}
+
+__device__ __forceinline__ float fma2_bf16_f32(uint32_t x2, uint32_t w2, float acc) {
+  asm("{\n\t.reg .b16 xl, xh, wl, wh;\n\t"
+      "mov.b32 {xl, xh}, %1;\n\t"
+      "mov.b32 {wl, wh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, xl, wl, %0;\n\t"
+      "fma.rn.f32.bf16 %0, xh, wh, %0;\n\t}"
+      : "+f"(acc) : "r"(x2), "r"(w2));
+  return acc;
+}
+
+__device__ __forceinline__ float h2f_bits(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+__device__ __forceinline__ float bf2f_bits(uint16_t h) { return __uint_as_float(((uint32_t)h) << 16); }
+
+template <bool BF16>
+__device__ __forceinline__ float x2f(uint16_t h) { return BF16 ? bf2f_bits(h) : h2f_bits(h); }
+
+__device__ __forceinline__ void store_out(void* Y, size_t i, float v, bool bf16) {
+  if (bf16) reinterpret_cast<__nv_bfloat16*>(Y)[i] = __float2bfloat16_rn(v);
+  else reinterpret_cast<__half*>(Y)[i] = __float2half_rn(v);
+}
+
+}  // namespace lbq

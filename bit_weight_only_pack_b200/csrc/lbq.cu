@@ -1,0 +1,607 @@
+// The C ABI of the lbq library (declared in include/lbq.h): argument checks,
+// shape-based kernel selection and launches. One translation unit includes
+// every kernel header, so the library builds as a single object.
+//
+// Kernel selection by shape mirrors BaseRT's practice of choosing kernels
+// from the layer shape ("BaseRT", kernel-selection section): M = 1 goes to
+// the CUDA-core GEMV, 2 <= M <= 16 to the tensor-core skinny kernel, larger M
+// to the tcgen05 prefill GEMM; split-K is chosen when the row tiles alone
+// cannot fill the SMs.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <algorithm>
+#include <map>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "pack_int4.cuh"
+#include "tma.cuh"
+#include "gemv_m1.cuh"
+#include "skinny.cuh"
+#include "gemm_tc.cuh"
+
+namespace lbq {
+
+static thread_local std::string g_last_error;
+static std::atomic<uint64_t> g_launches{0};
+
+static lbq_status fail(lbq_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+static lbq_status fail(lbq_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+static lbq_status cuda_check(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return fail(LBQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return LBQ_OK;
+}
+
+static lbq_status launch_check(const char* what) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cuda_check(cudaGetLastError(), what);
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int num_sms() {
+  static int sms = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  });
+  return sms;
+}
+
+static int log2_exact(int v) {
+  int l = 0;
+  while ((1 << l) < v) ++l;
+  return (1 << l) == v ? l : -1;
+}
+
+static lbq_status check_int4_shape(int K, int N, int group, int mode) {
+  if (mode != LBQ_MODE_SYM && mode != LBQ_MODE_ASYM)
+    return fail(LBQ_ERR_UNSUPPORTED, "mode %d is not an INT4 mode", mode);
+  if (group != 32 && group != 64 && group != 128)
+    return fail(LBQ_ERR_UNSUPPORTED, "group %d not in {32, 64, 128}", group);
+  if (K <= 0 || N <= 0) return fail(LBQ_ERR_INVALID_ARG, "K=%d N=%d must be positive", K, N);
+  if (K % group) return fail(LBQ_ERR_INVALID_ARG, "K=%d is not a multiple of group %d", K, group);
+  return LBQ_OK;
+}
+
+static lbq_status check_lut3_shape(int K, int N) {
+  if (K <= 0 || N <= 0) return fail(LBQ_ERR_INVALID_ARG, "K=%d N=%d must be positive", K, N);
+  if (K % 64 || N % 8) return fail(LBQ_ERR_INVALID_ARG, "LUT3 needs K %% 64 == 0 and N %% 8 == 0 (K=%d N=%d)", K, N);
+  return LBQ_OK;
+}
+
+__global__ void write_header_kernel(ImageHeader h, ImageHeader* dst) {
+  if (threadIdx.x == 0) *dst = h;
+}
+
+// Reads the image header (a synchronous 64-byte copy; used by the debug calls only).
+static lbq_status read_header(const void* image, ImageHeader* h) {
+  return cuda_check(cudaMemcpy(h, image, sizeof(ImageHeader), cudaMemcpyDeviceToHost), "reading the image header");
+}
+
+static lbq_status check_header(const ImageHeader& h, int K, int N, int group, int mode) {
+  const uint32_t magic = mode == LBQ_MODE_LUT3 ? kMagicLut3 : kMagicInt4;
+  if (h.magic != magic || h.version != kImageVersion)
+    return fail(LBQ_ERR_INVALID_ARG, "not an lbq image of this version (magic 0x%08x version %u)", h.magic, h.version);
+  if (h.K != K || h.N != N || h.mode != mode || (mode != LBQ_MODE_LUT3 && h.group != group))
+    return fail(LBQ_ERR_INVALID_ARG, "image holds K=%d N=%d group=%d mode=%d, call says K=%d N=%d group=%d mode=%d",
+                h.K, h.N, h.group, h.mode, K, N, group, mode);
+  return LBQ_OK;
+}
+
+// Resident blocks per SM for (kernel, block, dynamic smem). The first time a
+// kernel is seen its dynamic shared-memory limit is raised to the device's
+// opt-in maximum, once, so later calls with any smem size launch.
+static int occupancy_for(const void* fn, int block, int smem) {
+  static std::mutex mu;
+  static std::map<const void*, bool> raised;
+  static std::map<std::pair<const void*, long long>, int> cache;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!raised[fn]) {
+    int dev = 0, optin = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    cudaFuncAttributes fa{};
+    cudaFuncGetAttributes(&fa, fn);
+    cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes);
+    raised[fn] = true;
+  }
+  auto key = std::make_pair(fn, (long long)smem * 4096 + block);
+  auto itc = cache.find(key);
+  if (itc != cache.end()) return itc->second;
+  int occ = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, block, smem);
+  occ = std::max(occ, 1);
+  cache[key] = occ;
+  return occ;
+}
+
+// ----------------------------------------------------------------------------
+// M = 1 GEMV planning
+// ----------------------------------------------------------------------------
+
+struct M1Plan {
+  int splits, cps, cpt, rpt, tpr, phases, R;
+  int nqbox, sbox_w, nsbox, zbox_w, nzbox, off_s, off_z, slot_bytes, tx_bytes, stages;
+  int row_tiles, total_tiles, grid, block, smem;
+};
+
+static int g_force_splits = 0;  // test hook: force a split count (0 = shape-based choice)
+static int g_pdl = 0;           // launch GEMVs with programmatic dependent launch
+static int g_force_skinny = 0;  // test hook: route M = 1 to the tensor-core skinny kernel
+
+constexpr int kM1SlotTarget = 24 * 1024;
+constexpr int kM1RingBudget = 100 * 1024;
+
+static void m1_slot_geometry(M1Plan& p, int group, bool asym) {
+  const int gps = p.cps * 32 / group;  // groups per K-slice
+  p.nqbox = (p.cps * 16 + 255) / 256;
+  p.sbox_w = std::min(256, (gps + 7) / 8 * 8);
+  p.nsbox = (gps + p.sbox_w - 1) / p.sbox_w;
+  p.zbox_w = std::min(256, (gps + 15) / 16 * 16);
+  p.nzbox = asym ? (gps + p.zbox_w - 1) / p.zbox_w : 0;
+  const int qbytes = p.nqbox * p.R * 256;
+  p.off_s = (int)align_up(qbytes, 128);
+  const int sbytes = p.nsbox * p.R * p.sbox_w * 2;
+  p.off_z = (int)align_up(p.off_s + sbytes, 128);
+  const int zbytes = p.nzbox * p.R * p.zbox_w;
+  p.slot_bytes = (int)align_up(p.off_z + zbytes, 1024);
+  p.tx_bytes = qbytes + sbytes + zbytes;
+}
+
+// Shape-based plan: chunk split, threads per row, rows per slot, ring depth, grid.
+static M1Plan plan_m1(int K, int N, int group, bool asym, int force_splits) {
+  const int chunks = K / 32;
+  const int sms = num_sms();
+  const int target = 2 * sms;
+  M1Plan best{};
+  bool have = false;
+  const int max_splits = std::max(1, chunks / 64);
+  for (int splits = 1; splits <= max_splits; ++splits) {
+    if (force_splits > 0 && splits != std::min(force_splits, max_splits)) continue;
+    int cps = chunks;
+    if (splits > 1) cps = ((chunks + splits - 1) / splits + 63) / 64 * 64;  // slice starts on 2048-k boundaries
+    const int real_splits = (chunks + cps - 1) / cps;
+    if (real_splits != splits) continue;
+    const int cpt = cps <= 256 ? 1 : cps <= 512 ? 2 : cps <= 1024 ? 4 : 0;
+    if (cpt == 0) continue;
+    // one chunk per thread keeps the kernel within its register budget: split K instead
+    if (cpt > 1 && splits < max_splits && force_splits == 0) continue;
+    M1Plan p{};
+    p.splits = splits; p.cps = cps; p.cpt = cpt;
+    p.tpr = (((cps + cpt - 1) / cpt) + 31) / 32 * 32;
+    int phases = std::max(1, kM1MaxConsumerThreads / p.tpr);
+    while (phases > 1 && (long long)((N + 8 * phases - 1) / (8 * phases)) * splits < target) phases /= 2;
+    p.phases = phases;
+    const int max_rpt = cpt == 1 ? 8 : cpt == 2 ? 2 : 1;
+    p.rpt = 1;
+    for (int rpt = max_rpt; rpt >= 1; rpt /= 2) {
+      p.rpt = rpt;
+      p.R = rpt * phases;
+      m1_slot_geometry(p, group, asym);
+      if (p.slot_bytes <= kM1SlotTarget || rpt == 1) break;
+    }
+    p.stages = std::max(2, std::min(kM1MaxStages, kM1RingBudget / p.slot_bytes));
+    p.row_tiles = (N + 8 * phases - 1) / (8 * phases);
+    p.total_tiles = p.row_tiles * splits;
+    p.block = p.tpr * phases + 32;
+    p.smem = p.stages * p.slot_bytes + 1024;
+    best = p;
+    have = true;
+    if (force_splits > 0 || (long long)p.total_tiles >= target) break;
+  }
+  if (!have) return best;
+  best.grid = best.total_tiles;  // capped by occupancy at launch
+  return best;
+}
+
+static size_t m1_workspace_bytes(const M1Plan& p, int N) {
+  if (p.splits <= 1) return 0;
+  return align_up((size_t)p.splits * N * sizeof(float), 256) + align_up((size_t)p.row_tiles * sizeof(unsigned), 256);
+}
+
+typedef void (*M1Kernel)(CUtensorMap, CUtensorMap, CUtensorMap, GemvM1Args);
+
+template <bool B, bool A>
+static M1Kernel m1_kernel_for(int cpt, int rpt) {
+  if (cpt == 1) {
+    if (rpt == 8) return gemv_m1_kernel<B, A, 1, 8>;
+    if (rpt == 4) return gemv_m1_kernel<B, A, 1, 4>;
+    if (rpt == 2) return gemv_m1_kernel<B, A, 1, 2>;
+    return gemv_m1_kernel<B, A, 1, 1>;
+  }
+  if (cpt == 2) return rpt == 2 ? gemv_m1_kernel<B, A, 2, 2> : gemv_m1_kernel<B, A, 2, 1>;
+  return gemv_m1_kernel<B, A, 4, 1>;
+}
+
+static M1Kernel m1_kernel(bool bf16, bool asym, int cpt, int rpt) {
+  if (bf16) return asym ? m1_kernel_for<true, true>(cpt, rpt) : m1_kernel_for<true, false>(cpt, rpt);
+  return asym ? m1_kernel_for<false, true>(cpt, rpt) : m1_kernel_for<false, false>(cpt, rpt);
+}
+
+static lbq_status launch_kernel_ex(const void* fn, dim3 grid, dim3 block, int smem, cudaStream_t st, bool pdl,
+                                   void** args, const char* what) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  if (pdl) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  const cudaError_t e = cudaLaunchKernelExC(&cfg, fn, args);
+  if (e != cudaSuccess)
+    return fail(LBQ_ERR_CUDA, "%s (grid %u, block %u, smem %d, pdl %d): %s", what, grid.x, block.x, smem, (int)pdl,
+                cudaGetErrorString(e));
+  return LBQ_OK;
+}
+
+static lbq_status run_m1(const uint16_t* X, bool xbf16, const void* image, const Layout& L, void* Y, bool ybf16,
+                         void* ws, size_t ws_bytes, cudaStream_t st) {
+  const bool asym = L.mode == LBQ_MODE_ASYM;
+  M1Plan p = plan_m1(L.K, L.N, L.group, asym, g_force_splits);
+  if (p.block == 0) return fail(LBQ_ERR_UNSUPPORTED, "no GEMV plan for K=%d", L.K);
+  const size_t need = m1_workspace_bytes(p, L.N);
+  if (need > 0 && (ws == nullptr || ws_bytes < need))
+    return fail(LBQ_ERR_INVALID_ARG, "workspace of %zu bytes is too small (need %zu)", ws_bytes, need);
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  const int G = L.K / L.group;
+  CUtensorMap tq, ts, tz;
+  if (!make_tmap_2d(&tq, img + L.off0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.K / 2, (uint64_t)L.N,
+                    (uint64_t)L.K / 2, 256, (uint32_t)p.R, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&ts, img + L.off1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)G, (uint64_t)L.N, L.s_stride,
+                    (uint32_t)p.sbox_w, (uint32_t)p.R, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the GEMV tiles");
+  tz = ts;
+  if (asym && !make_tmap_2d(&tz, img + L.off2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)G, (uint64_t)L.N,
+                            L.z_stride, (uint32_t)p.zbox_w, (uint32_t)p.R, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the zero points");
+  GemvM1Args a{};
+  a.X = X;
+  a.Y = Y;
+  a.partials = need ? static_cast<float*>(ws) : nullptr;
+  a.counters = need ? reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + align_up((size_t)p.splits * L.N * sizeof(float), 256)) : nullptr;
+  a.K = L.K; a.N = L.N; a.gshift = log2_exact(L.group / 32);
+  a.cps = p.cps; a.splits = p.splits; a.tpr = p.tpr; a.phases = p.phases; a.rows_per_stage = p.R;
+  a.stages = p.stages; a.nqbox = p.nqbox; a.sbox_w = p.sbox_w; a.nsbox = p.nsbox; a.zbox_w = p.zbox_w;
+  a.nzbox = p.nzbox; a.off_s = p.off_s; a.off_z = p.off_z; a.slot_bytes = p.slot_bytes; a.tx_bytes = p.tx_bytes;
+  a.row_tiles = p.row_tiles; a.total_tiles = p.total_tiles; a.y_bf16 = ybf16 ? 1 : 0;
+  M1Kernel fn = m1_kernel(xbf16, asym, p.cpt, p.rpt);
+  const int occ = occupancy_for((const void*)fn, p.block, p.smem);
+  const int grid = std::min(p.total_tiles, num_sms() * occ);
+  void* args[] = {&tq, &ts, &tz, &a};
+  return launch_kernel_ex((const void*)fn, dim3(grid), dim3(p.block), p.smem, st, g_pdl != 0, args, "gemv_m1 launch");
+}
+
+// ----------------------------------------------------------------------------
+// 2 <= M <= 16: tensor-core skinny kernel
+// ----------------------------------------------------------------------------
+
+struct SkPlan {
+  int nt, gc, row_tiles, total_stages, sps, splits, total_tiles, smem, slot;
+};
+
+static SkPlan plan_skinny(int K, int N, int M, int group, bool asym, int force_splits) {
+  SkPlan p{};
+  p.nt = M <= 8 ? 1 : 2;
+  p.gc = group / 32;
+  p.row_tiles = (N + kSkRows - 1) / kSkRows;
+  p.total_stages = (K + 255) / 256;
+  const int target = 2 * num_sms();
+  int splits = 1;
+  if (force_splits > 0) splits = std::min(force_splits, p.total_stages);
+  else
+    while (p.row_tiles * splits < target && splits < p.total_stages) ++splits;
+  p.sps = (p.total_stages + splits - 1) / splits;
+  p.splits = (p.total_stages + p.sps - 1) / p.sps;
+  p.total_tiles = p.row_tiles * p.splits;
+  p.slot = kSkWBytes + 4 * p.nt * 1024 + kSkSBytes + (asym ? kSkZBytes : 0);
+  p.smem = kSkStages * p.slot + 1024;
+  return p;
+}
+
+static size_t skinny_workspace_bytes(const SkPlan& p, int M, int N) {
+  if (p.splits <= 1) return 0;
+  return align_up((size_t)p.splits * M * N * sizeof(float), 256) + align_up((size_t)p.row_tiles * sizeof(unsigned), 256);
+}
+
+typedef void (*SkKernel)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, SkinnyArgs);
+
+template <bool B, bool A, int NT, bool KF>
+static SkKernel sk_for_gc(int gc) {
+  if (gc == 1) return skinny_kernel<B, A, NT, 1, KF>;
+  if (gc == 2) return skinny_kernel<B, A, NT, 2, KF>;
+  return skinny_kernel<B, A, NT, 4, KF>;
+}
+
+template <bool B, bool A>
+static SkKernel sk_for_nt(int nt, int gc, bool kfull) {
+  if (nt == 1) return kfull ? sk_for_gc<B, A, 1, true>(gc) : sk_for_gc<B, A, 1, false>(gc);
+  return kfull ? sk_for_gc<B, A, 2, true>(gc) : sk_for_gc<B, A, 2, false>(gc);
+}
+
+static SkKernel sk_kernel(bool bf16, bool asym, int nt, int gc, bool kfull) {
+  if (bf16) return asym ? sk_for_nt<true, true>(nt, gc, kfull) : sk_for_nt<true, false>(nt, gc, kfull);
+  return asym ? sk_for_nt<false, true>(nt, gc, kfull) : sk_for_nt<false, false>(nt, gc, kfull);
+}
+
+static lbq_status run_skinny(const void* X, bool xbf16, int M, const void* image, const Layout& L, void* Y,
+                             bool ybf16, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const bool asym = L.mode == LBQ_MODE_ASYM;
+  const SkPlan p = plan_skinny(L.K, L.N, M, L.group, asym, g_force_splits);
+  const size_t need = skinny_workspace_bytes(p, M, L.N);
+  if (need > 0 && (ws == nullptr || ws_bytes < need))
+    return fail(LBQ_ERR_INVALID_ARG, "workspace of %zu bytes is too small (need %zu)", ws_bytes, need);
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  const int G = L.K / L.group;
+  CUtensorMap tw, tx, ts, tz;
+  bool ok = make_tmap_2d(&tw, img + L.off0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.K / 2, (uint64_t)L.N,
+                         (uint64_t)L.K / 2, 128, kSkRows, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)L.K, (uint64_t)M, (uint64_t)L.K * 2, 64,
+                         (uint32_t)M, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            make_tmap_2d(&ts, img + L.off1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)G, (uint64_t)L.N, L.s_stride,
+                         8, kSkRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+  tz = ts;
+  if (ok && asym)
+    ok = make_tmap_2d(&tz, img + L.off2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)G, (uint64_t)L.N, L.z_stride,
+                      16, kSkRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!ok) return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the skinny kernel");
+  SkinnyArgs a{};
+  a.Y = Y;
+  a.partials = need ? static_cast<float*>(ws) : nullptr;
+  a.counters = need ? reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) +
+                                                  align_up((size_t)p.splits * M * L.N * sizeof(float), 256)) : nullptr;
+  a.K = L.K; a.N = L.N; a.M = M;
+  a.stages_per_split = p.sps; a.splits = p.splits; a.row_tiles = p.row_tiles; a.total_tiles = p.total_tiles;
+  a.y_bf16 = ybf16 ? 1 : 0;
+  SkKernel fn = sk_kernel(xbf16, asym, p.nt, p.gc, L.K % 256 == 0);
+  const int occ = occupancy_for((const void*)fn, kSkThreads, p.smem);
+  const int grid = std::min(p.total_tiles, num_sms() * occ);
+  void* args[] = {&tw, &tx, &ts, &tz, &a};
+  return launch_kernel_ex((const void*)fn, dim3(grid), dim3(kSkThreads), p.smem, st, g_pdl != 0, args,
+                          "skinny launch");
+}
+
+// ----------------------------------------------------------------------------
+// M > 16: tcgen05 prefill GEMM
+// ----------------------------------------------------------------------------
+
+static int g_force_tc = 0;  // test hook: route every lbq_gemm call to the tcgen05 kernel
+
+static lbq_status run_gemm_tc(const void* X, bool xbf16, int M, const void* image, const Layout& L, void* Y,
+                              bool ybf16, cudaStream_t st) {
+  const bool asym = L.mode == LBQ_MODE_ASYM;
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  const int G = L.K / L.group;
+  CUtensorMap tx, tq, ts, tz;
+  bool ok = make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)L.K, (uint64_t)M, (uint64_t)L.K * 2,
+                         kTcBK, kTcBM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            make_tmap_2d(&tq, img + L.off0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.K / 2, (uint64_t)L.N,
+                         (uint64_t)L.K / 2, kTcBK / 2, kTcBN, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+            make_tmap_2d(&ts, img + L.off1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)G, (uint64_t)L.N, L.s_stride,
+                         8, kTcBN, CU_TENSOR_MAP_SWIZZLE_NONE);
+  tz = ts;
+  if (ok && asym)
+    ok = make_tmap_2d(&tz, img + L.off2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)G, (uint64_t)L.N, L.z_stride,
+                      16, kTcBN, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!ok) return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the prefill GEMM");
+  GemmTcArgs a{};
+  a.Y = Y;
+  a.M = M; a.N = L.N; a.K = L.K; a.gshift64 = log2_exact(L.group / 32);
+  a.m_tiles = (M + kTcBM - 1) / kTcBM;
+  a.n_tiles = (L.N + kTcBN - 1) / kTcBN;
+  a.k_blocks = (L.K + kTcBK - 1) / kTcBK;
+  a.y_bf16 = ybf16 ? 1 : 0;
+  const void* fn = xbf16 ? (asym ? (const void*)gemm_tc_kernel<true, true> : (const void*)gemm_tc_kernel<true, false>)
+                         : (asym ? (const void*)gemm_tc_kernel<false, true> : (const void*)gemm_tc_kernel<false, false>);
+  occupancy_for(fn, kTcThreads, kTcSmem);
+  const int grid = std::min(a.m_tiles * a.n_tiles, num_sms());
+  void* args[] = {&tx, &tq, &ts, &tz, &a};
+  return launch_kernel_ex(fn, dim3(grid), dim3(kTcThreads), kTcSmem, st, false, args, "prefill GEMM launch");
+}
+
+static lbq_status check_compute_args(const void* X, int x_dtype, int M, const void* image, void* Y, int y_dtype) {
+  if (!X || !image || !Y) return fail(LBQ_ERR_INVALID_ARG, "X, image and Y must be non-null");
+  if (!aligned16(X) || !aligned16(image) || !aligned16(Y))
+    return fail(LBQ_ERR_INVALID_ARG, "X, image and Y must be 16-byte aligned");
+  if (x_dtype != LBQ_DTYPE_F16 && x_dtype != LBQ_DTYPE_BF16) return fail(LBQ_ERR_UNSUPPORTED, "x_dtype %d", x_dtype);
+  if (y_dtype != LBQ_DTYPE_F16 && y_dtype != LBQ_DTYPE_BF16) return fail(LBQ_ERR_UNSUPPORTED, "y_dtype %d", y_dtype);
+  if (M <= 0) return fail(LBQ_ERR_INVALID_ARG, "M=%d must be positive", M);
+  return LBQ_OK;
+}
+
+}  // namespace lbq
+
+using namespace lbq;
+
+extern "C" {
+
+const char* lbq_last_error(void) { return g_last_error.c_str(); }
+
+int lbq_version(void) { return 100; }
+
+uint64_t lbq_launch_count(void) { return g_launches.load(); }
+
+// Test hook (not in the public header): force the split-K count of the M = 1
+// GEMV; 0 restores the shape-based choice.
+void lbq_debug_force_splits(int splits) { g_force_splits = splits < 0 ? 0 : splits; }
+
+// Test hook (not in the public header): route every lbq_gemm call, any M, to
+// the tcgen05 prefill kernel.
+void lbq_debug_force_tc(int on) { g_force_tc = on ? 1 : 0; }
+
+// Test hook (not in the public header): route M = 1 through the skinny kernel.
+void lbq_debug_force_skinny(int on) { g_force_skinny = on ? 1 : 0; }
+
+lbq_status lbq_set_option(int option, int value) {
+  if (option == LBQ_OPT_PDL) {
+    g_pdl = value ? 1 : 0;
+    return LBQ_OK;
+  }
+  return fail(LBQ_ERR_INVALID_ARG, "unknown option %d", option);
+}
+
+lbq_status lbq_packed_size(int K, int N, int group, int mode, size_t* bytes) {
+  if (!bytes) return fail(LBQ_ERR_INVALID_ARG, "bytes must be non-null");
+  lbq_status st = mode == LBQ_MODE_LUT3 ? check_lut3_shape(K, N) : check_int4_shape(K, N, group, mode);
+  if (st != LBQ_OK) return st;
+  *bytes = make_layout(K, N, mode == LBQ_MODE_LUT3 ? 0 : group, mode).total;
+  return LBQ_OK;
+}
+
+lbq_status lbq_pack(const float* W, int K, int N, int group, int mode, void* image, size_t image_bytes, void* stream) {
+  lbq_status st = check_int4_shape(K, N, group, mode);
+  if (st != LBQ_OK) return st;
+  if (!W || !image) return fail(LBQ_ERR_INVALID_ARG, "W and image must be non-null");
+  if (!aligned16(W) || !aligned16(image)) return fail(LBQ_ERR_INVALID_ARG, "W and image must be 16-byte aligned");
+  const Layout L = make_layout(K, N, group, mode);
+  if (image_bytes < L.total) return fail(LBQ_ERR_INVALID_ARG, "image buffer %zu bytes < %zu needed", image_bytes, L.total);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* img = static_cast<uint8_t*>(image);
+  write_header_kernel<<<1, 32, 0, s>>>(make_header(L), reinterpret_cast<ImageHeader*>(img));
+  if ((st = launch_check("header launch")) != LBQ_OK) return st;
+  // zero the scale / zero-point regions so their row padding is deterministic
+  if ((st = cuda_check(cudaMemsetAsync(img + L.off1, 0, L.total - L.off1, s), "clearing the scale regions")) != LBQ_OK)
+    return st;
+  const long long work = (long long)(K / group) * N;
+  const int block = 256;
+  const unsigned grid = (unsigned)((work + block - 1) / block);
+  if (mode == LBQ_MODE_SYM)
+    quantize_pack_int4_kernel<false><<<grid, block, 0, s>>>(W, K, N, group, img + L.off0, img + L.off1, nullptr,
+                                                             (int)L.s_stride, (int)L.z_stride);
+  else
+    quantize_pack_int4_kernel<true><<<grid, block, 0, s>>>(W, K, N, group, img + L.off0, img + L.off1, img + L.off2,
+                                                            (int)L.s_stride, (int)L.z_stride);
+  return launch_check("quantize_pack launch");
+}
+
+lbq_status lbq_pack_lut3(const uint8_t* idx, const uint8_t* codebooks, const uint8_t* exponents, int K, int N,
+                         void* image, size_t image_bytes, void* stream) {
+  (void)idx; (void)codebooks; (void)exponents; (void)K; (void)N; (void)image; (void)image_bytes; (void)stream;
+  return fail(LBQ_ERR_UNSUPPORTED, "LUT3 packing is not built yet");
+}
+
+lbq_status lbq_workspace_size(int op, int M, int K, int N, int group, int mode, size_t* bytes) {
+  if (!bytes) return fail(LBQ_ERR_INVALID_ARG, "bytes must be non-null");
+  *bytes = 0;
+  if (op == 0 || op == 1) {
+    lbq_status st = check_int4_shape(K, N, group, mode);
+    if (st != LBQ_OK) return st;
+    if (M <= 0) return fail(LBQ_ERR_INVALID_ARG, "M must be positive");
+    if (op == 1 && (M > 16 || g_force_tc)) return LBQ_OK;  // the prefill GEMM needs no workspace
+    if (M == 1 && !g_force_skinny) {
+      const M1Plan p = plan_m1(K, N, group, mode == LBQ_MODE_ASYM, g_force_splits);
+      *bytes = m1_workspace_bytes(p, N);
+    } else if (M <= 16) {
+      const SkPlan p = plan_skinny(K, N, M, group, mode == LBQ_MODE_ASYM, g_force_splits);
+      *bytes = skinny_workspace_bytes(p, M, N);
+    }
+    return LBQ_OK;
+  }
+  if (op == 2) return check_lut3_shape(K, N);
+  return fail(LBQ_ERR_INVALID_ARG, "op %d not in {0, 1, 2}", op);
+}
+
+lbq_status lbq_gemv(const void* X, int x_dtype, int M, int K, int N, int group, int mode, const void* image, void* Y,
+                    int y_dtype, void* ws, size_t ws_bytes, void* stream) {
+  lbq_status st = check_int4_shape(K, N, group, mode);
+  if (st != LBQ_OK) return st;
+  if ((st = check_compute_args(X, x_dtype, M, image, Y, y_dtype)) != LBQ_OK) return st;
+  if (M > 16) return fail(LBQ_ERR_UNSUPPORTED, "lbq_gemv takes M <= 16 (M=%d); use lbq_gemm", M);
+  const Layout L = make_layout(K, N, group, mode);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 1 && !g_force_skinny)
+    return run_m1(static_cast<const uint16_t*>(X), x_dtype == LBQ_DTYPE_BF16, image, L, Y, y_dtype == LBQ_DTYPE_BF16,
+                  ws, ws_bytes, s);
+  return run_skinny(X, x_dtype == LBQ_DTYPE_BF16, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, ws, ws_bytes, s);
+}
+
+lbq_status lbq_gemm(const void* X, int x_dtype, int M, int K, int N, int group, int mode, const void* image, void* Y,
+                    int y_dtype, void* ws, size_t ws_bytes, void* stream) {
+  if (M <= 16 && !g_force_tc) return lbq_gemv(X, x_dtype, M, K, N, group, mode, image, Y, y_dtype, ws, ws_bytes, stream);
+  lbq_status st = check_int4_shape(K, N, group, mode);
+  if (st != LBQ_OK) return st;
+  if ((st = check_compute_args(X, x_dtype, M, image, Y, y_dtype)) != LBQ_OK) return st;
+  return run_gemm_tc(X, x_dtype == LBQ_DTYPE_BF16, M, image, make_layout(K, N, group, mode), Y,
+                     y_dtype == LBQ_DTYPE_BF16, static_cast<cudaStream_t>(stream));
+}
+
+lbq_status lbq_lut3_gemm(const void* X, int x_dtype, int M, int K, int N, const void* image, void* Y, int y_dtype,
+                         void* ws, size_t ws_bytes, void* stream) {
+  (void)X; (void)x_dtype; (void)M; (void)K; (void)N; (void)image; (void)Y; (void)y_dtype; (void)ws; (void)ws_bytes; (void)stream;
+  return fail(LBQ_ERR_UNSUPPORTED, "the LUT3 kernels are not built yet");
+}
+
+lbq_status lbq_unpack_canonical(const void* image, int K, int N, int group, int mode, uint8_t* q_packed,
+                                uint16_t* scales, int8_t* zp, void* stream) {
+  lbq_status st = check_int4_shape(K, N, group, mode);
+  if (st != LBQ_OK) return st;
+  if (!image || !q_packed || !scales) return fail(LBQ_ERR_INVALID_ARG, "image, q_packed and scales must be non-null");
+  if (mode == LBQ_MODE_ASYM && !zp) return fail(LBQ_ERR_INVALID_ARG, "zp must be non-null for ASYM");
+  ImageHeader h;
+  if ((st = read_header(image, &h)) != LBQ_OK) return st;
+  if ((st = check_header(h, K, N, group, mode)) != LBQ_OK) return st;
+  const Layout L = make_layout(K, N, group, mode);
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  const long long work = (long long)(K / 2) * N;
+  unpack_int4_kernel<<<(unsigned)((work + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      img + L.off0, img + L.off1, mode == LBQ_MODE_ASYM ? img + L.off2 : nullptr, K, N, group, (int)L.s_stride,
+      (int)L.z_stride, q_packed, scales, mode == LBQ_MODE_ASYM ? zp : nullptr);
+  return launch_check("unpack launch");
+}
+
+lbq_status lbq_unpack_lut3_canonical(const void* image, int K, int N, uint8_t* idx_stream, uint8_t* codebooks,
+                                     uint8_t* exponents, void* stream) {
+  (void)image; (void)K; (void)N; (void)idx_stream; (void)codebooks; (void)exponents; (void)stream;
+  return fail(LBQ_ERR_UNSUPPORTED, "LUT3 is not built yet");
+}
+
+lbq_status lbq_dequant(const void* image, int K, int N, int group, int mode, float* W_out, void* stream) {
+  lbq_status st = mode == LBQ_MODE_LUT3 ? check_lut3_shape(K, N) : check_int4_shape(K, N, group, mode);
+  if (st != LBQ_OK) return st;
+  if (!image || !W_out) return fail(LBQ_ERR_INVALID_ARG, "image and W_out must be non-null");
+  ImageHeader h;
+  if ((st = read_header(image, &h)) != LBQ_OK) return st;
+  if ((st = check_header(h, K, N, group, mode)) != LBQ_OK) return st;
+  if (mode == LBQ_MODE_LUT3) return fail(LBQ_ERR_UNSUPPORTED, "LUT3 is not built yet");
+  const Layout L = make_layout(K, N, group, mode);
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  const long long work = (long long)K * N;
+  dequant_int4_kernel<<<(unsigned)((work + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      img + L.off0, img + L.off1, mode == LBQ_MODE_ASYM ? img + L.off2 : nullptr, K, N, group, (int)L.s_stride,
+      (int)L.z_stride, W_out);
+  return launch_check("dequant launch");
+}
+
+lbq_status lbq_device_status(void* stream) {
+  lbq_status st = cuda_check(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)), "stream synchronize");
+  if (st != LBQ_OK) return st;
+  unsigned int v = 0;
+  const unsigned int zero = 0;
+  if ((st = cuda_check(cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)), "reading the device flag")) != LBQ_OK) return st;
+  if (v == 0) return LBQ_OK;
+  if ((st = cuda_check(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)), "clearing the device flag")) != LBQ_OK) return st;
+  return fail(LBQ_ERR_DEVICE, "a kernel reported device error flags 0x%x", v);
+}
+
+}  // extern "C"

@@ -1,0 +1,204 @@
+/*
+ * lbq.h -- low-bit weight-only GEMV / GEMM for NVIDIA B200 (sm_100a).
+ *
+ * The operation (problem statement of "Low Bit Metal Kernels", INT4 dequant +
+ * matmul listing):  Y[M, N] = X[M, K] . dequant(Wq)[K, N],
+ * X and Y row-major FP16 or BF16, FP32 accumulation, Y rounded to nearest.
+ *
+ * Two weight formats:
+ *  - INT4, two codes per byte, one FP16 scale per group of `group` (32, 64,
+ *    128) consecutive k of a column, symmetric value (q - 8) * s or asymmetric
+ *    value (q - zp) * s with an int8 zero point ("Low Bit Metal Kernels",
+ *    dequant lines of the INT4 listing; "Low Bit ARM kernels", group-wise
+ *    scale section).
+ *  - LUT3: a 3-bit index into an 8-entry E4M3 codebook shared by a tile of 8
+ *    output channels x 64 k, times one UE8M0 exponent 2^(E-127) per tile
+ *    (vLLM PR 62759 write-up, format section).
+ *
+ * Conventions for every call:
+ *  - Pointers marked (device) are CUDA device pointers, (host) host pointers.
+ *    The caller owns and allocates every buffer; the library never allocates
+ *    device memory and keeps no pointer after a call returns.
+ *  - Calls that take a `stream` only enqueue work on it (cudaStream_t passed as
+ *    void*, 0 = legacy default stream) and return without synchronising. They
+ *    are safe to capture in a CUDA graph.
+ *  - Every call returns an lbq_status. On failure nothing is enqueued and
+ *    lbq_last_error() (thread-local) describes the cause. The library never
+ *    throws, aborts or exits.
+ *  - Compute calls trust that K, N, group and mode match the image (checking
+ *    the device header would cost a dependent memory round trip per launch);
+ *    the debug calls (unpack / dequant) do read and check the header.
+ *  - A kernel that detects a problem on the device (a pipeline wait that ran
+ *    past its bound) abandons its work and raises a flag that
+ *    lbq_device_status() reports; no kernel waits without a bound.
+ *  - Device pointers must be 16-byte aligned; K, N, M must be > 0 unless stated.
+ *
+ * The device image (what lbq_pack / lbq_pack_lut3 write) is an opaque blob of
+ * lbq_packed_size() bytes: a 256-byte header followed by the repacked codes,
+ * scales and zero points (or LUT3 indices, codebooks and exponents). Its
+ * layout is fixed by this library version; lbq_unpack_canonical /
+ * lbq_unpack_lut3_canonical recover the canonical arrays from it bit-exactly.
+ */
+#ifndef LBQ_H
+#define LBQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LBQ_OK = 0,
+  LBQ_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, buffer too small */
+  LBQ_ERR_UNSUPPORTED = 2,  /* a combination this version does not implement */
+  LBQ_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  LBQ_ERR_DEVICE = 4        /* a kernel reported a problem (lbq_device_status) */
+} lbq_status;
+
+typedef enum { LBQ_MODE_SYM = 0, LBQ_MODE_ASYM = 1, LBQ_MODE_LUT3 = 2 } lbq_mode;
+typedef enum { LBQ_DTYPE_F16 = 0, LBQ_DTYPE_BF16 = 1 } lbq_dtype;
+
+/* Human-readable description of the last failure on the calling thread. */
+const char* lbq_last_error(void);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int lbq_version(void);
+
+/*
+ * Size in bytes of the device image for a K x N weight in `mode`.
+ * INT4 (SYM/ASYM): group in {32, 64, 128}, K % group == 0, N >= 1.
+ * LUT3: group is ignored (pass 0), K % 64 == 0, N % 8 == 0.
+ * Writes *bytes (host). No device work.
+ */
+lbq_status lbq_packed_size(int K, int N, int group, int mode, size_t* bytes);
+
+/*
+ * Quantise and repack an FP32 weight into the device image (INT4 only).
+ *   W      (device) float32 [K, N] row-major, the logical weight of Y = X . W.
+ *   image  (device) lbq_packed_size() bytes, written entirely.
+ * Quantisation ("Low Bit ARM kernels", group-wise scale section; formulas of
+ * the INT4 listing in "Low Bit Metal Kernels"), per group of `group` k of a
+ * column n, all in IEEE FP32 with round-half-to-even:
+ *   SYM : s = fp16(max|w| / 7);           q = clamp(rint(w / s) + 8, 0, 15)
+ *   ASYM: s = fp16((max w - min w) / 15); zp = clamp(rint(-min w / s), -128, 127);
+ *         q = clamp(rint(w / s) + zp, 0, 15)
+ * where s in the divisions is the stored FP16 scale widened to FP32; a group
+ * whose stored scale is 0 gets q = 8 (SYM) or zp = 0, q = 0 (ASYM).
+ * W must be finite. Asynchronous on `stream`.
+ */
+lbq_status lbq_pack(const float* W, int K, int N, int group, int mode,
+                    void* image, size_t image_bytes, void* stream);
+
+/*
+ * Build a LUT3 device image from the format's canonical arrays (vLLM PR 62759
+ * write-up, format section).
+ *   idx        (device) uint8 [K, N], values 0..7 (weight (k, n)'s index)
+ *   codebooks  (device) uint8 [K/64, N/8, 8]  E4M3 ("fn") bytes per tile
+ *   exponents  (device) uint8 [K/64, N/8]     UE8M0 bytes per tile (bias 127)
+ * Weight value = e4m3(codebooks[k/64][n/8][idx[k][n]]) * 2^(exponents[k/64][n/8] - 127).
+ * Indices > 7 are taken modulo 8; NaN codebook bytes (0x7F/0xFF) and NaN
+ * exponents (0xFF) are the caller's responsibility (they decode to NaN).
+ * Asynchronous on `stream`.
+ */
+lbq_status lbq_pack_lut3(const uint8_t* idx, const uint8_t* codebooks, const uint8_t* exponents,
+                         int K, int N, void* image, size_t image_bytes, void* stream);
+
+/*
+ * Workspace needed by lbq_gemv / lbq_gemm / lbq_lut3_gemm for this shape:
+ * the split-K partial sums and tile counters of the dispatch the library
+ * would pick. op: 0 = lbq_gemv, 1 = lbq_gemm, 2 = lbq_lut3_gemm.
+ * Writes *bytes (host); 0 means the call needs no workspace (ws may be null).
+ * A workspace must be zero-filled before its first use; every call leaves it
+ * zero-filled again, so one buffer can be reused by consecutive calls on one
+ * stream (not by calls running concurrently).
+ */
+lbq_status lbq_workspace_size(int op, int M, int K, int N, int group, int mode, size_t* bytes);
+
+/*
+ * Decode GEMV / skinny GEMM on INT4 weights, 1 <= M <= 16.
+ *   X      (device) [M, K] row-major, x_dtype (LBQ_DTYPE_F16 / BF16)
+ *   image  (device) from lbq_pack with the same K, N, group, mode
+ *   Y      (device) [M, N] row-major, y_dtype, fully overwritten
+ *   ws     (device) >= lbq_workspace_size(0, ...) bytes, zero-filled (see above)
+ * y[m][n] = sum_k x[m][k] * (q[k][n] - z) * s[k/group][n], accumulated in FP32
+ * ("Low Bit ARM kernels": decode at batch 1 is a GEMV; the page's Metal
+ * kernel does the dequantisation inside the inner loop). Asynchronous.
+ */
+lbq_status lbq_gemv(const void* X, int x_dtype, int M, int K, int N, int group, int mode,
+                    const void* image, void* Y, int y_dtype, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/*
+ * Prefill GEMM on INT4 weights, any M >= 1 (M <= 16 is routed to lbq_gemv's
+ * kernels). Same arguments and result as lbq_gemv. Weights are dequantised
+ * to BF16 in shared memory and multiplied on the tensor cores; X must be BF16
+ * for M > 16. Asynchronous.
+ */
+lbq_status lbq_gemm(const void* X, int x_dtype, int M, int K, int N, int group, int mode,
+                    const void* image, void* Y, int y_dtype, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/*
+ * GEMV / GEMM on LUT3 weights (image from lbq_pack_lut3), any M >= 1.
+ * X must be BF16. y[m][n] = sum_k x[m][k] * w[k][n] with w the decoded
+ * LUT3 value (exact in BF16 for the exponents the format's workloads use).
+ */
+lbq_status lbq_lut3_gemm(const void* X, int x_dtype, int M, int K, int N,
+                         const void* image, void* Y, int y_dtype, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/*
+ * Debug / parity: recover the canonical arrays from an INT4 image.
+ *   q_packed (device) uint8 [K/2, N]: byte[j][n] = q[2j][n] | q[2j+1][n] << 4
+ *   scales   (device) uint16 [K/group, N]: FP16 bit patterns
+ *   zp       (device) int8 [K/group, N] (ASYM; may be null, ignored for SYM)
+ */
+lbq_status lbq_unpack_canonical(const void* image, int K, int N, int group, int mode,
+                                uint8_t* q_packed, uint16_t* scales, int8_t* zp, void* stream);
+
+/*
+ * Debug / parity: recover the canonical LUT3 arrays from a LUT3 image.
+ *   idx_stream (device) uint8 [K/64, N/8, 8, 24]: per tile and channel, the 64
+ *              indices as a little-endian 192-bit string, index i in bits [3i, 3i+3)
+ *   codebooks  (device) uint8 [K/64, N/8, 8];  exponents (device) uint8 [K/64, N/8]
+ */
+lbq_status lbq_unpack_lut3_canonical(const void* image, int K, int N, uint8_t* idx_stream,
+                                     uint8_t* codebooks, uint8_t* exponents, void* stream);
+
+/*
+ * Debug / parity: the exact dequantised weight, W_out (device) float32 [K, N].
+ * INT4: (q - z) * s; LUT3: e4m3(cb) * 2^(E-127). Both are exact in FP32.
+ */
+lbq_status lbq_dequant(const void* image, int K, int N, int group, int mode,
+                       float* W_out, void* stream);
+
+/*
+ * Synchronise `stream` and report (then clear) the device-side error flag the
+ * kernels raise on this device: LBQ_OK, or LBQ_ERR_DEVICE with the reason in
+ * lbq_last_error().
+ */
+lbq_status lbq_device_status(void* stream);
+
+/*
+ * Process-wide launch options.
+ *   LBQ_OPT_PDL (value 0/1, default 0): launch the GEMV kernels with
+ *   programmatic dependent launch. A kernel may then start, and stream its
+ *   weight image, while the previous kernel in the stream is still running;
+ *   it reads X and writes Y only after that kernel has completed. Enable it
+ *   only when no preceding kernel in the stream writes the image (images are
+ *   normally written once by lbq_pack and then only read), e.g. for the
+ *   back-to-back projections of a decode step.
+ */
+typedef enum { LBQ_OPT_PDL = 1 } lbq_option;
+lbq_status lbq_set_option(int option, int value);
+
+/* Number of kernel launches the library has enqueued so far in this process. */
+uint64_t lbq_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LBQ_H */

@@ -1,0 +1,252 @@
+"""INT4 parity on the GPU: packing and dequantisation bit-exact against the
+oracle, GEMV outputs within |y - y_ref| <= 4e-3*S + ulp16(|y_ref|)."""
+
+import numpy as np
+import pytest
+
+import workloads
+from helpers import check_outputs, oracle_int4, sample_columns
+from oracle import int4
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch():
+    import torch
+    assert torch.cuda.is_available(), "these tests need a CUDA device"
+    return torch
+
+
+@pytest.fixture(scope="module")
+def lbq():
+    import bit_weight_only_pack_b200 as lbq
+    return lbq
+
+
+def _special_groups(W, group):
+    """Plant the degenerate and one-sided groups the quantiser has to handle."""
+    K, N = W.shape
+    if N >= 4 and K >= 2 * group:
+        W[:group, 0] = 0.0                                   # all-zero group
+        W[group:2 * group, 1] = 0.37                         # constant group
+        W[:group, 2] = np.abs(W[:group, 2]) + 0.01           # all-positive group
+        W[group:2 * group, 3] = -np.abs(W[group:2 * group, 3]) - 0.5  # all-negative, far from 0
+    return W
+
+
+def _pack_and_compare(torch, lbq, W, group, mode):
+    K, N = W.shape
+    ref = oracle_int4(W, group, mode)
+    img = lbq.pack(torch.from_numpy(W).cuda(), group, mode)
+    q, s, z = lbq.unpack_canonical(img, K, N, group, mode)
+    assert np.array_equal(q.cpu().numpy(), ref["packed"])
+    assert np.array_equal(s.cpu().view(torch.int16).numpy(), ref["s"].view(np.int16))
+    if mode == "asym":
+        assert np.array_equal(z.cpu().numpy(), ref["zp"])
+    deq = lbq.dequant(img, K, N, group, mode).cpu().numpy()
+    assert np.array_equal(deq.astype(np.float64), ref["deq"])
+    return img, ref
+
+
+SHAPES = [
+    (4096, 4096, 32, "sym"),     # the single-GEMV workload
+    (4096, 1024, 32, "asym"),    # k/v projection of the decode step
+    (14336, 64, 32, "asym"),     # down projection, a column slice
+    (96, 40, 32, "asym"),        # three chunks, ragged N
+    (128, 8, 64, "sym"),
+    (256, 24, 128, "asym"),
+    (32, 1, 32, "sym"),          # one chunk, one column
+]
+
+
+@pytest.mark.parametrize("K,N,group,mode", SHAPES)
+def test_pack_and_dequant_bit_exact(torch, lbq, K, N, group, mode):
+    W = _special_groups(workloads.weights_host(11 + K + N, K, N), group)
+    _pack_and_compare(torch, lbq, W, group, mode)
+
+
+def test_pack_outliers_bit_exact(torch, lbq):
+    W = workloads.weights_host(3, 1024, 512, outlier_frac=1e-3, outlier_mult=20.0)
+    for group in (64, 128):
+        _pack_and_compare(torch, lbq, W, group, "sym")
+
+
+@pytest.mark.parametrize("K,N,group,mode", SHAPES)
+@pytest.mark.parametrize("xdt", ["f16", "bf16"])
+def test_gemv_m1_parity(torch, lbq, K, N, group, mode, xdt):
+    W = _special_groups(workloads.weights_host(11 + K + N, K, N), group)
+    img, ref = _pack_and_compare(torch, lbq, W, group, mode)
+    X = workloads.activations_host(5 + K, 1, K, xdt)
+    for ydt in ("f16", "bf16"):
+        Y = lbq.gemv(X.cuda(), img, N, group, mode, y_dtype=ydt)
+        torch.cuda.synchronize()
+        check_outputs(Y.cpu(), X, ref["deq"])
+
+
+@pytest.mark.parametrize("splits", [2, 3, 4, 7])
+def test_gemv_m1_forced_split_k(torch, lbq, splits):
+    K, N, group, mode = 14336, 1000, 32, "asym"   # K-slices start on 2048-k boundaries
+    W = workloads.weights_host(77, K, N)
+    img, ref = _pack_and_compare(torch, lbq, W, group, mode)
+    X = workloads.activations_host(77, 1, K, "f16")
+    lbq.lbq_debug_force_splits(splits)
+    try:
+        ws = lbq.workspace(0, 1, K, N, group, mode)
+        assert ws is not None and int(ws.count_nonzero()) == 0
+        Ys = [lbq.gemv(X.cuda(), img, N, group, mode, ws=ws) for _ in range(3)]
+        torch.cuda.synchronize()
+        counters_at = -(-splits * N * 4 // 256) * 256
+        assert int(ws[counters_at:].count_nonzero()) == 0  # tile counters left zeroed
+        for Y in Ys:
+            check_outputs(Y.cpu(), X, ref["deq"])
+        assert all(torch.equal(Ys[0], Y) for Y in Ys[1:])  # deterministic, workspace reusable
+    finally:
+        lbq.lbq_debug_force_splits(0)
+
+
+def test_decode_step_layer_shapes(torch, lbq):
+    """One Llama-3-8B-shaped layer of the decode step, full size, every column."""
+    for p, (name, K, N) in enumerate(workloads.LLAMA3_8B_PROJ):
+        seed = workloads.c2_seed(0, p)
+        W = workloads.weights_host(seed, K, N)
+        ref = oracle_int4(W, 32, "asym")
+        img = lbq.pack(torch.from_numpy(W).cuda(), 32, "asym")
+        X = workloads.activations_host(seed, 1, K, "f16")
+        Y = lbq.gemv(X.cuda(), img, N, 32, "asym")
+        torch.cuda.synchronize()
+        check_outputs(Y.cpu(), X, ref["deq"])
+
+
+@pytest.mark.parametrize("group", [64, 128])
+def test_batch_sweep_full_size_sampled(torch, lbq, group):
+    """K=8192, N=28672 with 0.1% x20 outliers, BF16 X, M in {1,2,4,8,16}; outputs
+    checked on sampled columns, codes on the same columns bit-exactly."""
+    K, N = 8192, 28672
+    W = workloads.weights_host(3, K, N, outlier_frac=1e-3, outlier_mult=20.0)
+    Wd = torch.from_numpy(W).cuda()
+    img = lbq.pack(Wd, group, "sym")
+    del Wd
+    cols = sample_columns(N, 384, seed=group)
+    ref = oracle_int4(np.ascontiguousarray(W[:, cols]), group, "sym")
+    q, s, _ = lbq.unpack_canonical(img, K, N, group, "sym")
+    assert np.array_equal(q.cpu().numpy()[:, cols], ref["packed"])
+    assert np.array_equal(s.cpu().view(torch.int16).numpy()[:, cols], ref["s"].view(np.int16))
+    for M in (1, 2, 4, 8, 16):
+        X = workloads.activations_host(3, M, K, "bf16")
+        Y = lbq.gemv(X.cuda(), img, N, group, "sym")
+        torch.cuda.synchronize()
+        check_outputs(Y.cpu(), X, ref["deq"], cols)
+
+
+def test_large_activation_magnitudes(torch, lbq):
+    K, N = 2048, 256
+    W = workloads.weights_host(5, K, N)
+    ref = oracle_int4(W, 32, "asym")
+    img = lbq.pack(torch.from_numpy(W).cuda(), 32, "asym")
+    X = (workloads.activations_host(5, 1, K, "f16").float() * 100).half()
+    Y = lbq.gemv(X.cuda(), img, N, 32, "asym")
+    torch.cuda.synchronize()
+    check_outputs(Y.cpu(), X, ref["deq"])
+
+
+def test_wrong_header_is_reported_by_debug_calls(torch, lbq):
+    W = workloads.weights_host(1, 64, 8)
+    img = lbq.pack(torch.from_numpy(W).cuda(), 32, "sym")
+    with pytest.raises(lbq.LbqError):
+        lbq.unpack_canonical(img, 64, 16, 32, "sym")   # N does not match the image
+    with pytest.raises(lbq.LbqError):
+        lbq.dequant(img, 64, 8, 32, "asym")             # mode does not match
+
+
+def test_pdl_back_to_back_graph(torch, lbq):
+    """Programmatic dependent launch: a graph of GEMVs where each X is the
+    previous GEMV's output (a real dependency), results equal to the oracle."""
+    K = N = 1024
+    Ws = [workloads.weights_host(40 + i, K, N) for i in range(4)]
+    refs = [oracle_int4(W, 64, "sym") for W in Ws]
+    imgs = [lbq.pack(torch.from_numpy(W).cuda(), 64, "sym") for W in Ws]
+    X0 = workloads.activations_host(40, 1, K, "f16").cuda()
+    lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 1)
+    try:
+        bufs = [X0] + [torch.empty((1, N), dtype=torch.float16, device="cuda") for _ in imgs]
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for i, img in enumerate(imgs):
+                lbq.gemv(bufs[i], img, N, 64, "sym", Y=bufs[i + 1])
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        eager = [b.clone() for b in bufs[1:]]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i, img in enumerate(imgs):
+                lbq.gemv(bufs[i], img, N, 64, "sym", Y=bufs[i + 1])
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        lbq.device_status()
+    finally:
+        lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 0)
+    for i in range(len(imgs)):
+        assert torch.equal(eager[i], bufs[i + 1])
+        check_outputs(bufs[i + 1].cpu(), bufs[i].cpu(), refs[i]["deq"])
+
+
+SKINNY_SHAPES = [
+    (4096, 1000, 32, "asym", "f16"),
+    (512, 72, 64, "sym", "bf16"),
+    (1024, 130, 128, "asym", "bf16"),
+    (96, 40, 32, "sym", "f16"),       # K below one 256-k stage, ragged N
+    (8320, 64, 128, "sym", "f16"),    # K not a multiple of 256
+]
+
+
+@pytest.mark.parametrize("M", [2, 3, 8, 9, 16])
+@pytest.mark.parametrize("K,N,group,mode,xdt", SKINNY_SHAPES)
+def test_skinny_parity(torch, lbq, M, K, N, group, mode, xdt):
+    W = _special_groups(workloads.weights_host(300 + K + N, K, N), group)
+    ref = oracle_int4(W, group, mode)
+    img = lbq.pack(torch.from_numpy(W).cuda(), group, mode)
+    X = workloads.activations_host(300 + M, M, K, xdt)
+    for ydt in ("f16", "bf16"):
+        Y = lbq.gemv(X.cuda(), img, N, group, mode, y_dtype=ydt)
+        torch.cuda.synchronize()
+        check_outputs(Y.cpu(), X, ref["deq"])
+
+
+@pytest.mark.parametrize("splits", [1, 2, 5])
+def test_skinny_forced_split_k(torch, lbq, splits):
+    K, N, M = 4096, 520, 5
+    W = workloads.weights_host(91, K, N)
+    ref = oracle_int4(W, 64, "asym")
+    img = lbq.pack(torch.from_numpy(W).cuda(), 64, "asym")
+    X = workloads.activations_host(91, M, K, "bf16")
+    lbq.lbq_debug_force_splits(splits)
+    try:
+        ws = lbq.workspace(0, M, K, N, 64, "asym")
+        Ys = [lbq.gemv(X.cuda(), img, N, 64, "asym", ws=ws) for _ in range(3)]
+        torch.cuda.synchronize()
+        for Y in Ys:
+            check_outputs(Y.cpu(), X, ref["deq"])
+        assert all(torch.equal(Ys[0], Y) for Y in Ys[1:])
+        if ws is not None:
+            counters_at = -(-splits * M * N * 4 // 256) * 256
+            assert int(ws[counters_at:].count_nonzero()) == 0
+    finally:
+        lbq.lbq_debug_force_splits(0)
+
+
+def test_m1_through_the_skinny_kernel(torch, lbq):
+    K, N = 4096, 1024
+    W = workloads.weights_host(93, K, N)
+    ref = oracle_int4(W, 32, "asym")
+    img = lbq.pack(torch.from_numpy(W).cuda(), 32, "asym")
+    X = workloads.activations_host(93, 1, K, "f16")
+    lbq.lbq_debug_force_skinny(1)
+    try:
+        Y = lbq.gemv(X.cuda(), img, N, 32, "asym")
+        torch.cuda.synchronize()
+    finally:
+        lbq.lbq_debug_force_skinny(0)
+    check_outputs(Y.cpu(), X, ref["deq"])
