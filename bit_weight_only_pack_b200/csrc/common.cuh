@@ -28,14 +28,21 @@ __device__ unsigned int g_device_error;
 //                    kSlot[i] (bits 4*slot .. 4*slot+3). The slot order puts
 //                    (k, k+1) pairs in the two 16-bit halves of the same mask,
 //                    so one AND/OR turns two codes into a half2/bf16x2.
-//   S region         FP16 scales, N rows of K/group values (row n = the
-//                    groups of column n), row stride padded to 16 bytes.
-//   Z region (ASYM)  int8 zero points, same shape, row stride padded to 16 bytes.
+//   S region         FP16 scales tiled by 128 output channels: the scale of
+//                    (channel n, group gi) is element ((n/128)*G + gi)*128 + n%128
+//                    (G = K/group; N padded to a multiple of 128 with zeros), so
+//                    the scales of one 128-channel tile for a run of groups are
+//                    one contiguous block.
+//   Z region (ASYM)  int8 zero points, same tiling.
 // LUT3:
-//   I region         N rows of (K/64)*24 bytes: row n = channel n, 24 bytes
-//                    per 64-k tile, in the kernel order of lut3.cuh.
-//   C region         codebooks, [N/8][K/64][8] E4M3 bytes.
-//   E region         exponents, [N/8][K/64] UE8M0 bytes.
+//   I region         indices, tile-major: [K/64][N][24 bytes] (the 64 indices
+//                    of channel n in 64-k tile kt, in the order of lut3.cuh).
+//   C region         codebooks, N/8 rows of K/64 x 8 E4M3 bytes (stride padded to 16).
+//   E region         exponents, N/8 rows of K/64 UE8M0 bytes (stride padded to 16).
+//   T region         per tile, the 8 decoded weights e4m3(cb[j]) * 2^(E-127) as
+//                    BF16 in a byte-planar 16 bytes (low bytes of entries 0..7,
+//                    then high bytes), [K/64][N/8][16]: what the kernels read.
+//                    C and E keep the format's own bytes for exact recovery.
 // Every region starts on a 256-byte boundary.
 // ----------------------------------------------------------------------------
 
@@ -55,36 +62,45 @@ struct ImageHeader {
   int32_t K, N, group, mode;
   uint64_t off0, off1, off2;  // INT4: Q, S, Z   LUT3: I, C, E
   uint64_t total;
+  uint64_t off3;              // LUT3: T
 };
 static_assert(sizeof(ImageHeader) <= kHeaderBytes, "header too large");
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Element index of (channel n, group gi) in the 128-channel-tiled S / Z regions.
+__host__ __device__ inline size_t meta_index(int n, int gi, int G) {
+  return ((size_t)(n >> 7) * G + gi) * 128 + (n & 127);
+}
+
 struct Layout {
   int K, N, group, mode;
-  size_t off0, off1, off2, total;
-  size_t bytes0, bytes1, bytes2;
-  size_t s_stride, z_stride;  // INT4: padded row strides (bytes) of the S and Z regions
+  size_t off0, off1, off2, off3, total;
+  size_t bytes0, bytes1, bytes2, bytes3;
+  size_t s_stride, z_stride;  // LUT3: padded row strides (bytes) of the C and E regions
 };
 
 inline Layout make_layout(int K, int N, int group, int mode) {
   Layout L{};
   L.K = K; L.N = N; L.group = group; L.mode = mode;
   if (mode == LBQ_MODE_LUT3) {
+    L.s_stride = align_up((size_t)(K / 64) * 8, 16);  // codebook row stride
+    L.z_stride = align_up((size_t)(K / 64), 16);      // exponent row stride
     L.bytes0 = (size_t)N * (size_t)(K / 64) * 24;
-    L.bytes1 = (size_t)(N / 8) * (size_t)(K / 64) * 8;
-    L.bytes2 = (size_t)(N / 8) * (size_t)(K / 64);
+    L.bytes1 = (size_t)(N / 8) * L.s_stride;
+    L.bytes2 = (size_t)(N / 8) * L.z_stride;
+    L.bytes3 = (size_t)(K / 64) * (size_t)(N / 8) * 16;
   } else {
-    L.s_stride = align_up((size_t)(K / group) * 2, 16);
-    L.z_stride = align_up((size_t)(K / group), 16);
+    const size_t tiles128 = (size_t)(N + 127) / 128;
     L.bytes0 = (size_t)N * (size_t)(K / 2);
-    L.bytes1 = (size_t)N * L.s_stride;
-    L.bytes2 = mode == LBQ_MODE_ASYM ? (size_t)N * L.z_stride : 0;
+    L.bytes1 = tiles128 * (size_t)(K / group) * 128 * 2;
+    L.bytes2 = mode == LBQ_MODE_ASYM ? tiles128 * (size_t)(K / group) * 128 : 0;
   }
   L.off0 = kHeaderBytes;
   L.off1 = align_up(L.off0 + L.bytes0, kRegionAlign);
   L.off2 = align_up(L.off1 + L.bytes1, kRegionAlign);
-  L.total = align_up(L.off2 + L.bytes2, kRegionAlign);
+  L.off3 = align_up(L.off2 + L.bytes2, kRegionAlign);
+  L.total = align_up(L.off3 + L.bytes3, kRegionAlign);
   return L;
 }
 
@@ -93,7 +109,7 @@ inline ImageHeader make_header(const Layout& L) {
   h.magic = L.mode == LBQ_MODE_LUT3 ? kMagicLut3 : kMagicInt4;
   h.version = kImageVersion;
   h.K = L.K; h.N = L.N; h.group = L.group; h.mode = L.mode;
-  h.off0 = L.off0; h.off1 = L.off1; h.off2 = L.off2; h.total = L.total;
+  h.off0 = L.off0; h.off1 = L.off1; h.off2 = L.off2; h.total = L.total; h.off3 = L.off3;
   return h;
 }
 

@@ -10,7 +10,8 @@
 // One persistent CTA per SM, tiles of BM = 128 tokens x BN = 256 outputs,
 // k-blocks of 64. Warp roles:
 //   warp 0      TMA producer: X tile (128 x 64, 128-byte swizzle), packed
-//               code tile (256 rows x 32 bytes), scale and zero-point boxes;
+//               code tile (256 rows x 32 bytes), and bulk copies of the
+//               block's scales / zero points (contiguous per 128-channel tile);
 //               one mbarrier per stage, ring of kTcStages.
 //   warp 1      TMEM owner (alloc / dealloc of 512 columns) and MMA issuer:
 //               one thread issues 4 x tcgen05.mma.kind::f16 (M=128, N=256,
@@ -33,6 +34,7 @@
 
 #include "common.cuh"
 #include "tma.cuh"
+#include "lut3_gemv.cuh"
 
 namespace lbq {
 
@@ -43,15 +45,18 @@ constexpr int kTcDqWarps = 4, kTcEpWarps = 4;
 constexpr int kTcThreads = (2 + kTcDqWarps + kTcEpWarps) * 32;
 constexpr int kTcABytes = kTcBM * kTcBK * 2;   // 16 KB
 constexpr int kTcPBytes = kTcBN * kTcBK / 2;   // 8 KB of codes
-constexpr int kTcSBytes = kTcBN * 16;          // 16-byte scale box per row
-constexpr int kTcZBytes = kTcBN * 16;          // 16-byte zero-point box per row
-constexpr int kTcStageBytes = kTcABytes + kTcPBytes + kTcSBytes + kTcZBytes;  // 32 KB
+constexpr int kTcSBytes = 1024;                // scales: 2 channel tiles x up to 2 groups x 128 x 2 B
+constexpr int kTcZBytes = 1024;                // zero points: 2 x 2 x 128 x 1 B (padded)
+constexpr int kTcStageBytes = kTcABytes + kTcPBytes + kTcSBytes + kTcZBytes;  // 26 KB, 1024-aligned
 constexpr int kTcBBytes = kTcBN * kTcBK * 2;   // 32 KB
 constexpr int kTcSmem = kTcStages * kTcStageBytes + kTcBStages * kTcBBytes + 1024;
 constexpr uint32_t kTcTmemCols = 512;
 
 struct GemmTcArgs {
   void* Y;
+  const uint8_t* s_region;  // INT4: 128-channel-tiled scales; LUT3: I region (indices)
+  const uint8_t* z_region;  // INT4: 128-channel-tiled zero points (ASYM); LUT3: T region (tables)
+  int G, tiles128;          // groups per channel, 128-channel tiles
   int M, N, K, gshift64;   // gshift64: log2(group / 32)
   int m_tiles, n_tiles, k_blocks;
   int y_bf16;
@@ -140,10 +145,10 @@ __device__ __forceinline__ uint32_t scale_pair(uint16_t s_bits) {
   return (uint32_t)u | ((uint32_t)u << 16);
 }
 
-template <bool BF16, bool ASYM>
+// LUT: false = INT4 image, true = LUT3 image (BF16 activations only).
+template <bool BF16, bool ASYM, bool LUT>
 __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
-    const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tq,
-    const __grid_constant__ CUtensorMap ts, const __grid_constant__ CUtensorMap tz, const GemmTcArgs a) {
+    const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tq, const GemmTcArgs a) {
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t full_ap[kTcStages], empty_ap[kTcStages];
   __shared__ __align__(8) uint64_t full_b[kTcBStages], empty_b[kTcBStages];
@@ -186,9 +191,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
     if (lane == 0) {
       tma_prefetch_desc(&tx);
       tma_prefetch_desc(&tq);
-      tma_prefetch_desc(&ts);
-      if (ASYM) tma_prefetch_desc(&tz);
-      const uint32_t tx_bytes = kTcABytes + kTcPBytes + kTcSBytes + (ASYM ? kTcZBytes : 0);
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
@@ -197,12 +199,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
           const int s = it % kTcStages;
           if (it >= kTcStages && !mbar_wait(&empty_ap[s], ((it / kTcStages) & 1) ^ 1)) { ok = false; break; }
           uint8_t* st = ring + s * kTcStageBytes;
+          if (LUT) {
+            // tile kb of the indices and tables of channels nb*256 .. (contiguous, tile-major)
+            const int rows = min(kTcBN, a.N - nb * kTcBN);
+            mbar_arrive_expect_tx(&full_ap[s], (uint32_t)(kTcABytes + rows * 24 + (rows / 8) * 16));
+            tma_load_2d(st, &tx, kb * kTcBK, mb * kTcBM, &full_ap[s]);
+            bulk_load(st + kTcABytes, a.s_region + ((size_t)kb * a.N + nb * kTcBN) * 24, (uint32_t)(rows * 24),
+                      &full_ap[s]);
+            bulk_load(st + kTcABytes + kTcPBytes, a.z_region + ((size_t)kb * (a.N / 8) + nb * (kTcBN / 8)) * 16,
+                      (uint32_t)((rows / 8) * 16), &full_ap[s]);
+            continue;
+          }
           const int g0 = (kb * 2) >> a.gshift64;  // first group of the k-block
-          mbar_arrive_expect_tx(&full_ap[s], tx_bytes);
+          const int ng = min(a.gshift64 == 0 ? 2 : 1, a.G - g0);  // groups of the k-block
+          const int ntl = min(2, a.tiles128 - 2 * nb);  // 128-channel tiles of this 256-wide block
+          mbar_arrive_expect_tx(&full_ap[s], (uint32_t)(kTcABytes + kTcPBytes + ntl * ng * 128 * (ASYM ? 3 : 2)));
           tma_load_2d(st, &tx, kb * kTcBK, mb * kTcBM, &full_ap[s]);
           tma_load_2d(st + kTcABytes, &tq, kb * (kTcBK / 2), nb * kTcBN, &full_ap[s]);
-          tma_load_2d(st + kTcABytes + kTcPBytes, &ts, (g0 / 8) * 8, nb * kTcBN, &full_ap[s]);
-          if (ASYM) tma_load_2d(st + kTcABytes + kTcPBytes + kTcSBytes, &tz, (g0 / 16) * 16, nb * kTcBN, &full_ap[s]);
+          for (int tl = 0; tl < ntl; ++tl) {
+            const size_t meta0 = ((size_t)(2 * nb + tl) * a.G + g0) * 128;
+            bulk_load(st + kTcABytes + kTcPBytes + tl * ng * 256, a.s_region + meta0 * 2, (uint32_t)(ng * 256), &full_ap[s]);
+            if (ASYM)
+              bulk_load(st + kTcABytes + kTcPBytes + kTcSBytes + tl * ng * 128, a.z_region + meta0, (uint32_t)(ng * 128),
+                        &full_ap[s]);
+          }
         }
       }
     }
@@ -240,6 +260,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
     int it = 0, bit = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      const int nb = tile / a.m_tiles;
       for (int kb = 0; kb < a.k_blocks; ++kb, ++it, ++bit) {
         const int s = it % kTcStages;
         const int sb = bit % kTcBStages;
@@ -247,8 +268,40 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
         if (bit >= kTcBStages && !mbar_wait(&empty_b[sb], ((bit / kTcBStages) & 1) ^ 1)) { ok = false; break; }
         const uint32_t st = smem_u32(ring + s * kTcStageBytes);
         const uint32_t bt = smem_u32(btile + sb * kTcBBytes);
+        if (LUT) {
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            const int n = dt + 128 * hr;
+            if (nb * kTcBN + n >= a.N) continue;
+            // 24 bytes of indices per channel: 8-byte aligned, so three 8-byte loads
+            const uint8_t* ip = ring + s * kTcStageBytes + kTcABytes + n * 24;
+            const uint2 p0 = *reinterpret_cast<const uint2*>(ip);
+            const uint2 p1 = *reinterpret_cast<const uint2*>(ip + 8);
+            const uint2 p2 = *reinterpret_cast<const uint2*>(ip + 16);
+            const uint32_t w[6] = {p0.x, p0.y, p1.x, p1.y, p2.x, p2.y};
+            const uint4 tab = lds128(st + kTcABytes + kTcPBytes + (n >> 3) * 16);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                uint32_t pr[4];
+                lut3_decode8(lut3_selector(w[3 * h + (t < 2 ? 0 : 1)], w[3 * h + 2], t), tab, pr);
+                const int c = 4 * h + t;
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                             :: "r"(bt + (uint32_t)(n * 128 + ((c ^ (n & 7)) << 4))), "r"(pr[0]), "r"(pr[1]),
+                                "r"(pr[2]), "r"(pr[3]) : "memory");
+              }
+          }
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&full_b[sb]);
+            mbar_arrive(&empty_ap[s]);
+          }
+          continue;
+        }
         const int g0 = (kb * 2) >> a.gshift64;
-        const int sx0 = (g0 / 8) * 8, zx0 = (g0 / 16) * 16;
+        const int ng = min(a.gshift64 == 0 ? 2 : 1, a.G - g0);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int n = dt + 128 * h;
@@ -259,13 +312,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
           for (int half = 0; half < 2; ++half) {
             // words 4*half .. 4*half+3 cover k = 32*half .. 32*half+31 of the k-block
             const int gi = (kb * 2 + half) >> a.gshift64;
-            uint16_t sbits;
-            asm volatile("ld.shared.u16 %0, [%1];" : "=h"(sbits)
-                         : "r"(st + kTcABytes + kTcPBytes + n * 16 + (gi - sx0) * 2));
+            const int mi = ((n >> 7) * ng + (gi - g0)) * 128 + (n & 127);  // (tile, group, row) in the stage
+            uint16_t sbits = 0;
             int z = 8;
-            if (ASYM)
-              asm volatile("ld.shared.s8 %0, [%1];" : "=r"(z)
-                           : "r"(st + kTcABytes + kTcPBytes + kTcSBytes + n * 16 + (gi - zx0)));
+            if (nb * kTcBN + n < a.N && gi - g0 < ng) {
+              asm volatile("ld.shared.u16 %0, [%1];" : "=h"(sbits) : "r"(st + kTcABytes + kTcPBytes + mi * 2));
+              if (ASYM) asm volatile("ld.shared.s8 %0, [%1];" : "=r"(z) : "r"(st + kTcABytes + kTcPBytes + kTcSBytes + mi));
+            }
             uint32_t c1, c2;
             zero_consts<BF16>(z, c1, c2);
             const uint32_t s2 = scale_pair<BF16>(sbits);

@@ -5,8 +5,9 @@
 // lanes and reduces. On B200 this kernel is HBM-bound, so it is built to keep
 // enough bytes in flight and to touch every weight byte once:
 //
-//  * One producer thread streams tiles of the image (the codes of R_s rows
-//    for this CTA's K-slice, plus their scales and zero points) into a ring of
+//  * One producer thread streams tiles of the image (the codes of 8 rows for
+//    this CTA's K-slice, plus their scales and zero points: 16-byte-wide boxes
+//    of the 128-channel-tiled scale / zero-point regions) into a ring of
 //    shared-memory slots with 2-D TMA copies, running up to `stages` slots
 //    ahead of the consumers (mbarrier full/empty handshake, bounded waits).
 //  * A consumer thread owns one 16-byte chunk (32 consecutive k, one scale)
@@ -38,19 +39,20 @@ namespace lbq {
 constexpr int kM1MaxStages = 8;
 constexpr int kM1MaxConsumerThreads = 256;
 
+constexpr int kM1SlotRows = 8;  // rows of the weight per ring slot
+
 struct GemvM1Args {
   const uint16_t* X;        // [K] FP16/BF16 bits
   void* Y;                  // [N]
   float* partials;          // [splits][N] FP32 (splits > 1)
   unsigned int* counters;   // [row_tiles] (splits > 1)
-  int K, N, gshift;         // chunk c lies in group c >> gshift
+  int K, N, G, gshift;      // chunk c lies in group c >> gshift
   int cps, splits;          // chunks per split (a multiple of 64 when splits > 1)
   int tpr, phases;          // consumer threads per row group (multiple of 32), row groups
-  int rows_per_stage;       // R_s = RPT * phases
   int stages;               // ring depth
   int nqbox;                // 256-byte code boxes per slot row
-  int sbox_w, nsbox;        // scale box width (elements) and count
-  int zbox_w, nzbox;        // zero-point box width (bytes) and count
+  int sbox_h, nsbox;        // groups per scale box and box count
+  int zbox_h, nzbox;        // groups per zero-point box and box count
   int off_s, off_z, slot_bytes, tx_bytes;
   int row_tiles, total_tiles;  // tile = 8*phases rows of one K-slice
   int y_bf16;
@@ -122,7 +124,7 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" :: "r"(nthreads) : "memory");
 }
 
-template <bool BF16, bool ASYM, int CPT, int RPT>
+template <bool BF16, bool ASYM, int RPT>
 __global__ void __launch_bounds__(kM1MaxConsumerThreads + 32, 2) gemv_m1_kernel(
     const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap ts,
     const __grid_constant__ CUtensorMap tz, const GemvM1Args a) {
@@ -136,7 +138,8 @@ __global__ void __launch_bounds__(kM1MaxConsumerThreads + 32, 2) gemv_m1_kernel(
   const int nthreads_c = a.tpr * a.phases;
   const int ncw = nthreads_c >> 5;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int R = a.rows_per_stage;
+  constexpr int R = kM1SlotRows;
+  constexpr int CPT = 1;
   const int rows_per_tile = 8 * a.phases;
 
   if (tid == 0) {
@@ -172,11 +175,13 @@ __global__ void __launch_bounds__(kM1MaxConsumerThreads + 32, 2) gemv_m1_kernel(
           }
           mbar_arrive_expect_tx(&full_bar[slot], (uint32_t)a.tx_bytes);
           for (int b = 0; b < a.nqbox; ++b) tma_load_2d(dst + b * R * 256, &tq, c0 * 16 + b * 256, r0, &full_bar[slot]);
+          // scales / zero points: rows r0..r0+7 of the 128-channel tile, groups g0..
+          const int my = (r0 >> 7) * a.G + g0;
           for (int b = 0; b < a.nsbox; ++b)
-            tma_load_2d(dst + a.off_s + b * R * a.sbox_w * 2, &ts, g0 + b * a.sbox_w, r0, &full_bar[slot]);
+            tma_load_2d(dst + a.off_s + b * a.sbox_h * 16, &ts, r0 & 127, my + b * a.sbox_h, &full_bar[slot]);
           if (ASYM)
             for (int b = 0; b < a.nzbox; ++b)
-              tma_load_2d(dst + a.off_z + b * R * a.zbox_w, &tz, g0 + b * a.zbox_w, r0, &full_bar[slot]);
+              tma_load_2d(dst + a.off_z + b * a.zbox_h * 16, &tz, (r0 & 127) & ~15, my + b * a.zbox_h, &full_bar[slot]);
         }
       }
     }
@@ -195,8 +200,8 @@ __global__ void __launch_bounds__(kM1MaxConsumerThreads + 32, 2) gemv_m1_kernel(
   uint32_t q_off[CPT], s_off[CPT], z_off[CPT];
   bool c_ok[CPT];
   const uint32_t q_rstride = (uint32_t)(a.phases * 256);
-  const uint32_t s_rstride = (uint32_t)(a.phases * a.sbox_w * 2);
-  const uint32_t z_rstride = (uint32_t)(a.phases * a.zbox_w);
+  const uint32_t s_rstride = (uint32_t)(a.phases * 2);
+  const uint32_t z_rstride = (uint32_t)a.phases;
   int cur_split = -1;
   int it = 0;
   int buf = 0;
@@ -215,12 +220,11 @@ __global__ void __launch_bounds__(kM1MaxConsumerThreads + 32, 2) gemv_m1_kernel(
 #pragma unroll
       for (int j = 0; j < CPT; ++j) {
         const int c = lt + j * a.tpr;
-        const int gi = c >> a.gshift;
-        const int sbx = gi / a.sbox_w, zbx = gi / a.zbox_w;
+        const int gi = c >> a.gshift;  // group within the K-slice
         c_ok[j] = c < nch;
         q_off[j] = (uint32_t)((c >> 4) * R * 256 + (c & 15) * 16 + phase * 256);
-        s_off[j] = (uint32_t)(a.off_s + (sbx * R + phase) * a.sbox_w * 2 + (gi - sbx * a.sbox_w) * 2);
-        z_off[j] = (uint32_t)(a.off_z + (zbx * R + phase) * a.zbox_w + (gi - zbx * a.zbox_w));
+        s_off[j] = (uint32_t)(a.off_s + gi * 16 + phase * 2);
+        z_off[j] = (uint32_t)(a.off_z + gi * 16 + phase);  // + the slot's row offset in its 16-row box
         float sA = 0.0f, sB = 0.0f;
         if (c_ok[j]) {
           const uint4* xp = reinterpret_cast<const uint4*>(a.X + (size_t)(c0 + c) * 32);
@@ -254,6 +258,7 @@ __global__ void __launch_bounds__(kM1MaxConsumerThreads + 32, 2) gemv_m1_kernel(
       const int slot = it % a.stages;
       if (!mbar_wait(&full_bar[slot], (it / a.stages) & 1)) { timed_out = true; break; }
       const uint32_t sb = smem_u32(ring + (size_t)slot * a.slot_bytes);
+      const uint32_t zrow = (uint32_t)((rt * rows_per_tile + st * R) & 8);  // 8-row half of the 16-row zp box
 #pragma unroll
       for (int i = 0; i < RPT; ++i) {
 #pragma unroll
@@ -265,7 +270,7 @@ __global__ void __launch_bounds__(kM1MaxConsumerThreads + 32, 2) gemv_m1_kernel(
             float corr = xoff[j];
             if (ASYM) {
               int zv;
-              asm volatile("ld.shared.s8 %0, [%1];" : "=r"(zv) : "r"(sb + z_off[j] + i * z_rstride));
+              asm volatile("ld.shared.s8 %0, [%1];" : "=r"(zv) : "r"(sb + z_off[j] + zrow + i * z_rstride));
               corr = fmaf((float)zv, xsum[j], corr);
             }
             const float acc = chunk_acc<BF16>(w, xr[j]);

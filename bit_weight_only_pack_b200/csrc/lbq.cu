@@ -18,9 +18,11 @@
 
 #include "common.cuh"
 #include "pack_int4.cuh"
+#include "lut3.cuh"
 #include "tma.cuh"
 #include "gemv_m1.cuh"
 #include "skinny.cuh"
+#include "lut3_gemv.cuh"
 #include "gemm_tc.cuh"
 
 namespace lbq {
@@ -136,77 +138,64 @@ static int occupancy_for(const void* fn, int block, int smem) {
 // ----------------------------------------------------------------------------
 
 struct M1Plan {
-  int splits, cps, cpt, rpt, tpr, phases, R;
-  int nqbox, sbox_w, nsbox, zbox_w, nzbox, off_s, off_z, slot_bytes, tx_bytes, stages;
-  int row_tiles, total_tiles, grid, block, smem;
+  int splits, cps, rpt, tpr, phases;
+  int nqbox, sbox_h, nsbox, zbox_h, nzbox, off_s, off_z, slot_bytes, tx_bytes, stages;
+  int row_tiles, total_tiles, block, smem;
 };
 
 static int g_force_splits = 0;  // test hook: force a split count (0 = shape-based choice)
 static int g_pdl = 0;           // launch GEMVs with programmatic dependent launch
 static int g_force_skinny = 0;  // test hook: route M = 1 to the tensor-core skinny kernel
 
-constexpr int kM1SlotTarget = 24 * 1024;
 constexpr int kM1RingBudget = 100 * 1024;
+constexpr int kM1MaxChunksPerSplit = 128;  // K-slices of at most 4096 k keep a ring slot near 20 KB
 
 static void m1_slot_geometry(M1Plan& p, int group, bool asym) {
   const int gps = p.cps * 32 / group;  // groups per K-slice
   p.nqbox = (p.cps * 16 + 255) / 256;
-  p.sbox_w = std::min(256, (gps + 7) / 8 * 8);
-  p.nsbox = (gps + p.sbox_w - 1) / p.sbox_w;
-  p.zbox_w = std::min(256, (gps + 15) / 16 * 16);
-  p.nzbox = asym ? (gps + p.zbox_w - 1) / p.zbox_w : 0;
-  const int qbytes = p.nqbox * p.R * 256;
+  p.sbox_h = std::min(256, gps);
+  p.nsbox = (gps + p.sbox_h - 1) / p.sbox_h;
+  p.zbox_h = p.sbox_h;
+  p.nzbox = asym ? p.nsbox : 0;
+  const int qbytes = p.nqbox * kM1SlotRows * 256;
   p.off_s = (int)align_up(qbytes, 128);
-  const int sbytes = p.nsbox * p.R * p.sbox_w * 2;
+  const int sbytes = p.nsbox * p.sbox_h * 16;
   p.off_z = (int)align_up(p.off_s + sbytes, 128);
-  const int zbytes = p.nzbox * p.R * p.zbox_w;
+  const int zbytes = p.nzbox * p.zbox_h * 16;
   p.slot_bytes = (int)align_up(p.off_z + zbytes, 1024);
   p.tx_bytes = qbytes + sbytes + zbytes;
 }
 
-// Shape-based plan: chunk split, threads per row, rows per slot, ring depth, grid.
+// Shape-based plan: K-slices (split-K), threads per row, ring depth.
 static M1Plan plan_m1(int K, int N, int group, bool asym, int force_splits) {
   const int chunks = K / 32;
-  const int sms = num_sms();
-  const int target = 2 * sms;
+  const int target = 2 * num_sms();
   M1Plan best{};
-  bool have = false;
   const int max_splits = std::max(1, chunks / 64);
   for (int splits = 1; splits <= max_splits; ++splits) {
     if (force_splits > 0 && splits != std::min(force_splits, max_splits)) continue;
     int cps = chunks;
-    if (splits > 1) cps = ((chunks + splits - 1) / splits + 63) / 64 * 64;  // slice starts on 2048-k boundaries
-    const int real_splits = (chunks + cps - 1) / cps;
-    if (real_splits != splits) continue;
-    const int cpt = cps <= 256 ? 1 : cps <= 512 ? 2 : cps <= 1024 ? 4 : 0;
-    if (cpt == 0) continue;
-    // one chunk per thread keeps the kernel within its register budget: split K instead
-    if (cpt > 1 && splits < max_splits && force_splits == 0) continue;
+    if (splits > 1) cps = ((chunks + splits - 1) / splits + 63) / 64 * 64;  // slices start on 2048-k boundaries
+    if ((chunks + cps - 1) / cps != splits) continue;
+    if (cps > kM1MaxChunksPerSplit && splits < max_splits && force_splits == 0) continue;
     M1Plan p{};
-    p.splits = splits; p.cps = cps; p.cpt = cpt;
-    p.tpr = (((cps + cpt - 1) / cpt) + 31) / 32 * 32;
-    int phases = std::max(1, kM1MaxConsumerThreads / p.tpr);
+    p.splits = splits;
+    p.cps = cps;
+    p.tpr = (cps + 31) / 32 * 32;
+    if (p.tpr > kM1MaxConsumerThreads) continue;
+    int phases = std::min(8, std::max(1, kM1MaxConsumerThreads / p.tpr));
     while (phases > 1 && (long long)((N + 8 * phases - 1) / (8 * phases)) * splits < target) phases /= 2;
     p.phases = phases;
-    const int max_rpt = cpt == 1 ? 8 : cpt == 2 ? 2 : 1;
-    p.rpt = 1;
-    for (int rpt = max_rpt; rpt >= 1; rpt /= 2) {
-      p.rpt = rpt;
-      p.R = rpt * phases;
-      m1_slot_geometry(p, group, asym);
-      if (p.slot_bytes <= kM1SlotTarget || rpt == 1) break;
-    }
+    p.rpt = kM1SlotRows / phases;
+    m1_slot_geometry(p, group, asym);
     p.stages = std::max(2, std::min(kM1MaxStages, kM1RingBudget / p.slot_bytes));
     p.row_tiles = (N + 8 * phases - 1) / (8 * phases);
     p.total_tiles = p.row_tiles * splits;
     p.block = p.tpr * phases + 32;
     p.smem = p.stages * p.slot_bytes + 1024;
     best = p;
-    have = true;
     if (force_splits > 0 || (long long)p.total_tiles >= target) break;
   }
-  if (!have) return best;
-  best.grid = best.total_tiles;  // capped by occupancy at launch
   return best;
 }
 
@@ -218,20 +207,16 @@ static size_t m1_workspace_bytes(const M1Plan& p, int N) {
 typedef void (*M1Kernel)(CUtensorMap, CUtensorMap, CUtensorMap, GemvM1Args);
 
 template <bool B, bool A>
-static M1Kernel m1_kernel_for(int cpt, int rpt) {
-  if (cpt == 1) {
-    if (rpt == 8) return gemv_m1_kernel<B, A, 1, 8>;
-    if (rpt == 4) return gemv_m1_kernel<B, A, 1, 4>;
-    if (rpt == 2) return gemv_m1_kernel<B, A, 1, 2>;
-    return gemv_m1_kernel<B, A, 1, 1>;
-  }
-  if (cpt == 2) return rpt == 2 ? gemv_m1_kernel<B, A, 2, 2> : gemv_m1_kernel<B, A, 2, 1>;
-  return gemv_m1_kernel<B, A, 4, 1>;
+static M1Kernel m1_kernel_for(int rpt) {
+  if (rpt == 8) return gemv_m1_kernel<B, A, 8>;
+  if (rpt == 4) return gemv_m1_kernel<B, A, 4>;
+  if (rpt == 2) return gemv_m1_kernel<B, A, 2>;
+  return gemv_m1_kernel<B, A, 1>;
 }
 
-static M1Kernel m1_kernel(bool bf16, bool asym, int cpt, int rpt) {
-  if (bf16) return asym ? m1_kernel_for<true, true>(cpt, rpt) : m1_kernel_for<true, false>(cpt, rpt);
-  return asym ? m1_kernel_for<false, true>(cpt, rpt) : m1_kernel_for<false, false>(cpt, rpt);
+static M1Kernel m1_kernel(bool bf16, bool asym, int rpt) {
+  if (bf16) return asym ? m1_kernel_for<true, true>(rpt) : m1_kernel_for<true, false>(rpt);
+  return asym ? m1_kernel_for<false, true>(rpt) : m1_kernel_for<false, false>(rpt);
 }
 
 static lbq_status launch_kernel_ex(const void* fn, dim3 grid, dim3 block, int smem, cudaStream_t st, bool pdl,
@@ -259,34 +244,35 @@ static lbq_status launch_kernel_ex(const void* fn, dim3 grid, dim3 block, int sm
 static lbq_status run_m1(const uint16_t* X, bool xbf16, const void* image, const Layout& L, void* Y, bool ybf16,
                          void* ws, size_t ws_bytes, cudaStream_t st) {
   const bool asym = L.mode == LBQ_MODE_ASYM;
-  M1Plan p = plan_m1(L.K, L.N, L.group, asym, g_force_splits);
+  const M1Plan p = plan_m1(L.K, L.N, L.group, asym, g_force_splits);
   if (p.block == 0) return fail(LBQ_ERR_UNSUPPORTED, "no GEMV plan for K=%d", L.K);
   const size_t need = m1_workspace_bytes(p, L.N);
   if (need > 0 && (ws == nullptr || ws_bytes < need))
     return fail(LBQ_ERR_INVALID_ARG, "workspace of %zu bytes is too small (need %zu)", ws_bytes, need);
   const uint8_t* img = static_cast<const uint8_t*>(image);
   const int G = L.K / L.group;
+  const uint64_t meta_rows = (uint64_t)((L.N + 127) / 128) * G;  // (channel tile, group) rows of 128 entries
   CUtensorMap tq, ts, tz;
   if (!make_tmap_2d(&tq, img + L.off0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.K / 2, (uint64_t)L.N,
-                    (uint64_t)L.K / 2, 256, (uint32_t)p.R, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_tmap_2d(&ts, img + L.off1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)G, (uint64_t)L.N, L.s_stride,
-                    (uint32_t)p.sbox_w, (uint32_t)p.R, CU_TENSOR_MAP_SWIZZLE_NONE))
+                    (uint64_t)L.K / 2, 256, kM1SlotRows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&ts, img + L.off1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, 128, meta_rows, 256, 8, (uint32_t)p.sbox_h,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the GEMV tiles");
   tz = ts;
-  if (asym && !make_tmap_2d(&tz, img + L.off2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)G, (uint64_t)L.N,
-                            L.z_stride, (uint32_t)p.zbox_w, (uint32_t)p.R, CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (asym && !make_tmap_2d(&tz, img + L.off2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, meta_rows, 128, 16,
+                            (uint32_t)p.zbox_h, CU_TENSOR_MAP_SWIZZLE_NONE))
     return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the zero points");
   GemvM1Args a{};
   a.X = X;
   a.Y = Y;
   a.partials = need ? static_cast<float*>(ws) : nullptr;
   a.counters = need ? reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + align_up((size_t)p.splits * L.N * sizeof(float), 256)) : nullptr;
-  a.K = L.K; a.N = L.N; a.gshift = log2_exact(L.group / 32);
-  a.cps = p.cps; a.splits = p.splits; a.tpr = p.tpr; a.phases = p.phases; a.rows_per_stage = p.R;
-  a.stages = p.stages; a.nqbox = p.nqbox; a.sbox_w = p.sbox_w; a.nsbox = p.nsbox; a.zbox_w = p.zbox_w;
+  a.K = L.K; a.N = L.N; a.G = G; a.gshift = log2_exact(L.group / 32);
+  a.cps = p.cps; a.splits = p.splits; a.tpr = p.tpr; a.phases = p.phases;
+  a.stages = p.stages; a.nqbox = p.nqbox; a.sbox_h = p.sbox_h; a.nsbox = p.nsbox; a.zbox_h = p.zbox_h;
   a.nzbox = p.nzbox; a.off_s = p.off_s; a.off_z = p.off_z; a.slot_bytes = p.slot_bytes; a.tx_bytes = p.tx_bytes;
   a.row_tiles = p.row_tiles; a.total_tiles = p.total_tiles; a.y_bf16 = ybf16 ? 1 : 0;
-  M1Kernel fn = m1_kernel(xbf16, asym, p.cpt, p.rpt);
+  const M1Kernel fn = m1_kernel(xbf16, asym, p.rpt);
   const int occ = occupancy_for((const void*)fn, p.block, p.smem);
   const int grid = std::min(p.total_tiles, num_sms() * occ);
   void* args[] = {&tq, &ts, &tz, &a};
@@ -298,34 +284,11 @@ static lbq_status run_m1(const uint16_t* X, bool xbf16, const void* image, const
 // ----------------------------------------------------------------------------
 
 struct SkPlan {
-  int nt, gc, row_tiles, total_stages, sps, splits, total_tiles, smem, slot;
+  int nt, gc, row_tiles, stages_per_tile, max_slots, grid, smem, slot;
+  long long units;
 };
 
-static SkPlan plan_skinny(int K, int N, int M, int group, bool asym, int force_splits) {
-  SkPlan p{};
-  p.nt = M <= 8 ? 1 : 2;
-  p.gc = group / 32;
-  p.row_tiles = (N + kSkRows - 1) / kSkRows;
-  p.total_stages = (K + 255) / 256;
-  const int target = 2 * num_sms();
-  int splits = 1;
-  if (force_splits > 0) splits = std::min(force_splits, p.total_stages);
-  else
-    while (p.row_tiles * splits < target && splits < p.total_stages) ++splits;
-  p.sps = (p.total_stages + splits - 1) / splits;
-  p.splits = (p.total_stages + p.sps - 1) / p.sps;
-  p.total_tiles = p.row_tiles * p.splits;
-  p.slot = kSkWBytes + 4 * p.nt * 1024 + kSkSBytes + (asym ? kSkZBytes : 0);
-  p.smem = kSkStages * p.slot + 1024;
-  return p;
-}
-
-static size_t skinny_workspace_bytes(const SkPlan& p, int M, int N) {
-  if (p.splits <= 1) return 0;
-  return align_up((size_t)p.splits * M * N * sizeof(float), 256) + align_up((size_t)p.row_tiles * sizeof(unsigned), 256);
-}
-
-typedef void (*SkKernel)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, SkinnyArgs);
+typedef void (*SkKernel)(CUtensorMap, CUtensorMap, SkinnyArgs);
 
 template <bool B, bool A, int NT, bool KF>
 static SkKernel sk_for_gc(int gc) {
@@ -345,40 +308,57 @@ static SkKernel sk_kernel(bool bf16, bool asym, int nt, int gc, bool kfull) {
   return asym ? sk_for_nt<false, true>(nt, gc, kfull) : sk_for_nt<false, false>(nt, gc, kfull);
 }
 
+// Stream-K plan: units = row tiles x 256-k stages, split evenly over one wave
+// of resident CTAs.
+static SkPlan plan_skinny(int K, int N, int M, int group, bool asym, bool xbf16) {
+  SkPlan p{};
+  p.nt = M <= 8 ? 1 : 2;
+  p.gc = group / 32;
+  p.row_tiles = (N + kSkRows - 1) / kSkRows;
+  p.stages_per_tile = (K + 255) / 256;
+  p.units = (long long)p.row_tiles * p.stages_per_tile;
+  p.slot = kSkWBytes + 4 * p.nt * 1024 + kSkSBytes + (asym ? kSkZBytes : 0);  // a multiple of 1024
+  p.smem = kSkStages * p.slot + 1024;
+  const SkKernel fn = sk_kernel(xbf16, asym, p.nt, p.gc, K % 256 == 0);
+  const int occ = occupancy_for((const void*)fn, kSkThreads, p.smem);
+  p.grid = (int)std::min<long long>(p.units, (long long)num_sms() * occ);
+  const long long per = std::max<long long>(1, p.units / p.grid);
+  p.max_slots = (int)((p.stages_per_tile + per - 1) / per + 1);
+  return p;
+}
+
+static size_t skinny_workspace_bytes(const SkPlan& p, int M) {
+  return align_up((size_t)p.row_tiles * p.max_slots * M * kSkRows * sizeof(float), 256) +
+         align_up((size_t)p.row_tiles * sizeof(unsigned), 256);
+}
+
 static lbq_status run_skinny(const void* X, bool xbf16, int M, const void* image, const Layout& L, void* Y,
                              bool ybf16, void* ws, size_t ws_bytes, cudaStream_t st) {
   const bool asym = L.mode == LBQ_MODE_ASYM;
-  const SkPlan p = plan_skinny(L.K, L.N, M, L.group, asym, g_force_splits);
-  const size_t need = skinny_workspace_bytes(p, M, L.N);
-  if (need > 0 && (ws == nullptr || ws_bytes < need))
+  const SkPlan p = plan_skinny(L.K, L.N, M, L.group, asym, xbf16);
+  const size_t need = skinny_workspace_bytes(p, M);
+  if (ws == nullptr || ws_bytes < need)
     return fail(LBQ_ERR_INVALID_ARG, "workspace of %zu bytes is too small (need %zu)", ws_bytes, need);
   const uint8_t* img = static_cast<const uint8_t*>(image);
-  const int G = L.K / L.group;
-  CUtensorMap tw, tx, ts, tz;
-  bool ok = make_tmap_2d(&tw, img + L.off0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.K / 2, (uint64_t)L.N,
-                         (uint64_t)L.K / 2, 128, kSkRows, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)L.K, (uint64_t)M, (uint64_t)L.K * 2, 64,
-                         (uint32_t)M, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            make_tmap_2d(&ts, img + L.off1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)G, (uint64_t)L.N, L.s_stride,
-                         8, kSkRows, CU_TENSOR_MAP_SWIZZLE_NONE);
-  tz = ts;
-  if (ok && asym)
-    ok = make_tmap_2d(&tz, img + L.off2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)G, (uint64_t)L.N, L.z_stride,
-                      16, kSkRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+  CUtensorMap tw, tx;
+  const bool ok = make_tmap_2d(&tw, img + L.off0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.K / 2, (uint64_t)L.N,
+                               (uint64_t)L.K / 2, 128, kSkRows, CU_TENSOR_MAP_SWIZZLE_128B) &&
+                  make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)L.K, (uint64_t)M,
+                               (uint64_t)L.K * 2, 64, (uint32_t)M, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the skinny kernel");
   SkinnyArgs a{};
   a.Y = Y;
-  a.partials = need ? static_cast<float*>(ws) : nullptr;
-  a.counters = need ? reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) +
-                                                  align_up((size_t)p.splits * M * L.N * sizeof(float), 256)) : nullptr;
-  a.K = L.K; a.N = L.N; a.M = M;
-  a.stages_per_split = p.sps; a.splits = p.splits; a.row_tiles = p.row_tiles; a.total_tiles = p.total_tiles;
+  a.partials = static_cast<float*>(ws);
+  a.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) +
+                                           align_up((size_t)p.row_tiles * p.max_slots * M * kSkRows * sizeof(float), 256));
+  a.s_region = img + L.off1;
+  a.z_region = asym ? img + L.off2 : nullptr;
+  a.K = L.K; a.N = L.N; a.M = M; a.G = L.K / L.group;
+  a.stages_per_tile = p.stages_per_tile; a.row_tiles = p.row_tiles; a.max_slots = p.max_slots; a.units = p.units;
   a.y_bf16 = ybf16 ? 1 : 0;
-  SkKernel fn = sk_kernel(xbf16, asym, p.nt, p.gc, L.K % 256 == 0);
-  const int occ = occupancy_for((const void*)fn, kSkThreads, p.smem);
-  const int grid = std::min(p.total_tiles, num_sms() * occ);
-  void* args[] = {&tw, &tx, &ts, &tz, &a};
-  return launch_kernel_ex((const void*)fn, dim3(grid), dim3(kSkThreads), p.smem, st, g_pdl != 0, args,
+  const SkKernel fn = sk_kernel(xbf16, asym, p.nt, p.gc, L.K % 256 == 0);
+  void* args[] = {&tw, &tx, &a};
+  return launch_kernel_ex((const void*)fn, dim3(p.grid), dim3(kSkThreads), p.smem, st, g_pdl != 0, args,
                           "skinny launch");
 }
 
@@ -392,32 +372,99 @@ static lbq_status run_gemm_tc(const void* X, bool xbf16, int M, const void* imag
                               bool ybf16, cudaStream_t st) {
   const bool asym = L.mode == LBQ_MODE_ASYM;
   const uint8_t* img = static_cast<const uint8_t*>(image);
-  const int G = L.K / L.group;
-  CUtensorMap tx, tq, ts, tz;
-  bool ok = make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)L.K, (uint64_t)M, (uint64_t)L.K * 2,
-                         kTcBK, kTcBM, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            make_tmap_2d(&tq, img + L.off0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.K / 2, (uint64_t)L.N,
-                         (uint64_t)L.K / 2, kTcBK / 2, kTcBN, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-            make_tmap_2d(&ts, img + L.off1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)G, (uint64_t)L.N, L.s_stride,
-                         8, kTcBN, CU_TENSOR_MAP_SWIZZLE_NONE);
-  tz = ts;
-  if (ok && asym)
-    ok = make_tmap_2d(&tz, img + L.off2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)G, (uint64_t)L.N, L.z_stride,
-                      16, kTcBN, CU_TENSOR_MAP_SWIZZLE_NONE);
+  CUtensorMap tx, tq;
+  const bool ok = make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)L.K, (uint64_t)M,
+                               (uint64_t)L.K * 2, kTcBK, kTcBM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+                  make_tmap_2d(&tq, img + L.off0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.K / 2, (uint64_t)L.N,
+                               (uint64_t)L.K / 2, kTcBK / 2, kTcBN, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the prefill GEMM");
   GemmTcArgs a{};
   a.Y = Y;
+  a.s_region = img + L.off1;
+  a.z_region = asym ? img + L.off2 : nullptr;
+  a.G = L.K / L.group;
+  a.tiles128 = (L.N + 127) / 128;
   a.M = M; a.N = L.N; a.K = L.K; a.gshift64 = log2_exact(L.group / 32);
   a.m_tiles = (M + kTcBM - 1) / kTcBM;
   a.n_tiles = (L.N + kTcBN - 1) / kTcBN;
   a.k_blocks = (L.K + kTcBK - 1) / kTcBK;
   a.y_bf16 = ybf16 ? 1 : 0;
-  const void* fn = xbf16 ? (asym ? (const void*)gemm_tc_kernel<true, true> : (const void*)gemm_tc_kernel<true, false>)
-                         : (asym ? (const void*)gemm_tc_kernel<false, true> : (const void*)gemm_tc_kernel<false, false>);
+  const void* fn = xbf16 ? (asym ? (const void*)gemm_tc_kernel<true, true, false> : (const void*)gemm_tc_kernel<true, false, false>)
+                         : (asym ? (const void*)gemm_tc_kernel<false, true, false> : (const void*)gemm_tc_kernel<false, false, false>);
   occupancy_for(fn, kTcThreads, kTcSmem);
   const int grid = std::min(a.m_tiles * a.n_tiles, num_sms());
-  void* args[] = {&tx, &tq, &ts, &tz, &a};
+  void* args[] = {&tx, &tq, &a};
   return launch_kernel_ex(fn, dim3(grid), dim3(kTcThreads), kTcSmem, st, false, args, "prefill GEMM launch");
+}
+
+// ----------------------------------------------------------------------------
+// LUT3: skinny (M <= 16) and tcgen05 (M > 16)
+// ----------------------------------------------------------------------------
+
+static SkPlan plan_lut3(int K, int N, int M) {
+  SkPlan p{};
+  p.nt = M <= 8 ? 1 : 2;
+  p.row_tiles = (N + kSkRows - 1) / kSkRows;
+  p.stages_per_tile = (K + 255) / 256;
+  p.units = (long long)p.row_tiles * p.stages_per_tile;
+  p.slot = 13312 + 4 * p.nt * 1024;
+  p.smem = kL3Stages * p.slot + 1024;
+  const void* fn = p.nt == 1 ? (const void*)lut3_skinny_kernel<1> : (const void*)lut3_skinny_kernel<2>;
+  const int occ = occupancy_for(fn, kSkThreads, p.smem);
+  p.grid = (int)std::min<long long>(p.units, (long long)num_sms() * occ);
+  const long long per = std::max<long long>(1, p.units / p.grid);
+  p.max_slots = (int)((p.stages_per_tile + per - 1) / per + 1);
+  return p;
+}
+
+static lbq_status run_lut3_skinny(const void* X, int M, const void* image, const Layout& L, void* Y, bool ybf16,
+                                  void* ws, size_t ws_bytes, cudaStream_t st) {
+  const SkPlan p = plan_lut3(L.K, L.N, M);
+  const size_t need = skinny_workspace_bytes(p, M);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(LBQ_ERR_INVALID_ARG, "workspace of %zu bytes is too small (need %zu)", ws_bytes, need);
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  CUtensorMap tx;
+  if (!make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)L.K, (uint64_t)M, (uint64_t)L.K * 2, 64,
+                    (uint32_t)M, CU_TENSOR_MAP_SWIZZLE_128B))
+    return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the LUT3 GEMV");
+  Lut3SkinnyArgs a{};
+  a.Y = Y;
+  a.partials = static_cast<float*>(ws);
+  a.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) +
+                                           align_up((size_t)p.row_tiles * p.max_slots * M * kSkRows * sizeof(float), 256));
+  a.i_region = img + L.off0;
+  a.t_region = img + L.off3;
+  a.K = L.K; a.N = L.N; a.M = M;
+  a.stages_per_tile = p.stages_per_tile; a.row_tiles = p.row_tiles; a.max_slots = p.max_slots; a.units = p.units;
+  a.y_bf16 = ybf16 ? 1 : 0;
+  const void* fn = p.nt == 1 ? (const void*)lut3_skinny_kernel<1> : (const void*)lut3_skinny_kernel<2>;
+  void* args[] = {&tx, &a};
+  return launch_kernel_ex(fn, dim3(p.grid), dim3(kSkThreads), p.smem, st, g_pdl != 0, args, "lut3 skinny launch");
+}
+
+static lbq_status run_lut3_gemm_tc(const void* X, int M, const void* image, const Layout& L, void* Y, bool ybf16,
+                                   cudaStream_t st) {
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  CUtensorMap tx, tq;
+  if (!make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)L.K, (uint64_t)M, (uint64_t)L.K * 2, kTcBK,
+                    kTcBM, CU_TENSOR_MAP_SWIZZLE_128B))
+    return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the LUT3 GEMM");
+  tq = tx;  // unused by the LUT3 producer
+  GemmTcArgs a{};
+  a.Y = Y;
+  a.s_region = img + L.off0;  // indices
+  a.z_region = img + L.off3;  // tables
+  a.M = M; a.N = L.N; a.K = L.K; a.gshift64 = 1;
+  a.m_tiles = (M + kTcBM - 1) / kTcBM;
+  a.n_tiles = (L.N + kTcBN - 1) / kTcBN;
+  a.k_blocks = L.K / kTcBK;
+  a.y_bf16 = ybf16 ? 1 : 0;
+  const void* fn = (const void*)gemm_tc_kernel<true, false, true>;
+  occupancy_for(fn, kTcThreads, kTcSmem);
+  const int grid = std::min(a.m_tiles * a.n_tiles, num_sms());
+  void* args[] = {&tx, &tq, &a};
+  return launch_kernel_ex(fn, dim3(grid), dim3(kTcThreads), kTcSmem, st, false, args, "LUT3 GEMM launch");
 }
 
 static lbq_status check_compute_args(const void* X, int x_dtype, int M, const void* image, void* Y, int y_dtype) {
@@ -487,18 +534,31 @@ lbq_status lbq_pack(const float* W, int K, int N, int group, int mode, void* ima
   const int block = 256;
   const unsigned grid = (unsigned)((work + block - 1) / block);
   if (mode == LBQ_MODE_SYM)
-    quantize_pack_int4_kernel<false><<<grid, block, 0, s>>>(W, K, N, group, img + L.off0, img + L.off1, nullptr,
-                                                             (int)L.s_stride, (int)L.z_stride);
+    quantize_pack_int4_kernel<false><<<grid, block, 0, s>>>(W, K, N, group, img + L.off0, img + L.off1, nullptr);
   else
-    quantize_pack_int4_kernel<true><<<grid, block, 0, s>>>(W, K, N, group, img + L.off0, img + L.off1, img + L.off2,
-                                                            (int)L.s_stride, (int)L.z_stride);
+    quantize_pack_int4_kernel<true><<<grid, block, 0, s>>>(W, K, N, group, img + L.off0, img + L.off1, img + L.off2);
   return launch_check("quantize_pack launch");
 }
 
 lbq_status lbq_pack_lut3(const uint8_t* idx, const uint8_t* codebooks, const uint8_t* exponents, int K, int N,
                          void* image, size_t image_bytes, void* stream) {
-  (void)idx; (void)codebooks; (void)exponents; (void)K; (void)N; (void)image; (void)image_bytes; (void)stream;
-  return fail(LBQ_ERR_UNSUPPORTED, "LUT3 packing is not built yet");
+  lbq_status st = check_lut3_shape(K, N);
+  if (st != LBQ_OK) return st;
+  if (!idx || !codebooks || !exponents || !image)
+    return fail(LBQ_ERR_INVALID_ARG, "idx, codebooks, exponents and image must be non-null");
+  if (!aligned16(image)) return fail(LBQ_ERR_INVALID_ARG, "image must be 16-byte aligned");
+  const Layout L = make_layout(K, N, 0, LBQ_MODE_LUT3);
+  if (image_bytes < L.total) return fail(LBQ_ERR_INVALID_ARG, "image buffer %zu bytes < %zu needed", image_bytes, L.total);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* img = static_cast<uint8_t*>(image);
+  write_header_kernel<<<1, 32, 0, s>>>(make_header(L), reinterpret_cast<ImageHeader*>(img));
+  if ((st = launch_check("header launch")) != LBQ_OK) return st;
+  if ((st = cuda_check(cudaMemsetAsync(img + L.off1, 0, L.total - L.off1, s), "clearing the table regions")) != LBQ_OK)
+    return st;
+  const long long work = (long long)(K / 64) * N;
+  pack_lut3_kernel<<<(unsigned)((work + 255) / 256), 256, 0, s>>>(idx, codebooks, exponents, K, N, img + L.off0,
+                                                                  img + L.off1, img + L.off2, img + L.off3);
+  return launch_check("pack_lut3 launch");
 }
 
 lbq_status lbq_workspace_size(int op, int M, int K, int N, int group, int mode, size_t* bytes) {
@@ -513,12 +573,21 @@ lbq_status lbq_workspace_size(int op, int M, int K, int N, int group, int mode, 
       const M1Plan p = plan_m1(K, N, group, mode == LBQ_MODE_ASYM, g_force_splits);
       *bytes = m1_workspace_bytes(p, N);
     } else if (M <= 16) {
-      const SkPlan p = plan_skinny(K, N, M, group, mode == LBQ_MODE_ASYM, g_force_splits);
-      *bytes = skinny_workspace_bytes(p, M, N);
+      // the plan depends on the activation dtype only through the kernel's
+      // occupancy; take the larger of the two
+      const SkPlan p0 = plan_skinny(K, N, M, group, mode == LBQ_MODE_ASYM, false);
+      const SkPlan p1 = plan_skinny(K, N, M, group, mode == LBQ_MODE_ASYM, true);
+      *bytes = std::max(skinny_workspace_bytes(p0, M), skinny_workspace_bytes(p1, M));
     }
     return LBQ_OK;
   }
-  if (op == 2) return check_lut3_shape(K, N);
+  if (op == 2) {
+    lbq_status st = check_lut3_shape(K, N);
+    if (st != LBQ_OK) return st;
+    if (M <= 0) return fail(LBQ_ERR_INVALID_ARG, "M must be positive");
+    if (M <= 16 && !g_force_tc) *bytes = skinny_workspace_bytes(plan_lut3(K, N, M), M);
+    return LBQ_OK;
+  }
   return fail(LBQ_ERR_INVALID_ARG, "op %d not in {0, 1, 2}", op);
 }
 
@@ -548,8 +617,14 @@ lbq_status lbq_gemm(const void* X, int x_dtype, int M, int K, int N, int group, 
 
 lbq_status lbq_lut3_gemm(const void* X, int x_dtype, int M, int K, int N, const void* image, void* Y, int y_dtype,
                          void* ws, size_t ws_bytes, void* stream) {
-  (void)X; (void)x_dtype; (void)M; (void)K; (void)N; (void)image; (void)Y; (void)y_dtype; (void)ws; (void)ws_bytes; (void)stream;
-  return fail(LBQ_ERR_UNSUPPORTED, "the LUT3 kernels are not built yet");
+  lbq_status st = check_lut3_shape(K, N);
+  if (st != LBQ_OK) return st;
+  if ((st = check_compute_args(X, x_dtype, M, image, Y, y_dtype)) != LBQ_OK) return st;
+  if (x_dtype != LBQ_DTYPE_BF16) return fail(LBQ_ERR_UNSUPPORTED, "LUT3 kernels take BF16 activations");
+  const Layout L = make_layout(K, N, 0, LBQ_MODE_LUT3);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M <= 16 && !g_force_tc) return run_lut3_skinny(X, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, ws, ws_bytes, s);
+  return run_lut3_gemm_tc(X, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);
 }
 
 lbq_status lbq_unpack_canonical(const void* image, int K, int N, int group, int mode, uint8_t* q_packed,
@@ -565,15 +640,26 @@ lbq_status lbq_unpack_canonical(const void* image, int K, int N, int group, int 
   const uint8_t* img = static_cast<const uint8_t*>(image);
   const long long work = (long long)(K / 2) * N;
   unpack_int4_kernel<<<(unsigned)((work + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      img + L.off0, img + L.off1, mode == LBQ_MODE_ASYM ? img + L.off2 : nullptr, K, N, group, (int)L.s_stride,
-      (int)L.z_stride, q_packed, scales, mode == LBQ_MODE_ASYM ? zp : nullptr);
+      img + L.off0, img + L.off1, mode == LBQ_MODE_ASYM ? img + L.off2 : nullptr, K, N, group, q_packed, scales,
+      mode == LBQ_MODE_ASYM ? zp : nullptr);
   return launch_check("unpack launch");
 }
 
 lbq_status lbq_unpack_lut3_canonical(const void* image, int K, int N, uint8_t* idx_stream, uint8_t* codebooks,
                                      uint8_t* exponents, void* stream) {
-  (void)image; (void)K; (void)N; (void)idx_stream; (void)codebooks; (void)exponents; (void)stream;
-  return fail(LBQ_ERR_UNSUPPORTED, "LUT3 is not built yet");
+  lbq_status st = check_lut3_shape(K, N);
+  if (st != LBQ_OK) return st;
+  if (!image || !idx_stream || !codebooks || !exponents)
+    return fail(LBQ_ERR_INVALID_ARG, "image, idx_stream, codebooks and exponents must be non-null");
+  ImageHeader h;
+  if ((st = read_header(image, &h)) != LBQ_OK) return st;
+  if ((st = check_header(h, K, N, 0, LBQ_MODE_LUT3)) != LBQ_OK) return st;
+  const Layout L = make_layout(K, N, 0, LBQ_MODE_LUT3);
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  const long long work = (long long)(K / 64) * N;
+  unpack_lut3_kernel<<<(unsigned)((work + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      img + L.off0, img + L.off1, img + L.off2, K, N, idx_stream, codebooks, exponents);
+  return launch_check("unpack_lut3 launch");
 }
 
 lbq_status lbq_dequant(const void* image, int K, int N, int group, int mode, float* W_out, void* stream) {
@@ -583,13 +669,19 @@ lbq_status lbq_dequant(const void* image, int K, int N, int group, int mode, flo
   ImageHeader h;
   if ((st = read_header(image, &h)) != LBQ_OK) return st;
   if ((st = check_header(h, K, N, group, mode)) != LBQ_OK) return st;
-  if (mode == LBQ_MODE_LUT3) return fail(LBQ_ERR_UNSUPPORTED, "LUT3 is not built yet");
+  if (mode == LBQ_MODE_LUT3) {
+    const Layout L = make_layout(K, N, 0, LBQ_MODE_LUT3);
+    const uint8_t* img = static_cast<const uint8_t*>(image);
+    const long long work = (long long)K * N;
+    dequant_lut3_kernel<<<(unsigned)((work + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        img + L.off0, img + L.off1, img + L.off2, K, N, W_out);
+    return launch_check("dequant_lut3 launch");
+  }
   const Layout L = make_layout(K, N, group, mode);
   const uint8_t* img = static_cast<const uint8_t*>(image);
   const long long work = (long long)K * N;
   dequant_int4_kernel<<<(unsigned)((work + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      img + L.off0, img + L.off1, mode == LBQ_MODE_ASYM ? img + L.off2 : nullptr, K, N, group, (int)L.s_stride,
-      (int)L.z_stride, W_out);
+      img + L.off0, img + L.off1, mode == LBQ_MODE_ASYM ? img + L.off2 : nullptr, K, N, group, W_out);
   return launch_check("dequant launch");
 }
 

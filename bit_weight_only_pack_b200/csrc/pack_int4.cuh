@@ -18,8 +18,7 @@ namespace lbq {
 template <bool ASYM>
 __global__ void __launch_bounds__(256) quantize_pack_int4_kernel(
     const float* __restrict__ W, int K, int N, int group,
-    uint8_t* __restrict__ q_region, uint8_t* __restrict__ s_region, uint8_t* __restrict__ z_region,
-    int s_stride, int z_stride) {
+    uint8_t* __restrict__ q_region, uint8_t* __restrict__ s_region, uint8_t* __restrict__ z_region) {
   const int G = K / group;
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= (long long)G * N) return;
@@ -72,8 +71,8 @@ __global__ void __launch_bounds__(256) quantize_pack_int4_kernel(
     }
     *reinterpret_cast<uint4*>(row + (size_t)(c0 + c) * 16) = make_uint4(words[0], words[1], words[2], words[3]);
   }
-  reinterpret_cast<uint16_t*>(s_region + (size_t)n * s_stride)[gi] = __half_as_ushort(s16);
-  if (ASYM) reinterpret_cast<int8_t*>(z_region + (size_t)n * z_stride)[gi] = (int8_t)(int)zp;
+  reinterpret_cast<uint16_t*>(s_region)[meta_index(n, gi, G)] = __half_as_ushort(s16);
+  if (ASYM) reinterpret_cast<int8_t*>(z_region)[meta_index(n, gi, G)] = (int8_t)(int)zp;
 }
 
 __device__ __forceinline__ uint32_t image_code(const uint8_t* q_region, int K, int k, int n) {
@@ -85,7 +84,7 @@ __device__ __forceinline__ uint32_t image_code(const uint8_t* q_region, int K, i
 // zero points transposed back to [K/group][N].
 __global__ void __launch_bounds__(256) unpack_int4_kernel(
     const uint8_t* __restrict__ q_region, const uint8_t* __restrict__ s_region,
-    const uint8_t* __restrict__ z_region, int K, int N, int group, int s_stride, int z_stride,
+    const uint8_t* __restrict__ z_region, int K, int N, int group,
     uint8_t* __restrict__ q_packed, uint16_t* __restrict__ s_out, int8_t* __restrict__ z_out) {
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long nbytes = (long long)(K / 2) * N;
@@ -100,9 +99,8 @@ __global__ void __launch_bounds__(256) unpack_int4_kernel(
   if (t < (long long)G * N) {
     const int n = (int)(t % N);
     const int gi = (int)(t / N);
-    s_out[t] = reinterpret_cast<const uint16_t*>(s_region + (size_t)n * s_stride)[gi];
-    if (z_out != nullptr && z_region != nullptr)
-      z_out[t] = reinterpret_cast<const int8_t*>(z_region + (size_t)n * z_stride)[gi];
+    s_out[t] = reinterpret_cast<const uint16_t*>(s_region)[meta_index(n, gi, G)];
+    if (z_out != nullptr && z_region != nullptr) z_out[t] = reinterpret_cast<const int8_t*>(z_region)[meta_index(n, gi, G)];
   }
 }
 
@@ -110,15 +108,14 @@ __global__ void __launch_bounds__(256) unpack_int4_kernel(
 // FP16 scale multiply exactly in FP32).
 __global__ void __launch_bounds__(256) dequant_int4_kernel(
     const uint8_t* __restrict__ q_region, const uint8_t* __restrict__ s_region,
-    const uint8_t* __restrict__ z_region, int K, int N, int group, int s_stride, int z_stride,
-    float* __restrict__ W_out) {
+    const uint8_t* __restrict__ z_region, int K, int N, int group, float* __restrict__ W_out) {
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= (long long)K * N) return;
   const int n = (int)(t % N);
   const int k = (int)(t / N);
-  const int gi = k / group;
-  const float s = h2f_bits(reinterpret_cast<const uint16_t*>(s_region + (size_t)n * s_stride)[gi]);
-  const int z = z_region ? (int)reinterpret_cast<const int8_t*>(z_region + (size_t)n * z_stride)[gi] : 8;
+  const int gi = k / group, G = K / group;
+  const float s = h2f_bits(reinterpret_cast<const uint16_t*>(s_region)[meta_index(n, gi, G)]);
+  const int z = z_region ? (int)reinterpret_cast<const int8_t*>(z_region)[meta_index(n, gi, G)] : 8;
   const int q = (int)image_code(q_region, K, k, n);
   W_out[t] = (float)(q - z) * s;
 }

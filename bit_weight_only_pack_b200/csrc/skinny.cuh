@@ -16,21 +16,24 @@
 //    D = sum x (1024 + q) - (1024 + z) sum x = sum x (q - z), accumulated in
 //    FP32 inside the tensor core. No weight is ever rounded.
 //  * Per group, acc += s[row] * D (FP32 FMAs on the accumulator fragment);
-//    FP16's upper-nibble class carries a factor 16, removed by using s/16.
+//    FP16's upper-nibble class carries a factor 16, removed before scaling.
 //  * The weight rows are the MMA "M" side (16 output channels per
 //    mma.m16n8k16) and the batch is the MMA "N" side (8 or 16 columns), so no
 //    batch padding to 128 is streamed ("no swap-AB" is one of the reasons the
 //    vLLM LUT-B kernel loses at small batch).
 //  * Producer warp: per 256-k stage, TMA loads of a 128-row x 128-byte code
-//    tile (128-byte swizzle), the 64-k activation boxes (128-byte swizzle) and
-//    16-byte boxes of the rows' scales / zero points, completing on one
-//    mbarrier; a ring of kSkStages stages feeds 8 consumer warps (16 rows
+//    tile (128-byte swizzle) and the 64-k activation boxes (128-byte
+//    swizzle), and one bulk copy each of the tile's scales / zero points for
+//    the stage's groups (contiguous in the 128-channel-tiled image), all
+//    completing on one mbarrier; a ring of kSkStages stages feeds 8 consumer warps (16 rows
 //    each). ldmatrix.x4 hands each thread the code words of rows r and r+8 for
 //    two 32-k chunks; within a chunk the k order is permuted identically for A
 //    and B so that thread t's MMA k-slots are exactly the 16 bytes of
 //    activations it reads with one shared-memory load.
-//  * Split-K: FP32 partials and a last-CTA reduction in slice order (the
-//    workspace's counters are reset, so it is left zeroed).
+//  * Stream-K: every CTA takes an equal contiguous range of (row tile, stage)
+//    units, so all SMs stream the same number of bytes whatever the shape;
+//    shared row tiles are finished by the CTA completing their stage count
+//    (FP32 partials added in slot order; counters reset, workspace left zeroed).
 #pragma once
 
 #include "common.cuh"
@@ -43,26 +46,34 @@ constexpr int kSkWarps = 8;                 // consumer warps, 16 rows each
 constexpr int kSkRows = kSkWarps * 16;      // rows of W per CTA tile
 constexpr int kSkThreads = (kSkWarps + 1) * 32;
 constexpr int kSkWBytes = kSkRows * 128;    // 16 KB of codes per 256-k stage
-constexpr int kSkSBytes = kSkRows * 16;     // 16-byte scale box per row
-constexpr int kSkZBytes = kSkRows * 16;     // 16-byte zero-point box per row
+constexpr int kSkSBytes = 8 * kSkRows * 2;  // scales of up to 8 groups for the tile's 128 rows
+constexpr int kSkZBytes = 8 * kSkRows;      // zero points of up to 8 groups
 
+// Stream-K work split: the (row tile, 256-k stage) units, row tile major,
+// are divided into equal contiguous ranges, one per CTA, so every CTA streams
+// the same number of bytes. A row tile covered by one CTA is written directly;
+// a row tile shared by several CTAs gets FP32 partials in per-CTA slots, and
+// the CTA that completes its stage count adds the slots in order.
 struct SkinnyArgs {
   void* Y;                   // [M][N]
-  float* partials;           // [splits][M][N]
+  float* partials;           // [row_tiles][max_slots][M][kSkRows]
   unsigned int* counters;    // [row_tiles]
-  int K, N, M;
-  int stages_per_split, splits, row_tiles, total_tiles;
+  const uint8_t* s_region;   // 128-channel-tiled scales of the image
+  const uint8_t* z_region;   // 128-channel-tiled zero points (ASYM)
+  int K, N, M, G;
+  int stages_per_tile, row_tiles, max_slots;
+  long long units;           // row_tiles * stages_per_tile
   int y_bf16;
 };
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1, bool bf16) {
   if (bf16)
-    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
                  "{%8, %9}, {%0, %1, %2, %3};"
                  : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
                  : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
   else
-    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
                  "{%8, %9}, {%0, %1, %2, %3};"
                  : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
                  : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -106,10 +117,27 @@ __device__ __forceinline__ void zero_consts(int z, uint32_t& c1, uint32_t& c2) {
   }
 }
 
+// CTA that owns unit u when `units` units are split evenly over `grid` CTAs.
+__device__ __forceinline__ int sk_owner(long long u, long long units, int grid) {
+  return (int)(((u + 1) * grid - 1) / units);
+}
+
+__device__ __forceinline__ void mma_16816_zc(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1, bool bf16) {
+  if (bf16)
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                 "{%8, %9}, {%10, %10, %10, %10};"
+                 : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+  else
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                 "{%8, %9}, {%10, %10, %10, %10};"
+                 : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
 template <bool BF16, bool ASYM, int NT, int GC, bool KFULL>
 __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
-    const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tx,
-    const __grid_constant__ CUtensorMap ts, const __grid_constant__ CUtensorMap tz, const SkinnyArgs a) {
+    const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tx, const SkinnyArgs a) {
   constexpr int kXBox = NT * 1024;  // one 64-k activation box (8*NT rows x 128 B)
   constexpr int kOffX = kSkWBytes;
   constexpr int kOffS = kOffX + 4 * kXBox;
@@ -119,11 +147,15 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
   __shared__ __align__(8) uint64_t full_bar[kSkStages];
   __shared__ __align__(8) uint64_t empty_bar[kSkStages];
   __shared__ unsigned int s_last;
-  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+  __shared__ uint2 zlut[ASYM ? 256 : 1];  // z + 128 -> constant A operands {class A, class B}
+  // ring base: the first 1024-byte boundary of the dynamic shared memory
+  uint8_t* ring = dsmem + ((1024u - (smem_u32(dsmem) & 1023u)) & 1023u);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int K = a.K, M = a.M;
-  const int total_stages = (K + 255) / 256;
+  const int S_t = a.stages_per_tile;
+  const long long u_begin = (long long)blockIdx.x * a.units / gridDim.x;
+  const long long u_end = (long long)(blockIdx.x + 1) * a.units / gridDim.x;
 
   if (tid == 0) {
     for (int i = 0; i < kSkStages; ++i) {
@@ -131,6 +163,13 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
       mbar_init(&empty_bar[i], kSkWarps);
     }
     fence_barrier_init();
+  }
+  if (ASYM) {
+    for (int i = tid; i < 256; i += kSkThreads) {
+      const float z = (float)(i - 128);
+      zlut[i] = BF16 ? make_uint2(pack_bf16x2(-(128.0f + z)), 0u)
+                     : make_uint2(pack_f16x2(-(1024.0f + z)), pack_f16x2(-(1024.0f + 16.0f * z)));
+    }
   }
   __syncthreads();
   asm volatile("griddepcontrol.launch_dependents;" :::);
@@ -140,27 +179,38 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
     if (lane == 0) {
       tma_prefetch_desc(&tw);
       tma_prefetch_desc(&tx);
-      tma_prefetch_desc(&ts);
-      if (ASYM) tma_prefetch_desc(&tz);
-      asm volatile("griddepcontrol.wait;" ::: "memory");  // X may come from the previous kernel
+      // The weights (codes, scales, zero points) are only read, so the first
+      // ring slots are filled before waiting on the previous kernel; the
+      // activations, which that kernel may write, are loaded after the wait.
+      const int nfirst = (int)min((long long)kSkStages, u_end - u_begin);
       int it = 0;
-      for (int tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x) {
-        const int split = tile / a.row_tiles;
-        const int rt = tile - split * a.row_tiles;
-        const int s0 = split * a.stages_per_split;
-        const int s1 = min(s0 + a.stages_per_split, total_stages);
-        for (int st = s0; st < s1; ++st, ++it) {
-          const int slot = it % kSkStages;
-          if (it >= kSkStages && !mbar_wait(&empty_bar[slot], ((it / kSkStages) & 1) ^ 1)) return;
-          uint8_t* dst = ring + (size_t)slot * kSlot;
-          const int gs0 = st * 8 / GC;  // first group of the stage
-          const int nxb = KFULL ? 4 : min(4, (K - st * 256 + 63) / 64);  // activation boxes that start inside K
-          mbar_arrive_expect_tx(&full_bar[slot],
-                                (uint32_t)(kSkWBytes + nxb * M * 128 + kSkSBytes + (ASYM ? kSkZBytes : 0)));
-          tma_load_2d(dst, &tw, st * 128, rt * kSkRows, &full_bar[slot]);
+      for (long long u = u_begin; u < u_end; ++u, ++it) {
+        const int rt = (int)(u / S_t);
+        const int st = (int)(u - (long long)rt * S_t);
+        const int slot = it % kSkStages;
+        if (it >= kSkStages && !mbar_wait(&empty_bar[slot], ((it / kSkStages) & 1) ^ 1)) return;
+        uint8_t* dst = ring + (size_t)slot * kSlot;
+        const int gs0 = st * 8 / GC;  // first group of the stage
+        const int ng = min(8 / GC, a.G - gs0);  // groups of the stage
+        const int nxb = KFULL ? 4 : min(4, (K - st * 256 + 63) / 64);  // activation boxes that start inside K
+        mbar_arrive_expect_tx(&full_bar[slot],
+                              (uint32_t)(kSkWBytes + nxb * M * 128 + ng * kSkRows * (ASYM ? 3 : 2)));
+        tma_load_2d(dst, &tw, st * 128, rt * kSkRows, &full_bar[slot]);
+        const size_t meta0 = ((size_t)rt * a.G + gs0) * kSkRows;  // element index of (tile rt, group gs0, row 0)
+        bulk_load(dst + kOffS, a.s_region + meta0 * 2, (uint32_t)(ng * kSkRows * 2), &full_bar[slot]);
+        if (ASYM) bulk_load(dst + kOffZ, a.z_region + meta0, (uint32_t)(ng * kSkRows), &full_bar[slot]);
+        if (it + 1 == nfirst) {
+          asm volatile("griddepcontrol.wait;" ::: "memory");  // X may come from the previous kernel
+          for (int i = 0; i <= it; ++i) {  // activations of the slots filled so far
+            const long long ui = u_begin + i;
+            const int sti = (int)(ui - (ui / S_t) * S_t);
+            const int nxi = KFULL ? 4 : min(4, (K - sti * 256 + 63) / 64);
+            uint8_t* di = ring + (size_t)(i % kSkStages) * kSlot;
+            for (int j = 0; j < nxi; ++j)
+              tma_load_2d(di + kOffX + j * kXBox, &tx, sti * 256 + 64 * j, 0, &full_bar[i % kSkStages]);
+          }
+        } else if (it >= nfirst) {
           for (int j = 0; j < nxb; ++j) tma_load_2d(dst + kOffX + j * kXBox, &tx, st * 256 + 64 * j, 0, &full_bar[slot]);
-          tma_load_2d(dst + kOffS, &ts, (gs0 / 8) * 8, rt * kSkRows, &full_bar[slot]);
-          if (ASYM) tma_load_2d(dst + kOffZ, &tz, (gs0 / 16) * 16, rt * kSkRows, &full_bar[slot]);
         }
       }
     }
@@ -172,8 +222,9 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
   const int lrow = warp * 16 + g;  // this thread's rows: lrow and lrow + 8
   // ldmatrix row address of this lane: matrix i = lane/8 -> rows +8*(i&1), chunk +(i>>1)
   const int lm_row = warp * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
-  const uint32_t lm_off[4] = {sw128(lm_row, 0 + (lane >> 4)), sw128(lm_row, 2 + (lane >> 4)),
-                              sw128(lm_row, 4 + (lane >> 4)), sw128(lm_row, 6 + (lane >> 4))};
+  uint32_t lm_off[4];
+#pragma unroll
+  for (int cp = 0; cp < 4; ++cp) lm_off[cp] = sw128(lm_row, 2 * cp + (lane >> 4));
   // activation fragment offsets of this thread: column m = g + 8n, chunk half (ci & 1)
   uint32_t x_off[NT][2];
   bool x_ok[NT];
@@ -183,8 +234,8 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
     x_off[n][0] = (uint32_t)(kOffX + sw128(g + 8 * n, t));
     x_off[n][1] = (uint32_t)(kOffX + sw128(g + 8 * n, 4 + t));
   }
-  const uint32_t s_off_r = (uint32_t)(kOffS + lrow * 16), s_off_r8 = s_off_r + 8 * 16;
-  const uint32_t z_off_r = (uint32_t)(kOffZ + lrow * 16), z_off_r8 = z_off_r + 8 * 16;
+  const int s_off_r = kOffS + lrow * 2, s_off_r8 = s_off_r + 8 * 2;
+  const int z_off_r = kOffZ + lrow, z_off_r8 = z_off_r + 8;
   // constant A operands of the offset-removing MMAs (symmetric: z = 8)
   uint32_t ca_r = BF16 ? pack_bf16x2(-136.0f) : pack_f16x2(-1032.0f);
   uint32_t cb_r = BF16 ? 0u : pack_f16x2(-1152.0f);  // -(1024 + 16*8)
@@ -192,11 +243,11 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
 
   int it = 0;
   bool ok = true;
-  for (int tile = blockIdx.x; tile < a.total_tiles && ok; tile += gridDim.x) {
-    const int split = tile / a.row_tiles;
-    const int rt = tile - split * a.row_tiles;
-    const int s0 = split * a.stages_per_split;
-    const int s1 = min(s0 + a.stages_per_split, total_stages);
+  long long u = u_begin;
+  while (u < u_end && ok) {
+    const int rt = (int)(u / S_t);
+    const int st0 = (int)(u - (long long)rt * S_t);
+    const int st1 = (int)min((long long)S_t, st0 + (u_end - u));
     float acc[NT][4];
 #pragma unroll
     for (int n = 0; n < NT; ++n)
@@ -205,100 +256,86 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
     float dA[NT][4], dB[NT][4];
     float s_r = 0.0f, s_r8 = 0.0f;
 
-    for (int st = s0; st < s1; ++st, ++it) {
+    for (int st = st0; st < st1; ++st, ++it) {
       const int slot = it % kSkStages;
       if (!mbar_wait(&full_bar[slot], (it / kSkStages) & 1)) { ok = false; break; }
-      const uint32_t sb = smem_u32(ring + (size_t)slot * kSlot);
+      const uint8_t* sp = ring + (size_t)slot * kSlot;
+      const uint32_t sb = smem_u32(sp);
       const int k0 = st * 256;
-      const int gs0 = st * 8 / GC;
-      const int sx0 = (gs0 / 8) * 8, zx0 = (gs0 / 16) * 16;
+      uint32_t wr[4][4];
 #pragma unroll
-      for (int cp = 0; cp < 4; ++cp) {
-        if (!KFULL && k0 + 64 * cp >= K) continue;
-        uint32_t wr[4];
-        ldmatrix_x4(wr, sb + lm_off[cp]);
+      for (int cp = 0; cp < 4; ++cp) ldmatrix_x4(wr[cp], sb + lm_off[cp]);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int ci = 2 * cp + h;
-          if (!KFULL && k0 + 32 * ci >= K) continue;
-          if (ci % GC == 0) {
-            const int gl = gs0 + ci / GC;
-            uint16_t b0, b1;
-            asm volatile("ld.shared.u16 %0, [%1];" : "=h"(b0) : "r"(sb + s_off_r + (gl - sx0) * 2));
-            asm volatile("ld.shared.u16 %0, [%1];" : "=h"(b1) : "r"(sb + s_off_r8 + (gl - sx0) * 2));
-            s_r = h2f_bits(b0);
-            s_r8 = h2f_bits(b1);
-            if (ASYM) {
-              int z0, z1;
-              asm volatile("ld.shared.s8 %0, [%1];" : "=r"(z0) : "r"(sb + z_off_r + (gl - zx0)));
-              asm volatile("ld.shared.s8 %0, [%1];" : "=r"(z1) : "r"(sb + z_off_r8 + (gl - zx0)));
-              if (BF16) {
-                ca_r = pack_bf16x2(-(128.0f + (float)z0));
-                ca_r8 = pack_bf16x2(-(128.0f + (float)z1));
-              } else {
-                ca_r = pack_f16x2(-(1024.0f + (float)z0));
-                ca_r8 = pack_f16x2(-(1024.0f + (float)z1));
-                cb_r = pack_f16x2(-(1024.0f + 16.0f * (float)z0));
-                cb_r8 = pack_f16x2(-(1024.0f + 16.0f * (float)z1));
-              }
-            }
-#pragma unroll
-            for (int n = 0; n < NT; ++n)
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                dA[n][i] = 0.0f;
-                dB[n][i] = 0.0f;
-              }
+      for (int ci = 0; ci < 8; ++ci) {
+        if (!KFULL && k0 + 32 * ci >= K) continue;
+        const bool group_start = (ci % GC == 0);
+        if (group_start) {
+          const int gl = ci / GC;  // group within the stage
+          s_r = h2f_bits(*reinterpret_cast<const uint16_t*>(sp + s_off_r + gl * kSkRows * 2));
+          s_r8 = h2f_bits(*reinterpret_cast<const uint16_t*>(sp + s_off_r8 + gl * kSkRows * 2));
+          if (ASYM) {
+            const int z0 = *reinterpret_cast<const int8_t*>(sp + z_off_r + gl * kSkRows);
+            const int z1 = *reinterpret_cast<const int8_t*>(sp + z_off_r8 + gl * kSkRows);
+            const uint2 c0 = zlut[z0 + 128], c1 = zlut[z1 + 128];
+            ca_r = c0.x; cb_r = c0.y;
+            ca_r8 = c1.x; cb_r8 = c1.y;
           }
-          const uint32_t wa = wr[h ? 2 : 0], wb = wr[h ? 3 : 1];
-          const uint32_t ca[4] = {ca_r, ca_r8, ca_r, ca_r8};
-          if (!BF16) {
-            // class A: (k0,k1) (k4,k5) = 1024+q;  class B: (k2,k3) (k6,k7) = 1024+16q
-            const uint32_t ta = wa >> 8, tb = wb >> 8;
-            const uint32_t aA[4] = {and_or(wa, 0x000F000Fu, 0x64006400u), and_or(wb, 0x000F000Fu, 0x64006400u),
-                                    and_or(ta, 0x000F000Fu, 0x64006400u), and_or(tb, 0x000F000Fu, 0x64006400u)};
-            const uint32_t aB[4] = {and_or(wa, 0x00F000F0u, 0x64006400u), and_or(wb, 0x00F000F0u, 0x64006400u),
-                                    and_or(ta, 0x00F000F0u, 0x64006400u), and_or(tb, 0x00F000F0u, 0x64006400u)};
-            const uint32_t cb[4] = {cb_r, cb_r8, cb_r, cb_r8};
+        }
+        const uint32_t wa = wr[ci >> 1][(ci & 1) ? 2 : 0], wb = wr[ci >> 1][(ci & 1) ? 3 : 1];
+        const uint32_t ca[4] = {ca_r, ca_r8, ca_r, ca_r8};
+        if (!BF16) {
+          // class A: (k0,k1) (k4,k5) = 1024+q;  class B: (k2,k3) (k6,k7) = 1024+16q
+          const uint32_t ta = wa >> 8, tb = wb >> 8;
+          const uint32_t aA[4] = {and_or(wa, 0x000F000Fu, 0x64006400u), and_or(wb, 0x000F000Fu, 0x64006400u),
+                                  and_or(ta, 0x000F000Fu, 0x64006400u), and_or(tb, 0x000F000Fu, 0x64006400u)};
+          const uint32_t aB[4] = {and_or(wa, 0x00F000F0u, 0x64006400u), and_or(wb, 0x00F000F0u, 0x64006400u),
+                                  and_or(ta, 0x00F000F0u, 0x64006400u), and_or(tb, 0x00F000F0u, 0x64006400u)};
+          const uint32_t cb[4] = {cb_r, cb_r8, cb_r, cb_r8};
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
-              uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-              if (x_ok[n]) xv = lds128(sb + x_off[n][h] + (ci >> 1) * kXBox);
+          for (int n = 0; n < NT; ++n) {
+            uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+            if (x_ok[n]) xv = *reinterpret_cast<const uint4*>(sp + x_off[n][ci & 1] + (ci >> 1) * kXBox);
+            if (group_start) {
+              mma_16816_zc(dA[n], aA, xv.x, xv.z, false);
+              mma_16816_zc(dB[n], aB, xv.y, xv.w, false);
+            } else {
               mma_16816(dA[n], aA, xv.x, xv.z, false);
-              mma_16816(dA[n], ca, xv.x, xv.z, false);
               mma_16816(dB[n], aB, xv.y, xv.w, false);
-              mma_16816(dB[n], cb, xv.y, xv.w, false);
             }
-          } else {
-            const uint32_t a0[4] = {and_or(wa, 0x000F000Fu, 0x43004300u), and_or(wb, 0x000F000Fu, 0x43004300u),
-                                    and_or(wa >> 4, 0x000F000Fu, 0x43004300u), and_or(wb >> 4, 0x000F000Fu, 0x43004300u)};
-            const uint32_t a1[4] = {and_or(wa >> 8, 0x000F000Fu, 0x43004300u), and_or(wb >> 8, 0x000F000Fu, 0x43004300u),
-                                    and_or(wa >> 12, 0x000F000Fu, 0x43004300u), and_or(wb >> 12, 0x000F000Fu, 0x43004300u)};
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-              uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-              if (x_ok[n]) xv = lds128(sb + x_off[n][h] + (ci >> 1) * kXBox);
-              mma_16816(dA[n], a0, xv.x, xv.y, true);
-              mma_16816(dA[n], ca, xv.x, xv.y, true);
-              mma_16816(dA[n], a1, xv.z, xv.w, true);
-              mma_16816(dA[n], ca, xv.z, xv.w, true);
-            }
+            mma_16816(dA[n], ca, xv.x, xv.z, false);
+            mma_16816(dB[n], cb, xv.y, xv.w, false);
           }
-          const bool group_end = (ci % GC == GC - 1) || (!KFULL && k0 + 32 * ci + 32 >= K);
-          if (group_end) {
+        } else {
+          const uint32_t a0[4] = {and_or(wa, 0x000F000Fu, 0x43004300u), and_or(wb, 0x000F000Fu, 0x43004300u),
+                                  and_or(wa >> 4, 0x000F000Fu, 0x43004300u), and_or(wb >> 4, 0x000F000Fu, 0x43004300u)};
+          const uint32_t a1[4] = {and_or(wa >> 8, 0x000F000Fu, 0x43004300u), and_or(wb >> 8, 0x000F000Fu, 0x43004300u),
+                                  and_or(wa >> 12, 0x000F000Fu, 0x43004300u), and_or(wb >> 12, 0x000F000Fu, 0x43004300u)};
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
-              acc[n][0] = fmaf(s_r, dA[n][0], acc[n][0]);
-              acc[n][1] = fmaf(s_r, dA[n][1], acc[n][1]);
-              acc[n][2] = fmaf(s_r8, dA[n][2], acc[n][2]);
-              acc[n][3] = fmaf(s_r8, dA[n][3], acc[n][3]);
-              if (!BF16) {
-                acc[n][0] = fmaf(s_r * 0.0625f, dB[n][0], acc[n][0]);
-                acc[n][1] = fmaf(s_r * 0.0625f, dB[n][1], acc[n][1]);
-                acc[n][2] = fmaf(s_r8 * 0.0625f, dB[n][2], acc[n][2]);
-                acc[n][3] = fmaf(s_r8 * 0.0625f, dB[n][3], acc[n][3]);
-              }
+          for (int n = 0; n < NT; ++n) {
+            uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+            if (x_ok[n]) xv = *reinterpret_cast<const uint4*>(sp + x_off[n][ci & 1] + (ci >> 1) * kXBox);
+            // dA: first half of the chunk's k + the second half's correction; dB the other way round
+            if (group_start) {
+              mma_16816_zc(dA[n], a0, xv.x, xv.y, true);
+              mma_16816_zc(dB[n], a1, xv.z, xv.w, true);
+            } else {
+              mma_16816(dA[n], a0, xv.x, xv.y, true);
+              mma_16816(dB[n], a1, xv.z, xv.w, true);
             }
+            mma_16816(dB[n], ca, xv.x, xv.y, true);
+            mma_16816(dA[n], ca, xv.z, xv.w, true);
+          }
+        }
+        const bool group_end = (ci % GC == GC - 1) || (!KFULL && k0 + 32 * ci + 32 >= K);
+        if (group_end) {
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            // FP16: D = dA + dB/16 (class B carries 16 q); BF16: D = dA + dB
+            const float f = BF16 ? 1.0f : 0.0625f;
+            acc[n][0] = fmaf(s_r, fmaf(dB[n][0], f, dA[n][0]), acc[n][0]);
+            acc[n][1] = fmaf(s_r, fmaf(dB[n][1], f, dA[n][1]), acc[n][1]);
+            acc[n][2] = fmaf(s_r8, fmaf(dB[n][2], f, dA[n][2]), acc[n][2]);
+            acc[n][3] = fmaf(s_r8, fmaf(dB[n][3], f, dA[n][3]), acc[n][3]);
           }
         }
       }
@@ -309,45 +346,58 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
 
     // ---------------------------------------------------------------- output
     const int n0 = rt * kSkRows + lrow;
+    const bool whole = (st0 == 0 && st1 == S_t);
+    if (whole) {
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
+      for (int n = 0; n < NT; ++n)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int m = 8 * n + 2 * t + (i & 1);
-        const int nn = n0 + ((i & 2) ? 8 : 0);
-        if (m < M && nn < a.N) {
-          if (a.splits == 1) store_out(a.Y, (size_t)m * a.N + nn, acc[n][i], a.y_bf16);
-          else a.partials[((size_t)split * M + m) * a.N + nn] = acc[n][i];
+        for (int i = 0; i < 4; ++i) {
+          const int m = 8 * n + 2 * t + (i & 1);
+          const int nn = n0 + ((i & 2) ? 8 : 0);
+          if (m < M && nn < a.N) store_out(a.Y, (size_t)m * a.N + nn, acc[n][i], a.y_bf16);
         }
-      }
-    }
-    if (a.splits > 1) {
+    } else {
+      const long long tile_u0 = (long long)rt * S_t;
+      const int first = sk_owner(tile_u0, a.units, gridDim.x);
+      const int slot_id = blockIdx.x - first;
+      float* base = a.partials + (size_t)rt * a.max_slots * M * kSkRows;
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = 8 * n + 2 * t + (i & 1);
+          const int r = lrow + ((i & 2) ? 8 : 0);
+          if (m < M) base[((size_t)slot_id * M + m) * kSkRows + r] = acc[n][i];
+        }
       __threadfence();
       asm volatile("bar.sync 1, %0;" :: "r"(kSkWarps * 32) : "memory");
       if (tid == 0) {
-        const unsigned int prev = atomicAdd(&a.counters[rt], 1u);
-        s_last = (prev == (unsigned int)(a.splits - 1));
+        const unsigned int add = (unsigned int)(st1 - st0);
+        const unsigned int prev = atomicAdd(&a.counters[rt], add);
+        s_last = (prev + add == (unsigned int)S_t);
       }
       asm volatile("bar.sync 1, %0;" :: "r"(kSkWarps * 32) : "memory");
       if (s_last) {
         __threadfence();
+        const int nslots = sk_owner(tile_u0 + S_t - 1, a.units, gridDim.x) - first + 1;
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
+        for (int n = 0; n < NT; ++n)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int m = 8 * n + 2 * t + (i & 1);
-            const int nn = n0 + ((i & 2) ? 8 : 0);
+            const int r = lrow + ((i & 2) ? 8 : 0);
+            const int nn = rt * kSkRows + r;
             if (m < M && nn < a.N) {
               float sum = 0.0f;
-              for (int sp = 0; sp < a.splits; ++sp) sum += __ldcg(a.partials + ((size_t)sp * M + m) * a.N + nn);
+              for (int sl = 0; sl < nslots; ++sl) sum += __ldcg(base + ((size_t)sl * M + m) * kSkRows + r);
               store_out(a.Y, (size_t)m * a.N + nn, sum, a.y_bf16);
             }
           }
-        }
         if (tid == 0) a.counters[rt] = 0u;
       }
       asm volatile("bar.sync 1, %0;" :: "r"(kSkWarps * 32) : "memory");
     }
+    u += st1 - st0;
   }
 }
 
