@@ -1,0 +1,158 @@
+"""3-bit LUT parity on the GPU: the packed image's indices, codebooks and
+exponents recovered bit-exactly, the decode exact against the oracle, and the
+GEMV / GEMM outputs within |y - y_ref| <= 4e-3*S + ulp16(|y_ref|)."""
+
+import numpy as np
+import pytest
+
+import workloads
+from helpers import check_outputs, sample_columns
+from oracle import lut3
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch():
+    import torch
+    assert torch.cuda.is_available(), "these tests need a CUDA device"
+    return torch
+
+
+@pytest.fixture(scope="module")
+def lbq():
+    import bit_weight_only_pack_b200 as lbq
+    return lbq
+
+
+def _inputs(seed, K, N):
+    idx, cb, ex = workloads.lut3_host(seed, K, N)
+    if K >= 128 and N >= 16:
+        # planted edge cases: a tile whose codebook holds the E4M3 extremes
+        # (+-448, +-smallest subnormal, +-0, +-1), every entry in use; a tile
+        # whose indices are all 7; a tile with a tiny and one with a large
+        # exponent (kept small enough that FP16 outputs stay finite)
+        idx[:64, :8] = np.arange(64)[:, None] % 8
+        cb[0, 0] = [0x7E, 0xFE, 0x01, 0x81, 0x00, 0x80, 0x38, 0xB8]
+        idx[64:128, :8] = 7
+        ex[1, 0] = 127 - 60
+        ex[0, 1] = 127 + 4
+    return idx, cb, ex
+
+
+def _image(torch, lbq, idx, cb, ex):
+    return lbq.pack_lut3(*(torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in (idx, cb, ex)))
+
+
+PACK_SHAPES = [
+    (4096, 14336),   # the 3-bit LUT workload
+    (64, 8),         # one tile
+    (320, 200),      # K not a multiple of 256, N not a multiple of 128
+    (1024, 136),
+]
+
+
+@pytest.mark.parametrize("K,N", PACK_SHAPES)
+def test_pack_unpack_and_decode_bit_exact(torch, lbq, K, N):
+    idx, cb, ex = _inputs(40 + K + N, K, N)
+    img = _image(torch, lbq, idx, cb, ex)
+    stream, cb_out, ex_out = lbq.unpack_lut3_canonical(img, K, N)
+    if K * N > 1 << 22:  # full size: compare the canonical stream on a slice of tiles
+        kt = slice(0, 4)
+        assert np.array_equal(stream.cpu().numpy()[kt], lut3.pack_indices(idx[:256]))
+        assert np.array_equal(lut3.unpack_indices(stream.cpu().numpy()), idx)
+    else:
+        assert np.array_equal(stream.cpu().numpy(), lut3.pack_indices(idx))
+    assert np.array_equal(cb_out.cpu().numpy(), cb)
+    assert np.array_equal(ex_out.cpu().numpy(), ex)
+    cols = sample_columns(N // 8, 64, seed=K) if K * N > 1 << 22 else np.arange(N // 8)
+    ch = (cols[:, None] * 8 + np.arange(8)[None, :]).reshape(-1)
+    W = lbq.dequant(img, K, N, 0, "lut3").cpu().numpy()[:, ch]
+    ref = lut3.dequant(idx[:, ch], cb[:, cols], ex[:, cols])
+    assert np.array_equal(W.astype(np.float64), ref)
+
+
+def _check_gemm(torch, lbq, idx, cb, ex, img, X, groups=None, y_dtype=None):
+    """Run lut3_gemm and check it against the oracle on the 8-channel groups given (all by default)."""
+    K, N = idx.shape
+    Y = lbq.lut3_gemm(X.cuda(), img, N, y_dtype=y_dtype)
+    torch.cuda.synchronize()
+    if groups is None:
+        groups = np.arange(N // 8)
+    ch = (groups[:, None] * 8 + np.arange(8)[None, :]).reshape(-1)
+    deq = lut3.dequant(np.ascontiguousarray(idx[:, ch]), cb[:, groups], ex[:, groups])
+    return check_outputs(Y.cpu(), X, deq, ch), Y
+
+
+SKINNY_SHAPES = [
+    (4096, 1024),    # whole 256-k stages, whole 128-channel tiles
+    (320, 200),      # a 64-k tail stage, ragged last tile
+    (64, 8),         # one tile
+    (14336, 264),    # long K over few tiles: stream-K shares tiles between CTAs
+]
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16])
+@pytest.mark.parametrize("K,N", SKINNY_SHAPES)
+def test_lut3_gemv_parity(torch, lbq, M, K, N):
+    idx, cb, ex = _inputs(70 + K + N, K, N)
+    img = _image(torch, lbq, idx, cb, ex)
+    X = workloads.activations_host(70 + M, M, K, "bf16")
+    for ydt in ("bf16", "f16"):
+        _check_gemm(torch, lbq, idx, cb, ex, img, X, y_dtype=ydt)
+    lbq.device_status()
+
+
+@pytest.mark.parametrize("M", [17, 130, 300])
+@pytest.mark.parametrize("K,N", [(1024, 512), (320, 264), (4096, 1032)])
+def test_lut3_gemm_parity(torch, lbq, M, K, N):
+    idx, cb, ex = _inputs(90 + K + N, K, N)
+    img = _image(torch, lbq, idx, cb, ex)
+    X = workloads.activations_host(90 + M, M, K, "bf16")
+    _check_gemm(torch, lbq, idx, cb, ex, img, X, y_dtype="bf16")
+    lbq.device_status()
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+def test_lut3_tcgen05_kernel_at_decode_batch(torch, lbq, M):
+    """The tcgen05 kernel itself at M <= 16 (normally routed to the GEMV)."""
+    K, N = 1024, 264
+    idx, cb, ex = _inputs(95, K, N)
+    img = _image(torch, lbq, idx, cb, ex)
+    X = workloads.activations_host(95 + M, M, K, "bf16")
+    lbq.lbq_debug_force_tc(1)
+    try:
+        _check_gemm(torch, lbq, idx, cb, ex, img, X)
+    finally:
+        lbq.lbq_debug_force_tc(0)
+
+
+def test_lut3_repeat_calls_identical(torch, lbq):
+    """Three calls on one workspace (shared tiles, so the counters must reset)."""
+    K, N, M = 14336, 264, 4
+    idx, cb, ex = _inputs(97, K, N)
+    img = _image(torch, lbq, idx, cb, ex)
+    X = workloads.activations_host(97, M, K, "bf16").cuda()
+    ws = lbq.workspace(2, M, K, N, 0, "lut3")
+    Ys = [lbq.lut3_gemm(X, img, N, ws=ws) for _ in range(3)]
+    torch.cuda.synchronize()
+    assert all(torch.equal(Ys[0], Y) for Y in Ys[1:])
+
+
+@pytest.mark.parametrize("M", [1, 16, 2048])
+def test_lut3_full_size_sampled(torch, lbq, M):
+    """K=4096, N=14336 (the 3-bit LUT workload): every row, sampled 8-channel groups."""
+    K, N = 4096, 14336
+    idx, cb, ex = workloads.lut3_host(5, K, N)
+    img = _image(torch, lbq, idx, cb, ex)
+    X = workloads.activations_host(5 + M, M, K, "bf16")
+    _check_gemm(torch, lbq, idx, cb, ex, img, X, groups=sample_columns(N // 8, 48, seed=M))
+
+
+def test_lut3_rejects_fp16_activations(torch, lbq):
+    K, N = 128, 16
+    idx, cb, ex = _inputs(99, K, N)
+    img = _image(torch, lbq, idx, cb, ex)
+    X = workloads.activations_host(99, 1, K, "f16").cuda()
+    with pytest.raises(lbq.LbqError):
+        lbq.lut3_gemm(X, img, N)
