@@ -112,16 +112,23 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- distributed
 
-def dist_setup(args):
+def dist_setup(backend=None):
+    """Rank / world from the torchrun environment; for world > 1 a process group
+    with a short timeout (NCCL on GPUs; gloo when no GPU is visible, which is how
+    the host logic is tested)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if backend is None:
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -134,10 +141,12 @@ def barrier(world):
 
 
 def max_over_ranks(world, value):
+    """The largest of the ranks' values (every rank gets it)."""
     import torch
     if world == 1:
         return value
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -165,7 +174,9 @@ class DecodeStep:
         self.x_all = torch.empty(x_len, dtype=torch.float16, device=device)
         self.y_all = torch.empty(y_len, dtype=torch.float16, device=device)
         xo = yo = 0
-        ws_bytes = 0
+        # one workspace per (K, N): a workspace is reused only by calls of one
+        # shape, whose tile counters sit at the same place every time
+        self.ws = {}
         for layer in range(layers):
             for p, (name, K, N) in enumerate(workloads.LLAMA3_8B_PROJ):
                 seed = workloads.c2_seed(layer, p)
@@ -177,19 +188,20 @@ class DecodeStep:
                 y = self.y_all[yo:yo + N].view(1, N)
                 xo += K
                 yo += N
-                self.projs.append((K, N, img, x, y))
+                if (K, N) not in self.ws:
+                    self.ws[(K, N)] = torch.zeros(max(lbq.lbq_workspace_size(0, 1, K, N, 32, 1), 256),
+                                                  dtype=torch.uint8, device=device)
+                self.projs.append((K, N, img, x, y, self.ws[(K, N)]))
                 self.bytes += int4_bytes(K, N, 32, "asym")
-                ws_bytes = max(ws_bytes, lbq.lbq_workspace_size(0, 1, K, N, 32, 1))
-        self.ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=device)
         self.lbq = lbq
         torch.cuda.synchronize()
 
     def launch_all(self):
         lbq = self.lbq
         stream = self.torch.cuda.current_stream().cuda_stream
-        for K, N, img, x, y in self.projs:
+        for K, N, img, x, y, ws in self.projs:
             lbq.lbq_gemv(x.data_ptr(), 0, 1, K, N, 32, 1, img.data_ptr(), y.data_ptr(), 0,
-                         self.ws.data_ptr(), self.ws.numel(), stream)
+                         ws.data_ptr(), ws.numel(), stream)
 
     def capture(self):
         torch = self.torch
@@ -224,19 +236,14 @@ def time_graph(torch, graph, steps, warmup, world):
     return e0.elapsed_time(e1)
 
 
-def rotating_gemv_ms(torch, lbq, images, X, N, group, mode, ws, reps=5):
-    """Per-launch time of one GEMV shape, cycling through distinct weight copies
-    (their total exceeds L2) inside one CUDA graph."""
-    Y = torch.empty((X.shape[0], N), dtype=X.dtype, device=X.device)
-    xdt = 0 if X.dtype == torch.float16 else 1
-    stream_of = lambda: torch.cuda.current_stream().cuda_stream
-    m = {"sym": 0, "asym": 1}[mode]
-
+def rotating_ms(torch, call, images, reps=5):
+    """Per-launch time of call(image, stream) cycling through distinct weight
+    copies (their total exceeds L2) inside one CUDA graph, CUDA events around
+    `reps` replays on the capturing stream's successor (the current stream)."""
     def run():
-        s = stream_of()
+        s = torch.cuda.current_stream().cuda_stream
         for img in images:
-            lbq.lbq_gemm(X.data_ptr(), xdt, X.shape[0], X.shape[1], N, group, m, img.data_ptr(), Y.data_ptr(), xdt,
-                         ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0, s)
+            call(img, s)
 
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
@@ -256,7 +263,37 @@ def rotating_gemv_ms(torch, lbq, images, X, N, group, mode, ws, reps=5):
         g.replay()
     e1.record()
     torch.cuda.synchronize()
+    del g
     return e0.elapsed_time(e1) / (reps * len(images))
+
+
+def rotating_gemv_ms(torch, lbq, images, X, N, group, mode, ws, reps=5):
+    """INT4 lbq_gemm over rotating weight copies (M <= 16 takes the GEMV kernels)."""
+    Y = torch.empty((X.shape[0], N), dtype=X.dtype, device=X.device)
+    xdt = 0 if X.dtype == torch.float16 else 1
+    m = {"sym": 0, "asym": 1}[mode]
+
+    def call(img, s):
+        lbq.lbq_gemm(X.data_ptr(), xdt, X.shape[0], X.shape[1], N, group, m, img.data_ptr(), Y.data_ptr(), xdt,
+                     ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0, s)
+
+    return rotating_ms(torch, call, images, reps)
+
+
+def rotating_lut3_ms(torch, lbq, images, X, N, ws, reps=5):
+    Y = torch.empty((X.shape[0], N), dtype=X.dtype, device=X.device)
+
+    def call(img, s):
+        lbq.lbq_lut3_gemm(X.data_ptr(), 1, X.shape[0], X.shape[1], N, img.data_ptr(), Y.data_ptr(), 1,
+                          ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0, s)
+
+    return rotating_ms(torch, call, images, reps)
+
+
+def weight_copies(img0, l2_bytes, minimum=3):
+    """img0 plus clones so that the copies together exceed 3x L2."""
+    copies = max(minimum, (3 * l2_bytes) // img0.numel() + 1)
+    return [img0] + [img0.clone() for _ in range(copies - 1)]
 
 
 def secondary_measurements(torch, lbq, workloads, device, peaks, quick):
@@ -304,6 +341,38 @@ def secondary_measurements(torch, lbq, workloads, device, peaks, quick):
                                                                 "frac_hbm": b / ms / 1e6 / hbm}
         del images, img0
     del W
+    # c4: prefill GEMM K=4096 N=14336 asym g128, bf16 X and Y, tcgen05
+    tc_peak, tc_sus = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
+    K, N = 4096, 14336
+    W = workloads.weights_device(4, K, N, device)
+    images = weight_copies(lbq.pack(W, 128, "asym"), l2_bytes)
+    del W
+    for M in (512, 2048, 8192):
+        X = workloads.activations_device(4, M, K, "bf16", device)
+        ms = rotating_gemv_ms(torch, lbq, images, X, N, 128, "asym", None, reps=3)
+        tf = 2.0 * M * K * N / ms / 1e9
+        out[f"c4_gemm_m{M}"] = {"us": ms * 1e3, "TFLOPs": tf, "frac_bf16_peak": tf / tc_peak,
+                                "frac_bf16_sustained": tf / tc_sus, "weight_copies": len(images)}
+        del X
+    del images
+    # c5: LUT3 K=4096 N=14336, M=1 (GB/s of the format's bytes) and M=2048 (TFLOP/s)
+    idx, cb, ex = workloads.lut3_device(5, K, N, device)
+    images = weight_copies(lbq.pack_lut3(idx, cb, ex), l2_bytes)
+    del idx, cb, ex
+    b = lut3_bytes(K, N)
+    for M in (1, 2048):
+        X = workloads.activations_device(5, M, K, "bf16", device)
+        ws = lbq.workspace(2, M, K, N, 0, "lut3")
+        ms = rotating_lut3_ms(torch, lbq, images, X, N, ws, reps=3)
+        if M == 1:
+            out["c5_lut3_m1"] = {"us": ms * 1e3, "GBps": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm,
+                                 "image_bytes_read": images[0].numel(), "weight_copies": len(images)}
+        else:
+            tf = 2.0 * M * K * N / ms / 1e9
+            out[f"c5_lut3_m{M}"] = {"us": ms * 1e3, "TFLOPs": tf, "frac_bf16_peak": tf / tc_peak,
+                                    "frac_bf16_sustained": tf / tc_sus}
+        del X
+    del images
     return out
 
 
@@ -428,22 +497,28 @@ def run_profile_case(name):
 
 # ----------------------------------------------------------------------------- main
 
-def traffic_from_profiles(kernel):
-    """DRAM bytes per launch recorded by the last ncu capture of `kernel`, if the
-    kernel source has not changed since (hash recorded beside the figure)."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(path):
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) from ncu captures
+# summarised under profiles/, with a hash of the kernel sources at capture time:
+# name -> (bytes, {source file: sha256[:16]}, summary file).
+NCU_TRAFFIC = {}
+
+
+def source_hash(name):
+    import hashlib
+    with open(os.path.join(ROOT, "bit_weight_only_pack_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_from_profiles(name):
+    """The recorded DRAM bytes for `name`, or None when there is no record or a
+    kernel source changed since the capture."""
+    rec = NCU_TRAFFIC.get(name)
+    if rec is None:
         return None
+    nbytes, sources, _summary = rec
     try:
-        import hashlib
-        with open(path) as f:
-            rec = json.load(f).get(kernel)
-        if not rec:
-            return None
-        src = os.path.join(ROOT, "bit_weight_only_pack_b200", "csrc", rec["source"])
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        return rec["dram_bytes_per_launch_full"] if h == rec["source_sha"] else None
-    except Exception:
+        return nbytes if all(source_hash(f) == h for f, h in sources.items()) else None
+    except OSError:
         return None
 
 
@@ -473,7 +548,7 @@ def main():
     import bit_weight_only_pack_b200 as lbq
     import workloads
 
-    world, rank, local = dist_setup(args)
+    world, rank, local = dist_setup()
     device = torch.device("cuda", local)
     peaks = load_peaks()
 
@@ -495,14 +570,17 @@ def main():
     ms_per_step = elapsed_ms / args.steps
     value = world * step.bytes / (ms_per_step / 1e3) / 1e9
 
-    # end to end: pinned host X in, pinned host Y out, every step
+    # end to end through the public C-ABI call: every step copies its
+    # activations in from pinned host memory, makes the 224 lbq_gemv calls
+    # (no graph) and copies the outputs back to pinned host memory
     x_host = torch.empty_like(step.x_all, device="cpu").pin_memory()
     x_host.copy_(step.x_all.cpu())
     y_host = torch.empty_like(step.y_all, device="cpu").pin_memory()
-    x_stage = torch.empty_like(step.x_all)
+    lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 0 if args.no_pdl else 1)
+    launches_before = lbq.lbq_launch_count()
     for _ in range(args.warmup):
         step.x_all.copy_(x_host, non_blocking=True)
-        graph.replay()
+        step.launch_all()
         y_host.copy_(step.y_all, non_blocking=True)
     torch.cuda.synchronize()
     barrier(world)
@@ -510,12 +588,14 @@ def main():
     e0.record()
     for _ in range(args.steps):
         step.x_all.copy_(x_host, non_blocking=True)
-        graph.replay()
+        step.launch_all()
         y_host.copy_(step.y_all, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
+    lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 0)
+    e2e_launches = lbq.lbq_launch_count() - launches_before
     e2e_ms = max_over_ranks(world, e0.elapsed_time(e1)) / args.steps
-    del x_stage
+    lbq.device_status()
 
     secondary = None
     if not args.no_secondary:
@@ -528,11 +608,13 @@ def main():
     hbm = peaks["hbm_gbs"]
     per_gpu = step.bytes / (ms_per_step / 1e3) / 1e9
     launches = step.launches_per_step
-    traffic = traffic_from_profiles("gemv_m1_kernel")
+    # DRAM bytes of one step's launches from an ncu capture (see profiles/), per launch on average
+    traffic_step = traffic_from_profiles("decode_step_per_layer")
+    traffic = traffic_step * args.layers / launches if traffic_step is not None else None
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16 x int4 -> f32 accumulate", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
         "config": {"workload": "c2: Llama-3-8B-shaped decode step at M=1, 7 projections x %d layers, asymmetric "
                                "INT4 group 32 (fp16 scale + int8 zp), fp16 X, fp16 Y" % args.layers,
                    "weight_bytes_per_step": step.bytes, "gemvs_per_step": len(step.projs),
@@ -543,15 +625,20 @@ def main():
                    "parallelism": "replicas" if world > 1 else "1 GPU"},
         "frac_hbm": per_gpu / hbm,
         "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": hbm, "unit": "GB/s", "frac": per_gpu / hbm,
-                     "peak_source": peaks["source"],
-                     "traffic": (traffic * launches if traffic is not None else None),
-                     "traffic_note": "DRAM bytes per step from ncu (sum over the step's launches) when the "
-                                     "kernel source is unchanged since the capture, else null",
-                     "kernel": "gemv_m1_kernel", "algorithmic_bytes_per_step": step.bytes},
+                     "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peaks["source"],
+                     "traffic": traffic,
+                     "kernel": "gemv_m1_kernel (every launch of the step)",
+                     "per_launch": "algorithmic bytes per launch averaged over the step's %d launches (%.0f B) / "
+                                   "average launch time (step time / launches); traffic = ncu DRAM read+write "
+                                   "bytes per launch, averaged the same way, null if the kernel source changed "
+                                   "since the capture" % (launches, step.bytes / max(launches, 1)),
+                     "algorithmic_bytes_per_step": step.bytes},
         "clocks": clocks,
         "e2e": {"value": world * step.bytes / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": step.x_all.numel() * 2, "d2h_bytes_per_step": step.y_all.numel() * 2,
-                "ms_per_step": e2e_ms},
+                "ms_per_step": e2e_ms, "kernel_launches": e2e_launches,
+                "how": "per step: pinned host X -> device, 224 lbq_gemv C-ABI calls (no graph), device Y -> "
+                       "pinned host; CUDA events on the launching stream"},
         "gpu_launches": launches * args.steps,
         "cpu_baseline": cpu,
         "secondary": secondary,
