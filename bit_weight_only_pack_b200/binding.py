@@ -55,6 +55,7 @@ _SIGS = {
     "lbq_dequant": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp], _c_int),
     "lbq_device_status": ([_vp], _c_int),
     "lbq_set_option": ([_c_int, _c_int], _c_int),
+    "lbq_gemv_noalloc": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp], _c_int),
     "lbq_debug_force_splits": ([_c_int], None),
     "lbq_debug_force_skinny": ([_c_int], None),
     "lbq_debug_force_tc": ([_c_int], None),
@@ -133,6 +134,10 @@ def lbq_dequant(image, K, N, group, mode, W_out, stream):
 
 def lbq_device_status(stream):
     _check(_lib.lbq_device_status(stream))
+
+
+def lbq_gemv_noalloc(X, x_dtype, M, K, N, group, mode, image, Y, y_dtype, stream):
+    _check(_lib.lbq_gemv_noalloc(X, x_dtype, M, K, N, group, mode, image, Y, y_dtype, stream))
 
 
 LBQ_OPT_PDL = 1
@@ -284,6 +289,16 @@ def dequant(image, K, N, group, mode):
     W = torch.empty((K, N), dtype=torch.float32, device=image.device)
     lbq_dequant(image.data_ptr(), K, N, group, _mode(mode), W.data_ptr(), _stream())
     return W
+
+
+def gemv_noalloc(X, image, N, group, mode, y_dtype=None, Y=None):
+    """lbq_gemv with the library's fixed scratch instead of a workspace."""
+    _need_cuda(X, image, Y)
+    M, K = X.shape
+    Y = _out(X, N, y_dtype) if Y is None else Y
+    lbq_gemv_noalloc(X.data_ptr(), _dt(X), M, K, N, group, _mode(mode), image.data_ptr(), Y.data_ptr(), _dt(Y),
+                     _stream())
+    return Y
 
 
 def device_status():

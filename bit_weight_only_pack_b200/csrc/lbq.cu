@@ -477,6 +477,47 @@ static lbq_status check_compute_args(const void* X, int x_dtype, int M, const vo
   return LBQ_OK;
 }
 
+// ----------------------------------------------------------------------------
+// Fixed scratch for lbq_gemv_noalloc
+// ----------------------------------------------------------------------------
+//
+// Some callers cannot hand the library a workspace: a C program with no device
+// allocator of its own, or a serving process whose device memory is carved up
+// once at start-up and must not grow (or fragment) while requests are served.
+// For them the split-K partial sums and tile counters of the GEMV live in this
+// module-level array, which the CUDA runtime places when it loads the module;
+// no call ever allocates or frees device memory.
+
+constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;  // 8 MiB per device
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the first lookup may load the module, so it must not happen
+// while the stream is being captured).
+static uint8_t* noalloc_scratch(lbq_status* st) {
+  static std::mutex mu;
+  static uint8_t* ptr[kNoAllocMaxDevices] = {};
+  int dev = 0;
+  if ((*st = cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) != LBQ_OK) return nullptr;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) {
+    *st = fail(LBQ_ERR_UNSUPPORTED, "device %d is beyond the %d devices the fixed scratch supports", dev,
+               kNoAllocMaxDevices);
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if ((*st = cuda_check(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress of the fixed scratch")) !=
+        LBQ_OK)
+      return nullptr;
+    ptr[dev] = static_cast<uint8_t*>(p);
+  }
+  *st = LBQ_OK;
+  return ptr[dev];
+}
+
 }  // namespace lbq
 
 using namespace lbq;
@@ -694,6 +735,48 @@ lbq_status lbq_device_status(void* stream) {
   if (v == 0) return LBQ_OK;
   if ((st = cuda_check(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)), "clearing the device flag")) != LBQ_OK) return st;
   return fail(LBQ_ERR_DEVICE, "a kernel reported device error flags 0x%x", v);
+}
+
+lbq_status lbq_gemv_noalloc(const void* X, int x_dtype, int M, int K, int N, int group, int mode, const void* image,
+                            void* Y, int y_dtype, void* stream) {
+  lbq_status st = check_int4_shape(K, N, group, mode);
+  if (st != LBQ_OK) return st;
+  if ((st = check_compute_args(X, x_dtype, M, image, Y, y_dtype)) != LBQ_OK) return st;
+  if (M > 16) return fail(LBQ_ERR_UNSUPPORTED, "lbq_gemv_noalloc takes M <= 16 (M=%d)", M);
+  // The scratch the dispatch of lbq_gemv needs for this call, and where in it
+  // the tile counters sit (the same plans lbq_gemv makes).
+  const bool asym = mode == LBQ_MODE_ASYM;
+  size_t need = 0, cnt_off = 0, cnt_bytes = 0;
+  if (M == 1 && !g_force_skinny) {
+    const M1Plan p = plan_m1(K, N, group, asym, g_force_splits);
+    need = p.block == 0 ? 0 : m1_workspace_bytes(p, N);
+    if (need) {
+      cnt_off = align_up((size_t)p.splits * N * sizeof(float), 256);
+      cnt_bytes = (size_t)p.row_tiles * sizeof(unsigned);
+    }
+  } else {
+    const SkPlan p = plan_skinny(K, N, M, group, asym, x_dtype == LBQ_DTYPE_BF16);
+    need = skinny_workspace_bytes(p, M);
+    cnt_off = align_up((size_t)p.row_tiles * p.max_slots * M * kSkRows * sizeof(float), 256);
+    cnt_bytes = (size_t)p.row_tiles * sizeof(unsigned);
+  }
+  if (need > kNoAllocScratchBytes)
+    return fail(LBQ_ERR_UNSUPPORTED,
+                "lbq_gemv_noalloc: M=%d K=%d N=%d needs %zu bytes of scratch, more than its fixed %zu; use lbq_gemv "
+                "with a workspace",
+                M, K, N, need, kNoAllocScratchBytes);
+  uint8_t* scratch = nullptr;
+  if (need) {
+    scratch = noalloc_scratch(&st);
+    if (!scratch) return st;
+    // The counters must be zero when the kernel starts; the previous call may
+    // have left partial sums where this shape keeps its counters.
+    if ((st = cuda_check(cudaMemsetAsync(scratch + cnt_off, 0, cnt_bytes, static_cast<cudaStream_t>(stream)),
+                         "clearing the fixed scratch's tile counters")) != LBQ_OK)
+      return st;
+  }
+  return lbq_gemv(X, x_dtype, M, K, N, group, mode, image, Y, y_dtype, scratch, need ? kNoAllocScratchBytes : 0,
+                  stream);
 }
 
 }  // extern "C"

@@ -110,9 +110,11 @@ lbq_status lbq_pack_lut3(const uint8_t* idx, const uint8_t* codebooks, const uin
  * the split-K partial sums and tile counters of the dispatch the library
  * would pick. op: 0 = lbq_gemv, 1 = lbq_gemm, 2 = lbq_lut3_gemm.
  * Writes *bytes (host); 0 means the call needs no workspace (ws may be null).
- * A workspace must be zero-filled before its first use; every call leaves it
- * zero-filled again, so one buffer can be reused by consecutive calls on one
- * stream (not by calls running concurrently).
+ * The workspace's tile counters must be zero when a call starts: zero-fill a
+ * new workspace before its first use; every call that completes returns its
+ * counters to zero (its partial sums are left behind), so one buffer can be
+ * reused by consecutive calls of the same shape on one stream (not by calls
+ * running concurrently). Reusing it for another shape needs a new zero fill.
  */
 lbq_status lbq_workspace_size(int op, int M, int K, int N, int group, int mode, size_t* bytes);
 
@@ -193,6 +195,29 @@ lbq_status lbq_device_status(void* stream);
  */
 typedef enum { LBQ_OPT_PDL = 1 } lbq_option;
 lbq_status lbq_set_option(int option, int value);
+
+/*
+ * lbq_gemv without a caller-provided workspace: same arguments (minus ws,
+ * ws_bytes), same kernels, same result. The pages describe no such call; it
+ * serves callers that cannot give the library device memory (a plain C
+ * program without a device allocator, or a process whose device memory is
+ * partitioned once at start-up). Nothing is allocated or freed, ever.
+ *   Scratch: one fixed module-level device array of 8 MiB per device, placed
+ *   by the CUDA runtime when it loads the library's module. A call whose
+ *   dispatch needs more (roughly (296 + 2 * ceil(N/128)) * M * 512 bytes for
+ *   2 <= M <= 16) fails with LBQ_ERR_UNSUPPORTED and launches nothing; use
+ *   lbq_gemv with a workspace for it.
+ *   Zero state: nothing has to be zero beforehand; each call clears the tile
+ *   counters it will use (one memset on `stream`) before its kernel.
+ *   First call: looks up the array's device address once per device (the
+ *   lookup may load the module); make it outside stream capture.
+ *   Concurrency: all calls on one device share the one array, so two calls
+ *   whose work can overlap (different streams, or host threads racing on one
+ *   stream) corrupt each other's partial sums. Serialise them.
+ * Asynchronous on `stream`.
+ */
+lbq_status lbq_gemv_noalloc(const void* X, int x_dtype, int M, int K, int N, int group, int mode,
+                            const void* image, void* Y, int y_dtype, void* stream);
 
 /* Number of kernel launches the library has enqueued so far in this process. */
 uint64_t lbq_launch_count(void);
