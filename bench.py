@@ -296,6 +296,10 @@ def weight_copies(img0, l2_bytes, minimum=3):
     return [img0] + [img0.clone() for _ in range(copies - 1)]
 
 
+# the GEMV kernels the library does not pick by default, timed beside the default
+GEMV_ALT_PATHS = (("cudacore_m1_kernel", 1), ("warp_mma_kernel", 2), ("tcgen05_kernel", 3))
+
+
 def secondary_measurements(torch, lbq, workloads, device, peaks, quick):
     out = {}
     hbm = peaks["hbm_gbs"]
@@ -312,10 +316,11 @@ def secondary_measurements(torch, lbq, workloads, device, peaks, quick):
     b = int4_bytes(K, N, 32, "sym")
     out["c1_gemv_4096x4096_sym_g32_m1"] = {"us": ms * 1e3, "GBps": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm,
                                            "weight_copies": copies}
-    lbq.lbq_debug_force_skinny(1)
-    ms = rotating_gemv_ms(torch, lbq, images, X, N, 32, "sym", lbq.workspace(0, 1, K, N, 32, "sym"))
-    lbq.lbq_debug_force_skinny(0)
-    out["c1_gemv_m1_on_tensor_core_kernel"] = {"us": ms * 1e3, "GBps": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm}
+    for name, path in GEMV_ALT_PATHS:
+        lbq.lbq_debug_gemv_path(path)
+        ms = rotating_gemv_ms(torch, lbq, images, X, N, 32, "sym", lbq.workspace(0, 1, K, N, 32, "sym"))
+        lbq.lbq_debug_gemv_path(0)
+        out[f"c1_gemv_m1_{name}"] = {"us": ms * 1e3, "GBps": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm}
     del images, img0
     if quick:
         return out
@@ -332,13 +337,16 @@ def secondary_measurements(torch, lbq, workloads, device, peaks, quick):
             ws = lbq.workspace(0, M, K, N, group, "sym")
             ms = rotating_gemv_ms(torch, lbq, images, X, N, group, "sym", ws, reps=3)
             out[f"c3_g{group}_m{M}"] = {"us": ms * 1e3, "GBps": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm}
-            if M == 1:
-                lbq.lbq_debug_force_skinny(1)
-                ws = lbq.workspace(0, M, K, N, group, "sym")
-                ms = rotating_gemv_ms(torch, lbq, images, X, N, group, "sym", ws, reps=3)
-                lbq.lbq_debug_force_skinny(0)
-                out[f"c3_g{group}_m1_on_tensor_core_kernel"] = {"us": ms * 1e3, "GBps": b / ms / 1e6,
-                                                                "frac_hbm": b / ms / 1e6 / hbm}
+            if M in (1, 16):
+                for name, path in GEMV_ALT_PATHS:
+                    if path == 1 and M != 1 or path == 2 and M != 1:
+                        continue
+                    lbq.lbq_debug_gemv_path(path)
+                    ws = lbq.workspace(0, M, K, N, group, "sym")
+                    ms = rotating_gemv_ms(torch, lbq, images, X, N, group, "sym", ws, reps=3)
+                    lbq.lbq_debug_gemv_path(0)
+                    out[f"c3_g{group}_m{M}_{name}"] = {"us": ms * 1e3, "GBps": b / ms / 1e6,
+                                                       "frac_hbm": b / ms / 1e6 / hbm}
         del images, img0
     del W
     # c4: prefill GEMM K=4096 N=14336 asym g128, bf16 X and Y, tcgen05

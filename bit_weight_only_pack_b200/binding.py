@@ -59,6 +59,7 @@ _SIGS = {
     "lbq_debug_force_splits": ([_c_int], None),
     "lbq_debug_force_skinny": ([_c_int], None),
     "lbq_debug_force_tc": ([_c_int], None),
+    "lbq_debug_gemv_path": ([_c_int], None),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -153,6 +154,11 @@ def lbq_debug_force_splits(splits):
 
 def lbq_debug_force_tc(on):
     _lib.lbq_debug_force_tc(1 if on else 0)
+
+
+def lbq_debug_gemv_path(path):
+    """Test hook: GEMV kernel for M <= 16 (0 auto, 1 CUDA-core M=1, 2 warp MMA, 3 tcgen05)."""
+    _lib.lbq_debug_gemv_path(path)
 
 
 def lbq_debug_force_skinny(on):

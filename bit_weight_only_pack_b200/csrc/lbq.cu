@@ -24,6 +24,7 @@
 #include "skinny.cuh"
 #include "lut3_gemv.cuh"
 #include "gemm_tc.cuh"
+#include "tc_gemv.cuh"
 
 namespace lbq {
 
@@ -146,6 +147,10 @@ struct M1Plan {
 static int g_force_splits = 0;  // test hook: force a split count (0 = shape-based choice)
 static int g_pdl = 0;           // launch GEMVs with programmatic dependent launch
 static int g_force_skinny = 0;  // test hook: route M = 1 to the tensor-core skinny kernel
+// test hook: GEMV kernel for M <= 16. 0 = the library's choice, 1 = the CUDA-core
+// M = 1 kernel, 2 = the warp-MMA skinny kernel, 3 = the tcgen05 kernel.
+static int g_gemv_path = 0;
+enum { kPathAuto = 0, kPathM1 = 1, kPathMma = 2, kPathTc = 3 };
 
 constexpr int kM1RingBudget = 100 * 1024;
 constexpr int kM1MaxChunksPerSplit = 128;  // K-slices of at most 4096 k keep a ring slot near 20 KB
@@ -363,6 +368,114 @@ static lbq_status run_skinny(const void* X, bool xbf16, int M, const void* image
 }
 
 // ----------------------------------------------------------------------------
+// 1 <= M <= 16: tcgen05 GEMV (weights as the A operand in tensor memory)
+// ----------------------------------------------------------------------------
+
+typedef void (*TgKernel)(CUtensorMap, CUtensorMap, TcGemvArgs);
+
+template <bool B, bool A, int MC>
+static TgKernel tg_for_gc(int gc) {
+  if (gc == 1) return tc_gemv_kernel<B, A, MC, 1>;
+  if (gc == 2) return tc_gemv_kernel<B, A, MC, 2>;
+  return tc_gemv_kernel<B, A, MC, 4>;
+}
+
+template <bool B, bool A>
+static TgKernel tg_for_mc(int M, int gc) {
+  if (M == 1) return tg_for_gc<B, A, 1>(gc);
+  if (M <= 8) return tg_for_gc<B, A, 8>(gc);
+  return tg_for_gc<B, A, 16>(gc);
+}
+
+static TgKernel tg_kernel(bool xbf16, bool asym, int M, int gc) {
+  if (xbf16) return asym ? tg_for_mc<true, true>(M, gc) : tg_for_mc<true, false>(M, gc);
+  return asym ? tg_for_mc<false, true>(M, gc) : tg_for_mc<false, false>(M, gc);
+}
+
+// One CTA per SM (the kernel holds all 512 tensor-memory columns).
+static SkPlan plan_tcgemv(int K, int N) {
+  SkPlan p{};
+  p.row_tiles = (N + 127) / 128;
+  p.stages_per_tile = (K + 255) / 256;
+  p.units = (long long)p.row_tiles * p.stages_per_tile;
+  p.smem = kTgSmem;
+  p.grid = (int)std::min<long long>(p.units, (long long)num_sms());
+  const long long per = std::max<long long>(1, p.units / p.grid);
+  p.max_slots = (int)((p.stages_per_tile + per - 1) / per + 1);
+  return p;
+}
+
+static lbq_status run_tcgemv(const void* X, bool xbf16, int M, const void* image, const Layout& L, void* Y,
+                             bool ybf16, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const bool asym = L.mode == LBQ_MODE_ASYM;
+  const SkPlan p = plan_tcgemv(L.K, L.N);
+  const size_t need = skinny_workspace_bytes(p, M);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(LBQ_ERR_INVALID_ARG, "workspace of %zu bytes is too small (need %zu)", ws_bytes, need);
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  CUtensorMap tw, tx;
+  const bool ok = make_tmap_2d(&tw, img + L.off0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.K / 2, (uint64_t)L.N,
+                               (uint64_t)L.K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+                  make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)L.K, (uint64_t)M,
+                               (uint64_t)L.K * 2, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the tcgen05 GEMV");
+  TcGemvArgs a{};
+  a.Y = Y;
+  a.partials = static_cast<float*>(ws);
+  a.counters = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) +
+                                           align_up((size_t)p.row_tiles * p.max_slots * M * kSkRows * sizeof(float), 256));
+  a.s_region = img + L.off1;
+  a.z_region = asym ? img + L.off2 : nullptr;
+  a.K = L.K; a.N = L.N; a.M = M; a.G = L.K / L.group;
+  a.stages_per_tile = p.stages_per_tile; a.row_tiles = p.row_tiles; a.max_slots = p.max_slots; a.units = p.units;
+  a.y_bf16 = ybf16 ? 1 : 0;
+  const TgKernel fn = tg_kernel(xbf16, asym, M, L.group / 32);
+  occupancy_for((const void*)fn, kTgThreads, kTgSmem);
+  void* args[] = {&tw, &tx, &a};
+  return launch_kernel_ex((const void*)fn, dim3(p.grid), dim3(kTgThreads), kTgSmem, st, g_pdl != 0, args,
+                          "tcgen05 GEMV launch");
+}
+
+// The kernel lbq_gemv runs for M <= 16. Measured on B200: at M = 1 the
+// CUDA-core kernel is faster up to ~10^8 weights (the warp-MMA kernel spends an
+// MMA, 7/8 wasted, per 256 weights, and legacy MMA throughput is the limit);
+// from M = 2 the warp-MMA kernel wins. The tcgen05 kernel is slower at every
+// batch size here (a 128 x 16 x N MMA costs the same ~185 cycles for N = 16
+// as for N = 256), so it is never the default.
+static int gemv_path(int M, long long weights) {
+  if (g_gemv_path == kPathM1 && M == 1) return kPathM1;
+  if (g_gemv_path == kPathMma || g_gemv_path == kPathTc) return g_gemv_path;
+  if (g_force_skinny) return kPathMma;
+  if (M == 1 && (g_force_splits || weights < (1LL << 27))) return kPathM1;
+  return kPathMma;
+}
+
+// Scratch of that kernel for one call: total bytes and where the tile counters
+// sit (they must be zero when the kernel starts).
+struct GemvScratch {
+  size_t need, cnt_off, cnt_bytes;
+};
+
+static GemvScratch gemv_scratch(int M, int K, int N, int group, bool asym, bool xbf16) {
+  GemvScratch g{0, 0, 0};
+  const int path = gemv_path(M, (long long)K * N);
+  if (path == kPathM1) {
+    const M1Plan p = plan_m1(K, N, group, asym, g_force_splits);
+    g.need = p.block == 0 ? 0 : m1_workspace_bytes(p, N);
+    if (g.need) {
+      g.cnt_off = align_up((size_t)p.splits * N * sizeof(float), 256);
+      g.cnt_bytes = (size_t)p.row_tiles * sizeof(unsigned);
+    }
+    return g;
+  }
+  const SkPlan p = path == kPathMma ? plan_skinny(K, N, M, group, asym, xbf16) : plan_tcgemv(K, N);
+  g.need = skinny_workspace_bytes(p, M);
+  g.cnt_off = align_up((size_t)p.row_tiles * p.max_slots * M * kSkRows * sizeof(float), 256);
+  g.cnt_bytes = (size_t)p.row_tiles * sizeof(unsigned);
+  return g;
+}
+
+// ----------------------------------------------------------------------------
 // M > 16: tcgen05 prefill GEMM
 // ----------------------------------------------------------------------------
 
@@ -541,6 +654,10 @@ void lbq_debug_force_tc(int on) { g_force_tc = on ? 1 : 0; }
 // Test hook (not in the public header): route M = 1 through the skinny kernel.
 void lbq_debug_force_skinny(int on) { g_force_skinny = on ? 1 : 0; }
 
+// Test hook (not in the public header): pick the GEMV kernel for M <= 16
+// (0 = the library's choice, 1 = CUDA-core M = 1, 2 = warp MMA, 3 = tcgen05).
+void lbq_debug_gemv_path(int path) { g_gemv_path = (path >= 0 && path <= 3) ? path : 0; }
+
 lbq_status lbq_set_option(int option, int value) {
   if (option == LBQ_OPT_PDL) {
     g_pdl = value ? 1 : 0;
@@ -610,15 +727,11 @@ lbq_status lbq_workspace_size(int op, int M, int K, int N, int group, int mode, 
     if (st != LBQ_OK) return st;
     if (M <= 0) return fail(LBQ_ERR_INVALID_ARG, "M must be positive");
     if (op == 1 && (M > 16 || g_force_tc)) return LBQ_OK;  // the prefill GEMM needs no workspace
-    if (M == 1 && !g_force_skinny) {
-      const M1Plan p = plan_m1(K, N, group, mode == LBQ_MODE_ASYM, g_force_splits);
-      *bytes = m1_workspace_bytes(p, N);
-    } else if (M <= 16) {
-      // the plan depends on the activation dtype only through the kernel's
+    if (M <= 16) {
+      // the plan may depend on the activation dtype through a kernel's
       // occupancy; take the larger of the two
-      const SkPlan p0 = plan_skinny(K, N, M, group, mode == LBQ_MODE_ASYM, false);
-      const SkPlan p1 = plan_skinny(K, N, M, group, mode == LBQ_MODE_ASYM, true);
-      *bytes = std::max(skinny_workspace_bytes(p0, M), skinny_workspace_bytes(p1, M));
+      const bool asym = mode == LBQ_MODE_ASYM;
+      *bytes = std::max(gemv_scratch(M, K, N, group, asym, false).need, gemv_scratch(M, K, N, group, asym, true).need);
     }
     return LBQ_OK;
   }
@@ -640,10 +753,13 @@ lbq_status lbq_gemv(const void* X, int x_dtype, int M, int K, int N, int group, 
   if (M > 16) return fail(LBQ_ERR_UNSUPPORTED, "lbq_gemv takes M <= 16 (M=%d); use lbq_gemm", M);
   const Layout L = make_layout(K, N, group, mode);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (M == 1 && !g_force_skinny)
+  const int path = gemv_path(M, (long long)K * N);
+  if (path == kPathM1)
     return run_m1(static_cast<const uint16_t*>(X), x_dtype == LBQ_DTYPE_BF16, image, L, Y, y_dtype == LBQ_DTYPE_BF16,
                   ws, ws_bytes, s);
-  return run_skinny(X, x_dtype == LBQ_DTYPE_BF16, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, ws, ws_bytes, s);
+  if (path == kPathMma)
+    return run_skinny(X, x_dtype == LBQ_DTYPE_BF16, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, ws, ws_bytes, s);
+  return run_tcgemv(X, x_dtype == LBQ_DTYPE_BF16, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, ws, ws_bytes, s);
 }
 
 lbq_status lbq_gemm(const void* X, int x_dtype, int M, int K, int N, int group, int mode, const void* image, void* Y,
@@ -745,21 +861,8 @@ lbq_status lbq_gemv_noalloc(const void* X, int x_dtype, int M, int K, int N, int
   if (M > 16) return fail(LBQ_ERR_UNSUPPORTED, "lbq_gemv_noalloc takes M <= 16 (M=%d)", M);
   // The scratch the dispatch of lbq_gemv needs for this call, and where in it
   // the tile counters sit (the same plans lbq_gemv makes).
-  const bool asym = mode == LBQ_MODE_ASYM;
-  size_t need = 0, cnt_off = 0, cnt_bytes = 0;
-  if (M == 1 && !g_force_skinny) {
-    const M1Plan p = plan_m1(K, N, group, asym, g_force_splits);
-    need = p.block == 0 ? 0 : m1_workspace_bytes(p, N);
-    if (need) {
-      cnt_off = align_up((size_t)p.splits * N * sizeof(float), 256);
-      cnt_bytes = (size_t)p.row_tiles * sizeof(unsigned);
-    }
-  } else {
-    const SkPlan p = plan_skinny(K, N, M, group, asym, x_dtype == LBQ_DTYPE_BF16);
-    need = skinny_workspace_bytes(p, M);
-    cnt_off = align_up((size_t)p.row_tiles * p.max_slots * M * kSkRows * sizeof(float), 256);
-    cnt_bytes = (size_t)p.row_tiles * sizeof(unsigned);
-  }
+  const GemvScratch g = gemv_scratch(M, K, N, group, mode == LBQ_MODE_ASYM, x_dtype == LBQ_DTYPE_BF16);
+  const size_t need = g.need, cnt_off = g.cnt_off, cnt_bytes = g.cnt_bytes;
   if (need > kNoAllocScratchBytes)
     return fail(LBQ_ERR_UNSUPPORTED,
                 "lbq_gemv_noalloc: M=%d K=%d N=%d needs %zu bytes of scratch, more than its fixed %zu; use lbq_gemv "

@@ -42,8 +42,21 @@ __host__ __device__ constexpr int lut3_hi_pos(int i) {
 // position of index i's two low bits in the chunk's A (i < 16) or B word
 __host__ __device__ constexpr int lut3_lo_pos(int i) { return 4 * (i & 7) + (((i >> 3) & 1) ? 2 : 0); }
 
-// One thread per (channel n, 64-k tile kt).
 __device__ inline float e4m3_to_float(uint32_t b);
+
+// BF16 bit pattern of e4m3(b) * 2^(e - 127). The product has at most four
+// significant bits, so while it is a normal FP32 number its FP32 pattern ends in
+// 16 zero bits and its top half is the exact BF16 pattern; outside that range
+// (|value| below 2^-126 or NaN) the value is rounded to nearest even.
+__device__ inline uint32_t lut3_table_entry(uint32_t b, uint32_t e) {
+  if (e == 255u) return 0x7FC0u;
+  const uint32_t f = __float_as_uint(ldexpf(e4m3_to_float(b), (int)e - 127));
+  if ((f & 0xFFFFu) == 0u) return f >> 16;
+  const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(f));
+  return (uint32_t)__bfloat16_as_ushort(h);
+}
+
+// One thread per (channel n, 64-k tile kt).
 
 __global__ void __launch_bounds__(256) pack_lut3_kernel(const uint8_t* __restrict__ idx, const uint8_t* __restrict__ cb,
                                                         const uint8_t* __restrict__ ex, int K, int N,
@@ -67,16 +80,15 @@ __global__ void __launch_bounds__(256) pack_lut3_kernel(const uint8_t* __restric
   if ((n & 7) == 0) {
     const int grp = n >> 3;
     const uint8_t e = ex[(size_t)kt * (N / 8) + grp];
-    uint8_t* tt = t_region + ((size_t)kt * (N / 8) + grp) * 16;
+    uint32_t lo[2] = {0u, 0u}, hi[2] = {0u, 0u};
     for (int j = 0; j < 8; ++j) {
       const uint8_t b = cb[((size_t)kt * (N / 8) + grp) * 8 + j];
       c_region[(size_t)grp * lut3_c_stride(K) + kt * 8 + j] = b;
-      const float v = e == 255 ? __int_as_float(0x7FC00000) : ldexpf(e4m3_to_float(b), (int)e - 127);
-      const __nv_bfloat16 h = __float2bfloat16_rn(v);
-      const uint16_t bits = *reinterpret_cast<const uint16_t*>(&h);
-      tt[j] = (uint8_t)(bits & 0xFF);
-      tt[8 + j] = (uint8_t)(bits >> 8);
+      const uint32_t bits = lut3_table_entry(b, e);
+      lo[j >> 2] |= (bits & 0xFFu) << (8 * (j & 3));
+      hi[j >> 2] |= (bits >> 8) << (8 * (j & 3));
     }
+    *reinterpret_cast<uint4*>(t_region + ((size_t)kt * (N / 8) + grp) * 16) = make_uint4(lo[0], lo[1], hi[0], hi[1]);
     e_region[(size_t)grp * lut3_e_stride(K) + kt] = e;
   }
 }

@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
   __shared__ __align__(8) uint64_t full_bar[kSkStages];
   __shared__ __align__(8) uint64_t empty_bar[kSkStages];
   __shared__ unsigned int s_last;
-  __shared__ uint2 zlut[ASYM ? 256 : 1];  // z + 128 -> constant A operands {class A, class B}
+  __shared__ uint2 zlut[ASYM ? 256 : 1];  // z + 128 -> zero-point constants {za, zb}
   // ring base: the first 1024-byte boundary of the dynamic shared memory
   uint8_t* ring = dsmem + ((1024u - (smem_u32(dsmem) & 1023u)) & 1023u);
 
@@ -167,8 +167,8 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
   if (ASYM) {
     for (int i = tid; i < 256; i += kSkThreads) {
       const float z = (float)(i - 128);
-      zlut[i] = BF16 ? make_uint2(pack_bf16x2(-(128.0f + z)), 0u)
-                     : make_uint2(pack_f16x2(-(1024.0f + z)), pack_f16x2(-(1024.0f + 16.0f * z)));
+      zlut[i] = BF16 ? make_uint2(pack_bf16x2(128.0f + z), 0u)
+                     : make_uint2(pack_f16x2(1024.0f + z), pack_f16x2(-(64.0f + z)));
     }
   }
   __syncthreads();
@@ -236,10 +236,11 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
   }
   const int s_off_r = kOffS + lrow * 2, s_off_r8 = s_off_r + 8 * 2;
   const int z_off_r = kOffZ + lrow, z_off_r8 = z_off_r + 8;
-  // constant A operands of the offset-removing MMAs (symmetric: z = 8)
-  uint32_t ca_r = BF16 ? pack_bf16x2(-136.0f) : pack_f16x2(-1032.0f);
-  uint32_t cb_r = BF16 ? 0u : pack_f16x2(-1152.0f);  // -(1024 + 16*8)
-  uint32_t ca_r8 = ca_r, cb_r8 = cb_r;
+  // zero-point constants of rows lrow / lrow + 8 (symmetric: z = 8)
+  //   FP16: za = (1024 + z) pair, zb = -(64 + z) pair;  BF16: za = (128 + z) pair
+  uint32_t za_r = BF16 ? pack_bf16x2(136.0f) : pack_f16x2(1032.0f);
+  uint32_t zb_r = BF16 ? 0u : pack_f16x2(-72.0f);
+  uint32_t za_r8 = za_r, zb_r8 = zb_r;
 
   int it = 0;
   bool ok = true;
@@ -253,7 +254,7 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
     for (int n = 0; n < NT; ++n)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[n][i] = 0.0f;
-    float dA[NT][4], dB[NT][4];
+    float d[NT][4];
     float s_r = 0.0f, s_r8 = 0.0f;
 
     for (int st = st0; st < st1; ++st, ++it) {
@@ -277,65 +278,53 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
             const int z0 = *reinterpret_cast<const int8_t*>(sp + z_off_r + gl * kSkRows);
             const int z1 = *reinterpret_cast<const int8_t*>(sp + z_off_r8 + gl * kSkRows);
             const uint2 c0 = zlut[z0 + 128], c1 = zlut[z1 + 128];
-            ca_r = c0.x; cb_r = c0.y;
-            ca_r8 = c1.x; cb_r8 = c1.y;
+            za_r = c0.x; zb_r = c0.y;
+            za_r8 = c1.x; zb_r8 = c1.y;
           }
         }
         const uint32_t wa = wr[ci >> 1][(ci & 1) ? 2 : 0], wb = wr[ci >> 1][(ci & 1) ? 3 : 1];
-        const uint32_t ca[4] = {ca_r, ca_r8, ca_r, ca_r8};
+        uint32_t a0[4], a1[4];
         if (!BF16) {
-          // class A: (k0,k1) (k4,k5) = 1024+q;  class B: (k2,k3) (k6,k7) = 1024+16q
+          // (k0,k1) (k4,k5): 1024 + q minus (1024 + z);  (k2,k3) (k6,k7): (1024 + 16 q) / 16 - (64 + z)
           const uint32_t ta = wa >> 8, tb = wb >> 8;
-          const uint32_t aA[4] = {and_or(wa, 0x000F000Fu, 0x64006400u), and_or(wb, 0x000F000Fu, 0x64006400u),
-                                  and_or(ta, 0x000F000Fu, 0x64006400u), and_or(tb, 0x000F000Fu, 0x64006400u)};
-          const uint32_t aB[4] = {and_or(wa, 0x00F000F0u, 0x64006400u), and_or(wb, 0x00F000F0u, 0x64006400u),
-                                  and_or(ta, 0x00F000F0u, 0x64006400u), and_or(tb, 0x00F000F0u, 0x64006400u)};
-          const uint32_t cb[4] = {cb_r, cb_r8, cb_r, cb_r8};
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-            if (x_ok[n]) xv = *reinterpret_cast<const uint4*>(sp + x_off[n][ci & 1] + (ci >> 1) * kXBox);
-            if (group_start) {
-              mma_16816_zc(dA[n], aA, xv.x, xv.z, false);
-              mma_16816_zc(dB[n], aB, xv.y, xv.w, false);
-            } else {
-              mma_16816(dA[n], aA, xv.x, xv.z, false);
-              mma_16816(dB[n], aB, xv.y, xv.w, false);
-            }
-            mma_16816(dA[n], ca, xv.x, xv.z, false);
-            mma_16816(dB[n], cb, xv.y, xv.w, false);
-          }
+          a0[0] = hsub2_u32(and_or(wa, 0x000F000Fu, 0x64006400u), za_r);
+          a0[1] = hsub2_u32(and_or(wb, 0x000F000Fu, 0x64006400u), za_r8);
+          a0[2] = hsub2_u32(and_or(ta, 0x000F000Fu, 0x64006400u), za_r);
+          a0[3] = hsub2_u32(and_or(tb, 0x000F000Fu, 0x64006400u), za_r8);
+          a1[0] = hfma2_u32(and_or(wa, 0x00F000F0u, 0x64006400u), 0x2C002C00u, zb_r);
+          a1[1] = hfma2_u32(and_or(wb, 0x00F000F0u, 0x64006400u), 0x2C002C00u, zb_r8);
+          a1[2] = hfma2_u32(and_or(ta, 0x00F000F0u, 0x64006400u), 0x2C002C00u, zb_r);
+          a1[3] = hfma2_u32(and_or(tb, 0x00F000F0u, 0x64006400u), 0x2C002C00u, zb_r8);
         } else {
-          const uint32_t a0[4] = {and_or(wa, 0x000F000Fu, 0x43004300u), and_or(wb, 0x000F000Fu, 0x43004300u),
-                                  and_or(wa >> 4, 0x000F000Fu, 0x43004300u), and_or(wb >> 4, 0x000F000Fu, 0x43004300u)};
-          const uint32_t a1[4] = {and_or(wa >> 8, 0x000F000Fu, 0x43004300u), and_or(wb >> 8, 0x000F000Fu, 0x43004300u),
-                                  and_or(wa >> 12, 0x000F000Fu, 0x43004300u), and_or(wb >> 12, 0x000F000Fu, 0x43004300u)};
+          // pairs (k0,k1) (k2,k3) | (k4,k5) (k6,k7): 128 + q minus (128 + z)
+          a0[0] = bsub2_u32(and_or(wa, 0x000F000Fu, 0x43004300u), za_r);
+          a0[1] = bsub2_u32(and_or(wb, 0x000F000Fu, 0x43004300u), za_r8);
+          a0[2] = bsub2_u32(and_or(wa >> 4, 0x000F000Fu, 0x43004300u), za_r);
+          a0[3] = bsub2_u32(and_or(wb >> 4, 0x000F000Fu, 0x43004300u), za_r8);
+          a1[0] = bsub2_u32(and_or(wa >> 8, 0x000F000Fu, 0x43004300u), za_r);
+          a1[1] = bsub2_u32(and_or(wb >> 8, 0x000F000Fu, 0x43004300u), za_r8);
+          a1[2] = bsub2_u32(and_or(wa >> 12, 0x000F000Fu, 0x43004300u), za_r);
+          a1[3] = bsub2_u32(and_or(wb >> 12, 0x000F000Fu, 0x43004300u), za_r8);
+        }
 #pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-            if (x_ok[n]) xv = *reinterpret_cast<const uint4*>(sp + x_off[n][ci & 1] + (ci >> 1) * kXBox);
-            // dA: first half of the chunk's k + the second half's correction; dB the other way round
-            if (group_start) {
-              mma_16816_zc(dA[n], a0, xv.x, xv.y, true);
-              mma_16816_zc(dB[n], a1, xv.z, xv.w, true);
-            } else {
-              mma_16816(dA[n], a0, xv.x, xv.y, true);
-              mma_16816(dB[n], a1, xv.z, xv.w, true);
-            }
-            mma_16816(dB[n], ca, xv.x, xv.y, true);
-            mma_16816(dA[n], ca, xv.z, xv.w, true);
-          }
+        for (int n = 0; n < NT; ++n) {
+          uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+          if (x_ok[n]) xv = *reinterpret_cast<const uint4*>(sp + x_off[n][ci & 1] + (ci >> 1) * kXBox);
+          // FP16: a0 holds k-slots {0,1 | 4,5} of the 8-k word, a1 {2,3 | 6,7};
+          // BF16: a0 {0,1 | 2,3}, a1 {4,5 | 6,7}
+          const uint32_t b00 = xv.x, b01 = BF16 ? xv.y : xv.z, b10 = BF16 ? xv.z : xv.y, b11 = xv.w;
+          if (group_start) mma_16816_zc(d[n], a0, b00, b01, BF16);
+          else mma_16816(d[n], a0, b00, b01, BF16);
+          mma_16816(d[n], a1, b10, b11, BF16);
         }
         const bool group_end = (ci % GC == GC - 1) || (!KFULL && k0 + 32 * ci + 32 >= K);
         if (group_end) {
 #pragma unroll
           for (int n = 0; n < NT; ++n) {
-            // FP16: D = dA + dB/16 (class B carries 16 q); BF16: D = dA + dB
-            const float f = BF16 ? 1.0f : 0.0625f;
-            acc[n][0] = fmaf(s_r, fmaf(dB[n][0], f, dA[n][0]), acc[n][0]);
-            acc[n][1] = fmaf(s_r, fmaf(dB[n][1], f, dA[n][1]), acc[n][1]);
-            acc[n][2] = fmaf(s_r8, fmaf(dB[n][2], f, dA[n][2]), acc[n][2]);
-            acc[n][3] = fmaf(s_r8, fmaf(dB[n][3], f, dA[n][3]), acc[n][3]);
+            acc[n][0] = fmaf(s_r, d[n][0], acc[n][0]);
+            acc[n][1] = fmaf(s_r, d[n][1], acc[n][1]);
+            acc[n][2] = fmaf(s_r8, d[n][2], acc[n][2]);
+            acc[n][3] = fmaf(s_r8, d[n][3], acc[n][3]);
           }
         }
       }

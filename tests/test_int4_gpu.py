@@ -72,16 +72,35 @@ def test_pack_outliers_bit_exact(torch, lbq):
         _pack_and_compare(torch, lbq, W, group, "sym")
 
 
+PATHS = {"auto": 0, "cudacore_m1": 1, "warp_mma": 2, "tcgen05": 3}
+
+
+class gemv_path:
+    """Route lbq_gemv to one kernel for the duration of a block (test hook)."""
+
+    def __init__(self, lbq, name):
+        self.lbq, self.path = lbq, PATHS[name]
+
+    def __enter__(self):
+        self.lbq.lbq_debug_gemv_path(self.path)
+
+    def __exit__(self, *exc):
+        self.lbq.lbq_debug_gemv_path(0)
+
+
 @pytest.mark.parametrize("K,N,group,mode", SHAPES)
 @pytest.mark.parametrize("xdt", ["f16", "bf16"])
-def test_gemv_m1_parity(torch, lbq, K, N, group, mode, xdt):
+@pytest.mark.parametrize("path", ["auto", "warp_mma", "tcgen05"])
+def test_gemv_m1_parity(torch, lbq, K, N, group, mode, xdt, path):
     W = _special_groups(workloads.weights_host(11 + K + N, K, N), group)
     img, ref = _pack_and_compare(torch, lbq, W, group, mode)
     X = workloads.activations_host(5 + K, 1, K, xdt)
-    for ydt in ("f16", "bf16"):
-        Y = lbq.gemv(X.cuda(), img, N, group, mode, y_dtype=ydt)
-        torch.cuda.synchronize()
-        check_outputs(Y.cpu(), X, ref["deq"])
+    with gemv_path(lbq, path):
+        for ydt in ("f16", "bf16"):
+            Y = lbq.gemv(X.cuda(), img, N, group, mode, y_dtype=ydt)
+            torch.cuda.synchronize()
+            check_outputs(Y.cpu(), X, ref["deq"])
+    lbq.device_status()
 
 
 @pytest.mark.parametrize("splits", [2, 3, 4, 7])
@@ -204,19 +223,23 @@ SKINNY_SHAPES = [
 
 @pytest.mark.parametrize("M", [2, 3, 8, 9, 16])
 @pytest.mark.parametrize("K,N,group,mode,xdt", SKINNY_SHAPES)
-def test_skinny_parity(torch, lbq, M, K, N, group, mode, xdt):
+@pytest.mark.parametrize("path", ["auto", "tcgen05"])
+def test_skinny_parity(torch, lbq, M, K, N, group, mode, xdt, path):
     W = _special_groups(workloads.weights_host(300 + K + N, K, N), group)
     ref = oracle_int4(W, group, mode)
     img = lbq.pack(torch.from_numpy(W).cuda(), group, mode)
     X = workloads.activations_host(300 + M, M, K, xdt)
-    for ydt in ("f16", "bf16"):
-        Y = lbq.gemv(X.cuda(), img, N, group, mode, y_dtype=ydt)
-        torch.cuda.synchronize()
-        check_outputs(Y.cpu(), X, ref["deq"])
+    with gemv_path(lbq, path):
+        for ydt in ("f16", "bf16"):
+            Y = lbq.gemv(X.cuda(), img, N, group, mode, y_dtype=ydt)
+            torch.cuda.synchronize()
+            check_outputs(Y.cpu(), X, ref["deq"])
+    lbq.device_status()
 
 
-@pytest.mark.parametrize("K,N,M", [(4096, 520, 5), (14336, 1000, 16), (8192, 128, 3)])
-def test_skinny_stream_k_shared_tiles(torch, lbq, K, N, M):
+@pytest.mark.parametrize("K,N,M", [(4096, 520, 5), (14336, 1000, 16), (8192, 128, 3), (14336, 264, 1)])
+@pytest.mark.parametrize("path", ["auto", "tcgen05"])
+def test_skinny_stream_k_shared_tiles(torch, lbq, K, N, M, path):
     """Few row tiles over many CTAs: row tiles are shared between CTAs and
     finished by the last one; three calls on one workspace give identical,
     correct results (so the tile counters are reset after every call)."""
@@ -224,10 +247,12 @@ def test_skinny_stream_k_shared_tiles(torch, lbq, K, N, M):
     ref = oracle_int4(W, 64, "asym")
     img = lbq.pack(torch.from_numpy(W).cuda(), 64, "asym")
     X = workloads.activations_host(91, M, K, "bf16")
-    ws = lbq.workspace(0, M, K, N, 64, "asym")
-    assert ws is not None
-    Ys = [lbq.gemv(X.cuda(), img, N, 64, "asym", ws=ws) for _ in range(3)]
-    torch.cuda.synchronize()
+    with gemv_path(lbq, path):
+        ws = lbq.workspace(0, M, K, N, 64, "asym")
+        assert ws is not None
+        Ys = [lbq.gemv(X.cuda(), img, N, 64, "asym", ws=ws) for _ in range(3)]
+        torch.cuda.synchronize()
+    lbq.device_status()
     for Y in Ys:
         check_outputs(Y.cpu(), X, ref["deq"])
     assert all(torch.equal(Ys[0], Y) for Y in Ys[1:])

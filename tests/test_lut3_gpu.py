@@ -70,6 +70,20 @@ def test_pack_unpack_and_decode_bit_exact(torch, lbq, K, N):
     W = lbq.dequant(img, K, N, 0, "lut3").cpu().numpy()[:, ch]
     ref = lut3.dequant(idx[:, ch], cb[:, cols], ex[:, cols])
     assert np.array_equal(W.astype(np.float64), ref)
+    _check_tables(torch, img, K, N, cb, ex)
+
+
+def _check_tables(torch, img, K, N, cb, ex):
+    """The image's per-tile decode tables (what the GEMV / GEMM kernels read):
+    the tile's 8 weights e4m3(cb) * 2^(E-127) as BF16, low bytes then high bytes."""
+    raw = img.cpu().numpy()
+    off3 = int(raw[56:64].view(np.uint64)[0])
+    T = raw[off3:off3 + (K // 64) * (N // 8) * 16].reshape(K // 64, N // 8, 16)
+    got = T[..., :8].astype(np.uint16) | (T[..., 8:].astype(np.uint16) << 8)
+    vals = lut3.E4M3_TABLE[cb] * np.ldexp(1.0, ex.astype(np.int64) - 127)[..., None]
+    want = torch.from_numpy(vals.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(vals.astype(np.float32).astype(np.float64), vals)  # exact in FP32, hence in BF16
+    assert np.array_equal(got, want)
 
 
 def _check_gemm(torch, lbq, idx, cb, ex, img, X, groups=None, y_dtype=None):
