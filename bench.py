@@ -297,7 +297,8 @@ def weight_copies(img0, l2_bytes, minimum=3):
 
 
 # the GEMV kernels the library does not pick by default, timed beside the default
-GEMV_ALT_PATHS = (("cudacore_m1_kernel", 1), ("warp_mma_kernel", 2), ("tcgen05_kernel", 3))
+GEMV_ALT_PATHS = (("tma_cudacore_m1_kernel", 1), ("direct_m1_kernel", 4), ("warp_mma_kernel", 2),
+                  ("tcgen05_kernel", 3))
 
 
 def secondary_measurements(torch, lbq, workloads, device, peaks, quick):
@@ -339,7 +340,7 @@ def secondary_measurements(torch, lbq, workloads, device, peaks, quick):
             out[f"c3_g{group}_m{M}"] = {"us": ms * 1e3, "GBps": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm}
             if M in (1, 16):
                 for name, path in GEMV_ALT_PATHS:
-                    if path == 1 and M != 1 or path == 2 and M != 1:
+                    if path in (1, 2, 4) and M != 1:
                         continue
                     lbq.lbq_debug_gemv_path(path)
                     ws = lbq.workspace(0, M, K, N, group, "sym")

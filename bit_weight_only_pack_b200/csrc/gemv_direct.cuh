@@ -1,0 +1,161 @@
+// Decode GEMV at batch 1 on INT4 weights with plain vector loads:
+// y[n] = sum_k x[k] * (q[k][n] - z) * s.
+//
+// At batch 1 every weight is used once, so the kernel is a stream: the code
+// bytes go from HBM straight to registers (16-byte non-allocating loads, 512
+// contiguous bytes per warp instruction), with no staging through shared
+// memory and no producer/consumer handshakes.
+//
+//  * A CTA owns blocks of 8 output rows (grid-stride) and the whole K range;
+//    lane l of warp w takes the 32-k chunk c = 32w + l (K <= 16384). Its
+//    activations (32 values per chunk) and their offset sums stay in registers
+//    for all the CTA's row blocks.
+//  * Per row block and chunk a lane loads the 8 rows' 16-byte code chunks,
+//    one 16-byte load of the 8 rows' scales and one 8-byte load of their zero
+//    points (the image stores them 128 channels at a time, so 8 consecutive
+//    rows are contiguous). The next row block's codes are loaded before the
+//    current one is computed.
+//  * Codes become FP16 (BF16) operands 1024 + q (128 + q) with one AND/OR per
+//    pair, multiplied by x with FP32 accumulation (exact products); per chunk
+//    the offset and the zero point are removed with the chunk's activation sum,
+//    then the scale is applied.
+//  * Each warp reduces its 8 row partials over its lanes (transposing
+//    butterfly); the warps of the CTA are added in a fixed order through shared
+//    memory, so results do not depend on timing.
+#pragma once
+
+#include "common.cuh"
+#include "gemv_m1.cuh"
+
+namespace lbq {
+
+constexpr int kGdMaxWarps = 16;
+
+struct GemvDirectArgs {
+  const uint16_t* X;       // [K] FP16/BF16 bits
+  void* Y;                 // [N]
+  const uint8_t* q;        // [N][K/2]
+  const uint8_t* s;        // 128-channel-tiled FP16 scales
+  const uint8_t* z;        // 128-channel-tiled int8 zero points (ASYM)
+  int K, N, G;
+  int row_blocks;          // ceil(N / 8)
+  int y_bf16;
+};
+
+// sum over one 16-byte chunk (32 k) of x * (offset-form weight), FP32.
+template <bool BF16>
+__device__ __forceinline__ float gd_chunk(const uint4 w, const uint32_t (&x)[16]) { return chunk_acc<BF16>(w, x); }
+
+// One chunk per lane: K <= 32 * 32 * kGdMaxWarps.
+template <bool BF16, bool ASYM>
+__global__ void __launch_bounds__(kGdMaxWarps * 32, 1) gemv_direct_kernel(const GemvDirectArgs a) {
+  constexpr int J = 1;
+  __shared__ float red[kGdMaxWarps][8];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nw = blockDim.x >> 5;
+  const int chunks = a.K >> 5;
+  const size_t rowb = (size_t)(a.K >> 1);  // code bytes per row
+  const int gpc = (a.K / a.G) >> 5;        // chunks per group (1, 2 or 4)
+
+  // this lane's chunks and their activations (read once for all row blocks)
+  uint32_t xr[J][16];
+  float xoff[J], xsum[J];
+  int cidx[J];
+  bool cok[J];
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    cidx[j] = warp * 32 + lane + j * nw * 32;
+    cok[j] = cidx[j] < chunks;
+  }
+
+  // codes of the current and the next row block
+  uint4 cur[J][8], nxt[J][8];
+  auto load_block = [&](int rb, uint4 (&w)[J][8]) {
+    const int r0 = rb * 8;
+#pragma unroll
+    for (int j = 0; j < J; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        w[j][i] = make_uint4(0u, 0u, 0u, 0u);
+        if (cok[j] && r0 + i < a.N) w[j][i] = ld_stream_v4(a.q + (size_t)(r0 + i) * rowb + (size_t)cidx[j] * 16);
+      }
+  };
+
+  // The weights are only read, so the first row block is requested before
+  // waiting for the previous kernel in the stream (which may write X).
+  int rb = blockIdx.x;
+  if (rb < a.row_blocks) load_block(rb, cur);
+  griddep_launch_dependents();
+  griddep_wait();
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int c = cidx[j];
+    float sA = 0.0f, sB = 0.0f;
+    if (cok[j]) {
+      const uint4* xp = reinterpret_cast<const uint4*>(a.X + (size_t)c * 32);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 u = ld_nc_v4(xp + v);
+        xr[j][4 * v + 0] = u.x; xr[j][4 * v + 1] = u.y; xr[j][4 * v + 2] = u.z; xr[j][4 * v + 3] = u.w;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float lo = x2f<BF16>((uint16_t)(xr[j][i] & 0xFFFFu));
+        const float hi = x2f<BF16>((uint16_t)(xr[j][i] >> 16));
+        if ((i & 1) == 0) sA += lo + hi; else sB += lo + hi;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) xr[j][i] = 0u;
+    }
+    const float xs = sA + sB;
+    xsum[j] = xs;
+    // FP16: slots of class A carry 1024 + q, class B (1024 + 16 q)/16 after chunk_acc
+    xoff[j] = (BF16 ? 128.0f * xs : 1024.0f * sA + 64.0f * sB) + (ASYM ? 0.0f : 8.0f * xs);
+  }
+
+  for (; rb < a.row_blocks; rb += gridDim.x) {
+    const int rbn = rb + gridDim.x;
+    if (rbn < a.row_blocks) load_block(rbn, nxt);
+    const int r0 = rb * 8;
+    float part[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) part[i] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      if (!cok[j]) continue;
+      const int g = cidx[j] / gpc;
+      const size_t m0 = ((size_t)(r0 >> 7) * a.G + g) * 128 + (r0 & 127);  // 8 consecutive rows, 16-byte aligned
+      const uint4 sv = ld_nc_v4(a.s + m0 * 2);
+      uint2 zv = make_uint2(0u, 0u);
+      if (ASYM) zv = *reinterpret_cast<const uint2*>(a.z + m0);
+      const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float acc = gd_chunk<BF16>(cur[j][i], xr[j]);
+        float corr = xoff[j];
+        if (ASYM) {
+          const int zi = (int)(int8_t)(((i < 4 ? zv.x : zv.y) >> (8 * (i & 3))) & 0xFFu);
+          corr = fmaf((float)zi, xsum[j], corr);
+        }
+        const float sc = h2f_bits((uint16_t)(sw[i >> 1] >> (16 * (i & 1))));
+        part[i] = fmaf(sc, acc - corr, part[i]);
+      }
+    }
+    const float total = butterfly8(part, lane);
+    if ((lane & 3) == 0) red[warp][butterfly8_row(lane)] = total;
+    __syncthreads();
+    if (warp == 0 && lane < 8) {
+      float sum = 0.0f;
+      for (int w = 0; w < nw; ++w) sum += red[w][lane];
+      if (r0 + lane < a.N) store_out(a.Y, (size_t)(r0 + lane), sum, a.y_bf16);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < J; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) cur[j][i] = nxt[j][i];
+  }
+}
+
+}  // namespace lbq

@@ -25,6 +25,7 @@
 #include "lut3_gemv.cuh"
 #include "gemm_tc.cuh"
 #include "tc_gemv.cuh"
+#include "gemv_direct.cuh"
 
 namespace lbq {
 
@@ -147,10 +148,11 @@ struct M1Plan {
 static int g_force_splits = 0;  // test hook: force a split count (0 = shape-based choice)
 static int g_pdl = 0;           // launch GEMVs with programmatic dependent launch
 static int g_force_skinny = 0;  // test hook: route M = 1 to the tensor-core skinny kernel
-// test hook: GEMV kernel for M <= 16. 0 = the library's choice, 1 = the CUDA-core
-// M = 1 kernel, 2 = the warp-MMA skinny kernel, 3 = the tcgen05 kernel.
+// test hook: GEMV kernel for M <= 16. 0 = the library's choice, 1 = the
+// TMA-pipelined CUDA-core M = 1 kernel, 2 = the warp-MMA skinny kernel, 3 = the
+// tcgen05 kernel, 4 = the direct-load CUDA-core M = 1 kernel.
 static int g_gemv_path = 0;
-enum { kPathAuto = 0, kPathM1 = 1, kPathMma = 2, kPathTc = 3 };
+enum { kPathAuto = 0, kPathM1 = 1, kPathMma = 2, kPathTc = 3, kPathDirect = 4 };
 
 constexpr int kM1RingBudget = 100 * 1024;
 constexpr int kM1MaxChunksPerSplit = 128;  // K-slices of at most 4096 k keep a ring slot near 20 KB
@@ -436,17 +438,46 @@ static lbq_status run_tcgemv(const void* X, bool xbf16, int M, const void* image
                           "tcgen05 GEMV launch");
 }
 
+// M = 1, direct loads (no workspace).
+static lbq_status run_direct(const uint16_t* X, bool xbf16, const void* image, const Layout& L, void* Y, bool ybf16,
+                             cudaStream_t st) {
+  const bool asym = L.mode == LBQ_MODE_ASYM;
+  const int chunks = L.K / 32;
+  const int nw = (chunks + 31) / 32;
+  if (nw > kGdMaxWarps) return fail(LBQ_ERR_UNSUPPORTED, "direct GEMV needs K <= %d", 32 * 32 * kGdMaxWarps);
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  GemvDirectArgs a{};
+  a.X = X;
+  a.Y = Y;
+  a.q = img + L.off0;
+  a.s = img + L.off1;
+  a.z = asym ? img + L.off2 : nullptr;
+  a.K = L.K; a.N = L.N; a.G = L.K / L.group;
+  a.row_blocks = (L.N + 7) / 8;
+  a.y_bf16 = ybf16 ? 1 : 0;
+  const void* fn = xbf16 ? (asym ? (const void*)gemv_direct_kernel<true, true> : (const void*)gemv_direct_kernel<true, false>)
+                         : (asym ? (const void*)gemv_direct_kernel<false, true> : (const void*)gemv_direct_kernel<false, false>);
+  const int occ = std::max(1, occupancy_for(fn, nw * 32, 0));
+  const int grid = std::min(a.row_blocks, num_sms() * occ);
+  void* args[] = {&a};
+  return launch_kernel_ex(fn, dim3(grid), dim3(nw * 32), 0, st, g_pdl != 0, args, "direct GEMV launch");
+}
+
 // The kernel lbq_gemv runs for M <= 16. Measured on B200: at M = 1 the
-// CUDA-core kernel is faster up to ~10^8 weights (the warp-MMA kernel spends an
-// MMA, 7/8 wasted, per 256 weights, and legacy MMA throughput is the limit);
-// from M = 2 the warp-MMA kernel wins. The tcgen05 kernel is slower at every
-// batch size here (a 128 x 16 x N MMA costs the same ~185 cycles for N = 16
-// as for N = 256), so it is never the default.
-static int gemv_path(int M, long long weights) {
+// direct-load CUDA-core kernel is the fastest at every size it supports
+// (K <= 16384; the warp-MMA kernel spends an MMA, 7/8 wasted, per 256 weights
+// and legacy MMA throughput is its limit); from M = 2 the warp-MMA kernel wins.
+// The tcgen05 kernel is slower at every batch size here (a 128 x 16 x N MMA
+// costs the same ~185 cycles for N = 16 as for N = 256), so it is never the
+// default.
+static int gemv_path(int M, int K, long long weights) {
+  const bool direct_ok = M == 1 && K <= 32 * 32 * kGdMaxWarps;
   if (g_gemv_path == kPathM1 && M == 1) return kPathM1;
+  if (g_gemv_path == kPathDirect && direct_ok) return kPathDirect;
   if (g_gemv_path == kPathMma || g_gemv_path == kPathTc) return g_gemv_path;
   if (g_force_skinny) return kPathMma;
-  if (M == 1 && (g_force_splits || weights < (1LL << 27))) return kPathM1;
+  if (M == 1 && g_force_splits) return kPathM1;
+  if (M == 1) return direct_ok ? kPathDirect : (weights < (1LL << 27) ? kPathM1 : kPathMma);
   return kPathMma;
 }
 
@@ -458,7 +489,8 @@ struct GemvScratch {
 
 static GemvScratch gemv_scratch(int M, int K, int N, int group, bool asym, bool xbf16) {
   GemvScratch g{0, 0, 0};
-  const int path = gemv_path(M, (long long)K * N);
+  const int path = gemv_path(M, K, (long long)K * N);
+  if (path == kPathDirect) return g;
   if (path == kPathM1) {
     const M1Plan p = plan_m1(K, N, group, asym, g_force_splits);
     g.need = p.block == 0 ? 0 : m1_workspace_bytes(p, N);
@@ -655,8 +687,9 @@ void lbq_debug_force_tc(int on) { g_force_tc = on ? 1 : 0; }
 void lbq_debug_force_skinny(int on) { g_force_skinny = on ? 1 : 0; }
 
 // Test hook (not in the public header): pick the GEMV kernel for M <= 16
-// (0 = the library's choice, 1 = CUDA-core M = 1, 2 = warp MMA, 3 = tcgen05).
-void lbq_debug_gemv_path(int path) { g_gemv_path = (path >= 0 && path <= 3) ? path : 0; }
+// (0 = the library's choice, 1 = TMA-pipelined CUDA-core M = 1, 2 = warp MMA,
+// 3 = tcgen05, 4 = direct-load CUDA-core M = 1).
+void lbq_debug_gemv_path(int path) { g_gemv_path = (path >= 0 && path <= 4) ? path : 0; }
 
 lbq_status lbq_set_option(int option, int value) {
   if (option == LBQ_OPT_PDL) {
@@ -753,7 +786,10 @@ lbq_status lbq_gemv(const void* X, int x_dtype, int M, int K, int N, int group, 
   if (M > 16) return fail(LBQ_ERR_UNSUPPORTED, "lbq_gemv takes M <= 16 (M=%d); use lbq_gemm", M);
   const Layout L = make_layout(K, N, group, mode);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int path = gemv_path(M, (long long)K * N);
+  const int path = gemv_path(M, K, (long long)K * N);
+  if (path == kPathDirect)
+    return run_direct(static_cast<const uint16_t*>(X), x_dtype == LBQ_DTYPE_BF16, image, L, Y,
+                      y_dtype == LBQ_DTYPE_BF16, s);
   if (path == kPathM1)
     return run_m1(static_cast<const uint16_t*>(X), x_dtype == LBQ_DTYPE_BF16, image, L, Y, y_dtype == LBQ_DTYPE_BF16,
                   ws, ws_bytes, s);

@@ -72,7 +72,7 @@ def test_pack_outliers_bit_exact(torch, lbq):
         _pack_and_compare(torch, lbq, W, group, "sym")
 
 
-PATHS = {"auto": 0, "cudacore_m1": 1, "warp_mma": 2, "tcgen05": 3}
+PATHS = {"auto": 0, "cudacore_m1": 1, "warp_mma": 2, "tcgen05": 3, "direct_m1": 4}
 
 
 class gemv_path:
@@ -90,7 +90,7 @@ class gemv_path:
 
 @pytest.mark.parametrize("K,N,group,mode", SHAPES)
 @pytest.mark.parametrize("xdt", ["f16", "bf16"])
-@pytest.mark.parametrize("path", ["auto", "warp_mma", "tcgen05"])
+@pytest.mark.parametrize("path", ["auto", "cudacore_m1", "warp_mma", "tcgen05"])
 def test_gemv_m1_parity(torch, lbq, K, N, group, mode, xdt, path):
     W = _special_groups(workloads.weights_host(11 + K + N, K, N), group)
     img, ref = _pack_and_compare(torch, lbq, W, group, mode)
@@ -238,7 +238,7 @@ def test_skinny_parity(torch, lbq, M, K, N, group, mode, xdt, path):
 
 
 @pytest.mark.parametrize("K,N,M", [(4096, 520, 5), (14336, 1000, 16), (8192, 128, 3), (14336, 264, 1)])
-@pytest.mark.parametrize("path", ["auto", "tcgen05"])
+@pytest.mark.parametrize("path", ["warp_mma", "tcgen05"])
 def test_skinny_stream_k_shared_tiles(torch, lbq, K, N, M, path):
     """Few row tiles over many CTAs: row tiles are shared between CTAs and
     finished by the last one; three calls on one workspace give identical,
