@@ -20,8 +20,9 @@
 //    the offset and the zero point are removed with the chunk's activation sum,
 //    then the scale is applied.
 //  * Each warp reduces its 8 row partials over its lanes (transposing
-//    butterfly); the warps of the CTA are added in a fixed order through shared
-//    memory, so results do not depend on timing.
+//    butterfly) and parks them in shared memory; after its last row block the
+//    CTA adds the warps' sums in a fixed order (one barrier per CTA, none per
+//    row block), so results do not depend on timing.
 #pragma once
 
 #include "common.cuh"
@@ -46,11 +47,12 @@ struct GemvDirectArgs {
 template <bool BF16>
 __device__ __forceinline__ float gd_chunk(const uint4 w, const uint32_t (&x)[16]) { return chunk_acc<BF16>(w, x); }
 
-// One chunk per lane: K <= 32 * 32 * kGdMaxWarps.
+// One chunk per lane: K <= 32 * 32 * kGdMaxWarps. Dynamic shared memory:
+// float [row blocks of this CTA][warps][8] of per-warp row sums.
 template <bool BF16, bool ASYM>
 __global__ void __launch_bounds__(kGdMaxWarps * 32, 1) gemv_direct_kernel(const GemvDirectArgs a) {
   constexpr int J = 1;
-  __shared__ float red[kGdMaxWarps][8];
+  extern __shared__ float red[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nw = blockDim.x >> 5;
   const int chunks = a.K >> 5;
@@ -114,7 +116,8 @@ __global__ void __launch_bounds__(kGdMaxWarps * 32, 1) gemv_direct_kernel(const 
     xoff[j] = (BF16 ? 128.0f * xs : 1024.0f * sA + 64.0f * sB) + (ASYM ? 0.0f : 8.0f * xs);
   }
 
-  for (; rb < a.row_blocks; rb += gridDim.x) {
+  int lb = 0;  // row block index within this CTA
+  for (; rb < a.row_blocks; rb += gridDim.x, ++lb) {
     const int rbn = rb + gridDim.x;
     if (rbn < a.row_blocks) load_block(rbn, nxt);
     const int r0 = rb * 8;
@@ -131,30 +134,35 @@ __global__ void __launch_bounds__(kGdMaxWarps * 32, 1) gemv_direct_kernel(const 
       if (ASYM) zv = *reinterpret_cast<const uint2*>(a.z + m0);
       const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float acc = gd_chunk<BF16>(cur[j][i], xr[j]);
-        float corr = xoff[j];
-        if (ASYM) {
-          const int zi = (int)(int8_t)(((i < 4 ? zv.x : zv.y) >> (8 * (i & 3))) & 0xFFu);
-          corr = fmaf((float)zi, xsum[j], corr);
+      for (int i = 0; i < 8; i += 2) {
+        const float2 sc = __half22float2(*reinterpret_cast<const __half2*>(&sw[i >> 1]));
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float acc = gd_chunk<BF16>(cur[j][i + h], xr[j]);
+          float corr = xoff[j];
+          if (ASYM) {
+            const int zi = (int)(int8_t)(((i < 4 ? zv.x : zv.y) >> (8 * ((i + h) & 3))) & 0xFFu);
+            corr = fmaf((float)zi, xsum[j], corr);
+          }
+          part[i + h] = fmaf(h ? sc.y : sc.x, acc - corr, part[i + h]);
         }
-        const float sc = h2f_bits((uint16_t)(sw[i >> 1] >> (16 * (i & 1))));
-        part[i] = fmaf(sc, acc - corr, part[i]);
       }
     }
     const float total = butterfly8(part, lane);
-    if ((lane & 3) == 0) red[warp][butterfly8_row(lane)] = total;
-    __syncthreads();
-    if (warp == 0 && lane < 8) {
-      float sum = 0.0f;
-      for (int w = 0; w < nw; ++w) sum += red[w][lane];
-      if (r0 + lane < a.N) store_out(a.Y, (size_t)(r0 + lane), sum, a.y_bf16);
-    }
-    __syncthreads();
+    if ((lane & 3) == 0) red[(lb * nw + warp) * 8 + butterfly8_row(lane)] = total;
 #pragma unroll
     for (int j = 0; j < J; ++j)
 #pragma unroll
       for (int i = 0; i < 8; ++i) cur[j][i] = nxt[j][i];
+  }
+  // the warps' row sums of every row block of this CTA, added in warp order
+  __syncthreads();
+  for (int t = tid; t < lb * 8; t += blockDim.x) {
+    const int l = t >> 3, row = t & 7;
+    const int r = (blockIdx.x + l * gridDim.x) * 8 + row;
+    float sum = 0.0f;
+    for (int w = 0; w < nw; ++w) sum += red[(l * nw + w) * 8 + row];
+    if (r < a.N) store_out(a.Y, (size_t)r, sum, a.y_bf16);
   }
 }
 

@@ -457,10 +457,16 @@ static lbq_status run_direct(const uint16_t* X, bool xbf16, const void* image, c
   a.y_bf16 = ybf16 ? 1 : 0;
   const void* fn = xbf16 ? (asym ? (const void*)gemv_direct_kernel<true, true> : (const void*)gemv_direct_kernel<true, false>)
                          : (asym ? (const void*)gemv_direct_kernel<false, true> : (const void*)gemv_direct_kernel<false, false>);
-  const int occ = std::max(1, occupancy_for(fn, nw * 32, 0));
-  const int grid = std::min(a.row_blocks, num_sms() * occ);
+  // one wave of CTAs; each keeps 8 floats per warp per row block in shared memory
+  int occ = std::max(1, occupancy_for(fn, nw * 32, 0));
+  int grid = std::min(a.row_blocks, num_sms() * occ);
+  int smem = ((a.row_blocks + grid - 1) / grid) * nw * 8 * (int)sizeof(float);
+  while (smem > 96 * 1024 && grid < a.row_blocks) {  // very tall matrices: more CTAs, fewer blocks each
+    grid = std::min(a.row_blocks, grid * 2);
+    smem = ((a.row_blocks + grid - 1) / grid) * nw * 8 * (int)sizeof(float);
+  }
   void* args[] = {&a};
-  return launch_kernel_ex(fn, dim3(grid), dim3(nw * 32), 0, st, g_pdl != 0, args, "direct GEMV launch");
+  return launch_kernel_ex(fn, dim3(grid), dim3(nw * 32), smem, st, g_pdl != 0, args, "direct GEMV launch");
 }
 
 // The kernel lbq_gemv runs for M <= 16. Measured on B200: at M = 1 the
