@@ -60,6 +60,7 @@ _SIGS = {
     "lbq_debug_force_skinny": ([_c_int], None),
     "lbq_debug_force_tc": ([_c_int], None),
     "lbq_debug_gemv_path": ([_c_int], None),
+    "lbq_debug_gemm_path": ([_c_int], None),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -159,6 +160,11 @@ def lbq_debug_force_tc(on):
 def lbq_debug_gemv_path(path):
     """Test hook: GEMV kernel for M <= 16 (0 auto, 1 CUDA-core M=1, 2 warp MMA, 3 tcgen05)."""
     _lib.lbq_debug_gemv_path(path)
+
+
+def lbq_debug_gemm_path(path):
+    """Test hook: prefill kernel (0 weights in tensor memory, 1 weights dequantised into shared memory)."""
+    _lib.lbq_debug_gemm_path(path)
 
 
 def lbq_debug_force_skinny(on):

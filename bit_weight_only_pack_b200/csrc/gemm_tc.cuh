@@ -17,10 +17,11 @@
 //               one thread issues 4 x tcgen05.mma.kind::f16 (M=128, N=256,
 //               K=16) per k-block into one of two TMEM accumulators and
 //               commits to the stage / B-tile / accumulator barriers.
-//   warps 2..5  dequantisers: codes -> BF16 (or FP16) weights written straight
-//               into the K-major 128-byte-swizzled layout the UMMA shared-
-//               memory descriptor describes; fence.proxy.async, then arrive.
-//   warps 6..9  epilogue: tcgen05.ld the finished accumulator (each warp its
+//   warps 2..9  dequantisers (one weight row each): codes -> BF16 (or FP16)
+//               weights written straight into the K-major 128-byte-swizzled
+//               layout the UMMA shared-memory descriptor describes;
+//               fence.proxy.async, then arrive.
+//   warps 10-13 epilogue: tcgen05.ld the finished accumulator (each warp its
 //               32 TMEM lanes = 32 tokens), round to BF16/FP16, store to Y;
 //               runs while the MMA fills the other accumulator.
 //
@@ -40,8 +41,9 @@ namespace lbq {
 
 constexpr int kTcBM = 128, kTcBN = 256, kTcBK = 64;
 constexpr int kTcStages = 4;                   // X + codes ring
-constexpr int kTcBStages = 2;                  // dequantised weight tiles
-constexpr int kTcDqWarps = 4, kTcEpWarps = 4;
+constexpr int kTcBStages = 3;                  // dequantised weight tiles
+constexpr int kTcDqWarps = 8, kTcEpWarps = 4;
+constexpr int kTcDqRows = kTcBN / (kTcDqWarps * 32);  // weight rows per dequantiser thread
 constexpr int kTcThreads = (2 + kTcDqWarps + kTcEpWarps) * 32;
 constexpr int kTcABytes = kTcBM * kTcBK * 2;   // 16 KB
 constexpr int kTcPBytes = kTcBN * kTcBK / 2;   // 8 KB of codes
@@ -256,7 +258,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
     }
   } else if (warp < 2 + kTcDqWarps) {
     // ------------------------------------------------------------------ dequantisers
-    const int dt = tid - 64;  // 0..127: rows dt and dt + 128 of the weight tile
+    const int dt = tid - 64;  // rows dt + kTcDqWarps * 32 * i of the weight tile
     int it = 0, bit = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
@@ -270,8 +272,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
         const uint32_t bt = smem_u32(btile + sb * kTcBBytes);
         if (LUT) {
 #pragma unroll
-          for (int hr = 0; hr < 2; ++hr) {
-            const int n = dt + 128 * hr;
+          for (int hr = 0; hr < kTcDqRows; ++hr) {
+            const int n = dt + kTcDqWarps * 32 * hr;
             if (nb * kTcBN + n >= a.N) continue;
             // 24 bytes of indices per channel: 8-byte aligned, so three 8-byte loads
             const uint8_t* ip = ring + s * kTcStageBytes + kTcABytes + n * 24;
@@ -303,8 +305,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(
         const int g0 = (kb * 2) >> a.gshift64;
         const int ng = min(a.gshift64 == 0 ? 2 : 1, a.G - g0);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int n = dt + 128 * h;
+        for (int h = 0; h < kTcDqRows; ++h) {
+          const int n = dt + kTcDqWarps * 32 * h;
           const uint4 p0 = lds128(st + kTcABytes + n * 32);
           const uint4 p1 = lds128(st + kTcABytes + n * 32 + 16);
           const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};

@@ -1,0 +1,278 @@
+// Prefill GEMM with the weights as the tcgen05 A operand in tensor memory:
+// Y^T[N, M] = dequant(W)^T[N, K] . X^T[K, M], tiles of 128 output channels
+// (the 128 TMEM lanes) x 256 tokens (the MMA's N).
+//
+// Putting the weights on the M side of the MMA makes every dequantised weight
+// serve 256 tokens (twice the reuse of a 128-token tile) and keeps the
+// dequantised operand out of shared memory: converter threads write it to
+// tensor memory with tcgen05.st, so shared memory only carries the TMA'd
+// activations (read once by the tensor core) and the packed codes.
+//
+//   warp 0      TMA producer: per 128-k block two activation boxes (256 tokens x
+//               64 k, 128-byte swizzle = the K-major B-operand layout), the
+//               channels' codes (128 rows x 64 bytes) and the block's scales /
+//               zero points (INT4) or LUT3 indices and decode tables.
+//   warp 1      TMEM owner and MMA issuer: 8 x tcgen05.mma (M = 128, N = 256,
+//               K = 16, A from tensor memory) per k-block into one accumulator
+//               (256 columns); commits free the A buffer and the stage. A
+//               barrier wait costs a few hundred cycles on this GPU, so the
+//               blocks are large enough that the waits hide behind the MMAs.
+//   warps 2..9  converters: thread (quarter q, lane l) owns channel 32q + l and
+//               two 32-k chunks of the k-block; INT4: w = (q - z) * s rounded once to the
+//               activation type (nibble -> 1024 + q / 128 + q by AND/OR, an
+//               exact packed subtract, one packed multiply); LUT3: the exact
+//               BF16 weight from the tile's table (byte permutes). 16 pairs
+//               per tcgen05.st. Four A buffers of 64 columns.
+//   warps 10-13 epilogue: tcgen05.ld the finished accumulator (thread = one
+//               channel, columns = tokens), round, store Y[token][channel].
+#pragma once
+
+#include "common.cuh"
+#include "tma.cuh"
+#include "skinny.cuh"
+#include "gemm_tc.cuh"
+#include "tc_gemv.cuh"
+#include "lut3_gemv.cuh"
+
+namespace lbq {
+
+constexpr int kTsBN = 128;                 // channels per tile (TMEM lanes)
+constexpr int kTsBM = 256;                 // tokens per tile (MMA N)
+constexpr int kTsBK = 128;                 // k per block: 8 MMAs per pair of barrier waits
+constexpr int kTsStages = 3;
+constexpr int kTsABufs = 4;                // A (weights) buffers in tensor memory, 64 columns each
+constexpr int kTsConvWarps = 8, kTsEpWarps = 4;
+// 32-k chunks per converter thread per block: the block's kTsBK / 32 chunks are
+// split over the kTsConvWarps / 4 warps that share a TMEM lane quarter
+constexpr int kTsChunksPerConv = (kTsBK / 32) / (kTsConvWarps / 4);
+static_assert(kTsChunksPerConv >= 1 && kTsChunksPerConv * (kTsConvWarps / 4) * 32 == kTsBK, "converter split");
+constexpr int kTsThreads = (2 + kTsConvWarps + kTsEpWarps) * 32;
+constexpr int kTsXBox = kTsBM * 64 * 2;             // one 64-k activation box (32 KB)
+constexpr int kTsXBytes = 2 * kTsXBox;              // 64 KB
+constexpr int kTsCBytes = kTsBN * 64;               // 8 KB codes (INT4) / 6 KB indices (LUT3)
+constexpr int kTsMBytes = 2048;                     // scales + zero points (INT4) / tables (LUT3)
+constexpr int kTsOffC = kTsXBytes, kTsOffM = kTsOffC + kTsCBytes;
+constexpr int kTsStageBytes = kTsOffM + kTsMBytes;  // 74 KB, a multiple of 1024
+constexpr int kTsSmem = kTsStages * kTsStageBytes + 1024;
+constexpr uint32_t kTsColA = 0, kTsColD = 256;
+static_assert(kTsStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
+
+struct GemmTsArgs {
+  void* Y;                   // [M][N]
+  const uint8_t* meta0;      // INT4: 128-channel-tiled scales; LUT3: I region (indices)
+  const uint8_t* meta1;      // INT4: 128-channel-tiled zero points (ASYM); LUT3: T region (tables)
+  int M, N, K, G, group;
+  int n_tiles, m_tiles, k_blocks;  // channel tiles, token tiles, 64-k blocks
+  int y_bf16;
+};
+
+template <bool BF16, bool ASYM, bool LUT>
+__global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_constant__ CUtensorMap tx,
+                                                                const __grid_constant__ CUtensorMap tq,
+                                                                const GemmTsArgs a) {
+  extern __shared__ uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t full_bar[kTsStages], empty_bar[kTsStages];
+  __shared__ __align__(8) uint64_t a_full[kTsABufs], a_empty[kTsABufs], d_full, d_empty;
+  __shared__ uint32_t tmem_base_sh;
+  uint8_t* ring = dsmem + ((1024u - (smem_u32(dsmem) & 1023u)) & 1023u);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int total_tiles = a.n_tiles * a.m_tiles;
+  const int nkb = a.k_blocks;
+
+  if (tid == 0) {
+    for (int i = 0; i < kTsStages; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1 + kTsConvWarps);
+    }
+    for (int i = 0; i < kTsABufs; ++i) {
+      mbar_init(&a_full[i], kTsConvWarps);
+      mbar_init(&a_empty[i], 1);
+    }
+    mbar_init(&d_full, 1);
+    mbar_init(&d_empty, kTsEpWarps);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(&tmem_base_sh)), "r"(512u) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tx);
+      if (!LUT) tma_prefetch_desc(&tq);
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;  // token tiles inner: codes reused from L2
+        const int rows = min(kTsBN, a.N - nt * kTsBN);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kTsStages;
+          if (it >= kTsStages && !mbar_wait(&empty_bar[s], ((it / kTsStages) & 1) ^ 1)) { ok = false; break; }
+          uint8_t* st = ring + (size_t)s * kTsStageBytes;
+          const int nxb = min(2, (a.K - kb * kTsBK + 63) / 64);  // 64-k activation boxes inside K
+          if (LUT) {
+            // the block's two 64-k LUT tiles: indices (24 B per channel) and tables (16 B per 8 channels)
+            mbar_arrive_expect_tx(&full_bar[s], (uint32_t)(nxb * (kTsXBox + rows * 24 + (rows / 8) * 16)));
+            for (int j = 0; j < nxb; ++j) {
+              const int kt = kb * 2 + j;
+              tma_load_2d(st + j * kTsXBox, &tx, kt * 64, mt * kTsBM, &full_bar[s]);
+              bulk_load(st + kTsOffC + j * (kTsBN * 24), a.meta0 + ((size_t)kt * a.N + nt * kTsBN) * 24,
+                        (uint32_t)(rows * 24), &full_bar[s]);
+              bulk_load(st + kTsOffM + j * 256, a.meta1 + ((size_t)kt * (a.N / 8) + nt * (kTsBN / 8)) * 16,
+                        (uint32_t)((rows / 8) * 16), &full_bar[s]);
+            }
+          } else {
+            const int g0 = (kb * kTsBK) / a.group;
+            const int ng = min(max(1, kTsBK / a.group), a.G - g0);  // K may end inside the block
+            mbar_arrive_expect_tx(&full_bar[s], (uint32_t)(nxb * kTsXBox + kTsCBytes + ng * 128 * (ASYM ? 3 : 2)));
+            for (int j = 0; j < nxb; ++j) tma_load_2d(st + j * kTsXBox, &tx, kb * kTsBK + 64 * j, mt * kTsBM, &full_bar[s]);
+            tma_load_2d(st + kTsOffC, &tq, kb * (kTsBK / 2), nt * kTsBN, &full_bar[s]);
+            const size_t m0 = ((size_t)nt * a.G + g0) * 128;
+            bulk_load(st + kTsOffM, a.meta0 + m0 * 2, (uint32_t)(ng * 256), &full_bar[s]);
+            if (ASYM) bulk_load(st + kTsOffM + 1024, a.meta1 + m0, (uint32_t)(ng * 128), &full_bar[s]);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_m128(BF16, kTsBM);
+      int it = 0, t_iter = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t_iter) {
+        if (t_iter >= 1 && !mbar_wait(&d_empty, (t_iter - 1) & 1)) break;
+        tc_fence_after();
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kTsStages, b = it % kTsABufs;
+          if (!mbar_wait(&full_bar[s], (it / kTsStages) & 1)) { ok = false; break; }
+          if (!mbar_wait(&a_full[b], (it / kTsABufs) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t xb = smem_u32(ring + (size_t)s * kTsStageBytes);
+          const int nkk = min(kTsBK, a.K - kb * kTsBK + 15) / 16;  // 16-k slices inside K (K % 32 == 0)
+          for (int kk = 0; kk < nkk; ++kk) {
+            const uint64_t db = umma_desc_sw128(xb + (uint32_t)(kk >> 2) * kTsXBox) + (uint64_t)((kk & 3) * 2);
+            umma_ts(tmem + kTsColD, tmem + kTsColA + (uint32_t)b * 64 + (uint32_t)kk * 8, db, idesc,
+                    (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty_bar[s]);
+          umma_commit(&a_empty[b]);
+        }
+        if (ok) umma_commit(&d_full);
+      }
+    }
+  } else if (warp < 2 + kTsConvWarps) {
+    // ------------------------------------------------------------------ converters
+    const int cw = warp - 2;
+    const int q = warp & 3;          // TMEM lane quarter this warp may access
+    const int part = cw >> 2;        // which chunks of the k-block this warp converts
+    const int r = 32 * q + lane;     // channel within the tile
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      const int nt = tile / a.m_tiles;
+      const bool row_ok = nt * kTsBN + r < a.N;
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
+        const int s = it % kTsStages, b = it % kTsABufs;
+        if (ok && !mbar_wait(&full_bar[s], (it / kTsStages) & 1)) ok = false;
+        if (ok && it >= kTsABufs && !mbar_wait(&a_empty[b], ((it / kTsABufs) & 1) ^ 1)) ok = false;
+        tc_fence_after();
+        const uint8_t* st = ring + (size_t)s * kTsStageBytes;
+        // this thread's chunks of the block (32 k, 16 pairs each)
+#pragma unroll
+        for (int j = 0; j < kTsChunksPerConv; ++j) {
+          const int ci = part * kTsChunksPerConv + j;  // chunk 0..3 of the block
+          const int kc = ci * 32;                      // its first k within the block
+          uint32_t o[16];
+          if (ok && row_ok && kb * kTsBK + kc < a.K) {
+            if (LUT) {
+              const uint8_t* tile = st + kTsOffC + (ci >> 1) * (kTsBN * 24);  // LUT tile kb*2 + ci/2
+              const uint32_t* w = reinterpret_cast<const uint32_t*>(tile + r * 24 + (ci & 1) * 12);
+              const uint32_t wa = w[0], wb = w[1], wc = w[2];
+              const uint4 tab = lds128(smem_u32(st + kTsOffM + (ci >> 1) * 256 + (r >> 3) * 16));
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                uint32_t p[4];
+                lut3_decode8(lut3_selector(t < 2 ? wa : wb, wc, t), tab, p);
+                o[4 * t + 0] = p[0]; o[4 * t + 1] = p[1]; o[4 * t + 2] = p[2]; o[4 * t + 3] = p[3];
+              }
+            } else {
+              const int gl = kc / a.group;  // group of the chunk among the block's groups
+              const uint16_t sbits = *reinterpret_cast<const uint16_t*>(st + kTsOffM + (gl * 128 + r) * 2);
+              const int z = ASYM ? (int)*reinterpret_cast<const int8_t*>(st + kTsOffM + 1024 + gl * 128 + r) : 8;
+              uint32_t c1, c2;
+              zero_consts<BF16>(z, c1, c2);
+              const uint32_t s2 = scale_pair<BF16>(sbits);
+              const uint4 wv = lds128(smem_u32(st + kTsOffC + r * 64 + kc / 2));
+              const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+              constexpr uint32_t magic = BF16 ? 0x43004300u : 0x64006400u;
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const uint32_t pq = and_or(wd[q4] >> (4 * e), 0x000F000Fu, magic);
+                  o[4 * q4 + e] = BF16 ? bmul2_u32(bsub2_u32(pq, c1), s2) : hmul2_u32(hsub2_u32(pq, c1), s2);
+                }
+              }
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = 0u;
+          }
+          tmem_st16(lane_base + kTsColA + (uint32_t)b * 64 + (uint32_t)(kc / 2), o);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0 && ok) {
+          mbar_arrive(&a_full[b]);
+          mbar_arrive(&empty_bar[s]);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int r = 32 * q + lane;  // channel within the tile
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+    int t_iter = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++t_iter) {
+      const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;
+      if (!mbar_wait(&d_full, t_iter & 1)) break;
+      tc_fence_after();
+      const int n = nt * kTsBN + r;
+#pragma unroll 1
+      for (int j = 0; j < kTsBM / 32; ++j) {
+        uint32_t v[32];
+        tmem_ld32(lane_base + kTsColD + (uint32_t)(j * 32), v);
+        const int m0 = mt * kTsBM + j * 32;
+        if (n < a.N) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (m0 + i < a.M) store_out(a.Y, (size_t)(m0 + i) * a.N + n, __uint_as_float(v[i]), a.y_bf16);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&d_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(512u) : "memory");
+  }
+}
+
+}  // namespace lbq

@@ -26,6 +26,7 @@
 #include "gemm_tc.cuh"
 #include "tc_gemv.cuh"
 #include "gemv_direct.cuh"
+#include "gemm_ts.cuh"
 
 namespace lbq {
 
@@ -518,6 +519,46 @@ static GemvScratch gemv_scratch(int M, int K, int N, int group, bool asym, bool 
 // ----------------------------------------------------------------------------
 
 static int g_force_tc = 0;  // test hook: route every lbq_gemm call to the tcgen05 kernel
+// test hook: prefill kernel. 0 = weights in tensor memory (A operand), 1 = the
+// kernel with the weights dequantised into shared memory (B operand).
+static int g_gemm_path = 0;
+
+typedef void (*TsKernel)(CUtensorMap, CUtensorMap, GemmTsArgs);
+
+// Prefill GEMM with the weights as the A operand in tensor memory (INT4 or LUT3).
+static lbq_status run_gemm_ts(const void* X, bool xbf16, int M, const void* image, const Layout& L, void* Y,
+                              bool ybf16, cudaStream_t st) {
+  const bool lut = L.mode == LBQ_MODE_LUT3, asym = L.mode == LBQ_MODE_ASYM;
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  CUtensorMap tx, tq;
+  if (!make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)L.K, (uint64_t)M, (uint64_t)L.K * 2, 64,
+                    kTsBM, CU_TENSOR_MAP_SWIZZLE_128B))
+    return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the prefill activations");
+  tq = tx;
+  if (!lut && !make_tmap_2d(&tq, img + L.off0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.K / 2, (uint64_t)L.N,
+                            (uint64_t)L.K / 2, kTsBK / 2, kTsBN, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the prefill codes");
+  GemmTsArgs a{};
+  a.Y = Y;
+  a.meta0 = lut ? img + L.off0 : img + L.off1;
+  a.meta1 = lut ? img + L.off3 : (asym ? img + L.off2 : nullptr);
+  a.M = M; a.N = L.N; a.K = L.K;
+  a.group = lut ? 64 : L.group;
+  a.G = L.K / a.group;
+  a.n_tiles = (L.N + kTsBN - 1) / kTsBN;
+  a.m_tiles = (M + kTsBM - 1) / kTsBM;
+  a.k_blocks = (L.K + kTsBK - 1) / kTsBK;
+  a.y_bf16 = ybf16 ? 1 : 0;
+  TsKernel fn;
+  if (lut) fn = gemm_ts_kernel<true, false, true>;
+  else if (xbf16) fn = asym ? gemm_ts_kernel<true, true, false> : gemm_ts_kernel<true, false, false>;
+  else fn = asym ? gemm_ts_kernel<false, true, false> : gemm_ts_kernel<false, false, false>;
+  occupancy_for((const void*)fn, kTsThreads, kTsSmem);
+  const int grid = std::min(a.n_tiles * a.m_tiles, num_sms());
+  void* args[] = {&tx, &tq, &a};
+  return launch_kernel_ex((const void*)fn, dim3(grid), dim3(kTsThreads), kTsSmem, st, false, args,
+                          "prefill GEMM launch");
+}
 
 static lbq_status run_gemm_tc(const void* X, bool xbf16, int M, const void* image, const Layout& L, void* Y,
                               bool ybf16, cudaStream_t st) {
@@ -692,6 +733,10 @@ void lbq_debug_force_tc(int on) { g_force_tc = on ? 1 : 0; }
 // Test hook (not in the public header): route M = 1 through the skinny kernel.
 void lbq_debug_force_skinny(int on) { g_force_skinny = on ? 1 : 0; }
 
+// Test hook (not in the public header): pick the prefill kernel (0 = weights in
+// tensor memory, 1 = weights dequantised into shared memory).
+void lbq_debug_gemm_path(int path) { g_gemm_path = path == 1 ? 1 : 0; }
+
 // Test hook (not in the public header): pick the GEMV kernel for M <= 16
 // (0 = the library's choice, 1 = TMA-pipelined CUDA-core M = 1, 2 = warp MMA,
 // 3 = tcgen05, 4 = direct-load CUDA-core M = 1).
@@ -810,6 +855,9 @@ lbq_status lbq_gemm(const void* X, int x_dtype, int M, int K, int N, int group, 
   lbq_status st = check_int4_shape(K, N, group, mode);
   if (st != LBQ_OK) return st;
   if ((st = check_compute_args(X, x_dtype, M, image, Y, y_dtype)) != LBQ_OK) return st;
+  if (g_gemm_path == 0)
+    return run_gemm_ts(X, x_dtype == LBQ_DTYPE_BF16, M, image, make_layout(K, N, group, mode), Y,
+                       y_dtype == LBQ_DTYPE_BF16, static_cast<cudaStream_t>(stream));
   return run_gemm_tc(X, x_dtype == LBQ_DTYPE_BF16, M, image, make_layout(K, N, group, mode), Y,
                      y_dtype == LBQ_DTYPE_BF16, static_cast<cudaStream_t>(stream));
 }
@@ -823,6 +871,7 @@ lbq_status lbq_lut3_gemm(const void* X, int x_dtype, int M, int K, int N, const 
   const Layout L = make_layout(K, N, 0, LBQ_MODE_LUT3);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (M <= 16 && !g_force_tc) return run_lut3_skinny(X, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, ws, ws_bytes, s);
+  if (g_gemm_path == 0) return run_gemm_ts(X, true, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);
   return run_lut3_gemm_tc(X, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);
 }
 

@@ -35,15 +35,20 @@ GEMM_SHAPES = [
 
 
 @pytest.mark.parametrize("M,K,N,group,mode,xdt", GEMM_SHAPES)
-def test_gemm_parity(torch, lbq, M, K, N, group, mode, xdt):
+@pytest.mark.parametrize("path", [0, 1])  # 0: weights in tensor memory, 1: weights in shared memory
+def test_gemm_parity(torch, lbq, M, K, N, group, mode, xdt, path):
     W = workloads.weights_host(500 + K + N, K, N)
     ref = oracle_int4(W, group, mode)
     img = lbq.pack(torch.from_numpy(W).cuda(), group, mode)
     X = workloads.activations_host(500 + M, M, K, xdt)
-    for ydt in ("bf16", "f16"):
-        Y = lbq.gemm(X.cuda(), img, N, group, mode, y_dtype=ydt)
-        torch.cuda.synchronize()
-        check_outputs(Y.cpu(), X, ref["deq"])
+    lbq.lbq_debug_gemm_path(path)
+    try:
+        for ydt in ("bf16", "f16"):
+            Y = lbq.gemm(X.cuda(), img, N, group, mode, y_dtype=ydt)
+            torch.cuda.synchronize()
+            check_outputs(Y.cpu(), X, ref["deq"])
+    finally:
+        lbq.lbq_debug_gemm_path(0)
     lbq.device_status()
 
 

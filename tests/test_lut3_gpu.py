@@ -119,11 +119,16 @@ def test_lut3_gemv_parity(torch, lbq, M, K, N):
 
 @pytest.mark.parametrize("M", [17, 130, 300])
 @pytest.mark.parametrize("K,N", [(1024, 512), (320, 264), (4096, 1032)])
-def test_lut3_gemm_parity(torch, lbq, M, K, N):
+@pytest.mark.parametrize("path", [0, 1])  # 0: weights in tensor memory, 1: weights in shared memory
+def test_lut3_gemm_parity(torch, lbq, M, K, N, path):
     idx, cb, ex = _inputs(90 + K + N, K, N)
     img = _image(torch, lbq, idx, cb, ex)
     X = workloads.activations_host(90 + M, M, K, "bf16")
-    _check_gemm(torch, lbq, idx, cb, ex, img, X, y_dtype="bf16")
+    lbq.lbq_debug_gemm_path(path)
+    try:
+        _check_gemm(torch, lbq, idx, cb, ex, img, X, y_dtype="bf16")
+    finally:
+        lbq.lbq_debug_gemm_path(0)
     lbq.device_status()
 
 
