@@ -27,6 +27,7 @@
 #include "tc_gemv.cuh"
 #include "gemv_direct.cuh"
 #include "gemm_ts.cuh"
+#include "lut3_direct.cuh"
 
 namespace lbq {
 
@@ -635,6 +636,33 @@ static lbq_status run_lut3_skinny(const void* X, int M, const void* image, const
   return launch_kernel_ex(fn, dim3(p.grid), dim3(kSkThreads), p.smem, st, g_pdl != 0, args, "lut3 skinny launch");
 }
 
+// LUT3, M = 1, direct loads (no workspace).
+static bool lut3_direct_ok(int M, int K) { return M == 1 && K / 64 <= 32 * kLdMaxWarps && g_gemv_path != kPathMma; }
+
+static lbq_status run_lut3_direct(const void* X, const void* image, const Layout& L, void* Y, bool ybf16,
+                                  cudaStream_t st) {
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  Lut3DirectArgs a{};
+  a.X = static_cast<const uint16_t*>(X);
+  a.Y = Y;
+  a.i_region = img + L.off0;
+  a.t_region = img + L.off3;
+  a.K = L.K; a.N = L.N;
+  a.row_blocks = L.N / 8;
+  a.y_bf16 = ybf16 ? 1 : 0;
+  const int nw = (L.K / 64 + 31) / 32;
+  const void* fn = (const void*)lut3_direct_kernel;
+  const int occ = std::max(1, occupancy_for(fn, nw * 32, 0));
+  int grid = std::min(a.row_blocks, num_sms() * occ);
+  int smem = ((a.row_blocks + grid - 1) / grid) * nw * 8 * (int)sizeof(float);
+  while (smem > 96 * 1024 && grid < a.row_blocks) {
+    grid = std::min(a.row_blocks, grid * 2);
+    smem = ((a.row_blocks + grid - 1) / grid) * nw * 8 * (int)sizeof(float);
+  }
+  void* args[] = {&a};
+  return launch_kernel_ex(fn, dim3(grid), dim3(nw * 32), smem, st, g_pdl != 0, args, "LUT3 direct GEMV launch");
+}
+
 static lbq_status run_lut3_gemm_tc(const void* X, int M, const void* image, const Layout& L, void* Y, bool ybf16,
                                    cudaStream_t st) {
   const uint8_t* img = static_cast<const uint8_t*>(image);
@@ -823,7 +851,7 @@ lbq_status lbq_workspace_size(int op, int M, int K, int N, int group, int mode, 
     lbq_status st = check_lut3_shape(K, N);
     if (st != LBQ_OK) return st;
     if (M <= 0) return fail(LBQ_ERR_INVALID_ARG, "M must be positive");
-    if (M <= 16 && !g_force_tc) *bytes = skinny_workspace_bytes(plan_lut3(K, N, M), M);
+    if (M <= 16 && !g_force_tc && !lut3_direct_ok(M, K)) *bytes = skinny_workspace_bytes(plan_lut3(K, N, M), M);
     return LBQ_OK;
   }
   return fail(LBQ_ERR_INVALID_ARG, "op %d not in {0, 1, 2}", op);
@@ -870,6 +898,7 @@ lbq_status lbq_lut3_gemm(const void* X, int x_dtype, int M, int K, int N, const 
   if (x_dtype != LBQ_DTYPE_BF16) return fail(LBQ_ERR_UNSUPPORTED, "LUT3 kernels take BF16 activations");
   const Layout L = make_layout(K, N, 0, LBQ_MODE_LUT3);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (lut3_direct_ok(M, K) && !g_force_tc) return run_lut3_direct(X, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);
   if (M <= 16 && !g_force_tc) return run_lut3_skinny(X, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, ws, ws_bytes, s);
   if (g_gemm_path == 0) return run_gemm_ts(X, true, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);
   return run_lut3_gemm_tc(X, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);

@@ -108,12 +108,17 @@ SKINNY_SHAPES = [
 
 @pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16])
 @pytest.mark.parametrize("K,N", SKINNY_SHAPES)
-def test_lut3_gemv_parity(torch, lbq, M, K, N):
+@pytest.mark.parametrize("path", [0, 2])  # 0: library's choice (direct loads at M = 1), 2: warp-MMA kernel
+def test_lut3_gemv_parity(torch, lbq, M, K, N, path):
     idx, cb, ex = _inputs(70 + K + N, K, N)
     img = _image(torch, lbq, idx, cb, ex)
     X = workloads.activations_host(70 + M, M, K, "bf16")
-    for ydt in ("bf16", "f16"):
-        _check_gemm(torch, lbq, idx, cb, ex, img, X, y_dtype=ydt)
+    lbq.lbq_debug_gemv_path(path)
+    try:
+        for ydt in ("bf16", "f16"):
+            _check_gemm(torch, lbq, idx, cb, ex, img, X, y_dtype=ydt)
+    finally:
+        lbq.lbq_debug_gemv_path(0)
     lbq.device_status()
 
 
