@@ -163,45 +163,71 @@ def physical_gpu_index(local):
 # ----------------------------------------------------------------------------- the decode step
 
 class DecodeStep:
-    """224 asym INT4 g32 GEMVs (32 layers x 7 projections), images resident in HBM."""
+    """224 asym INT4 g32 GEMVs (32 layers x 7 projections), images resident in HBM.
 
-    def __init__(self, torch, lbq, workloads, device, layers):
+    As in a decoder layer, q, k and v read one activation vector and gate and
+    up another; with grouped=True each of those sets is one lbq_gemv_grouped
+    launch (4 launches per layer), otherwise every projection is its own
+    lbq_gemv call (7 per layer)."""
+
+    # projection groups sharing X: (q, k, v), (o), (gate, up), (down)
+    GROUPS = ((0, 1, 2), (3,), (4, 5), (6,))
+
+    def __init__(self, torch, lbq, workloads, device, layers, grouped=True):
         self.torch = torch
-        self.projs = []
+        self.lbq = lbq
+        self.grouped = grouped
         self.bytes = 0
-        x_len = sum(K for _ in range(layers) for (_, K, _) in workloads.LLAMA3_8B_PROJ)
-        y_len = sum(N for _ in range(layers) for (_, _, N) in workloads.LLAMA3_8B_PROJ)
+        self.calls = []  # per launch: list of (K, N, img, x, y, ws)
+        proj = workloads.LLAMA3_8B_PROJ
+        x_len = layers * sum(proj[g[0]][1] for g in self.GROUPS)
+        y_len = layers * sum(N for (_, _, N) in proj)
         self.x_all = torch.empty(x_len, dtype=torch.float16, device=device)
         self.y_all = torch.empty(y_len, dtype=torch.float16, device=device)
+        self.n_gemvs = layers * len(proj)
         xo = yo = 0
         # one workspace per (K, N): a workspace is reused only by calls of one
         # shape, whose tile counters sit at the same place every time
         self.ws = {}
         for layer in range(layers):
-            for p, (name, K, N) in enumerate(workloads.LLAMA3_8B_PROJ):
-                seed = workloads.c2_seed(layer, p)
-                W = workloads.weights_device(seed, K, N, device)
-                img = lbq.pack(W, 32, "asym")
-                del W
+            for grp in self.GROUPS:
+                K = proj[grp[0]][1]
                 x = self.x_all[xo:xo + K].view(1, K)
-                x.copy_(workloads.activations_device(seed, 1, K, "f16", device))
-                y = self.y_all[yo:yo + N].view(1, N)
+                x.copy_(workloads.activations_device(workloads.c2_seed(layer, grp[0]), 1, K, "f16", device))
                 xo += K
-                yo += N
-                if (K, N) not in self.ws:
-                    self.ws[(K, N)] = torch.zeros(max(lbq.lbq_workspace_size(0, 1, K, N, 32, 1), 256),
-                                                  dtype=torch.uint8, device=device)
-                self.projs.append((K, N, img, x, y, self.ws[(K, N)]))
-                self.bytes += int4_bytes(K, N, 32, "asym")
-        self.lbq = lbq
+                members = []
+                for p in grp:
+                    _, Kp, N = proj[p]
+                    W = workloads.weights_device(workloads.c2_seed(layer, p), Kp, N, device)
+                    img = lbq.pack(W, 32, "asym")
+                    del W
+                    y = self.y_all[yo:yo + N].view(1, N)
+                    yo += N
+                    if (Kp, N) not in self.ws:
+                        self.ws[(Kp, N)] = torch.zeros(max(lbq.lbq_workspace_size(0, 1, Kp, N, 32, 1), 256),
+                                                       dtype=torch.uint8, device=device)
+                    members.append((Kp, N, img, x, y, self.ws[(Kp, N)]))
+                    self.bytes += int4_bytes(Kp, N, 32, "asym")
+                if grouped and len(members) > 1:
+                    items = lbq.make_gemv_items([(x.data_ptr(), img.data_ptr(), y.data_ptr(), N)
+                                                 for (_, N, img, x, y, _) in members])
+                    self.calls.append(("grouped", K, items, len(members), members))
+                else:
+                    for m in members:
+                        self.calls.append(("single",) + m)
         torch.cuda.synchronize()
 
     def launch_all(self):
         lbq = self.lbq
         stream = self.torch.cuda.current_stream().cuda_stream
-        for K, N, img, x, y, ws in self.projs:
-            lbq.lbq_gemv(x.data_ptr(), 0, 1, K, N, 32, 1, img.data_ptr(), y.data_ptr(), 0,
-                         ws.data_ptr(), ws.numel(), stream)
+        for c in self.calls:
+            if c[0] == "grouped":
+                _, K, items, n, _members = c
+                lbq.lbq_gemv_grouped(items, n, K, 32, 1, 0, 0, stream)
+            else:
+                _, K, N, img, x, y, ws = c
+                lbq.lbq_gemv(x.data_ptr(), 0, 1, K, N, 32, 1, img.data_ptr(), y.data_ptr(), 0,
+                             ws.data_ptr(), ws.numel(), stream)
 
     def capture(self):
         torch = self.torch
@@ -542,6 +568,8 @@ def main():
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch the decode-step GEMVs without programmatic dependent launch")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--ungrouped", action="store_true",
+                    help="one lbq_gemv launch per projection instead of grouped q/k/v and gate/up")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", default=None, choices=sorted(PROFILE_CASES),
                     help="run a small case for ncu (a few launches over weight copies larger than L2) and exit")
@@ -561,7 +589,7 @@ def main():
     device = torch.device("cuda", local)
     peaks = load_peaks()
 
-    step = DecodeStep(torch, lbq, workloads, device, args.layers)
+    step = DecodeStep(torch, lbq, workloads, device, args.layers, grouped=not args.ungrouped)
     # the step's weights are written once and then only read, so the GEMVs may
     # overlap their weight streaming with the previous kernel's tail
     lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 0 if args.no_pdl else 1)
@@ -580,7 +608,7 @@ def main():
     value = world * step.bytes / (ms_per_step / 1e3) / 1e9
 
     # end to end through the public C-ABI call: every step copies its
-    # activations in from pinned host memory, makes the 224 lbq_gemv calls
+    # activations in from pinned host memory, makes the step's C-ABI calls
     # (no graph) and copies the outputs back to pinned host memory
     x_host = torch.empty_like(step.x_all, device="cpu").pin_memory()
     x_host.copy_(step.x_all.cpu())
@@ -624,9 +652,12 @@ def main():
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": {"workload": "c2: Llama-3-8B-shaped decode step at M=1, 7 projections x %d layers, asymmetric "
+        "config": {"workload": "Llama-3-8B-shaped decode step at M=1, 7 projections x %d layers, asymmetric "
                                "INT4 group 32 (fp16 scale + int8 zp), fp16 X, fp16 Y" % args.layers,
-                   "weight_bytes_per_step": step.bytes, "gemvs_per_step": len(step.projs),
+                   "weight_bytes_per_step": step.bytes, "gemvs_per_step": step.n_gemvs,
+                   "launches_per_step": step.launches_per_step,
+                   "grouping": "q/k/v and gate/up share X and run as one grouped launch each"
+                               if step.grouped else "one launch per projection",
                    "l2": "inputs larger than L2 (%.2f GB of weights per step vs %d MB L2); no flush"
                          % (step.bytes / 1e9, torch.cuda.get_device_properties(device).L2_cache_size >> 20),
                    "timing": "CUDA events around K replays of one CUDA graph holding the step",
@@ -636,7 +667,7 @@ def main():
         "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": hbm, "unit": "GB/s", "frac": per_gpu / hbm,
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peaks["source"],
                      "traffic": traffic,
-                     "kernel": "gemv_m1_kernel (every launch of the step)",
+                     "kernel": "gemv_direct_kernel (every launch of the step)",
                      "per_launch": "algorithmic bytes per launch averaged over the step's %d launches (%.0f B) / "
                                    "average launch time (step time / launches); traffic = ncu DRAM read+write "
                                    "bytes per launch, averaged the same way, null if the kernel source changed "
@@ -646,7 +677,8 @@ def main():
         "e2e": {"value": world * step.bytes / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": step.x_all.numel() * 2, "d2h_bytes_per_step": step.y_all.numel() * 2,
                 "ms_per_step": e2e_ms, "kernel_launches": e2e_launches,
-                "how": "per step: pinned host X -> device, 224 lbq_gemv C-ABI calls (no graph), device Y -> "
+                "how": "per step: pinned host X -> device, the step's lbq_gemv / lbq_gemv_grouped C-ABI calls "
+                       "(no graph), device Y -> "
                        "pinned host; CUDA events on the launching stream"},
         "gpu_launches": launches * args.steps,
         "cpu_baseline": cpu,

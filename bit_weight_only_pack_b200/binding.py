@@ -39,6 +39,11 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 _c_int, _c_size, _vp, _u64 = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_uint64
 
+class lbq_gemv_item(ctypes.Structure):
+    """One GEMV of lbq_gemv_grouped (include/lbq.h)."""
+    _fields_ = [("X", ctypes.c_void_p), ("image", ctypes.c_void_p), ("Y", ctypes.c_void_p), ("N", ctypes.c_int)]
+
+
 _SIGS = {
     "lbq_last_error": ([], ctypes.c_char_p),
     "lbq_version": ([], _c_int),
@@ -56,6 +61,7 @@ _SIGS = {
     "lbq_device_status": ([_vp], _c_int),
     "lbq_set_option": ([_c_int, _c_int], _c_int),
     "lbq_gemv_noalloc": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp], _c_int),
+    "lbq_gemv_grouped": ([ctypes.POINTER(lbq_gemv_item), _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp], _c_int),
     "lbq_debug_force_splits": ([_c_int], None),
     "lbq_debug_force_skinny": ([_c_int], None),
     "lbq_debug_force_tc": ([_c_int], None),
@@ -136,6 +142,19 @@ def lbq_dequant(image, K, N, group, mode, W_out, stream):
 
 def lbq_device_status(stream):
     _check(_lib.lbq_device_status(stream))
+
+
+def lbq_gemv_grouped(items, count, K, group, mode, x_dtype, y_dtype, stream):
+    """items: a ctypes array of lbq_gemv_item (host memory)."""
+    _check(_lib.lbq_gemv_grouped(items, count, K, group, mode, x_dtype, y_dtype, stream))
+
+
+def make_gemv_items(triples):
+    """[(X ptr, image ptr, Y ptr, N), ...] -> ctypes array for lbq_gemv_grouped."""
+    arr = (lbq_gemv_item * len(triples))()
+    for i, (x, img, y, n) in enumerate(triples):
+        arr[i] = lbq_gemv_item(x, img, y, n)
+    return arr
 
 
 def lbq_gemv_noalloc(X, x_dtype, M, K, N, group, mode, image, Y, y_dtype, stream):
@@ -301,6 +320,25 @@ def dequant(image, K, N, group, mode):
     W = torch.empty((K, N), dtype=torch.float32, device=image.device)
     lbq_dequant(image.data_ptr(), K, N, group, _mode(mode), W.data_ptr(), _stream())
     return W
+
+
+def gemv_grouped(problems, group, mode, y_dtype=None):
+    """Batch-1 GEMVs in one launch. problems: [(X [1, K], image, N), ...] with a
+    common K; returns the list of Y [1, N]."""
+    torch = _torch()
+    K = problems[0][0].shape[1]
+    Ys = []
+    rows = []
+    for X, img, N in problems:
+        _need_cuda(X, img)
+        if X.shape != (1, K) or X.dtype != problems[0][0].dtype:
+            raise ValueError("grouped GEMVs need X [1, K] of one K and dtype")
+        Y = _out(X, N, y_dtype)
+        Ys.append(Y)
+        rows.append((X.data_ptr(), img.data_ptr(), Y.data_ptr(), N))
+    lbq_gemv_grouped(make_gemv_items(rows), len(rows), K, group, _mode(mode), _dt(problems[0][0]), _dt(Ys[0]),
+                     _stream())
+    return Ys
 
 
 def gemv_noalloc(X, image, N, group, mode, y_dtype=None, Y=None):

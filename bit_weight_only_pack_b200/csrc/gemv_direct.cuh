@@ -9,7 +9,11 @@
 //  * A CTA owns blocks of 8 output rows (grid-stride) and the whole K range;
 //    lane l of warp w takes the 32-k chunk c = 32w + l (K <= 16384). Its
 //    activations (32 values per chunk) and their offset sums stay in registers
-//    for all the CTA's row blocks.
+//    while the CTA's row blocks use the same X.
+//  * One launch may carry up to 4 GEMVs with the same K, group, mode and
+//    dtypes (the projections that read one activation vector, e.g. q/k/v or
+//    gate/up of a decoder layer): their row blocks are numbered one after the
+//    other and spread over the same grid.
 //  * Per row block and chunk a lane loads the 8 rows' 16-byte code chunks,
 //    one 16-byte load of the 8 rows' scales and one 8-byte load of their zero
 //    points (the image stores them 128 channels at a time, so 8 consecutive
@@ -31,15 +35,21 @@
 namespace lbq {
 
 constexpr int kGdMaxWarps = 16;
+constexpr int kGdMaxItems = 4;  // GEMVs of one launch (same K, group, mode and dtypes)
 
+// One launch computes up to kGdMaxItems GEMVs; their 8-row blocks are numbered
+// consecutively, item i owning blocks [rb_end[i-1], rb_end[i]).
 struct GemvDirectArgs {
-  const uint16_t* X;       // [K] FP16/BF16 bits
-  void* Y;                 // [N]
-  const uint8_t* q;        // [N][K/2]
-  const uint8_t* s;        // 128-channel-tiled FP16 scales
-  const uint8_t* z;        // 128-channel-tiled int8 zero points (ASYM)
-  int K, N, G;
-  int row_blocks;          // ceil(N / 8)
+  const uint16_t* X[kGdMaxItems];  // [K] FP16/BF16 bits
+  void* Y[kGdMaxItems];            // [N]
+  const uint8_t* q[kGdMaxItems];   // [N][K/2]
+  const uint8_t* s[kGdMaxItems];   // 128-channel-tiled FP16 scales
+  const uint8_t* z[kGdMaxItems];   // 128-channel-tiled int8 zero points (ASYM)
+  int N[kGdMaxItems];
+  int rb_end[kGdMaxItems];
+  int items;
+  int K, G;
+  int row_blocks;                  // total over the items
   int y_bf16;
 };
 
@@ -51,36 +61,30 @@ __device__ __forceinline__ float gd_chunk(const uint4 w, const uint32_t (&x)[16]
 // float [row blocks of this CTA][warps][8] of per-warp row sums.
 template <bool BF16, bool ASYM>
 __global__ void __launch_bounds__(kGdMaxWarps * 32, 1) gemv_direct_kernel(const GemvDirectArgs a) {
-  constexpr int J = 1;
   extern __shared__ float red[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nw = blockDim.x >> 5;
   const int chunks = a.K >> 5;
   const size_t rowb = (size_t)(a.K >> 1);  // code bytes per row
   const int gpc = (a.K / a.G) >> 5;        // chunks per group (1, 2 or 4)
+  const int c = warp * 32 + lane;          // this lane's 32-k chunk
+  const bool cok = c < chunks;
 
-  // this lane's chunks and their activations (read once for all row blocks)
-  uint32_t xr[J][16];
-  float xoff[J], xsum[J];
-  int cidx[J];
-  bool cok[J];
-#pragma unroll
-  for (int j = 0; j < J; ++j) {
-    cidx[j] = warp * 32 + lane + j * nw * 32;
-    cok[j] = cidx[j] < chunks;
-  }
-
+  auto item_of = [&](int rb) {
+    int i = 0;
+    while (i + 1 < a.items && rb >= a.rb_end[i]) ++i;
+    return i;
+  };
   // codes of the current and the next row block
-  uint4 cur[J][8], nxt[J][8];
-  auto load_block = [&](int rb, uint4 (&w)[J][8]) {
-    const int r0 = rb * 8;
+  uint4 cur[8], nxt[8];
+  auto load_block = [&](int rb, uint4 (&w)[8]) {
+    const int it = item_of(rb);
+    const int r0 = (rb - (it ? a.rb_end[it - 1] : 0)) * 8;
 #pragma unroll
-    for (int j = 0; j < J; ++j)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        w[j][i] = make_uint4(0u, 0u, 0u, 0u);
-        if (cok[j] && r0 + i < a.N) w[j][i] = ld_stream_v4(a.q + (size_t)(r0 + i) * rowb + (size_t)cidx[j] * 16);
-      }
+    for (int i = 0; i < 8; ++i) {
+      w[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (cok && r0 + i < a.N[it]) w[i] = ld_stream_v4(a.q[it] + (size_t)(r0 + i) * rowb + (size_t)c * 16);
+    }
   };
 
   // The weights are only read, so the first row block is requested before
@@ -89,60 +93,63 @@ __global__ void __launch_bounds__(kGdMaxWarps * 32, 1) gemv_direct_kernel(const 
   if (rb < a.row_blocks) load_block(rb, cur);
   griddep_launch_dependents();
   griddep_wait();
-#pragma unroll
-  for (int j = 0; j < J; ++j) {
-    const int c = cidx[j];
+
+  // this lane's activations and their offset sums, for the item being worked on
+  uint32_t xr[16];
+  float xoff = 0.0f, xsum = 0.0f;
+  const uint16_t* x_loaded = nullptr;
+  auto load_x = [&](const uint16_t* X) {
+    x_loaded = X;
     float sA = 0.0f, sB = 0.0f;
-    if (cok[j]) {
-      const uint4* xp = reinterpret_cast<const uint4*>(a.X + (size_t)c * 32);
+    if (cok) {
+      const uint4* xp = reinterpret_cast<const uint4*>(X + (size_t)c * 32);
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
         const uint4 u = ld_nc_v4(xp + v);
-        xr[j][4 * v + 0] = u.x; xr[j][4 * v + 1] = u.y; xr[j][4 * v + 2] = u.z; xr[j][4 * v + 3] = u.w;
+        xr[4 * v + 0] = u.x; xr[4 * v + 1] = u.y; xr[4 * v + 2] = u.z; xr[4 * v + 3] = u.w;
       }
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float lo = x2f<BF16>((uint16_t)(xr[j][i] & 0xFFFFu));
-        const float hi = x2f<BF16>((uint16_t)(xr[j][i] >> 16));
+        const float lo = x2f<BF16>((uint16_t)(xr[i] & 0xFFFFu));
+        const float hi = x2f<BF16>((uint16_t)(xr[i] >> 16));
         if ((i & 1) == 0) sA += lo + hi; else sB += lo + hi;
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) xr[j][i] = 0u;
+      for (int i = 0; i < 16; ++i) xr[i] = 0u;
     }
-    const float xs = sA + sB;
-    xsum[j] = xs;
+    xsum = sA + sB;
     // FP16: slots of class A carry 1024 + q, class B (1024 + 16 q)/16 after chunk_acc
-    xoff[j] = (BF16 ? 128.0f * xs : 1024.0f * sA + 64.0f * sB) + (ASYM ? 0.0f : 8.0f * xs);
-  }
+    xoff = (BF16 ? 128.0f * xsum : 1024.0f * sA + 64.0f * sB) + (ASYM ? 0.0f : 8.0f * xsum);
+  };
 
   int lb = 0;  // row block index within this CTA
   for (; rb < a.row_blocks; rb += gridDim.x, ++lb) {
     const int rbn = rb + gridDim.x;
     if (rbn < a.row_blocks) load_block(rbn, nxt);
-    const int r0 = rb * 8;
+    const int it = item_of(rb);
+    if (a.X[it] != x_loaded) load_x(a.X[it]);
+    const int r0 = (rb - (it ? a.rb_end[it - 1] : 0)) * 8;
     float part[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) part[i] = 0.0f;
-#pragma unroll
-    for (int j = 0; j < J; ++j) {
-      if (!cok[j]) continue;
-      const int g = cidx[j] / gpc;
+    if (cok) {
+      const int g = c / gpc;
       const size_t m0 = ((size_t)(r0 >> 7) * a.G + g) * 128 + (r0 & 127);  // 8 consecutive rows, 16-byte aligned
-      const uint4 sv = ld_nc_v4(a.s + m0 * 2);
+      const uint4 sv = ld_nc_v4(a.s[it] + m0 * 2);
       uint2 zv = make_uint2(0u, 0u);
-      if (ASYM) zv = *reinterpret_cast<const uint2*>(a.z + m0);
+      if (ASYM) zv = *reinterpret_cast<const uint2*>(a.z[it] + m0);
       const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
       for (int i = 0; i < 8; i += 2) {
         const float2 sc = __half22float2(*reinterpret_cast<const __half2*>(&sw[i >> 1]));
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const float acc = gd_chunk<BF16>(cur[j][i + h], xr[j]);
-          float corr = xoff[j];
+          const float acc = gd_chunk<BF16>(cur[i + h], xr);
+          float corr = xoff;
           if (ASYM) {
             const int zi = (int)(int8_t)(((i < 4 ? zv.x : zv.y) >> (8 * ((i + h) & 3))) & 0xFFu);
-            corr = fmaf((float)zi, xsum[j], corr);
+            corr = fmaf((float)zi, xsum, corr);
           }
           part[i + h] = fmaf(h ? sc.y : sc.x, acc - corr, part[i + h]);
         }
@@ -151,18 +158,18 @@ __global__ void __launch_bounds__(kGdMaxWarps * 32, 1) gemv_direct_kernel(const 
     const float total = butterfly8(part, lane);
     if ((lane & 3) == 0) red[(lb * nw + warp) * 8 + butterfly8_row(lane)] = total;
 #pragma unroll
-    for (int j = 0; j < J; ++j)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) cur[j][i] = nxt[j][i];
+    for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
   }
   // the warps' row sums of every row block of this CTA, added in warp order
   __syncthreads();
   for (int t = tid; t < lb * 8; t += blockDim.x) {
     const int l = t >> 3, row = t & 7;
-    const int r = (blockIdx.x + l * gridDim.x) * 8 + row;
+    const int rbo = blockIdx.x + l * gridDim.x;
+    const int it = item_of(rbo);
+    const int r = (rbo - (it ? a.rb_end[it - 1] : 0)) * 8 + row;
     float sum = 0.0f;
     for (int w = 0; w < nw; ++w) sum += red[(l * nw + w) * 8 + row];
-    if (r < a.N) store_out(a.Y, (size_t)r, sum, a.y_bf16);
+    if (r < a.N[it]) store_out(a.Y[it], (size_t)r, sum, a.y_bf16);
   }
 }
 

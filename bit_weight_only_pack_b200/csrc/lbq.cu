@@ -440,27 +440,37 @@ static lbq_status run_tcgemv(const void* X, bool xbf16, int M, const void* image
                           "tcgen05 GEMV launch");
 }
 
-// M = 1, direct loads (no workspace).
-static lbq_status run_direct(const uint16_t* X, bool xbf16, const void* image, const Layout& L, void* Y, bool ybf16,
+// M = 1, direct loads (no workspace): `count` GEMVs of the same K / group /
+// mode / dtypes in one launch.
+static lbq_status run_direct(const lbq_gemv_item* items, int count, int K, int group, int mode, bool xbf16, bool ybf16,
                              cudaStream_t st) {
-  const bool asym = L.mode == LBQ_MODE_ASYM;
-  const int chunks = L.K / 32;
+  const bool asym = mode == LBQ_MODE_ASYM;
+  const int chunks = K / 32;
   const int nw = (chunks + 31) / 32;
   if (nw > kGdMaxWarps) return fail(LBQ_ERR_UNSUPPORTED, "direct GEMV needs K <= %d", 32 * 32 * kGdMaxWarps);
-  const uint8_t* img = static_cast<const uint8_t*>(image);
+  if (count < 1 || count > kGdMaxItems) return fail(LBQ_ERR_INVALID_ARG, "count=%d not in 1..%d", count, kGdMaxItems);
   GemvDirectArgs a{};
-  a.X = X;
-  a.Y = Y;
-  a.q = img + L.off0;
-  a.s = img + L.off1;
-  a.z = asym ? img + L.off2 : nullptr;
-  a.K = L.K; a.N = L.N; a.G = L.K / L.group;
-  a.row_blocks = (L.N + 7) / 8;
+  int rbs = 0;
+  for (int i = 0; i < count; ++i) {
+    const Layout L = make_layout(K, items[i].N, group, mode);
+    const uint8_t* img = static_cast<const uint8_t*>(items[i].image);
+    a.X[i] = static_cast<const uint16_t*>(items[i].X);
+    a.Y[i] = items[i].Y;
+    a.q[i] = img + L.off0;
+    a.s[i] = img + L.off1;
+    a.z[i] = asym ? img + L.off2 : nullptr;
+    a.N[i] = items[i].N;
+    rbs += (items[i].N + 7) / 8;
+    a.rb_end[i] = rbs;
+  }
+  a.items = count;
+  a.K = K; a.G = K / group;
+  a.row_blocks = rbs;
   a.y_bf16 = ybf16 ? 1 : 0;
   const void* fn = xbf16 ? (asym ? (const void*)gemv_direct_kernel<true, true> : (const void*)gemv_direct_kernel<true, false>)
                          : (asym ? (const void*)gemv_direct_kernel<false, true> : (const void*)gemv_direct_kernel<false, false>);
   // one wave of CTAs; each keeps 8 floats per warp per row block in shared memory
-  int occ = std::max(1, occupancy_for(fn, nw * 32, 0));
+  const int occ = std::max(1, occupancy_for(fn, nw * 32, 0));
   int grid = std::min(a.row_blocks, num_sms() * occ);
   int smem = ((a.row_blocks + grid - 1) / grid) * nw * 8 * (int)sizeof(float);
   while (smem > 96 * 1024 && grid < a.row_blocks) {  // very tall matrices: more CTAs, fewer blocks each
@@ -866,9 +876,10 @@ lbq_status lbq_gemv(const void* X, int x_dtype, int M, int K, int N, int group, 
   const Layout L = make_layout(K, N, group, mode);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int path = gemv_path(M, K, (long long)K * N);
-  if (path == kPathDirect)
-    return run_direct(static_cast<const uint16_t*>(X), x_dtype == LBQ_DTYPE_BF16, image, L, Y,
-                      y_dtype == LBQ_DTYPE_BF16, s);
+  if (path == kPathDirect) {
+    const lbq_gemv_item item{X, image, Y, N};
+    return run_direct(&item, 1, K, group, mode, x_dtype == LBQ_DTYPE_BF16, y_dtype == LBQ_DTYPE_BF16, s);
+  }
   if (path == kPathM1)
     return run_m1(static_cast<const uint16_t*>(X), x_dtype == LBQ_DTYPE_BF16, image, L, Y, y_dtype == LBQ_DTYPE_BF16,
                   ws, ws_bytes, s);
@@ -971,6 +982,20 @@ lbq_status lbq_device_status(void* stream) {
   if (v == 0) return LBQ_OK;
   if ((st = cuda_check(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)), "clearing the device flag")) != LBQ_OK) return st;
   return fail(LBQ_ERR_DEVICE, "a kernel reported device error flags 0x%x", v);
+}
+
+lbq_status lbq_gemv_grouped(const lbq_gemv_item* items, int count, int K, int group, int mode, int x_dtype,
+                            int y_dtype, void* stream) {
+  if (!items) return fail(LBQ_ERR_INVALID_ARG, "items must be non-null");
+  if (count < 1 || count > kGdMaxItems) return fail(LBQ_ERR_INVALID_ARG, "count=%d not in 1..%d", count, kGdMaxItems);
+  if (K > 32 * 32 * kGdMaxWarps) return fail(LBQ_ERR_UNSUPPORTED, "lbq_gemv_grouped needs K <= %d", 32 * 32 * kGdMaxWarps);
+  for (int i = 0; i < count; ++i) {
+    lbq_status st = check_int4_shape(K, items[i].N, group, mode);
+    if (st != LBQ_OK) return st;
+    if ((st = check_compute_args(items[i].X, x_dtype, 1, items[i].image, items[i].Y, y_dtype)) != LBQ_OK) return st;
+  }
+  return run_direct(items, count, K, group, mode, x_dtype == LBQ_DTYPE_BF16, y_dtype == LBQ_DTYPE_BF16,
+                    static_cast<cudaStream_t>(stream));
 }
 
 lbq_status lbq_gemv_noalloc(const void* X, int x_dtype, int M, int K, int N, int group, int mode, const void* image,

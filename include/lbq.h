@@ -133,6 +133,25 @@ lbq_status lbq_gemv(const void* X, int x_dtype, int M, int K, int N, int group, 
                     void* stream);
 
 /*
+ * Several batch-1 INT4 GEMVs in one launch, e.g. the projections of a decoder
+ * layer that read the same activation vector (q, k, v; gate, up). Item i:
+ *   X      (device) [1, K], x_dtype
+ *   image  (device) from lbq_pack with K, items[i].N, group, mode
+ *   Y      (device) [1, items[i].N], y_dtype, fully overwritten
+ * items is a host array of 1..4 entries; all share K (<= 16384), group, mode
+ * and the dtypes. No workspace. The result of each item equals that of
+ * lbq_gemv with M = 1 on it. Asynchronous on `stream`.
+ */
+typedef struct {
+  const void* X;
+  const void* image;
+  void* Y;
+  int N;
+} lbq_gemv_item;
+lbq_status lbq_gemv_grouped(const lbq_gemv_item* items, int count, int K, int group, int mode,
+                            int x_dtype, int y_dtype, void* stream);
+
+/*
  * Prefill GEMM on INT4 weights, any M >= 1 (M <= 16 is routed to lbq_gemv's
  * kernels). Same arguments and result as lbq_gemv. Weights are dequantised
  * to BF16 in shared memory and multiplied on the tensor cores; X must be BF16

@@ -271,3 +271,35 @@ def test_m1_through_the_skinny_kernel(torch, lbq):
     finally:
         lbq.lbq_debug_force_skinny(0)
     check_outputs(Y.cpu(), X, ref["deq"])
+
+
+@pytest.mark.parametrize("shared_x", [True, False])
+@pytest.mark.parametrize("xdt,mode,group", [("f16", "asym", 32), ("bf16", "sym", 128)])
+def test_gemv_grouped_matches_single_calls(torch, lbq, shared_x, xdt, mode, group):
+    """Three GEMVs in one launch (q/k/v-like widths, one ragged): each output
+    equals the single-GEMV output bit for bit and passes the oracle check."""
+    K, Ns = 1024, (512, 128, 72)
+    Ws = [workloads.weights_host(950 + i, K, N) for i, N in enumerate(Ns)]
+    refs = [oracle_int4(W, group, mode) for W in Ws]
+    imgs = [lbq.pack(torch.from_numpy(W).cuda(), group, mode) for W in Ws]
+    Xs = [workloads.activations_host(960 + (0 if shared_x else i), 1, K, xdt) for i in range(len(Ns))]
+    Xd = [X.cuda() for X in Xs]
+    Ys = lbq.gemv_grouped([(Xd[i], imgs[i], N) for i, N in enumerate(Ns)], group, mode)
+    singles = [lbq.gemv(Xd[i], imgs[i], N, group, mode) for i, N in enumerate(Ns)]
+    torch.cuda.synchronize()
+    lbq.device_status()
+    for i in range(len(Ns)):
+        assert torch.equal(Ys[i], singles[i])
+        check_outputs(Ys[i].cpu(), Xs[i], refs[i]["deq"])
+
+
+def test_gemv_grouped_rejects_bad_groups(torch, lbq):
+    W = workloads.weights_host(970, 256, 64)
+    img = lbq.pack(torch.from_numpy(W).cuda(), 32, "sym")
+    X = workloads.activations_host(970, 1, 256, "f16").cuda()
+    with pytest.raises(lbq.LbqError):
+        lbq.gemv_grouped([(X, img, 64)] * 5, 32, "sym")   # more than 4 items
+    Y = torch.empty((1, 64), dtype=torch.float16, device="cuda")
+    items = lbq.make_gemv_items([(X.data_ptr(), img.data_ptr(), Y.data_ptr(), 64)])
+    with pytest.raises(lbq.LbqError):
+        lbq.lbq_gemv_grouped(items, 1, 32768, 32, 0, 0, 0, None)  # K beyond the direct kernel
