@@ -489,16 +489,19 @@ def run_reference(args):
 
 # ----------------------------------------------------------------------------- ncu cases
 
-# name -> (K, N, group, mode, x dtype, M); a "_tc" suffix routes M = 1 through the tensor-core kernel
+# name -> (K, N, group, mode, x dtype, M, GEMV path or None); the path is the
+# test hook's kernel choice (1 TMA CUDA-core, 2 warp MMA, 3 tcgen05, 4 direct)
 PROFILE_CASES = {
-    "c1": (4096, 4096, 32, "sym", "f16", 1),
-    "c2gate": (4096, 14336, 32, "asym", "f16", 1),
-    "c2gate_tc": (4096, 14336, 32, "asym", "f16", 1),
-    "c4m2048": (4096, 14336, 128, "asym", "bf16", 2048),
-    "c2down": (14336, 4096, 32, "asym", "f16", 1),
-    "c2kv": (4096, 1024, 32, "asym", "f16", 1),
-    "c3m1": (8192, 28672, 128, "sym", "bf16", 1),
-    "c3m16": (8192, 28672, 128, "sym", "bf16", 16),
+    "c1": (4096, 4096, 32, "sym", "f16", 1, None),
+    "c2gate": (4096, 14336, 32, "asym", "f16", 1, None),
+    "c2down": (14336, 4096, 32, "asym", "f16", 1, None),
+    "c2kv": (4096, 1024, 32, "asym", "f16", 1, None),
+    "c2gate_mma": (4096, 14336, 32, "asym", "f16", 1, 2),
+    "c3m1": (8192, 28672, 128, "sym", "bf16", 1, None),
+    "c3m16": (8192, 28672, 128, "sym", "bf16", 16, None),
+    "c4m2048": (4096, 14336, 128, "asym", "bf16", 2048, None),
+    "c5m1": (4096, 14336, 0, "lut3", "bf16", 1, None),
+    "c5m2048": (4096, 14336, 0, "lut3", "bf16", 2048, None),
 }
 
 
@@ -508,25 +511,34 @@ def run_profile_case(name):
     import torch
     import bit_weight_only_pack_b200 as lbq
     import workloads
-    K, N, group, mode, xdt, M = PROFILE_CASES[name]
+    K, N, group, mode, xdt, M, path = PROFILE_CASES[name]
     device = torch.device("cuda", 0)
     torch.cuda.set_device(0)
-    W = workloads.weights_device(7, K, N, device)
-    img0 = lbq.pack(W, group, mode)
-    del W
+    if mode == "lut3":
+        idx, cb, ex = workloads.lut3_device(7, K, N, device)
+        img0 = lbq.pack_lut3(idx, cb, ex)
+        del idx, cb, ex
+    else:
+        W = workloads.weights_device(7, K, N, device)
+        img0 = lbq.pack(W, group, mode)
+        del W
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    copies = max(3, (3 * l2) // img0.numel() + 1)
-    images = [img0] + [img0.clone() for _ in range(copies - 1)]
+    images = weight_copies(img0, l2)
     X = workloads.activations_device(7, M, K, xdt, device)
-    if name.endswith("_tc"):
-        lbq.lbq_debug_force_skinny(1)
-    ws = lbq.workspace(0, M, K, N, group, mode)
-    for img in images:
-        lbq.gemm(X, img, N, group, mode, ws=ws)
+    if path is not None:
+        lbq.lbq_debug_gemv_path(path)
+    if mode == "lut3":
+        ws = lbq.workspace(2, M, K, N, 0, "lut3")
+        for img in images:
+            lbq.lut3_gemm(X, img, N, ws=ws)
+    else:
+        ws = lbq.workspace(0, M, K, N, group, mode)
+        for img in images:
+            lbq.gemm(X, img, N, group, mode, ws=ws)
     torch.cuda.synchronize()
-    lbq.lbq_debug_force_skinny(0)
+    lbq.lbq_debug_gemv_path(0)
     lbq.device_status()
-    print(f"profile case {name}: {copies} launches of K={K} N={N} g={group} {mode} M={M}", flush=True)
+    print(f"profile case {name}: {len(images)} launches of K={K} N={N} {mode} M={M}", flush=True)
     return 0
 
 
