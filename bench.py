@@ -547,7 +547,12 @@ def run_profile_case(name):
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) from ncu captures
 # summarised under profiles/, with a hash of the kernel sources at capture time:
 # name -> (bytes, {source file: sha256[:16]}, summary file).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # mean DRAM bytes per gemv_direct_kernel launch of the decode step
+    "decode_step_per_launch": (32422922, {"gemv_direct.cuh": "4aad9b641ebb822e", "gemv_m1.cuh": "36b10f852f538832",
+                                          "common.cuh": "57fbadb552e32665"},
+                               "profiles/decode_step_launch_list.md"),
+}
 
 
 def source_hash(name):
@@ -657,9 +662,8 @@ def main():
     hbm = peaks["hbm_gbs"]
     per_gpu = step.bytes / (ms_per_step / 1e3) / 1e9
     launches = step.launches_per_step
-    # DRAM bytes of one step's launches from an ncu capture (see profiles/), per launch on average
-    traffic_step = traffic_from_profiles("decode_step_per_layer")
-    traffic = traffic_step * args.layers / launches if traffic_step is not None else None
+    # DRAM bytes per launch of the step from an ncu capture (see profiles/), for the default step only
+    traffic = traffic_from_profiles("decode_step_per_launch") if (args.layers == 32 and not args.ungrouped) else None
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
