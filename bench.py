@@ -549,7 +549,7 @@ def run_profile_case(name):
 # name -> (bytes, {source file: sha256[:16]}, summary file).
 NCU_TRAFFIC = {
     # mean DRAM bytes per gemv_direct_kernel launch of the decode step
-    "decode_step_per_launch": (32422922, {"gemv_direct.cuh": "4aad9b641ebb822e", "gemv_m1.cuh": "36b10f852f538832",
+    "decode_step_per_launch": (32422922, {"gemv_direct.cuh": "4aad9b641ebb822e", "gemv_m1.cuh": "a992f85dd1acbd76",
                                           "common.cuh": "57fbadb552e32665"},
                                "profiles/decode_step_launch_list.md"),
 }

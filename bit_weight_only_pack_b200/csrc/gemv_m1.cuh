@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kM1MaxConsumerThreads + 32, 2) gemv_m1_kernel(
 
   griddep_wait();  // X may be written by the previous kernel in the stream
 
-  for (int tile = blockIdx.x; tile < a.total_tiles && !timed_out; tile += gridDim.x) {
+  for (int tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x) {
     const int split = tile / a.row_tiles;
     const int rt = tile - split * a.row_tiles;
 
@@ -256,7 +256,10 @@ __global__ void __launch_bounds__(kM1MaxConsumerThreads + 32, 2) gemv_m1_kernel(
 #pragma unroll
     for (int st = 0; st < 8 / RPT; ++st, ++it) {
       const int slot = it % a.stages;
-      if (!mbar_wait(&full_bar[slot], (it / a.stages) & 1)) { timed_out = true; break; }
+      // after a timed-out wait the warp skips its work but keeps the same
+      // sequence of consumer barriers as the other warps
+      if (!timed_out && !mbar_wait(&full_bar[slot], (it / a.stages) & 1)) timed_out = true;
+      if (timed_out) continue;
       const uint32_t sb = smem_u32(ring + (size_t)slot * a.slot_bytes);
       const uint32_t zrow = (uint32_t)((rt * rows_per_tile + st * R) & 8);  // 8-row half of the 16-row zp box
 #pragma unroll
@@ -281,7 +284,6 @@ __global__ void __launch_bounds__(kM1MaxConsumerThreads + 32, 2) gemv_m1_kernel(
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[slot]);
     }
-    if (timed_out) break;
 
     const float total = butterfly8(part, lane);
     if ((lane & 3) == 0) red[buf][warp][butterfly8_row(lane)] = total;
@@ -294,7 +296,7 @@ __global__ void __launch_bounds__(kM1MaxConsumerThreads + 32, 2) gemv_m1_kernel(
       float sum = 0.0f;
       for (int w = w0; w < w1; ++w) sum += red[buf][w][idx];
       const int n = row0 + tid;
-      if (n < a.N) {
+      if (n < a.N && !timed_out) {
         if (a.splits == 1) store_out(a.Y, n, sum, a.y_bf16);
         else a.partials[(size_t)split * a.N + n] = sum;
       }
@@ -303,8 +305,8 @@ __global__ void __launch_bounds__(kM1MaxConsumerThreads + 32, 2) gemv_m1_kernel(
       __threadfence();
       consumer_sync(nthreads_c);
       if (tid == 0) {
-        const unsigned int prev = atomicAdd(&a.counters[rt], 1u);
-        s_last = (prev == (unsigned int)(a.splits - 1));
+        s_last = 0u;
+        if (!timed_out) s_last = (atomicAdd(&a.counters[rt], 1u) == (unsigned int)(a.splits - 1));
       }
       consumer_sync(nthreads_c);
       if (s_last) {

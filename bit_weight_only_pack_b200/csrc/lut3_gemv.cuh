@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(kSkThreads, 2) lut3_skinny_kernel(const __grid
   int it = 0;
   bool ok = true;
   long long u = u_begin;
-  while (u < u_end && ok) {
+  while (u < u_end) {
     const int rt = (int)(u / S_t);
     const int st0 = (int)(u - (long long)rt * S_t);
     const int st1 = (int)min((long long)S_t, st0 + (u_end - u));
@@ -150,7 +150,10 @@ __global__ void __launch_bounds__(kSkThreads, 2) lut3_skinny_kernel(const __grid
 
     for (int st = st0; st < st1; ++st, ++it) {
       const int slot = it % kL3Stages;
-      if (!mbar_wait(&full_bar[slot], (it / kL3Stages) & 1)) { ok = false; break; }
+      // after a timed-out wait the warp skips its work but keeps the same
+      // sequence of named barriers as the other consumer warps
+      if (ok && !mbar_wait(&full_bar[slot], (it / kL3Stages) & 1)) ok = false;
+      if (!ok) continue;
       const uint8_t* sp = ring + (size_t)slot * kSlot;
       const int ntile = min(4, K / 64 - st * 4);
 #pragma unroll
@@ -184,7 +187,6 @@ __global__ void __launch_bounds__(kSkThreads, 2) lut3_skinny_kernel(const __grid
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[slot]);
     }
-    if (!ok) break;
 
     const int n0 = rt * kSkRows + lrow;
     const bool whole = (st0 == 0 && st1 == S_t);
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(kSkThreads, 2) lut3_skinny_kernel(const __grid
         for (int i = 0; i < 4; ++i) {
           const int m = 8 * n + 2 * t + (i & 1);
           const int nn = n0 + ((i & 2) ? 8 : 0);
-          if (m < M && nn < N) store_out(a.Y, (size_t)m * N + nn, acc[n][i], a.y_bf16);
+          if (ok && m < M && nn < N) store_out(a.Y, (size_t)m * N + nn, acc[n][i], a.y_bf16);
         }
     } else {
       const long long tile_u0 = (long long)rt * S_t;
@@ -208,14 +210,17 @@ __global__ void __launch_bounds__(kSkThreads, 2) lut3_skinny_kernel(const __grid
         for (int i = 0; i < 4; ++i) {
           const int m = 8 * n + 2 * t + (i & 1);
           const int r = lrow + ((i & 2) ? 8 : 0);
-          if (m < M) base[((size_t)slot_id * M + m) * kSkRows + r] = acc[n][i];
+          if (ok && m < M) base[((size_t)slot_id * M + m) * kSkRows + r] = acc[n][i];
         }
       __threadfence();
       asm volatile("bar.sync 1, %0;" :: "r"(kSkWarps * 32) : "memory");
       if (tid == 0) {
-        const unsigned int add = (unsigned int)(st1 - st0);
-        const unsigned int prev = atomicAdd(&a.counters[rt], add);
-        s_last = (prev + add == (unsigned int)S_t);
+        s_last = 0u;
+        if (ok) {
+          const unsigned int add = (unsigned int)(st1 - st0);
+          const unsigned int prev = atomicAdd(&a.counters[rt], add);
+          s_last = (prev + add == (unsigned int)S_t);
+        }
       }
       asm volatile("bar.sync 1, %0;" :: "r"(kSkWarps * 32) : "memory");
       if (s_last) {

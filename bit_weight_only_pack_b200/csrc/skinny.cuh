@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
   int it = 0;
   bool ok = true;
   long long u = u_begin;
-  while (u < u_end && ok) {
+  while (u < u_end) {
     const int rt = (int)(u / S_t);
     const int st0 = (int)(u - (long long)rt * S_t);
     const int st1 = (int)min((long long)S_t, st0 + (u_end - u));
@@ -259,7 +259,10 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
 
     for (int st = st0; st < st1; ++st, ++it) {
       const int slot = it % kSkStages;
-      if (!mbar_wait(&full_bar[slot], (it / kSkStages) & 1)) { ok = false; break; }
+      // after a timed-out wait the warp skips its work but keeps the same
+      // sequence of named barriers as the other consumer warps
+      if (ok && !mbar_wait(&full_bar[slot], (it / kSkStages) & 1)) ok = false;
+      if (!ok) continue;
       const uint8_t* sp = ring + (size_t)slot * kSlot;
       const uint32_t sb = smem_u32(sp);
       const int k0 = st * 256;
@@ -331,7 +334,6 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[slot]);
     }
-    if (!ok) break;
 
     // ---------------------------------------------------------------- output
     const int n0 = rt * kSkRows + lrow;
@@ -343,7 +345,7 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
         for (int i = 0; i < 4; ++i) {
           const int m = 8 * n + 2 * t + (i & 1);
           const int nn = n0 + ((i & 2) ? 8 : 0);
-          if (m < M && nn < a.N) store_out(a.Y, (size_t)m * a.N + nn, acc[n][i], a.y_bf16);
+          if (ok && m < M && nn < a.N) store_out(a.Y, (size_t)m * a.N + nn, acc[n][i], a.y_bf16);
         }
     } else {
       const long long tile_u0 = (long long)rt * S_t;
@@ -356,14 +358,17 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
         for (int i = 0; i < 4; ++i) {
           const int m = 8 * n + 2 * t + (i & 1);
           const int r = lrow + ((i & 2) ? 8 : 0);
-          if (m < M) base[((size_t)slot_id * M + m) * kSkRows + r] = acc[n][i];
+          if (ok && m < M) base[((size_t)slot_id * M + m) * kSkRows + r] = acc[n][i];
         }
       __threadfence();
       asm volatile("bar.sync 1, %0;" :: "r"(kSkWarps * 32) : "memory");
       if (tid == 0) {
-        const unsigned int add = (unsigned int)(st1 - st0);
-        const unsigned int prev = atomicAdd(&a.counters[rt], add);
-        s_last = (prev + add == (unsigned int)S_t);
+        s_last = 0u;
+        if (ok) {
+          const unsigned int add = (unsigned int)(st1 - st0);
+          const unsigned int prev = atomicAdd(&a.counters[rt], add);
+          s_last = (prev + add == (unsigned int)S_t);
+        }
       }
       asm volatile("bar.sync 1, %0;" :: "r"(kSkWarps * 32) : "memory");
       if (s_last) {
