@@ -303,3 +303,41 @@ def test_gemv_grouped_rejects_bad_groups(torch, lbq):
     items = lbq.make_gemv_items([(X.data_ptr(), img.data_ptr(), Y.data_ptr(), 64)])
     with pytest.raises(lbq.LbqError):
         lbq.lbq_gemv_grouped(items, 1, 32768, 32, 0, 0, 0, None)  # K beyond the direct kernel
+
+
+@pytest.mark.parametrize("K,N,group,mode", [
+    (16384, 9, 32, "sym"),       # the longest K the direct kernel takes, one partial row block
+    (16416, 200, 32, "asym"),    # one chunk past it: the TMA batch-1 kernel
+    (28672, 136, 128, "asym"),   # long K (a 70B-class down projection), ragged N
+    (4096, 3, 128, "asym"),      # fewer columns than one row block
+])
+@pytest.mark.parametrize("xdt", ["f16", "bf16"])
+def test_m1_dispatch_boundaries(torch, lbq, K, N, group, mode, xdt):
+    """Batch 1 through the library's own kernel choice on both sides of the
+    K limit of the direct kernel, every column."""
+    W = _special_groups(workloads.weights_host(90 + K + N, K, N), group)
+    img, ref = _pack_and_compare(torch, lbq, W, group, mode)
+    X = workloads.activations_host(90 + K, 1, K, xdt)
+    for ydt in ("f16", "bf16"):
+        Y = lbq.gemv(X.cuda(), img, N, group, mode, y_dtype=ydt)
+        torch.cuda.synchronize()
+        check_outputs(Y.cpu(), X, ref["deq"])
+    lbq.device_status()
+
+
+def test_m1_long_k_many_weights_sampled(torch, lbq):
+    """K=16512, N=8200: past the direct kernel's K limit and over 2^27 weights,
+    where batch 1 goes to the warp-MMA kernel; sampled columns."""
+    K, N, group = 16512, 8200, 128
+    W = workloads.weights_host(31, K, N)
+    Wd = torch.from_numpy(W).cuda()
+    img = lbq.pack(Wd, group, "asym")
+    del Wd
+    cols = sample_columns(N, 256, seed=31)
+    ref = oracle_int4(np.ascontiguousarray(W[:, cols]), group, "asym")
+    del W
+    X = workloads.activations_host(31, 1, K, "bf16")
+    Y = lbq.gemv(X.cuda(), img, N, group, "asym")
+    torch.cuda.synchronize()
+    check_outputs(Y.cpu(), X, ref["deq"], cols)
+    lbq.device_status()

@@ -180,3 +180,15 @@ def test_lut3_rejects_fp16_activations(torch, lbq):
     X = workloads.activations_host(99, 1, K, "f16").cuda()
     with pytest.raises(lbq.LbqError):
         lbq.lut3_gemm(X, img, N)
+
+
+@pytest.mark.parametrize("K,N", [(16384, 72), (16448, 40)])
+def test_lut3_m1_direct_kernel_k_limit(torch, lbq, K, N):
+    """Batch 1 at the longest K the direct LUT3 kernel takes (256 tiles) and
+    one tile past it (the warp-MMA kernel), every channel."""
+    idx, cb, ex = _inputs(60 + K, K, N)
+    img = _image(torch, lbq, idx, cb, ex)
+    X = workloads.activations_host(60 + K, 1, K, "bf16")
+    for ydt in ("bf16", "f16"):
+        _check_gemm(torch, lbq, idx, cb, ex, img, X, y_dtype=ydt)
+    lbq.device_status()
