@@ -548,9 +548,9 @@ def run_profile_case(name):
 # summarised under profiles/, with a hash of the kernel sources at capture time:
 # name -> (bytes, {source file: sha256[:16]}, summary file).
 NCU_TRAFFIC = {
-    # mean DRAM bytes per gemv_direct_kernel launch of the decode step
-    "decode_step_per_launch": (32422922, {"gemv_direct.cuh": "4aad9b641ebb822e", "gemv_m1.cuh": "a992f85dd1acbd76",
-                                          "common.cuh": "57fbadb552e32665"},
+    # mean DRAM bytes per launch of the decode step (all gemv_direct_async_kernel)
+    "decode_step_per_launch": (32428280, {"gemv_direct.cuh": "d619e61ab3b68780", "common.cuh": "84092f83f8c9f1ae",
+                                          "lbq.cu": "f96dbd717a90b246"},
                                "profiles/decode_step_launch_list.md"),
 }
 
@@ -568,6 +568,8 @@ def traffic_from_profiles(name):
     if rec is None:
         return None
     nbytes, sources, _summary = rec
+    if nbytes is None:
+        return None
     try:
         return nbytes if all(source_hash(f) == h for f, h in sources.items()) else None
     except OSError:
@@ -683,7 +685,7 @@ def main():
         "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": hbm, "unit": "GB/s", "frac": per_gpu / hbm,
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peaks["source"],
                      "traffic": traffic,
-                     "kernel": "gemv_direct_kernel (every launch of the step)",
+                     "kernel": "gemv_direct_async_kernel (every launch of the step)",
                      "per_launch": "algorithmic bytes per launch averaged over the step's %d launches (%.0f B) / "
                                    "average launch time (step time / launches); traffic = ncu DRAM read+write "
                                    "bytes per launch, averaged the same way, null if the kernel source changed "

@@ -67,6 +67,7 @@ _SIGS = {
     "lbq_debug_force_tc": ([_c_int], None),
     "lbq_debug_gemv_path": ([_c_int], None),
     "lbq_debug_gemm_path": ([_c_int], None),
+    "lbq_debug_direct_variant": ([_c_int, _c_int], None),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -179,6 +180,12 @@ def lbq_debug_force_tc(on):
 def lbq_debug_gemv_path(path):
     """Test hook: GEMV kernel for M <= 16 (0 auto, 1 CUDA-core M=1, 2 warp MMA, 3 tcgen05)."""
     _lib.lbq_debug_gemv_path(path)
+
+
+def lbq_debug_direct_variant(variant, ctas_per_sm=0):
+    """Test hook: batch-1 direct kernel variant (-1 library's choice, 0 registers, 2..4 staged copies,
+    1 / 5 tensor cores with exact / offset-form operands) and a CTAs-per-SM cap."""
+    _lib.lbq_debug_direct_variant(variant, ctas_per_sm)
 
 
 def lbq_debug_gemm_path(path):

@@ -173,4 +173,134 @@ __global__ void __launch_bounds__(kGdMaxWarps * 32, 1) gemv_direct_kernel(const 
   }
 }
 
+// The same GEMV with the weights staged through shared memory by per-thread
+// asynchronous copies: each lane keeps S row blocks of its chunk (8 rows of
+// codes, their scales and zero points) in flight in its own shared-memory
+// slots, so the bytes in flight per SM no longer depend on registers, and the
+// scale and zero-point reads are prefetched with the codes. A lane reads back
+// only what it copied itself, so a per-thread wait on its copy groups is the
+// only synchronisation. Dynamic shared memory: uint4 codes [S][8][T], uint4
+// scales [S][T], uint2 zero points [S][T] (T threads), then the row sums as in
+// gemv_direct_kernel.
+template <int S>
+constexpr int gd_stage_bytes_per_thread() { return S * (8 * 16 + 16 + 8); }
+
+template <bool BF16, bool ASYM, int S>
+__global__ void __launch_bounds__(kGdMaxWarps * 32) gemv_direct_async_kernel(const GemvDirectArgs a) {
+  extern __shared__ __align__(16) uint8_t gd_smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int T = blockDim.x, nw = T >> 5;
+  uint4* sq = reinterpret_cast<uint4*>(gd_smem);
+  uint4* ss = sq + S * 8 * T;
+  uint2* sz = reinterpret_cast<uint2*>(ss + S * T);
+  float* red = reinterpret_cast<float*>(sz + S * T);
+  const int chunks = a.K >> 5;
+  const size_t rowb = (size_t)(a.K >> 1);
+  const int gpc = (a.K / a.G) >> 5;
+  const int c = warp * 32 + lane;
+  const bool cok = c < chunks;
+
+  auto item_of = [&](int rb) {
+    int i = 0;
+    while (i + 1 < a.items && rb >= a.rb_end[i]) ++i;
+    return i;
+  };
+  // copy row block rb's codes, scales and zero points for this lane into stage st
+  auto issue = [&](int rb, int st) {
+    if (cok && rb < a.row_blocks) {
+      const int it = item_of(rb);
+      const int r0 = (rb - (it ? a.rb_end[it - 1] : 0)) * 8;
+      const uint8_t* qc = a.q[it] + (size_t)c * 16;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const bool ok = r0 + i < a.N[it];  // rows past N read nothing and stage zeros
+        cp_async16(&sq[(st * 8 + i) * T + tid], qc + (size_t)(ok ? r0 + i : 0) * rowb, ok ? 16 : 0);
+      }
+      const size_t m0 = ((size_t)(r0 >> 7) * a.G + c / gpc) * 128 + (r0 & 127);
+      cp_async16(&ss[st * T + tid], a.s[it] + m0 * 2, 16);
+      if (ASYM) cp_async8(&sz[st * T + tid], a.z[it] + m0);
+    }
+    cp_async_commit();  // one group per stage, empty or not, keeps the wait count fixed
+  };
+
+  int rb = blockIdx.x;
+  // the weights are only read: the first S row blocks are requested before
+  // waiting for the previous kernel in the stream
+#pragma unroll
+  for (int st = 0; st < S; ++st) issue(rb + st * (int)gridDim.x, st);
+  griddep_launch_dependents();
+  griddep_wait();
+
+  uint32_t xr[16];
+  float xoff = 0.0f, xsum = 0.0f;
+  const uint16_t* x_loaded = nullptr;
+  auto load_x = [&](const uint16_t* X) {
+    x_loaded = X;
+    float sA = 0.0f, sB = 0.0f;
+    if (cok) {
+      const uint4* xp = reinterpret_cast<const uint4*>(X + (size_t)c * 32);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 u = ld_nc_v4(xp + v);
+        xr[4 * v + 0] = u.x; xr[4 * v + 1] = u.y; xr[4 * v + 2] = u.z; xr[4 * v + 3] = u.w;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float lo = x2f<BF16>((uint16_t)(xr[i] & 0xFFFFu));
+        const float hi = x2f<BF16>((uint16_t)(xr[i] >> 16));
+        if ((i & 1) == 0) sA += lo + hi; else sB += lo + hi;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) xr[i] = 0u;
+    }
+    xsum = sA + sB;
+    xoff = (BF16 ? 128.0f * xsum : 1024.0f * sA + 64.0f * sB) + (ASYM ? 0.0f : 8.0f * xsum);
+  };
+
+  int lb = 0, st = 0;
+  for (; rb < a.row_blocks; rb += gridDim.x, ++lb) {
+    cp_async_wait<S - 1>();  // this lane's copies of row block rb have landed
+    const int it = item_of(rb);
+    if (a.X[it] != x_loaded) load_x(a.X[it]);
+    float part[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) part[i] = 0.0f;
+    if (cok) {
+      const uint4 sv = ss[st * T + tid];
+      const uint2 zv = ASYM ? sz[st * T + tid] : make_uint2(0u, 0u);
+      const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        const float2 sc = __half22float2(*reinterpret_cast<const __half2*>(&sw[i >> 1]));
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float acc = gd_chunk<BF16>(sq[(st * 8 + i + h) * T + tid], xr);
+          float corr = xoff;
+          if (ASYM) {
+            const int zi = (int)(int8_t)(((i < 4 ? zv.x : zv.y) >> (8 * ((i + h) & 3))) & 0xFFu);
+            corr = fmaf((float)zi, xsum, corr);
+          }
+          part[i + h] = fmaf(h ? sc.y : sc.x, acc - corr, part[i + h]);
+        }
+      }
+    }
+    const float total = butterfly8(part, lane);
+    if ((lane & 3) == 0) red[(lb * nw + warp) * 8 + butterfly8_row(lane)] = total;
+    issue(rb + S * (int)gridDim.x, st);  // refill the stage just read
+    st = st + 1 == S ? 0 : st + 1;
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  for (int t = tid; t < lb * 8; t += blockDim.x) {
+    const int l = t >> 3, row = t & 7;
+    const int rbo = blockIdx.x + l * gridDim.x;
+    const int it = item_of(rbo);
+    const int r = (rbo - (it ? a.rb_end[it - 1] : 0)) * 8 + row;
+    float sum = 0.0f;
+    for (int w = 0; w < nw; ++w) sum += red[(l * nw + w) * 8 + row];
+    if (r < a.N[it]) store_out(a.Y[it], (size_t)r, sum, a.y_bf16);
+  }
+}
+
 }  // namespace lbq

@@ -341,3 +341,61 @@ def test_m1_long_k_many_weights_sampled(torch, lbq):
     torch.cuda.synchronize()
     check_outputs(Y.cpu(), X, ref["deq"], cols)
     lbq.device_status()
+
+
+class direct_variant:
+    """Route the batch-1 direct GEMV to one of its variants for a block (test hook):
+    0 = CUDA cores, weights pipelined through registers; 2..4 = CUDA cores with
+    that many row blocks staged through shared memory; 1 = multiply-adds on
+    the tensor cores with exact (q - z) operands, 5 = the same with
+    offset-form operands."""
+
+    def __init__(self, lbq, variant):
+        self.lbq, self.variant = lbq, variant
+
+    def __enter__(self):
+        self.lbq.lbq_debug_direct_variant(self.variant, 0)
+
+    def __exit__(self, *exc):
+        self.lbq.lbq_debug_direct_variant(-1, 0)
+
+
+@pytest.mark.parametrize("K,N,group,mode", SHAPES + [(14336, 136, 128, "asym"), (16384, 40, 64, "sym"),
+                                                     (1056, 24, 32, "asym"), (2080, 17, 32, "sym")])
+@pytest.mark.parametrize("xdt", ["f16", "bf16"])
+@pytest.mark.parametrize("variant", [0, 1, 2, 3, 5])
+def test_gemv_m1_direct_variants(torch, lbq, K, N, group, mode, xdt, variant):
+    W = _special_groups(workloads.weights_host(11 + K + N, K, N), group)
+    img, ref = _pack_and_compare(torch, lbq, W, group, mode)
+    X = workloads.activations_host(5 + K, 1, K, xdt)
+    with gemv_path(lbq, "direct_m1"), direct_variant(lbq, variant):
+        for ydt in ("f16", "bf16"):
+            Y = lbq.gemv(X.cuda(), img, N, group, mode, y_dtype=ydt)
+            torch.cuda.synchronize()
+            check_outputs(Y.cpu(), X, ref["deq"])
+    lbq.device_status()
+
+
+@pytest.mark.parametrize("variant", [0, 1, 2, 3, 5])
+@pytest.mark.parametrize("shared_x", [True, False])
+def test_gemv_grouped_direct_variants(torch, lbq, variant, shared_x):
+    """Grouped launches (distinct or shared X) on each direct-kernel variant
+    match single calls on the same variant bit for bit, and the oracle."""
+    K, group, mode = 4096, 32, "asym"
+    Ns = (4096, 1024, 1000)
+    imgs, refs = [], []
+    for i, N in enumerate(Ns):
+        W = workloads.weights_host(200 + i, K, N)
+        img, ref = _pack_and_compare(torch, lbq, W, group, mode)
+        imgs.append(img)
+        refs.append(ref)
+    Xs = [workloads.activations_host(300 + (0 if shared_x else i), 1, K, "f16") for i in range(len(Ns))]
+    Xd = [Xs[0].cuda()] * len(Ns) if shared_x else [X.cuda() for X in Xs]  # shared: one device vector
+    with direct_variant(lbq, variant):
+        singles = [lbq.gemv(X, img, N, group, mode) for X, img, N in zip(Xd, imgs, Ns)]
+        grouped = lbq.gemv_grouped([(X, img, N) for X, img, N in zip(Xd, imgs, Ns)], group, mode)
+        torch.cuda.synchronize()
+    for Ys, Yg, X, ref in zip(singles, grouped, Xs, refs):
+        assert torch.equal(Ys, Yg)
+        check_outputs(Yg.cpu(), X, ref["deq"])
+    lbq.device_status()
