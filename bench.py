@@ -328,6 +328,16 @@ GEMV_ALT_PATHS = (("tma_cudacore_m1_kernel", 1), ("direct_m1_kernel", 4), ("warp
 
 
 def secondary_measurements(torch, lbq, workloads, device, peaks, quick):
+    # GEMVs are launched as in the step, with programmatic dependent launch
+    # (the GEMMs never use it); weights rotate through copies larger than L2
+    lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 1)
+    try:
+        return _secondary_measurements(torch, lbq, workloads, device, peaks, quick)
+    finally:
+        lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 0)
+
+
+def _secondary_measurements(torch, lbq, workloads, device, peaks, quick):
     out = {}
     hbm = peaks["hbm_gbs"]
     l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size

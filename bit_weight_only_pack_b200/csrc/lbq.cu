@@ -752,6 +752,10 @@ static lbq_status run_lut3_skinny(const void* X, int M, const void* image, const
 // LUT3, M = 1, direct loads (no workspace).
 static bool lut3_direct_ok(int M, int K) { return M == 1 && K / 64 <= 32 * kLdMaxWarps && g_gemv_path != kPathMma; }
 
+// test hook: LUT3 batch-1 kernel (-1 = the library's choice, 0 = indices
+// pipelined through registers, 2 / 3 = staged through shared memory)
+static int g_lut3_stages = -1;
+
 static lbq_status run_lut3_direct(const void* X, const void* image, const Layout& L, void* Y, bool ybf16,
                                   cudaStream_t st) {
   const uint8_t* img = static_cast<const uint8_t*>(image);
@@ -764,16 +768,23 @@ static lbq_status run_lut3_direct(const void* X, const void* image, const Layout
   a.row_blocks = L.N / 8;
   a.y_bf16 = ybf16 ? 1 : 0;
   const int nw = (L.K / 64 + 31) / 32;
-  const void* fn = (const void*)lut3_direct_kernel;
-  const int occ = std::max(1, occupancy_for(fn, nw * 32, 0));
+  const int T = nw * 32;
+  int stages = g_lut3_stages < 0 ? 0 : g_lut3_stages;  // registers: staging measured slower here
+  while (stages >= 2 && (size_t)stages * 13 * T * 16 > 200 * 1024) --stages;
+  if (stages < 2) stages = 0;
+  const int stage_bytes = stages * 13 * T * 16;
+  const void* fn = stages == 0 ? (const void*)lut3_direct_kernel
+                 : stages == 2 ? (const void*)lut3_direct_async_kernel<2> : (const void*)lut3_direct_async_kernel<3>;
+  const int occ = std::max(1, occupancy_for(fn, T, stage_bytes + 1024));
   int grid = std::min(a.row_blocks, num_sms() * occ);
   int smem = ((a.row_blocks + grid - 1) / grid) * nw * 8 * (int)sizeof(float);
-  while (smem > 96 * 1024 && grid < a.row_blocks) {
+  while (smem > (stages ? 4096 : 96 * 1024) && grid < a.row_blocks) {
     grid = std::min(a.row_blocks, grid * 2);
     smem = ((a.row_blocks + grid - 1) / grid) * nw * 8 * (int)sizeof(float);
   }
+  smem += stage_bytes;
   void* args[] = {&a};
-  return launch_kernel_ex(fn, dim3(grid), dim3(nw * 32), smem, st, g_pdl != 0, args, "LUT3 direct GEMV launch");
+  return launch_kernel_ex(fn, dim3(grid), dim3(T), smem, st, g_pdl != 0, args, "LUT3 direct GEMV launch");
 }
 
 static lbq_status run_lut3_gemm_tc(const void* X, int M, const void* image, const Layout& L, void* Y, bool ybf16,
@@ -888,6 +899,11 @@ void lbq_debug_gemv_path(int path) { g_gemv_path = (path >= 0 && path <= 4) ? pa
 // 2..4 = staged through shared memory with that many row blocks in flight,
 // 1 = tensor-core kernel with exact (q - z) operands, 5 = tensor-core kernel
 // with offset-form operands) and a cap on resident CTAs per SM.
+// Test hook (not in the public header): LUT3 batch-1 kernel variant (-1 = the
+// library's choice, 0 = indices pipelined through registers, 2 / 3 = staged
+// through shared memory with that many row blocks in flight).
+void lbq_debug_lut3_variant(int variant) { g_lut3_stages = (variant == 0 || variant == 2 || variant == 3) ? variant : -1; }
+
 void lbq_debug_direct_variant(int variant, int ctas_per_sm) {
   g_direct_stages = (variant == 0 || (variant >= 2 && variant <= 4)) ? variant : -1;
   g_direct_ctas = ctas_per_sm > 0 ? ctas_per_sm : 0;

@@ -112,4 +112,100 @@ __global__ void __launch_bounds__(kLdMaxWarps * 32, 1) lut3_direct_kernel(const 
   }
 }
 
+// The same GEMV with each lane's indices and table staged through shared
+// memory by per-thread asynchronous copies, S row blocks ahead: the 208 bytes
+// per lane and block no longer sit in registers (251 -> under 100 per
+// thread), so more warps fit an SM and the loads run ahead of the decode.
+// A lane reads back only what it copied, so its own copy-group wait is the
+// only synchronisation. Dynamic shared memory: uint4 [S][13][T] (12 chunks of
+// indices, then the table), then the row sums as in lut3_direct_kernel.
+template <int S>
+__global__ void __launch_bounds__(kLdMaxWarps * 32) lut3_direct_async_kernel(const Lut3DirectArgs a) {
+  extern __shared__ __align__(16) uint8_t ld_smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int T = blockDim.x, nw = T >> 5;
+  const int kt = warp * 32 + lane;
+  const bool tok = kt < (a.K >> 6);
+  uint4* ring = reinterpret_cast<uint4*>(ld_smem);
+  float* red = reinterpret_cast<float*>(ring + (size_t)S * 13 * T);
+
+  auto issue = [&](int rb, int st) {
+    if (tok && rb < a.row_blocks) {
+      const uint8_t* base = a.i_region + ((size_t)kt * a.N + (size_t)rb * 8) * 24;
+#pragma unroll
+      for (int v = 0; v < 12; ++v) cp_async16(&ring[((size_t)st * 13 + v) * T + tid], base + 16 * v, 16);
+      cp_async16(&ring[((size_t)st * 13 + 12) * T + tid], a.t_region + ((size_t)kt * (a.N >> 3) + rb) * 16, 16);
+    }
+    cp_async_commit();  // one group per row block, empty or not, keeps the wait count fixed
+  };
+
+  int rb = blockIdx.x;
+  // the weights are only read: the first S row blocks are requested before
+  // waiting for the previous kernel in the stream
+#pragma unroll
+  for (int st = 0; st < S; ++st) issue(rb + st * (int)gridDim.x, st);
+  griddep_launch_dependents();
+  griddep_wait();
+  uint32_t xr[32];  // this tile's 64 activations as BF16 pairs
+  if (tok) {
+    const uint4* xp = reinterpret_cast<const uint4*>(a.X + (size_t)kt * 64);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const uint4 u = ld_nc_v4(xp + v);
+      xr[4 * v + 0] = u.x; xr[4 * v + 1] = u.y; xr[4 * v + 2] = u.z; xr[4 * v + 3] = u.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) xr[i] = 0u;
+  }
+
+  int lb = 0, st = 0;
+  for (; rb < a.row_blocks; rb += gridDim.x, ++lb) {
+    cp_async_wait<S - 1>();  // this lane's copies of row block rb have landed
+    float part[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) part[i] = 0.0f;
+    if (tok) {
+      const uint4 tab = ring[((size_t)st * 13 + 12) * T + tid];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        // row i's 24 bytes: words 6i .. 6i+5 of the staged 48
+        uint32_t wr[6];
+#pragma unroll
+        for (int e = 0; e < 6; ++e) {
+          const int wi = 6 * i + e;
+          const uint4 u = ring[((size_t)st * 13 + (wi >> 2)) * T + tid];
+          wr[e] = (wi & 3) == 0 ? u.x : (wi & 3) == 1 ? u.y : (wi & 3) == 2 ? u.z : u.w;
+        }
+        float acc = 0.0f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t wa = wr[3 * h], wb = wr[3 * h + 1], wc = wr[3 * h + 2];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            uint32_t p[4];
+            lut3_decode8(lut3_selector(t < 2 ? wa : wb, wc, t), tab, p);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc = fma2_bf16_f32(xr[16 * h + 4 * t + e], p[e], acc);
+          }
+        }
+        part[i] = acc;
+      }
+    }
+    const float total = butterfly8(part, lane);
+    if ((lane & 3) == 0) red[(lb * nw + warp) * 8 + butterfly8_row(lane)] = total;
+    issue(rb + S * (int)gridDim.x, st);  // refill the stage just read
+    st = st + 1 == S ? 0 : st + 1;
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  for (int t = tid; t < lb * 8; t += blockDim.x) {
+    const int l = t >> 3, row = t & 7;
+    const int r = (blockIdx.x + l * gridDim.x) * 8 + row;
+    float sum = 0.0f;
+    for (int w = 0; w < nw; ++w) sum += red[(l * nw + w) * 8 + row];
+    if (r < a.N) store_out(a.Y, (size_t)r, sum, a.y_bf16);
+  }
+}
+
 }  // namespace lbq
