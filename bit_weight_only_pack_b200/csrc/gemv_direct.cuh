@@ -190,35 +190,46 @@ __global__ void __launch_bounds__(kGdMaxWarps * 32) gemv_direct_async_kernel(con
   extern __shared__ __align__(16) uint8_t gd_smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = blockDim.x, nw = T >> 5;
-  uint4* sq = reinterpret_cast<uint4*>(gd_smem);
-  uint4* ss = sq + S * 8 * T;
-  uint2* sz = reinterpret_cast<uint2*>(ss + S * T);
-  float* red = reinterpret_cast<float*>(sz + S * T);
+  // 32-bit shared addresses of this thread's slots: codes [S][8][T] x 16 B,
+  // scales [S][T] x 16 B, zero points [S][T] x 8 B (lane-contiguous, so a
+  // warp's copies of one row fill 512 contiguous bytes)
+  const uint32_t T16 = (uint32_t)T * 16;
+  const uint32_t sq_s = (uint32_t)__cvta_generic_to_shared(gd_smem) + (uint32_t)tid * 16;
+  const uint32_t ss_s = sq_s + (uint32_t)S * 8 * T16;
+  const uint32_t sz_s = (uint32_t)__cvta_generic_to_shared(gd_smem) + (uint32_t)S * 9 * T16 + (uint32_t)tid * 8;
+  float* red = reinterpret_cast<float*>(gd_smem + (size_t)S * (9 * 16 + 8) * T);
   const int chunks = a.K >> 5;
   const size_t rowb = (size_t)(a.K >> 1);
   const int gpc = (a.K / a.G) >> 5;
   const int c = warp * 32 + lane;
   const bool cok = c < chunks;
+  const int gidx = cok ? c / gpc : 0;  // this lane's group
 
-  auto item_of = [&](int rb) {
-    int i = 0;
-    while (i + 1 < a.items && rb >= a.rb_end[i]) ++i;
-    return i;
+  // the two row-block cursors (copies, compute) only move forward, so each
+  // keeps its GEMV index
+  int it_copy = 0, it_comp = 0;
+  auto item_adv = [&](int& it, int rb) {
+    while (it + 1 < a.items && rb >= a.rb_end[it]) ++it;
   };
   // copy row block rb's codes, scales and zero points for this lane into stage st
   auto issue = [&](int rb, int st) {
     if (cok && rb < a.row_blocks) {
-      const int it = item_of(rb);
+      item_adv(it_copy, rb);
+      const int it = it_copy;
       const int r0 = (rb - (it ? a.rb_end[it - 1] : 0)) * 8;
-      const uint8_t* qc = a.q[it] + (size_t)c * 16;
+      const uint8_t* qc = a.q[it] + (size_t)r0 * rowb + (size_t)c * 16;
+      const uint32_t dst = sq_s + (uint32_t)st * 8 * T16;
+      const int nr = a.N[it] - r0;
+      if (nr >= 8) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const bool ok = r0 + i < a.N[it];  // rows past N read nothing and stage zeros
-        cp_async16(&sq[(st * 8 + i) * T + tid], qc + (size_t)(ok ? r0 + i : 0) * rowb, ok ? 16 : 0);
+        for (int i = 0; i < 8; ++i) cp_async16_s(dst + i * T16, qc + (size_t)i * rowb, 16);
+      } else {  // rows past N read nothing and stage zeros
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cp_async16_s(dst + i * T16, i < nr ? qc + (size_t)i * rowb : qc, i < nr ? 16 : 0);
       }
-      const size_t m0 = ((size_t)(r0 >> 7) * a.G + c / gpc) * 128 + (r0 & 127);
-      cp_async16(&ss[st * T + tid], a.s[it] + m0 * 2, 16);
-      if (ASYM) cp_async8(&sz[st * T + tid], a.z[it] + m0);
+      const size_t m0 = ((size_t)(r0 >> 7) * a.G + gidx) * 128 + (r0 & 127);
+      cp_async16_s(ss_s + (uint32_t)st * T16, a.s[it] + m0 * 2, 16);
+      if (ASYM) cp_async8_s(sz_s + (uint32_t)st * 8 * T, a.z[it] + m0);
     }
     cp_async_commit();  // one group per stage, empty or not, keeps the wait count fixed
   };
@@ -261,21 +272,23 @@ __global__ void __launch_bounds__(kGdMaxWarps * 32) gemv_direct_async_kernel(con
   int lb = 0, st = 0;
   for (; rb < a.row_blocks; rb += gridDim.x, ++lb) {
     cp_async_wait<S - 1>();  // this lane's copies of row block rb have landed
-    const int it = item_of(rb);
+    item_adv(it_comp, rb);
+    const int it = it_comp;
     if (a.X[it] != x_loaded) load_x(a.X[it]);
     float part[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) part[i] = 0.0f;
     if (cok) {
-      const uint4 sv = ss[st * T + tid];
-      const uint2 zv = ASYM ? sz[st * T + tid] : make_uint2(0u, 0u);
+      const uint32_t src = sq_s + (uint32_t)st * 8 * T16;
+      const uint4 sv = lds128(ss_s + (uint32_t)st * T16);
+      const uint2 zv = ASYM ? lds64(sz_s + (uint32_t)st * 8 * T) : make_uint2(0u, 0u);
       const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
       for (int i = 0; i < 8; i += 2) {
         const float2 sc = __half22float2(*reinterpret_cast<const __half2*>(&sw[i >> 1]));
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const float acc = gd_chunk<BF16>(sq[(st * 8 + i + h) * T + tid], xr);
+          const float acc = gd_chunk<BF16>(lds128(src + (uint32_t)(i + h) * T16), xr);
           float corr = xoff;
           if (ASYM) {
             const int zi = (int)(int8_t)(((i < 4 ? zv.x : zv.y) >> (8 * ((i + h) & 3))) & 0xFFu);
@@ -292,10 +305,11 @@ __global__ void __launch_bounds__(kGdMaxWarps * 32) gemv_direct_async_kernel(con
   }
   cp_async_wait<0>();
   __syncthreads();
+  int it = 0;
   for (int t = tid; t < lb * 8; t += blockDim.x) {
     const int l = t >> 3, row = t & 7;
     const int rbo = blockIdx.x + l * gridDim.x;
-    const int it = item_of(rbo);
+    item_adv(it, rbo);
     const int r = (rbo - (it ? a.rb_end[it - 1] : 0)) * 8 + row;
     float sum = 0.0f;
     for (int w = 0; w < nw; ++w) sum += red[(l * nw + w) * 8 + row];
