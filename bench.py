@@ -559,8 +559,8 @@ def run_profile_case(name):
 # name -> (bytes, {source file: sha256[:16]}, summary file).
 NCU_TRAFFIC = {
     # mean DRAM bytes per launch of the decode step (all gemv_direct_async_kernel)
-    "decode_step_per_launch": (32428280, {"gemv_direct.cuh": "d619e61ab3b68780", "common.cuh": "84092f83f8c9f1ae",
-                                          "lbq.cu": "f96dbd717a90b246"},
+    "decode_step_per_launch": (32426732, {"gemv_direct.cuh": "b7b97f59eb923d87", "common.cuh": "eb93cb6f87fb3da4",
+                                          "lbq.cu": "4a964504cf4b33d9"},
                                "profiles/decode_step_launch_list.md"),
 }
 
