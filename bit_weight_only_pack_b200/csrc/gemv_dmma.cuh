@@ -104,6 +104,10 @@ __global__ void __launch_bounds__(kDmMaxWarps * 32, 1) gemv_dmma_kernel(const Ge
     c0 = (warp * spw + cu.ss) * 8;
   };
   const size_t thr_off = (size_t)g * rowb + (size_t)t * 16;  // this thread's row / chunk within a pass
+  const size_t rowb8 = rowb * 8;
+  // 32-bit shared address of this thread's ring element (slot 0, j = 0); elements are T * 16 bytes apart
+  const uint32_t T16 = (uint32_t)T * 16;
+  const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring) + (uint32_t)tid * 16;
   // Copy a pass's codes (slot element j = 4h + 2f + e: row r + 16h + 8e,
   // chunk c0 + t + 4f) and, cooperatively, its scales and zero points.
   auto issue = [&](Cursor& cu, int slot) {
@@ -112,13 +116,18 @@ __global__ void __launch_bounds__(kDmMaxWarps * 32, 1) gemv_dmma_kernel(const Ge
     if (rt < a.row_tiles) {
       const int it = cu.it, N = a.N[it];
       const uint8_t* qb = a.q[it] + (size_t)n0 * rowb + (size_t)c0 * 16 + thr_off;
-      const bool full = n0 + kDmRows <= N && c0 + 8 <= chunks;
+      const uint32_t dst = ring_s + (uint32_t)slot * 8 * T16;
+      if (n0 + kDmRows <= N && c0 + 8 <= chunks) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int dr = 16 * (j >> 2) + 8 * (j & 1), dc = 4 * ((j >> 1) & 1);
-        const bool ok = full || (n0 + dr + g < N && c0 + dc + t < chunks);  // outside: nothing read, zeros staged
-        cp_async16(&ring[((size_t)slot * 8 + j) * T + tid], ok ? qb + (size_t)dr * rowb + dc * 16 : a.q[it],
-                   ok ? 16 : 0);
+        for (int j = 0; j < 8; ++j)
+          cp_async16_s(dst + j * T16, qb + (size_t)(2 * (j >> 2) + (j & 1)) * rowb8 + 64 * ((j >> 1) & 1), 16);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int dr = 16 * (j >> 2) + 8 * (j & 1), dc = 4 * ((j >> 1) & 1);
+          const bool ok = n0 + dr + g < N && c0 + dc + t < chunks;  // outside: nothing read, zeros staged
+          cp_async16_s(dst + j * T16, ok ? qb + (size_t)dr * rowb + dc * 16 : a.q[it], ok ? 16 : 0);
+        }
       }
       uint8_t* ms = mring + ((size_t)slot * nw + warp) * kDmMetaBytes;
       const int np = 8 >> gshift, gb = c0 >> gshift;
@@ -213,7 +222,7 @@ __global__ void __launch_bounds__(kDmMaxWarps * 32, 1) gemv_dmma_kernel(const Ge
     uint32_t w[8][4], za[8], zb[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const uint4 v = ring[((size_t)slot * 8 + j) * T + tid];
+      const uint4 v = lds128(ring_s + ((uint32_t)slot * 8 + j) * T16);
       w[j][0] = v.x; w[j][1] = v.y; w[j][2] = v.z; w[j][3] = v.w;
       if (ASYM && !OFF) {
         const int lg = (t + 4 * ((j >> 1) & 1)) >> gshift;
