@@ -8,7 +8,7 @@ indexed [k][n]). Groups run along K: one FP16 scale (and, for the asymmetric
 form, one int8 zero point) per (group of ``group`` consecutive k, column n);
 "Low Bit ARM kernels", group-wise scale section (group size 32, 64 or 128).
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * The scale is computed in FP32 and stored as FP16 (round to nearest even);
   the codes are computed by dividing by the *stored* scale widened back to FP32,

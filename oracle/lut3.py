@@ -10,7 +10,7 @@ small tiles out of the E4M3 subnormal range, so a weight's value is
 codebook[idx] * 2^(E - 127). E4M3 and UE8M0 are the OCP Microscaling (MX)
 element and scale types that page links to.
 
-Readings taken where the page is silent (listed in the design doc):
+Readings taken where the page is silent:
 
 * E4M3 is the "fn" variant: bias 7, subnormals, max 448, 0x7F / 0xFF are NaN.
 * UE8M0 has bias 127 and 0xFF is NaN.
