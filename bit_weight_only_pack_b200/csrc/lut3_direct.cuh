@@ -126,15 +126,20 @@ __global__ void __launch_bounds__(kLdMaxWarps * 32) lut3_direct_async_kernel(con
   const int T = blockDim.x, nw = T >> 5;
   const int kt = warp * 32 + lane;
   const bool tok = kt < (a.K >> 6);
-  uint4* ring = reinterpret_cast<uint4*>(ld_smem);
-  float* red = reinterpret_cast<float*>(ring + (size_t)S * 13 * T);
+  // 32-bit shared address of this thread's element 0 of stage 0; elements are T * 16 bytes apart
+  const uint32_t T16 = (uint32_t)T * 16;
+  const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ld_smem) + (uint32_t)tid * 16;
+  float* red = reinterpret_cast<float*>(ld_smem + (size_t)S * 13 * T16);
+  const uint8_t* ibase = a.i_region + (size_t)kt * a.N * 24;  // this lane's tile row of indices
+  const uint8_t* tbase = a.t_region + (size_t)kt * (a.N >> 3) * 16;
 
   auto issue = [&](int rb, int st) {
     if (tok && rb < a.row_blocks) {
-      const uint8_t* base = a.i_region + ((size_t)kt * a.N + (size_t)rb * 8) * 24;
+      const uint8_t* base = ibase + (size_t)rb * 192;
+      const uint32_t dst = ring_s + (uint32_t)st * 13 * T16;
 #pragma unroll
-      for (int v = 0; v < 12; ++v) cp_async16(&ring[((size_t)st * 13 + v) * T + tid], base + 16 * v, 16);
-      cp_async16(&ring[((size_t)st * 13 + 12) * T + tid], a.t_region + ((size_t)kt * (a.N >> 3) + rb) * 16, 16);
+      for (int v = 0; v < 12; ++v) cp_async16_s(dst + v * T16, base + 16 * v, 16);
+      cp_async16_s(dst + 12 * T16, tbase + (size_t)rb * 16, 16);
     }
     cp_async_commit();  // one group per row block, empty or not, keeps the wait count fixed
   };
@@ -166,30 +171,32 @@ __global__ void __launch_bounds__(kLdMaxWarps * 32) lut3_direct_async_kernel(con
 #pragma unroll
     for (int i = 0; i < 8; ++i) part[i] = 0.0f;
     if (tok) {
-      const uint4 tab = ring[((size_t)st * 13 + 12) * T + tid];
+      const uint32_t src = ring_s + (uint32_t)st * 13 * T16;
+      const uint4 tab = lds128(src + 12 * T16);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        // row i's 24 bytes: words 6i .. 6i+5 of the staged 48
-        uint32_t wr[6];
+      for (int i = 0; i < 8; i += 2) {
+        // rows i and i+1: 48 bytes, words 6i .. 6i+11 = chunks 3i/2 .. 3i/2+2
+        const uint4 u0 = lds128(src + (uint32_t)(3 * i / 2) * T16);
+        const uint4 u1 = lds128(src + (uint32_t)(3 * i / 2 + 1) * T16);
+        const uint4 u2 = lds128(src + (uint32_t)(3 * i / 2 + 2) * T16);
+        const uint32_t w12[12] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w, u2.x, u2.y, u2.z, u2.w};
 #pragma unroll
-        for (int e = 0; e < 6; ++e) {
-          const int wi = 6 * i + e;
-          const uint4 u = ring[((size_t)st * 13 + (wi >> 2)) * T + tid];
-          wr[e] = (wi & 3) == 0 ? u.x : (wi & 3) == 1 ? u.y : (wi & 3) == 2 ? u.z : u.w;
-        }
-        float acc = 0.0f;
+        for (int r = 0; r < 2; ++r) {
+          const uint32_t* wr = w12 + 6 * r;
+          float acc = 0.0f;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t wa = wr[3 * h], wb = wr[3 * h + 1], wc = wr[3 * h + 2];
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t wa = wr[3 * h], wb = wr[3 * h + 1], wc = wr[3 * h + 2];
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            uint32_t p[4];
-            lut3_decode8(lut3_selector(t < 2 ? wa : wb, wc, t), tab, p);
+            for (int t = 0; t < 4; ++t) {
+              uint32_t p[4];
+              lut3_decode8(lut3_selector(t < 2 ? wa : wb, wc, t), tab, p);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc = fma2_bf16_f32(xr[16 * h + 4 * t + e], p[e], acc);
+              for (int e = 0; e < 4; ++e) acc = fma2_bf16_f32(xr[16 * h + 4 * t + e], p[e], acc);
+            }
           }
+          part[i + r] = acc;
         }
-        part[i] = acc;
       }
     }
     const float total = butterfly8(part, lane);
