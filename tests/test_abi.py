@@ -91,3 +91,33 @@ def test_workspace_query_is_host_only():
     assert lbq.lbq_workspace_size(0, 1, 4096, 4096, 32, 0) >= 0
     with pytest.raises(lbq.LbqError):
         lbq.lbq_workspace_size(9, 1, 4096, 4096, 32, 0)
+
+
+def test_grouped_noalloc_and_lut3_calls_reject_bad_arguments_on_the_host():
+    """Argument checks of the grouped, no-alloc and LUT3 calls run before any
+    device work: each bad call returns its status and launches nothing."""
+    import bit_weight_only_pack_b200 as lbq
+    b = lbq.binding
+    before = lbq.lbq_launch_count()
+    good = [(16, 32, 48, 64)]  # X, image, Y (16-byte aligned fake addresses), N
+    cases = [
+        (lambda: lbq.lbq_gemv_grouped(None, 1, 64, 32, 0, 0, 0, None), b.LBQ_ERR_INVALID_ARG),          # no items
+        (lambda: lbq.lbq_gemv_grouped(lbq.make_gemv_items(good), 0, 64, 32, 0, 0, 0, None), b.LBQ_ERR_INVALID_ARG),
+        (lambda: lbq.lbq_gemv_grouped(lbq.make_gemv_items(good * 5), 5, 64, 32, 0, 0, 0, None), b.LBQ_ERR_INVALID_ARG),
+        (lambda: lbq.lbq_gemv_grouped(lbq.make_gemv_items(good), 1, 32768, 32, 0, 0, 0, None), b.LBQ_ERR_UNSUPPORTED),
+        (lambda: lbq.lbq_gemv_grouped(lbq.make_gemv_items(good), 1, 64, 48, 0, 0, 0, None), b.LBQ_ERR_UNSUPPORTED),
+        (lambda: lbq.lbq_gemv_grouped(lbq.make_gemv_items([(8, 32, 48, 64)]), 1, 64, 32, 0, 0, 0, None),
+         b.LBQ_ERR_INVALID_ARG),                                                                        # misaligned X
+        (lambda: lbq.lbq_gemv_grouped(lbq.make_gemv_items(good), 1, 64, 32, 0, 2, 0, None), b.LBQ_ERR_UNSUPPORTED),
+        (lambda: lbq.lbq_gemv_noalloc(16, 0, 17, 64, 8, 32, 0, 32, 48, 0, None), b.LBQ_ERR_UNSUPPORTED),  # M > 16
+        (lambda: lbq.lbq_gemv_noalloc(16, 0, 1, 60, 8, 32, 0, 32, 48, 0, None), b.LBQ_ERR_INVALID_ARG),   # K % group
+        (lambda: lbq.lbq_lut3_gemm(16, 1, 1, 96, 8, 32, 48, 1, None, 0, None), b.LBQ_ERR_INVALID_ARG),    # K % 64
+        (lambda: lbq.lbq_lut3_gemm(16, 1, 1, 128, 12, 32, 48, 1, None, 0, None), b.LBQ_ERR_INVALID_ARG),  # N % 8
+        (lambda: lbq.lbq_lut3_gemm(16, 0, 1, 128, 8, 32, 48, 1, None, 0, None), b.LBQ_ERR_UNSUPPORTED),   # FP16 X
+    ]
+    for call, status in cases:
+        with pytest.raises(lbq.LbqError) as e:
+            call()
+        assert e.value.status == status, lbq.lbq_last_error()
+        assert lbq.lbq_last_error()
+    assert lbq.lbq_launch_count() == before
