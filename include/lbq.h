@@ -153,9 +153,12 @@ lbq_status lbq_gemv_grouped(const lbq_gemv_item* items, int count, int K, int gr
 
 /*
  * Prefill GEMM on INT4 weights, any M >= 1 (M <= 16 is routed to lbq_gemv's
- * kernels). Same arguments and result as lbq_gemv. Weights are dequantised
- * to BF16 in shared memory and multiplied on the tensor cores; X must be BF16
- * for M > 16. Asynchronous.
+ * kernels). Same arguments and result as lbq_gemv; X may be FP16 or BF16.
+ * For M > 16 the weights are dequantised into the activation type ((q - z)
+ * formed exactly, the product with the scale rounded once) straight into
+ * tensor memory and multiplied on the tcgen05 tensor cores with FP32
+ * accumulation ("Low Bit Metal Kernels": dequantise just before the
+ * multiply). Needs no workspace for M > 16. Asynchronous.
  */
 lbq_status lbq_gemm(const void* X, int x_dtype, int M, int K, int N, int group, int mode,
                     const void* image, void* Y, int y_dtype, void* ws, size_t ws_bytes,
