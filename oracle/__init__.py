@@ -15,6 +15,9 @@ What it computes, and where each step comes from:
   codebook shared by a tile of 8 output channels x 64 K, scaled by one UE8M0
   exponent per tile; its canonical index bit stream and its exact decode.
   Source: vLLM PR 62759 write-up (format section; tile and memory budget).
+* ``oracle.mxfp8``  -- MXFP8 activations (E4M3 elements, one UE8M0 scale per
+  32 k) and the LUT3 x MXFP8 product: the activation format of the same page's
+  native and emulated LUT-B paths (the next row after the BF16 LUT3 path).
 * ``oracle.matmul`` -- Y = X . W accumulated in FP64, the error scale
   S = |X| . |W|, and the acceptance test |y - y_ref| <= 4e-3*S + ulp16(|y_ref|).
 
@@ -29,4 +32,4 @@ decoders, nearest-level characterisation of the quantiser). Quantisation
 and it is out of scope.
 """
 
-from . import int4, lut3, matmul  # noqa: F401
+from . import int4, lut3, matmul, mxfp8  # noqa: F401

@@ -325,3 +325,118 @@ def test_int4_algorithmic_bytes():
     # bits per weight: 4 + 16/g (sym), 4 + 24/g (asym)
     assert int4.algorithmic_bytes(4096, 4096, 32, "sym") == 4096 * 4096 * 4.5 / 8
     assert int4.algorithmic_bytes(4096, 14336, 128, "asym") == 4096 * 14336 * (4 + 24 / 128) / 8
+
+
+# ----------------------------------------------------------------------------- MXFP8 activations
+
+def _e4m3_neighbours_midpoints():
+    vals = sorted({v for v in lut3.E4M3_TABLE.tolist() if not math.isnan(v) and v >= 0})
+    return [(a + b) / 2 for a, b in zip(vals, vals[1:])]
+
+
+def test_e4m3_rounding_matches_torch_and_ml_dtypes_in_range():
+    """Round-to-nearest-even into E4M3 equals the libraries' casts for every
+    value the libraries convert without saturation (|v| <= 448): random
+    values across all binades, every midpoint between neighbours (ties), and
+    values that underflow."""
+    import ml_dtypes
+    import torch
+    from oracle import mxfp8
+    rng = np.random.default_rng(17)
+    mags = np.ldexp(rng.uniform(1.0, 2.0, 4000), rng.integers(-14, 9, 4000))
+    mids = np.array(_e4m3_neighbours_midpoints())
+    v = np.concatenate([mags, mids, [2.0 ** -10, 2.0 ** -11, 3 * 2.0 ** -11, 1e-9, 448.0]])
+    v = v[v <= 448.0]
+    v = np.concatenate([v, -v]).astype(np.float32)  # values exact in FP32 (midpoints included)
+    ours = np.array([mxfp8.e4m3_byte(mxfp8.round_e4m3(float(x))) for x in v], dtype=np.uint8)
+    tor = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    lib = v.astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    assert np.array_equal(ours, tor)
+    assert np.array_equal(ours, lib)
+
+
+def test_e4m3_rounding_saturates_above_448():
+    from oracle import mxfp8
+    assert [mxfp8.round_e4m3(x) for x in (448.0, 463.9, 464.0, 511.9, -500.0)] == [448.0] * 4 + [-448.0]
+
+
+def test_mx_scale_rule_hand_examples():
+    """Scale byte = floor(log2 amax) - 8 + 127 and elements x / 2^(that - 127):
+    amax 1 -> scale 2^-8 and x = 1 becomes 256; amax 448 -> scale 1; amax 500
+    -> scale 1 and 500 saturates to 448; amax 0.75 -> scale 2^-9 and 0.75
+    becomes 384; amax 2^-130 -> the smallest scale 2^-127 (clamped), so it
+    becomes 2^-3; a zero block stores scale 1."""
+    from oracle import mxfp8
+    def block(first, rest=0.0):
+        return np.array([[first] + [rest] * 31])
+    cases = [
+        (1.0, 119, 256.0), (448.0, 127, 448.0), (500.0, 127, 448.0), (0.75, 118, 384.0),
+        (2.0 ** -130, 0, 2.0 ** -3), (0.0, 127, 0.0),
+    ]
+    for amax, sbyte, elem in cases:
+        codes, scales = mxfp8.quantize(block(amax))
+        assert scales[0, 0] == sbyte
+        assert lut3.E4M3_TABLE[codes[0, 0]] == elem
+        assert mxfp8.dequant(codes, scales)[0, 0] == elem * 2.0 ** (sbyte - 127)
+    # a second element is scaled by the same power of two: 0.3 * 256 = 76.8 -> 80 (quantum 8)
+    codes, scales = mxfp8.quantize(block(1.0, 0.3))
+    assert lut3.E4M3_TABLE[codes[0, 1]] == 80.0
+
+
+def test_mx_block_maximum_lands_in_the_top_binade_and_error_is_bounded():
+    """Every block's largest element is in [256, 448] after scaling, and each
+    element's error is at most half an E4M3 step: 2^-4 relative in the normal
+    range, 2^-10 of the scale in the subnormal range."""
+    from oracle import mxfp8
+    rng = np.random.default_rng(5)
+    X = (rng.standard_normal((4, 256)) * np.ldexp(1.0, rng.integers(-20, 20, (4, 1)))).astype(np.float32)
+    codes, scales = mxfp8.quantize(X)
+    Xq = mxfp8.dequant(codes, scales)
+    elems = np.abs(lut3.E4M3_TABLE[codes]).reshape(4, 8, 32)
+    assert np.all(elems.max(axis=2) >= 256.0) and np.all(elems.max(axis=2) <= 448.0)
+    scale = np.ldexp(1.0, scales.astype(np.int64) - 127)[:, np.arange(256) // 32]
+    x = X.astype(np.float64)
+    scaled = np.abs(x) / scale
+    normal = (scaled >= 2.0 ** -6) & (scaled < 448.0)
+    assert np.all(np.abs(Xq - x)[normal] <= 2.0 ** -4 * np.abs(x)[normal])
+    assert np.all(np.abs(Xq - x)[scaled < 2.0 ** -6] <= 2.0 ** -10 * scale[scaled < 2.0 ** -6])
+
+
+def test_mx_representable_blocks_round_trip_exactly():
+    """A block that already is E4M3 values times one power of two, with its
+    largest element in [256, 448], comes back bit for bit."""
+    from oracle import mxfp8
+    rng = np.random.default_rng(9)
+    finite = [b for b in range(256) if not math.isnan(lut3.E4M3_TABLE[b])]
+    top = [b for b in finite if 256.0 <= abs(lut3.E4M3_TABLE[b]) <= 448.0]
+    for s in (-20, 0, 7):
+        bytes_ = rng.choice(finite, size=(3, 64))
+        bytes_[:, 0] = rng.choice(top, size=3)
+        bytes_[:, 32] = rng.choice(top, size=3)
+        vals = np.abs(lut3.E4M3_TABLE[bytes_]).reshape(3, 2, 32)
+        assert np.all(vals.max(axis=2) <= 448.0)
+        X = lut3.E4M3_TABLE[bytes_] * 2.0 ** s
+        codes, scales = mxfp8.quantize(X)
+        assert np.array_equal(mxfp8.dequant(codes, scales), X)
+        assert np.all(scales == 127 + s)
+
+
+def test_lut3_mxfp8_product_matches_exact_rational_brute_force():
+    """The LUT3 x MXFP8 product equals the exact rational sum of the exact
+    products of the dequantised operands (one 64 x 8 tile, two rows)."""
+    from fractions import Fraction
+    from oracle import mxfp8
+    rng = np.random.default_rng(21)
+    K, N, M = 64, 8, 2
+    idx = rng.integers(0, 8, size=(K, N)).astype(np.uint8)
+    cb = np.array([[[0x38, 0xB8, 0x40, 0x30, 0x7E, 0x01, 0x00, 0xC4]]], dtype=np.uint8)
+    ex = np.array([[120]], dtype=np.uint8)
+    X = rng.standard_normal((M, K)).astype(np.float32)
+    Y = mxfp8.lut3_matmul(X, idx, cb, ex)
+    codes, scales = mxfp8.quantize(X)
+    Xq = mxfp8.dequant(codes, scales)
+    W = lut3.dequant(idx, cb, ex)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(float(Xq[m, k])) * Fraction(float(W[k, n])) for k in range(K))
+            assert abs(Fraction(float(Y[m, n])) - exact) <= abs(exact) * Fraction(1, 2 ** 50) + Fraction(1, 2 ** 200)
