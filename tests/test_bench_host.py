@@ -70,3 +70,22 @@ def test_single_process_needs_no_group(monkeypatch):
         monkeypatch.delenv(k, raising=False)
     assert bench.dist_setup("gloo") == (1, 0, 0)
     assert bench.max_over_ranks(1, 4.0) == 4.0
+
+
+def test_bench_byte_counts_match_the_oracle_and_the_library():
+    """The bytes bench.py divides by (its GB/s) are the format's algorithmic
+    bytes as the oracle defines them, and the decode step's total is the sum
+    over its 224 projections; the library's image for INT4 adds only padding
+    and a header on top of them."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads
+    import bit_weight_only_pack_b200 as lbq
+    from oracle import int4, lut3
+    for K, N, g, mode in [(4096, 4096, 32, "sym"), (4096, 14336, 32, "asym"), (8192, 28672, 128, "sym"),
+                          (14336, 4096, 64, "asym")]:
+        assert bench.int4_bytes(K, N, g, mode) == int4.algorithmic_bytes(K, N, g, mode)
+        assert lbq.lbq_packed_size(K, N, g, 0 if mode == "sym" else 1) >= bench.int4_bytes(K, N, g, mode)
+    assert bench.lut3_bytes(4096, 14336) == lut3.algorithmic_bytes(4096, 14336)
+    step = 32 * sum(int4.algorithmic_bytes(K, N, 32, "asym") for _, K, N in workloads.LLAMA3_8B_PROJ)
+    assert step == 4143972352
