@@ -507,6 +507,7 @@ PROFILE_CASES = {
     "c2down": (14336, 4096, 32, "asym", "f16", 1, None),
     "c2kv": (4096, 1024, 32, "asym", "f16", 1, None),
     "c2gate_mma": (4096, 14336, 32, "asym", "f16", 1, 2),
+    "c2gate_regs": (4096, 14336, 32, "asym", "f16", 1, 4, 0),  # batch-1 kernel variant: weights in registers
     "c3m1": (8192, 28672, 128, "sym", "bf16", 1, None),
     "c3m16": (8192, 28672, 128, "sym", "bf16", 16, None),
     "c4m2048": (4096, 14336, 128, "asym", "bf16", 2048, None),
@@ -521,7 +522,8 @@ def run_profile_case(name):
     import torch
     import bit_weight_only_pack_b200 as lbq
     import workloads
-    K, N, group, mode, xdt, M, path = PROFILE_CASES[name]
+    K, N, group, mode, xdt, M, path = PROFILE_CASES[name][:7]
+    variant = PROFILE_CASES[name][7] if len(PROFILE_CASES[name]) > 7 else None
     device = torch.device("cuda", 0)
     torch.cuda.set_device(0)
     if mode == "lut3":
@@ -537,6 +539,8 @@ def run_profile_case(name):
     X = workloads.activations_device(7, M, K, xdt, device)
     if path is not None:
         lbq.lbq_debug_gemv_path(path)
+    if variant is not None:
+        lbq.lbq_debug_direct_variant(variant)
     if mode == "lut3":
         ws = lbq.workspace(2, M, K, N, 0, "lut3")
         for img in images:
@@ -547,6 +551,7 @@ def run_profile_case(name):
             lbq.gemm(X, img, N, group, mode, ws=ws)
     torch.cuda.synchronize()
     lbq.lbq_debug_gemv_path(0)
+    lbq.lbq_debug_direct_variant(-1)
     lbq.device_status()
     print(f"profile case {name}: {len(images)} launches of K={K} N={N} {mode} M={M}", flush=True)
     return 0
