@@ -62,6 +62,7 @@ _SIGS = {
     "lbq_set_option": ([_c_int, _c_int], _c_int),
     "lbq_gemv_noalloc": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp], _c_int),
     "lbq_gemv_grouped": ([ctypes.POINTER(lbq_gemv_item), _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp], _c_int),
+    "lbq_quantize_mxfp8": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
     "lbq_debug_force_splits": ([_c_int], None),
     "lbq_debug_force_skinny": ([_c_int], None),
     "lbq_debug_force_tc": ([_c_int], None),
@@ -164,6 +165,21 @@ def lbq_gemv_noalloc(X, x_dtype, M, K, N, group, mode, image, Y, y_dtype, stream
 
 
 LBQ_OPT_PDL = 1
+
+
+def lbq_quantize_mxfp8(X, x_dtype, M, K, codes, scales, stream):
+    _check(_lib.lbq_quantize_mxfp8(X, x_dtype, M, K, codes, scales, stream))
+
+
+def quantize_mxfp8(X):
+    """MXFP8 activations: X [M, K] FP16/BF16 -> (codes uint8 [M, K] E4M3, scales uint8 [M, K/32] UE8M0)."""
+    torch = _torch()
+    _need_cuda(X)
+    M, K = X.shape
+    codes = torch.empty((M, K), dtype=torch.uint8, device=X.device)
+    scales = torch.empty((M, K // 32), dtype=torch.uint8, device=X.device)
+    lbq_quantize_mxfp8(X.data_ptr(), _dt(X), M, K, codes.data_ptr(), scales.data_ptr(), _stream())
+    return codes, scales
 
 
 def lbq_set_option(option, value):

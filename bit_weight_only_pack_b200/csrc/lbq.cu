@@ -27,6 +27,7 @@
 #include "tc_gemv.cuh"
 #include "gemv_direct.cuh"
 #include "gemv_dmma.cuh"
+#include "mxfp8.cuh"
 #include "gemm_ts.cuh"
 #include "lut3_direct.cuh"
 
@@ -1126,6 +1127,23 @@ lbq_status lbq_gemv_grouped(const lbq_gemv_item* items, int count, int K, int gr
   }
   return run_direct(items, count, K, group, mode, x_dtype == LBQ_DTYPE_BF16, y_dtype == LBQ_DTYPE_BF16,
                     static_cast<cudaStream_t>(stream));
+}
+
+lbq_status lbq_quantize_mxfp8(const void* X, int x_dtype, int M, int K, uint8_t* codes, uint8_t* scales,
+                              void* stream) {
+  if (!X || !codes || !scales) return fail(LBQ_ERR_INVALID_ARG, "X, codes and scales must be non-null");
+  if (M <= 0 || K <= 0 || K % 32) return fail(LBQ_ERR_INVALID_ARG, "M=%d K=%d: need M >= 1 and K a multiple of 32", M, K);
+  if (!aligned16(X) || !aligned16(codes))
+    return fail(LBQ_ERR_INVALID_ARG, "X and codes must be 16-byte aligned");
+  if (x_dtype != LBQ_DTYPE_F16 && x_dtype != LBQ_DTYPE_BF16) return fail(LBQ_ERR_UNSUPPORTED, "x_dtype %d", x_dtype);
+  const long long blocks = (long long)M * (K / 32);
+  const unsigned grid = (unsigned)((blocks + 255) / 256);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (x_dtype == LBQ_DTYPE_BF16)
+    quantize_mxfp8_kernel<true><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(X), codes, scales, blocks);
+  else
+    quantize_mxfp8_kernel<false><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(X), codes, scales, blocks);
+  return launch_check("MXFP8 quantisation launch");
 }
 
 lbq_status lbq_gemv_noalloc(const void* X, int x_dtype, int M, int K, int N, int group, int mode, const void* image,

@@ -241,6 +241,23 @@ lbq_status lbq_set_option(int option, int value);
 lbq_status lbq_gemv_noalloc(const void* X, int x_dtype, int M, int K, int N, int group, int mode,
                             const void* image, void* Y, int y_dtype, void* stream);
 
+/*
+ * MXFP8 quantisation of activations (vLLM PR 62759 write-up: MXFP8
+ * activations = E4M3 elements with one UE8M0 scale per 1 x 32 block; OCP MX
+ * element and scale types): the activation side of a LUT3 x MXFP8 product.
+ *   X      (device) [M, K] row-major FP16 / BF16 (x_dtype), finite, 16-byte aligned
+ *   K      a multiple of 32; block b of row m is k = 32 b .. 32 b + 31
+ *   codes  (device) uint8 [M, K], E4M3 bytes, 16-byte aligned
+ *   scales (device) uint8 [M, K/32], UE8M0 bytes
+ * Per block: scale byte = floor(log2 amax) - 8 + 127 clamped to [0, 254]
+ * (127 for an all-zero block), amax its largest |x|; each element is
+ * x * 2^(127 - byte) rounded to nearest E4M3, ties to even, saturating at
+ * +-448 (zeros keep their sign). Bit-identical to the CPU reference.
+ * Asynchronous on `stream`; argument errors are reported before any launch.
+ */
+lbq_status lbq_quantize_mxfp8(const void* X, int x_dtype, int M, int K, uint8_t* codes, uint8_t* scales,
+                              void* stream);
+
 /* Number of kernel launches the library has enqueued so far in this process. */
 uint64_t lbq_launch_count(void);
 
