@@ -564,7 +564,7 @@ def run_profile_case(name):
 # name -> (bytes, {source file: sha256[:16]}, summary file).
 NCU_TRAFFIC = {
     # mean DRAM bytes per launch of the decode step (all gemv_direct_async_kernel)
-    "decode_step_per_launch": (32426732, {"gemv_direct.cuh": "b7b97f59eb923d87", "common.cuh": "eb93cb6f87fb3da4",
+    "decode_step_per_launch": (32426732, {"gemv_direct.cuh": "80c3d5258f32c480", "common.cuh": "eb93cb6f87fb3da4",
                                           "lbq.cu": "18ec92ef2e5d8cd1"},
                                "profiles/decode_step_launch_list.md"),
 }

@@ -182,9 +182,6 @@ __global__ void __launch_bounds__(kGdMaxWarps * 32, 1) gemv_direct_kernel(const 
 // only synchronisation. Dynamic shared memory: uint4 codes [S][8][T], uint4
 // scales [S][T], uint2 zero points [S][T] (T threads), then the row sums as in
 // gemv_direct_kernel.
-template <int S>
-constexpr int gd_stage_bytes_per_thread() { return S * (8 * 16 + 16 + 8); }
-
 template <bool BF16, bool ASYM, int S>
 __global__ void __launch_bounds__(kGdMaxWarps * 32) gemv_direct_async_kernel(const GemvDirectArgs a) {
   extern __shared__ __align__(16) uint8_t gd_smem[];
