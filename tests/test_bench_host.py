@@ -89,3 +89,26 @@ def test_bench_byte_counts_match_the_oracle_and_the_library():
     assert bench.lut3_bytes(4096, 14336) == lut3.algorithmic_bytes(4096, 14336)
     step = 32 * sum(int4.algorithmic_bytes(K, N, 32, "asym") for _, K, N in workloads.LLAMA3_8B_PROJ)
     assert step == 4143972352
+
+
+def test_profile_summaries_name_commands_that_exist():
+    """Every summary under profiles/ gives the command that made it, and that
+    command runs committed files only: bench.py with a profile case it defines
+    or with flags its parser accepts."""
+    import glob
+    import re
+    sys.path.insert(0, ROOT)
+    import bench
+    files = sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md")))
+    assert files
+    for path in files:
+        text = open(path).read()
+        cmds = re.findall(r"python bench\.py[^\n`]*", text)
+        assert cmds, f"{os.path.basename(path)} gives no command"
+        for cmd in cmds:
+            m = re.search(r"--profile (\S+)", cmd)
+            if m:
+                assert m.group(1) in bench.PROFILE_CASES, (path, m.group(1))
+            for flag in re.findall(r"(--[a-z-]+)", cmd):
+                assert flag in ("--profile", "--steps", "--warmup", "--no-secondary", "--no-cpu-baseline",
+                                "--gpus", "--impl", "--quick", "--ungrouped", "--no-pdl", "--layers"), (path, flag)
