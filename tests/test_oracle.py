@@ -221,6 +221,38 @@ def test_ulp16_values():
     assert u.tolist() == [2.0 ** -10, 2.0 ** -10, 2.0 ** -9, 0.5, 2.0 ** -24, 2.0 ** -24, 2.0 ** -24, 2.0 ** -9]
 
 
+def test_abs_scale_hand_values(golden):
+    """S = sum_k |x_k w_kn| against hand sums: a mixed-sign 2x3 . 3x2 case with
+    cancelling terms, and the sym 4x4 fixture (S far above |y| in column 0)."""
+    g = golden("acceptance_2x3x2.json")
+    X, W = np.array(g["X"]), np.array(g["W"])
+    assert matmul.matmul_f64(X, W).tolist() == g["Y"]
+    assert matmul.abs_scale(X, W).tolist() == g["S"]
+    assert matmul.ulp16(np.array(g["Y"])).tolist() == g["ulp16"]
+    g4 = golden("int4_sym_4x4.json")
+    assert matmul.abs_scale(np.array(g4["X"]), np.array(g4["dequant"])).tolist() == g4["S"]
+
+
+@pytest.mark.parametrize("factor,accepted", [(1.5, False), (1.05, False), (0.9, True), (0.5, True)])
+def test_acceptance_bound_is_tight(golden, factor, accepted):
+    """An output off by `factor` hand-derived bounds is rejected above 1 and
+    accepted below it, element by element, and error_ratio reports the factor:
+    a 2x change in the 4e-3 factor or in S moves 1.5 or 0.9 across 1."""
+    g = golden("acceptance_2x3x2.json")
+    X, W = np.array(g["X"]), np.array(g["W"])
+    Y_ref = np.array(g["Y"])
+    bound = np.array(g["bound"])
+    S = matmul.abs_scale(X, W)
+    for sign in (1.0, -1.0):
+        for m in range(2):
+            for n in range(2):
+                Y = Y_ref.copy()
+                Y[m, n] += sign * factor * bound[m, n]
+                r = matmul.error_ratio(Y, Y_ref, S)
+                assert r[m, n] == pytest.approx(factor, rel=1e-12)
+                assert matmul.check(Y, Y_ref, S)[0] is accepted
+
+
 def test_tolerance_accepts_fp32_accumulation_and_rejects_mistakes():
     rng = np.random.default_rng(17)
     M, K, N = 2, 512, 64
