@@ -838,10 +838,13 @@ constexpr int kNoAllocMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device (the first lookup may load the module, so it must not happen
-// while the stream is being captured).
-static uint8_t* noalloc_scratch(lbq_status* st) {
+// Device address of g_noalloc_scratch on the current device. Outside stream
+// capture it is looked up on every call (cheap once the module is loaded), so
+// a module reloaded after cudaDeviceReset is found at its new address; while
+// `stream` is being captured the address of the last uncaptured call on this
+// device is used, because the first lookup may load the module, which capture
+// does not allow.
+static uint8_t* noalloc_scratch(cudaStream_t stream, lbq_status* st) {
   static std::mutex mu;
   static uint8_t* ptr[kNoAllocMaxDevices] = {};
   int dev = 0;
@@ -851,13 +854,20 @@ static uint8_t* noalloc_scratch(lbq_status* st) {
                kNoAllocMaxDevices);
     return nullptr;
   }
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if ((*st = cuda_check(cudaStreamIsCapturing(stream, &cap), "cudaStreamIsCapturing")) != LBQ_OK) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (ptr[dev] == nullptr) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     if ((*st = cuda_check(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress of the fixed scratch")) !=
         LBQ_OK)
       return nullptr;
     ptr[dev] = static_cast<uint8_t*>(p);
+  } else if (ptr[dev] == nullptr) {
+    *st = fail(LBQ_ERR_INVALID_ARG,
+               "lbq_gemv_noalloc: the first call on a device must come before any stream capture (it looks up the "
+               "fixed scratch's address)");
+    return nullptr;
   }
   *st = LBQ_OK;
   return ptr[dev];
@@ -1163,7 +1173,7 @@ lbq_status lbq_gemv_noalloc(const void* X, int x_dtype, int M, int K, int N, int
                 M, K, N, need, kNoAllocScratchBytes);
   uint8_t* scratch = nullptr;
   if (need) {
-    scratch = noalloc_scratch(&st);
+    scratch = noalloc_scratch(static_cast<cudaStream_t>(stream), &st);
     if (!scratch) return st;
     // The counters must be zero when the kernel starts; the previous call may
     // have left partial sums where this shape keeps its counters.

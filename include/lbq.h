@@ -68,9 +68,22 @@ int lbq_version(void);
 
 /*
  * Size in bytes of the device image for a K x N weight in `mode`.
- * INT4 (SYM/ASYM): group in {32, 64, 128}, K % group == 0, N >= 1.
- * LUT3: group is ignored (pass 0), K % 64 == 0, N % 8 == 0.
- * Writes *bytes (host). No device work.
+ * INT4 (SYM/ASYM): group in {32, 64, 128}, K % group == 0, N >= 1. The
+ *   format holds two codes per byte ("Low Bit Metal Kernels", INT4 listing:
+ *   one byte = two nibbles) plus one FP16 scale, and for ASYM one int8 zero
+ *   point, per group of a column ("Low Bit ARM kernels", group-wise scale
+ *   section): K*N/2 + (K/group)*N*(2 or 3) bytes. The image adds a 256-byte
+ *   header, 256-byte region alignment and the scales / zero points padded to
+ *   128-channel tiles.
+ * LUT3: group is ignored (pass 0), K % 64 == 0, N % 8 == 0. The format is a
+ *   3-bit index per weight, 8 E4M3 codebook bytes and one UE8M0 exponent per
+ *   8-channel x 64-k tile: 3 + 72/512 = 3.140625 bits per weight, the write-up's
+ *   "about 3.14 bits/weight", with 6144 index bytes per 128 x 128 block (vLLM
+ *   PR 62759 write-up, format section and its tile / memory budget). The image
+ *   adds the header, a 16-byte BF16 table per tile and alignment.
+ * Writes *bytes (host). No device work. Errors: LBQ_ERR_UNSUPPORTED for an
+ * unknown mode or group, LBQ_ERR_INVALID_ARG for sizes the format cannot hold
+ * or a null `bytes`.
  */
 lbq_status lbq_packed_size(int K, int N, int group, int mode, size_t* bytes);
 
@@ -108,7 +121,11 @@ lbq_status lbq_pack_lut3(const uint8_t* idx, const uint8_t* codebooks, const uin
 /*
  * Workspace needed by lbq_gemv / lbq_gemm / lbq_lut3_gemm for this shape:
  * the split-K partial sums and tile counters of the dispatch the library
- * would pick. op: 0 = lbq_gemv, 1 = lbq_gemm, 2 = lbq_lut3_gemm.
+ * would pick. Decode at batch 1 is a GEMV whose rows are split over many
+ * lanes and reduced ("Low Bit ARM kernels": decode is a GEMV; "BaseRT",
+ * kernel-selection section: SIMD groups share one weight row); when the rows
+ * alone cannot fill the 148 SMs the K range is split as well, and the slices'
+ * FP32 partial sums meet here. op: 0 = lbq_gemv, 1 = lbq_gemm, 2 = lbq_lut3_gemm.
  * Writes *bytes (host); 0 means the call needs no workspace (ws may be null).
  * The workspace's tile counters must be zero when a call starts: zero-fill a
  * new workspace before its first use; every call that completes returns its
@@ -174,7 +191,12 @@ lbq_status lbq_lut3_gemm(const void* X, int x_dtype, int M, int K, int N,
                          void* stream);
 
 /*
- * Debug / parity: recover the canonical arrays from an INT4 image.
+ * Debug / parity: recover the canonical arrays from an INT4 image, the exact
+ * inverse of the repack: two codes per byte with the low nibble the even k
+ * ("Low Bit Metal Kernels", INT4 listing: the low nibble is taken first), the
+ * FP16 scale and int8 zero point per group ("Low Bit ARM kernels", group-wise
+ * scale section). Reads and checks the image header (synchronous 64-byte copy);
+ * LBQ_ERR_INVALID_ARG if it does not match K, N, group, mode.
  *   q_packed (device) uint8 [K/2, N]: byte[j][n] = q[2j][n] | q[2j+1][n] << 4
  *   scales   (device) uint16 [K/group, N]: FP16 bit patterns
  *   zp       (device) int8 [K/group, N] (ASYM; may be null, ignored for SYM)
@@ -183,7 +205,10 @@ lbq_status lbq_unpack_canonical(const void* image, int K, int N, int group, int 
                                 uint8_t* q_packed, uint16_t* scales, int8_t* zp, void* stream);
 
 /*
- * Debug / parity: recover the canonical LUT3 arrays from a LUT3 image.
+ * Debug / parity: recover the canonical LUT3 arrays from a LUT3 image (the
+ * format of the vLLM PR 62759 write-up, format section: 3-bit indices, 8 E4M3
+ * codebook bytes and one UE8M0 exponent per 8-channel x 64-k tile). Reads and
+ * checks the image header; LBQ_ERR_INVALID_ARG if it does not match K, N.
  *   idx_stream (device) uint8 [K/64, N/8, 8, 24]: per tile and channel, the 64
  *              indices as a little-endian 192-bit string, index i in bits [3i, 3i+3)
  *   codebooks  (device) uint8 [K/64, N/8, 8];  exponents (device) uint8 [K/64, N/8]
@@ -193,7 +218,10 @@ lbq_status lbq_unpack_lut3_canonical(const void* image, int K, int N, uint8_t* i
 
 /*
  * Debug / parity: the exact dequantised weight, W_out (device) float32 [K, N].
- * INT4: (q - z) * s; LUT3: e4m3(cb) * 2^(E-127). Both are exact in FP32.
+ * INT4: (q - z) * s ("Low Bit Metal Kernels", INT4 listing: (nibble - 8) *
+ * scale; "Low Bit ARM kernels": (q - zp) * s with a zero point);
+ * LUT3: e4m3(cb) * 2^(E-127) (vLLM PR 62759 write-up, format section).
+ * Both are exact in FP32. Reads and checks the image header.
  */
 lbq_status lbq_dequant(const void* image, int K, int N, int group, int mode,
                        float* W_out, void* stream);
@@ -231,8 +259,12 @@ lbq_status lbq_set_option(int option, int value);
  *   lbq_gemv with a workspace for it.
  *   Zero state: nothing has to be zero beforehand; each call clears the tile
  *   counters it will use (one memset on `stream`) before its kernel.
- *   First call: looks up the array's device address once per device (the
- *   lookup may load the module); make it outside stream capture.
+ *   Address: outside stream capture every call looks the array's device
+ *   address up (cheap once loaded; a module reloaded after cudaDeviceReset
+ *   is found at its new place). Under capture the address of the last
+ *   uncaptured call on the device is used, so the first call on each device
+ *   must come before any capture (LBQ_ERR_INVALID_ARG otherwise), and a
+ *   cudaDeviceReset must be followed by an uncaptured call before capturing.
  *   Concurrency: all calls on one device share the one array, so two calls
  *   whose work can overlap (different streams, or host threads racing on one
  *   stream) corrupt each other's partial sums. Serialise them.
