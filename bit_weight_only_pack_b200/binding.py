@@ -70,6 +70,9 @@ _SIGS = {
     "lbq_debug_gemm_path": ([_c_int], None),
     "lbq_debug_direct_variant": ([_c_int, _c_int], None),
     "lbq_debug_lut3_variant": ([_c_int], None),
+    "lbq_debug_tmma_default": ([_c_int], None),
+    "lbq_debug_tmma_split": ([_c_int], None),
+    "lbq_debug_drop_copies": ([_c_int], None),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -195,8 +198,25 @@ def lbq_debug_force_tc(on):
 
 
 def lbq_debug_gemv_path(path):
-    """Test hook: GEMV kernel for M <= 16 (0 auto, 1 CUDA-core M=1, 2 warp MMA, 3 tcgen05)."""
+    """Test hook: GEMV kernel for M <= 16 (0 auto, 1 CUDA-core M=1, 2 warp MMA, 3 tcgen05,
+    4 direct-load CUDA-core M=1, 5 TMA-fed warp-MMA M=1)."""
     _lib.lbq_debug_gemv_path(path)
+
+
+def lbq_debug_tmma_default(mode):
+    """Test hook: when the TMA-fed warp-MMA kernel is the batch-1 choice (0 never, 1 always,
+    2 launches of >= 4 16-row tiles per SM with K <= 4096)."""
+    _lib.lbq_debug_tmma_default(int(mode))
+
+
+def lbq_debug_drop_copies(on):
+    """Test hook: TMA-fed GEMV launches issue no copies, so their bounded waits run out."""
+    _lib.lbq_debug_drop_copies(1 if on else 0)
+
+
+def lbq_debug_tmma_split(r):
+    """Test hook: force the TMA-fed kernel's K split into r in {1, 2, 4} ranges (0 = its own choice)."""
+    _lib.lbq_debug_tmma_split(r)
 
 
 def lbq_debug_direct_variant(variant, ctas_per_sm=0):

@@ -15,6 +15,7 @@
 #include <map>
 #include <mutex>
 #include <string>
+#include <tuple>
 
 #include "common.cuh"
 #include "pack_int4.cuh"
@@ -26,6 +27,7 @@
 #include "gemm_tc.cuh"
 #include "tc_gemv.cuh"
 #include "gemv_direct.cuh"
+#include "gemv_tmma.cuh"
 #include "gemv_dmma.cuh"
 #include "mxfp8.cuh"
 #include "gemm_ts.cuh"
@@ -156,7 +158,7 @@ static int g_force_skinny = 0;  // test hook: route M = 1 to the tensor-core ski
 // TMA-pipelined CUDA-core M = 1 kernel, 2 = the warp-MMA skinny kernel, 3 = the
 // tcgen05 kernel, 4 = the direct-load CUDA-core M = 1 kernel.
 static int g_gemv_path = 0;
-enum { kPathAuto = 0, kPathM1 = 1, kPathMma = 2, kPathTc = 3, kPathDirect = 4 };
+enum { kPathAuto = 0, kPathM1 = 1, kPathMma = 2, kPathTc = 3, kPathDirect = 4, kPathTmma = 5 };
 
 constexpr int kM1RingBudget = 100 * 1024;
 constexpr int kM1MaxChunksPerSplit = 128;  // K-slices of at most 4096 k keep a ring slot near 20 KB
@@ -585,6 +587,210 @@ static lbq_status run_direct(const lbq_gemv_item* items, int count, int K, int g
   return launch_kernel_ex(fn, dim3(grid), dim3(T), smem, st, g_pdl != 0, args, "direct GEMV launch");
 }
 
+// ----------------------------------------------------------------------------
+// M = 1: TMA-fed warp-MMA GEMV
+// ----------------------------------------------------------------------------
+
+// Tensor maps are encoded on the host; a decode step reuses the same images
+// every step, so each (base, shape, box) is encoded once.
+static bool cached_tmap_2d(CUtensorMap* out, const void* base, CUtensorMapDataType dt, int elem, uint64_t cols,
+                           uint64_t rows, uint64_t row_stride, uint32_t box_cols, uint32_t box_rows,
+                           CUtensorMapSwizzle swz) {
+  struct Key {
+    uintptr_t base;
+    uint64_t cols, rows, stride;
+    uint32_t bc, br;
+    int dt, swz;
+    bool operator<(const Key& o) const {
+      return std::tie(base, cols, rows, stride, bc, br, dt, swz) <
+             std::tie(o.base, o.cols, o.rows, o.stride, o.bc, o.br, o.dt, o.swz);
+    }
+  };
+  struct Entry {
+    alignas(64) CUtensorMap map;
+  };
+  static std::mutex mu;
+  static std::map<Key, Entry> cache;
+  const Key k{reinterpret_cast<uintptr_t>(base), cols, rows, row_stride, box_cols, box_rows, (int)dt, (int)swz};
+  std::lock_guard<std::mutex> lk(mu);
+  auto itc = cache.find(k);
+  if (itc != cache.end()) {
+    *out = itc->second.map;
+    return true;
+  }
+  Entry e;
+  if (!make_tmap_2d(&e.map, base, dt, elem, cols, rows, row_stride, box_cols, box_rows, swz)) return false;
+  if (cache.size() >= 8192) cache.clear();
+  cache.emplace(k, e);
+  *out = e.map;
+  return true;
+}
+
+// The codes [N][K/2] viewed as [K/256 slices][N rows][128 bytes] (row stride
+// K/2, slice stride 128), box 128 x 16 rows x nsl slices, 128-byte swizzle.
+static bool cached_tmap_3d(CUtensorMap* out, const void* base, uint64_t N, uint64_t K, uint32_t nsl) {
+  struct Key {
+    uintptr_t base;
+    uint64_t N, K;
+    uint32_t nsl;
+    bool operator<(const Key& o) const { return std::tie(base, N, K, nsl) < std::tie(o.base, o.N, o.K, o.nsl); }
+  };
+  struct Entry {
+    alignas(64) CUtensorMap map;
+  };
+  static std::mutex mu;
+  static std::map<Key, Entry> cache;
+  const Key k{reinterpret_cast<uintptr_t>(base), N, K, nsl};
+  std::lock_guard<std::mutex> lk(mu);
+  auto itc = cache.find(k);
+  if (itc != cache.end()) {
+    *out = itc->second.map;
+    return true;
+  }
+  Entry e;
+  if (!make_tmap_3d(&e.map, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, N, K / 256, K / 2, 128, 128, kTmRows, nsl,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return false;
+  if (cache.size() >= 8192) cache.clear();
+  cache.emplace(k, e);
+  *out = e.map;
+  return true;
+}
+
+struct TmPlan {
+  int R, nsl, krg, row_tiles, grid, stages, stage_bytes, s_off, z_off, smem, block, max_units;
+  size_t ws, cnt_off;
+};
+
+static int max_dynamic_smem() {
+  static int optin = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  });
+  return optin;
+}
+
+// K is cut into R ranges of nsl 256-k slices (one consumer warp each, at most
+// 16): the smallest R in {1, 2, 4} that fits (one CTA per SM, a fixed range per
+// CTA). Several GEMVs in one launch keep R = 1 (no workspace).
+static int g_tmma_split = 0;  // test hook: force the number of K-ranges (0 = the plan's choice)
+static int g_debug_drop = 0;  // test hook: the TMA GEMV's producer issues nothing (its waits must give up)
+
+static TmPlan plan_tmma(int K, const int* Ns, int count, int group, bool asym, bool allow_split = true) {
+  TmPlan p{};
+  const int chunks = K / 32;
+  for (int i = 0; i < count; ++i) p.row_tiles += (Ns[i] + kTmRows - 1) / kTmRows;
+  const int sms = num_sms();
+  // the fewest ranges that fit: each range's CTA pays a fixed cost per unit
+  // and the split adds a workspace pass, which balance rarely repays
+  for (int R = 1; R <= 4; R *= 2) {
+    if ((count > 1 || !allow_split) && R > 1) break;
+    if (g_tmma_split > 0 && R != g_tmma_split && !((count > 1 || !allow_split) && R == 1)) continue;
+    const int nsl = (chunks + 8 * R - 1) / (8 * R);
+    if (nsl > kTmMaxSlices || (R - 1) * nsl * 8 >= chunks) continue;  // no range may be empty
+    p.R = R;
+    p.nsl = nsl;
+    break;
+  }
+  if (p.nsl == 0) return p;
+  p.krg = p.nsl * 256 / group;
+  p.grid = p.R * std::max(1, std::min(p.row_tiles, sms / p.R));
+  p.s_off = p.nsl * kTmSliceBytes;
+  p.z_off = (int)align_up((size_t)p.s_off + (size_t)p.krg * 32, 128);
+  p.stage_bytes = (int)align_up(asym ? (size_t)p.z_off + (size_t)p.krg * 16 : (size_t)p.z_off, 1024);
+  const int cpk = p.grid / p.R;
+  p.max_units = (p.row_tiles + cpk - 1) / cpk;
+  const int avail = max_dynamic_smem() - 2 * kTmMaxStages * 8 - 1024;
+  const int red_bytes = p.max_units * p.nsl * 16 * 4 + p.max_units * 4;
+  int S = kTmMaxStages;
+  while (S >= 2 && S * p.stage_bytes + red_bytes > avail) --S;
+  p.stages = S;
+  p.smem = 1024 + S * p.stage_bytes + red_bytes;
+  p.block = (p.nsl + 1) * 32;
+  if (p.R > 1) {
+    p.cnt_off = align_up((size_t)p.R * Ns[0] * sizeof(float), 256);
+    p.ws = p.cnt_off + align_up((size_t)p.row_tiles * sizeof(unsigned), 256);
+  }
+  return p;
+}
+
+// Shapes the TMA-fed kernel takes: a 16-row box of codes and whole 256-k
+// slices must fit the matrix; several GEMVs per launch need K <= 4096 (one
+// range, no workspace).
+static bool tmma_ok(int M, int K, const int* Ns, int count) {
+  if (M != 1 || K < 256 || K > 16384 || K % 256) return false;
+  if (count > 1 && K > 32 * 8 * kTmMaxSlices) return false;
+  for (int i = 0; i < count; ++i)
+    if (Ns[i] < kTmRows) return false;
+  return true;
+}
+
+static const void* tmma_kernel(bool bf16, bool asym, int gshift) {
+#define LBQ_TMK(GS)                                                                                        \
+  (bf16 ? (asym ? (const void*)gemv_tmma_kernel<true, true, GS> : (const void*)gemv_tmma_kernel<true, false, GS>)   \
+        : (asym ? (const void*)gemv_tmma_kernel<false, true, GS> : (const void*)gemv_tmma_kernel<false, false, GS>))
+  return gshift == 0 ? LBQ_TMK(0) : gshift == 1 ? LBQ_TMK(1) : LBQ_TMK(2);
+#undef LBQ_TMK
+}
+
+static lbq_status run_tmma(const lbq_gemv_item* items, int count, int K, int group, int mode, bool xbf16, bool ybf16,
+                           void* ws, size_t ws_bytes, cudaStream_t st, bool allow_split = true) {
+  const bool asym = mode == LBQ_MODE_ASYM;
+  if (count < 1 || count > kTmMaxItems) return fail(LBQ_ERR_INVALID_ARG, "count=%d not in 1..%d", count, kTmMaxItems);
+  int Ns[kTmMaxItems];
+  for (int i = 0; i < count; ++i) Ns[i] = items[i].N;
+  const TmPlan p = plan_tmma(K, Ns, count, group, asym, allow_split);
+  if (p.nsl == 0 || p.stages < 2) return fail(LBQ_ERR_UNSUPPORTED, "no TMA GEMV plan for K=%d", K);
+  GemvTmmaArgs a{};
+  GemvTmmaMaps m;
+  std::memset(&m, 0, sizeof(m));
+  int tiles = 0;
+  for (int i = 0; i < count; ++i) {
+    const Layout L = make_layout(K, items[i].N, group, mode);
+    const uint8_t* img = static_cast<const uint8_t*>(items[i].image);
+    const uint64_t meta_rows = (uint64_t)((items[i].N + 127) / 128) * (uint64_t)(K / group);
+    if (!cached_tmap_3d(&m.q[i], img + L.off0, (uint64_t)items[i].N, (uint64_t)K, (uint32_t)p.nsl) ||
+        !cached_tmap_2d(&m.s[i], img + L.off1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, 128, meta_rows, 256, 16,
+                        (uint32_t)p.krg, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        (asym && !cached_tmap_2d(&m.z[i], img + L.off2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, meta_rows, 128, 16,
+                                 (uint32_t)p.krg, CU_TENSOR_MAP_SWIZZLE_NONE)))
+      return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the GEMV image %d", i);
+    a.X[i] = static_cast<const uint16_t*>(items[i].X);
+    a.Y[i] = items[i].Y;
+    a.N[i] = items[i].N;
+    tiles += (items[i].N + kTmRows - 1) / kTmRows;
+    a.rt_end[i] = tiles;
+  }
+  if (p.R > 1) {
+    if (!ws || ws_bytes < p.ws || !aligned16(ws))
+      return fail(LBQ_ERR_INVALID_ARG, "workspace of %zu bytes (16-byte aligned) needed, got %zu", p.ws, ws_bytes);
+    a.partials = static_cast<float*>(ws);
+    a.counters = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + p.cnt_off);
+  }
+  a.items = count;
+  a.K = K;
+  a.G = K / group;
+  a.gshift = group == 32 ? 0 : group == 64 ? 1 : 2;
+  a.R = p.R;
+  a.nsl = p.nsl;
+  a.krg = p.krg;
+  a.row_tiles = p.row_tiles;
+  a.stages = p.stages;
+  a.stage_bytes = p.stage_bytes;
+  a.s_off = p.s_off;
+  a.z_off = p.z_off;
+  a.max_units = p.max_units;
+  a.y_bf16 = ybf16 ? 1 : 0;
+  a.debug_drop = g_debug_drop;
+  const void* fn = tmma_kernel(xbf16, asym, a.gshift);
+  occupancy_for(fn, p.block, p.smem);  // raises the kernel's dynamic shared-memory limit once
+  void* args[] = {&m, &a};
+  return launch_kernel_ex(fn, dim3(p.grid), dim3(p.block), p.smem, st, g_pdl != 0, args, "TMA GEMV launch");
+}
+
 // The kernel lbq_gemv runs for M <= 16. Measured on B200: at M = 1 the
 // direct-load CUDA-core kernel is the fastest at every size it supports
 // (K <= 16384; the warp-MMA kernel spends an MMA, 7/8 wasted, per 256 weights
@@ -592,13 +798,33 @@ static lbq_status run_direct(const lbq_gemv_item* items, int count, int K, int g
 // The tcgen05 kernel is slower at every batch size here (a 128 x 16 x N MMA
 // costs the same ~185 cycles for N = 16 as for N = 256), so it is never the
 // default.
-static int gemv_path(int M, int K, long long weights) {
+// When the TMA-fed warp-MMA kernel is the M = 1 choice: 2 (the default) for
+// launches of at least kTmmaMinTilesPerSm 16-row tiles per SM with K <= 4096,
+// where it was measured faster than the staged CUDA-core kernel (the gate/up
+// launch of the decode step: 4.74 against 4.32 TB/s; the step 1078 against
+// 1127 us); smaller launches and longer K stay on the staged kernel, which
+// starts streaming sooner. Test hook values: 0 never, 1 always.
+static int g_tmma_default = 2;
+constexpr int kTmmaMinTilesPerSm = 4;
+
+static bool tmma_preferred(int K, const int* Ns, int count) {
+  if (g_tmma_default == 1) return true;
+  if (g_tmma_default != 2) return false;
+  int tiles = 0;
+  for (int i = 0; i < count; ++i) tiles += (Ns[i] + 15) / 16;
+  return K <= 4096 && tiles >= kTmmaMinTilesPerSm * num_sms();
+}
+
+static int gemv_path(int M, int K, int N) {
+  const long long weights = (long long)K * N;
   const bool direct_ok = M == 1 && K <= 32 * 32 * kGdMaxWarps;
+  if (g_gemv_path == kPathTmma && tmma_ok(M, K, &N, 1)) return kPathTmma;
   if (g_gemv_path == kPathM1 && M == 1) return kPathM1;
   if (g_gemv_path == kPathDirect && direct_ok) return kPathDirect;
   if (g_gemv_path == kPathMma || g_gemv_path == kPathTc) return g_gemv_path;
   if (g_force_skinny) return kPathMma;
   if (M == 1 && g_force_splits) return kPathM1;
+  if (M == 1 && g_gemv_path == kPathAuto && tmma_preferred(K, &N, 1) && tmma_ok(M, K, &N, 1)) return kPathTmma;
   if (M == 1) return direct_ok ? kPathDirect : (weights < (1LL << 27) ? kPathM1 : kPathMma);
   return kPathMma;
 }
@@ -611,8 +837,17 @@ struct GemvScratch {
 
 static GemvScratch gemv_scratch(int M, int K, int N, int group, bool asym, bool xbf16) {
   GemvScratch g{0, 0, 0};
-  const int path = gemv_path(M, K, (long long)K * N);
+  const int path = gemv_path(M, K, N);
   if (path == kPathDirect) return g;
+  if (path == kPathTmma) {
+    const TmPlan p = plan_tmma(K, &N, 1, group, asym);
+    g.need = p.ws;
+    if (g.need) {
+      g.cnt_off = p.cnt_off;
+      g.cnt_bytes = (size_t)p.row_tiles * sizeof(unsigned);
+    }
+    return g;
+  }
   if (path == kPathM1) {
     const M1Plan p = plan_m1(K, N, group, asym, g_force_splits);
     g.need = p.block == 0 ? 0 : m1_workspace_bytes(p, N);
@@ -902,8 +1137,24 @@ void lbq_debug_gemm_path(int path) { g_gemm_path = path == 1 ? 1 : 0; }
 
 // Test hook (not in the public header): pick the GEMV kernel for M <= 16
 // (0 = the library's choice, 1 = TMA-pipelined CUDA-core M = 1, 2 = warp MMA,
-// 3 = tcgen05, 4 = direct-load CUDA-core M = 1).
-void lbq_debug_gemv_path(int path) { g_gemv_path = (path >= 0 && path <= 4) ? path : 0; }
+// 3 = tcgen05, 4 = direct-load CUDA-core M = 1, 5 = TMA-fed warp-MMA M = 1).
+void lbq_debug_gemv_path(int path) { g_gemv_path = (path >= 0 && path <= 5) ? path : 0; }
+
+// Test hook (not in the public header): when the TMA-fed warp-MMA kernel is
+// the batch-1 choice: 0 never, 1 always, 2 (and any other value: the library's
+// default) for launches of at least 4 16-row tiles per SM with K <= 4096.
+void lbq_debug_tmma_default(int mode) { g_tmma_default = (mode >= 0 && mode <= 2) ? mode : 2; }
+
+// Test hook (not in the public header): force the TMA-fed kernel's K split
+// (1, 2 or 4 ranges; 0 = the plan's choice). A forced split that the shape
+// cannot take leaves the kernel without a plan (the call then fails).
+void lbq_debug_tmma_split(int r) { g_tmma_split = (r == 1 || r == 2 || r == 4) ? r : 0; }
+
+// Test hook (not in the public header): the next TMA-fed GEMV launches issue
+// no copies, so every consumer wait runs out (after a short spin limit); the
+// kernel returns without writing Y and raises the device flag that
+// lbq_device_status() reports. No copy is in flight when the CTA exits.
+void lbq_debug_drop_copies(int on) { g_debug_drop = on ? 1 : 0; }
 
 // Test hook (not in the public header): direct batch-1 kernel variant
 // (-1 = the library's choice, 0 = weights pipelined through registers,
@@ -1016,9 +1267,12 @@ lbq_status lbq_gemv(const void* X, int x_dtype, int M, int K, int N, int group, 
   if (M > 16) return fail(LBQ_ERR_UNSUPPORTED, "lbq_gemv takes M <= 16 (M=%d); use lbq_gemm", M);
   const Layout L = make_layout(K, N, group, mode);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int path = gemv_path(M, K, (long long)K * N);
-  if (path == kPathDirect) {
+  const int path = gemv_path(M, K, N);
+  if (path == kPathDirect || path == kPathTmma) {
     const lbq_gemv_item item{X, image, Y, N};
+    if (path == kPathTmma)
+      return run_tmma(&item, 1, K, group, mode, x_dtype == LBQ_DTYPE_BF16, y_dtype == LBQ_DTYPE_BF16, ws, ws_bytes,
+                      s);
     return run_direct(&item, 1, K, group, mode, x_dtype == LBQ_DTYPE_BF16, y_dtype == LBQ_DTYPE_BF16, s);
   }
   if (path == kPathM1)
@@ -1135,6 +1389,14 @@ lbq_status lbq_gemv_grouped(const lbq_gemv_item* items, int count, int K, int gr
     if (st != LBQ_OK) return st;
     if ((st = check_compute_args(items[i].X, x_dtype, 1, items[i].image, items[i].Y, y_dtype)) != LBQ_OK) return st;
   }
+  int Ns[kGdMaxItems];
+  for (int i = 0; i < count; ++i) Ns[i] = items[i].N;
+  const bool tmma = (g_gemv_path == kPathTmma || (g_gemv_path == kPathAuto && tmma_preferred(K, Ns, count))) &&
+                    tmma_ok(1, K, Ns, count) && count <= kTmMaxItems &&
+                    plan_tmma(K, Ns, count, group, mode == LBQ_MODE_ASYM, false).nsl > 0;
+  if (tmma)
+    return run_tmma(items, count, K, group, mode, x_dtype == LBQ_DTYPE_BF16, y_dtype == LBQ_DTYPE_BF16, nullptr, 0,
+                    static_cast<cudaStream_t>(stream), false);
   return run_direct(items, count, K, group, mode, x_dtype == LBQ_DTYPE_BF16, y_dtype == LBQ_DTYPE_BF16,
                     static_cast<cudaStream_t>(stream));
 }
