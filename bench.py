@@ -418,22 +418,41 @@ def _secondary_measurements(torch, lbq, workloads, device, peaks, quick):
                                     "frac_bf16_sustained": tf / tc_sus}
         del X
     del images
+    # MXFP8 activation quantiser (the activation side of the LUT3 x MXFP8
+    # product): M=2048 K=4096 BF16, 2 bytes read and 1 + 1/32 written per value
+    M, K = 2048, 4096
+    xs = [workloads.activations_device(50 + i, M, K, "bf16", device)
+          for i in range(max(3, 3 * l2_bytes // (M * K * 2) + 1))]
+    codes = torch.empty((M, K), dtype=torch.uint8, device=device)
+    scales = torch.empty((M, K // 32), dtype=torch.uint8, device=device)
+
+    def qcall(X, s):
+        lbq.lbq_quantize_mxfp8(X.data_ptr(), 1, M, K, codes.data_ptr(), scales.data_ptr(), s)
+
+    ms = rotating_ms(torch, qcall, xs, reps=3)
+    b = M * K * 2 + M * K + M * K // 32
+    out["mxfp8_quantize_m2048_k4096"] = {"us": ms * 1e3, "GBps": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm,
+                                         "bytes_per_launch": b, "input_copies": len(xs)}
+    del xs
     return out
 
 
 # ----------------------------------------------------------------------------- CPU baseline (oracle)
 
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count()
+
+
 def oracle_sample(seconds_target, layer=0, max_proj=7):
     """Time the oracle (dequant + FP64 matmul) on the first projections of one
     layer of the decode step, host-generated and quantised outside the timer."""
-    import numpy as np
     import workloads
     from oracle import int4, matmul
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count()
+    cores = _blas_threads()
     done_bytes, spent, names = 0, 0.0, []
     for p, (name, K, N) in enumerate(workloads.LLAMA3_8B_PROJ[:max_proj]):
         seed = workloads.c2_seed(layer, p)
@@ -451,6 +470,62 @@ def oracle_sample(seconds_target, layer=0, max_proj=7):
     return {"value": done_bytes / spent / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": f"layer {layer} projections {'+'.join(names)} of the decode step: exact dequant + FP64 "
                       f"matmul (numpy), {done_bytes} weight bytes in {spent:.2f} s"}
+
+
+def oracle_per_config(column_budget=1024):
+    """The oracle on a bounded sample of every other configuration: a K x
+    min(N, column_budget) weight of the configuration's distribution and seed,
+    dequant + FP64 matmul timed, reported as that configuration's metric
+    (weight-GB/s of the sampled columns; GFLOP/s as well for the GEMMs)."""
+    import workloads
+    from oracle import int4, lut3, matmul
+    out = {}
+
+    def timed(fn):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+    def int4_case(name, seed, K, N, group, mode, Ms, xdt, **kw):
+        n = min(N, column_budget)
+        W = workloads.weights_host(seed, K, n, **kw)
+        q, s, z = int4.quantize(W, group, mode)
+        for M in Ms:
+            X = workloads.activations_host(seed, M, K, xdt)
+            dt = timed(lambda: matmul.matmul_f64(X, int4.dequant(q, s, group, z)))
+            rec = {"columns": n, "seconds": dt, "GBps": int4_bytes(K, n, group, mode) / dt / 1e9}
+            if M > 16:
+                rec["GFLOPs"] = 2.0 * M * K * n / dt / 1e9
+            out[f"{name}_m{M}"] = rec
+
+    int4_case("c1_4096x4096_sym_g32", 0, 4096, 4096, 32, "sym", (1,), "f16")
+    int4_case("c3_8192x28672_sym_g64", 3, 8192, 28672, 64, "sym", (1, 16), "bf16", outlier_frac=1e-3,
+              outlier_mult=20.0)
+    int4_case("c3_8192x28672_sym_g128", 3, 8192, 28672, 128, "sym", (1, 16), "bf16", outlier_frac=1e-3,
+              outlier_mult=20.0)
+    int4_case("c4_4096x14336_asym_g128", 4, 4096, 14336, 128, "asym", (512, 2048), "bf16")
+    K, n = 4096, min(14336, column_budget)
+    idx, cb, ex = workloads.lut3_host(5, K, n)
+    for M in (1, 2048):
+        X = workloads.activations_host(5, M, K, "bf16")
+        dt = timed(lambda: matmul.matmul_f64(X, lut3.dequant(idx, cb, ex)))
+        rec = {"columns": n, "seconds": dt, "GBps": lut3_bytes(K, n) / dt / 1e9}
+        if M > 16:
+            rec["GFLOPs"] = 2.0 * M * K * n / dt / 1e9
+        out[f"c5_4096x14336_lut3_m{M}"] = rec
+    return out
+
+
+def oracle_one_core(seconds_target=4.0):
+    """oracle_sample with the BLAS pool limited to one thread."""
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:
+        return None
+    with threadpool_limits(limits=1):
+        r = oracle_sample(seconds_target, max_proj=7)
+    r["cores"] = 1
+    return r
 
 
 def run_reference(args):
@@ -479,11 +554,7 @@ def run_reference(args):
             total_bytes += int4_bytes(K, N, 32, "asym")
             total_s += dt
     value = total_bytes / total_s / 1e9
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count()
+    cores = _blas_threads()
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_s / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -500,19 +571,31 @@ def run_reference(args):
 # ----------------------------------------------------------------------------- ncu cases
 
 # name -> (K, N, group, mode, x dtype, M, GEMV path or None); the path is the
-# test hook's kernel choice (1 TMA CUDA-core, 2 warp MMA, 3 tcgen05, 4 direct)
+# test hook's kernel choice (1 TMA CUDA-core, 2 warp MMA, 3 tcgen05, 4 direct,
+# 5 TMA-fed warp MMA). A tuple N is one grouped launch of GEMVs sharing X, as
+# the decode step runs q/k/v and gate/up.
 PROFILE_CASES = {
     "c1": (4096, 4096, 32, "sym", "f16", 1, None),
+    "c2qkv": (4096, (4096, 1024, 1024), 32, "asym", "f16", 1, None),
+    "c2o": (4096, 4096, 32, "asym", "f16", 1, None),
+    "c2gateup": (4096, (14336, 14336), 32, "asym", "f16", 1, None),
     "c2gate": (4096, 14336, 32, "asym", "f16", 1, None),
     "c2down": (14336, 4096, 32, "asym", "f16", 1, None),
     "c2kv": (4096, 1024, 32, "asym", "f16", 1, None),
     "c2gate_mma": (4096, 14336, 32, "asym", "f16", 1, 2),
+    "c2gate_direct": (4096, 14336, 32, "asym", "f16", 1, 4),
+    "c2gate_tmma": (4096, 14336, 32, "asym", "f16", 1, 5),
+    "c2o_tmma": (4096, 4096, 32, "asym", "f16", 1, 5),
+    "c2down_tmma": (14336, 4096, 32, "asym", "f16", 1, 5),
     "c2gate_regs": (4096, 14336, 32, "asym", "f16", 1, 4, 0),  # batch-1 kernel variant: weights in registers
     "c3m1": (8192, 28672, 128, "sym", "bf16", 1, None),
     "c3m16": (8192, 28672, 128, "sym", "bf16", 16, None),
+    "c4m512": (4096, 14336, 128, "asym", "bf16", 512, None),
     "c4m2048": (4096, 14336, 128, "asym", "bf16", 2048, None),
     "c5m1": (4096, 14336, 0, "lut3", "bf16", 1, None),
+    "c5m16": (4096, 14336, 0, "lut3", "bf16", 16, None),
     "c5m2048": (4096, 14336, 0, "lut3", "bf16", 2048, None),
+    "mxfp8q": (4096, 0, 0, "mxfp8", "bf16", 2048, None),
 }
 
 
@@ -526,16 +609,32 @@ def run_profile_case(name):
     variant = PROFILE_CASES[name][7] if len(PROFILE_CASES[name]) > 7 else None
     device = torch.device("cuda", 0)
     torch.cuda.set_device(0)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    if mode == "mxfp8":
+        # activation quantiser: copies of X larger than L2 in total
+        xs = [workloads.activations_device(7 + i, M, K, xdt, device)
+              for i in range(max(3, 3 * l2 // (M * K * 2) + 1))]
+        for X in xs:
+            lbq.quantize_mxfp8(X)
+        torch.cuda.synchronize()
+        lbq.device_status()
+        print(f"profile case {name}: {len(xs)} launches of M={M} K={K}", flush=True)
+        return 0
+    Ns = N if isinstance(N, tuple) else (N,)
     if mode == "lut3":
         idx, cb, ex = workloads.lut3_device(7, K, N, device)
         img0 = lbq.pack_lut3(idx, cb, ex)
         del idx, cb, ex
+        img0s = [img0]
     else:
-        W = workloads.weights_device(7, K, N, device)
-        img0 = lbq.pack(W, group, mode)
-        del W
-    l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    images = weight_copies(img0, l2)
+        img0s = []
+        for i, n in enumerate(Ns):
+            W = workloads.weights_device(7 + i, K, n, device)
+            img0s.append(lbq.pack(W, group, mode))
+            del W
+    per_launch = sum(int(i.numel()) for i in img0s)
+    copies = max(3, (3 * l2) // per_launch + 1)
+    sets = [img0s] + [[i.clone() for i in img0s] for _ in range(copies - 1)]
     X = workloads.activations_device(7, M, K, xdt, device)
     if path is not None:
         lbq.lbq_debug_gemv_path(path)
@@ -543,52 +642,83 @@ def run_profile_case(name):
         lbq.lbq_debug_direct_variant(variant)
     if mode == "lut3":
         ws = lbq.workspace(2, M, K, N, 0, "lut3")
-        for img in images:
-            lbq.lut3_gemm(X, img, N, ws=ws)
+        for imgs in sets:
+            lbq.lut3_gemm(X, imgs[0], N, ws=ws)
+    elif len(Ns) > 1:
+        for imgs in sets:
+            lbq.gemv_grouped([(X, img, n) for img, n in zip(imgs, Ns)], group, mode)
     else:
         ws = lbq.workspace(1, M, K, N, group, mode)
-        for img in images:
-            lbq.gemm(X, img, N, group, mode, ws=ws)
+        for imgs in sets:
+            lbq.gemm(X, imgs[0], N, group, mode, ws=ws)
     torch.cuda.synchronize()
     lbq.lbq_debug_gemv_path(0)
     lbq.lbq_debug_direct_variant(-1)
     lbq.device_status()
-    print(f"profile case {name}: {len(images)} launches of K={K} N={N} {mode} M={M}", flush=True)
+    print(f"profile case {name}: {len(sets)} launches of K={K} N={N} {mode} M={M}", flush=True)
     return 0
 
 
 # ----------------------------------------------------------------------------- main
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) from ncu captures
-# summarised under profiles/, with a hash of the kernel sources at capture time:
-# name -> (bytes, {source file: sha256[:16]}, summary file).
-NCU_TRAFFIC = {
-    # mean DRAM bytes per launch of the decode step (all gemv_direct_async_kernel)
-    "decode_step_per_launch": (32426732, {"gemv_direct.cuh": "80c3d5258f32c480", "common.cuh": "eb93cb6f87fb3da4",
-                                          "lbq.cu": "18ec92ef2e5d8cd1"},
-                               "profiles/decode_step_launch_list.md"),
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# decode step's four launch shapes (q/k/v grouped, o, gate/up grouped, down),
+# each from a one-launch ncu capture of its profile case summarised under
+# profiles/, with hashes of the kernel's sources and of its planner at capture
+# time: shape -> (bytes, {source: sha256[:16]}, summary file). Each shape runs
+# once per layer, so the step's traffic per launch is their mean.
+STEP_KERNEL = ("gemv_tmma_kernel (gate/up) and gemv_direct_async_kernel (q/k/v, o, down)")
+STEP_SOURCES = ("gemv_tmma.cuh", "gemv_direct.cuh", "gemv_m1.cuh", "tma.cuh", "common.cuh", "lbq.cu#tmma-plan",
+                "lbq.cu#direct-plan")
+STEP_CAPTURE_HASHES = {
+    "gemv_tmma.cuh": "d81c29e83ca35ffb",
+    "gemv_direct.cuh": "80c3d5258f32c480",
+    "gemv_m1.cuh": "a992f85dd1acbd76",
+    "tma.cuh": "fc6224a6c6bf092f",
+    "common.cuh": "eb93cb6f87fb3da4",
+    "lbq.cu#tmma-plan": "e30dce5cede0f3f4",
+    "lbq.cu#direct-plan": "7afca7967200d200",
 }
+STEP_TRAFFIC = {
+    "c2qkv": (14980864, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
+    "c2o": (9997312, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
+    "c2gateup": (70369536, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
+    "c2down": (34921728, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
+}
+# the planner sections of lbq.cu (kernel choice, launch shape, K split, stages)
+PLAN_MARKERS = {"tmma-plan": ("// M = 1: TMA-fed warp-MMA GEMV", "// Scratch of that kernel for one call"),
+                "direct-plan": ("static lbq_status run_direct(", "// ----------------------------------------------------------------------------\n// M = 1: TMA-fed")}
 
 
 def source_hash(name):
+    """sha256[:16] of a kernel source, or of the marked planner section of lbq.cu."""
     import hashlib
-    with open(os.path.join(ROOT, "bit_weight_only_pack_b200", "csrc", name), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    fname, _, section = name.partition("#")
+    with open(os.path.join(ROOT, "bit_weight_only_pack_b200", "csrc", fname), "rb") as f:
+        data = f.read()
+    if section:
+        a, b = (m.encode() for m in PLAN_MARKERS[section])
+        i, j = data.find(a), data.find(b)
+        if i < 0 or j < i:
+            return None
+        data = data[i:j]
+    return hashlib.sha256(data).hexdigest()[:16]
 
 
-def traffic_from_profiles(name):
-    """The recorded DRAM bytes for `name`, or None when there is no record or a
-    kernel source changed since the capture."""
-    rec = NCU_TRAFFIC.get(name)
-    if rec is None:
-        return None
-    nbytes, sources, _summary = rec
-    if nbytes is None:
-        return None
-    try:
-        return nbytes if all(source_hash(f) == h for f, h in sources.items()) else None
-    except OSError:
-        return None
+def current_hashes():
+    return {f: source_hash(f) for f in STEP_SOURCES}
+
+
+def traffic_from_profiles():
+    """Mean recorded DRAM bytes per launch of the step, or None when a shape has
+    no record or a kernel source or the planner changed since its capture."""
+    vals = []
+    now = current_hashes()
+    for nbytes, sources, _summary in STEP_TRAFFIC.values():
+        if nbytes is None or sources != now:
+            return None
+        vals.append(nbytes)
+    return sum(vals) / len(vals)
 
 
 def main():
@@ -648,13 +778,13 @@ def main():
     x_host.copy_(step.x_all.cpu())
     y_host = torch.empty_like(step.y_all, device="cpu").pin_memory()
     lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 0 if args.no_pdl else 1)
-    launches_before = lbq.lbq_launch_count()
     for _ in range(args.warmup):
         step.x_all.copy_(x_host, non_blocking=True)
         step.launch_all()
         y_host.copy_(step.y_all, non_blocking=True)
     torch.cuda.synchronize()
     barrier(world)
+    launches_before = lbq.lbq_launch_count()  # the timed steps' launches only
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
@@ -670,17 +800,23 @@ def main():
 
     secondary = None
     if not args.no_secondary:
+        sec_sampler = ClockSampler(physical_gpu_index(local))
+        sec_sampler.start()
+        time.sleep(0.25)
         secondary = secondary_measurements(torch, lbq, workloads, device, peaks, args.quick)
+        secondary["clocks"] = sec_sampler.stop()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample(10.0)
+        cpu["one_core"] = oracle_one_core(4.0)
+        cpu["per_config"] = oracle_per_config()
 
     hbm = peaks["hbm_gbs"]
     per_gpu = step.bytes / (ms_per_step / 1e3) / 1e9
     launches = step.launches_per_step
     # DRAM bytes per launch of the step from an ncu capture (see profiles/), for the default step only
-    traffic = traffic_from_profiles("decode_step_per_launch") if (args.layers == 32 and not args.ungrouped) else None
+    traffic = traffic_from_profiles() if (args.layers == 32 and not args.ungrouped) else None
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -700,11 +836,12 @@ def main():
         "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": hbm, "unit": "GB/s", "frac": per_gpu / hbm,
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peaks["source"],
                      "traffic": traffic,
-                     "kernel": "gemv_direct_async_kernel (every launch of the step)",
+                     "kernel": STEP_KERNEL,
                      "per_launch": "algorithmic bytes per launch averaged over the step's %d launches (%.0f B) / "
                                    "average launch time (step time / launches); traffic = ncu DRAM read+write "
-                                   "bytes per launch, averaged the same way, null if the kernel source changed "
-                                   "since the capture" % (launches, step.bytes / max(launches, 1)),
+                                   "bytes per launch of the step's four launch shapes (one-launch captures), "
+                                   "their mean; null if the kernel or its planner changed since the capture"
+                                   % (launches, step.bytes / max(launches, 1)),
                      "algorithmic_bytes_per_step": step.bytes},
         "clocks": clocks,
         "e2e": {"value": world * step.bytes / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",

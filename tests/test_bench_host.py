@@ -112,3 +112,41 @@ def test_profile_summaries_name_commands_that_exist():
             for flag in re.findall(r"(--[a-z-]+)", cmd):
                 assert flag in ("--profile", "--steps", "--warmup", "--no-secondary", "--no-cpu-baseline",
                                 "--gpus", "--impl", "--quick", "--ungrouped", "--no-pdl", "--layers"), (path, flag)
+
+
+def test_profile_commands_stay_within_the_capture_rules():
+    """Every ncu command under profiles/ either records launch times only
+    (gpu__time_duration.sum) or captures one kernel (-k) for at most three
+    launches (-c); none collects more over a whole run."""
+    import glob
+    import re
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        text = open(path).read().replace("\\\n", " ")
+        for cmd in re.findall(r"^\s*ncu [^\n`]*", text, flags=re.M):
+            assert "--clock-control none" in cmd, (path, cmd)
+            m = re.search(r"--metrics (\S+)", cmd)
+            times_only = m is not None and m.group(1) == "gpu__time_duration.sum" and "--set" not in cmd \
+                and "--section" not in cmd
+            if times_only:
+                continue
+            assert re.search(r"-k (regex:)?\S+", cmd), (path, cmd)
+            c = re.search(r"-c (\d+)", cmd)
+            assert c and int(c.group(1)) <= 3, (path, cmd)
+
+
+def test_step_traffic_records_are_consistent():
+    """The decode step's traffic figure is reported only when every launch
+    shape has a record taken with the current kernel sources and planner, and
+    every record names a committed summary."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert set(bench.STEP_TRAFFIC) == {"c2qkv", "c2o", "c2gateup", "c2down"}
+    for name, (nbytes, sources, summary) in bench.STEP_TRAFFIC.items():
+        assert name in bench.PROFILE_CASES
+        assert os.path.exists(os.path.join(ROOT, summary)) or nbytes is None, summary
+        if nbytes is not None:
+            assert set(sources) == set(bench.STEP_SOURCES)
+    now = bench.current_hashes()
+    assert all(v is not None for v in now.values())
+    complete = all(r[0] is not None and r[1] == now for r in bench.STEP_TRAFFIC.values())
+    assert (bench.traffic_from_profiles() is not None) == complete
