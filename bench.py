@@ -418,6 +418,28 @@ def _secondary_measurements(torch, lbq, workloads, device, peaks, quick):
                                     "frac_bf16_sustained": tf / tc_sus}
         del X
     del images
+    # LUT3 x MXFP8 on the block-scaled FP8 tensor path, M=2048 (activations
+    # already in MXFP8: codes + scales), against an FP8 peak of 2x the BF16 one
+    # (the FP8 dense rate is twice the BF16 rate on this GPU; only BF16 is measured)
+    idx, cb, ex = workloads.lut3_device(5, K, N, device)
+    images = weight_copies(lbq.pack_lut3(idx, cb, ex), l2_bytes)
+    del idx, cb, ex
+    for M in (2048, 8192):
+        codes_h, scales_h = workloads.mx_activations_host(60 + M, M, K)
+        codes, scales = torch.from_numpy(codes_h).to(device), torch.from_numpy(scales_h).to(device)
+        Ymx = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+
+        def mxcall(img, s):
+            lbq.lbq_lut3_mx_gemm(codes.data_ptr(), scales.data_ptr(), M, K, N, img.data_ptr(), Ymx.data_ptr(), 1, s)
+
+        ms = rotating_ms(torch, mxcall, images, reps=3)
+        tf = 2.0 * M * K * N / ms / 1e9
+        out[f"c5_lut3_mxfp8_m{M}"] = {"us": ms * 1e3, "TFLOPs": tf, "frac_fp8_peak": tf / (2 * tc_peak),
+                                      "fp8_peak_tflops": 2 * tc_peak,
+                                      "fp8_peak_source": "2 x the BF16 figure (%s)" % peaks["source"],
+                                      "frac_bf16_peak": tf / tc_peak}
+        del codes, scales, Ymx
+    del images
     # MXFP8 activation quantiser (the activation side of the LUT3 x MXFP8
     # product): M=2048 K=4096 BF16, 2 bytes read and 1 + 1/32 written per value
     M, K = 2048, 4096
@@ -596,6 +618,7 @@ PROFILE_CASES = {
     "c5m16": (4096, 14336, 0, "lut3", "bf16", 16, None),
     "c5m2048": (4096, 14336, 0, "lut3", "bf16", 2048, None),
     "mxfp8q": (4096, 0, 0, "mxfp8", "bf16", 2048, None),
+    "c5mx2048": (4096, 14336, 0, "lut3mx", "mxfp8", 2048, None),
 }
 
 
@@ -619,6 +642,19 @@ def run_profile_case(name):
         torch.cuda.synchronize()
         lbq.device_status()
         print(f"profile case {name}: {len(xs)} launches of M={M} K={K}", flush=True)
+        return 0
+    if mode == "lut3mx":
+        # LUT3 x MXFP8: activations drawn in the format, weight copies larger than L2
+        idx, cb, ex = workloads.lut3_device(7, K, N, device)
+        images = weight_copies(lbq.pack_lut3(idx, cb, ex), l2)
+        del idx, cb, ex
+        codes_h, scales_h = workloads.mx_activations_host(7, M, K)
+        codes, scales = torch.from_numpy(codes_h).to(device), torch.from_numpy(scales_h).to(device)
+        for img in images:
+            lbq.lut3_mx_gemm(codes, scales, img, N)
+        torch.cuda.synchronize()
+        lbq.device_status()
+        print(f"profile case {name}: {len(images)} launches of K={K} N={N} M={M}", flush=True)
         return 0
     Ns = N if isinstance(N, tuple) else (N,)
     if mode == "lut3":

@@ -63,6 +63,7 @@ _SIGS = {
     "lbq_gemv_noalloc": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp], _c_int),
     "lbq_gemv_grouped": ([ctypes.POINTER(lbq_gemv_item), _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp], _c_int),
     "lbq_quantize_mxfp8": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
+    "lbq_lut3_mx_gemm": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp], _c_int),
     "lbq_debug_force_splits": ([_c_int], None),
     "lbq_debug_force_skinny": ([_c_int], None),
     "lbq_debug_force_tc": ([_c_int], None),
@@ -183,6 +184,21 @@ def quantize_mxfp8(X):
     scales = torch.empty((M, K // 32), dtype=torch.uint8, device=X.device)
     lbq_quantize_mxfp8(X.data_ptr(), _dt(X), M, K, codes.data_ptr(), scales.data_ptr(), _stream())
     return codes, scales
+
+
+def lbq_lut3_mx_gemm(codes, scales, M, K, N, image, Y, y_dtype, stream):
+    _check(_lib.lbq_lut3_mx_gemm(codes, scales, M, K, N, image, Y, y_dtype, stream))
+
+
+def lut3_mx_gemm(codes, scales, image, N, y_dtype="bf16", Y=None):
+    """Y[M, N] = MXFP8 activations (codes uint8 [M, K], scales uint8 [M, K/32]) . LUT3 weights."""
+    torch = _torch()
+    _need_cuda(codes, scales, image, Y)
+    M, K = codes.shape
+    if Y is None:
+        Y = torch.empty((M, N), dtype={"f16": torch.float16, "bf16": torch.bfloat16}[y_dtype], device=codes.device)
+    lbq_lut3_mx_gemm(codes.data_ptr(), scales.data_ptr(), M, K, N, image.data_ptr(), Y.data_ptr(), _dt(Y), _stream())
+    return Y
 
 
 def lbq_set_option(option, value):

@@ -31,6 +31,7 @@
 #include "gemv_dmma.cuh"
 #include "mxfp8.cuh"
 #include "gemm_ts.cuh"
+#include "gemm_mx.cuh"
 #include "lut3_direct.cuh"
 
 namespace lbq {
@@ -1047,6 +1048,44 @@ static lbq_status run_lut3_gemm_tc(const void* X, int M, const void* image, cons
   return launch_kernel_ex(fn, dim3(grid), dim3(kTcThreads), kTcSmem, st, false, args, "LUT3 GEMM launch");
 }
 
+// ----------------------------------------------------------------------------
+// LUT3 x MXFP8 on the block-scaled FP8 tensor path
+// ----------------------------------------------------------------------------
+
+static lbq_status run_lut3_mx(const uint8_t* codes, const uint8_t* scales, int M, const void* image, const Layout& L,
+                              void* Y, bool ybf16, cudaStream_t st) {
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  const int cb_rows = std::min(16, L.N / 8);
+  CUtensorMap tx, ts, tc, te, ty;
+  if (!make_tmap_2d(&ty, Y, ybf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)L.N,
+                    (uint64_t)M, (uint64_t)L.N * 2, kMxBN, 32, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&tx, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.K, (uint64_t)M, (uint64_t)L.K, kMxBK,
+                    kMxBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&ts, scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.K / 32, (uint64_t)M,
+                    (uint64_t)L.K / 32, 16, kMxBM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&tc, img + L.off1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.s_stride, (uint64_t)L.N / 8,
+                    (uint64_t)L.s_stride, 16, (uint32_t)cb_rows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&te, img + L.off2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.z_stride, (uint64_t)L.N / 8,
+                    (uint64_t)L.z_stride, 16, (uint32_t)cb_rows, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the LUT3 x MXFP8 operands");
+  GemmMxArgs a{};
+  a.Y = Y;
+  a.i_region = img + L.off0;
+  a.M = M;
+  a.N = L.N;
+  a.K = L.K;
+  a.n_tiles = (L.N + kMxBN - 1) / kMxBN;
+  a.m_tiles = (M + kMxBM - 1) / kMxBM;
+  a.k_blocks = L.K / kMxBK;
+  a.cb_rows = cb_rows;
+  a.y_bf16 = ybf16 ? 1 : 0;
+  const void* fn = (const void*)gemm_mx_lut3_kernel;
+  occupancy_for(fn, kMxThreads, kMxSmem);
+  const int grid = std::min(a.n_tiles * a.m_tiles, num_sms());
+  void* args[] = {&tx, &ts, &tc, &te, &ty, &a};
+  return launch_kernel_ex(fn, dim3(grid), dim3(kMxThreads), kMxSmem, st, false, args, "LUT3 x MXFP8 GEMM launch");
+}
+
 static lbq_status check_compute_args(const void* X, int x_dtype, int M, const void* image, void* Y, int y_dtype) {
   if (!X || !image || !Y) return fail(LBQ_ERR_INVALID_ARG, "X, image and Y must be non-null");
   if (!aligned16(X) || !aligned16(image) || !aligned16(Y))
@@ -1445,6 +1484,20 @@ lbq_status lbq_gemv_noalloc(const void* X, int x_dtype, int M, int K, int N, int
   }
   return lbq_gemv(X, x_dtype, M, K, N, group, mode, image, Y, y_dtype, scratch, need ? kNoAllocScratchBytes : 0,
                   stream);
+}
+
+lbq_status lbq_lut3_mx_gemm(const uint8_t* codes, const uint8_t* scales, int M, int K, int N, const void* image,
+                            void* Y, int y_dtype, void* stream) {
+  lbq_status st = check_lut3_shape(K, N);
+  if (st != LBQ_OK) return st;
+  if (K % 512) return fail(LBQ_ERR_UNSUPPORTED, "lbq_lut3_mx_gemm needs K %% 512 == 0 (K=%d)", K);
+  if (M <= 0) return fail(LBQ_ERR_INVALID_ARG, "M=%d must be positive", M);
+  if (!codes || !scales || !image || !Y) return fail(LBQ_ERR_INVALID_ARG, "codes, scales, image and Y must be non-null");
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(image) || !aligned16(Y))
+    return fail(LBQ_ERR_INVALID_ARG, "codes, scales, image and Y must be 16-byte aligned");
+  if (y_dtype != LBQ_DTYPE_F16 && y_dtype != LBQ_DTYPE_BF16) return fail(LBQ_ERR_UNSUPPORTED, "y_dtype %d", y_dtype);
+  return run_lut3_mx(codes, scales, M, image, make_layout(K, N, 0, LBQ_MODE_LUT3), Y, y_dtype == LBQ_DTYPE_BF16,
+                     static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -290,6 +290,29 @@ lbq_status lbq_gemv_noalloc(const void* X, int x_dtype, int M, int K, int N, int
 lbq_status lbq_quantize_mxfp8(const void* X, int x_dtype, int M, int K, uint8_t* codes, uint8_t* scales,
                               void* stream);
 
+/*
+ * LUT3 weights x MXFP8 activations on the block-scaled FP8 tensor path (vLLM
+ * PR 62759 write-up: LUT-B weights with MXFP8 activations, E4M3 elements and
+ * one UE8M0 scale per 1 x 32 block; its format section: the tile's UE8M0
+ * exponent maps onto the weight operand's per-32-k block scale). The decoded
+ * weight of a LUT3 index is its codebook's E4M3 byte, the tile exponent its
+ * block scale, so the product runs as tcgen05.mma.kind::mxf8f6f4.block_scale
+ * with every product exact and FP32 accumulation:
+ *   y[m][n] = sum_k e4m3(codes[m][k]) 2^(scales[m][k/32] - 127)
+ *                   * e4m3(cb[k/64][n/8][idx[k][n]]) 2^(E[k/64][n/8] - 127)
+ *   codes  (device) uint8 [M, K], E4M3 bytes (e.g. from lbq_quantize_mxfp8)
+ *   scales (device) uint8 [M, K/32], UE8M0 bytes
+ *   image  (device) from lbq_pack_lut3 with this K, N
+ *   Y      (device) [M, N] row-major, y_dtype, fully overwritten
+ * K % 512 == 0 (the block scales are read 16 bytes, 512 k, at a time), N % 8
+ * == 0, M >= 1; every pointer 16-byte aligned. NaN codes (0x7F / 0xFF) or scale
+ * bytes (0xFF) give NaN outputs. Errors: LBQ_ERR_INVALID_ARG for null or
+ * misaligned pointers or bad sizes, LBQ_ERR_UNSUPPORTED for K % 512 != 0 or an
+ * unknown y_dtype, before any launch. Asynchronous on `stream`.
+ */
+lbq_status lbq_lut3_mx_gemm(const uint8_t* codes, const uint8_t* scales, int M, int K, int N, const void* image,
+                            void* Y, int y_dtype, void* stream);
+
 /* Number of kernel launches the library has enqueued so far in this process. */
 uint64_t lbq_launch_count(void);
 

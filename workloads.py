@@ -87,6 +87,17 @@ def lut3_host(seed, K, N):
     return idx, cb, ex
 
 
+def mx_activations_host(seed, M, K, scale_lo=118, scale_hi=134):
+    """MXFP8 activations drawn directly in the format: E4M3 codes uint8 [M, K]
+    uniform over the non-NaN bytes, UE8M0 scale bytes uint8 [M, K/32] uniform
+    over scale_lo..scale_hi."""
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(0, 256, size=(M, K), dtype=np.uint8)
+    codes[(codes & 0x7F) == 0x7F] -= 1
+    scales = rng.integers(scale_lo, scale_hi + 1, size=(M, K // 32), dtype=np.uint8)
+    return codes, scales
+
+
 # ----------------------------------------------------------------------------- device (torch)
 
 def _gen(seed, device):
