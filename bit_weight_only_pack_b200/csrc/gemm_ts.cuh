@@ -23,8 +23,10 @@
 //               exact packed subtract, one packed multiply); LUT3: the exact
 //               BF16 weight from the tile's table (byte permutes). 16 pairs
 //               per tcgen05.st. Four A buffers of 64 columns.
-//   warps 10-13 epilogue: tcgen05.ld the finished accumulator (thread = one
-//               channel, columns = tokens), round, store Y[token][channel].
+//   warps 10-13 epilogue: tcgen05.ld the finished accumulator 32 tokens at a
+//               time (thread = one channel), round into a [32 tokens][128
+//               channels] shared-memory tile and write it with one TMA store
+//               (two tiles alternate).
 #pragma once
 
 #include "common.cuh"
@@ -39,7 +41,13 @@ namespace lbq {
 constexpr int kTsBN = 128;                 // channels per tile (TMEM lanes)
 constexpr int kTsBM = 256;                 // tokens per tile (MMA N)
 constexpr int kTsBK = 128;                 // k per block: 8 MMAs per pair of barrier waits
-constexpr int kTsStages = 3;
+// TMA ring depth: INT4 keeps three 74 KB stages and stores Y element by
+// element; LUT3 trades one stage for two 8 KB output tiles written by TMA
+// stores (measured on B200, K=4096 N=14336 M=2048: INT4 811 TFLOP/s with three
+// stages against 812 with two plus TMA stores, and 779 against 817 at M=8192;
+// LUT3 864 -> 907 TFLOP/s with the TMA stores)
+__host__ __device__ constexpr int ts_stages(bool lut) { return lut ? 2 : 3; }
+constexpr int kTsMaxStages = 3;
 constexpr int kTsABufs = 4;                // A (weights) buffers in tensor memory, 64 columns each
 constexpr int kTsConvWarps = 8, kTsEpWarps = 4;
 // 32-k chunks per converter thread per block: the block's kTsBK / 32 chunks are
@@ -53,7 +61,8 @@ constexpr int kTsCBytes = kTsBN * 64;               // 8 KB codes (INT4) / 6 KB 
 constexpr int kTsMBytes = 2048;                     // scales + zero points (INT4) / tables (LUT3)
 constexpr int kTsOffC = kTsXBytes, kTsOffM = kTsOffC + kTsCBytes;
 constexpr int kTsStageBytes = kTsOffM + kTsMBytes;  // 74 KB, a multiple of 1024
-constexpr int kTsSmem = kTsStages * kTsStageBytes + 1024;
+constexpr int kTsOutBytes = 32 * kTsBN * 2;          // one [32 tokens][128 channels] output tile
+__host__ __device__ constexpr int ts_smem(bool lut) { return ts_stages(lut) * kTsStageBytes + (lut ? 2 * kTsOutBytes : 0) + 1024; }
 constexpr uint32_t kTsColA = 0, kTsColD = 256;
 static_assert(kTsStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
 
@@ -64,17 +73,21 @@ struct GemmTsArgs {
   int M, N, K, G, group;
   int n_tiles, m_tiles, k_blocks;  // channel tiles, token tiles, 64-k blocks
   int y_bf16;
+  int tma_out;               // 1: Y written by TMA stores (N % 8 == 0, 16-byte aligned Y); 0: element stores
 };
 
 template <bool BF16, bool ASYM, bool LUT>
 __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_constant__ CUtensorMap tx,
                                                                 const __grid_constant__ CUtensorMap tq,
+                                                                const __grid_constant__ CUtensorMap ty,
                                                                 const GemmTsArgs a) {
   extern __shared__ uint8_t dsmem[];
-  __shared__ __align__(8) uint64_t full_bar[kTsStages], empty_bar[kTsStages];
+  constexpr int kTsStages = ts_stages(LUT);
+  __shared__ __align__(8) uint64_t full_bar[kTsMaxStages], empty_bar[kTsMaxStages];
   __shared__ __align__(8) uint64_t a_full[kTsABufs], a_empty[kTsABufs], d_full, d_empty;
   __shared__ uint32_t tmem_base_sh;
   uint8_t* ring = dsmem + ((1024u - (smem_u32(dsmem) & 1023u)) & 1023u);
+  uint8_t* obuf = ring + (size_t)kTsStages * kTsStageBytes;  // two output tiles (LUT3)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int total_tiles = a.n_tiles * a.m_tiles;
@@ -241,30 +254,64 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
     }
   } else {
     // ------------------------------------------------------------------ epilogue
+    // every epilogue warp runs every chunk and both named barriers of it, also
+    // after a timed-out wait (then it loads and stores nothing)
     const int q = warp & 3;
     const int r = 32 * q + lane;  // channel within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-    int t_iter = 0;
+    const bool issuer = warp == 2 + kTsConvWarps && lane == 0;
+    if (issuer) tma_prefetch_desc(&ty);
+    int t_iter = 0, ob = 0;
+    bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++t_iter) {
       const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;
-      if (!mbar_wait(&d_full, t_iter & 1)) break;
+      if (ok && !mbar_wait(&d_full, t_iter & 1)) ok = false;
       tc_fence_after();
-      const int n = nt * kTsBN + r;
 #pragma unroll 1
       for (int j = 0; j < kTsBM / 32; ++j) {
         uint32_t v[32];
-        tmem_ld32(lane_base + kTsColD + (uint32_t)(j * 32), v);
-        const int m0 = mt * kTsBM + j * 32;
-        if (n < a.N) {
+        if (ok) {
+          tmem_ld32(lane_base + kTsColD + (uint32_t)(j * 32), v);
+        } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (m0 + i < a.M) store_out(a.Y, (size_t)(m0 + i) * a.N + n, __uint_as_float(v[i]), a.y_bf16);
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
         }
+        if (j == kTsBM / 32 - 1) {  // the accumulator is in registers: the MMAs may start the next tile
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0 && ok) mbar_arrive(&d_empty);
+        }
+        if (LUT && issuer) bulk_wait_read<1>();  // the tile written two chunks ago has been read
+        asm volatile("bar.sync 2, %0;" :: "r"(kTsEpWarps * 32) : "memory");
+        uint8_t* ot = obuf + (size_t)ob * kTsOutBytes;
+        const int m0 = mt * kTsBM + j * 32;
+        if (!a.tma_out) {  // rows of Y not 16-byte aligned: element stores
+          const int n = nt * kTsBN + r;
+          if (ok && n < a.N) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (m0 + i < a.M) store_out(a.Y, (size_t)(m0 + i) * a.N + n, __uint_as_float(v[i]), a.y_bf16);
+          }
+        }
+        if (LUT && a.tma_out) {  // the staging tiles exist only in the LUT3 kernel's shared memory
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float f = __uint_as_float(v[i]);
+            const uint16_t h =
+                a.y_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(f)) : __half_as_ushort(__float2half_rn(f));
+            *reinterpret_cast<uint16_t*>(ot + (i * kTsBN + r) * 2) = h;
+          }
+        }
+        fence_proxy_async();  // the tile, to the TMA unit
+        asm volatile("bar.sync 2, %0;" :: "r"(kTsEpWarps * 32) : "memory");
+        if (LUT && issuer && ok && a.tma_out && m0 < a.M) {
+          tma_store_2d(&ty, ot, nt * kTsBN, m0);
+          bulk_commit();
+        }
+        ob ^= 1;
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&d_empty);
     }
+    if (LUT && issuer) bulk_wait<0>();  // every output store has landed
   }
 
   tc_fence_before();

@@ -874,14 +874,14 @@ static int g_force_tc = 0;  // test hook: route every lbq_gemm call to the tcgen
 // kernel with the weights dequantised into shared memory (B operand).
 static int g_gemm_path = 0;
 
-typedef void (*TsKernel)(CUtensorMap, CUtensorMap, GemmTsArgs);
+typedef void (*TsKernel)(CUtensorMap, CUtensorMap, CUtensorMap, GemmTsArgs);
 
 // Prefill GEMM with the weights as the A operand in tensor memory (INT4 or LUT3).
 static lbq_status run_gemm_ts(const void* X, bool xbf16, int M, const void* image, const Layout& L, void* Y,
                               bool ybf16, cudaStream_t st) {
   const bool lut = L.mode == LBQ_MODE_LUT3, asym = L.mode == LBQ_MODE_ASYM;
   const uint8_t* img = static_cast<const uint8_t*>(image);
-  CUtensorMap tx, tq;
+  CUtensorMap tx, tq, ty;
   if (!make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)L.K, (uint64_t)M, (uint64_t)L.K * 2, 64,
                     kTsBM, CU_TENSOR_MAP_SWIZZLE_128B))
     return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the prefill activations");
@@ -900,14 +900,22 @@ static lbq_status run_gemm_ts(const void* X, bool xbf16, int M, const void* imag
   a.m_tiles = (M + kTsBM - 1) / kTsBM;
   a.k_blocks = (L.K + kTsBK - 1) / kTsBK;
   a.y_bf16 = ybf16 ? 1 : 0;
+  // LUT3 writes output tiles by TMA store where Y's rows allow it (16-byte row
+  // stride and base); INT4 stores elements (its kernel keeps a deeper ring instead)
+  a.tma_out = (lut && L.N % 8 == 0 && aligned16(Y)) ? 1 : 0;
+  ty = tx;
+  if (a.tma_out && !make_tmap_2d(&ty, Y, ybf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                                 (uint64_t)L.N, (uint64_t)M, (uint64_t)L.N * 2, kTsBN, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the prefill output");
   TsKernel fn;
   if (lut) fn = gemm_ts_kernel<true, false, true>;
   else if (xbf16) fn = asym ? gemm_ts_kernel<true, true, false> : gemm_ts_kernel<true, false, false>;
   else fn = asym ? gemm_ts_kernel<false, true, false> : gemm_ts_kernel<false, false, false>;
-  occupancy_for((const void*)fn, kTsThreads, kTsSmem);
+  const int smem = ts_smem(lut);
+  occupancy_for((const void*)fn, kTsThreads, smem);
   const int grid = std::min(a.n_tiles * a.m_tiles, num_sms());
-  void* args[] = {&tx, &tq, &a};
-  return launch_kernel_ex((const void*)fn, dim3(grid), dim3(kTsThreads), kTsSmem, st, false, args,
+  void* args[] = {&tx, &tq, &ty, &a};
+  return launch_kernel_ex((const void*)fn, dim3(grid), dim3(kTsThreads), smem, st, false, args,
                           "prefill GEMM launch");
 }
 
