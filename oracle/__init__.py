@@ -18,6 +18,10 @@ What it computes, and where each step comes from:
 * ``oracle.mxfp8``  -- MXFP8 activations (E4M3 elements, one UE8M0 scale per
   32 k) and the LUT3 x MXFP8 product: the activation format of the same page's
   native and emulated LUT-B paths (the next row after the BF16 LUT3 path).
+* ``oracle.affine`` -- generic b-bit (1..8) affine group-wise weights: the
+  quantiser, the canonical per-column little-endian bit stream and the exact
+  dequantisation ("Low Bit ARM kernels": one kernel per bit width in a
+  bit-width x tile table; group-wise scale and zero point).
 * ``oracle.matmul`` -- Y = X . W accumulated in FP64, the error scale
   S = |X| . |W|, and the acceptance test |y - y_ref| <= 4e-3*S + ulp16(|y_ref|).
 
@@ -32,4 +36,4 @@ decoders, nearest-level characterisation of the quantiser). Quantisation
 and it is out of scope.
 """
 
-from . import int4, lut3, matmul, mxfp8  # noqa: F401
+from . import affine, int4, lut3, matmul, mxfp8  # noqa: F401

@@ -472,3 +472,62 @@ def test_lut3_mxfp8_product_matches_exact_rational_brute_force():
         for n in range(N):
             exact = sum(Fraction(float(Xq[m, k])) * Fraction(float(W[k, n])) for k in range(K))
             assert abs(Fraction(float(Y[m, n])) - exact) <= abs(exact) * Fraction(1, 2 ** 50) + Fraction(1, 2 ** 200)
+
+
+# ----------------------------------------------------------------------------- generic b-bit affine
+
+from oracle import affine  # noqa: E402
+
+
+def test_affine_b3_golden(golden):
+    g = golden("affine_b3_8x2.json")
+    W = np.array(g["W"], dtype=np.float32)
+    q, s, zp = affine.quantize(W, g["group"], g["bits"])
+    assert q.tolist() == g["q"]
+    assert s.astype(np.float64).tolist() == g["scale"]
+    assert zp.tolist() == g["zp"]
+    assert affine.pack(q, g["bits"]).tolist() == g["packed"]
+    assert affine.unpack(np.array(g["packed"], dtype=np.uint8), g["bits"], g["K"]).tolist() == g["q"]
+    assert affine.dequant(q, s, g["group"], zp).tolist() == g["dequant"]
+
+
+def test_affine_4_bit_is_the_asymmetric_int4_form():
+    """b = 4 reduces to the (separately pinned) asymmetric INT4 quantiser and
+    its canonical two-nibbles-per-byte packing."""
+    W = (np.random.default_rng(21).standard_normal((256, 40)) * 0.02).astype(np.float32)
+    q, s, zp = affine.quantize(W, 32, 4)
+    q4, s4, zp4 = int4.quantize_asym(W, 32)
+    assert np.array_equal(q, q4) and np.array_equal(s.view(np.int16), s4.view(np.int16)) and np.array_equal(zp, zp4)
+    assert np.array_equal(affine.pack(q, 4), int4.pack_nibbles(q4))
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 5, 6, 7, 8])
+def test_affine_codes_are_nearest_levels_and_round_trip(bits):
+    """Every code is the nearest of the L + 1 levels (q - zp) s to w, clamped
+    to the range; packing round-trips; the bit stream holds exactly b bits per
+    code (brute force over the stream)."""
+    rng = np.random.default_rng(30 + bits)
+    K, N, group = 64, 12, 32
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    q, s, zp = affine.quantize(W, group, bits)
+    L = (1 << bits) - 1
+    assert q.max() <= L
+    deq = affine.dequant(q, s, group, zp)
+    s_k = np.repeat(s.astype(np.float64), group, axis=0)
+    z_k = np.repeat(zp.astype(np.float64), group, axis=0)
+    lv = (np.arange(L + 1)[None, None, :] - z_k[:, :, None]) * s_k[:, :, None]     # [K, N, L+1]
+    best = np.min(np.abs(lv - W[:, :, None].astype(np.float64)), axis=2)
+    # the chosen level is a nearest one, up to the FP32 rounding of w / s
+    assert np.all(np.abs(deq - W) <= best + 1e-6 * s_k + 1e-12)
+    packed = affine.pack(q, bits)
+    assert packed.shape == (K * bits // 8, N)
+    assert np.array_equal(affine.unpack(packed, bits, K), q)
+    stream = np.unpackbits(packed, axis=0, bitorder="little")   # [K*bits, N]
+    for k in (0, 1, K - 1):
+        val = sum(int(stream[bits * k + i, 0]) << i for i in range(bits))
+        assert val == int(q[k, 0])
+
+
+def test_affine_algorithmic_bytes():
+    assert affine.algorithmic_bytes(4096, 4096, 32, 3) == 4096 * 4096 * 3 // 8 + 128 * 4096 * 3
+    assert affine.algorithmic_bytes(4096, 14336, 64, 4) == int4.algorithmic_bytes(4096, 14336, 64, "asym")
