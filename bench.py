@@ -10,7 +10,8 @@ per second, against the measured HBM copy bandwidth. The step's weights
 (4.14 GB) are far larger than L2, so no flush is needed between steps.
 
 Secondary numbers (same JSON line, key "secondary"): the single 4096x4096
-GEMV, the K=8192 N=28672 batch sweep, the prefill GEMM and the LUT3 path.
+GEMV, the K=8192 N=28672 batch sweep, the prefill GEMM, the LUT3 path, LUT3 x
+MXFP8 with its activation quantiser, and the 1..8-bit affine GEMV.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lbq|reference]
 Multi-GPU: one process per GPU under torchrun; each rank runs its own decode
@@ -46,6 +47,12 @@ def load_peaks():
 
 def int4_bytes(K, N, group, mode):
     return K * N // 2 + (K // group) * N * (3 if mode == "asym" else 2)
+
+
+def affine_bytes(K, N, group, bits):
+    """Algorithmic bytes of a b-bit affine weight: K N b / 8 code bytes plus an
+    FP16 scale and an int8 zero point per group of a column."""
+    return K * N * bits // 8 + (K // group) * N * 3
 
 
 def lut3_bytes(K, N):
@@ -456,6 +463,25 @@ def _secondary_measurements(torch, lbq, workloads, device, peaks, quick):
     out["mxfp8_quantize_m2048_k4096"] = {"us": ms * 1e3, "GBps": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm,
                                          "bytes_per_launch": b, "input_copies": len(xs)}
     del xs
+    # generic b-bit affine GEMV, b = 1..8, at the gate/up shape K=4096 N=14336
+    # g64, batch 1 (and batch 4 for 3 bits), FP16 X: GB/s of the format's bytes
+    K, N, group = 4096, 14336, 64
+    W = workloads.weights_device(8, K, N, device)
+    for bits in range(1, 9):
+        images = weight_copies(lbq.pack_affine(W, group, bits), l2_bytes)
+        b = affine_bytes(K, N, group, bits)
+        for M in ((1, 4) if bits == 3 else (1,)):
+            X = workloads.activations_device(8, M, K, "f16", device)
+            Ya = torch.empty((M, N), dtype=torch.float16, device=device)
+
+            def acall(img, s):
+                lbq.lbq_affine_gemv(X.data_ptr(), 0, M, K, N, group, bits, img.data_ptr(), Ya.data_ptr(), 0, s)
+
+            ms = rotating_ms(torch, acall, images, reps=3)
+            out[f"affine_b{bits}_g64_m{M}"] = {"us": ms * 1e3, "GBps": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm,
+                                              "bytes_per_launch": b, "weight_copies": len(images)}
+        del images
+    del W
     return out
 
 
@@ -619,6 +645,8 @@ PROFILE_CASES = {
     "c5m2048": (4096, 14336, 0, "lut3", "bf16", 2048, None),
     "mxfp8q": (4096, 0, 0, "mxfp8", "bf16", 2048, None),
     "c5mx2048": (4096, 14336, 0, "lut3mx", "mxfp8", 2048, None),
+    "affine2": (4096, 14336, 64, "affine2", "f16", 1, None),
+    "affine3": (4096, 14336, 64, "affine3", "f16", 1, None),
 }
 
 
@@ -655,6 +683,19 @@ def run_profile_case(name):
         torch.cuda.synchronize()
         lbq.device_status()
         print(f"profile case {name}: {len(images)} launches of K={K} N={N} M={M}", flush=True)
+        return 0
+    if mode.startswith("affine"):
+        # b-bit affine GEMV: weight copies larger than L2
+        bits = int(mode[len("affine"):])
+        W = workloads.weights_device(7, K, N, device)
+        images = weight_copies(lbq.pack_affine(W, group, bits), l2)
+        del W
+        X = workloads.activations_device(7, M, K, xdt, device)
+        for img in images:
+            lbq.affine_gemv(X, img, N, group, bits)
+        torch.cuda.synchronize()
+        lbq.device_status()
+        print(f"profile case {name}: {len(images)} launches of K={K} N={N} bits={bits} M={M}", flush=True)
         return 0
     Ns = N if isinstance(N, tuple) else (N,)
     if mode == "lut3":

@@ -19,7 +19,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "liblbq.so")
 
 LBQ_OK, LBQ_ERR_INVALID_ARG, LBQ_ERR_UNSUPPORTED, LBQ_ERR_CUDA, LBQ_ERR_DEVICE = range(5)
-MODES = {"sym": 0, "asym": 1, "lut3": 2}
+MODES = {"sym": 0, "asym": 1, "lut3": 2, "affine": 3}
 DTYPES = {"f16": 0, "bf16": 1}
 STATUS_NAMES = {0: "LBQ_OK", 1: "LBQ_ERR_INVALID_ARG", 2: "LBQ_ERR_UNSUPPORTED", 3: "LBQ_ERR_CUDA",
                 4: "LBQ_ERR_DEVICE"}
@@ -64,6 +64,10 @@ _SIGS = {
     "lbq_gemv_grouped": ([ctypes.POINTER(lbq_gemv_item), _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp], _c_int),
     "lbq_quantize_mxfp8": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
     "lbq_lut3_mx_gemm": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp], _c_int),
+    "lbq_affine_packed_size": ([_c_int, _c_int, _c_int, _c_int, ctypes.POINTER(_c_size)], _c_int),
+    "lbq_pack_affine": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _c_size, _vp], _c_int),
+    "lbq_affine_gemv": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp], _c_int),
+    "lbq_unpack_affine_canonical": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp], _c_int),
     "lbq_debug_force_splits": ([_c_int], None),
     "lbq_debug_force_skinny": ([_c_int], None),
     "lbq_debug_force_tc": ([_c_int], None),
@@ -199,6 +203,24 @@ def lut3_mx_gemm(codes, scales, image, N, y_dtype="bf16", Y=None):
         Y = torch.empty((M, N), dtype={"f16": torch.float16, "bf16": torch.bfloat16}[y_dtype], device=codes.device)
     lbq_lut3_mx_gemm(codes.data_ptr(), scales.data_ptr(), M, K, N, image.data_ptr(), Y.data_ptr(), _dt(Y), _stream())
     return Y
+
+
+def lbq_affine_packed_size(K, N, group, bits):
+    n = _c_size(0)
+    _check(_lib.lbq_affine_packed_size(K, N, group, bits, ctypes.byref(n)))
+    return n.value
+
+
+def lbq_pack_affine(W, K, N, group, bits, image, image_bytes, stream):
+    _check(_lib.lbq_pack_affine(W, K, N, group, bits, image, image_bytes, stream))
+
+
+def lbq_affine_gemv(X, x_dtype, M, K, N, group, bits, image, Y, y_dtype, stream):
+    _check(_lib.lbq_affine_gemv(X, x_dtype, M, K, N, group, bits, image, Y, y_dtype, stream))
+
+
+def lbq_unpack_affine_canonical(image, K, N, group, bits, q_stream, scales, zp, stream):
+    _check(_lib.lbq_unpack_affine_canonical(image, K, N, group, bits, q_stream, scales, zp, stream))
 
 
 def lbq_set_option(option, value):
@@ -414,6 +436,36 @@ def gemv_noalloc(X, image, N, group, mode, y_dtype=None, Y=None):
     lbq_gemv_noalloc(X.data_ptr(), _dt(X), M, K, N, group, _mode(mode), image.data_ptr(), Y.data_ptr(), _dt(Y),
                      _stream())
     return Y
+
+
+def pack_affine(W, group, bits):
+    """Quantise + repack a float32 [K, N] CUDA tensor to b-bit affine codes; returns the uint8 image."""
+    torch = _torch()
+    _need_cuda(W)
+    K, N = W.shape
+    img = torch.empty(lbq_affine_packed_size(K, N, group, bits), dtype=torch.uint8, device=W.device)
+    lbq_pack_affine(W.data_ptr(), K, N, group, bits, img.data_ptr(), img.numel(), _stream())
+    return img
+
+
+def affine_gemv(X, image, N, group, bits, y_dtype=None, Y=None):
+    """Y[M, N] = X[M, K] . dequant(image) for a b-bit affine image, 1 <= M <= 16."""
+    _need_cuda(X, image, Y)
+    M, K = X.shape
+    Y = _out(X, N, y_dtype) if Y is None else Y
+    lbq_affine_gemv(X.data_ptr(), _dt(X), M, K, N, group, bits, image.data_ptr(), Y.data_ptr(), _dt(Y), _stream())
+    return Y
+
+
+def unpack_affine_canonical(image, K, N, group, bits):
+    """(q_stream uint8 [K*bits/8, N], scale fp16 [K/group, N], zp int8 [K/group, N])."""
+    torch = _torch()
+    q = torch.empty((K * bits // 8, N), dtype=torch.uint8, device=image.device)
+    s = torch.empty((K // group, N), dtype=torch.int16, device=image.device)
+    z = torch.empty((K // group, N), dtype=torch.int8, device=image.device)
+    lbq_unpack_affine_canonical(image.data_ptr(), K, N, group, bits, q.data_ptr(), s.data_ptr(), z.data_ptr(),
+                                _stream())
+    return q, s.view(torch.float16), z
 
 
 def device_status():

@@ -43,11 +43,16 @@ __device__ unsigned int g_device_error;
 //                    BF16 in a byte-planar 16 bytes (low bytes of entries 0..7,
 //                    then high bytes), [K/64][N/8][16]: what the kernels read.
 //                    C and E keep the format's own bytes for exact recovery.
+// AFFINE (b-bit codes, b = 1..8, in the header's `bits`):
+//   Q region         N rows of K*b/8 bytes, chunks of 32 k of b 32-bit words
+//                    each (layout in affine.cuh).
+//   S, Z regions     FP16 scales and int8 zero points, tiled as for INT4.
 // Every region starts on a 256-byte boundary.
 // ----------------------------------------------------------------------------
 
 constexpr uint32_t kMagicInt4 = 0x3451424Cu;  // "LBQ4"
 constexpr uint32_t kMagicLut3 = 0x3351424Cu;  // "LBQ3"
+constexpr uint32_t kMagicAffine = 0x4151424Cu;  // "LBQA"
 constexpr uint32_t kImageVersion = 1;
 constexpr size_t kHeaderBytes = 256;
 constexpr size_t kRegionAlign = 256;
@@ -63,6 +68,7 @@ struct ImageHeader {
   uint64_t off0, off1, off2;  // INT4: Q, S, Z   LUT3: I, C, E
   uint64_t total;
   uint64_t off3;              // LUT3: T
+  int32_t bits;               // AFFINE: code width (0 for the other formats)
 };
 static_assert(sizeof(ImageHeader) <= kHeaderBytes, "header too large");
 
@@ -74,16 +80,22 @@ __host__ __device__ inline size_t meta_index(int n, int gi, int G) {
 }
 
 struct Layout {
-  int K, N, group, mode;
+  int K, N, group, mode, bits;
   size_t off0, off1, off2, off3, total;
   size_t bytes0, bytes1, bytes2, bytes3;
   size_t s_stride, z_stride;  // LUT3: padded row strides (bytes) of the C and E regions
 };
 
-inline Layout make_layout(int K, int N, int group, int mode) {
+inline Layout make_layout(int K, int N, int group, int mode, int bits = 0) {
   Layout L{};
   L.K = K; L.N = N; L.group = group; L.mode = mode;
-  if (mode == LBQ_MODE_LUT3) {
+  L.bits = mode == LBQ_MODE_AFFINE ? bits : 0;
+  if (mode == LBQ_MODE_AFFINE) {
+    const size_t tiles128 = (size_t)(N + 127) / 128;
+    L.bytes0 = (size_t)N * (size_t)(K / 32) * 4 * (size_t)bits;
+    L.bytes1 = tiles128 * (size_t)(K / group) * 128 * 2;
+    L.bytes2 = tiles128 * (size_t)(K / group) * 128;
+  } else if (mode == LBQ_MODE_LUT3) {
     L.s_stride = align_up((size_t)(K / 64) * 8, 16);  // codebook row stride
     L.z_stride = align_up((size_t)(K / 64), 16);      // exponent row stride
     L.bytes0 = (size_t)N * (size_t)(K / 64) * 24;
@@ -106,7 +118,8 @@ inline Layout make_layout(int K, int N, int group, int mode) {
 
 inline ImageHeader make_header(const Layout& L) {
   ImageHeader h{};
-  h.magic = L.mode == LBQ_MODE_LUT3 ? kMagicLut3 : kMagicInt4;
+  h.magic = L.mode == LBQ_MODE_LUT3 ? kMagicLut3 : L.mode == LBQ_MODE_AFFINE ? kMagicAffine : kMagicInt4;
+  h.bits = L.bits;
   h.version = kImageVersion;
   h.K = L.K; h.N = L.N; h.group = L.group; h.mode = L.mode;
   h.off0 = L.off0; h.off1 = L.off1; h.off2 = L.off2; h.total = L.total; h.off3 = L.off3;

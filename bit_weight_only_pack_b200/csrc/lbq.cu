@@ -33,6 +33,7 @@
 #include "gemm_ts.cuh"
 #include "gemm_mx.cuh"
 #include "lut3_direct.cuh"
+#include "affine.cuh"
 
 namespace lbq {
 
@@ -1094,6 +1095,72 @@ static lbq_status run_lut3_mx(const uint8_t* codes, const uint8_t* scales, int M
   return launch_kernel_ex(fn, dim3(grid), dim3(kMxThreads), kMxSmem, st, false, args, "LUT3 x MXFP8 GEMM launch");
 }
 
+// ----------------------------------------------------------------------------
+// Generic b-bit affine weights
+// ----------------------------------------------------------------------------
+
+static lbq_status check_affine_shape(int K, int N, int group, int bits) {
+  if (bits < 1 || bits > 8) return fail(LBQ_ERR_UNSUPPORTED, "bits %d not in 1..8", bits);
+  if (group != 32 && group != 64 && group != 128)
+    return fail(LBQ_ERR_UNSUPPORTED, "group %d not in {32, 64, 128}", group);
+  if (K <= 0 || N <= 0) return fail(LBQ_ERR_INVALID_ARG, "K=%d N=%d must be positive", K, N);
+  if (K % group) return fail(LBQ_ERR_INVALID_ARG, "K=%d is not a multiple of group %d", K, group);
+  return LBQ_OK;
+}
+
+static lbq_status check_affine_header(const ImageHeader& h, int K, int N, int group, int bits) {
+  if (h.magic != kMagicAffine || h.version != kImageVersion)
+    return fail(LBQ_ERR_INVALID_ARG, "not an lbq affine image of this version (magic 0x%08x version %u)", h.magic,
+                h.version);
+  if (h.K != K || h.N != N || h.group != group || h.bits != bits || h.mode != LBQ_MODE_AFFINE)
+    return fail(LBQ_ERR_INVALID_ARG, "image holds K=%d N=%d group=%d bits=%d, call says K=%d N=%d group=%d bits=%d",
+                h.K, h.N, h.group, h.bits, K, N, group, bits);
+  return LBQ_OK;
+}
+
+// The bit-width x batch-tile kernel table: [x dtype][bits - 1][tile], tiles
+// of 1, 2 and 4 rows of X (8, 4 and 2 output channels per row block).
+#define LBQ_AG_TILES(B, BF) \
+  { (const void*)affine_gemv_kernel<B, BF, 1>, (const void*)affine_gemv_kernel<B, BF, 2>, \
+    (const void*)affine_gemv_kernel<B, BF, 4> }
+#define LBQ_AG_BITS(BF) \
+  { LBQ_AG_TILES(1, BF), LBQ_AG_TILES(2, BF), LBQ_AG_TILES(3, BF), LBQ_AG_TILES(4, BF), \
+    LBQ_AG_TILES(5, BF), LBQ_AG_TILES(6, BF), LBQ_AG_TILES(7, BF), LBQ_AG_TILES(8, BF) }
+static const void* const kAffineGemv[2][8][3] = {LBQ_AG_BITS(false), LBQ_AG_BITS(true)};
+#undef LBQ_AG_BITS
+#undef LBQ_AG_TILES
+
+static lbq_status run_affine_gemv(const uint16_t* X, bool xbf16, int M, const uint8_t* image, const Layout& L,
+                                  void* Y, bool ybf16, cudaStream_t st) {
+  const int chunks = L.K / 32;
+  const int nw = (chunks + 31) / 32;
+  if (nw > kAgMaxWarps) return fail(LBQ_ERR_UNSUPPORTED, "affine GEMV needs K <= %d", 32 * 32 * kAgMaxWarps);
+  const int T = nw * 32;
+  const int smem = 2 * nw * 8 * (int)sizeof(float);
+  for (int m0 = 0; m0 < M; m0 += 4) {
+    const int mv = std::min(4, M - m0);
+    const int tile = mv == 1 ? 0 : mv == 2 ? 1 : 2;
+    const int R = 8 >> tile;
+    const void* fn = kAffineGemv[xbf16 ? 1 : 0][L.bits - 1][tile];
+    AffineGemvArgs a{};
+    a.X = X + (size_t)m0 * L.K;
+    a.Y = static_cast<uint8_t*>(Y) + (size_t)m0 * L.N * 2;
+    a.q = image + L.off0;
+    a.s = image + L.off1;
+    a.z = image + L.off2;
+    a.K = L.K; a.N = L.N; a.G = L.K / L.group; a.gshift = log2_exact(L.group / 32);
+    a.m_valid = mv;
+    a.row_blocks = (L.N + R - 1) / R;
+    a.y_bf16 = ybf16 ? 1 : 0;
+    const int occ = std::max(1, occupancy_for(fn, T, smem));
+    const int grid = std::min(a.row_blocks, num_sms() * occ);
+    void* args[] = {&a};
+    lbq_status s = launch_kernel_ex(fn, dim3(grid), dim3(T), smem, st, false, args, "affine GEMV launch");
+    if (s != LBQ_OK) return s;
+  }
+  return LBQ_OK;
+}
+
 static lbq_status check_compute_args(const void* X, int x_dtype, int M, const void* image, void* Y, int y_dtype) {
   if (!X || !image || !Y) return fail(LBQ_ERR_INVALID_ARG, "X, image and Y must be non-null");
   if (!aligned16(X) || !aligned16(image) || !aligned16(Y))
@@ -1413,6 +1480,63 @@ lbq_status lbq_dequant(const void* image, int K, int N, int group, int mode, flo
   dequant_int4_kernel<<<(unsigned)((work + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       img + L.off0, img + L.off1, mode == LBQ_MODE_ASYM ? img + L.off2 : nullptr, K, N, group, W_out);
   return launch_check("dequant launch");
+}
+
+lbq_status lbq_affine_packed_size(int K, int N, int group, int bits, size_t* bytes) {
+  if (!bytes) return fail(LBQ_ERR_INVALID_ARG, "bytes must be non-null");
+  lbq_status st = check_affine_shape(K, N, group, bits);
+  if (st != LBQ_OK) return st;
+  *bytes = make_layout(K, N, group, LBQ_MODE_AFFINE, bits).total;
+  return LBQ_OK;
+}
+
+lbq_status lbq_pack_affine(const float* W, int K, int N, int group, int bits, void* image, size_t image_bytes,
+                           void* stream) {
+  lbq_status st = check_affine_shape(K, N, group, bits);
+  if (st != LBQ_OK) return st;
+  if (!W || !image) return fail(LBQ_ERR_INVALID_ARG, "W and image must be non-null");
+  if (!aligned16(W) || !aligned16(image)) return fail(LBQ_ERR_INVALID_ARG, "W and image must be 16-byte aligned");
+  const Layout L = make_layout(K, N, group, LBQ_MODE_AFFINE, bits);
+  if (image_bytes < L.total) return fail(LBQ_ERR_INVALID_ARG, "image buffer %zu bytes < %zu needed", image_bytes, L.total);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* img = static_cast<uint8_t*>(image);
+  write_header_kernel<<<1, 32, 0, s>>>(make_header(L), reinterpret_cast<ImageHeader*>(img));
+  if ((st = launch_check("header launch")) != LBQ_OK) return st;
+  if ((st = cuda_check(cudaMemsetAsync(img + L.off1, 0, L.total - L.off1, s), "clearing the scale regions")) != LBQ_OK)
+    return st;
+  const long long work = (long long)(K / group) * N;
+  quantize_pack_affine_kernel<<<(unsigned)((work + 255) / 256), 256, 0, s>>>(W, K, N, group, bits, img + L.off0,
+                                                                           img + L.off1, img + L.off2);
+  return launch_check("quantize_pack_affine launch");
+}
+
+lbq_status lbq_affine_gemv(const void* X, int x_dtype, int M, int K, int N, int group, int bits, const void* image,
+                           void* Y, int y_dtype, void* stream) {
+  lbq_status st = check_affine_shape(K, N, group, bits);
+  if (st != LBQ_OK) return st;
+  if ((st = check_compute_args(X, x_dtype, M, image, Y, y_dtype)) != LBQ_OK) return st;
+  if (M > 16) return fail(LBQ_ERR_UNSUPPORTED, "lbq_affine_gemv takes 1 <= M <= 16 (M=%d)", M);
+  const Layout L = make_layout(K, N, group, LBQ_MODE_AFFINE, bits);
+  return run_affine_gemv(static_cast<const uint16_t*>(X), x_dtype == LBQ_DTYPE_BF16, M,
+                         static_cast<const uint8_t*>(image), L, Y, y_dtype == LBQ_DTYPE_BF16,
+                         static_cast<cudaStream_t>(stream));
+}
+
+lbq_status lbq_unpack_affine_canonical(const void* image, int K, int N, int group, int bits, uint8_t* q_stream,
+                                       uint16_t* scales, int8_t* zp, void* stream) {
+  lbq_status st = check_affine_shape(K, N, group, bits);
+  if (st != LBQ_OK) return st;
+  if (!image || !q_stream || !scales || !zp)
+    return fail(LBQ_ERR_INVALID_ARG, "image, q_stream, scales and zp must be non-null");
+  ImageHeader h;
+  if ((st = read_header(image, &h)) != LBQ_OK) return st;
+  if ((st = check_affine_header(h, K, N, group, bits)) != LBQ_OK) return st;
+  const Layout L = make_layout(K, N, group, LBQ_MODE_AFFINE, bits);
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  const long long work = (long long)(K / 8) * bits * N;
+  unpack_affine_kernel<<<(unsigned)((work + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      img + L.off0, img + L.off1, img + L.off2, K, N, group, bits, q_stream, scales, zp);
+  return launch_check("unpack_affine launch");
 }
 
 lbq_status lbq_device_status(void* stream) {

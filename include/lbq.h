@@ -57,7 +57,7 @@ typedef enum {
   LBQ_ERR_DEVICE = 4        /* a kernel reported a problem (lbq_device_status) */
 } lbq_status;
 
-typedef enum { LBQ_MODE_SYM = 0, LBQ_MODE_ASYM = 1, LBQ_MODE_LUT3 = 2 } lbq_mode;
+typedef enum { LBQ_MODE_SYM = 0, LBQ_MODE_ASYM = 1, LBQ_MODE_LUT3 = 2, LBQ_MODE_AFFINE = 3 } lbq_mode;
 typedef enum { LBQ_DTYPE_F16 = 0, LBQ_DTYPE_BF16 = 1 } lbq_dtype;
 
 /* Human-readable description of the last failure on the calling thread. */
@@ -312,6 +312,66 @@ lbq_status lbq_quantize_mxfp8(const void* X, int x_dtype, int M, int K, uint8_t*
  */
 lbq_status lbq_lut3_mx_gemm(const uint8_t* codes, const uint8_t* scales, int M, int K, int N, const void* image,
                             void* Y, int y_dtype, void* stream);
+
+/*
+ * Generic b-bit affine weights, b = 1..8 ("Low Bit ARM kernels": one GEMV
+ * micro-kernel and one unpack routine per bit width 1..8 in a bit-width x tile
+ * table; 3-bit weights as an accuracy point between 2 and 4 bits; the
+ * group-wise scale section for the affine form). A weight is a code q in
+ * 0 .. 2^bits - 1 with value (q - zp) * s, one FP16 scale s and one int8 zero
+ * point zp per group of `group` (32, 64, 128) consecutive k of a column.
+ * bits = 4 is the asymmetric INT4 format in another image layout.
+ *
+ * lbq_affine_packed_size: size of the device image, K*N*bits/8 code bytes
+ *   plus the scales and zero points padded to 128-channel tiles, a 256-byte
+ *   header and 256-byte region alignment. Writes *bytes (host); no device work.
+ *   Errors: LBQ_ERR_UNSUPPORTED for bits outside 1..8 or group outside
+ *   {32, 64, 128}; LBQ_ERR_INVALID_ARG for K % group != 0, K or N <= 0, or a
+ *   null `bytes`.
+ */
+lbq_status lbq_affine_packed_size(int K, int N, int group, int bits, size_t* bytes);
+
+/*
+ * Quantise and repack an FP32 weight into a b-bit affine image.
+ *   W      (device) float32 [K, N] row-major, finite, 16-byte aligned
+ *   image  (device) lbq_affine_packed_size() bytes, written entirely
+ * Per group of a column, in IEEE FP32 with round-half-to-even, L = 2^bits - 1:
+ *   s = fp16((max w - min w) / L); zp = clamp(rint(-min w / s), -128, 127);
+ *   q = clamp(rint(w / s) + zp, 0, L)
+ * (s in the divisions is the stored FP16 scale widened to FP32; a group whose
+ * stored scale is 0 gets zp = 0, q = 0). Asynchronous on `stream`.
+ */
+lbq_status lbq_pack_affine(const float* W, int K, int N, int group, int bits, void* image, size_t image_bytes,
+                           void* stream);
+
+/*
+ * Decode GEMV on b-bit affine weights, 1 <= M <= 16:
+ *   Y[m][n] = sum_k X[m][k] (q[k][n] - zp) s, FP32 accumulation, Y rounded to
+ *   nearest in y_dtype.
+ *   X      (device) [M, K] row-major, x_dtype (LBQ_DTYPE_F16 / BF16), finite
+ *   image  (device) from lbq_pack_affine with this K, N, group, bits
+ *   Y      (device) [M, N] row-major, y_dtype, fully overwritten
+ * K <= 16384. X is read in tiles of up to 4 rows (one launch per tile; each
+ * launch streams the whole weight once). No workspace. Errors:
+ * LBQ_ERR_INVALID_ARG / LBQ_ERR_UNSUPPORTED before any launch, as above, and
+ * LBQ_ERR_UNSUPPORTED for M > 16 or K > 16384. Asynchronous on `stream`.
+ */
+lbq_status lbq_affine_gemv(const void* X, int x_dtype, int M, int K, int N, int group, int bits, const void* image,
+                           void* Y, int y_dtype, void* stream);
+
+/*
+ * Recover the canonical arrays of a b-bit affine image bit-exactly (debug /
+ * parity). Reads and checks the image header (a synchronous 64-byte copy).
+ *   q_stream (device) uint8 [K*bits/8, N]: per column n one little-endian bit
+ *            stream, code k at bits [bits*k, bits*k + bits); byte j of column
+ *            n's stream at q_stream[j][n]
+ *   scales   (device) uint16 [K/group, N] FP16 bits
+ *   zp       (device) int8 [K/group, N]
+ * Errors: LBQ_ERR_INVALID_ARG for null pointers or a header that does not
+ * match the call. The copy-out kernels run asynchronously on `stream`.
+ */
+lbq_status lbq_unpack_affine_canonical(const void* image, int K, int N, int group, int bits, uint8_t* q_stream,
+                                       uint16_t* scales, int8_t* zp, void* stream);
 
 /* Number of kernel launches the library has enqueued so far in this process. */
 uint64_t lbq_launch_count(void);
