@@ -22,6 +22,10 @@ What it computes, and where each step comes from:
   quantiser, the canonical per-column little-endian bit stream and the exact
   dequantisation ("Low Bit ARM kernels": one kernel per bit width in a
   bit-width x tile table; group-wise scale and zero point).
+* ``oracle.w4a8``   -- dynamic INT8 activations (symmetric, one FP32 scale per
+  32-k block of a row) and the W4A8 product from exact integer block sums
+  ("Low Bit ARM kernels": 4-bit weights with dynamic INT8 activations, group
+  32, integer inner loop, group scales applied after it).
 * ``oracle.matmul`` -- Y = X . W accumulated in FP64, the error scale
   S = |X| . |W|, and the acceptance test |y - y_ref| <= 4e-3*S + ulp16(|y_ref|).
 
@@ -36,4 +40,4 @@ decoders, nearest-level characterisation of the quantiser). Quantisation
 and it is out of scope.
 """
 
-from . import affine, int4, lut3, matmul, mxfp8  # noqa: F401
+from . import affine, int4, lut3, matmul, mxfp8, w4a8  # noqa: F401

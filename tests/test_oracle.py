@@ -531,3 +531,119 @@ def test_affine_codes_are_nearest_levels_and_round_trip(bits):
 def test_affine_algorithmic_bytes():
     assert affine.algorithmic_bytes(4096, 4096, 32, 3) == 4096 * 4096 * 3 // 8 + 128 * 4096 * 3
     assert affine.algorithmic_bytes(4096, 14336, 64, 4) == int4.algorithmic_bytes(4096, 14336, 64, "asym")
+
+
+# ----------------------------------------------------------------------------- W4A8
+
+from oracle import w4a8  # noqa: E402
+
+
+def _w4a8_golden_inputs(g):
+    K, group = g["K"], g["group"]
+    q = np.full((K, 2), 8, dtype=np.uint8)
+    q[:, 0] = g["q_col0"]
+    q[:, 1] = g["q_col1_default"]
+    q[0, 1] = g["q_col1_k0"]
+    sw = np.array(g["sw"], dtype=np.float16)
+    return q, sw, group
+
+
+def test_w4a8_activation_golden(golden):
+    g = golden("w4a8_block_1x64.json")
+    X = np.array(g["x"], dtype=np.float16).astype(np.float32)
+    assert np.array_equal(X, np.array(g["x"], dtype=np.float64))   # every value is exact in FP16
+    xq, s = w4a8.quantize_activations(X)
+    assert xq.tolist() == g["xq"]
+    assert s.tolist() == g["s"]
+
+
+@pytest.mark.parametrize("mode", ["sym", "asym"])
+def test_w4a8_product_golden(golden, mode):
+    g = golden("w4a8_block_1x64.json")
+    q, sw, group = _w4a8_golden_inputs(g)
+    xq = np.array(g["xq"], dtype=np.int8)
+    sx = np.array(g["s"], dtype=np.float32)
+    zp = None if mode == "sym" else np.array(g["zp_asym"], dtype=np.int8)
+    y = w4a8.matmul(xq, sx, q, sw, zp, group)
+    assert y.tolist() == g["y_" + mode]
+
+
+def test_w4a8_activation_invariants():
+    rng = np.random.default_rng(21)
+    X = (rng.standard_normal((5, 256)) * np.exp(rng.uniform(-6, 4, (5, 1)))).astype(np.float16).astype(np.float32)
+    X[0, 32:64] = 0.0                        # zero block
+    X[1, 64:96] = np.float32(np.float16(6e-8))  # FP16 subnormals only
+    xq, s = w4a8.quantize_activations(X)
+    Xb = X.reshape(5, 8, 32)
+    qb = xq.reshape(5, 8, 32).astype(np.int64)
+    assert np.all(np.abs(qb) <= 127)
+    assert np.all(qb[0, 1] == 0) and s[0, 1] == 0
+    amax_pos = np.abs(Xb).argmax(axis=2)
+    for m in range(5):
+        for b in range(8):
+            if s[m, b] == 0:
+                continue
+            i = amax_pos[m, b]
+            assert abs(qb[m, b, i]) == 127                     # the block maximum takes the extreme code
+            err = np.abs(Xb[m, b].astype(np.float64) - qb[m, b] * np.float64(s[m, b]))
+            assert np.all(err <= np.float64(s[m, b]) * (0.5 + 1e-6))   # nearest level
+    # odd symmetry and exact power-of-two scaling
+    xqn, sn = w4a8.quantize_activations(-X)
+    assert np.array_equal(xqn, -xq) and np.array_equal(sn, s)
+    xq2, s2 = w4a8.quantize_activations(X * np.float32(4.0))
+    assert np.array_equal(xq2, xq) and np.array_equal(s2, s * np.float32(4.0))
+
+
+def test_w4a8_scale_is_fp32_quotient_and_codes_are_fp32_rint():
+    """Against a scalar restatement with Python floats rounded through struct:
+    s = f32(amax / 127); xq = rint(f32(x / s)) with ties to even."""
+    rng = np.random.default_rng(22)
+    X = rng.standard_normal((3, 96)).astype(np.float16).astype(np.float32)
+    xq, s = w4a8.quantize_activations(X)
+
+    def f32(v):
+        return struct.unpack("<f", struct.pack("<f", v))[0]
+
+    for m in range(3):
+        for b in range(3):
+            blk = [float(v) for v in X[m, 32 * b:32 * b + 32]]
+            amax = max(abs(v) for v in blk)
+            sb = f32(amax / 127.0)
+            assert float(s[m, b]) == sb
+            for i, v in enumerate(blk):
+                r = round(f32(v / sb))          # Python's round() is half-to-even
+                assert int(xq[m, 32 * b + i]) == max(-127, min(127, r))
+
+
+def test_w4a8_product_matches_exact_rational_brute_force():
+    rng = np.random.default_rng(23)
+    M, K, N, group = 2, 64, 3, 32
+    xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    sx = rng.uniform(0.001, 0.1, (M, K // 32)).astype(np.float32)
+    q = rng.integers(0, 16, (K, N)).astype(np.uint8)
+    sw = rng.uniform(0.001, 0.1, (K // group, N)).astype(np.float16)
+    zp = rng.integers(-128, 128, (K // group, N)).astype(np.int8)
+    for z in (None, zp):
+        y = w4a8.matmul(xq, sx, q, sw, z, group)
+        for m in range(M):
+            for n in range(N):
+                exact = Fraction(0)
+                for k in range(K):
+                    zz = 8 if z is None else int(z[k // group, n])
+                    exact += (Fraction(int(xq[m, k])) * Fraction(float(sx[m, k // 32]))
+                              * (int(q[k, n]) - zz) * Fraction(float(sw[k // group, n])))
+                assert abs(Fraction(float(y[m, n])) - exact) <= abs(exact) * Fraction(1, 2 ** 50) + Fraction(1, 2 ** 80)
+
+
+def test_w4a8_product_is_the_product_of_the_dequantised_operands():
+    """The integer-block form equals the FP64 product of the dequantised
+    activations with the INT4 oracle's dequantised weight (both paths)."""
+    rng = np.random.default_rng(24)
+    X = rng.standard_normal((3, 256)).astype(np.float16).astype(np.float32)
+    W = (rng.standard_normal((256, 40)) * 0.02).astype(np.float32)
+    xq, sx = w4a8.quantize_activations(X)
+    for group, mode in ((32, "sym"), (64, "asym"), (128, "asym")):
+        q, s, zp = int4.quantize(W, group, mode)
+        y = w4a8.matmul(xq, sx, q, s, zp if mode == "asym" else None, group)
+        ref = matmul.matmul_f64(w4a8.dequant_activations(xq, sx), int4.dequant(q, s, group, zp))
+        assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
