@@ -180,10 +180,11 @@ class DecodeStep:
     # projection groups sharing X: (q, k, v), (o), (gate, up), (down)
     GROUPS = ((0, 1, 2), (3,), (4, 5), (6,))
 
-    def __init__(self, torch, lbq, workloads, device, layers, grouped=True):
+    def __init__(self, torch, lbq, workloads, device, layers, grouped=True, w4a8=False):
         self.torch = torch
         self.lbq = lbq
         self.grouped = grouped
+        self.w4a8 = w4a8  # W4A8: each shared X is quantised to INT8 once, then its GEMVs run on the codes
         self.bytes = 0
         self.calls = []  # per launch: list of (K, N, img, x, y, ws)
         proj = workloads.LLAMA3_8B_PROJ
@@ -215,7 +216,13 @@ class DecodeStep:
                                                        dtype=torch.uint8, device=device)
                     members.append((Kp, N, img, x, y, self.ws[(Kp, N)]))
                     self.bytes += int4_bytes(Kp, N, 32, "asym")
-                if grouped and len(members) > 1:
+                if w4a8:
+                    xq = torch.empty((1, K), dtype=torch.int8, device=device)
+                    sx = torch.empty((1, K // 32), dtype=torch.float32, device=device)
+                    items = lbq.make_w4a8_items([(xq.data_ptr(), sx.data_ptr(), img.data_ptr(), y.data_ptr(), N)
+                                                 for (_, N, img, x, y, _) in members])
+                    self.calls.append(("w4a8", K, x, xq, sx, items, len(members), members))
+                elif grouped and len(members) > 1:
                     items = lbq.make_gemv_items([(x.data_ptr(), img.data_ptr(), y.data_ptr(), N)
                                                  for (_, N, img, x, y, _) in members])
                     self.calls.append(("grouped", K, items, len(members), members))
@@ -228,7 +235,11 @@ class DecodeStep:
         lbq = self.lbq
         stream = self.torch.cuda.current_stream().cuda_stream
         for c in self.calls:
-            if c[0] == "grouped":
+            if c[0] == "w4a8":
+                _, K, x, xq, sx, items, n, _members = c
+                lbq.lbq_quantize_int8(x.data_ptr(), 0, 1, K, xq.data_ptr(), sx.data_ptr(), stream)
+                lbq.lbq_w4a8_gemv_grouped(items, n, K, 32, 1, 0, stream)
+            elif c[0] == "grouped":
                 _, K, items, n, _members = c
                 lbq.lbq_gemv_grouped(items, n, K, 32, 1, 0, 0, stream)
             else:
@@ -463,6 +474,29 @@ def _secondary_measurements(torch, lbq, workloads, device, peaks, quick):
     out["mxfp8_quantize_m2048_k4096"] = {"us": ms * 1e3, "GBps": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm,
                                          "bytes_per_launch": b, "input_copies": len(xs)}
     del xs
+    # the decode step in W4A8 form: 32 layers, per shared activation vector one
+    # INT8 quantisation and one grouped W4A8 launch (8 launches per layer), one
+    # CUDA graph with programmatic dependent launch; GB/s of the INT4 weight bytes
+    lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 1)
+    wstep = DecodeStep(torch, lbq, workloads, device, 32, w4a8=True)
+    g = wstep.capture()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(10):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / 10
+    out["c2_step_w4a8_32layers"] = {"us": ms * 1e3, "GBps": wstep.bytes / ms / 1e6,
+                                     "frac_hbm": wstep.bytes / ms / 1e6 / hbm,
+                                     "launches_per_step": wstep.launches_per_step,
+                                     "weight_bytes_per_step": wstep.bytes,
+                                     "activations": "INT8, one FP32 scale per 32 k (lbq_quantize_int8), once per "
+                                                    "shared X"}
+    del g, wstep
     # generic b-bit affine GEMV, b = 1..8, at the gate/up shape K=4096 N=14336
     # g64, batch 1 (and batch 4 for 3 bits), FP16 X: GB/s of the format's bytes
     K, N, group = 4096, 14336, 64
@@ -646,6 +680,7 @@ PROFILE_CASES = {
     "mxfp8q": (4096, 0, 0, "mxfp8", "bf16", 2048, None),
     "c5mx2048": (4096, 14336, 0, "lut3mx", "mxfp8", 2048, None),
     "affine2": (4096, 14336, 64, "affine2", "f16", 1, None),
+    "w4a8gate": (4096, 14336, 32, "w4a8", "f16", 1, None),
     "affine3": (4096, 14336, 64, "affine3", "f16", 1, None),
 }
 
@@ -683,6 +718,19 @@ def run_profile_case(name):
         torch.cuda.synchronize()
         lbq.device_status()
         print(f"profile case {name}: {len(images)} launches of K={K} N={N} M={M}", flush=True)
+        return 0
+    if mode == "w4a8":
+        # W4A8 batch-1 GEMV on asym INT4 weights: X quantised once, weight copies larger than L2
+        W = workloads.weights_device(7, K, N, device)
+        images = weight_copies(lbq.pack(W, group, "asym"), l2)
+        del W
+        X = workloads.activations_device(7, M, K, xdt, device)
+        xq, sx = lbq.quantize_int8(X)
+        for img in images:
+            lbq.w4a8_gemv(xq, sx, img, N, group, "asym")
+        torch.cuda.synchronize()
+        lbq.device_status()
+        print(f"profile case {name}: {len(images)} launches of K={K} N={N} W4A8 M={M}", flush=True)
         return 0
     if mode.startswith("affine"):
         # b-bit affine GEMV: weight copies larger than L2

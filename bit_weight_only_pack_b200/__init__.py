@@ -4,7 +4,8 @@ Y[M, N] = X[M, K] . dequant(Wq)[K, N] for INT4 (group-wise FP16 scales,
 symmetric or asymmetric with an int8 zero point) and 3-bit LUT weights
 (E4M3 codebook per 8 x 64 tile, UE8M0 exponent), as a decode GEMV / skinny
 GEMM and as a tcgen05 prefill GEMM; LUT3 weights with MXFP8 activations on the
-block-scaled FP8 tensor path; generic 1..8-bit affine weights as a decode GEMV.
+block-scaled FP8 tensor path; generic 1..8-bit affine weights as a decode GEMV;
+INT4 weights with dynamic INT8 activations (W4A8) as a decode GEMV.
 The work is done by liblbq.so (C ABI in include/lbq.h); this package is its
 thin Python binding.
 """
@@ -16,5 +17,6 @@ from .binding import (  # noqa: F401
     lbq_launch_count, lbq_lut3_gemm, lbq_pack, lbq_set_option, LBQ_OPT_PDL, lbq_pack_lut3, lbq_packed_size, lbq_unpack_canonical,
     lbq_unpack_lut3_canonical, lbq_version, lbq_workspace_size, lbq_quantize_mxfp8, lbq_lut3_mx_gemm,
     affine_gemv, pack_affine, unpack_affine_canonical, lbq_affine_gemv, lbq_affine_packed_size, lbq_pack_affine,
-    lbq_unpack_affine_canonical,
+    lbq_unpack_affine_canonical, quantize_int8, w4a8_gemv, lbq_quantize_int8, lbq_w4a8_gemv,
+    w4a8_gemv_grouped, lbq_w4a8_gemv_grouped, lbq_debug_w4a8_tiled, make_w4a8_items,
 )

@@ -44,6 +44,12 @@ class lbq_gemv_item(ctypes.Structure):
     _fields_ = [("X", ctypes.c_void_p), ("image", ctypes.c_void_p), ("Y", ctypes.c_void_p), ("N", ctypes.c_int)]
 
 
+class lbq_w4a8_item(ctypes.Structure):
+    """One GEMV of lbq_w4a8_gemv_grouped (include/lbq.h)."""
+    _fields_ = [("xq", ctypes.c_void_p), ("sx", ctypes.c_void_p), ("image", ctypes.c_void_p), ("Y", ctypes.c_void_p),
+                ("N", ctypes.c_int)]
+
+
 _SIGS = {
     "lbq_last_error": ([], ctypes.c_char_p),
     "lbq_version": ([], _c_int),
@@ -68,6 +74,11 @@ _SIGS = {
     "lbq_pack_affine": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _c_size, _vp], _c_int),
     "lbq_affine_gemv": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp], _c_int),
     "lbq_unpack_affine_canonical": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp], _c_int),
+    "lbq_quantize_int8": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
+    "lbq_w4a8_gemv": ([_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp], _c_int),
+    "lbq_w4a8_gemv_grouped": ([ctypes.POINTER(lbq_w4a8_item), _c_int, _c_int, _c_int, _c_int, _c_int, _vp],
+                              _c_int),
+    "lbq_debug_w4a8_tiled": ([_c_int], None),
     "lbq_debug_force_splits": ([_c_int], None),
     "lbq_debug_force_skinny": ([_c_int], None),
     "lbq_debug_force_tc": ([_c_int], None),
@@ -223,6 +234,31 @@ def lbq_unpack_affine_canonical(image, K, N, group, bits, q_stream, scales, zp, 
     _check(_lib.lbq_unpack_affine_canonical(image, K, N, group, bits, q_stream, scales, zp, stream))
 
 
+def lbq_quantize_int8(X, x_dtype, M, K, xq, sx, stream):
+    _check(_lib.lbq_quantize_int8(X, x_dtype, M, K, xq, sx, stream))
+
+
+def lbq_w4a8_gemv(xq, sx, M, K, N, group, mode, image, Y, y_dtype, stream):
+    _check(_lib.lbq_w4a8_gemv(xq, sx, M, K, N, group, mode, image, Y, y_dtype, stream))
+
+
+def lbq_w4a8_gemv_grouped(items, count, K, group, mode, y_dtype, stream):
+    _check(_lib.lbq_w4a8_gemv_grouped(items, count, K, group, mode, y_dtype, stream))
+
+
+def make_w4a8_items(rows):
+    """ctypes array of lbq_w4a8_item from (xq_ptr, sx_ptr, image_ptr, Y_ptr, N) tuples."""
+    arr = (lbq_w4a8_item * len(rows))()
+    for i, (xq, sx, img, Y, N) in enumerate(rows):
+        arr[i].xq, arr[i].sx, arr[i].image, arr[i].Y, arr[i].N = xq, sx, img, Y, N
+    return arr
+
+
+def lbq_debug_w4a8_tiled(on):
+    """Test hook: batch-1 W4A8 on the tiled kernel instead of the staged one."""
+    _lib.lbq_debug_w4a8_tiled(1 if on else 0)
+
+
 def lbq_set_option(option, value):
     _check(_lib.lbq_set_option(option, value))
 
@@ -340,6 +376,11 @@ def _out(X, N, y_dtype):
     torch = _torch()
     dt = {None: X.dtype, "f16": torch.float16, "bf16": torch.bfloat16}[y_dtype] if not hasattr(y_dtype, "is_floating_point") else y_dtype
     return torch.empty((X.shape[0], N), dtype=dt, device=X.device)
+
+
+def _out_dt(M, N, y_dtype, device):
+    torch = _torch()
+    return torch.empty((M, N), dtype={"f16": torch.float16, "bf16": torch.bfloat16}[y_dtype], device=device)
 
 
 def gemv(X, image, N, group, mode, y_dtype=None, ws=None, Y=None):
@@ -466,6 +507,44 @@ def unpack_affine_canonical(image, K, N, group, bits):
     lbq_unpack_affine_canonical(image.data_ptr(), K, N, group, bits, q.data_ptr(), s.data_ptr(), z.data_ptr(),
                                 _stream())
     return q, s.view(torch.float16), z
+
+
+def quantize_int8(X):
+    """Dynamic INT8 activations of X [M, K]: (xq int8 [M, K], sx float32 [M, K/32])."""
+    torch = _torch()
+    _need_cuda(X)
+    M, K = X.shape
+    xq = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    sx = torch.empty((M, K // 32), dtype=torch.float32, device=X.device)
+    lbq_quantize_int8(X.data_ptr(), _dt(X), M, K, xq.data_ptr(), sx.data_ptr(), _stream())
+    return xq, sx
+
+
+def w4a8_gemv(xq, sx, image, N, group, mode, y_dtype="f16", Y=None):
+    """Y[M, N] = dequant(xq, sx) . dequant(image) for an INT4 image, 1 <= M <= 16
+    (xq, sx from :func:`quantize_int8`)."""
+    _need_cuda(xq, sx, image, Y)
+    M, K = xq.shape
+    Y = _out_dt(M, N, y_dtype, xq.device) if Y is None else Y
+    lbq_w4a8_gemv(xq.data_ptr(), sx.data_ptr(), M, K, N, group, _mode(mode), image.data_ptr(), Y.data_ptr(), _dt(Y),
+                  _stream())
+    return Y
+
+
+def w4a8_gemv_grouped(problems, group, mode, y_dtype="f16"):
+    """Batch-1 W4A8 GEMVs in one launch. problems: [(xq [1, K], sx [1, K/32],
+    image, N), ...] with a common K; returns the list of Y [1, N]."""
+    K = problems[0][0].shape[1]
+    Ys, rows = [], []
+    for xq, sx, img, N in problems:
+        _need_cuda(xq, sx, img)
+        if xq.shape != (1, K):
+            raise ValueError("grouped GEMVs need xq [1, K] of one K")
+        Y = _out_dt(1, N, y_dtype, xq.device)
+        Ys.append(Y)
+        rows.append((xq.data_ptr(), sx.data_ptr(), img.data_ptr(), Y.data_ptr(), N))
+    lbq_w4a8_gemv_grouped(make_w4a8_items(rows), len(rows), K, group, _mode(mode), _dt(Ys[0]), _stream())
+    return Ys
 
 
 def device_status():

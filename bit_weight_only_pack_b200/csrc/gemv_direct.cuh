@@ -31,6 +31,7 @@
 
 #include "common.cuh"
 #include "gemv_m1.cuh"
+#include "w4a8.cuh"
 
 namespace lbq {
 
@@ -40,7 +41,8 @@ constexpr int kGdMaxItems = 4;  // GEMVs of one launch (same K, group, mode and 
 // One launch computes up to kGdMaxItems GEMVs; their 8-row blocks are numbered
 // consecutively, item i owning blocks [rb_end[i-1], rb_end[i]).
 struct GemvDirectArgs {
-  const uint16_t* X[kGdMaxItems];  // [K] FP16/BF16 bits
+  const uint16_t* X[kGdMaxItems];  // [K] FP16/BF16 bits (the A8 kernel: [K] INT8 codes)
+  const float* SX[kGdMaxItems];    // the A8 kernel: [K/32] activation scales
   void* Y[kGdMaxItems];            // [N]
   const uint8_t* q[kGdMaxItems];   // [N][K/2]
   const uint8_t* s[kGdMaxItems];   // 128-channel-tiled FP16 scales
@@ -182,7 +184,14 @@ __global__ void __launch_bounds__(kGdMaxWarps * 32, 1) gemv_direct_kernel(const 
 // only synchronisation. Dynamic shared memory: uint4 codes [S][8][T], uint4
 // scales [S][T], uint2 zero points [S][T] (T threads), then the row sums as in
 // gemv_direct_kernel.
-template <bool BF16, bool ASYM, int S>
+//
+// A8 = true is the W4A8 form of the same kernel ("Low Bit ARM kernels": 4-bit
+// weights with dynamic INT8 activations): X holds INT8 codes and SX one FP32
+// scale per 32-k block (from lbq_quantize_int8); a chunk of a row is four
+// pairs of byte dot products (dp4a) on the low nibbles and the in-place high
+// nibbles (16 q), exact in int32; per chunk (s_w s_x) (sum xq q - z sum xq) is
+// added in FP32.
+template <bool BF16, bool ASYM, int S, bool A8 = false>
 __global__ void __launch_bounds__(kGdMaxWarps * 32) gemv_direct_async_kernel(const GemvDirectArgs a) {
   extern __shared__ __align__(16) uint8_t gd_smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -241,9 +250,25 @@ __global__ void __launch_bounds__(kGdMaxWarps * 32) gemv_direct_async_kernel(con
 
   uint32_t xr[16];
   float xoff = 0.0f, xsum = 0.0f;
+  float sx8 = 0.0f;  // A8: the block's activation scale and code sum
+  int xs8 = 0;
   const uint16_t* x_loaded = nullptr;
   auto load_x = [&](const uint16_t* X) {
     x_loaded = X;
+    if constexpr (A8) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) xr[i] = 0u;
+      sx8 = 0.0f;
+      xs8 = 0;
+      if (cok) {
+        uint32_t lo[4], hi[4];
+        load_xq_block(reinterpret_cast<const int8_t*>(X) + (size_t)c * 32, lo, hi, xs8);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { xr[i] = lo[i]; xr[4 + i] = hi[i]; }
+        sx8 = __ldg(a.SX[it_comp] + c);
+      }
+      return;
+    }
     float sA = 0.0f, sB = 0.0f;
     if (cok) {
       const uint4* xp = reinterpret_cast<const uint4*>(X + (size_t)c * 32);
@@ -285,6 +310,19 @@ __global__ void __launch_bounds__(kGdMaxWarps * 32) gemv_direct_async_kernel(con
         const float2 sc = __half22float2(*reinterpret_cast<const __half2*>(&sw[i >> 1]));
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
+          if constexpr (A8) {
+            const uint4 wv = lds128(src + (uint32_t)(i + h) * T16);
+            const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+            int acc = 0, acc16 = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              acc = dp4a_us(wd[j] & 0x0F0F0F0Fu, xr[j], acc);
+              acc16 = dp4a_us(wd[j] & 0xF0F0F0F0u, xr[4 + j], acc16);
+            }
+            const int zi = ASYM ? (int)(int8_t)(((i < 4 ? zv.x : zv.y) >> (8 * ((i + h) & 3))) & 0xFFu) : 8;
+            part[i + h] = (float)(acc + (acc16 >> 4) - zi * xs8) * ((h ? sc.y : sc.x) * sx8);
+            continue;
+          }
           const float acc = gd_chunk<BF16>(lds128(src + (uint32_t)(i + h) * T16), xr);
           float corr = xoff;
           if (ASYM) {

@@ -34,6 +34,7 @@
 #include "gemm_mx.cuh"
 #include "lut3_direct.cuh"
 #include "affine.cuh"
+#include "w4a8.cuh"
 
 namespace lbq {
 
@@ -454,12 +455,17 @@ static lbq_status run_tcgemv(const void* X, bool xbf16, int M, const void* image
 static int g_direct_stages = -1;
 static int g_direct_ctas = 0;  // test hook: cap on resident CTAs per SM (0 = occupancy limit)
 
-static const void* direct_async_kernel(bool bf16, bool asym, int stages) {
-#define LBQ_GDA(S) (bf16 ? (asym ? (const void*)gemv_direct_async_kernel<true, true, S>              \
-                                 : (const void*)gemv_direct_async_kernel<true, false, S>)             \
-                         : (asym ? (const void*)gemv_direct_async_kernel<false, true, S>             \
-                                 : (const void*)gemv_direct_async_kernel<false, false, S>))
-  return stages >= 4 ? LBQ_GDA(4) : stages == 3 ? LBQ_GDA(3) : LBQ_GDA(2);
+static const void* direct_async_kernel(bool bf16, bool asym, int stages, bool a8 = false) {
+#define LBQ_GDA(S, A) (bf16 ? (asym ? (const void*)gemv_direct_async_kernel<true, true, S, A>              \
+                                    : (const void*)gemv_direct_async_kernel<true, false, S, A>)             \
+                            : (asym ? (const void*)gemv_direct_async_kernel<false, true, S, A>             \
+                                    : (const void*)gemv_direct_async_kernel<false, false, S, A>))
+#define LBQ_GDA8(S) (asym ? (const void*)gemv_direct_async_kernel<false, true, S, true> \
+                         : (const void*)gemv_direct_async_kernel<false, false, S, true>)
+  (void)bf16;
+  if (a8) return stages >= 4 ? LBQ_GDA8(4) : stages == 3 ? LBQ_GDA8(3) : LBQ_GDA8(2);
+#undef LBQ_GDA8
+  return stages >= 4 ? LBQ_GDA(4, false) : stages == 3 ? LBQ_GDA(3, false) : LBQ_GDA(2, false);
 #undef LBQ_GDA
 }
 
@@ -531,9 +537,12 @@ static lbq_status run_dmma(const lbq_gemv_item* items, int count, int K, int gro
   return fail(LBQ_ERR_UNSUPPORTED, "K=%d with %d distinct activation vectors does not fit shared memory", K, a.nx);
 }
 
+// sx != nullptr selects the W4A8 form: items[i].X are INT8 codes and sx[i]
+// their per-32-k scales.
 static lbq_status run_direct(const lbq_gemv_item* items, int count, int K, int group, int mode, bool xbf16, bool ybf16,
-                             cudaStream_t st) {
-  if (g_dmma) return run_dmma(items, count, K, group, mode, xbf16, ybf16, st);
+                             cudaStream_t st, const float* const* sx = nullptr) {
+  const bool a8 = sx != nullptr;
+  if (g_dmma && !a8) return run_dmma(items, count, K, group, mode, xbf16, ybf16, st);
   const bool asym = mode == LBQ_MODE_ASYM;
   const int chunks = K / 32;
   const int nw = (chunks + 31) / 32;
@@ -545,6 +554,7 @@ static lbq_status run_direct(const lbq_gemv_item* items, int count, int K, int g
     const Layout L = make_layout(K, items[i].N, group, mode);
     const uint8_t* img = static_cast<const uint8_t*>(items[i].image);
     a.X[i] = static_cast<const uint16_t*>(items[i].X);
+    a.SX[i] = a8 ? sx[i] : nullptr;
     a.Y[i] = items[i].Y;
     a.q[i] = img + L.off0;
     a.s[i] = img + L.off1;
@@ -573,8 +583,9 @@ static lbq_status run_direct(const lbq_gemv_item* items, int count, int K, int g
   // the most stages (<= the chosen count) whose slots fit a CTA
   while (stages >= 2 && (size_t)T * (size_t)(stages * (8 * 16 + 16 + 8)) > 220 * 1024) --stages;
   if (stages < 2) stages = 0;
+  if (a8 && stages == 0) stages = 2;  // the INT8-activation form exists only staged (2 stages always fit)
   const int stage_bytes = stages ? T * stages * (8 * 16 + 16 + 8) : 0;
-  const void* fn = stages == 0 ? reg_fn : direct_async_kernel(xbf16, asym, stages);
+  const void* fn = stages == 0 ? reg_fn : direct_async_kernel(xbf16, asym, stages, a8);
   // one wave of CTAs; each keeps 8 floats per warp per row block in shared memory
   int occ = std::max(1, occupancy_for(fn, T, stage_bytes + 4096));
   if (g_direct_ctas > 0) occ = std::min(occ, g_direct_ctas);
@@ -1161,6 +1172,61 @@ static lbq_status run_affine_gemv(const uint16_t* X, bool xbf16, int M, const ui
   return LBQ_OK;
 }
 
+// ----------------------------------------------------------------------------
+// W4A8: INT4 weights x dynamic INT8 activations
+// ----------------------------------------------------------------------------
+
+static int g_w4a8_tiled = 0;  // test hook: batch-1 W4A8 on the tiled kernel instead of the staged one
+
+// [asym][tile of 1, 2, 4 rows of X]
+static const void* const kW4a8Gemv[2][3] = {
+    {(const void*)w4a8_gemv_kernel<false, 1>, (const void*)w4a8_gemv_kernel<false, 2>,
+     (const void*)w4a8_gemv_kernel<false, 4>},
+    {(const void*)w4a8_gemv_kernel<true, 1>, (const void*)w4a8_gemv_kernel<true, 2>,
+     (const void*)w4a8_gemv_kernel<true, 4>}};
+
+static lbq_status run_w4a8_gemv(const int8_t* XQ, const float* SX, int M, const uint8_t* image, const Layout& L,
+                                void* Y, bool ybf16, cudaStream_t st) {
+  const int chunks = L.K / 32;
+  const int nw = (chunks + 31) / 32;
+  if (nw > kW8MaxWarps) return fail(LBQ_ERR_UNSUPPORTED, "W4A8 GEMV needs K <= %d", 32 * 32 * kW8MaxWarps);
+  const int T = nw * 32;
+  const int smem = 2 * nw * 8 * (int)sizeof(float);
+  const bool asym = L.mode == LBQ_MODE_ASYM;
+  for (int m0 = 0; m0 < M; m0 += 4) {
+    const int mv = std::min(4, M - m0);
+    const int tile = mv == 1 ? 0 : mv == 2 ? 1 : 2;
+    const int R = 8 >> tile;
+    const void* fn = kW4a8Gemv[asym ? 1 : 0][tile];
+    W4a8Args a{};
+    a.XQ = XQ + (size_t)m0 * L.K;
+    a.SX = SX + (size_t)m0 * (L.K / 32);
+    a.Y = static_cast<uint8_t*>(Y) + (size_t)m0 * L.N * 2;
+    a.q = image + L.off0;
+    a.s = image + L.off1;
+    a.z = asym ? image + L.off2 : nullptr;
+    a.K = L.K; a.N = L.N; a.G = L.K / L.group; a.gshift = log2_exact(L.group / 32);
+    a.m_valid = mv;
+    a.row_blocks = (L.N + R - 1) / R;
+    a.y_bf16 = ybf16 ? 1 : 0;
+    const int occ = std::max(1, occupancy_for(fn, T, smem));
+    const int grid = std::min(a.row_blocks, num_sms() * occ);
+    void* args[] = {&a};
+    lbq_status s = launch_kernel_ex(fn, dim3(grid), dim3(T), smem, st, g_pdl != 0, args, "W4A8 GEMV launch");
+    if (s != LBQ_OK) return s;
+  }
+  return LBQ_OK;
+}
+
+static lbq_status check_w4a8_args(const int8_t* xq, const float* sx, int M, const void* image, void* Y, int y_dtype) {
+  if (!xq || !sx || !image || !Y) return fail(LBQ_ERR_INVALID_ARG, "xq, sx, image and Y must be non-null");
+  if (!aligned16(xq) || !aligned16(image) || !aligned16(Y) || (reinterpret_cast<uintptr_t>(sx) & 3u))
+    return fail(LBQ_ERR_INVALID_ARG, "xq, image and Y must be 16-byte aligned, sx 4-byte aligned");
+  if (y_dtype != LBQ_DTYPE_F16 && y_dtype != LBQ_DTYPE_BF16) return fail(LBQ_ERR_UNSUPPORTED, "y_dtype %d", y_dtype);
+  if (M <= 0) return fail(LBQ_ERR_INVALID_ARG, "M=%d must be positive", M);
+  return LBQ_OK;
+}
+
 static lbq_status check_compute_args(const void* X, int x_dtype, int M, const void* image, void* Y, int y_dtype) {
   if (!X || !image || !Y) return fail(LBQ_ERR_INVALID_ARG, "X, image and Y must be non-null");
   if (!aligned16(X) || !aligned16(image) || !aligned16(Y))
@@ -1285,6 +1351,10 @@ void lbq_debug_direct_variant(int variant, int ctas_per_sm) {
   g_direct_ctas = ctas_per_sm > 0 ? ctas_per_sm : 0;
   g_dmma = variant == 1 ? 1 : variant == 5 ? 2 : 0;
 }
+
+// Test hook (not in the public header): batch-1 lbq_w4a8_gemv on the tiled
+// W4A8 kernel (the one for M > 1) instead of the staged direct kernel.
+void lbq_debug_w4a8_tiled(int on) { g_w4a8_tiled = on ? 1 : 0; }
 
 lbq_status lbq_set_option(int option, int value) {
   if (option == LBQ_OPT_PDL) {
@@ -1537,6 +1607,52 @@ lbq_status lbq_unpack_affine_canonical(const void* image, int K, int N, int grou
   unpack_affine_kernel<<<(unsigned)((work + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       img + L.off0, img + L.off1, img + L.off2, K, N, group, bits, q_stream, scales, zp);
   return launch_check("unpack_affine launch");
+}
+
+lbq_status lbq_quantize_int8(const void* X, int x_dtype, int M, int K, int8_t* xq, float* sx, void* stream) {
+  if (!X || !xq || !sx) return fail(LBQ_ERR_INVALID_ARG, "X, xq and sx must be non-null");
+  if (!aligned16(X) || !aligned16(xq)) return fail(LBQ_ERR_INVALID_ARG, "X and xq must be 16-byte aligned");
+  if (x_dtype != LBQ_DTYPE_F16 && x_dtype != LBQ_DTYPE_BF16) return fail(LBQ_ERR_UNSUPPORTED, "x_dtype %d", x_dtype);
+  if (M <= 0 || K <= 0 || K % 32) return fail(LBQ_ERR_INVALID_ARG, "M=%d K=%d: need M > 0 and K a positive multiple of 32", M, K);
+  const long long warps = (long long)M * (K / 32);  // one warp per 32-k block
+  const unsigned grid = (unsigned)((warps * 32 + 255) / 256);
+  const void* fn = x_dtype == LBQ_DTYPE_BF16 ? (const void*)quantize_int8_kernel<true>
+                                             : (const void*)quantize_int8_kernel<false>;
+  const uint16_t* Xp = static_cast<const uint16_t*>(X);
+  void* args[] = {(void*)&Xp, (void*)&M, (void*)&K, (void*)&xq, (void*)&sx};
+  return launch_kernel_ex(fn, dim3(grid), dim3(256), 0, static_cast<cudaStream_t>(stream), g_pdl != 0, args,
+                          "quantize_int8 launch");
+}
+
+lbq_status lbq_w4a8_gemv_grouped(const lbq_w4a8_item* items, int count, int K, int group, int mode, int y_dtype,
+                                 void* stream) {
+  if (!items || count < 1 || count > kGdMaxItems) return fail(LBQ_ERR_INVALID_ARG, "count=%d not in 1..%d", count, kGdMaxItems);
+  lbq_status st;
+  lbq_gemv_item gi[kGdMaxItems];
+  const float* sx[kGdMaxItems];
+  for (int i = 0; i < count; ++i) {
+    if ((st = check_int4_shape(K, items[i].N, group, mode)) != LBQ_OK) return st;
+    if ((st = check_w4a8_args(items[i].xq, items[i].sx, 1, items[i].image, items[i].Y, y_dtype)) != LBQ_OK) return st;
+    gi[i] = lbq_gemv_item{items[i].xq, items[i].image, items[i].Y, items[i].N};
+    sx[i] = items[i].sx;
+  }
+  return run_direct(gi, count, K, group, mode, false, y_dtype == LBQ_DTYPE_BF16, static_cast<cudaStream_t>(stream), sx);
+}
+
+lbq_status lbq_w4a8_gemv(const int8_t* xq, const float* sx, int M, int K, int N, int group, int mode,
+                         const void* image, void* Y, int y_dtype, void* stream) {
+  lbq_status st = check_int4_shape(K, N, group, mode);
+  if (st != LBQ_OK) return st;
+  if ((st = check_w4a8_args(xq, sx, M, image, Y, y_dtype)) != LBQ_OK) return st;
+  if (M > 16) return fail(LBQ_ERR_UNSUPPORTED, "lbq_w4a8_gemv takes 1 <= M <= 16 (M=%d)", M);
+  if (M == 1 && !g_w4a8_tiled) {
+    const lbq_gemv_item item{xq, image, Y, N};
+    return run_direct(&item, 1, K, group, mode, false, y_dtype == LBQ_DTYPE_BF16, static_cast<cudaStream_t>(stream),
+                      &sx);
+  }
+  const Layout L = make_layout(K, N, group, mode);
+  return run_w4a8_gemv(xq, sx, M, static_cast<const uint8_t*>(image), L, Y, y_dtype == LBQ_DTYPE_BF16,
+                       static_cast<cudaStream_t>(stream));
 }
 
 lbq_status lbq_device_status(void* stream) {

@@ -373,6 +373,64 @@ lbq_status lbq_affine_gemv(const void* X, int x_dtype, int M, int K, int N, int 
 lbq_status lbq_unpack_affine_canonical(const void* image, int K, int N, int group, int bits, uint8_t* q_stream,
                                        uint16_t* scales, int8_t* zp, void* stream);
 
+/*
+ * Dynamic INT8 activations for W4A8 ("Low Bit ARM kernels": 4-bit weights
+ * with dynamic INT8 activations, group size 32, an integer inner loop with
+ * int32 accumulation and the group scales applied after it). Each row of X is
+ * quantised in blocks of 32 consecutive k, symmetric, in IEEE FP32:
+ *   s = amax / 127 (amax the block's largest |x|);
+ *   xq = clamp(rint(x / s), -127, 127), ties to even; an all-zero block has
+ *   s = 0 and xq = 0.
+ *   X   (device) [M, K] row-major, x_dtype (LBQ_DTYPE_F16 / BF16), finite
+ *   xq  (device) int8 [M, K], 16-byte aligned
+ *   sx  (device) float32 [M, K/32]
+ * K % 32 == 0. Bit-identical to the CPU reference. Errors: LBQ_ERR_INVALID_ARG
+ * for null or misaligned pointers or bad sizes, LBQ_ERR_UNSUPPORTED for an
+ * unknown x_dtype, before any launch. Asynchronous on `stream`.
+ */
+lbq_status lbq_quantize_int8(const void* X, int x_dtype, int M, int K, int8_t* xq, float* sx, void* stream);
+
+/*
+ * W4A8 decode GEMV, 1 <= M <= 16: INT4 weights (an lbq_pack image, SYM or
+ * ASYM) times INT8 activations from lbq_quantize_int8 ("Low Bit ARM kernels":
+ * the integer inner loop with int32 accumulation, group scales after it). Per
+ * 32-k block b of row m and column n the integer sum
+ * I = sum xq q - z sum xq is exact (z = 8 for SYM, the zero point for ASYM), and
+ *   Y[m][n] = sum_b sx[m][b] s_w[group of b][n] I[m][b][n]
+ * accumulated in FP32, rounded to nearest in y_dtype.
+ *   xq     (device) int8 [M, K], 16-byte aligned
+ *   sx     (device) float32 [M, K/32]
+ *   image  (device) from lbq_pack with this K, N, group, mode
+ *   Y      (device) [M, N] row-major, y_dtype, fully overwritten
+ * K <= 16384. M = 1 runs as the staged batch-1 kernel; larger M in tiles of
+ * up to 4 rows (one launch per tile; each launch streams the whole weight
+ * once). No workspace. Errors: LBQ_ERR_INVALID_ARG / LBQ_ERR_UNSUPPORTED for
+ * bad pointers, sizes or modes, M > 16 or K > 16384, before any launch.
+ * Asynchronous on `stream`.
+ */
+lbq_status lbq_w4a8_gemv(const int8_t* xq, const float* sx, int M, int K, int N, int group, int mode,
+                         const void* image, void* Y, int y_dtype, void* stream);
+
+/*
+ * Several batch-1 W4A8 GEMVs in one launch (the projections of a decoder
+ * layer that read the same activation vector, quantised once). Item i:
+ *   xq, sx (device) [1, K] INT8 codes and [1, K/32] scales (lbq_quantize_int8)
+ *   image  (device) from lbq_pack with K, items[i].N, group, mode
+ *   Y      (device) [1, items[i].N], y_dtype, fully overwritten
+ * items is a host array of 1..4 entries sharing K (<= 16384), group and mode;
+ * each item's result equals lbq_w4a8_gemv with M = 1 on it. No workspace.
+ * Errors as lbq_w4a8_gemv, before any launch. Asynchronous on `stream`.
+ */
+typedef struct {
+  const int8_t* xq;
+  const float* sx;
+  const void* image;
+  void* Y;
+  int N;
+} lbq_w4a8_item;
+lbq_status lbq_w4a8_gemv_grouped(const lbq_w4a8_item* items, int count, int K, int group, int mode, int y_dtype,
+                                 void* stream);
+
 /* Number of kernel launches the library has enqueued so far in this process. */
 uint64_t lbq_launch_count(void);
 
