@@ -26,6 +26,10 @@ What it computes, and where each step comes from:
   32-k block of a row) and the W4A8 product from exact integer block sums
   ("Low Bit ARM kernels": 4-bit weights with dynamic INT8 activations, group
   32, integer inner loop, group scales applied after it).
+* ``oracle.moe``    -- the grouped MoE GEMM of LUT3 experts with MXFP8
+  activations: moe_align_block_size (expert-sorted, block-padded pair lists)
+  and the gathered product with zero rows for non-local experts (vLLM PR
+  62759 write-up, gather and expert-parallelism sections).
 * ``oracle.matmul`` -- Y = X . W accumulated in FP64, the error scale
   S = |X| . |W|, and the acceptance test |y - y_ref| <= 4e-3*S + ulp16(|y_ref|).
 
@@ -40,4 +44,4 @@ decoders, nearest-level characterisation of the quantiser). Quantisation
 and it is out of scope.
 """
 
-from . import affine, int4, lut3, matmul, mxfp8, w4a8  # noqa: F401
+from . import affine, int4, lut3, matmul, moe, mxfp8, w4a8  # noqa: F401

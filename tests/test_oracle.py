@@ -647,3 +647,70 @@ def test_w4a8_product_is_the_product_of_the_dequantised_operands():
         y = w4a8.matmul(xq, sx, q, s, zp if mode == "asym" else None, group)
         ref = matmul.matmul_f64(w4a8.dequant_activations(xq, sx), int4.dequant(q, s, group, zp))
         assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- MoE grouped GEMM
+
+from oracle import moe  # noqa: E402
+
+
+def test_moe_align_golden(golden):
+    g = golden("moe_align_6x2.json")
+    s, e, total = moe.align(np.array(g["topk_ids"]), g["num_experts"], g["block"])
+    assert s.tolist() == g["sorted_ids"] and e.tolist() == g["expert_ids"] and total == g["total"]
+    P = np.array(g["topk_ids"]).size
+    assert moe.max_padded(P, g["num_experts"], g["block"]) == g["max_padded"]
+
+
+def test_moe_align_invariants_and_bound():
+    rng = np.random.default_rng(31)
+    for T, top_k, E, block in ((1, 8, 256, 128), (37, 2, 8, 16), (300, 4, 16, 128), (5, 1, 3, 4)):
+        ids = rng.integers(0, E, size=(T, top_k))
+        s, e, total = moe.align(ids, E, block)
+        P = T * top_k
+        assert total % block == 0 and total <= moe.max_padded(P, E, block)
+        valid = s[s < P]
+        assert sorted(valid.tolist()) == list(range(P))          # every pair exactly once
+        assert np.all(s[s >= P] == P)                            # padding carries the one id
+        flat = ids.reshape(-1)
+        for b in range(total // block):
+            blk = s[b * block:(b + 1) * block]
+            assert np.all(flat[blk[blk < P]] == e[b])            # one expert per block
+            assert blk[0] < P                                    # no block is all padding
+        assert np.all(np.diff(e) >= 0)                           # experts in ascending order
+    # the bound is reached: every expert gets one pair
+    s, e, total = moe.align(np.arange(8).reshape(8, 1), 8, 4)
+    assert total == moe.max_padded(8, 8, 4) == 32
+
+
+def _tiny_experts(rng, E, K, N):
+    out = []
+    for _ in range(E):
+        idx = rng.integers(0, 8, size=(K, N), dtype=np.uint8)
+        cb = rng.integers(0, 0x7F, size=(K // 64, N // 8, 8), dtype=np.uint8)   # finite E4M3 bytes
+        ex = rng.integers(117, 128, size=(K // 64, N // 8), dtype=np.uint8)
+        out.append((idx, cb, ex))
+    return out
+
+
+def test_moe_gathered_product_equals_the_routed_definition():
+    """The aligned, gathered, padded form reproduces the pair-by-pair routing
+    definition (an independent loop without sorting), also with a map that
+    takes some experts off this rank."""
+    rng = np.random.default_rng(32)
+    T, top_k, E, K, N, block = 7, 3, 5, 64, 16, 4
+    codes = rng.integers(0, 256, size=(T, K), dtype=np.uint8)
+    codes[(codes & 0x7F) == 0x7F] -= 1
+    scales = rng.integers(120, 130, size=(T, K // 32), dtype=np.uint8)
+    ids = rng.integers(0, E, size=(T, top_k))
+    experts = _tiny_experts(rng, E, K, N)
+    s, e, total = moe.align(ids, E, block)
+    Y = moe.grouped_matmul(codes, scales, top_k, s, e, total, block, experts)
+    assert not np.any(np.isnan(Y))                              # every pair written
+    assert np.array_equal(Y, moe.routed_matmul(codes, scales, ids, experts))
+    emap = np.array([0, -1, 1, -1, 2])                           # experts 1 and 3 are remote
+    local = [experts[0], experts[2], experts[4]]
+    Ym = moe.grouped_matmul(codes, scales, top_k, s, e, total, block, local, emap)
+    assert np.array_equal(Ym, moe.routed_matmul(codes, scales, ids, local, emap))
+    remote = np.isin(ids.reshape(-1), [1, 3])
+    assert np.all(Ym[remote] == 0) and np.array_equal(Ym[~remote], Y[~remote])
