@@ -334,6 +334,30 @@ def rotating_lut3_ms(torch, lbq, images, X, N, ws, reps=5):
     return rotating_ms(torch, call, images, reps)
 
 
+# the MoE layer of the LUT-B write-up's latency table: 256 experts, top-8,
+# hidden 2048, expert intermediate 512 (gate and up side by side: N = 1024)
+MOE_LAYER = {"experts": 256, "top_k": 8, "hidden": 2048, "inter": 512}
+
+
+def moe_expert_images(torch, lbq, workloads, device, seed, K, N, E):
+    """E LUT3 expert images (seeded synthetic indices, codebooks, exponents) at one stride."""
+    experts = [workloads.lut3_device(seed + e, K, N, device) for e in range(E)]
+    images, stride = lbq.pack_lut3_experts(experts)
+    del experts
+    return images, stride
+
+
+def moe_inputs(torch, lbq, workloads, device, T, top_k, E, K):
+    """Seeded uniform routing (top_k distinct experts per token), its alignment
+    on the device, and MXFP8 activations [T, K] drawn in the format."""
+    import numpy as np
+    rng = np.random.default_rng(7 + T)
+    ids = np.stack([rng.choice(E, size=top_k, replace=False) for _ in range(T)]).astype(np.int32)
+    aligned = lbq.moe_align(torch.from_numpy(ids).to(device), E)
+    codes, scales = workloads.mx_activations_host(8 + T, T, K)
+    return aligned, torch.from_numpy(codes).to(device), torch.from_numpy(scales).to(device)
+
+
 def weight_copies(img0, l2_bytes, minimum=3):
     """img0 plus clones so that the copies together exceed 3x L2."""
     copies = max(minimum, (3 * l2_bytes) // img0.numel() + 1)
@@ -497,6 +521,43 @@ def _secondary_measurements(torch, lbq, workloads, device, peaks, quick):
                                      "activations": "INT8, one FP32 scale per 32 k (lbq_quantize_int8), once per "
                                                     "shared X"}
     del g, wstep
+    # grouped MoE GEMM of LUT3 experts x MXFP8 activations at the write-up's
+    # layer shape (E=256, top-8, H=2048, I=512): the gate/up GEMM (K=2048,
+    # N=1024) and the down GEMM (K=512, N=2048, one row per pair), with the
+    # device alignment, at 1, 16, 256 and 4096 tokens
+    E, top_k, H, I = MOE_LAYER["experts"], MOE_LAYER["top_k"], MOE_LAYER["hidden"], MOE_LAYER["inter"]
+    img1, st1 = moe_expert_images(torch, lbq, workloads, device, 1000, H, 2 * I, E)
+    img2, st2 = moe_expert_images(torch, lbq, workloads, device, 5000, I, H, E)
+    for T in (1, 16, 256, 4096):
+        aligned, c1, s1 = moe_inputs(torch, lbq, workloads, device, T, top_k, E, H)
+        ids_flat = None
+        import numpy as np
+        rng = np.random.default_rng(7 + T)
+        ids_flat = torch.from_numpy(np.stack([rng.choice(E, size=top_k, replace=False)
+                                              for _ in range(T)]).astype(np.int32).reshape(-1, 1)).to(device)
+        al2 = lbq.moe_align(ids_flat, E)
+        c2h, s2h = workloads.mx_activations_host(9 + T, T * top_k, I)
+        c2, s2 = torch.from_numpy(c2h).to(device), torch.from_numpy(s2h).to(device)
+        Y1 = torch.empty((T * top_k, 2 * I), dtype=torch.bfloat16, device=device)
+        Y2 = torch.empty((T * top_k, H), dtype=torch.bfloat16, device=device)
+        ids_dev = ids_flat.view(T, top_k)
+
+        def layer(_img, s):
+            lbq.lbq_moe_align(ids_dev.data_ptr(), T * top_k, E, 128, None, aligned[0].data_ptr(),
+                              aligned[1].data_ptr(), aligned[2].data_ptr(), aligned[0].numel(), s)
+            lbq.lbq_moe_lut3_mx_gemm(c1.data_ptr(), s1.data_ptr(), T, top_k, H, 2 * I, aligned[0].data_ptr(),
+                                     aligned[1].data_ptr(), aligned[2].data_ptr(), aligned[0].numel(),
+                                     img1.data_ptr(), st1, E, Y1.data_ptr(), 1, s)
+            lbq.lbq_moe_lut3_mx_gemm(c2.data_ptr(), s2.data_ptr(), T * top_k, 1, I, H, al2[0].data_ptr(),
+                                     al2[1].data_ptr(), al2[2].data_ptr(), al2[0].numel(),
+                                     img2.data_ptr(), st2, E, Y2.data_ptr(), 1, s)
+
+        ms = rotating_ms(torch, layer, [None], reps=10)
+        fl = 2.0 * T * top_k * (H * 2 * I + I * H)
+        out[f"moe_lut3_mx_layer_t{T}"] = {"us": ms * 1e3, "TFLOPs": fl / ms / 1e9,
+                                          "what": "align + gate/up GEMM + down GEMM (E=256, top-8, H=2048, I=512)"}
+        del c1, s1, c2, s2, Y1, Y2, aligned, al2
+    del img1, img2
     # generic b-bit affine GEMV, b = 1..8, at the gate/up shape K=4096 N=14336
     # g64, batch 1 (and batch 4 for 3 bits), FP16 X: GB/s of the format's bytes
     K, N, group = 4096, 14336, 64
@@ -681,6 +742,8 @@ PROFILE_CASES = {
     "c5mx2048": (4096, 14336, 0, "lut3mx", "mxfp8", 2048, None),
     "affine2": (4096, 14336, 64, "affine2", "f16", 1, None),
     "w4a8gate": (4096, 14336, 32, "w4a8", "f16", 1, None),
+    # grouped MoE GEMM (E=256, top-8, H=2048 -> 2 x I=1024), 256 tokens; N is the gate/up width
+    "moe256": (2048, 1024, 0, "moe", "mxfp8", 256, None),
     "affine3": (4096, 14336, 64, "affine3", "f16", 1, None),
 }
 
@@ -718,6 +781,16 @@ def run_profile_case(name):
         torch.cuda.synchronize()
         lbq.device_status()
         print(f"profile case {name}: {len(images)} launches of K={K} N={N} M={M}", flush=True)
+        return 0
+    if mode == "moe":
+        E, top_k, T = MOE_LAYER["experts"], MOE_LAYER["top_k"], M
+        images, stride = moe_expert_images(torch, lbq, workloads, device, 1000, K, N, E)
+        aligned, codes, scales = moe_inputs(torch, lbq, workloads, device, T, top_k, E, K)
+        for _ in range(3):
+            lbq.moe_lut3_mx_gemm(codes, scales, top_k, aligned, images, stride, E, N)
+        torch.cuda.synchronize()
+        lbq.device_status()
+        print(f"profile case {name}: 3 launches of T={T} top_k={top_k} E={E} K={K} N={N}", flush=True)
         return 0
     if mode == "w4a8":
         # W4A8 batch-1 GEMV on asym INT4 weights: X quantised once, weight copies larger than L2

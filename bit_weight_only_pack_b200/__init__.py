@@ -5,7 +5,8 @@ symmetric or asymmetric with an int8 zero point) and 3-bit LUT weights
 (E4M3 codebook per 8 x 64 tile, UE8M0 exponent), as a decode GEMV / skinny
 GEMM and as a tcgen05 prefill GEMM; LUT3 weights with MXFP8 activations on the
 block-scaled FP8 tensor path; generic 1..8-bit affine weights as a decode GEMV;
-INT4 weights with dynamic INT8 activations (W4A8) as a decode GEMV.
+INT4 weights with dynamic INT8 activations (W4A8) as a decode GEMV; a grouped
+MoE GEMM of LUT3 experts with MXFP8 activations gathered by expert.
 The work is done by liblbq.so (C ABI in include/lbq.h); this package is its
 thin Python binding.
 """
@@ -19,4 +20,5 @@ from .binding import (  # noqa: F401
     affine_gemv, pack_affine, unpack_affine_canonical, lbq_affine_gemv, lbq_affine_packed_size, lbq_pack_affine,
     lbq_unpack_affine_canonical, quantize_int8, w4a8_gemv, lbq_quantize_int8, lbq_w4a8_gemv,
     w4a8_gemv_grouped, lbq_w4a8_gemv_grouped, lbq_debug_w4a8_tiled, make_w4a8_items,
+    MOE_BLOCK, moe_align, moe_lut3_mx_gemm, pack_lut3_experts, lbq_moe_align, lbq_moe_lut3_mx_gemm, lbq_moe_max_padded,
 )

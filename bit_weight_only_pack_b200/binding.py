@@ -79,6 +79,10 @@ _SIGS = {
     "lbq_w4a8_gemv_grouped": ([ctypes.POINTER(lbq_w4a8_item), _c_int, _c_int, _c_int, _c_int, _c_int, _vp],
                               _c_int),
     "lbq_debug_w4a8_tiled": ([_c_int], None),
+    "lbq_moe_max_padded": ([_c_int, _c_int, _c_int, ctypes.POINTER(_c_int)], _c_int),
+    "lbq_moe_align": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_int, _vp], _c_int),
+    "lbq_moe_lut3_mx_gemm": ([_vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_int, _vp, _c_size, _c_int,
+                              _vp, _c_int, _vp], _c_int),
     "lbq_debug_force_splits": ([_c_int], None),
     "lbq_debug_force_skinny": ([_c_int], None),
     "lbq_debug_force_tc": ([_c_int], None),
@@ -257,6 +261,24 @@ def make_w4a8_items(rows):
 def lbq_debug_w4a8_tiled(on):
     """Test hook: batch-1 W4A8 on the tiled kernel instead of the staged one."""
     _lib.lbq_debug_w4a8_tiled(1 if on else 0)
+
+
+def lbq_moe_max_padded(num_pairs, num_experts, block):
+    n = _c_int(0)
+    _check(_lib.lbq_moe_max_padded(num_pairs, num_experts, block, ctypes.byref(n)))
+    return n.value
+
+
+def lbq_moe_align(topk_ids, num_pairs, num_experts, block, expert_map, sorted_ids, expert_ids, total, max_padded,
+                  stream):
+    _check(_lib.lbq_moe_align(topk_ids, num_pairs, num_experts, block, expert_map, sorted_ids, expert_ids, total,
+                              max_padded, stream))
+
+
+def lbq_moe_lut3_mx_gemm(codes, scales, T, top_k, K, N, sorted_ids, expert_ids, total, max_padded, images,
+                         image_stride, num_local_experts, Y, y_dtype, stream):
+    _check(_lib.lbq_moe_lut3_mx_gemm(codes, scales, T, top_k, K, N, sorted_ids, expert_ids, total, max_padded, images,
+                                     image_stride, num_local_experts, Y, y_dtype, stream))
 
 
 def lbq_set_option(option, value):
@@ -545,6 +567,53 @@ def w4a8_gemv_grouped(problems, group, mode, y_dtype="f16"):
         rows.append((xq.data_ptr(), sx.data_ptr(), img.data_ptr(), Y.data_ptr(), N))
     lbq_w4a8_gemv_grouped(make_w4a8_items(rows), len(rows), K, group, _mode(mode), _dt(Ys[0]), _stream())
     return Ys
+
+
+MOE_BLOCK = 128  # rows per tile of the grouped GEMM = the alignment block
+
+
+def moe_align(topk_ids, num_experts, expert_map=None, block=MOE_BLOCK):
+    """(sorted_ids int32 [max_padded], expert_ids int32 [max_padded / block],
+    total int32 [1]) on the device for topk_ids int32 [T, top_k]."""
+    torch = _torch()
+    _need_cuda(topk_ids, expert_map)
+    P = topk_ids.numel()
+    mp = lbq_moe_max_padded(P, num_experts, block)
+    s = torch.empty(mp, dtype=torch.int32, device=topk_ids.device)
+    e = torch.empty(mp // block, dtype=torch.int32, device=topk_ids.device)
+    t = torch.empty(1, dtype=torch.int32, device=topk_ids.device)
+    lbq_moe_align(topk_ids.data_ptr(), P, num_experts, block, expert_map.data_ptr() if expert_map is not None else None,
+                  s.data_ptr(), e.data_ptr(), t.data_ptr(), mp, _stream())
+    return s, e, t
+
+
+def pack_lut3_experts(experts):
+    """One uint8 buffer holding every expert's LUT3 image at a fixed stride:
+    experts = [(idx, codebooks, exponents), ...] (CUDA tensors, one K, N).
+    Returns (images, stride)."""
+    torch = _torch()
+    K, N = experts[0][0].shape
+    size = lbq_packed_size(K, N, 0, MODES["lut3"])
+    stride = -(-size // 256) * 256
+    buf = torch.empty(stride * len(experts), dtype=torch.uint8, device=experts[0][0].device)
+    for i, (idx, cb, ex) in enumerate(experts):
+        _need_cuda(idx, cb, ex)
+        lbq_pack_lut3(idx.data_ptr(), cb.data_ptr(), ex.data_ptr(), K, N, buf.data_ptr() + i * stride, stride,
+                      _stream())
+    return buf, stride
+
+
+def moe_lut3_mx_gemm(codes, scales, top_k, aligned, images, stride, num_local_experts, N, y_dtype="bf16", Y=None):
+    """Y [T * top_k, N] of the grouped GEMM; aligned = moe_align(...) with block 128."""
+    torch = _torch()
+    sorted_ids, expert_ids, total = aligned
+    _need_cuda(codes, scales, sorted_ids, expert_ids, total, images, Y)
+    T, K = codes.shape
+    Y = _out_dt(T * top_k, N, y_dtype, codes.device) if Y is None else Y
+    lbq_moe_lut3_mx_gemm(codes.data_ptr(), scales.data_ptr(), T, top_k, K, N, sorted_ids.data_ptr(),
+                         expert_ids.data_ptr(), total.data_ptr(), sorted_ids.numel(), images.data_ptr(), stride,
+                         num_local_experts, Y.data_ptr(), _dt(Y), _stream())
+    return Y
 
 
 def device_status():

@@ -1,0 +1,337 @@
+// Grouped MoE GEMM: LUT3 expert weights x MXFP8 activations, token rows
+// gathered through sorted_token_ids, plus the alignment that produces them.
+//
+// The vLLM PR 62759 write-up's native kernel is a grouped GEMM over the routed
+// experts: moe_align_block_size lists each expert's (token, choice) pairs
+// contiguously, padded to the M block, and the kernel takes one expert per M
+// block, gathers the token rows of A through the list (a padding entry's row
+// is filled with zeros through the copy's source size), and writes zeros for
+// the valid rows of a block whose expert is not on this rank.
+//
+// Here the product is the LUT3 x MXFP8 kernel of gemm_mx.cuh with a 128-token
+// tile (the write-up's M block) and three changes:
+//  * warps 10..13 gather: thread g owns row g of the block; per k-block it
+//    copies its token's 128 code bytes as eight 16-byte cp.async into the
+//    128-byte-swizzled operand tile (the layout a TMA copy would write) and the
+//    token's 4 scale bytes, source size 0 for a padding entry, then makes the
+//    stage's mbarrier track those copies (cp.async.mbarrier.arrive.noinc);
+//  * warp 0 copies the block's expert weights (indices, codebook and exponent
+//    rows) with bulk copies from that expert's image (the images sit at a fixed
+//    stride, so no per-expert tensor map is needed); for a non-local expert it
+//    copies nothing and the converters write zero weights;
+//  * the epilogue writes each finished row to Y[pair id] with 16-byte stores
+//    (rows of padding entries are not written).
+#pragma once
+
+#include "gemm_mx.cuh"
+
+namespace lbq {
+
+constexpr int kMoeBM = 128;  // tokens (sorted rows) per tile = the alignment block
+constexpr int kMoeGatherWarps = 4;
+constexpr int kMoeThreads = (2 + kMxConvWarps + kMxEpWarps + kMoeGatherWarps) * 32;
+using MoeStage = MxStage<kMoeBM>;
+constexpr int kMoeSmem = kMxStages * MoeStage::kBytes + kMxABufs * kMxABufBytes + 2 * kMxOutBytes + 1024;
+constexpr uint32_t kMoeColD = 0, kMoeColSF = 128;  // TMEM columns: accumulator, then 16 per A buffer
+constexpr uint32_t kMoeTmemCols = 256;
+
+struct GemmMoeArgs {
+  const uint8_t* codes;         // [T][K] E4M3 activations
+  const uint8_t* scales;        // [T][K/32] UE8M0
+  const int32_t* sorted_ids;    // [max_blocks * 128] pair ids, P = padding
+  const int32_t* expert_ids;    // [max_blocks] local expert of each block (< 0: not on this rank)
+  const int32_t* total;         // device scalar: entries of sorted_ids in use
+  const uint8_t* images;        // local expert e's LUT3 image at images + e * image_stride
+  size_t image_stride;
+  size_t off_i, off_c, off_e;   // region offsets inside an image
+  int s_stride, z_stride;       // codebook / exponent row strides (bytes)
+  void* Y;                      // [P][N]
+  int top_k, P, N, K;
+  int n_tiles, max_blocks, k_blocks, num_experts;
+  int y_bf16;
+};
+
+__device__ __forceinline__ void cp_async4_zfill(uint32_t smem, const void* gmem, int src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" :: "r"(smem), "l"(gmem), "r"(src_bytes) : "memory");
+}
+// The mbarrier completes one of its expected arrivals once every cp.async this
+// thread issued before has landed.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" :: "r"(smem_u32(bar)) : "memory");
+}
+
+__global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const GemmMoeArgs a) {
+  extern __shared__ uint8_t dsmem[];
+  __shared__ __align__(8) uint64_t full_bar[kMxStages], empty_bar[kMxStages];
+  __shared__ __align__(8) uint64_t a_full[kMxABufs], a_empty[kMxABufs], d_full, d_empty;
+  __shared__ uint32_t tmem_base_sh;
+  uint8_t* ring = dsmem + ((1024u - (smem_u32(dsmem) & 1023u)) & 1023u);
+  uint8_t* abuf = ring + (size_t)kMxStages * MoeStage::kBytes;
+  uint8_t* obuf = abuf + (size_t)kMxABufs * kMxABufBytes;  // two output tiles
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // every role derives the same tile sequence from the same total
+  const int nblk = min(max(__ldg(a.total), 0) / kMoeBM, a.max_blocks);
+  const int total_tiles = a.n_tiles * nblk;
+  const int nkb = a.k_blocks;
+  auto expert_of = [&](int mb) {
+    const int e = __ldg(a.expert_ids + mb);
+    return e < a.num_experts ? e : -1;  // ids past the images count as not local
+  };
+
+  if (tid == 0) {
+    for (int i = 0; i < kMxStages; ++i) {
+      mbar_init(&full_bar[i], 1 + kMoeGatherWarps * 32);
+      mbar_init(&empty_bar[i], 1 + kMxConvWarps);
+    }
+    for (int i = 0; i < kMxABufs; ++i) {
+      mbar_init(&a_full[i], kMxConvWarps);
+      mbar_init(&a_empty[i], 1);
+    }
+    mbar_init(&d_full, 1);
+    mbar_init(&d_empty, kMxEpWarps);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(&tmem_base_sh)), "r"(kMoeTmemCols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ expert weights
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      const int nt = tile / nblk, mb = tile - nt * nblk;  // blocks inner: one expert's blocks are adjacent
+      const int e = expert_of(mb);
+      const int rows = min(kMxBN, a.N - nt * kMxBN);  // a multiple of 8
+      const int groups = rows >> 3;
+      const uint8_t* img = a.images + (size_t)(e < 0 ? 0 : e) * a.image_stride;
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
+        const int s = it % kMxStages;
+        if (lane == 0 && it >= kMxStages && !mbar_wait(&empty_bar[s], ((it / kMxStages) & 1) ^ 1)) ok = false;
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (!ok) break;
+        uint8_t* st = ring + (size_t)s * MoeStage::kBytes;
+        if (lane == 0)
+          mbar_arrive_expect_tx(&full_bar[s], e < 0 ? 0u : (uint32_t)(2 * rows * 24 + 2 * 16 * groups));
+        __syncwarp();
+        if (e >= 0) {
+          if (lane < 2) {
+            const int kt = kb * 2 + lane;
+            bulk_load(st + MoeStage::kOffI + lane * (kMxBN * 24),
+                      img + a.off_i + ((size_t)kt * a.N + nt * kMxBN) * 24, (uint32_t)(rows * 24), &full_bar[s]);
+          }
+          const int g = lane & 15;
+          if (g < groups) {
+            const size_t row = (size_t)(nt * (kMxBN / 8) + g);
+            if (lane < 16)
+              bulk_load(st + MoeStage::kOffC + g * 16, img + a.off_c + row * a.s_stride + (size_t)kb * 16, 16u,
+                        &full_bar[s]);
+            else
+              bulk_load(st + MoeStage::kOffE + g * 16, img + a.off_e + row * a.z_stride + (size_t)(kb * 2 / 16) * 16,
+                        16u, &full_bar[s]);
+          }
+        }
+      }
+    }
+    // every copy this CTA issued lands before it may exit
+    if (lane == 0)
+      for (int v = max(0, it - kMxStages); v < it; ++v)
+        if (!mbar_wait(&full_bar[v % kMxStages], (v / kMxStages) & 1)) break;
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ scale copies + MMA issuer
+    if (lane == 0) {
+      int it = 0, t_iter = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t_iter) {
+        if (t_iter >= 1 && !mbar_wait(&d_empty, (t_iter - 1) & 1)) break;
+        tc_fence_after();
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kMxStages, b = it % kMxABufs;
+          if (!mbar_wait(&full_bar[s], (it / kMxStages) & 1)) { ok = false; break; }
+          if (!mbar_wait(&a_full[b], (it / kMxABufs) & 1)) { ok = false; break; }
+          fence_proxy_async();  // the gathered rows (cp.async writes), to the tensor core's proxy
+          tc_fence_after();
+          const uint32_t ab = smem_u32(abuf + (size_t)b * kMxABufBytes);
+          const uint32_t xb = smem_u32(ring + (size_t)s * MoeStage::kBytes + MoeStage::kOffX);
+          const uint32_t sf = tmem + kMoeColSF + (uint32_t)b * 16;
+          tmem_cp_sf(sf, sf_desc(ab + kMxOffSA));
+          tmem_cp_sf(sf + 4, sf_desc(ab + kMxOffSB));
+#pragma unroll
+          for (uint32_t kk = 0; kk < 4; ++kk) {
+            const uint64_t da = umma_desc_sw128(ab + kMxOffA) + (uint64_t)(kk * 2);
+            const uint64_t db = umma_desc_sw128(xb) + (uint64_t)(kk * 2);
+            umma_mx(tmem + kMoeColD, da, db, umma_idesc_mx(kk, kMoeBM), sf | (kk << 30), (sf + 4) | (kk << 30),
+                    (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty_bar[s]);
+          umma_commit(&a_empty[b]);
+        }
+        if (ok) umma_commit(&d_full);
+      }
+    }
+  } else if (warp < 2 + kMxConvWarps) {
+    // ------------------------------------------------------------------ converters
+    const int r = (warp - 2) * 32 + lane;  // channel within the tile / token row of the block
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      const int nt = tile / nblk, mb = tile - nt * nblk;
+      const bool row_ok = nt * kMxBN + r < a.N && expert_of(mb) >= 0;
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
+        const int s = it % kMxStages, b = it % kMxABufs;
+        if (ok && !mbar_wait(&full_bar[s], (it / kMxStages) & 1)) ok = false;
+        if (ok && it >= kMxABufs && !mbar_wait(&a_empty[b], ((it / kMxABufs) & 1) ^ 1)) ok = false;
+        tc_fence_after();
+        const uint8_t* st = ring + (size_t)s * MoeStage::kBytes;
+        uint8_t* ab = abuf + (size_t)b * kMxABufBytes;
+        if (ok) mx_convert_block<kMoeBM>(st, ab, r, kb, row_ok);
+        fence_proxy_async();  // the operand and scale writes, to the tensor core's proxy
+        __syncwarp();
+        if (lane == 0 && ok) {
+          mbar_arrive(&a_full[b]);
+          mbar_arrive(&empty_bar[s]);
+        }
+      }
+    }
+  } else if (warp < 2 + kMxConvWarps + kMxEpWarps) {
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int r = 32 * q + lane;  // channel within the tile
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+    const int ew = warp - (2 + kMxConvWarps);  // 0..3: rows 8 ew .. 8 ew + 7 of each 32-row chunk
+    // every epilogue warp runs every chunk and its named barrier, also after a
+    // timed-out wait (then it loads and stores nothing)
+    int t_iter = 0, ob = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++t_iter) {
+      const int nt = tile / nblk, mb = tile - nt * nblk;
+      const int rows = min(kMxBN, a.N - nt * kMxBN);
+      if (ok && !mbar_wait(&d_full, t_iter & 1)) ok = false;
+      tc_fence_after();
+#pragma unroll 1
+      for (int j = 0; j < kMoeBM / 32; ++j) {
+        uint32_t v[32];
+        if (ok) {
+          tmem_ld32(lane_base + kMoeColD + (uint32_t)(j * 32), v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        }
+        if (j == kMoeBM / 32 - 1) {  // the accumulator is in registers: the MMAs may start the next tile
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0 && ok) mbar_arrive(&d_empty);
+        }
+        uint8_t* ot = obuf + (size_t)ob * kMxOutBytes;  // [32 rows][128 channels]
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float f = __uint_as_float(v[i]);
+          const uint16_t h = a.y_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(f)) : __half_as_ushort(__float2half_rn(f));
+          *reinterpret_cast<uint16_t*>(ot + (i * kMxBN + r) * 2) = h;
+        }
+        consumer_named_sync(2, kMxEpWarps * 32);
+        // rows 8 ew .. 8 ew + 7 of the chunk: two rows per pass, 16 lanes x 16 B each
+#pragma unroll
+        for (int pass = 0; pass < 4; ++pass) {
+          const int i = 8 * ew + 2 * pass + (lane >> 4), cl = lane & 15;
+          const int sid = __ldg(a.sorted_ids + (size_t)mb * kMoeBM + j * 32 + i);
+          if (ok && sid >= 0 && sid < a.P && cl * 8 < rows) {
+            const uint4 val = *reinterpret_cast<const uint4*>(ot + i * (kMxBN * 2) + cl * 16);
+            *reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.Y) + ((size_t)sid * a.N + nt * kMxBN) * 2 + cl * 16) = val;
+          }
+        }
+        ob ^= 1;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ token-row gather
+    const int g = tid - (2 + kMxConvWarps + kMxEpWarps) * 32;  // row of the block
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      const int nt = tile / nblk, mb = tile - nt * nblk;
+      (void)nt;
+      const int sid = __ldg(a.sorted_ids + (size_t)mb * kMoeBM + g);
+      const bool valid = sid >= 0 && sid < a.P;
+      const int token = valid ? sid / a.top_k : 0;
+      const uint8_t* xsrc = a.codes + (size_t)token * a.K;
+      const uint8_t* ssrc = a.scales + (size_t)token * (a.K / 32);
+      const int nb = valid ? 16 : 0;
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
+        const int s = it % kMxStages;
+        if (lane == 0 && it >= kMxStages && !mbar_wait(&empty_bar[s], ((it / kMxStages) & 1) ^ 1)) ok = false;
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (!ok) break;
+        const uint32_t st = smem_u32(ring + (size_t)s * MoeStage::kBytes);
+        const uint32_t dst = st + MoeStage::kOffX + (uint32_t)g * 128u;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          cp_async16_s(dst + (((uint32_t)c ^ (uint32_t)(g & 7)) << 4), xsrc + (size_t)kb * kMxBK + c * 16, nb);
+        cp_async4_zfill(st + MoeStage::kOffS + (uint32_t)g * 16u + (uint32_t)(kb & 3) * 4u, ssrc + (size_t)kb * 4,
+                        valid ? 4 : 0);
+        cp_async_arrive_noinc(&full_bar[s]);
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's copies land before it may exit
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kMoeTmemCols) : "memory");
+  }
+}
+
+// moe_align_block_size on one CTA: per-expert counts, runs padded to `block`
+// in ascending expert order, the padding id P everywhere else, and each pair's
+// id scattered into its expert's run (pairs of one expert in arrival order of
+// the atomics: any order is as valid, each output row depends on its own pair).
+// Shared memory: counts [E], run starts [E + 1], cursors [E].
+__global__ void __launch_bounds__(1024) moe_align_kernel(const int32_t* __restrict__ topk_ids, int P, int E,
+                                                         int block, const int32_t* __restrict__ expert_map,
+                                                         int32_t* __restrict__ sorted_ids,
+                                                         int32_t* __restrict__ expert_ids, int32_t* __restrict__ total,
+                                                         int max_padded) {
+  extern __shared__ int moe_sm[];
+  int* cnt = moe_sm;
+  int* start = cnt + E;
+  int* cur = start + E + 1;
+  const int tid = threadIdx.x, nt = blockDim.x;
+  for (int e = tid; e < E; e += nt) { cnt[e] = 0; cur[e] = 0; }
+  __syncthreads();
+  for (int p = tid; p < P; p += nt) {
+    const int e = topk_ids[p];
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int o = 0;
+    for (int e = 0; e < E; ++e) {
+      start[e] = o;
+      o += (cnt[e] + block - 1) / block * block;
+    }
+    start[E] = o;
+    *total = o;
+  }
+  for (int i = tid; i < max_padded; i += nt) sorted_ids[i] = P;
+  for (int b = tid; b < max_padded / block; b += nt) expert_ids[b] = -1;
+  __syncthreads();
+  for (int e = tid; e < E; e += nt) {
+    const int le = expert_map ? expert_map[e] : e;
+    for (int b = start[e] / block; b < start[e + 1] / block; ++b) expert_ids[b] = le;
+  }
+  for (int p = tid; p < P; p += nt) {
+    const int e = topk_ids[p];
+    if (e >= 0 && e < E) sorted_ids[start[e] + atomicAdd(&cur[e], 1)] = p;
+  }
+}
+
+}  // namespace lbq

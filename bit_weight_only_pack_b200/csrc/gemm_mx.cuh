@@ -55,17 +55,26 @@ constexpr int kMxStages = 3;          // TMA ring
 constexpr int kMxABufs = 4;           // converted A tiles + scale atoms
 constexpr int kMxConvWarps = 4, kMxEpWarps = 4;
 constexpr int kMxThreads = (2 + kMxConvWarps + kMxEpWarps) * 32;
-// stage layout
-constexpr int kMxOffX = 0;                            // 256 x 128 B codes, 128-byte swizzle
-constexpr int kMxOffI = kMxOffX + kMxBM * kMxBK;      // 2 tiles x 128 channels x 24 B indices
-constexpr int kMxOffC = kMxOffI + 2 * kMxBN * 24;     // codebooks: 16 groups x 16 B (2 tiles x 8 B)
-constexpr int kMxOffE = kMxOffC + 16 * 16;            // exponents: 16 groups x 16 B (tiles in a 16-tile row)
-constexpr int kMxOffS = kMxOffE + 16 * 16;            // token scales: 256 x 16 B (4 blocks of a 512-k row)
-constexpr int kMxStageBytes = (kMxOffS + kMxBM * 16 + 1023) / 1024 * 1024;
+// stage layout for a tile of BM tokens
+template <int BM>
+struct MxStage {
+  static constexpr int kOffX = 0;                          // BM x 128 B codes, 128-byte swizzle
+  static constexpr int kOffI = kOffX + BM * kMxBK;         // 2 tiles x 128 channels x 24 B indices
+  static constexpr int kOffC = kOffI + 2 * kMxBN * 24;     // codebooks: 16 groups x 16 B (2 tiles x 8 B)
+  static constexpr int kOffE = kOffC + 16 * 16;            // exponents: 16 groups x 16 B (tiles in a 16-tile row)
+  static constexpr int kOffS = kOffE + 16 * 16;            // token scales: BM x 16 B (4 blocks of a 512-k row)
+  static constexpr int kBytes = (kOffS + BM * 16 + 1023) / 1024 * 1024;
+};
+constexpr int kMxOffX = MxStage<kMxBM>::kOffX;
+constexpr int kMxOffI = MxStage<kMxBM>::kOffI;
+constexpr int kMxOffC = MxStage<kMxBM>::kOffC;
+constexpr int kMxOffE = MxStage<kMxBM>::kOffE;
+constexpr int kMxOffS = MxStage<kMxBM>::kOffS;
+constexpr int kMxStageBytes = MxStage<kMxBM>::kBytes;
 // A buffer layout
 constexpr int kMxOffA = 0;                            // 128 x 128 B weights, 128-byte swizzle
 constexpr int kMxOffSA = kMxBN * kMxBK;               // A scale atom, 512 B
-constexpr int kMxOffSB = kMxOffSA + 512;              // two B scale atoms, 1024 B
+constexpr int kMxOffSB = kMxOffSA + 512;              // B scale atoms (one per 128 tokens), up to 1024 B
 constexpr int kMxABufBytes = (kMxOffSB + 1024 + 1023) / 1024 * 1024;
 constexpr int kMxOutBytes = 32 * kMxBN * 2;          // one [32 tokens][128 channels] output tile
 constexpr int kMxSmem = kMxStages * kMxStageBytes + kMxABufs * kMxABufBytes + 2 * kMxOutBytes + 1024;
@@ -84,8 +93,8 @@ struct GemmMxArgs {
 // Instruction descriptor of kind::mxf8f6f4.block_scale: A = B = E4M3, K-major,
 // D = FP32, UE8M0 scales, N = 256, M = 128; the scale IDs pick the k-step's
 // byte of each 32-bit scale column.
-__host__ __device__ constexpr uint32_t umma_idesc_mx(uint32_t step) {
-  return ((uint32_t)(kMxBM >> 3) << 17) | (1u << 23) | ((uint32_t)(kMxBN >> 4) << 24) | (step << 29) | (step << 4);
+__host__ __device__ constexpr uint32_t umma_idesc_mx(uint32_t step, int n = kMxBM) {
+  return ((uint32_t)(n >> 3) << 17) | (1u << 23) | ((uint32_t)(kMxBN >> 4) << 24) | (step << 29) | (step << 4);
 }
 
 // Shared-memory descriptor of a scale atom for tcgen05.cp: 32 rows of 16 bytes,
@@ -110,6 +119,61 @@ __device__ __forceinline__ void umma_mx(uint32_t d_tmem, uint64_t a_desc, uint64
                "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
                :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(acc)
                : "memory");
+}
+
+// Converter work of one k-block for channel r of the tile: the channel's 128
+// E4M3 weights into the swizzled A tile, its tile exponents into the A scale
+// atom (scale 1.0 and zero weights when the channel does not exist, row_ok
+// false), and the k-block's scale bytes of tokens r + 128 hh into the B scale
+// atoms. st is the stage (layout MxStage<BM>), ab the A buffer.
+template <int BM>
+__device__ __forceinline__ void mx_convert_block(const uint8_t* st, uint8_t* ab, int r, int kb, bool row_ok) {
+  using L = MxStage<BM>;
+  // weights: 2 tiles x 2 chunks x 4 groups of 8 k -> E4M3 bytes, 16 per swizzled chunk
+  const uint32_t arow = smem_u32(ab + kMxOffA) + (uint32_t)r * 128u;
+  uint32_t eword = 0x7F7F7F7Fu;  // scale 1.0 for channels past N
+  if (row_ok) {
+    uint32_t e2 = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(st + L::kOffI + h * (kMxBN * 24) + r * 24);
+      const uint2 cb = *reinterpret_cast<const uint2*>(st + L::kOffC + (r >> 3) * 16 + h * 8);
+      const uint32_t e = st[L::kOffE + (r >> 3) * 16 + ((kb * 2 + h) & 15)];
+      e2 |= (e | (e << 8)) << (16 * h);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const uint32_t wa = w[3 * c], wb = w[3 * c + 1], wc = w[3 * c + 2];
+#pragma unroll
+        for (int tp = 0; tp < 2; ++tp) {
+          uint32_t o[4];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int t = 2 * tp + u;
+            const uint32_t sel = lut3_selector(t < 2 ? wa : wb, wc, t);
+            o[2 * u] = prmt(cb.x, cb.y, sel);
+            o[2 * u + 1] = prmt(cb.x, cb.y, sel >> 16);
+          }
+          const uint32_t chunk = (uint32_t)(4 * h + 2 * c + tp);  // 16-k chunk of the 128-k block
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                       :: "r"(arow + ((chunk ^ (uint32_t)(r & 7)) << 4)), "r"(o[0]), "r"(o[1]), "r"(o[2]),
+                          "r"(o[3]) : "memory");
+        }
+      }
+    }
+    eword = e2;
+  } else {
+#pragma unroll
+    for (uint32_t chunk = 0; chunk < 8; ++chunk)
+      asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" :: "r"(arow + (chunk << 4)), "r"(0u) : "memory");
+  }
+  const uint32_t atom_off = (uint32_t)(16 * (r & 31) + 4 * (r >> 5));
+  *reinterpret_cast<uint32_t*>(ab + kMxOffSA + atom_off) = eword;
+  // token scales of this block: bytes 4 (kb % 4) .. +3 of each token's 16-byte row
+#pragma unroll
+  for (int hh = 0; hh < BM / 128; ++hh) {
+    const uint32_t sw = *reinterpret_cast<const uint32_t*>(st + L::kOffS + (hh * 128 + r) * 16 + (kb & 3) * 4);
+    *reinterpret_cast<uint32_t*>(ab + kMxOffSB + hh * 512 + atom_off) = sw;
+  }
 }
 
 __global__ void __launch_bounds__(kMxThreads, 1)
@@ -232,53 +296,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         tc_fence_after();
         const uint8_t* st = ring + (size_t)s * kMxStageBytes;
         uint8_t* ab = abuf + (size_t)b * kMxABufBytes;
-        if (ok) {
-          // weights: 2 tiles x 2 chunks x 4 groups of 8 k -> E4M3 bytes, 16 per swizzled chunk
-          const uint32_t arow = smem_u32(ab + kMxOffA) + (uint32_t)r * 128u;
-          uint32_t eword = 0x7F7F7F7Fu;  // scale 1.0 for channels past N
-          if (row_ok) {
-            uint32_t e2 = 0;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint32_t* w = reinterpret_cast<const uint32_t*>(st + kMxOffI + h * (kMxBN * 24) + r * 24);
-              const uint2 cb = *reinterpret_cast<const uint2*>(st + kMxOffC + (r >> 3) * 16 + h * 8);
-              const uint32_t e = st[kMxOffE + (r >> 3) * 16 + ((kb * 2 + h) & 15)];
-              e2 |= (e | (e << 8)) << (16 * h);
-#pragma unroll
-              for (int c = 0; c < 2; ++c) {
-                const uint32_t wa = w[3 * c], wb = w[3 * c + 1], wc = w[3 * c + 2];
-#pragma unroll
-                for (int tp = 0; tp < 2; ++tp) {
-                  uint32_t o[4];
-#pragma unroll
-                  for (int u = 0; u < 2; ++u) {
-                    const int t = 2 * tp + u;
-                    const uint32_t sel = lut3_selector(t < 2 ? wa : wb, wc, t);
-                    o[2 * u] = prmt(cb.x, cb.y, sel);
-                    o[2 * u + 1] = prmt(cb.x, cb.y, sel >> 16);
-                  }
-                  const uint32_t chunk = (uint32_t)(4 * h + 2 * c + tp);  // 16-k chunk of the 128-k block
-                  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
-                               :: "r"(arow + ((chunk ^ (uint32_t)(r & 7)) << 4)), "r"(o[0]), "r"(o[1]), "r"(o[2]),
-                                  "r"(o[3]) : "memory");
-                }
-              }
-            }
-            eword = e2;
-          } else {
-#pragma unroll
-            for (uint32_t chunk = 0; chunk < 8; ++chunk)
-              asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" :: "r"(arow + (chunk << 4)), "r"(0u) : "memory");
-          }
-          const uint32_t atom_off = (uint32_t)(16 * (r & 31) + 4 * (r >> 5));
-          *reinterpret_cast<uint32_t*>(ab + kMxOffSA + atom_off) = eword;
-          // token scales of this block: bytes 4 (kb % 4) .. +3 of each token's 16-byte row
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const uint32_t sw = *reinterpret_cast<const uint32_t*>(st + kMxOffS + (hh * 128 + r) * 16 + (kb & 3) * 4);
-            *reinterpret_cast<uint32_t*>(ab + kMxOffSB + hh * 512 + atom_off) = sw;
-          }
-        }
+        if (ok) mx_convert_block<kMxBM>(st, ab, r, kb, row_ok);
         fence_proxy_async();  // the operand and scale writes, to the tensor core's proxy
         __syncwarp();
         if (lane == 0 && ok) {

@@ -35,6 +35,7 @@
 #include "lut3_direct.cuh"
 #include "affine.cuh"
 #include "w4a8.cuh"
+#include "gemm_moe.cuh"
 
 namespace lbq {
 
@@ -1107,6 +1108,15 @@ static lbq_status run_lut3_mx(const uint8_t* codes, const uint8_t* scales, int M
 }
 
 // ----------------------------------------------------------------------------
+// Grouped MoE: LUT3 experts x MXFP8 activations
+// ----------------------------------------------------------------------------
+
+static int moe_max_padded(long long P, int E, int block) {
+  const long long runs = std::min<long long>(P, E);
+  return (int)((P + runs * (block - 1)) / block * block);
+}
+
+// ----------------------------------------------------------------------------
 // Generic b-bit affine weights
 // ----------------------------------------------------------------------------
 
@@ -1746,6 +1756,77 @@ lbq_status lbq_lut3_mx_gemm(const uint8_t* codes, const uint8_t* scales, int M, 
   if (y_dtype != LBQ_DTYPE_F16 && y_dtype != LBQ_DTYPE_BF16) return fail(LBQ_ERR_UNSUPPORTED, "y_dtype %d", y_dtype);
   return run_lut3_mx(codes, scales, M, image, make_layout(K, N, 0, LBQ_MODE_LUT3), Y, y_dtype == LBQ_DTYPE_BF16,
                      static_cast<cudaStream_t>(stream));
+}
+
+lbq_status lbq_moe_max_padded(int num_pairs, int num_experts, int block, int* max_padded) {
+  if (!max_padded) return fail(LBQ_ERR_INVALID_ARG, "max_padded must be non-null");
+  if (num_pairs <= 0 || num_experts <= 0 || block <= 0)
+    return fail(LBQ_ERR_INVALID_ARG, "num_pairs=%d num_experts=%d block=%d must be positive", num_pairs, num_experts, block);
+  const long long bound = (long long)num_pairs + (long long)std::min(num_pairs, num_experts) * (block - 1);
+  if (bound > (1LL << 30)) return fail(LBQ_ERR_INVALID_ARG, "the padded pair list would exceed 2^30 entries");
+  *max_padded = moe_max_padded(num_pairs, num_experts, block);
+  return LBQ_OK;
+}
+
+lbq_status lbq_moe_align(const int32_t* topk_ids, int num_pairs, int num_experts, int block, const int32_t* expert_map,
+                         int32_t* sorted_ids, int32_t* expert_ids, int32_t* total, int max_padded, void* stream) {
+  if (!topk_ids || !sorted_ids || !expert_ids || !total)
+    return fail(LBQ_ERR_INVALID_ARG, "topk_ids, sorted_ids, expert_ids and total must be non-null");
+  if (num_pairs <= 0 || num_experts <= 0 || num_experts > 2048 || block <= 0)
+    return fail(LBQ_ERR_INVALID_ARG, "num_pairs=%d num_experts=%d (1..2048) block=%d", num_pairs, num_experts, block);
+  int need = 0;
+  lbq_status st = lbq_moe_max_padded(num_pairs, num_experts, block, &need);
+  if (st != LBQ_OK) return st;
+  if (max_padded < need) return fail(LBQ_ERR_INVALID_ARG, "max_padded=%d < %d (lbq_moe_max_padded)", max_padded, need);
+  const int smem = (3 * num_experts + 1) * (int)sizeof(int);
+  void* args[] = {(void*)&topk_ids, (void*)&num_pairs, (void*)&num_experts, (void*)&block, (void*)&expert_map,
+                  (void*)&sorted_ids, (void*)&expert_ids, (void*)&total, (void*)&max_padded};
+  return launch_kernel_ex((const void*)moe_align_kernel, dim3(1), dim3(1024), smem, static_cast<cudaStream_t>(stream),
+                          false, args, "MoE align launch");
+}
+
+lbq_status lbq_moe_lut3_mx_gemm(const uint8_t* codes, const uint8_t* scales, int T, int top_k, int K, int N,
+                                const int32_t* sorted_ids, const int32_t* expert_ids, const int32_t* total,
+                                int max_padded, const void* images, size_t image_stride, int num_local_experts,
+                                void* Y, int y_dtype, void* stream) {
+  lbq_status st = check_lut3_shape(K, N);
+  if (st != LBQ_OK) return st;
+  if (K % 128) return fail(LBQ_ERR_UNSUPPORTED, "lbq_moe_lut3_mx_gemm needs K %% 128 == 0 (K=%d)", K);
+  if (T <= 0 || top_k <= 0 || num_local_experts <= 0)
+    return fail(LBQ_ERR_INVALID_ARG, "T=%d top_k=%d num_local_experts=%d must be positive", T, top_k, num_local_experts);
+  if ((long long)T * top_k >= (1LL << 30)) return fail(LBQ_ERR_INVALID_ARG, "T * top_k too large");
+  if (max_padded <= 0 || max_padded % kMoeBM)
+    return fail(LBQ_ERR_INVALID_ARG, "max_padded=%d must be a positive multiple of %d", max_padded, kMoeBM);
+  if (!codes || !scales || !sorted_ids || !expert_ids || !total || !images || !Y)
+    return fail(LBQ_ERR_INVALID_ARG, "codes, scales, sorted_ids, expert_ids, total, images and Y must be non-null");
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(images) || !aligned16(Y) || image_stride % 16)
+    return fail(LBQ_ERR_INVALID_ARG, "codes, scales, images, Y and image_stride must be 16-byte aligned");
+  if (y_dtype != LBQ_DTYPE_F16 && y_dtype != LBQ_DTYPE_BF16) return fail(LBQ_ERR_UNSUPPORTED, "y_dtype %d", y_dtype);
+  const Layout L = make_layout(K, N, 0, LBQ_MODE_LUT3);
+  if (image_stride < L.total) return fail(LBQ_ERR_INVALID_ARG, "image_stride %zu < image size %zu", image_stride, L.total);
+  GemmMoeArgs a{};
+  a.codes = codes;
+  a.scales = scales;
+  a.sorted_ids = sorted_ids;
+  a.expert_ids = expert_ids;
+  a.total = total;
+  a.images = static_cast<const uint8_t*>(images);
+  a.image_stride = image_stride;
+  a.off_i = L.off0; a.off_c = L.off1; a.off_e = L.off2;
+  a.s_stride = (int)L.s_stride; a.z_stride = (int)L.z_stride;
+  a.Y = Y;
+  a.top_k = top_k; a.P = T * top_k; a.N = N; a.K = K;
+  a.n_tiles = (N + kMxBN - 1) / kMxBN;
+  a.max_blocks = max_padded / kMoeBM;
+  a.k_blocks = K / kMxBK;
+  a.num_experts = num_local_experts;
+  a.y_bf16 = y_dtype == LBQ_DTYPE_BF16 ? 1 : 0;
+  const void* fn = (const void*)gemm_moe_lut3_mx_kernel;
+  occupancy_for(fn, kMoeThreads, kMoeSmem);
+  const int grid = (int)std::min<long long>((long long)a.n_tiles * a.max_blocks, num_sms());
+  void* args[] = {&a};
+  return launch_kernel_ex(fn, dim3(grid), dim3(kMoeThreads), kMoeSmem, static_cast<cudaStream_t>(stream), false, args,
+                          "MoE LUT3 x MXFP8 GEMM launch");
 }
 
 }  // extern "C"

@@ -431,6 +431,64 @@ typedef struct {
 lbq_status lbq_w4a8_gemv_grouped(const lbq_w4a8_item* items, int count, int K, int group, int mode, int y_dtype,
                                  void* stream);
 
+/*
+ * Grouped MoE GEMM of LUT3 expert weights with MXFP8 activations (vLLM PR
+ * 62759 write-up: the native grouped GEMM gathers token rows through
+ * sorted_token_ids from moe_align_block_size, takes one expert per M block,
+ * zero-fills the A rows of padding entries through the copy's source size,
+ * and writes zeros for the rows of a block whose expert is not on this rank).
+ *
+ * Pairs: pair p = t * top_k + j is token t's j-th choice, routed to expert
+ * topk_ids[p]; P = T * top_k pairs.
+ *
+ * lbq_moe_max_padded: *max_padded = the largest `total` lbq_moe_align can
+ *   produce, (P + min(P, E) (block - 1)) rounded down to a multiple of block:
+ *   the length to allocate for sorted_ids (and max_padded / block for
+ *   expert_ids). Host only. Errors: LBQ_ERR_INVALID_ARG for non-positive
+ *   arguments or a list longer than 2^30.
+ */
+lbq_status lbq_moe_max_padded(int num_pairs, int num_experts, int block, int* max_padded);
+
+/*
+ * moe_align_block_size on the device (one CTA):
+ *   topk_ids    (device) int32 [num_pairs], expert of each pair, 0 <= id < num_experts
+ *               (other ids are left out of the lists; their output rows are not written)
+ *   expert_map  (device) int32 [num_experts] global -> local expert (negative: not on
+ *               this rank), or null for the identity
+ *   sorted_ids  (device) int32 [max_padded]: each expert's pair ids contiguous (experts in
+ *               ascending id, the pairs of one expert in no fixed order), each run padded
+ *               to a multiple of `block` with the id num_pairs, which also fills the
+ *               entries past the total
+ *   expert_ids  (device) int32 [max_padded / block]: the (mapped) expert of each block,
+ *               -1 past the total
+ *   total       (device) int32 scalar: entries in use
+ * num_experts <= 2048; max_padded >= lbq_moe_max_padded(). Errors before any
+ * launch: LBQ_ERR_INVALID_ARG. Asynchronous on `stream`.
+ */
+lbq_status lbq_moe_align(const int32_t* topk_ids, int num_pairs, int num_experts, int block, const int32_t* expert_map,
+                         int32_t* sorted_ids, int32_t* expert_ids, int32_t* total, int max_padded, void* stream);
+
+/*
+ * The grouped GEMM, tile of 128 sorted rows (lbq_moe_align with block = 128):
+ *   Y[p][n] = sum_k e4m3(codes[p / top_k][k]) 2^(scales[p / top_k][k/32] - 127) * W_e[k][n]
+ * for every pair p listed in a block whose local expert e is in
+ * 0 .. num_local_experts - 1 (W_e the LUT3 decode of expert e's image, every
+ * product exact, FP32 accumulation); Y[p][:] = 0 for pairs of a block with a
+ * negative (or too large) expert id. Rows of pairs that are not listed are not written.
+ *   codes, scales (device) uint8 [T, K] E4M3 and [T, K/32] UE8M0 (lbq_quantize_mxfp8)
+ *   sorted_ids, expert_ids, total (device) from lbq_moe_align(block = 128)
+ *   images  (device) local expert e's lbq_pack_lut3 image (K, N) at images + e * image_stride
+ *   Y       (device) [T * top_k, N] row-major, y_dtype
+ * K % 128 == 0, N % 8 == 0; max_padded the value the lists were sized with
+ * (a multiple of 128); pointers and image_stride 16-byte aligned. Errors
+ * before any launch: LBQ_ERR_INVALID_ARG / LBQ_ERR_UNSUPPORTED. Asynchronous
+ * on `stream`.
+ */
+lbq_status lbq_moe_lut3_mx_gemm(const uint8_t* codes, const uint8_t* scales, int T, int top_k, int K, int N,
+                                const int32_t* sorted_ids, const int32_t* expert_ids, const int32_t* total,
+                                int max_padded, const void* images, size_t image_stride, int num_local_experts,
+                                void* Y, int y_dtype, void* stream);
+
 /* Number of kernel launches the library has enqueued so far in this process. */
 uint64_t lbq_launch_count(void);
 
