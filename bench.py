@@ -352,10 +352,11 @@ def moe_inputs(torch, lbq, workloads, device, T, top_k, E, K):
     on the device, and MXFP8 activations [T, K] drawn in the format."""
     import numpy as np
     rng = np.random.default_rng(7 + T)
-    ids = np.stack([rng.choice(E, size=top_k, replace=False) for _ in range(T)]).astype(np.int32)
-    aligned = lbq.moe_align(torch.from_numpy(ids).to(device), E)
+    ids = torch.from_numpy(np.stack([rng.choice(E, size=top_k, replace=False) for _ in range(T)]).astype(np.int32))
+    ids = ids.to(device)
+    aligned = lbq.moe_align(ids, E)
     codes, scales = workloads.mx_activations_host(8 + T, T, K)
-    return aligned, torch.from_numpy(codes).to(device), torch.from_numpy(scales).to(device)
+    return aligned, torch.from_numpy(codes).to(device), torch.from_numpy(scales).to(device), ids
 
 
 def weight_copies(img0, l2_bytes, minimum=3):
@@ -529,18 +530,12 @@ def _secondary_measurements(torch, lbq, workloads, device, peaks, quick):
     img1, st1 = moe_expert_images(torch, lbq, workloads, device, 1000, H, 2 * I, E)
     img2, st2 = moe_expert_images(torch, lbq, workloads, device, 5000, I, H, E)
     for T in (1, 16, 256, 4096):
-        aligned, c1, s1 = moe_inputs(torch, lbq, workloads, device, T, top_k, E, H)
-        ids_flat = None
-        import numpy as np
-        rng = np.random.default_rng(7 + T)
-        ids_flat = torch.from_numpy(np.stack([rng.choice(E, size=top_k, replace=False)
-                                              for _ in range(T)]).astype(np.int32).reshape(-1, 1)).to(device)
-        al2 = lbq.moe_align(ids_flat, E)
+        aligned, c1, s1, ids_dev = moe_inputs(torch, lbq, workloads, device, T, top_k, E, H)
+        al2 = lbq.moe_align(ids_dev.view(-1, 1), E)  # the down GEMM: one row per pair
         c2h, s2h = workloads.mx_activations_host(9 + T, T * top_k, I)
         c2, s2 = torch.from_numpy(c2h).to(device), torch.from_numpy(s2h).to(device)
         Y1 = torch.empty((T * top_k, 2 * I), dtype=torch.bfloat16, device=device)
         Y2 = torch.empty((T * top_k, H), dtype=torch.bfloat16, device=device)
-        ids_dev = ids_flat.view(T, top_k)
 
         def layer(_img, s):
             lbq.lbq_moe_align(ids_dev.data_ptr(), T * top_k, E, 128, None, aligned[0].data_ptr(),
@@ -785,7 +780,7 @@ def run_profile_case(name):
     if mode == "moe":
         E, top_k, T = MOE_LAYER["experts"], MOE_LAYER["top_k"], M
         images, stride = moe_expert_images(torch, lbq, workloads, device, 1000, K, N, E)
-        aligned, codes, scales = moe_inputs(torch, lbq, workloads, device, T, top_k, E, K)
+        aligned, codes, scales, _ = moe_inputs(torch, lbq, workloads, device, T, top_k, E, K)
         for _ in range(3):
             lbq.moe_lut3_mx_gemm(codes, scales, top_k, aligned, images, stride, E, N)
         torch.cuda.synchronize()
@@ -866,22 +861,23 @@ def run_profile_case(name):
 # time: shape -> (bytes, {source: sha256[:16]}, summary file). Each shape runs
 # once per layer, so the step's traffic per launch is their mean.
 STEP_KERNEL = ("gemv_tmma_kernel (gate/up) and gemv_direct_async_kernel (q/k/v, o, down)")
-STEP_SOURCES = ("gemv_tmma.cuh", "gemv_direct.cuh", "gemv_m1.cuh", "tma.cuh", "common.cuh", "lbq.cu#tmma-plan",
-                "lbq.cu#direct-plan")
+STEP_SOURCES = ("gemv_tmma.cuh", "gemv_direct.cuh", "gemv_m1.cuh", "w4a8.cuh", "tma.cuh", "common.cuh",
+                "lbq.cu#tmma-plan", "lbq.cu#direct-plan")
 STEP_CAPTURE_HASHES = {
     "gemv_tmma.cuh": "d81c29e83ca35ffb",
-    "gemv_direct.cuh": "80c3d5258f32c480",
+    "gemv_direct.cuh": "370710b80822d44e",
     "gemv_m1.cuh": "a992f85dd1acbd76",
-    "tma.cuh": "fc6224a6c6bf092f",
-    "common.cuh": "eb93cb6f87fb3da4",
+    "w4a8.cuh": "9b2ae43b5bafb58f",
+    "tma.cuh": "5f428384c68b0ba7",
+    "common.cuh": "6e369f75860e0aec",
     "lbq.cu#tmma-plan": "e30dce5cede0f3f4",
-    "lbq.cu#direct-plan": "7afca7967200d200",
+    "lbq.cu#direct-plan": "7020bd2977db6eb8",
 }
 STEP_TRAFFIC = {
     "c2qkv": (14980864, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
-    "c2o": (9997312, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
-    "c2gateup": (70369536, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
-    "c2down": (34921728, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
+    "c2o": (9998848, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
+    "c2gateup": (70426368, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
+    "c2down": (34921472, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
 }
 # the planner sections of lbq.cu (kernel choice, launch shape, K split, stages)
 PLAN_MARKERS = {"tmma-plan": ("// M = 1: TMA-fed warp-MMA GEMV", "// Scratch of that kernel for one call"),

@@ -15,10 +15,16 @@
 //    128-byte-swizzled operand tile (the layout a TMA copy would write) and the
 //    token's 4 scale bytes, source size 0 for a padding entry, then makes the
 //    stage's mbarrier track those copies (cp.async.mbarrier.arrive.noinc);
-//  * warp 0 copies the block's expert weights (indices, codebook and exponent
-//    rows) with bulk copies from that expert's image (the images sit at a fixed
-//    stride, so no per-expert tensor map is needed); for a non-local expert it
+//  * warp 0 copies the block's expert weights with bulk copies from that
+//    expert's image (the images sit at a fixed stride, so no per-expert tensor
+//    map is needed): per tile the 16 channel groups' codebook and exponent rows
+//    for the whole K range (contiguous rows of the image: two copies, into a
+//    double-buffered per-tile area), per k-block the two LUT3 tiles' indices.
+//    Every bulk copy is a separate request to the copy unit, so the rows go
+//    once per tile rather than 16 bytes per k-block. For a non-local expert it
 //    copies nothing and the converters write zero weights;
+//  * eight converter warps, one 64-k LUT3 tile of the k-block each (warps
+//    2..5 the first, 6..9 the second);
 //  * the epilogue writes each finished row to Y[pair id] with 16-byte stores
 //    (rows of padding entries are not written).
 #pragma once
@@ -28,12 +34,20 @@
 namespace lbq {
 
 constexpr int kMoeBM = 128;  // tokens (sorted rows) per tile = the alignment block
-constexpr int kMoeGatherWarps = 4;
-constexpr int kMoeThreads = (2 + kMxConvWarps + kMxEpWarps + kMoeGatherWarps) * 32;
+constexpr int kMoeStages = 3;  // ring depth (k-blocks of indices and gathered rows in flight)
+constexpr int kMoeConvWarps = 8, kMoeGatherWarps = 4;
+constexpr int kMoeWarpEp = 2 + kMoeConvWarps;             // first epilogue warp
+constexpr int kMoeWarpGather = kMoeWarpEp + kMxEpWarps;   // first gather warp
+constexpr int kMoeThreads = (kMoeWarpGather + kMoeGatherWarps) * 32;
+constexpr int kMoeMaxK = 8192;
 using MoeStage = MxStage<kMoeBM>;
-constexpr int kMoeSmem = kMxStages * MoeStage::kBytes + kMxABufs * kMxABufBytes + 2 * kMxOutBytes + 1024;
+// fixed part of the dynamic shared memory; two per-tile codebook / exponent
+// areas of moe_meta_bytes(K) follow
+constexpr int kMoeSmemBase = kMoeStages * MoeStage::kBytes + kMxABufs * kMxABufBytes + 2 * kMxOutBytes + 1024;
 constexpr uint32_t kMoeColD = 0, kMoeColSF = 128;  // TMEM columns: accumulator, then 16 per A buffer
 constexpr uint32_t kMoeTmemCols = 256;
+__host__ __device__ constexpr int moe_meta_bytes(int s_stride, int z_stride) { return 16 * (s_stride + z_stride); }
+static_assert(kMoeSmemBase + 2 * moe_meta_bytes(kMoeMaxK / 8, kMoeMaxK / 64) <= 227 * 1024, "MoE GEMM shared memory");
 
 struct GemmMoeArgs {
   const uint8_t* codes;         // [T][K] E4M3 activations
@@ -62,12 +76,16 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
 
 __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const GemmMoeArgs a) {
   extern __shared__ uint8_t dsmem[];
-  __shared__ __align__(8) uint64_t full_bar[kMxStages], empty_bar[kMxStages];
+  __shared__ __align__(8) uint64_t full_bar[kMoeStages], empty_bar[kMoeStages];
   __shared__ __align__(8) uint64_t a_full[kMxABufs], a_empty[kMxABufs], d_full, d_empty;
+  __shared__ __align__(8) uint64_t meta_full[2], meta_empty[2];
   __shared__ uint32_t tmem_base_sh;
   uint8_t* ring = dsmem + ((1024u - (smem_u32(dsmem) & 1023u)) & 1023u);
-  uint8_t* abuf = ring + (size_t)kMxStages * MoeStage::kBytes;
+  uint8_t* abuf = ring + (size_t)kMoeStages * MoeStage::kBytes;
   uint8_t* obuf = abuf + (size_t)kMxABufs * kMxABufBytes;  // two output tiles
+  uint8_t* meta = obuf + 2 * kMxOutBytes;                   // two per-tile areas: codebook rows, exponent rows
+  const int meta_bytes = moe_meta_bytes(a.s_stride, a.z_stride);
+  const int meta_e = 16 * a.s_stride;                        // exponent rows inside an area
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // every role derives the same tile sequence from the same total
@@ -80,13 +98,17 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
   };
 
   if (tid == 0) {
-    for (int i = 0; i < kMxStages; ++i) {
+    for (int i = 0; i < kMoeStages; ++i) {
       mbar_init(&full_bar[i], 1 + kMoeGatherWarps * 32);
-      mbar_init(&empty_bar[i], 1 + kMxConvWarps);
+      mbar_init(&empty_bar[i], 1 + kMoeConvWarps);
     }
     for (int i = 0; i < kMxABufs; ++i) {
-      mbar_init(&a_full[i], kMxConvWarps);
+      mbar_init(&a_full[i], kMoeConvWarps);
       mbar_init(&a_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&meta_full[i], 1);
+      mbar_init(&meta_empty[i], kMoeConvWarps);
     }
     mbar_init(&d_full, 1);
     mbar_init(&d_empty, kMxEpWarps);
@@ -104,46 +126,43 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
 
   if (warp == 0) {
     // ------------------------------------------------------------------ expert weights
-    int it = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-      const int nt = tile / nblk, mb = tile - nt * nblk;  // blocks inner: one expert's blocks are adjacent
-      const int e = expert_of(mb);
-      const int rows = min(kMxBN, a.N - nt * kMxBN);  // a multiple of 8
-      const int groups = rows >> 3;
-      const uint8_t* img = a.images + (size_t)(e < 0 ? 0 : e) * a.image_stride;
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int s = it % kMxStages;
-        if (lane == 0 && it >= kMxStages && !mbar_wait(&empty_bar[s], ((it / kMxStages) & 1) ^ 1)) ok = false;
-        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-        if (!ok) break;
-        uint8_t* st = ring + (size_t)s * MoeStage::kBytes;
-        if (lane == 0)
-          mbar_arrive_expect_tx(&full_bar[s], e < 0 ? 0u : (uint32_t)(2 * rows * 24 + 2 * 16 * groups));
-        __syncwarp();
+    if (lane == 0) {
+      int it = 0, t_iter = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t_iter) {
+        const int nt = tile / nblk, mb = tile - nt * nblk;  // blocks inner: one expert's blocks are adjacent
+        const int e = expert_of(mb);
+        const int rows = min(kMxBN, a.N - nt * kMxBN);  // a multiple of 8
+        const int groups = rows >> 3;
+        const uint8_t* img = a.images + (size_t)(e < 0 ? 0 : e) * a.image_stride;
+        // the tile's codebook and exponent rows (16 consecutive rows of each region)
+        const int mi = t_iter & 1;
+        if (t_iter >= 2 && !mbar_wait(&meta_empty[mi], ((t_iter >> 1) & 1) ^ 1)) { ok = false; break; }
+        uint8_t* mt = meta + (size_t)mi * meta_bytes;
+        const size_t g0 = (size_t)nt * (kMxBN / 8);
+        mbar_arrive_expect_tx(&meta_full[mi], e < 0 ? 0u : (uint32_t)(groups * (a.s_stride + a.z_stride)));
         if (e >= 0) {
-          if (lane < 2) {
-            const int kt = kb * 2 + lane;
-            bulk_load(st + MoeStage::kOffI + lane * (kMxBN * 24),
-                      img + a.off_i + ((size_t)kt * a.N + nt * kMxBN) * 24, (uint32_t)(rows * 24), &full_bar[s]);
-          }
-          const int g = lane & 15;
-          if (g < groups) {
-            const size_t row = (size_t)(nt * (kMxBN / 8) + g);
-            if (lane < 16)
-              bulk_load(st + MoeStage::kOffC + g * 16, img + a.off_c + row * a.s_stride + (size_t)kb * 16, 16u,
+          bulk_load(mt, img + a.off_c + g0 * a.s_stride, (uint32_t)(groups * a.s_stride), &meta_full[mi]);
+          bulk_load(mt + meta_e, img + a.off_e + g0 * a.z_stride, (uint32_t)(groups * a.z_stride), &meta_full[mi]);
+        }
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kMoeStages;
+          if (it >= kMoeStages && !mbar_wait(&empty_bar[s], ((it / kMoeStages) & 1) ^ 1)) { ok = false; break; }
+          uint8_t* st = ring + (size_t)s * MoeStage::kBytes;
+          mbar_arrive_expect_tx(&full_bar[s], e < 0 ? 0u : (uint32_t)(2 * rows * 24));
+          if (e >= 0)
+            for (int h = 0; h < 2; ++h)
+              bulk_load(st + MoeStage::kOffI + h * (kMxBN * 24),
+                        img + a.off_i + ((size_t)(kb * 2 + h) * a.N + nt * kMxBN) * 24, (uint32_t)(rows * 24),
                         &full_bar[s]);
-            else
-              bulk_load(st + MoeStage::kOffE + g * 16, img + a.off_e + row * a.z_stride + (size_t)(kb * 2 / 16) * 16,
-                        16u, &full_bar[s]);
-          }
         }
       }
+      // every copy this CTA issued lands before it may exit
+      for (int v = max(0, it - kMoeStages); v < it; ++v)
+        if (!mbar_wait(&full_bar[v % kMoeStages], (v / kMoeStages) & 1)) break;
+      for (int v = max(0, t_iter - 2); v < t_iter; ++v)
+        if (!mbar_wait(&meta_full[v & 1], (v >> 1) & 1)) break;
     }
-    // every copy this CTA issued lands before it may exit
-    if (lane == 0)
-      for (int v = max(0, it - kMxStages); v < it; ++v)
-        if (!mbar_wait(&full_bar[v % kMxStages], (v / kMxStages) & 1)) break;
   } else if (warp == 1) {
     // ------------------------------------------------------------------ scale copies + MMA issuer
     if (lane == 0) {
@@ -153,8 +172,8 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
         if (t_iter >= 1 && !mbar_wait(&d_empty, (t_iter - 1) & 1)) break;
         tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % kMxStages, b = it % kMxABufs;
-          if (!mbar_wait(&full_bar[s], (it / kMxStages) & 1)) { ok = false; break; }
+          const int s = it % kMoeStages, b = it % kMxABufs;
+          if (!mbar_wait(&full_bar[s], (it / kMoeStages) & 1)) { ok = false; break; }
           if (!mbar_wait(&a_full[b], (it / kMxABufs) & 1)) { ok = false; break; }
           fence_proxy_async();  // the gathered rows (cp.async writes), to the tensor core's proxy
           tc_fence_after();
@@ -176,22 +195,29 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
         if (ok) umma_commit(&d_full);
       }
     }
-  } else if (warp < 2 + kMxConvWarps) {
+  } else if (warp < kMoeWarpEp) {
     // ------------------------------------------------------------------ converters
-    const int r = (warp - 2) * 32 + lane;  // channel within the tile / token row of the block
-    int it = 0;
+    const int cw = warp - 2;
+    const int r = (cw & 3) * 32 + lane;  // channel within the tile / token row of the block
+    const int h = cw >> 2;               // this warp's LUT3 tile of each k-block
+    int it = 0, t_iter = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++t_iter) {
       const int nt = tile / nblk, mb = tile - nt * nblk;
       const bool row_ok = nt * kMxBN + r < a.N && expert_of(mb) >= 0;
+      const int mi = t_iter & 1;
+      if (ok && !mbar_wait(&meta_full[mi], (t_iter >> 1) & 1)) ok = false;
+      const uint8_t* mt = meta + (size_t)mi * meta_bytes;
       for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int s = it % kMxStages, b = it % kMxABufs;
-        if (ok && !mbar_wait(&full_bar[s], (it / kMxStages) & 1)) ok = false;
+        const int s = it % kMoeStages, b = it % kMxABufs;
+        if (ok && !mbar_wait(&full_bar[s], (it / kMoeStages) & 1)) ok = false;
         if (ok && it >= kMxABufs && !mbar_wait(&a_empty[b], ((it / kMxABufs) & 1) ^ 1)) ok = false;
         tc_fence_after();
         const uint8_t* st = ring + (size_t)s * MoeStage::kBytes;
         uint8_t* ab = abuf + (size_t)b * kMxABufBytes;
-        if (ok) mx_convert_block<kMoeBM>(st, ab, r, kb, row_ok);
+        if (ok)
+          mx_convert_block<kMoeBM>(st, ab, r, kb, row_ok, mt + (r >> 3) * a.s_stride + kb * 16,
+                                   mt + meta_e + (r >> 3) * a.z_stride + kb * 2, h, h + 1, h == 0);
         fence_proxy_async();  // the operand and scale writes, to the tensor core's proxy
         __syncwarp();
         if (lane == 0 && ok) {
@@ -199,13 +225,15 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
           mbar_arrive(&empty_bar[s]);
         }
       }
+      __syncwarp();
+      if (lane == 0 && ok) mbar_arrive(&meta_empty[mi]);
     }
-  } else if (warp < 2 + kMxConvWarps + kMxEpWarps) {
+  } else if (warp < kMoeWarpGather) {
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int r = 32 * q + lane;  // channel within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-    const int ew = warp - (2 + kMxConvWarps);  // 0..3: rows 8 ew .. 8 ew + 7 of each 32-row chunk
+    const int ew = warp - kMoeWarpEp;  // 0..3: rows 8 ew .. 8 ew + 7 of each 32-row chunk
     // every epilogue warp runs every chunk and its named barrier, also after a
     // timed-out wait (then it loads and stores nothing)
     int t_iter = 0, ob = 0;
@@ -217,6 +245,11 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
       tc_fence_after();
 #pragma unroll 1
       for (int j = 0; j < kMoeBM / 32; ++j) {
+        // the pair ids of this warp's rows of the chunk, requested before the accumulator is read
+        int sid[4];
+#pragma unroll
+        for (int pass = 0; pass < 4; ++pass)
+          sid[pass] = __ldg(a.sorted_ids + (size_t)mb * kMoeBM + j * 32 + 8 * ew + 2 * pass + (lane >> 4));
         uint32_t v[32];
         if (ok) {
           tmem_ld32(lane_base + kMoeColD + (uint32_t)(j * 32), v);
@@ -241,10 +274,10 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
 #pragma unroll
         for (int pass = 0; pass < 4; ++pass) {
           const int i = 8 * ew + 2 * pass + (lane >> 4), cl = lane & 15;
-          const int sid = __ldg(a.sorted_ids + (size_t)mb * kMoeBM + j * 32 + i);
-          if (ok && sid >= 0 && sid < a.P && cl * 8 < rows) {
+          if (ok && sid[pass] >= 0 && sid[pass] < a.P && cl * 8 < rows) {
             const uint4 val = *reinterpret_cast<const uint4*>(ot + i * (kMxBN * 2) + cl * 16);
-            *reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.Y) + ((size_t)sid * a.N + nt * kMxBN) * 2 + cl * 16) = val;
+            *reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.Y) + ((size_t)sid[pass] * a.N + nt * kMxBN) * 2 +
+                                      cl * 16) = val;
           }
         }
         ob ^= 1;
@@ -252,7 +285,7 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
     }
   } else {
     // ------------------------------------------------------------------ token-row gather
-    const int g = tid - (2 + kMxConvWarps + kMxEpWarps) * 32;  // row of the block
+    const int g = tid - kMoeWarpGather * 32;  // row of the block
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
@@ -265,8 +298,8 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
       const uint8_t* ssrc = a.scales + (size_t)token * (a.K / 32);
       const int nb = valid ? 16 : 0;
       for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int s = it % kMxStages;
-        if (lane == 0 && it >= kMxStages && !mbar_wait(&empty_bar[s], ((it / kMxStages) & 1) ^ 1)) ok = false;
+        const int s = it % kMoeStages;
+        if (lane == 0 && it >= kMoeStages && !mbar_wait(&empty_bar[s], ((it / kMoeStages) & 1) ^ 1)) ok = false;
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         if (!ok) break;
         const uint32_t st = smem_u32(ring + (size_t)s * MoeStage::kBytes);

@@ -121,25 +121,29 @@ __device__ __forceinline__ void umma_mx(uint32_t d_tmem, uint64_t a_desc, uint64
                : "memory");
 }
 
-// Converter work of one k-block for channel r of the tile: the channel's 128
-// E4M3 weights into the swizzled A tile, its tile exponents into the A scale
-// atom (scale 1.0 and zero weights when the channel does not exist, row_ok
-// false), and the k-block's scale bytes of tokens r + 128 hh into the B scale
-// atoms. st is the stage (layout MxStage<BM>), ab the A buffer.
+// Converter work of one k-block for channel r of the tile, LUT3 tiles
+// h = hb .. he - 1 of the block (64 k each): the channel's E4M3 weights into
+// the swizzled A tile and its tile exponents into the A scale atom (scale 1.0
+// and zero weights when the channel does not exist, row_ok false); with
+// copy_scales, also the k-block's scale bytes of tokens r + 128 hh into the B
+// scale atoms. cbp points at the channel group's 16 codebook bytes of the
+// block (tile h at cbp + 8 h), ep at its exponent byte of the block's first
+// tile (tile h at ep[h]); st is the stage (layout MxStage<BM>), ab the A buffer.
 template <int BM>
-__device__ __forceinline__ void mx_convert_block(const uint8_t* st, uint8_t* ab, int r, int kb, bool row_ok) {
+__device__ __forceinline__ void mx_convert_block(const uint8_t* st, uint8_t* ab, int r, int kb, bool row_ok,
+                                                 const uint8_t* cbp, const uint8_t* ep, int hb, int he,
+                                                 bool copy_scales) {
   using L = MxStage<BM>;
-  // weights: 2 tiles x 2 chunks x 4 groups of 8 k -> E4M3 bytes, 16 per swizzled chunk
   const uint32_t arow = smem_u32(ab + kMxOffA) + (uint32_t)r * 128u;
-  uint32_t eword = 0x7F7F7F7Fu;  // scale 1.0 for channels past N
-  if (row_ok) {
-    uint32_t e2 = 0;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
+  const uint32_t atom_off = (uint32_t)(16 * (r & 31) + 4 * (r >> 5));
+  for (int h = hb; h < he; ++h) {
+    uint32_t eh = 0x7F7Fu;  // scale 1.0 for channels past N
+    if (row_ok) {
+      // weights: 2 chunks x 4 groups of 8 k -> E4M3 bytes, 16 per swizzled chunk
       const uint32_t* w = reinterpret_cast<const uint32_t*>(st + L::kOffI + h * (kMxBN * 24) + r * 24);
-      const uint2 cb = *reinterpret_cast<const uint2*>(st + L::kOffC + (r >> 3) * 16 + h * 8);
-      const uint32_t e = st[L::kOffE + (r >> 3) * 16 + ((kb * 2 + h) & 15)];
-      e2 |= (e | (e << 8)) << (16 * h);
+      const uint2 cb = *reinterpret_cast<const uint2*>(cbp + h * 8);
+      const uint32_t e = ep[h];
+      eh = e | (e << 8);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const uint32_t wa = w[3 * c], wb = w[3 * c + 1], wc = w[3 * c + 2];
@@ -159,20 +163,21 @@ __device__ __forceinline__ void mx_convert_block(const uint8_t* st, uint8_t* ab,
                           "r"(o[3]) : "memory");
         }
       }
+    } else {
+#pragma unroll
+      for (uint32_t cc = 0; cc < 4; ++cc)
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" :: "r"(arow + ((4u * h + cc) << 4)), "r"(0u) : "memory");
     }
-    eword = e2;
-  } else {
-#pragma unroll
-    for (uint32_t chunk = 0; chunk < 8; ++chunk)
-      asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" :: "r"(arow + (chunk << 4)), "r"(0u) : "memory");
+    // the two k-steps of tile h take bytes 2h, 2h + 1 of the channel's scale word
+    *reinterpret_cast<uint16_t*>(ab + kMxOffSA + atom_off + 2 * h) = (uint16_t)eh;
   }
-  const uint32_t atom_off = (uint32_t)(16 * (r & 31) + 4 * (r >> 5));
-  *reinterpret_cast<uint32_t*>(ab + kMxOffSA + atom_off) = eword;
-  // token scales of this block: bytes 4 (kb % 4) .. +3 of each token's 16-byte row
+  if (copy_scales) {
+    // token scales of this block: bytes 4 (kb % 4) .. +3 of each token's 16-byte row
 #pragma unroll
-  for (int hh = 0; hh < BM / 128; ++hh) {
-    const uint32_t sw = *reinterpret_cast<const uint32_t*>(st + L::kOffS + (hh * 128 + r) * 16 + (kb & 3) * 4);
-    *reinterpret_cast<uint32_t*>(ab + kMxOffSB + hh * 512 + atom_off) = sw;
+    for (int hh = 0; hh < BM / 128; ++hh) {
+      const uint32_t sw = *reinterpret_cast<const uint32_t*>(st + L::kOffS + (hh * 128 + r) * 16 + (kb & 3) * 4);
+      *reinterpret_cast<uint32_t*>(ab + kMxOffSB + hh * 512 + atom_off) = sw;
+    }
   }
 }
 
@@ -296,7 +301,9 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         tc_fence_after();
         const uint8_t* st = ring + (size_t)s * kMxStageBytes;
         uint8_t* ab = abuf + (size_t)b * kMxABufBytes;
-        if (ok) mx_convert_block<kMxBM>(st, ab, r, kb, row_ok);
+        if (ok)
+          mx_convert_block<kMxBM>(st, ab, r, kb, row_ok, st + kMxOffC + (r >> 3) * 16,
+                                  st + kMxOffE + (r >> 3) * 16 + ((kb * 2) & 15), 0, 2, true);
         fence_proxy_async();  // the operand and scale writes, to the tensor core's proxy
         __syncwarp();
         if (lane == 0 && ok) {

@@ -1791,7 +1791,8 @@ lbq_status lbq_moe_lut3_mx_gemm(const uint8_t* codes, const uint8_t* scales, int
                                 void* Y, int y_dtype, void* stream) {
   lbq_status st = check_lut3_shape(K, N);
   if (st != LBQ_OK) return st;
-  if (K % 128) return fail(LBQ_ERR_UNSUPPORTED, "lbq_moe_lut3_mx_gemm needs K %% 128 == 0 (K=%d)", K);
+  if (K % 128 || K > kMoeMaxK)
+    return fail(LBQ_ERR_UNSUPPORTED, "lbq_moe_lut3_mx_gemm needs K %% 128 == 0 and K <= %d (K=%d)", kMoeMaxK, K);
   if (T <= 0 || top_k <= 0 || num_local_experts <= 0)
     return fail(LBQ_ERR_INVALID_ARG, "T=%d top_k=%d num_local_experts=%d must be positive", T, top_k, num_local_experts);
   if ((long long)T * top_k >= (1LL << 30)) return fail(LBQ_ERR_INVALID_ARG, "T * top_k too large");
@@ -1821,11 +1822,12 @@ lbq_status lbq_moe_lut3_mx_gemm(const uint8_t* codes, const uint8_t* scales, int
   a.k_blocks = K / kMxBK;
   a.num_experts = num_local_experts;
   a.y_bf16 = y_dtype == LBQ_DTYPE_BF16 ? 1 : 0;
+  const int smem = kMoeSmemBase + 2 * moe_meta_bytes(a.s_stride, a.z_stride);
   const void* fn = (const void*)gemm_moe_lut3_mx_kernel;
-  occupancy_for(fn, kMoeThreads, kMoeSmem);
+  occupancy_for(fn, kMoeThreads, smem);
   const int grid = (int)std::min<long long>((long long)a.n_tiles * a.max_blocks, num_sms());
   void* args[] = {&a};
-  return launch_kernel_ex(fn, dim3(grid), dim3(kMoeThreads), kMoeSmem, static_cast<cudaStream_t>(stream), false, args,
+  return launch_kernel_ex(fn, dim3(grid), dim3(kMoeThreads), smem, static_cast<cudaStream_t>(stream), false, args,
                           "MoE LUT3 x MXFP8 GEMM launch");
 }
 

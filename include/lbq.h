@@ -479,7 +479,7 @@ lbq_status lbq_moe_align(const int32_t* topk_ids, int num_pairs, int num_experts
  *   sorted_ids, expert_ids, total (device) from lbq_moe_align(block = 128)
  *   images  (device) local expert e's lbq_pack_lut3 image (K, N) at images + e * image_stride
  *   Y       (device) [T * top_k, N] row-major, y_dtype
- * K % 128 == 0, N % 8 == 0; max_padded the value the lists were sized with
+ * K % 128 == 0, K <= 8192, N % 8 == 0; max_padded the value the lists were sized with
  * (a multiple of 128); pointers and image_stride 16-byte aligned. Errors
  * before any launch: LBQ_ERR_INVALID_ARG / LBQ_ERR_UNSUPPORTED. Asynchronous
  * on `stream`.
