@@ -34,7 +34,10 @@
 namespace lbq {
 
 constexpr int kMoeBM = 128;  // tokens (sorted rows) per tile = the alignment block
-constexpr int kMoeStages = 3;  // ring depth (k-blocks of indices and gathered rows in flight)
+// Ring depth and converted weight tiles in flight. Measured at the write-up's
+// layer shape: 5 stages with 2 tiles, or 4 with 3, change the time by 5% at most.
+constexpr int kMoeStages = 3;
+constexpr int kMoeABufs = 4;
 constexpr int kMoeConvWarps = 8, kMoeGatherWarps = 4;
 constexpr int kMoeWarpEp = 2 + kMoeConvWarps;             // first epilogue warp
 constexpr int kMoeWarpGather = kMoeWarpEp + kMxEpWarps;   // first gather warp
@@ -43,7 +46,7 @@ constexpr int kMoeMaxK = 8192;
 using MoeStage = MxStage<kMoeBM>;
 // fixed part of the dynamic shared memory; two per-tile codebook / exponent
 // areas of moe_meta_bytes(K) follow
-constexpr int kMoeSmemBase = kMoeStages * MoeStage::kBytes + kMxABufs * kMxABufBytes + 2 * kMxOutBytes + 1024;
+constexpr int kMoeSmemBase = kMoeStages * MoeStage::kBytes + kMoeABufs * kMxABufBytes + 2 * kMxOutBytes + 1024;
 constexpr uint32_t kMoeColD = 0, kMoeColSF = 128;  // TMEM columns: accumulator, then 16 per A buffer
 constexpr uint32_t kMoeTmemCols = 256;
 __host__ __device__ constexpr int moe_meta_bytes(int s_stride, int z_stride) { return 16 * (s_stride + z_stride); }
@@ -77,12 +80,12 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
 __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const GemmMoeArgs a) {
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t full_bar[kMoeStages], empty_bar[kMoeStages];
-  __shared__ __align__(8) uint64_t a_full[kMxABufs], a_empty[kMxABufs], d_full, d_empty;
+  __shared__ __align__(8) uint64_t a_full[kMoeABufs], a_empty[kMoeABufs], d_full, d_empty;
   __shared__ __align__(8) uint64_t meta_full[2], meta_empty[2];
   __shared__ uint32_t tmem_base_sh;
   uint8_t* ring = dsmem + ((1024u - (smem_u32(dsmem) & 1023u)) & 1023u);
   uint8_t* abuf = ring + (size_t)kMoeStages * MoeStage::kBytes;
-  uint8_t* obuf = abuf + (size_t)kMxABufs * kMxABufBytes;  // two output tiles
+  uint8_t* obuf = abuf + (size_t)kMoeABufs * kMxABufBytes;  // two output tiles
   uint8_t* meta = obuf + 2 * kMxOutBytes;                   // two per-tile areas: codebook rows, exponent rows
   const int meta_bytes = moe_meta_bytes(a.s_stride, a.z_stride);
   const int meta_e = 16 * a.s_stride;                        // exponent rows inside an area
@@ -102,7 +105,7 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
       mbar_init(&full_bar[i], 1 + kMoeGatherWarps * 32);
       mbar_init(&empty_bar[i], 1 + kMoeConvWarps);
     }
-    for (int i = 0; i < kMxABufs; ++i) {
+    for (int i = 0; i < kMoeABufs; ++i) {
       mbar_init(&a_full[i], kMoeConvWarps);
       mbar_init(&a_empty[i], 1);
     }
@@ -172,9 +175,9 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
         if (t_iter >= 1 && !mbar_wait(&d_empty, (t_iter - 1) & 1)) break;
         tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % kMoeStages, b = it % kMxABufs;
+          const int s = it % kMoeStages, b = it % kMoeABufs;
           if (!mbar_wait(&full_bar[s], (it / kMoeStages) & 1)) { ok = false; break; }
-          if (!mbar_wait(&a_full[b], (it / kMxABufs) & 1)) { ok = false; break; }
+          if (!mbar_wait(&a_full[b], (it / kMoeABufs) & 1)) { ok = false; break; }
           fence_proxy_async();  // the gathered rows (cp.async writes), to the tensor core's proxy
           tc_fence_after();
           const uint32_t ab = smem_u32(abuf + (size_t)b * kMxABufBytes);
@@ -209,9 +212,9 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
       if (ok && !mbar_wait(&meta_full[mi], (t_iter >> 1) & 1)) ok = false;
       const uint8_t* mt = meta + (size_t)mi * meta_bytes;
       for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int s = it % kMoeStages, b = it % kMxABufs;
+        const int s = it % kMoeStages, b = it % kMoeABufs;
         if (ok && !mbar_wait(&full_bar[s], (it / kMoeStages) & 1)) ok = false;
-        if (ok && it >= kMxABufs && !mbar_wait(&a_empty[b], ((it / kMxABufs) & 1) ^ 1)) ok = false;
+        if (ok && it >= kMoeABufs && !mbar_wait(&a_empty[b], ((it / kMoeABufs) & 1) ^ 1)) ok = false;
         tc_fence_after();
         const uint8_t* st = ring + (size_t)s * MoeStage::kBytes;
         uint8_t* ab = abuf + (size_t)b * kMxABufBytes;
