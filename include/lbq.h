@@ -113,7 +113,12 @@ lbq_status lbq_pack(const float* W, int K, int N, int group, int mode,
  * Weight value = e4m3(codebooks[k/64][n/8][idx[k][n]]) * 2^(exponents[k/64][n/8] - 127).
  * Indices > 7 are taken modulo 8; NaN codebook bytes (0x7F/0xFF) and NaN
  * exponents (0xFF) are the caller's responsibility (they decode to NaN).
- * Asynchronous on `stream`.
+ * The BF16-activation kernels (lbq_lut3_gemm) decode through a per-tile BF16
+ * table that holds every weight exactly for 3 <= exponent <= 246 (E4M3
+ * magnitudes 2^-9 .. 448 times 2^(E-127) inside BF16's 2^-133 .. 2^128);
+ * outside that range its entries are the weights rounded to BF16 (down to 0,
+ * up to infinity at the extremes). The MXFP8 kernels read the format's own
+ * bytes and are exact for every exponent. Asynchronous on `stream`.
  */
 lbq_status lbq_pack_lut3(const uint8_t* idx, const uint8_t* codebooks, const uint8_t* exponents,
                          int K, int N, void* image, size_t image_bytes, void* stream);

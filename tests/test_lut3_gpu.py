@@ -213,3 +213,23 @@ def test_lut3_m1_variants(torch, lbq, K, N, variant):
     finally:
         lbq.lbq_debug_lut3_variant(-1)
     lbq.device_status()
+
+
+def test_tables_exact_at_the_exponent_range_ends(torch, lbq):
+    """The BF16 decode tables hold every weight e4m3(b) * 2^(E-127) exactly for
+    3 <= E <= 246 (E4M3 magnitudes run from 2^-9 to 448; BF16 from 2^-133 to
+    just under 2^128): tiles at E = 3, 4, 245 and 246 with the E4M3 extremes
+    in their codebooks decode bit-exactly, and the dequantised image equals the
+    oracle's exact decode."""
+    K, N = 256, 32
+    idx, cb, ex = workloads.lut3_host(701, K, N)
+    extremes = [0x7E, 0xFE, 0x01, 0x81, 0x00, 0x80, 0x08, 0xF8]  # +-448, +-2^-9, +-0, +-2^-6, -240
+    for kt, e in enumerate((3, 4, 245, 246)):
+        cb[kt, :] = extremes
+        ex[kt, :] = e
+        idx[64 * kt:64 * kt + 64, :] = np.arange(64)[:, None] % 8
+    img = _image(torch, lbq, idx, cb, ex)
+    _check_tables(torch, img, K, N, cb, ex)
+    W = lbq.dequant(img, K, N, 0, "lut3").cpu().numpy()
+    assert np.array_equal(W.astype(np.float64), lut3.dequant(idx, cb, ex))
+    lbq.device_status()

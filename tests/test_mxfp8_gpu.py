@@ -36,6 +36,16 @@ def _planted(torch, X):
     X[0, 192] = 1.0
     X[0, 193] = 1.0 / 256 * 1.03125                      # small elements next to a large one
     X[0, 194] = -(1.0 / 256) * 1.0625
+    if X.dtype == torch.bfloat16 and X.shape[1] >= 320:
+        # scale byte clamped to 0: amax 2^-125 asks for 2^(-125 - 8), below 2^-127
+        X[0, 224:256] = 0.0
+        X[0, 224] = 2.0 ** -125
+        X[0, 225] = -(2.0 ** -127) * 1.5
+        X[0, 226] = 2.0 ** -131                          # a BF16 subnormal in the same block
+        # the block's largest element is itself a BF16 subnormal
+        X[0, 288:320] = 0.0
+        X[0, 288] = -(2.0 ** -130) * 1.5
+        X[0, 289] = 2.0 ** -133
     return X
 
 
@@ -43,9 +53,11 @@ def _planted(torch, X):
 @pytest.mark.parametrize("M,K", [(1, 4096), (3, 96), (17, 1024)])
 def test_quantize_mxfp8_bit_exact(torch, lbq, xdt, M, K):
     X = workloads.activations_host(40 + M + K, M, K, xdt)
-    X = X * (torch.arange(M, dtype=torch.float32)[:, None] * 7 - 9).exp2().to(X.dtype)  # row magnitudes 2^-9 .. 2^103
-    if xdt == "f16":
-        X = workloads.activations_host(40 + M + K, M, K, xdt)
+    if xdt == "bf16":
+        X = X * (torch.arange(M, dtype=torch.float32)[:, None] * 7 - 9).exp2().to(X.dtype)  # rows 2^-9 .. 2^103
+    else:
+        # FP16 rows 2^-14 .. 2^4 (the small rows are largely FP16 subnormals)
+        X = (X.float() * (torch.arange(M, dtype=torch.float32)[:, None] % 4 * 6 - 14).exp2()).to(X.dtype)
     if K >= 256:
         X = _planted(torch, X.clone())
     codes, scales = lbq.quantize_mxfp8(X.cuda())
