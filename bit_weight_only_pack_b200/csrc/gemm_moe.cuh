@@ -47,8 +47,10 @@ using MoeStage = MxStage<kMoeBM>;
 // fixed part of the dynamic shared memory; two per-tile codebook / exponent
 // areas of moe_meta_bytes(K) follow
 constexpr int kMoeSmemBase = kMoeStages * MoeStage::kBytes + kMoeABufs * kMxABufBytes + 2 * kMxOutBytes + 1024;
-constexpr uint32_t kMoeColD = 0, kMoeColSF = 128;  // TMEM columns: accumulator, then 16 per A buffer
-constexpr uint32_t kMoeTmemCols = 256;
+// TMEM columns: two accumulators (the MMAs fill one while the epilogue drains
+// the other), then 16 per A buffer of scale atoms
+constexpr uint32_t kMoeColD = 0, kMoeColSF = 256;
+constexpr uint32_t kMoeTmemCols = 512;
 __host__ __device__ constexpr int moe_meta_bytes(int s_stride, int z_stride) { return 16 * (s_stride + z_stride); }
 static_assert(kMoeSmemBase + 2 * moe_meta_bytes(kMoeMaxK / 8, kMoeMaxK / 64) <= 227 * 1024, "MoE GEMM shared memory");
 
@@ -80,7 +82,7 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
 __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const GemmMoeArgs a) {
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t full_bar[kMoeStages], empty_bar[kMoeStages];
-  __shared__ __align__(8) uint64_t a_full[kMoeABufs], a_empty[kMoeABufs], d_full, d_empty;
+  __shared__ __align__(8) uint64_t a_full[kMoeABufs], a_empty[kMoeABufs], d_full[2], d_empty[2];
   __shared__ __align__(8) uint64_t meta_full[2], meta_empty[2];
   __shared__ uint32_t tmem_base_sh;
   uint8_t* ring = dsmem + ((1024u - (smem_u32(dsmem) & 1023u)) & 1023u);
@@ -113,8 +115,10 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
       mbar_init(&meta_full[i], 1);
       mbar_init(&meta_empty[i], kMoeConvWarps);
     }
-    mbar_init(&d_full, 1);
-    mbar_init(&d_empty, kMxEpWarps);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&d_full[i], 1);
+      mbar_init(&d_empty[i], kMxEpWarps);
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -172,7 +176,8 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
       int it = 0, t_iter = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t_iter) {
-        if (t_iter >= 1 && !mbar_wait(&d_empty, (t_iter - 1) & 1)) break;
+        const int ai = t_iter & 1;  // accumulator of this tile
+        if (t_iter >= 2 && !mbar_wait(&d_empty[ai], ((t_iter >> 1) & 1) ^ 1)) break;
         tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % kMoeStages, b = it % kMoeABufs;
@@ -189,13 +194,13 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
           for (uint32_t kk = 0; kk < 4; ++kk) {
             const uint64_t da = umma_desc_sw128(ab + kMxOffA) + (uint64_t)(kk * 2);
             const uint64_t db = umma_desc_sw128(xb) + (uint64_t)(kk * 2);
-            umma_mx(tmem + kMoeColD, da, db, umma_idesc_mx(kk, kMoeBM), sf | (kk << 30), (sf + 4) | (kk << 30),
-                    (kb > 0 || kk > 0) ? 1u : 0u);
+            umma_mx(tmem + kMoeColD + (uint32_t)ai * kMoeBM, da, db, umma_idesc_mx(kk, kMoeBM), sf | (kk << 30),
+                    (sf + 4) | (kk << 30), (kb > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&empty_bar[s]);
           umma_commit(&a_empty[b]);
         }
-        if (ok) umma_commit(&d_full);
+        if (ok) umma_commit(&d_full[ai]);
       }
     }
   } else if (warp < kMoeWarpEp) {
@@ -244,7 +249,8 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++t_iter) {
       const int nt = tile / nblk, mb = tile - nt * nblk;
       const int rows = min(kMxBN, a.N - nt * kMxBN);
-      if (ok && !mbar_wait(&d_full, t_iter & 1)) ok = false;
+      const int ai = t_iter & 1;
+      if (ok && !mbar_wait(&d_full[ai], (t_iter >> 1) & 1)) ok = false;
       tc_fence_after();
 #pragma unroll 1
       for (int j = 0; j < kMoeBM / 32; ++j) {
@@ -255,7 +261,7 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
           sid[pass] = __ldg(a.sorted_ids + (size_t)mb * kMoeBM + j * 32 + 8 * ew + 2 * pass + (lane >> 4));
         uint32_t v[32];
         if (ok) {
-          tmem_ld32(lane_base + kMoeColD + (uint32_t)(j * 32), v);
+          tmem_ld32(lane_base + kMoeColD + (uint32_t)ai * kMoeBM + (uint32_t)(j * 32), v);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = 0u;
@@ -263,7 +269,7 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
         if (j == kMoeBM / 32 - 1) {  // the accumulator is in registers: the MMAs may start the next tile
           tc_fence_before();
           __syncwarp();
-          if (lane == 0 && ok) mbar_arrive(&d_empty);
+          if (lane == 0 && ok) mbar_arrive(&d_empty[ai]);
         }
         uint8_t* ot = obuf + (size_t)ob * kMxOutBytes;  // [32 rows][128 channels]
 #pragma unroll
