@@ -1597,6 +1597,18 @@ lbq_status lbq_affine_gemv(const void* X, int x_dtype, int M, int K, int N, int 
   if ((st = check_compute_args(X, x_dtype, M, image, Y, y_dtype)) != LBQ_OK) return st;
   if (M > 16) return fail(LBQ_ERR_UNSUPPORTED, "lbq_affine_gemv takes 1 <= M <= 16 (M=%d)", M);
   const Layout L = make_layout(K, N, group, LBQ_MODE_AFFINE, bits);
+  // 4-bit codes: the image's chunks, scales and zero points are byte for byte
+  // the asymmetric INT4 image (pair-split nibbles = the INT4 slot order, same
+  // region offsets), so batch 1 runs on the INT4 GEMVs (none of them needs a
+  // workspace at batch 1 when the TMA-fed kernel takes the whole K range)
+  if (bits == 4 && M == 1 && K <= 32 * 32 * kGdMaxWarps) {
+    const lbq_gemv_item item{X, image, Y, N};
+    const bool xbf16 = x_dtype == LBQ_DTYPE_BF16, ybf16 = y_dtype == LBQ_DTYPE_BF16;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (tmma_ok(1, K, &N, 1) && tmma_preferred(K, &N, 1) && plan_tmma(K, &N, 1, group, true, false).nsl > 0)
+      return run_tmma(&item, 1, K, group, LBQ_MODE_ASYM, xbf16, ybf16, nullptr, 0, s, false);
+    return run_direct(&item, 1, K, group, LBQ_MODE_ASYM, xbf16, ybf16, s);
+  }
   return run_affine_gemv(static_cast<const uint16_t*>(X), x_dtype == LBQ_DTYPE_BF16, M,
                          static_cast<const uint8_t*>(image), L, Y, y_dtype == LBQ_DTYPE_BF16,
                          static_cast<cudaStream_t>(stream));
