@@ -137,7 +137,9 @@ __global__ void __launch_bounds__(256) unpack_affine_kernel(
 //    4 b bytes allow), one vector load of the R scales and one of the R zero
 //    points; consecutive lanes read consecutive chunks of a row, so a warp
 //    instruction covers 128 b contiguous bytes. Latency is hidden by the
-//    other warps resident on the SM (no staging, no handshakes).
+//    other warps resident on the SM (no staging, no handshakes); the first
+//    row block is requested before the kernel waits for its predecessor in
+//    the stream (programmatic dependent launch).
 //  * Per pair of k one shift + one AND/OR (four operations when the pair's
 //    field crosses a 16-bit boundary) give 2^F + q for both k, and two
 //    mixed-precision FMAs accumulate x (2^F + q) in FP32 for each batch row.
@@ -222,33 +224,11 @@ __global__ void __launch_bounds__(kAgMaxWarps * 32) affine_gemv_kernel(const Aff
   const size_t rowb = (size_t)chunks * 4 * B;
   const int gi = c >> a.gshift;
 
-  uint32_t x[MB][16];
-  float xs[MB];
-#pragma unroll
-  for (int m = 0; m < MB; ++m) {
-    xs[m] = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) x[m][i] = 0u;
-    if (cok && m < a.m_valid) {
-      const uint4* xp = reinterpret_cast<const uint4*>(a.X + (size_t)m * a.K + (size_t)c * 32);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 v = __ldg(xp + i);
-        x[m][4 * i] = v.x; x[m][4 * i + 1] = v.y; x[m][4 * i + 2] = v.z; x[m][4 * i + 3] = v.w;
-      }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        xs[m] += x2f<BF16>((uint16_t)(x[m][i] & 0xFFFFu));
-        xs[m] += x2f<BF16>((uint16_t)(x[m][i] >> 16));
-      }
-    }
-  }
-
-  int buf = 0;
-  for (int rb = blockIdx.x; rb < a.row_blocks; rb += gridDim.x) {
+  // codes, scales and zero points of row block rb
+  uint32_t w[R][B];
+  float s[R], zf[R];
+  auto load_rows = [&](int rb) {
     const int n0 = rb * R;
-    uint32_t w[R][B];
-    float s[R], zf[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
 #pragma unroll
@@ -296,6 +276,39 @@ __global__ void __launch_bounds__(kAgMaxWarps * 32) affine_gemv_kernel(const Aff
         zf[r] = (float)zb[r];
       }
     }
+  };
+  // the weights are only read: the first row block is requested before waiting
+  // for the previous kernel in the stream (which may write X)
+  if ((int)blockIdx.x < a.row_blocks) load_rows(blockIdx.x);
+  griddep_launch_dependents();
+  griddep_wait();
+
+  uint32_t x[MB][16];
+  float xs[MB];
+#pragma unroll
+  for (int m = 0; m < MB; ++m) {
+    xs[m] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[m][i] = 0u;
+    if (cok && m < a.m_valid) {
+      const uint4* xp = reinterpret_cast<const uint4*>(a.X + (size_t)m * a.K + (size_t)c * 32);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 v = __ldg(xp + i);
+        x[m][4 * i] = v.x; x[m][4 * i + 1] = v.y; x[m][4 * i + 2] = v.z; x[m][4 * i + 3] = v.w;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        xs[m] += x2f<BF16>((uint16_t)(x[m][i] & 0xFFFFu));
+        xs[m] += x2f<BF16>((uint16_t)(x[m][i] >> 16));
+      }
+    }
+  }
+
+  int buf = 0;
+  for (int rb = blockIdx.x; rb < a.row_blocks; rb += gridDim.x) {
+    const int n0 = rb * R;
+    if (rb != (int)blockIdx.x) load_rows(rb);
 
     float part[8];
 #pragma unroll

@@ -1176,7 +1176,7 @@ static lbq_status run_affine_gemv(const uint16_t* X, bool xbf16, int M, const ui
     const int occ = std::max(1, occupancy_for(fn, T, smem));
     const int grid = std::min(a.row_blocks, num_sms() * occ);
     void* args[] = {&a};
-    lbq_status s = launch_kernel_ex(fn, dim3(grid), dim3(T), smem, st, false, args, "affine GEMV launch");
+    lbq_status s = launch_kernel_ex(fn, dim3(grid), dim3(T), smem, st, g_pdl != 0, args, "affine GEMV launch");
     if (s != LBQ_OK) return s;
   }
   return LBQ_OK;
