@@ -14,7 +14,7 @@ thin Python binding.
 from .binding import (  # noqa: F401
     DTYPES, MODES, LbqError, dequant, device_status, gemm, gemv, gemv_grouped, gemv_noalloc, make_gemv_items, lut3_gemm, lut3_mx_gemm, pack, pack_lut3, quantize_mxfp8,
     unpack_canonical, unpack_lut3_canonical, workspace,
-    lbq_debug_force_splits, lbq_debug_force_skinny, lbq_debug_force_tc, lbq_debug_gemv_path, lbq_debug_gemm_path, lbq_debug_direct_variant, lbq_debug_lut3_variant, lbq_debug_tmma_default, lbq_debug_tmma_split, lbq_debug_drop_copies, lbq_dequant, lbq_device_status, lbq_gemm, lbq_gemv, lbq_gemv_grouped, lbq_gemv_noalloc, lbq_last_error,
+    lbq_debug_force_splits, lbq_debug_force_skinny, lbq_debug_force_tc, lbq_debug_gemv_path, lbq_debug_gemm_path, lbq_debug_direct_variant, lbq_debug_tmma_default, lbq_debug_tmma_split, lbq_debug_drop_copies, lbq_dequant, lbq_device_status, lbq_gemm, lbq_gemv, lbq_gemv_grouped, lbq_gemv_noalloc, lbq_last_error,
     lbq_launch_count, lbq_lut3_gemm, lbq_pack, lbq_set_option, LBQ_OPT_PDL, lbq_pack_lut3, lbq_packed_size, lbq_unpack_canonical,
     lbq_unpack_lut3_canonical, lbq_version, lbq_workspace_size, lbq_quantize_mxfp8, lbq_lut3_mx_gemm,
     affine_gemv, pack_affine, unpack_affine_canonical, lbq_affine_gemv, lbq_affine_packed_size, lbq_pack_affine,

@@ -89,7 +89,6 @@ _SIGS = {
     "lbq_debug_gemv_path": ([_c_int], None),
     "lbq_debug_gemm_path": ([_c_int], None),
     "lbq_debug_direct_variant": ([_c_int, _c_int], None),
-    "lbq_debug_lut3_variant": ([_c_int], None),
     "lbq_debug_tmma_default": ([_c_int], None),
     "lbq_debug_tmma_split": ([_c_int], None),
     "lbq_debug_drop_copies": ([_c_int], None),
@@ -319,11 +318,6 @@ def lbq_debug_direct_variant(variant, ctas_per_sm=0):
     """Test hook: batch-1 direct kernel variant (-1 library's choice, 0 registers, 2..4 staged copies,
     1 / 5 tensor cores with exact / offset-form operands) and a CTAs-per-SM cap."""
     _lib.lbq_debug_direct_variant(variant, ctas_per_sm)
-
-
-def lbq_debug_lut3_variant(variant):
-    """Test hook: LUT3 batch-1 kernel (-1 library's choice, 0 registers, 2 / 3 staged copies)."""
-    _lib.lbq_debug_lut3_variant(variant)
 
 
 def lbq_debug_gemm_path(path):

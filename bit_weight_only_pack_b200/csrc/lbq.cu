@@ -28,7 +28,6 @@
 #include "tc_gemv.cuh"
 #include "gemv_direct.cuh"
 #include "gemv_tmma.cuh"
-#include "gemv_dmma.cuh"
 #include "mxfp8.cuh"
 #include "gemm_ts.cuh"
 #include "gemm_mx.cuh"
@@ -452,7 +451,7 @@ static lbq_status run_tcgemv(const void* X, bool xbf16, int M, const void* image
 // mode / dtypes in one launch.
 // test hook: -1 = the library's choice, 0 = weights pipelined through
 // registers, 2..4 = staged through shared memory with that many row blocks in
-// flight (1 and 5 select the tensor-core kernel, see run_dmma)
+// flight
 static int g_direct_stages = -1;
 static int g_direct_ctas = 0;  // test hook: cap on resident CTAs per SM (0 = occupancy limit)
 
@@ -470,80 +469,11 @@ static const void* direct_async_kernel(bool bf16, bool asym, int stages, bool a8
 #undef LBQ_GDA
 }
 
-static int g_dmma = 0;  // test hook: batch-1 GEMVs on the tensor-core direct kernel
-
-static const void* dmma_kernel(bool bf16, bool asym, int stages, bool off) {
-#define LBQ_DM(S, O) (bf16 ? (asym ? (const void*)gemv_dmma_kernel<true, true, S, O> : (const void*)gemv_dmma_kernel<true, false, S, O>) \
-                           : (asym ? (const void*)gemv_dmma_kernel<false, true, S, O> : (const void*)gemv_dmma_kernel<false, false, S, O>))
-  if (off) return stages >= 4 ? LBQ_DM(4, true) : stages == 3 ? LBQ_DM(3, true) : LBQ_DM(2, true);
-  return stages >= 4 ? LBQ_DM(4, false) : stages == 3 ? LBQ_DM(3, false) : LBQ_DM(2, false);
-#undef LBQ_DM
-}
-
-// Batch-1 GEMVs (1..4 with one K, group, mode and dtypes) on the tensor-core
-// direct kernel.
-static lbq_status run_dmma(const lbq_gemv_item* items, int count, int K, int group, int mode, bool xbf16, bool ybf16,
-                           cudaStream_t st) {
-  const bool asym = mode == LBQ_MODE_ASYM;
-  if (count < 1 || count > kDmMaxItems) return fail(LBQ_ERR_INVALID_ARG, "count=%d not in 1..%d", count, kDmMaxItems);
-  const int chunks = K / 32;
-  const int passes = (chunks + 7) / 8;                        // 8-chunk passes along K
-  const int spw = (passes + kDmMaxWarps - 1) / kDmMaxWarps;  // passes per warp
-  const int nw = (passes + spw - 1) / spw;
-  const int T = nw * 32;
-  GemvDmmaArgs a{};
-  int tiles = 0;
-  for (int i = 0; i < count; ++i) {
-    const Layout L = make_layout(K, items[i].N, group, mode);
-    const uint8_t* img = static_cast<const uint8_t*>(items[i].image);
-    a.q[i] = img + L.off0;
-    a.s[i] = img + L.off1;
-    a.z[i] = asym ? img + L.off2 : nullptr;
-    a.Y[i] = items[i].Y;
-    a.N[i] = items[i].N;
-    tiles += (items[i].N + kDmRows - 1) / kDmRows;
-    a.rt_end[i] = tiles;
-    int v = 0;
-    while (v < a.nx && a.X[v] != items[i].X) ++v;
-    if (v == a.nx) a.X[a.nx++] = static_cast<const uint16_t*>(items[i].X);
-    a.xi[i] = v;
-  }
-  a.items = count;
-  a.K = K; a.G = K / group;
-  a.row_tiles = tiles;
-  a.spw = spw;
-  a.gshift = group == 32 ? 0 : group == 64 ? 1 : 2;
-  a.y_bf16 = ybf16 ? 1 : 0;
-  // the deepest ring (2..4 passes) that fits with the row sums of one wave
-  static int optin = 0;
-  if (optin == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  }
-  for (int stages = 4; stages >= 2; --stages) {
-    const void* fn = dmma_kernel(xbf16, asym, stages, g_dmma == 2);
-    const size_t fixed = dmma_smem_fixed(stages, T, a.nx, K);
-    const int occ = std::max(1, occupancy_for(fn, T, (int)fixed + 4096));
-    int grid = std::min(tiles, num_sms() * occ);
-    size_t smem = fixed + (size_t)((tiles + grid - 1) / grid) * nw * kDmRows * sizeof(float);
-    while (smem > (size_t)optin && grid < tiles) {  // tall matrices: more CTAs, fewer tiles each
-      grid = std::min(tiles, grid * 2);
-      smem = fixed + (size_t)((tiles + grid - 1) / grid) * nw * kDmRows * sizeof(float);
-    }
-    if (smem > (size_t)optin) continue;
-    void* args[] = {&a};
-    return launch_kernel_ex(fn, dim3(grid), dim3(T), (int)smem, st, g_pdl != 0, args, "tensor-core GEMV launch");
-  }
-  return fail(LBQ_ERR_UNSUPPORTED, "K=%d with %d distinct activation vectors does not fit shared memory", K, a.nx);
-}
-
 // sx != nullptr selects the W4A8 form: items[i].X are INT8 codes and sx[i]
 // their per-32-k scales.
 static lbq_status run_direct(const lbq_gemv_item* items, int count, int K, int group, int mode, bool xbf16, bool ybf16,
                              cudaStream_t st, const float* const* sx = nullptr) {
   const bool a8 = sx != nullptr;
-  if (g_dmma && !a8) return run_dmma(items, count, K, group, mode, xbf16, ybf16, st);
   const bool asym = mode == LBQ_MODE_ASYM;
   const int chunks = K / 32;
   const int nw = (chunks + 31) / 32;
@@ -1012,7 +942,6 @@ static bool lut3_direct_ok(int M, int K) { return M == 1 && K / 64 <= 32 * kLdMa
 
 // test hook: LUT3 batch-1 kernel (-1 = the library's choice, 0 = indices
 // pipelined through registers, 2 / 3 = staged through shared memory)
-static int g_lut3_stages = -1;
 
 static lbq_status run_lut3_direct(const void* X, const void* image, const Layout& L, void* Y, bool ybf16,
                                   cudaStream_t st) {
@@ -1027,20 +956,14 @@ static lbq_status run_lut3_direct(const void* X, const void* image, const Layout
   a.y_bf16 = ybf16 ? 1 : 0;
   const int nw = (L.K / 64 + 31) / 32;
   const int T = nw * 32;
-  int stages = g_lut3_stages < 0 ? 0 : g_lut3_stages;  // registers: staging measured slower here
-  while (stages >= 2 && (size_t)stages * 13 * T * 16 > 200 * 1024) --stages;
-  if (stages < 2) stages = 0;
-  const int stage_bytes = stages * 13 * T * 16;
-  const void* fn = stages == 0 ? (const void*)lut3_direct_kernel
-                 : stages == 2 ? (const void*)lut3_direct_async_kernel<2> : (const void*)lut3_direct_async_kernel<3>;
-  const int occ = std::max(1, occupancy_for(fn, T, stage_bytes + 1024));
+  const void* fn = (const void*)lut3_direct_kernel;
+  const int occ = std::max(1, occupancy_for(fn, T, 1024));
   int grid = std::min(a.row_blocks, num_sms() * occ);
   int smem = ((a.row_blocks + grid - 1) / grid) * nw * 8 * (int)sizeof(float);
-  while (smem > (stages ? 4096 : 96 * 1024) && grid < a.row_blocks) {
+  while (smem > 96 * 1024 && grid < a.row_blocks) {
     grid = std::min(a.row_blocks, grid * 2);
     smem = ((a.row_blocks + grid - 1) / grid) * nw * 8 * (int)sizeof(float);
   }
-  smem += stage_bytes;
   void* args[] = {&a};
   return launch_kernel_ex(fn, dim3(grid), dim3(T), smem, st, g_pdl != 0, args, "LUT3 direct GEMV launch");
 }
@@ -1347,19 +1270,12 @@ void lbq_debug_tmma_split(int r) { g_tmma_split = (r == 1 || r == 2 || r == 4) ?
 void lbq_debug_drop_copies(int on) { g_debug_drop = on ? 1 : 0; }
 
 // Test hook (not in the public header): direct batch-1 kernel variant
-// (-1 = the library's choice, 0 = weights pipelined through registers,
-// 2..4 = staged through shared memory with that many row blocks in flight,
-// 1 = tensor-core kernel with exact (q - z) operands, 5 = tensor-core kernel
-// with offset-form operands) and a cap on resident CTAs per SM.
-// Test hook (not in the public header): LUT3 batch-1 kernel variant (-1 = the
-// library's choice, 0 = indices pipelined through registers, 2 / 3 = staged
-// through shared memory with that many row blocks in flight).
-void lbq_debug_lut3_variant(int variant) { g_lut3_stages = (variant == 0 || variant == 2 || variant == 3) ? variant : -1; }
-
+// (-1 = the library's choice, 0 = weights pipelined through registers, 2..4 =
+// staged through shared memory with that many row blocks in flight) and a cap
+// on resident CTAs per SM.
 void lbq_debug_direct_variant(int variant, int ctas_per_sm) {
   g_direct_stages = (variant == 0 || (variant >= 2 && variant <= 4)) ? variant : -1;
   g_direct_ctas = ctas_per_sm > 0 ? ctas_per_sm : 0;
-  g_dmma = variant == 1 ? 1 : variant == 5 ? 2 : 0;
 }
 
 // Test hook (not in the public header): batch-1 lbq_w4a8_gemv on the tiled

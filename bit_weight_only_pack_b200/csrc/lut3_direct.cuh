@@ -112,107 +112,4 @@ __global__ void __launch_bounds__(kLdMaxWarps * 32, 1) lut3_direct_kernel(const 
   }
 }
 
-// The same GEMV with each lane's indices and table staged through shared
-// memory by per-thread asynchronous copies, S row blocks ahead: the 208 bytes
-// per lane and block no longer sit in registers (251 -> under 100 per
-// thread), so more warps fit an SM and the loads run ahead of the decode.
-// A lane reads back only what it copied, so its own copy-group wait is the
-// only synchronisation. Dynamic shared memory: uint4 [S][13][T] (12 chunks of
-// indices, then the table), then the row sums as in lut3_direct_kernel.
-template <int S>
-__global__ void __launch_bounds__(kLdMaxWarps * 32) lut3_direct_async_kernel(const Lut3DirectArgs a) {
-  extern __shared__ __align__(16) uint8_t ld_smem[];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int T = blockDim.x, nw = T >> 5;
-  const int kt = warp * 32 + lane;
-  const bool tok = kt < (a.K >> 6);
-  // 32-bit shared address of this thread's element 0 of stage 0; elements are T * 16 bytes apart
-  const uint32_t T16 = (uint32_t)T * 16;
-  const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ld_smem) + (uint32_t)tid * 16;
-  float* red = reinterpret_cast<float*>(ld_smem + (size_t)S * 13 * T16);
-  const uint8_t* ibase = a.i_region + (size_t)kt * a.N * 24;  // this lane's tile row of indices
-  const uint8_t* tbase = a.t_region + (size_t)kt * (a.N >> 3) * 16;
-
-  auto issue = [&](int rb, int st) {
-    if (tok && rb < a.row_blocks) {
-      const uint8_t* base = ibase + (size_t)rb * 192;
-      const uint32_t dst = ring_s + (uint32_t)st * 13 * T16;
-#pragma unroll
-      for (int v = 0; v < 12; ++v) cp_async16_s(dst + v * T16, base + 16 * v, 16);
-      cp_async16_s(dst + 12 * T16, tbase + (size_t)rb * 16, 16);
-    }
-    cp_async_commit();  // one group per row block, empty or not, keeps the wait count fixed
-  };
-
-  int rb = blockIdx.x;
-  // the weights are only read: the first S row blocks are requested before
-  // waiting for the previous kernel in the stream
-#pragma unroll
-  for (int st = 0; st < S; ++st) issue(rb + st * (int)gridDim.x, st);
-  griddep_launch_dependents();
-  griddep_wait();
-  uint32_t xr[32];  // this tile's 64 activations as BF16 pairs
-  if (tok) {
-    const uint4* xp = reinterpret_cast<const uint4*>(a.X + (size_t)kt * 64);
-#pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      const uint4 u = ld_nc_v4(xp + v);
-      xr[4 * v + 0] = u.x; xr[4 * v + 1] = u.y; xr[4 * v + 2] = u.z; xr[4 * v + 3] = u.w;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) xr[i] = 0u;
-  }
-
-  int lb = 0, st = 0;
-  for (; rb < a.row_blocks; rb += gridDim.x, ++lb) {
-    cp_async_wait<S - 1>();  // this lane's copies of row block rb have landed
-    float part[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) part[i] = 0.0f;
-    if (tok) {
-      const uint32_t src = ring_s + (uint32_t)st * 13 * T16;
-      const uint4 tab = lds128(src + 12 * T16);
-#pragma unroll
-      for (int i = 0; i < 8; i += 2) {
-        // rows i and i+1: 48 bytes, words 6i .. 6i+11 = chunks 3i/2 .. 3i/2+2
-        const uint4 u0 = lds128(src + (uint32_t)(3 * i / 2) * T16);
-        const uint4 u1 = lds128(src + (uint32_t)(3 * i / 2 + 1) * T16);
-        const uint4 u2 = lds128(src + (uint32_t)(3 * i / 2 + 2) * T16);
-        const uint32_t w12[12] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w, u2.x, u2.y, u2.z, u2.w};
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const uint32_t* wr = w12 + 6 * r;
-          float acc = 0.0f;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t wa = wr[3 * h], wb = wr[3 * h + 1], wc = wr[3 * h + 2];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              uint32_t p[4];
-              lut3_decode8(lut3_selector(t < 2 ? wa : wb, wc, t), tab, p);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) acc = fma2_bf16_f32(xr[16 * h + 4 * t + e], p[e], acc);
-            }
-          }
-          part[i + r] = acc;
-        }
-      }
-    }
-    const float total = butterfly8(part, lane);
-    if ((lane & 3) == 0) red[(lb * nw + warp) * 8 + butterfly8_row(lane)] = total;
-    issue(rb + S * (int)gridDim.x, st);  // refill the stage just read
-    st = st + 1 == S ? 0 : st + 1;
-  }
-  cp_async_wait<0>();
-  __syncthreads();
-  for (int t = tid; t < lb * 8; t += blockDim.x) {
-    const int l = t >> 3, row = t & 7;
-    const int r = (blockIdx.x + l * gridDim.x) * 8 + row;
-    float sum = 0.0f;
-    for (int w = 0; w < nw; ++w) sum += red[(l * nw + w) * 8 + row];
-    if (r < a.N) store_out(a.Y, (size_t)r, sum, a.y_bf16);
-  }
-}
-
 }  // namespace lbq
