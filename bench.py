@@ -759,11 +759,11 @@ def run_reference(args):
 # the decode step runs q/k/v and gate/up.
 PROFILE_CASES = {
     "c1": (4096, 4096, 32, "sym", "f16", 1, None),
-    "c2qkv": (4096, (4096, 1024, 1024), 32, "asym", "f16", 1, None),
-    "c2o": (4096, 4096, 32, "asym", "f16", 1, None),
-    "c2gateup": (4096, (14336, 14336), 32, "asym", "f16", 1, None),
+    "c2qkv": (14980608, (4096, 1024, 1024), 32, "asym", "f16", 1, None),
+    "c2o": (9997056, 4096, 32, "asym", "f16", 1, None),
+    "c2gateup": (70183168, (14336, 14336), 32, "asym", "f16", 1, None),
     "c2gate": (4096, 14336, 32, "asym", "f16", 1, None),
-    "c2down": (14336, 4096, 32, "asym", "f16", 1, None),
+    "c2down": (34921728, 4096, 32, "asym", "f16", 1, None),
     "c2kv": (4096, 1024, 32, "asym", "f16", 1, None),
     "c2gate_mma": (4096, 14336, 32, "asym", "f16", 1, 2),
     "c2gate_direct": (4096, 14336, 32, "asym", "f16", 1, 4),
@@ -916,13 +916,13 @@ STEP_CAPTURE_HASHES = {
     "tma.cuh": "5f428384c68b0ba7",
     "common.cuh": "6e369f75860e0aec",
     "lbq.cu#tmma-plan": "e30dce5cede0f3f4",
-    "lbq.cu#direct-plan": "7020bd2977db6eb8",
+    "lbq.cu#direct-plan": "b62033ebadd8a276",
 }
 STEP_TRAFFIC = {
-    "c2qkv": (14980864, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
-    "c2o": (9998848, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
-    "c2gateup": (70426368, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
-    "c2down": (34921472, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
+    "c2qkv": (14980608, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
+    "c2o": (9997056, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
+    "c2gateup": (70183168, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
+    "c2down": (34921728, STEP_CAPTURE_HASHES, "profiles/gemv_decode_step_shapes_4096x_asym_g32_m1.md"),
 }
 # the planner sections of lbq.cu (kernel choice, launch shape, K split, stages)
 PLAN_MARKERS = {"tmma-plan": ("// M = 1: TMA-fed warp-MMA GEMV", "// Scratch of that kernel for one call"),
