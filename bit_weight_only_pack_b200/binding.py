@@ -79,6 +79,7 @@ _SIGS = {
     "lbq_w4a8_gemv_grouped": ([ctypes.POINTER(lbq_w4a8_item), _c_int, _c_int, _c_int, _c_int, _c_int, _vp],
                               _c_int),
     "lbq_debug_w4a8_tiled": ([_c_int], None),
+    "lbq_debug_lut3_stages": ([_c_int], None),
     "lbq_moe_max_padded": ([_c_int, _c_int, _c_int, ctypes.POINTER(_c_int)], _c_int),
     "lbq_moe_align": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_int, _vp], _c_int),
     "lbq_moe_lut3_mx_gemm": ([_vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_int, _vp, _c_size, _c_int,
@@ -260,6 +261,11 @@ def make_w4a8_items(rows):
 def lbq_debug_w4a8_tiled(on):
     """Test hook: batch-1 W4A8 on the tiled kernel instead of the staged one."""
     _lib.lbq_debug_w4a8_tiled(1 if on else 0)
+
+
+def lbq_debug_lut3_stages(stages):
+    """Test hook: ring stages of the TMA-fed LUT3 batch-1 kernel (0 = the plan's choice)."""
+    _lib.lbq_debug_lut3_stages(int(stages))
 
 
 def lbq_moe_max_padded(num_pairs, num_experts, block):

@@ -32,6 +32,7 @@
 #include "gemm_ts.cuh"
 #include "gemm_mx.cuh"
 #include "lut3_direct.cuh"
+#include "lut3_tmma.cuh"
 #include "affine.cuh"
 #include "w4a8.cuh"
 #include "gemm_moe.cuh"
@@ -968,6 +969,74 @@ static lbq_status run_lut3_direct(const void* X, const void* image, const Layout
   return launch_kernel_ex(fn, dim3(grid), dim3(T), smem, st, g_pdl != 0, args, "LUT3 direct GEMV launch");
 }
 
+// LUT3, M = 1, TMA-fed warp-MMA kernel: one 8-row codebook group over all of
+// K per unit, K <= 8192 (at most 16 consumer warps of 4 or 8 tiles each).
+struct L3tPlan {
+  int kg, nw, grid, max_units, stage_bytes, t_off, stages, smem;
+};
+
+static int g_l3t_stages = 0;  // test hook: ring stages of the LUT3 TMA GEMV (0 = the plan's choice)
+static int g_l3t_default_stages = 4;
+
+static L3tPlan plan_lut3_tmma(int K, int N) {
+  L3tPlan p{};
+  const int KT = K / 64;
+  if (KT > 4 * 2 * kL3tMaxWarps) return p;
+  p.kg = KT <= 4 * kL3tMaxWarps ? 1 : 2;
+  p.nw = (KT + 4 * p.kg - 1) / (4 * p.kg);
+  const int units = N / 8;
+  p.grid = std::max(1, std::min(units, num_sms()));
+  p.max_units = (units + p.grid - 1) / p.grid;
+  p.t_off = (int)align_up((size_t)KT * 192, 128);
+  p.stage_bytes = p.t_off + (int)align_up((size_t)KT * 16, 128);
+  const int red_bytes = p.max_units * p.nw * 8 * 4;
+  const int avail = max_dynamic_smem() - 2 * kL3tMaxStages * 8 - 1024 - red_bytes;
+  // a short ring: copies in flight together land together (see the kernel)
+  const int want = g_l3t_stages ? g_l3t_stages : g_l3t_default_stages;
+  p.stages = std::min(std::min(std::min(p.max_units, want), kL3tMaxStages), avail / p.stage_bytes);
+  p.smem = 1024 + p.stages * p.stage_bytes + red_bytes;
+  return p;
+}
+
+static bool lut3_tmma_ok(int M, int K, int N, const void* X, const void* image) {
+  if (M != 1 || g_gemv_path == kPathMma || g_gemv_path == kPathDirect) return false;
+  if ((reinterpret_cast<uintptr_t>(X) & 15) || (reinterpret_cast<uintptr_t>(image) & 15)) return false;
+  const L3tPlan p = plan_lut3_tmma(K, N);
+  return p.nw > 0 && p.stages >= 1;
+}
+
+static lbq_status run_lut3_tmma(const void* X, const void* image, const Layout& L, void* Y, bool ybf16,
+                                cudaStream_t st) {
+  const L3tPlan p = plan_lut3_tmma(L.K, L.N);
+  if (p.nw == 0 || p.stages < 1) return fail(LBQ_ERR_UNSUPPORTED, "no LUT3 TMA GEMV plan for K=%d N=%d", L.K, L.N);
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  const int KT = L.K / 64;
+  CUtensorMap mi, mt;
+  // indices [K/64][N * 24 bytes] as 8-byte elements, box: one group's 192 bytes x every tile
+  if (!make_tmap_2d(&mi, img + L.off0, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, (uint64_t)L.N * 3, (uint64_t)KT,
+                    (uint64_t)L.N * 24, 24, (uint32_t)KT, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the LUT3 indices");
+  // tables [K/64][N/8 * 16 bytes], box: one group's 16 bytes x every tile
+  if (!make_tmap_2d(&mt, img + L.off3, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, (uint64_t)L.N / 4, (uint64_t)KT,
+                    (uint64_t)L.N * 2, 2, (uint32_t)KT, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the LUT3 tables");
+  Lut3TmmaArgs a{};
+  a.X = static_cast<const uint16_t*>(X);
+  a.Y = Y;
+  a.K = L.K; a.N = L.N;
+  a.units = L.N / 8;
+  a.nw = p.nw;
+  a.stages = p.stages; a.stage_bytes = p.stage_bytes; a.t_off = p.t_off;
+  a.max_units = p.max_units;
+  a.y_bf16 = ybf16 ? 1 : 0;
+  a.debug_drop = g_debug_drop;
+  const void* fn = p.kg == 1 ? (const void*)lut3_tmma_kernel<1> : (const void*)lut3_tmma_kernel<2>;
+  const int block = (p.nw + 1) * 32;
+  occupancy_for(fn, block, p.smem);  // raises the kernel's dynamic shared-memory limit once
+  void* args[] = {&mi, &mt, &a};
+  return launch_kernel_ex(fn, dim3(p.grid), dim3(block), p.smem, st, g_pdl != 0, args, "LUT3 TMA GEMV launch");
+}
+
 static lbq_status run_lut3_gemm_tc(const void* X, int M, const void* image, const Layout& L, void* Y, bool ybf16,
                                    cudaStream_t st) {
   const uint8_t* img = static_cast<const uint8_t*>(image);
@@ -1282,6 +1351,11 @@ void lbq_debug_direct_variant(int variant, int ctas_per_sm) {
 // W4A8 kernel (the one for M > 1) instead of the staged direct kernel.
 void lbq_debug_w4a8_tiled(int on) { g_w4a8_tiled = on ? 1 : 0; }
 
+// Test hook (not in the public header): ring stages of the TMA-fed LUT3
+// batch-1 kernel (1..16, capped by the CTA's units and shared memory; 0 = the
+// plan's choice).
+void lbq_debug_lut3_stages(int stages) { g_l3t_stages = (stages >= 1 && stages <= kL3tMaxStages) ? stages : 0; }
+
 lbq_status lbq_set_option(int option, int value) {
   if (option == LBQ_OPT_PDL) {
     g_pdl = value ? 1 : 0;
@@ -1414,6 +1488,7 @@ lbq_status lbq_lut3_gemm(const void* X, int x_dtype, int M, int K, int N, const 
   if (x_dtype != LBQ_DTYPE_BF16) return fail(LBQ_ERR_UNSUPPORTED, "LUT3 kernels take BF16 activations");
   const Layout L = make_layout(K, N, 0, LBQ_MODE_LUT3);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (lut3_tmma_ok(M, K, N, X, image) && !g_force_tc) return run_lut3_tmma(X, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);
   if (lut3_direct_ok(M, K) && !g_force_tc) return run_lut3_direct(X, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);
   if (M <= 16 && !g_force_tc) return run_lut3_skinny(X, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, ws, ws_bytes, s);
   if (g_gemm_path == 0) return run_gemm_ts(X, true, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);

@@ -108,7 +108,9 @@ SKINNY_SHAPES = [
 
 @pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16])
 @pytest.mark.parametrize("K,N", SKINNY_SHAPES)
-@pytest.mark.parametrize("path", [0, 2])  # 0: library's choice (direct loads at M = 1), 2: warp-MMA kernel
+# 0: library's choice (the TMA-fed warp-MMA kernel at M = 1 for K <= 8192),
+# 2: the skinny warp-MMA kernel
+@pytest.mark.parametrize("path", [0, 2])
 def test_lut3_gemv_parity(torch, lbq, M, K, N, path):
     idx, cb, ex = _inputs(70 + K + N, K, N)
     img = _image(torch, lbq, idx, cb, ex)
@@ -194,17 +196,77 @@ def test_lut3_m1_direct_kernel_k_limit(torch, lbq, K, N):
     lbq.device_status()
 
 
-@pytest.mark.parametrize("K,N", SKINNY_SHAPES + [(16384, 72), (1024, 8)])
-def test_lut3_m1_direct_kernel(torch, lbq, K, N):
-    """Batch 1 on the register-pipelined direct kernel, within the oracle's
-    tolerance, and the same bits on a repeated call."""
-    idx, cb, ex = _inputs(80 + K + N, K, N)
+M1_SHAPES = SKINNY_SHAPES + [
+    (16384, 72),     # the direct kernel's longest K (the TMA kernel takes K <= 8192)
+    (1024, 8),       # one codebook group: a one-CTA grid
+    (8192, 40),      # the TMA kernel's longest K: 8 tiles per lane quad
+    (4160, 16),      # past 4096: the two-group form with idle tiles in the last warp
+    (4096, 14336),   # the 3-bit LUT workload: 13 groups on the busiest CTAs
+]
+
+
+@pytest.mark.parametrize("K,N", M1_SHAPES)
+# (gemv path, ring stages): the library's choice; the TMA-fed kernel with a
+# one-stage ring (every unit waits for the previous one's release) and with
+# its longest ring; the register-pipelined direct kernel
+@pytest.mark.parametrize("path,stages", [(0, 0), (0, 1), (0, 16), (4, 0)])
+def test_lut3_m1_kernels(torch, lbq, K, N, path, stages):
+    """Batch 1 on the TMA-fed warp-MMA kernel (the default for K <= 8192, at
+    several ring lengths) and on the register-pipelined direct kernel, within
+    the oracle's tolerance (full size: on sampled channels), and the same bits
+    on a repeated call."""
+    if K * N > 1 << 24:
+        idx, cb, ex = workloads.lut3_host(5, K, N)
+        cols = sample_columns(N, 96, seed=K)
+    else:
+        idx, cb, ex = _inputs(80 + K + N, K, N)
+        cols = None
     img = _image(torch, lbq, idx, cb, ex)
     X = workloads.activations_host(80 + K, 1, K, "bf16")
-    _, Y = _check_gemm(torch, lbq, idx, cb, ex, img, X)
-    Y0 = lbq.lut3_gemm(X.cuda(), img, N)
-    torch.cuda.synchronize()
-    assert torch.equal(Y, Y0)
+    lbq.lbq_debug_gemv_path(path)
+    lbq.lbq_debug_lut3_stages(stages)
+    try:
+        if cols is None:
+            _, Y = _check_gemm(torch, lbq, idx, cb, ex, img, X)
+        else:
+            Y = lbq.lut3_gemm(X.cuda(), img, N)
+            torch.cuda.synchronize()
+            groups = np.unique(cols // 8)
+            ch = (groups[:, None] * 8 + np.arange(8)[None, :]).reshape(-1)
+            deq = lut3.dequant(np.ascontiguousarray(idx[:, ch]), cb[:, groups], ex[:, groups])
+            check_outputs(Y.cpu(), X, deq, ch)
+        Y0 = lbq.lut3_gemm(X.cuda(), img, N)
+        torch.cuda.synchronize()
+        assert torch.equal(Y, Y0)
+    finally:
+        lbq.lbq_debug_gemv_path(0)
+        lbq.lbq_debug_lut3_stages(0)
+    lbq.device_status()
+
+
+def test_lut3_m1_bounded_wait_runs_out_and_is_reported(torch, lbq):
+    """Failure detection without a GPU fault on the TMA-fed LUT3 kernel: with
+    the producer's copies withheld (test hook) on a one-CTA launch, every
+    consumer wait gives up after a short spin limit, Y is not written, the
+    device flag reads LBQ_ERR_DEVICE and is cleared, and the next call passes
+    parity."""
+    K, N = 1024, 8
+    idx, cb, ex = _inputs(360, K, N)
+    img = _image(torch, lbq, idx, cb, ex)
+    X = workloads.activations_host(361, 1, K, "bf16")
+    sentinel = torch.full((1, N), 7.0, dtype=torch.bfloat16, device="cuda")
+    lbq.device_status()  # nothing pending
+    lbq.lbq_debug_drop_copies(1)
+    try:
+        lbq.lut3_gemm(X.cuda(), img, N, Y=sentinel)
+        with pytest.raises(lbq.LbqError) as err:
+            lbq.device_status()
+        assert err.value.status == 4  # LBQ_ERR_DEVICE
+    finally:
+        lbq.lbq_debug_drop_copies(0)
+    assert torch.equal(sentinel.cpu(), torch.full((1, N), 7.0, dtype=torch.bfloat16))  # Y untouched
+    lbq.device_status()  # the flag was cleared
+    _check_gemm(torch, lbq, idx, cb, ex, img, X)
     lbq.device_status()
 
 
