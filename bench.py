@@ -499,7 +499,16 @@ def _secondary_measurements(torch, lbq, workloads, device, peaks, quick):
         ms = rotating_lut3_ms(torch, lbq, images, X, N, ws, reps=3)
         if M == 1:
             out["c5_lut3_m1"] = {"us": ms * 1e3, "GBps": b / ms / 1e6, "frac_hbm": b / ms / 1e6 / hbm,
-                                 "image_bytes_read": images[0].numel(), "weight_copies": len(images)}
+                                 "image_bytes_read": images[0].numel(), "weight_copies": len(images),
+                                 "kernel": "lut3_tmma_kernel"}
+            # the register-pipelined direct kernel (the default for 8192 < K <= 16384), timed beside it
+            lbq.lbq_debug_gemv_path(4)
+            try:
+                ms_d = rotating_lut3_ms(torch, lbq, images, X, N, ws, reps=3)
+            finally:
+                lbq.lbq_debug_gemv_path(0)
+            out["c5_lut3_m1_direct_kernel"] = {"us": ms_d * 1e3, "GBps": b / ms_d / 1e6,
+                                               "frac_hbm": b / ms_d / 1e6 / hbm}
         else:
             tf = 2.0 * M * K * N / ms / 1e9
             out[f"c5_lut3_m{M}"] = {"us": ms * 1e3, "TFLOPs": tf, "frac_bf16_peak": tf / tc_peak,
