@@ -360,8 +360,9 @@ static lbq_status run_skinny(const void* X, bool xbf16, int M, const void* image
   CUtensorMap tw, tx;
   const bool ok = make_tmap_2d(&tw, img + L.off0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.K / 2, (uint64_t)L.N,
                                (uint64_t)L.K / 2, 128, kSkRows, CU_TENSOR_MAP_SWIZZLE_128B) &&
-                  make_tmap_2d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, (uint64_t)L.K, (uint64_t)M,
-                               (uint64_t)L.K * 2, 64, (uint32_t)M, CU_TENSOR_MAP_SWIZZLE_128B);
+                  // X [M][K] as (32-k chunk, token, chunk index); box: 8 chunks of all M tokens
+                  make_tmap_3d(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT16, 32, (uint64_t)M, (uint64_t)L.K / 32,
+                               (uint64_t)L.K * 2, 64, 32, (uint32_t)M, 8, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the skinny kernel");
   SkinnyArgs a{};
   a.Y = Y;

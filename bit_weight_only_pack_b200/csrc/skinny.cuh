@@ -22,8 +22,10 @@
 //    batch padding to 128 is streamed ("no swap-AB" is one of the reasons the
 //    vLLM LUT-B kernel loses at small batch).
 //  * Producer warp: per 256-k stage, TMA loads of a 128-row x 128-byte code
-//    tile (128-byte swizzle) and the 64-k activation boxes (128-byte
-//    swizzle), and one bulk copy each of the tile's scales / zero points for
+//    tile (128-byte swizzle) and one box of the stage's activations (a 3-D
+//    view of X: 32-k chunk x token x chunk, so chunk j of token m lands at
+//    (j M + m) 64 bytes and a quarter-warp's two tokens fall in opposite bank
+//    halves), and one bulk copy each of the tile's scales / zero points for
 //    the stage's groups (contiguous in the 128-channel-tiled image), all
 //    completing on one mbarrier; a ring of kSkStages stages feeds 8 consumer warps (16 rows
 //    each). ldmatrix.x4 hands each thread the code words of rows r and r+8 for
@@ -138,9 +140,9 @@ __device__ __forceinline__ void mma_16816_zc(float (&d)[4], const uint32_t (&a)[
 template <bool BF16, bool ASYM, int NT, int GC, bool KFULL>
 __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
     const __grid_constant__ CUtensorMap tw, const __grid_constant__ CUtensorMap tx, const SkinnyArgs a) {
-  constexpr int kXBox = NT * 1024;  // one 64-k activation box (8*NT rows x 128 B)
+  constexpr int kXBytes = NT * 4096;  // the stage's activations: 8 chunks x up to 8*NT tokens x 64 B
   constexpr int kOffX = kSkWBytes;
-  constexpr int kOffS = kOffX + 4 * kXBox;
+  constexpr int kOffS = kOffX + kXBytes;
   constexpr int kOffZ = kOffS + kSkSBytes;
   constexpr int kSlot = kOffZ + (ASYM ? kSkZBytes : 0);
   extern __shared__ uint8_t dsmem[];
@@ -192,9 +194,9 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
         uint8_t* dst = ring + (size_t)slot * kSlot;
         const int gs0 = st * 8 / GC;  // first group of the stage
         const int ng = min(8 / GC, a.G - gs0);  // groups of the stage
-        const int nxb = KFULL ? 4 : min(4, (K - st * 256 + 63) / 64);  // activation boxes that start inside K
+        // the activation box counts in full (chunks past K read as zeros)
         mbar_arrive_expect_tx(&full_bar[slot],
-                              (uint32_t)(kSkWBytes + nxb * M * 128 + ng * kSkRows * (ASYM ? 3 : 2)));
+                              (uint32_t)(kSkWBytes + M * 512 + ng * kSkRows * (ASYM ? 3 : 2)));
         tma_load_2d(dst, &tw, st * 128, rt * kSkRows, &full_bar[slot]);
         const size_t meta0 = ((size_t)rt * a.G + gs0) * kSkRows;  // element index of (tile rt, group gs0, row 0)
         bulk_load(dst + kOffS, a.s_region + meta0 * 2, (uint32_t)(ng * kSkRows * 2), &full_bar[slot]);
@@ -204,13 +206,11 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
           for (int i = 0; i <= it; ++i) {  // activations of the slots filled so far
             const long long ui = u_begin + i;
             const int sti = (int)(ui - (ui / S_t) * S_t);
-            const int nxi = KFULL ? 4 : min(4, (K - sti * 256 + 63) / 64);
             uint8_t* di = ring + (size_t)(i % kSkStages) * kSlot;
-            for (int j = 0; j < nxi; ++j)
-              tma_load_2d(di + kOffX + j * kXBox, &tx, sti * 256 + 64 * j, 0, &full_bar[i % kSkStages]);
+            tma_load_3d(di + kOffX, &tx, 0, 0, sti * 8, &full_bar[i % kSkStages]);
           }
         } else if (it >= nfirst) {
-          for (int j = 0; j < nxb; ++j) tma_load_2d(dst + kOffX + j * kXBox, &tx, st * 256 + 64 * j, 0, &full_bar[slot]);
+          tma_load_3d(dst + kOffX, &tx, 0, 0, st * 8, &full_bar[slot]);
         }
       }
     }
@@ -225,14 +225,15 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
   uint32_t lm_off[4];
 #pragma unroll
   for (int cp = 0; cp < 4; ++cp) lm_off[cp] = sw128(lm_row, 2 * cp + (lane >> 4));
-  // activation fragment offsets of this thread: column m = g + 8n, chunk half (ci & 1)
-  uint32_t x_off[NT][2];
+  // activation fragment offsets of this thread: column m = g + 8n, 16 bytes t
+  // of each 32-k chunk ci at x_off[n] + ci * x_step
+  uint32_t x_off[NT];
   bool x_ok[NT];
+  const uint32_t x_step = (uint32_t)M * 64u;
 #pragma unroll
   for (int n = 0; n < NT; ++n) {
     x_ok[n] = (g + 8 * n) < M;
-    x_off[n][0] = (uint32_t)(kOffX + sw128(g + 8 * n, t));
-    x_off[n][1] = (uint32_t)(kOffX + sw128(g + 8 * n, 4 + t));
+    x_off[n] = (uint32_t)(kOffX + (g + 8 * n) * 64 + 16 * t);
   }
   const int s_off_r = kOffS + lrow * 2, s_off_r8 = s_off_r + 8 * 2;
   const int z_off_r = kOffZ + lrow, z_off_r8 = z_off_r + 8;
@@ -312,7 +313,7 @@ __global__ void __launch_bounds__(kSkThreads, 2) skinny_kernel(
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
           uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-          if (x_ok[n]) xv = *reinterpret_cast<const uint4*>(sp + x_off[n][ci & 1] + (ci >> 1) * kXBox);
+          if (x_ok[n]) xv = *reinterpret_cast<const uint4*>(sp + x_off[n] + ci * x_step);
           // FP16: a0 holds k-slots {0,1 | 4,5} of the 8-k word, a1 {2,3 | 6,7};
           // BF16: a0 {0,1 | 2,3}, a1 {4,5 | 6,7}
           const uint32_t b00 = xv.x, b01 = BF16 ? xv.y : xv.z, b10 = BF16 ? xv.z : xv.y, b11 = xv.w;
