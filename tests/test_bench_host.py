@@ -150,3 +150,24 @@ def test_step_traffic_records_are_consistent():
     assert all(v is not None for v in now.values())
     complete = all(r[0] is not None and r[1] == now for r in bench.STEP_TRAFFIC.values())
     assert (bench.traffic_from_profiles() is not None) == complete
+
+
+def test_profile_cases_are_the_shapes_they_name():
+    """Every profile case is a shape the library takes (K a multiple of 64 and
+    at most 65536, N positive, M in 1 .. 8192), and the decode step's cases
+    have the step's shapes (K = 4096, or 14336 for down)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    for name, case in bench.PROFILE_CASES.items():
+        K, N, group, mode, xdt, M = case[:6]
+        assert K % 64 == 0 and 64 <= K <= 65536, (name, K)
+        Ns = N if isinstance(N, tuple) else (N,)
+        assert all(0 <= n <= 1 << 20 for n in Ns), (name, N)
+        assert 1 <= M <= 8192, (name, M)
+    step = {"c2qkv": (4096, (4096, 1024, 1024)), "c2o": (4096, 4096), "c2gateup": (4096, (14336, 14336)),
+            "c2down": (14336, 4096)}
+    for name, (K, N) in step.items():
+        assert tuple(bench.PROFILE_CASES[name][:2]) == (K, N), name
+    # the step's traffic records: mean bytes per launch within 1% of the algorithmic bytes
+    mean = sum(r[0] for r in bench.STEP_TRAFFIC.values()) / len(bench.STEP_TRAFFIC)
+    assert abs(mean / 32374784 - 1.0) < 0.01
