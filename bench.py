@@ -270,10 +270,14 @@ class DecodeStep:
 class E2EStep:
     """One decode step through the public C-ABI calls (no graph) with its
     inputs copied in from pinned host memory and its outputs copied back. The
-    layers go in `chunks` groups: a copy stream brings each group's X in and
-    takes its Y out, and the compute stream waits only for its own group's X,
-    so the copies of the other groups overlap the GEMVs (the step's X vectors
-    are inputs of the step, as in the bench's graph)."""
+    layers go in `chunks` groups, with one copy stream bringing X in and one
+    taking Y out: a group's X for the next step is copied in as soon as this
+    step's GEMVs of that group have read it, and a group's Y goes out as soon as
+    its GEMVs are done, so the copies overlap the other groups' GEMVs (the
+    step's X vectors are inputs of the step, as in the bench's graph). Every
+    step's copies lie inside the timed region: the first step's inputs wait
+    for the compute stream (reset()), and finish() makes the compute stream
+    wait for the last outputs."""
 
     def __init__(self, torch, step, chunks=4):
         self.torch, self.step = torch, step
@@ -283,30 +287,46 @@ class E2EStep:
         self.x_host = torch.empty_like(step.x_all, device="cpu").pin_memory()
         self.x_host.copy_(step.x_all.cpu())
         self.y_host = torch.empty_like(step.y_all, device="cpu").pin_memory()
-        self.cs = torch.cuda.Stream()
-        self.ev_in = [torch.cuda.Event() for _ in self.groups]
-        self.ev_out = [torch.cuda.Event() for _ in self.groups]
+        self.cs_in, self.cs_out = torch.cuda.Stream(), torch.cuda.Stream()
+        self.ev_in = [torch.cuda.Event() for _ in self.groups]    # X of the group copied in
+        self.ev_used = [torch.cuda.Event() for _ in self.groups]  # the group's GEMVs done
+        self.ev_out = [torch.cuda.Event() for _ in self.groups]   # Y of the group copied out
         self.done = torch.cuda.Event()
+        self.started = False
+
+    def reset(self):
+        """The next step's input copies wait for the compute stream's work so far."""
+        self.started = False
 
     def run(self):
-        torch, step, cs = self.torch, self.step, self.cs
+        torch, step = self.torch, self.step
         main = torch.cuda.current_stream()
-        cs.wait_stream(main)
-        for g, ev in zip(self.groups, self.ev_in):
+        for i, g in enumerate(self.groups):
             (x0, _), (x1, _) = g[0][2], g[-1][2]
-            with torch.cuda.stream(cs):
+            with torch.cuda.stream(self.cs_in):
+                if self.started:
+                    self.cs_in.wait_event(self.ev_used[i])  # the previous step has read this X
+                else:
+                    self.cs_in.wait_stream(main)
                 step.x_all[x0:x1].copy_(self.x_host[x0:x1], non_blocking=True)
-                ev.record(cs)
-        for g, ev_in, ev_out in zip(self.groups, self.ev_in, self.ev_out):
-            main.wait_event(ev_in)
+                self.ev_in[i].record(self.cs_in)
+        for i, g in enumerate(self.groups):
+            main.wait_event(self.ev_in[i])
+            if self.started:
+                main.wait_event(self.ev_out[i])  # the previous step's Y of this group is out
             step.launch_all(step.calls[g[0][0]:g[-1][1]])
-            ev_out.record(main)
+            self.ev_used[i].record(main)
             (y0, _), (y1, _) = g[0][3], g[-1][3]
-            cs.wait_event(ev_out)
-            with torch.cuda.stream(cs):
+            with torch.cuda.stream(self.cs_out):
+                self.cs_out.wait_event(self.ev_used[i])
                 self.y_host[y0:y1].copy_(step.y_all[y0:y1], non_blocking=True)
-        self.done.record(cs)
-        main.wait_event(self.done)
+                self.ev_out[i].record(self.cs_out)
+        self.done.record(self.cs_out)
+        self.started = True
+
+    def finish(self):
+        """The compute stream waits for the last step's output copies."""
+        self.torch.cuda.current_stream().wait_event(self.done)
 
 
 def time_graph(torch, graph, steps, warmup, world):
@@ -1026,13 +1046,16 @@ def main():
     lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 0 if args.no_pdl else 1)
     for _ in range(args.warmup):
         e2e.run()
+    e2e.finish()
     torch.cuda.synchronize()
     barrier(world)
     launches_before = lbq.lbq_launch_count()  # the timed steps' launches only
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
+    e2e.reset()
     for _ in range(args.steps):
         e2e.run()
+    e2e.finish()
     e1.record()
     torch.cuda.synchronize()
     lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 0)
@@ -1090,9 +1113,11 @@ def main():
                 "h2d_bytes_per_step": step.x_all.numel() * 2, "d2h_bytes_per_step": step.y_all.numel() * 2,
                 "ms_per_step": e2e_ms, "kernel_launches": e2e_launches,
                 "how": "per step: pinned host X -> device, the step's lbq_gemv / lbq_gemv_grouped C-ABI calls "
-                       "(no graph), device Y -> pinned host; the copies run on a second stream in four groups of "
-                       "layers, each group's GEMVs waiting only for that group's X, so the other groups' copies "
-                       "overlap the GEMVs; CUDA events on the launching stream, which waits for the last copy"},
+                       "(no graph), device Y -> pinned host; in four groups of layers, X in on one copy stream "
+                       "(a group's next-step X as soon as this step's GEMVs of the group have read it), Y out on "
+                       "another (as soon as the group's GEMVs are done), each group's GEMVs waiting only for its "
+                       "own X and its previous Y copy; CUDA events on the launching stream, the first step's "
+                       "copies after the start event and the end event after the last copy"},
         "gpu_launches": launches * args.steps,
         "cpu_baseline": cpu,
         "secondary": secondary,
