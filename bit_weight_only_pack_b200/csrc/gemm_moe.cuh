@@ -354,14 +354,43 @@ __global__ void __launch_bounds__(1024) moe_align_kernel(const int32_t* __restri
     if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
   }
   __syncthreads();
-  if (tid == 0) {
-    int o = 0;
-    for (int e = 0; e < E; ++e) {
+  {
+    // start[e] = padded counts of the experts before e: each thread sums a
+    // contiguous range of experts, then an exclusive scan over the threads
+    // (warp shuffles, then one warp over the warp totals)
+    __shared__ int warp_sum[32];
+    const int per = (E + nt - 1) / nt, e0 = min(E, tid * per), e1 = min(E, e0 + per);
+    int mine = 0;
+    for (int e = e0; e < e1; ++e) mine += (cnt[e] + block - 1) / block * block;
+    const int lane = tid & 31, warp = tid >> 5;
+    int incl = mine;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+      if (lane >= d) incl += v;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int nwarps = nt >> 5;
+      int w = lane < nwarps ? warp_sum[lane] : 0;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, w, d);
+        if (lane >= d) w += v;
+      }
+      if (lane < nwarps) warp_sum[lane] = w;  // inclusive totals of warps 0..lane
+    }
+    __syncthreads();
+    int o = incl - mine + (warp > 0 ? warp_sum[warp - 1] : 0);
+    for (int e = e0; e < e1; ++e) {
       start[e] = o;
       o += (cnt[e] + block - 1) / block * block;
     }
-    start[E] = o;
-    *total = o;
+    if (tid == nt - 1) {
+      start[E] = o;
+      *total = o;
+    }
   }
   for (int i = tid; i < max_padded; i += nt) sorted_ids[i] = P;
   for (int b = tid; b < max_padded / block; b += nt) expert_ids[b] = -1;

@@ -58,7 +58,9 @@ def _check_align(torch, lbq, ids, E, emap=None, block=128):
     return s, e, total
 
 
-@pytest.mark.parametrize("T,top_k,E", [(1, 8, 256), (16, 8, 256), (256, 8, 64), (37, 2, 8), (300, 1, 3)])
+# the last two: more experts than the kernel's 1024 threads (each thread scans a range of experts)
+@pytest.mark.parametrize("T,top_k,E", [(1, 8, 256), (16, 8, 256), (256, 8, 64), (37, 2, 8), (300, 1, 3),
+                                       (300, 4, 1500), (5, 2, 2048)])
 def test_align_matches_the_oracle(torch, lbq, T, top_k, E):
     _check_align(torch, lbq, _routing(70 + T, T, top_k, E), E)
 
@@ -112,6 +114,8 @@ def _run_case(torch, lbq, T, top_k, E, K, N, ydt="bf16", emap=None, seed=80):
     (5, 3, 8, 128, 64),        # fewer rows than a block for every expert, one k-block
     (64, 8, 16, 2048, 256),    # the MoE layer's gate/up K, two channel tiles
     (200, 2, 2, 512, 128),     # experts with several blocks each
+    (1, 8, 32, 2048, 1024),    # one token over 8 of 32 experts at the layer's gate/up shape
+    (16, 8, 64, 512, 2056),    # 16 tokens, some experts with several pairs; a ragged last channel tile
 ])
 @pytest.mark.parametrize("ydt", ["bf16", "f16"])
 def test_grouped_gemm_matches_the_routing_definition(torch, lbq, T, top_k, E, K, N, ydt):
