@@ -279,7 +279,7 @@ class E2EStep:
     for the compute stream (reset()), and finish() makes the compute stream
     wait for the last outputs."""
 
-    def __init__(self, torch, step, chunks=4):
+    def __init__(self, torch, step, chunks=2):
         self.torch, self.step = torch, step
         n = len(step.layers)
         per = -(-n // chunks)
@@ -1003,6 +1003,8 @@ def main():
     ap.add_argument("--ungrouped", action="store_true",
                     help="one lbq_gemv launch per projection instead of grouped q/k/v and gate/up")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-groups", type=int, default=2,
+                    help="groups of layers whose host copies overlap the other groups' GEMVs in the e2e step")
     ap.add_argument("--profile", default=None, choices=sorted(PROFILE_CASES),
                     help="run a small case for ncu (a few launches over weight copies larger than L2) and exit")
     args = ap.parse_args()
@@ -1042,7 +1044,7 @@ def main():
     # end to end through the public C-ABI call: every step copies its
     # activations in from pinned host memory, makes the step's C-ABI calls
     # (no graph) and copies the outputs back to pinned host memory
-    e2e = E2EStep(torch, step)
+    e2e = E2EStep(torch, step, chunks=max(1, args.e2e_groups))
     lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 0 if args.no_pdl else 1)
     for _ in range(args.warmup):
         e2e.run()
@@ -1113,11 +1115,11 @@ def main():
                 "h2d_bytes_per_step": step.x_all.numel() * 2, "d2h_bytes_per_step": step.y_all.numel() * 2,
                 "ms_per_step": e2e_ms, "kernel_launches": e2e_launches,
                 "how": "per step: pinned host X -> device, the step's lbq_gemv / lbq_gemv_grouped C-ABI calls "
-                       "(no graph), device Y -> pinned host; in four groups of layers, X in on one copy stream "
+                       "(no graph), device Y -> pinned host; in %d groups of layers, X in on one copy stream "
                        "(a group's next-step X as soon as this step's GEMVs of the group have read it), Y out on "
                        "another (as soon as the group's GEMVs are done), each group's GEMVs waiting only for its "
                        "own X and its previous Y copy; CUDA events on the launching stream, the first step's "
-                       "copies after the start event and the end event after the last copy"},
+                       "copies after the start event and the end event after the last copy" % len(e2e.groups)},
         "gpu_launches": launches * args.steps,
         "cpu_baseline": cpu,
         "secondary": secondary,
