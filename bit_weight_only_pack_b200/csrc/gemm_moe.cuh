@@ -35,7 +35,8 @@ namespace lbq {
 
 constexpr int kMoeBM = 128;  // tokens (sorted rows) per tile = the alignment block
 // Ring depth and converted weight tiles in flight. Measured at the write-up's
-// layer shape: 5 stages with 2 tiles, or 4 with 3, change the time by 5% at most.
+// layer shape: 5 stages with 2 tiles, or 4 with 3 (or 2), change the time by 5%
+// at most, at 1, 16 and 256 tokens alike.
 constexpr int kMoeStages = 3;
 constexpr int kMoeABufs = 4;
 constexpr int kMoeConvWarps = 8, kMoeGatherWarps = 4;
