@@ -288,3 +288,39 @@ def test_tables_exact_at_the_exponent_range_ends(torch, lbq):
     W = lbq.dequant(img, K, N, 0, "lut3").cpu().numpy()
     assert np.array_equal(W.astype(np.float64), lut3.dequant(idx, cb, ex))
     lbq.device_status()
+
+
+def test_lut3_m1_pdl_graph(torch, lbq):
+    """The batch-1 LUT3 kernel with programmatic dependent launch inside a CUDA
+    graph: three back-to-back launches, each reading the previous one's output
+    as its activation (the weights stream before the wait, X only after it)."""
+    K = N = 4096
+    idx, cb, ex = workloads.lut3_host(342, K, N)
+    img = _image(torch, lbq, idx, cb, ex)
+    deq = lut3.dequant(idx, cb, ex)
+    X0 = workloads.activations_host(343, 1, K, "bf16").cuda()
+    bufs = [X0] + [torch.empty((1, N), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    ws = lbq.workspace(2, 1, K, N, 0, "lut3")
+    lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 1)
+    try:
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for i in range(3):
+                lbq.lut3_gemm(bufs[i], img, N, ws=ws, Y=bufs[i + 1])
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(3):
+                lbq.lut3_gemm(bufs[i], img, N, ws=ws, Y=bufs[i + 1])
+        for b in bufs[1:]:
+            b.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+    finally:
+        lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 0)
+    lbq.device_status()
+    # each stage against the oracle applied to the previous stage's GPU output
+    for i in range(3):
+        check_outputs(bufs[i + 1].cpu(), bufs[i].cpu(), deq)
