@@ -529,6 +529,20 @@ def _secondary_measurements(torch, lbq, workloads, device, peaks, quick):
                 lbq.lbq_debug_gemv_path(0)
             out["c5_lut3_m1_direct_kernel"] = {"us": ms_d * 1e3, "GBps": b / ms_d / 1e6,
                                                "frac_hbm": b / ms_d / 1e6 / hbm}
+            # batch 4 on the TMA-fed batch kernel, and on the skinny kernel beside it
+            X4 = workloads.activations_device(5, 4, K, "bf16", device)
+            ws4 = lbq.workspace(2, 4, K, N, 0, "lut3")
+            ms4 = rotating_lut3_ms(torch, lbq, images, X4, N, ws4, reps=3)
+            out["c5_lut3_m4"] = {"us": ms4 * 1e3, "GBps": b / ms4 / 1e6, "frac_hbm": b / ms4 / 1e6 / hbm,
+                                 "kernel": "lut3_tmma_batch_kernel"}
+            lbq.lbq_debug_lut3_batch_off(1)
+            try:
+                ms4s = rotating_lut3_ms(torch, lbq, images, X4, N, ws4, reps=3)
+            finally:
+                lbq.lbq_debug_lut3_batch_off(0)
+            out["c5_lut3_m4_skinny_kernel"] = {"us": ms4s * 1e3, "GBps": b / ms4s / 1e6,
+                                               "frac_hbm": b / ms4s / 1e6 / hbm}
+            del X4, ws4
         else:
             tf = 2.0 * M * K * N / ms / 1e9
             out[f"c5_lut3_m{M}"] = {"us": ms * 1e3, "TFLOPs": tf, "frac_bf16_peak": tf / tc_peak,

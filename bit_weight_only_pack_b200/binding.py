@@ -80,6 +80,7 @@ _SIGS = {
                               _c_int),
     "lbq_debug_w4a8_tiled": ([_c_int], None),
     "lbq_debug_lut3_stages": ([_c_int], None),
+    "lbq_debug_lut3_batch_off": ([_c_int], None),
     "lbq_moe_max_padded": ([_c_int, _c_int, _c_int, ctypes.POINTER(_c_int)], _c_int),
     "lbq_moe_align": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_int, _vp], _c_int),
     "lbq_moe_lut3_mx_gemm": ([_vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_int, _vp, _c_size, _c_int,
@@ -266,6 +267,11 @@ def lbq_debug_w4a8_tiled(on):
 def lbq_debug_lut3_stages(stages):
     """Test hook: ring stages of the TMA-fed LUT3 batch-1 kernel (0 = the plan's choice)."""
     _lib.lbq_debug_lut3_stages(int(stages))
+
+
+def lbq_debug_lut3_batch_off(on):
+    """Test hook: LUT3 at M = 2..8 on the skinny kernel instead of the TMA-fed batch kernel."""
+    _lib.lbq_debug_lut3_batch_off(1 if on else 0)
 
 
 def lbq_moe_max_padded(num_pairs, num_experts, block):

@@ -33,6 +33,7 @@
 #include "gemm_mx.cuh"
 #include "lut3_direct.cuh"
 #include "lut3_tmma.cuh"
+#include "lut3_tmma_batch.cuh"
 #include "affine.cuh"
 #include "w4a8.cuh"
 #include "gemm_moe.cuh"
@@ -1038,6 +1039,77 @@ static lbq_status run_lut3_tmma(const void* X, const void* image, const Layout& 
   return launch_kernel_ex(fn, dim3(p.grid), dim3(block), p.smem, st, g_pdl != 0, args, "LUT3 TMA GEMV launch");
 }
 
+// LUT3, M = 2..8, TMA-fed warp-MMA kernel with the batch on the MMA's columns.
+static int g_l3b_off = 0;  // test hook: 1 = M = 2..8 on the skinny kernel instead
+
+struct L3bPlan {
+  int kj, nw, grid, stage_bytes, t_off, stages, xs_off, red_off, smem;
+};
+
+static L3bPlan plan_lut3_batch(int M, int K, int N) {
+  L3bPlan p{};
+  const int KT = K / 64;
+  if (M < 2 || M > kL3bMaxM || KT > 8 * kL3tMaxWarps || (size_t)M * K * 2 > 64 * 1024) return p;
+  p.nw = std::min(kL3tMaxWarps, KT);
+  const int kj = (KT + p.nw - 1) / p.nw;
+  p.kj = kj <= 2 ? 2 : kj <= 4 ? 4 : 8;
+  const int tiles = (N + kL3bRows - 1) / kL3bRows;
+  p.grid = std::max(1, std::min(tiles, num_sms()));
+  const int max_units = (tiles + p.grid - 1) / p.grid;
+  p.t_off = (int)align_up((size_t)KT * 384, 128);
+  p.stage_bytes = p.t_off + (int)align_up((size_t)KT * 32, 128);
+  const int x_bytes = (int)align_up((size_t)M * K * 2, 128);
+  const int red_bytes = 2 * p.nw * 128 * (int)sizeof(float);
+  const int avail = max_dynamic_smem() - 2 * kL3tMaxStages * 8 - 1024 - x_bytes - red_bytes;
+  const int want = g_l3t_stages ? g_l3t_stages : g_l3t_default_stages;
+  p.stages = std::min(std::min(std::min(max_units, want), kL3tMaxStages), avail / p.stage_bytes);
+  p.xs_off = p.stages * p.stage_bytes;
+  p.red_off = p.xs_off + x_bytes;
+  p.smem = 1024 + p.red_off + red_bytes;
+  return p;
+}
+
+static bool lut3_batch_ok(int M, int K, int N, const void* X, const void* image) {
+  if (g_l3b_off || g_gemv_path == kPathMma) return false;
+  if ((reinterpret_cast<uintptr_t>(X) & 15) || (reinterpret_cast<uintptr_t>(image) & 15)) return false;
+  const L3bPlan p = plan_lut3_batch(M, K, N);
+  return p.nw > 0 && p.stages >= 1;
+}
+
+static lbq_status run_lut3_batch(const void* X, int M, const void* image, const Layout& L, void* Y, bool ybf16,
+                                 cudaStream_t st) {
+  const L3bPlan p = plan_lut3_batch(M, L.K, L.N);
+  if (p.nw == 0 || p.stages < 1) return fail(LBQ_ERR_UNSUPPORTED, "no LUT3 batch GEMV plan for M=%d K=%d", M, L.K);
+  const uint8_t* img = static_cast<const uint8_t*>(image);
+  const int KT = L.K / 64;
+  CUtensorMap mi, mt;
+  // indices [K/64][N * 24 bytes] as 8-byte words, box: two groups' 384 bytes x every tile
+  if (!make_tmap_2d(&mi, img + L.off0, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, (uint64_t)L.N * 3, (uint64_t)KT,
+                    (uint64_t)L.N * 24, 48, (uint32_t)KT, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the LUT3 indices");
+  // tables [K/64][N/8 * 16 bytes], box: two groups' 32 bytes x every tile
+  if (!make_tmap_2d(&mt, img + L.off3, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, (uint64_t)L.N / 4, (uint64_t)KT,
+                    (uint64_t)L.N * 2, 4, (uint32_t)KT, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the LUT3 tables");
+  Lut3BatchArgs a{};
+  a.X = static_cast<const uint16_t*>(X);
+  a.Y = Y;
+  a.K = L.K; a.N = L.N; a.M = M;
+  a.tiles = (L.N + kL3bRows - 1) / kL3bRows;
+  a.nw = p.nw;
+  a.stages = p.stages; a.stage_bytes = p.stage_bytes; a.t_off = p.t_off;
+  a.xs_off = p.xs_off; a.red_off = p.red_off;
+  a.y_bf16 = ybf16 ? 1 : 0;
+  a.debug_drop = g_debug_drop;
+  const void* fn = p.kj == 2 ? (const void*)lut3_tmma_batch_kernel<2>
+                 : p.kj == 4 ? (const void*)lut3_tmma_batch_kernel<4> : (const void*)lut3_tmma_batch_kernel<8>;
+  const int block = (p.nw + 1) * 32;
+  occupancy_for(fn, block, p.smem);  // raises the kernel's dynamic shared-memory limit once
+  void* args[] = {&mi, &mt, &a};
+  return launch_kernel_ex(fn, dim3(p.grid), dim3(block), p.smem, st, g_pdl != 0, args,
+                          "LUT3 TMA batch GEMV launch");
+}
+
 static lbq_status run_lut3_gemm_tc(const void* X, int M, const void* image, const Layout& L, void* Y, bool ybf16,
                                    cudaStream_t st) {
   const uint8_t* img = static_cast<const uint8_t*>(image);
@@ -1357,6 +1429,10 @@ void lbq_debug_w4a8_tiled(int on) { g_w4a8_tiled = on ? 1 : 0; }
 // plan's choice).
 void lbq_debug_lut3_stages(int stages) { g_l3t_stages = (stages >= 1 && stages <= kL3tMaxStages) ? stages : 0; }
 
+// Test hook (not in the public header): 1 = LUT3 at M = 2..8 on the skinny
+// kernel instead of the TMA-fed batch kernel (0 = the library's choice).
+void lbq_debug_lut3_batch_off(int on) { g_l3b_off = on ? 1 : 0; }
+
 lbq_status lbq_set_option(int option, int value) {
   if (option == LBQ_OPT_PDL) {
     g_pdl = value ? 1 : 0;
@@ -1491,6 +1567,8 @@ lbq_status lbq_lut3_gemm(const void* X, int x_dtype, int M, int K, int N, const 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (lut3_tmma_ok(M, K, N, X, image) && !g_force_tc) return run_lut3_tmma(X, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);
   if (lut3_direct_ok(M, K) && !g_force_tc) return run_lut3_direct(X, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);
+  if (lut3_batch_ok(M, K, N, X, image) && !g_force_tc)
+    return run_lut3_batch(X, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);
   if (M <= 16 && !g_force_tc) return run_lut3_skinny(X, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, ws, ws_bytes, s);
   if (g_gemm_path == 0) return run_gemm_ts(X, true, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);
   return run_lut3_gemm_tc(X, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);

@@ -244,17 +244,18 @@ def test_lut3_m1_kernels(torch, lbq, K, N, path, stages):
     lbq.device_status()
 
 
-def test_lut3_m1_bounded_wait_runs_out_and_is_reported(torch, lbq):
-    """Failure detection without a GPU fault on the TMA-fed LUT3 kernel: with
+@pytest.mark.parametrize("M", [1, 4])  # the batch-1 kernel; the batch kernel (16-row units, batch on the columns)
+def test_lut3_m1_bounded_wait_runs_out_and_is_reported(torch, lbq, M):
+    """Failure detection without a GPU fault on the TMA-fed LUT3 kernels: with
     the producer's copies withheld (test hook) on a one-CTA launch, every
-    consumer wait gives up after a short spin limit, Y is not written, the
-    device flag reads LBQ_ERR_DEVICE and is cleared, and the next call passes
-    parity."""
+    consumer wait gives up after a short spin limit (the batch kernel's warps
+    keep their named-barrier sequence), Y is not written, the device flag reads
+    LBQ_ERR_DEVICE and is cleared, and the next call passes parity."""
     K, N = 1024, 8
     idx, cb, ex = _inputs(360, K, N)
     img = _image(torch, lbq, idx, cb, ex)
-    X = workloads.activations_host(361, 1, K, "bf16")
-    sentinel = torch.full((1, N), 7.0, dtype=torch.bfloat16, device="cuda")
+    X = workloads.activations_host(361, M, K, "bf16")
+    sentinel = torch.full((M, N), 7.0, dtype=torch.bfloat16, device="cuda")
     lbq.device_status()  # nothing pending
     lbq.lbq_debug_drop_copies(1)
     try:
@@ -264,7 +265,7 @@ def test_lut3_m1_bounded_wait_runs_out_and_is_reported(torch, lbq):
         assert err.value.status == 4  # LBQ_ERR_DEVICE
     finally:
         lbq.lbq_debug_drop_copies(0)
-    assert torch.equal(sentinel.cpu(), torch.full((1, N), 7.0, dtype=torch.bfloat16))  # Y untouched
+    assert torch.equal(sentinel.cpu(), torch.full((M, N), 7.0, dtype=torch.bfloat16))  # Y untouched
     lbq.device_status()  # the flag was cleared
     _check_gemm(torch, lbq, idx, cb, ex, img, X)
     lbq.device_status()
@@ -290,17 +291,19 @@ def test_tables_exact_at_the_exponent_range_ends(torch, lbq):
     lbq.device_status()
 
 
-def test_lut3_m1_pdl_graph(torch, lbq):
-    """The batch-1 LUT3 kernel with programmatic dependent launch inside a CUDA
-    graph: three back-to-back launches, each reading the previous one's output
-    as its activation (the weights stream before the wait, X only after it)."""
+@pytest.mark.parametrize("M", [1, 4])  # the batch-1 kernel; the batch kernel
+def test_lut3_m1_pdl_graph(torch, lbq, M):
+    """The TMA-fed LUT3 kernels with programmatic dependent launch inside a
+    CUDA graph: three back-to-back launches, each reading the previous one's
+    output as its activation (the weights stream before the wait, X only
+    after it)."""
     K = N = 4096
     idx, cb, ex = workloads.lut3_host(342, K, N)
     img = _image(torch, lbq, idx, cb, ex)
     deq = lut3.dequant(idx, cb, ex)
-    X0 = workloads.activations_host(343, 1, K, "bf16").cuda()
-    bufs = [X0] + [torch.empty((1, N), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
-    ws = lbq.workspace(2, 1, K, N, 0, "lut3")
+    X0 = workloads.activations_host(343, M, K, "bf16").cuda()
+    bufs = [X0] + [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    ws = lbq.workspace(2, M, K, N, 0, "lut3")
     lbq.lbq_set_option(lbq.LBQ_OPT_PDL, 1)
     try:
         s = torch.cuda.Stream()
@@ -324,3 +327,20 @@ def test_lut3_m1_pdl_graph(torch, lbq):
     # each stage against the oracle applied to the previous stage's GPU output
     for i in range(3):
         check_outputs(bufs[i + 1].cpu(), bufs[i].cpu(), deq)
+
+
+@pytest.mark.parametrize("off", [0, 1])  # the TMA-fed batch kernel; the skinny kernel
+def test_lut3_batch_full_size_sampled(torch, lbq, off):
+    """The 3-bit LUT workload at batch 4 (K=4096, N=14336), sampled channel
+    groups, on the batch kernel and on the skinny kernel."""
+    K, N, M = 4096, 14336, 4
+    idx, cb, ex = workloads.lut3_host(5, K, N)
+    img = _image(torch, lbq, idx, cb, ex)
+    X = workloads.activations_host(344, M, K, "bf16")
+    groups = np.unique(sample_columns(N, 96, seed=344) // 8)
+    lbq.lbq_debug_lut3_batch_off(off)
+    try:
+        _check_gemm(torch, lbq, idx, cb, ex, img, X, groups=groups)
+    finally:
+        lbq.lbq_debug_lut3_batch_off(0)
+    lbq.device_status()
