@@ -502,10 +502,19 @@ def _secondary_measurements(torch, lbq, workloads, device, peaks, quick):
     del W
     for M in (512, 2048, 8192):
         X = workloads.activations_device(4, M, K, "bf16", device)
-        ms = rotating_gemv_ms(torch, lbq, images, X, N, 128, "asym", lbq.workspace(1, M, K, N, 128, "asym"), reps=3)
+        ws = lbq.workspace(1, M, K, N, 128, "asym")
+        ms = rotating_gemv_ms(torch, lbq, images, X, N, 128, "asym", ws, reps=3)
         tf = 2.0 * M * K * N / ms / 1e9
         out[f"c4_gemm_m{M}"] = {"us": ms * 1e3, "TFLOPs": tf, "frac_bf16_peak": tf / tc_peak,
-                                "frac_bf16_sustained": tf / tc_sus, "weight_copies": len(images)}
+                                "frac_bf16_sustained": tf / tc_sus, "weight_copies": len(images),
+                                "stream_k": ws is not None}
+        if ws is not None:  # the same launches with whole tiles only, for comparison
+            lbq.lbq_debug_gemm_stream_k(0)
+            try:
+                ms_w = rotating_gemv_ms(torch, lbq, images, X, N, 128, "asym", ws, reps=3)
+            finally:
+                lbq.lbq_debug_gemm_stream_k(1)
+            out[f"c4_gemm_m{M}"]["TFLOPs_whole_tiles"] = 2.0 * M * K * N / ms_w / 1e9
         del X
     del images
     # c5: LUT3 K=4096 N=14336, M=1 (GB/s of the format's bytes) and M=2048 (TFLOP/s)
@@ -546,7 +555,14 @@ def _secondary_measurements(torch, lbq, workloads, device, peaks, quick):
         else:
             tf = 2.0 * M * K * N / ms / 1e9
             out[f"c5_lut3_m{M}"] = {"us": ms * 1e3, "TFLOPs": tf, "frac_bf16_peak": tf / tc_peak,
-                                    "frac_bf16_sustained": tf / tc_sus}
+                                    "frac_bf16_sustained": tf / tc_sus, "stream_k": ws is not None}
+            if ws is not None:  # whole tiles only, for comparison
+                lbq.lbq_debug_gemm_stream_k(0)
+                try:
+                    ms_w = rotating_lut3_ms(torch, lbq, images, X, N, ws, reps=3)
+                finally:
+                    lbq.lbq_debug_gemm_stream_k(1)
+                out[f"c5_lut3_m{M}"]["TFLOPs_whole_tiles"] = 2.0 * M * K * N / ms_w / 1e9
         del X
     del images
     # LUT3 x MXFP8 on the block-scaled FP8 tensor path, M=2048 (activations

@@ -81,6 +81,10 @@ _SIGS = {
     "lbq_debug_w4a8_tiled": ([_c_int], None),
     "lbq_debug_lut3_stages": ([_c_int], None),
     "lbq_debug_lut3_batch_off": ([_c_int], None),
+    "lbq_debug_gemm_stream_k": ([_c_int], None),
+    "lbq_debug_gemm_hold": ([_c_int], None),
+    "lbq_debug_gemm_schedule": ([_c_int, _c_int, _c_int, _c_int, _c_int, ctypes.POINTER(_c_int),
+                                 ctypes.POINTER(_c_int), ctypes.POINTER(_c_int), _c_int], _c_int),
     "lbq_moe_max_padded": ([_c_int, _c_int, _c_int, ctypes.POINTER(_c_int)], _c_int),
     "lbq_moe_align": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_int, _vp], _c_int),
     "lbq_moe_lut3_mx_gemm": ([_vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_int, _vp, _c_size, _c_int,
@@ -272,6 +276,25 @@ def lbq_debug_lut3_stages(stages):
 def lbq_debug_lut3_batch_off(on):
     """Test hook: LUT3 at M = 2..8 on the skinny kernel instead of the TMA-fed batch kernel."""
     _lib.lbq_debug_lut3_batch_off(1 if on else 0)
+
+
+def lbq_debug_gemm_stream_k(on):
+    """Test hook: prefill stream-K on (the library's choice) or off (whole tiles only)."""
+    _lib.lbq_debug_gemm_stream_k(1 if on else 0)
+
+
+def lbq_debug_gemm_hold(polls):
+    """Test hook: with polls > 0 the prefill's parked parts are never flagged and the wait gives up after polls."""
+    _lib.lbq_debug_gemm_hold(int(polls))
+
+
+def lbq_debug_gemm_schedule(M, K, N, stream_k, cta):
+    """Test hook: (grid, k_blocks, [(tile, kb0, kb1, part), ...]) of one prefill CTA, as the kernel walks it."""
+    grid, nkb = _c_int(0), _c_int(0)
+    n = _lib.lbq_debug_gemm_schedule(M, K, N, 1 if stream_k else 0, cta, ctypes.byref(grid), ctypes.byref(nkb), None, 0)
+    buf = (_c_int * max(4 * n, 4))()
+    _lib.lbq_debug_gemm_schedule(M, K, N, 1 if stream_k else 0, cta, ctypes.byref(grid), ctypes.byref(nkb), buf, n)
+    return grid.value, nkb.value, [tuple(buf[4 * i:4 * i + 4]) for i in range(n)]
 
 
 def lbq_moe_max_padded(num_pairs, num_experts, block):

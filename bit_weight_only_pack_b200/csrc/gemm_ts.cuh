@@ -27,6 +27,17 @@
 //               time (thread = one channel), round into a [32 tokens][128
 //               channels] shared-memory tile and write it with one TMA store
 //               (two tiles alternate).
+//
+// Schedule: the CTAs (at most one per SM) take whole tiles strided over the
+// grid; when the tiles leave a part-filled last wave, the last two waves'
+// tiles are instead cut into (tile, 128-k block) items shared out evenly
+// (stream-K), so every SM ends at about the same time. Each CTA's share is at
+// least one tile long, so a tile is cut at most once: its earlier part ends
+// the share of CTA c - 1 and its later part starts the share of CTA c. The
+// later part finishes first (it is its CTA's first item of the phase), parks
+// its FP32 sums in workspace slot c and raises flag c; the earlier part waits
+// for the flag (bounded), adds the parked sums to its own in a fixed order and
+// writes the tile, so results do not depend on timing.
 #pragma once
 
 #include "common.cuh"
@@ -74,7 +85,61 @@ struct GemmTsArgs {
   int n_tiles, m_tiles, k_blocks;  // channel tiles, token tiles, 64-k blocks
   int y_bf16;
   int tma_out;               // 1: Y written by TMA stores (N % 8 == 0, 16-byte aligned Y); 0: element stores
+  int dp_tiles;              // tiles taken whole, strided over the grid (all of them without stream-K)
+  long long sk_items;        // (tile, k-block) items of the tiles after them, shared out evenly (0: none)
+  float* partials;           // [grid][kTsBM tokens][kTsBN channels] parked sums of cut tiles
+  unsigned* flags;           // [grid] 1 while slot c holds a later part's sums; reset by the reader
+  uint32_t flag_polls;       // bound on the wait for a parked part (about 1 us per poll)
+  int debug_hold;            // test hook: later parts never raise their flag
 };
+
+// One work item: k-blocks [kb0, kb1) of a tile. part 0: the whole tile;
+// 1: a later part (parks its sums in slot blockIdx.x); 2: an earlier part
+// (adds the sums parked in slot blockIdx.x + 1, then writes the tile).
+struct TsItem {
+  int tile, kb0, kb1, part;
+};
+
+// The items of CTA `cta` of `grid` in order; every role of the CTA walks the
+// same sequence (the host runs it too, for the schedule's checks).
+struct TsSched {
+  int tile, dp_tiles, step, nkb;
+  long long pos, end;
+  __host__ __device__ TsSched(int dp, long long sk_items, int k_blocks, int cta, int grid)
+      : tile(cta), dp_tiles(dp), step(grid), nkb(k_blocks) {
+    pos = sk_items * cta / grid;
+    end = sk_items * (cta + 1) / grid;
+  }
+  __device__ explicit TsSched(const GemmTsArgs& a)
+      : TsSched(a.dp_tiles, a.sk_items, a.k_blocks, (int)blockIdx.x, (int)gridDim.x) {}
+  __host__ __device__ bool next(TsItem& w) {
+    if (tile < dp_tiles) {
+      w.tile = tile;
+      w.kb0 = 0;
+      w.kb1 = nkb;
+      w.part = 0;
+      tile += step;
+      return true;
+    }
+    if (pos >= end) return false;
+    const long long t = pos / nkb;
+    w.tile = dp_tiles + (int)t;
+    w.kb0 = (int)(pos - t * nkb);
+    w.kb1 = (int)(end - pos < (long long)(nkb - w.kb0) ? w.kb0 + (end - pos) : nkb);
+    w.part = w.kb0 > 0 ? 1 : (w.kb1 < nkb ? 2 : 0);
+    pos += w.kb1 - w.kb0;
+    return true;
+  }
+};
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
 
 template <bool BF16, bool ASYM, bool LUT>
 __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_constant__ CUtensorMap tx,
@@ -86,12 +151,11 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
   __shared__ __align__(8) uint64_t full_bar[kTsMaxStages], empty_bar[kTsMaxStages];
   __shared__ __align__(8) uint64_t a_full[kTsABufs], a_empty[kTsABufs], d_full, d_empty;
   __shared__ uint32_t tmem_base_sh;
+  __shared__ int sk_ok_sh;  // the epilogue's wait for a parked part succeeded
   uint8_t* ring = dsmem + ((1024u - (smem_u32(dsmem) & 1023u)) & 1023u);
   uint8_t* obuf = ring + (size_t)kTsStages * kTsStageBytes;  // two output tiles (LUT3)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int total_tiles = a.n_tiles * a.m_tiles;
-  const int nkb = a.k_blocks;
 
   if (tid == 0) {
     for (int i = 0; i < kTsStages; ++i) {
@@ -123,10 +187,12 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
       if (!LUT) tma_prefetch_desc(&tq);
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;  // token tiles inner: codes reused from L2
+      TsSched sch(a);
+      TsItem w;
+      while (ok && sch.next(w)) {
+        const int nt = w.tile / a.m_tiles, mt = w.tile - nt * a.m_tiles;  // token tiles inner: codes reused from L2
         const int rows = min(kTsBN, a.N - nt * kTsBN);
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const int s = it % kTsStages;
           if (it >= kTsStages && !mbar_wait(&empty_bar[s], ((it / kTsStages) & 1) ^ 1)) { ok = false; break; }
           uint8_t* st = ring + (size_t)s * kTsStageBytes;
@@ -161,10 +227,12 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
       const uint32_t idesc = umma_idesc_m128(BF16, kTsBM);
       int it = 0, t_iter = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t_iter) {
+      TsSched sch(a);
+      TsItem w;
+      for (; ok && sch.next(w); ++t_iter) {
         if (t_iter >= 1 && !mbar_wait(&d_empty, (t_iter - 1) & 1)) break;
         tc_fence_after();
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const int s = it % kTsStages, b = it % kTsABufs;
           if (!mbar_wait(&full_bar[s], (it / kTsStages) & 1)) { ok = false; break; }
           if (!mbar_wait(&a_full[b], (it / kTsABufs) & 1)) { ok = false; break; }
@@ -174,7 +242,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
           for (int kk = 0; kk < nkk; ++kk) {
             const uint64_t db = umma_desc_sw128(xb + (uint32_t)(kk >> 2) * kTsXBox) + (uint64_t)((kk & 3) * 2);
             umma_ts(tmem + kTsColD, tmem + kTsColA + (uint32_t)b * 64 + (uint32_t)kk * 8, db, idesc,
-                    (kb > 0 || kk > 0) ? 1u : 0u);
+                    (kb > w.kb0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&empty_bar[s]);
           umma_commit(&a_empty[b]);
@@ -191,10 +259,12 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
     int it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      const int nt = tile / a.m_tiles;
+    TsSched sch(a);
+    TsItem w;
+    while (sch.next(w)) {
+      const int nt = w.tile / a.m_tiles;
       const bool row_ok = nt * kTsBN + r < a.N;
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
+      for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
         const int s = it % kTsStages, b = it % kTsABufs;
         if (ok && !mbar_wait(&full_bar[s], (it / kTsStages) & 1)) ok = false;
         if (ok && it >= kTsABufs && !mbar_wait(&a_empty[b], ((it / kTsABufs) & 1) ^ 1)) ok = false;
@@ -209,8 +279,8 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
           if (ok && row_ok && kb * kTsBK + kc < a.K) {
             if (LUT) {
               const uint8_t* tile = st + kTsOffC + (ci >> 1) * (kTsBN * 24);  // LUT tile kb*2 + ci/2
-              const uint32_t* w = reinterpret_cast<const uint32_t*>(tile + r * 24 + (ci & 1) * 12);
-              const uint32_t wa = w[0], wb = w[1], wc = w[2];
+              const uint32_t* wp = reinterpret_cast<const uint32_t*>(tile + r * 24 + (ci & 1) * 12);
+              const uint32_t wa = wp[0], wb = wp[1], wc = wp[2];
               const uint4 tab = lds128(smem_u32(st + kTsOffM + (ci >> 1) * 256 + (r >> 3) * 16));
 #pragma unroll
               for (int t = 0; t < 4; ++t) {
@@ -263,10 +333,32 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
     if (issuer) tma_prefetch_desc(&ty);
     int t_iter = 0, ob = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++t_iter) {
-      const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;
+    TsSched sch(a);
+    TsItem w;
+    for (; sch.next(w); ++t_iter) {
+      const int nt = w.tile / a.m_tiles, mt = w.tile - nt * a.m_tiles;
       if (ok && !mbar_wait(&d_full, t_iter & 1)) ok = false;
       tc_fence_after();
+      // an earlier part: wait for the later part's sums in slot blockIdx.x + 1
+      const float* park_in = a.partials + (size_t)(blockIdx.x + 1) * (kTsBM * kTsBN) + r;
+      float* park_out = a.partials + (size_t)blockIdx.x * (kTsBM * kTsBN) + r;
+      if (w.part == 2) {
+        if (issuer) {
+          bool got = false;
+          if (ok) {
+            unsigned* f = a.flags + blockIdx.x + 1;
+            for (uint32_t i = 0; i < a.flag_polls && !got; ++i) {
+              got = ld_acquire_u32(f) != 0u;
+              if (!got) __nanosleep(1000);
+            }
+            if (got) atomicExch(f, 0u);  // the slot is free for the next call
+            else atomicOr(&g_device_error, kDevErrTimeout);
+          }
+          sk_ok_sh = got ? 1 : 0;
+        }
+        asm volatile("bar.sync 2, %0;" :: "r"(kTsEpWarps * 32) : "memory");
+        ok = ok && sk_ok_sh != 0;
+      }
 #pragma unroll 1
       for (int j = 0; j < kTsBM / 32; ++j) {
         uint32_t v[32];
@@ -275,6 +367,11 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = 0u;
+        }
+        if (w.part == 2 && ok) {  // own sums + parked sums, in that order
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            v[i] = __float_as_uint(__uint_as_float(v[i]) + __ldcg(park_in + (j * 32 + i) * kTsBN));
         }
         if (j == kTsBM / 32 - 1) {  // the accumulator is in registers: the MMAs may start the next tile
           tc_fence_before();
@@ -285,7 +382,12 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
         asm volatile("bar.sync 2, %0;" :: "r"(kTsEpWarps * 32) : "memory");
         uint8_t* ot = obuf + (size_t)ob * kTsOutBytes;
         const int m0 = mt * kTsBM + j * 32;
-        if (!a.tma_out) {  // rows of Y not 16-byte aligned: element stores
+        if (w.part == 1) {  // a later part: park the FP32 sums (all 256 tokens; rows past M hold zeros)
+          if (ok) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) __stcg(park_out + (j * 32 + i) * kTsBN, __uint_as_float(v[i]));
+          }
+        } else if (!a.tma_out) {  // rows of Y not 16-byte aligned: element stores
           const int n = nt * kTsBN + r;
           if (ok && n < a.N) {
 #pragma unroll
@@ -293,7 +395,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
               if (m0 + i < a.M) store_out(a.Y, (size_t)(m0 + i) * a.N + n, __uint_as_float(v[i]), a.y_bf16);
           }
         }
-        if (LUT && a.tma_out) {  // the staging tiles exist only in the LUT3 kernel's shared memory
+        if (LUT && a.tma_out && w.part != 1) {  // the staging tiles exist only in the LUT3 kernel's shared memory
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float f = __uint_as_float(v[i]);
@@ -304,11 +406,16 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
         }
         fence_proxy_async();  // the tile, to the TMA unit
         asm volatile("bar.sync 2, %0;" :: "r"(kTsEpWarps * 32) : "memory");
-        if (LUT && issuer && ok && a.tma_out && m0 < a.M) {
+        if (LUT && issuer && ok && a.tma_out && w.part != 1 && m0 < a.M) {
           tma_store_2d(&ty, ot, nt * kTsBN, m0);
           bulk_commit();
         }
         ob ^= 1;
+      }
+      if (w.part == 1) {  // the parked sums are visible GPU-wide before the flag
+        __threadfence();
+        asm volatile("bar.sync 2, %0;" :: "r"(kTsEpWarps * 32) : "memory");
+        if (issuer && ok && !a.debug_hold) st_release_u32(a.flags + blockIdx.x, 1u);
       }
     }
     if (LUT && issuer) bulk_wait<0>();  // every output store has landed

@@ -823,8 +823,37 @@ static int g_gemm_path = 0;
 typedef void (*TsKernel)(CUtensorMap, CUtensorMap, CUtensorMap, GemmTsArgs);
 
 // Prefill GEMM with the weights as the A operand in tensor memory (INT4 or LUT3).
+// Prefill schedule: whole tiles strided over a grid of at most one CTA per
+// SM; when that leaves a part-filled last wave whose idle share is worth more
+// than the cut tiles' exchange (idle k-blocks per SM >= 4), the last two waves'
+// tiles are shared out by k-block (stream-K) through a workspace of one flag
+// and one FP32 tile per CTA.
+static int g_ts_stream_k = 1;       // test hook: 0 = whole tiles only
+static int g_ts_hold = 0;           // test hook: later parts never raise their flag
+static uint32_t g_ts_polls = 0;     // test hook: bound on the flag wait (0 = about 4 s)
+struct TsPlan {
+  int grid, dp_tiles;
+  long long sk_items;
+  size_t flags_bytes, ws_bytes;  // 0 without stream-K
+};
+static TsPlan plan_gemm_ts(int M, int K, int N) {
+  const int T = ((N + kTsBN - 1) / kTsBN) * ((M + kTsBM - 1) / kTsBM);
+  const int nkb = (K + kTsBK - 1) / kTsBK;
+  TsPlan p{};
+  p.grid = std::min(T, num_sms());
+  p.dp_tiles = T;
+  const int rem = T % p.grid;
+  if (T > p.grid && rem != 0 && (long long)nkb * (p.grid - rem) >= 4LL * p.grid) {
+    p.dp_tiles = (T / p.grid - 1) * p.grid;
+    p.sk_items = (long long)(T - p.dp_tiles) * nkb;
+    p.flags_bytes = ((size_t)p.grid * 4 + 255) / 256 * 256;
+    p.ws_bytes = p.flags_bytes + (size_t)p.grid * kTsBM * kTsBN * 4;
+  }
+  return p;
+}
+
 static lbq_status run_gemm_ts(const void* X, bool xbf16, int M, const void* image, const Layout& L, void* Y,
-                              bool ybf16, cudaStream_t st) {
+                              bool ybf16, void* ws, size_t ws_bytes, cudaStream_t st) {
   const bool lut = L.mode == LBQ_MODE_LUT3, asym = L.mode == LBQ_MODE_ASYM;
   const uint8_t* img = static_cast<const uint8_t*>(image);
   CUtensorMap tx, tq, ty;
@@ -859,7 +888,17 @@ static lbq_status run_gemm_ts(const void* X, bool xbf16, int M, const void* imag
   else fn = asym ? gemm_ts_kernel<false, true, false> : gemm_ts_kernel<false, false, false>;
   const int smem = ts_smem(lut);
   occupancy_for((const void*)fn, kTsThreads, smem);
-  const int grid = std::min(a.n_tiles * a.m_tiles, num_sms());
+  const TsPlan p = plan_gemm_ts(M, L.K, L.N);
+  const int grid = p.grid;
+  a.dp_tiles = a.n_tiles * a.m_tiles;
+  a.flag_polls = g_ts_polls ? g_ts_polls : (1u << 22);
+  a.debug_hold = g_ts_hold;
+  if (p.ws_bytes && g_ts_stream_k && ws && ws_bytes >= p.ws_bytes) {  // without the workspace: whole tiles
+    a.dp_tiles = p.dp_tiles;
+    a.sk_items = p.sk_items;
+    a.flags = static_cast<unsigned*>(ws);
+    a.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + p.flags_bytes);
+  }
   void* args[] = {&tx, &tq, &ty, &a};
   return launch_kernel_ex((const void*)fn, dim3(grid), dim3(kTsThreads), smem, st, false, args,
                           "prefill GEMM launch");
@@ -1433,6 +1472,46 @@ void lbq_debug_lut3_stages(int stages) { g_l3t_stages = (stages >= 1 && stages <
 // kernel instead of the TMA-fed batch kernel (0 = the library's choice).
 void lbq_debug_lut3_batch_off(int on) { g_l3b_off = on ? 1 : 0; }
 
+// Test hook (not in the public header): prefill stream-K on (1, the library's
+// choice) or off (0: whole tiles, as without a workspace).
+void lbq_debug_gemm_stream_k(int on) { g_ts_stream_k = on ? 1 : 0; }
+
+// Test hook (not in the public header): with polls > 0 the prefill's later
+// parts never raise their flag and each earlier part gives up after `polls`
+// waits of about 1 us: it writes nothing and raises the device flag that
+// lbq_device_status() reports. polls = 0 restores the library's behaviour.
+void lbq_debug_gemm_hold(int polls) {
+  g_ts_hold = polls > 0 ? 1 : 0;
+  g_ts_polls = polls > 0 ? (uint32_t)polls : 0u;
+}
+
+// Test hook (not in the public header): the prefill schedule of CTA `cta` for
+// this shape, as the kernel walks it. Writes up to `max_items` items as
+// (tile, kb0, kb1, part) int quadruples to `items` (host) and returns the
+// item count; *grid receives the grid size, *k_blocks the 128-k blocks per tile.
+int lbq_debug_gemm_schedule(int M, int K, int N, int stream_k, int cta, int* grid, int* k_blocks, int* items,
+                            int max_items) {
+  const TsPlan p = plan_gemm_ts(M, K, N);
+  const int nkb = (K + kTsBK - 1) / kTsBK;
+  *grid = p.grid;
+  *k_blocks = nkb;
+  const bool sk = stream_k && p.ws_bytes;
+  TsSched sch(sk ? p.dp_tiles : ((N + kTsBN - 1) / kTsBN) * ((M + kTsBM - 1) / kTsBM), sk ? p.sk_items : 0, nkb,
+              cta, p.grid);
+  TsItem w;
+  int n = 0;
+  while (sch.next(w)) {
+    if (n < max_items) {
+      items[4 * n] = w.tile;
+      items[4 * n + 1] = w.kb0;
+      items[4 * n + 2] = w.kb1;
+      items[4 * n + 3] = w.part;
+    }
+    ++n;
+  }
+  return n;
+}
+
 lbq_status lbq_set_option(int option, int value) {
   if (option == LBQ_OPT_PDL) {
     g_pdl = value ? 1 : 0;
@@ -1501,7 +1580,11 @@ lbq_status lbq_workspace_size(int op, int M, int K, int N, int group, int mode, 
     lbq_status st = check_int4_shape(K, N, group, mode);
     if (st != LBQ_OK) return st;
     if (M <= 0) return fail(LBQ_ERR_INVALID_ARG, "M must be positive");
-    if (op == 1 && (M > 16 || g_force_tc)) return LBQ_OK;  // the prefill GEMM needs no workspace
+    if (op == 1 && g_force_tc) return LBQ_OK;  // the alternative tensor-core GEMM needs no workspace
+    if (op == 1 && M > 16) {  // the prefill GEMM: stream-K's flags and parked tiles, where it cuts tiles
+      *bytes = plan_gemm_ts(M, K, N).ws_bytes;
+      return LBQ_OK;
+    }
     if (M <= 16) {
       // the plan may depend on the activation dtype through a kernel's
       // occupancy; take the larger of the two
@@ -1515,6 +1598,7 @@ lbq_status lbq_workspace_size(int op, int M, int K, int N, int group, int mode, 
     if (st != LBQ_OK) return st;
     if (M <= 0) return fail(LBQ_ERR_INVALID_ARG, "M must be positive");
     if (M <= 16 && !g_force_tc && !lut3_direct_ok(M, K)) *bytes = skinny_workspace_bytes(plan_lut3(K, N, M), M);
+    if (M > 16 && !g_force_tc) *bytes = plan_gemm_ts(M, K, N).ws_bytes;
     return LBQ_OK;
   }
   return fail(LBQ_ERR_INVALID_ARG, "op %d not in {0, 1, 2}", op);
@@ -1552,7 +1636,7 @@ lbq_status lbq_gemm(const void* X, int x_dtype, int M, int K, int N, int group, 
   if ((st = check_compute_args(X, x_dtype, M, image, Y, y_dtype)) != LBQ_OK) return st;
   if (g_gemm_path == 0)
     return run_gemm_ts(X, x_dtype == LBQ_DTYPE_BF16, M, image, make_layout(K, N, group, mode), Y,
-                       y_dtype == LBQ_DTYPE_BF16, static_cast<cudaStream_t>(stream));
+                       y_dtype == LBQ_DTYPE_BF16, ws, ws_bytes, static_cast<cudaStream_t>(stream));
   return run_gemm_tc(X, x_dtype == LBQ_DTYPE_BF16, M, image, make_layout(K, N, group, mode), Y,
                      y_dtype == LBQ_DTYPE_BF16, static_cast<cudaStream_t>(stream));
 }
@@ -1570,7 +1654,7 @@ lbq_status lbq_lut3_gemm(const void* X, int x_dtype, int M, int K, int N, const 
   if (lut3_batch_ok(M, K, N, X, image) && !g_force_tc)
     return run_lut3_batch(X, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);
   if (M <= 16 && !g_force_tc) return run_lut3_skinny(X, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, ws, ws_bytes, s);
-  if (g_gemm_path == 0) return run_gemm_ts(X, true, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);
+  if (g_gemm_path == 0) return run_gemm_ts(X, true, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, ws, ws_bytes, s);
   return run_lut3_gemm_tc(X, M, image, L, Y, y_dtype == LBQ_DTYPE_BF16, s);
 }
 

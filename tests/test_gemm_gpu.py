@@ -91,3 +91,69 @@ def test_prefill_full_size_sampled(torch, lbq, M):
     Y = lbq.gemm(X.cuda(), img, N, 128, "asym", y_dtype="bf16")
     torch.cuda.synchronize()
     check_outputs(Y.cpu(), X, ref["deq"], cols)
+
+
+SK_SHAPES = [
+    # more tiles than SMs with a part-filled last wave: the prefill cuts tiles (stream-K)
+    (300, 1024, 10000, 128, "asym", "bf16"),   # 158 tiles, ragged M and N, 8 k-blocks
+    (520, 2048, 9000, 64, "sym", "f16"),       # 213 tiles, 16 k-blocks
+    (700, 1056, 5000, 32, "asym", "bf16"),     # 120 tiles (no cut) ... and K ending inside a block
+    (1100, 1056, 4100, 32, "sym", "bf16"),     # 165 tiles, 9 k-blocks (the last part-filled), N % 8 != 0
+]
+
+
+@pytest.mark.parametrize("M,K,N,group,mode,xdt", SK_SHAPES)
+def test_gemm_stream_k_parity(torch, lbq, M, K, N, group, mode, xdt):
+    """With the workspace the last waves' tiles are cut by k-block; both
+    schedules match the oracle, repeated calls on one workspace are identical
+    and every flag is back at zero after each call."""
+    W = workloads.weights_host(800 + K + N, K, N)
+    ref = oracle_int4(W, group, mode)
+    img = lbq.pack(torch.from_numpy(W).cuda(), group, mode)
+    X = workloads.activations_host(800 + M, M, K, xdt).cuda()
+    ws = lbq.workspace(1, M, K, N, group, mode)
+    grid = lbq.lbq_debug_gemm_schedule(M, K, N, 1, 0)[0]
+    cut = ws is not None
+    assert cut == ((M, N) != (700, 5000))
+    Ys = [lbq.gemm(X, img, N, group, mode, ws=ws) for _ in range(3)]
+    torch.cuda.synchronize()
+    lbq.device_status()
+    assert all(torch.equal(Ys[0], Y) for Y in Ys[1:])
+    if cut:
+        assert int(ws[:grid * 4].view(torch.int32).abs().sum()) == 0
+    check_outputs(Ys[0].cpu(), X.cpu(), ref["deq"])
+    lbq.lbq_debug_gemm_stream_k(0)
+    try:
+        Y0 = lbq.gemm(X, img, N, group, mode, ws=ws)
+        torch.cuda.synchronize()
+    finally:
+        lbq.lbq_debug_gemm_stream_k(1)
+    check_outputs(Y0.cpu(), X.cpu(), ref["deq"])
+
+
+def test_gemm_stream_k_wait_runs_out_and_is_reported(torch, lbq):
+    """Failure detection without a GPU fault: with the later parts' flags
+    withheld (test hook), every earlier part's wait gives up after a short
+    bound, its tile is not written, the device flag is reported as
+    LBQ_ERR_DEVICE, and the next call on the same workspace passes parity."""
+    M, K, N, group, mode = 300, 1024, 10000, 128, "asym"
+    W = workloads.weights_host(810, K, N)
+    ref = oracle_int4(W, group, mode)
+    img = lbq.pack(torch.from_numpy(W).cuda(), group, mode)
+    X = workloads.activations_host(811, M, K, "bf16").cuda()
+    ws = lbq.workspace(1, M, K, N, group, mode)
+    assert ws is not None
+    lbq.device_status()  # nothing pending
+    lbq.lbq_debug_gemm_hold(2000)
+    try:
+        lbq.gemm(X, img, N, group, mode, ws=ws)
+        with pytest.raises(lbq.LbqError) as err:
+            lbq.device_status()
+        assert err.value.status == 4  # LBQ_ERR_DEVICE
+    finally:
+        lbq.lbq_debug_gemm_hold(0)
+    lbq.device_status()  # the flag was cleared by the report
+    Y = lbq.gemm(X, img, N, group, mode, ws=ws)
+    torch.cuda.synchronize()
+    lbq.device_status()
+    check_outputs(Y.cpu(), X.cpu(), ref["deq"])

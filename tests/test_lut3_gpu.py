@@ -153,6 +153,25 @@ def test_lut3_tcgen05_kernel_at_decode_batch(torch, lbq, M):
         lbq.lbq_debug_force_tc(0)
 
 
+@pytest.mark.parametrize("M,K,N", [(300, 1024, 10000), (1100, 1024, 4104)])
+def test_lut3_gemm_stream_k(torch, lbq, M, K, N):
+    """The LUT3 prefill with cut tiles (158 / 165 tiles on the SMs): against
+    the oracle, identical over repeated calls on one workspace, flags reset."""
+    idx, cb, ex = _inputs(98 + K + N, K, N)
+    img = _image(torch, lbq, idx, cb, ex)
+    X = workloads.activations_host(98 + M, M, K, "bf16").cuda()
+    ws = lbq.workspace(2, M, K, N, 0, "lut3")
+    assert ws is not None
+    grid = lbq.lbq_debug_gemm_schedule(M, K, N, 1, 0)[0]
+    Ys = [lbq.lut3_gemm(X, img, N, ws=ws) for _ in range(3)]
+    torch.cuda.synchronize()
+    lbq.device_status()
+    assert all(torch.equal(Ys[0], Y) for Y in Ys[1:])
+    assert int(ws[:grid * 4].view(torch.int32).abs().sum()) == 0
+    ch = np.arange(N)
+    check_outputs(Ys[0].cpu(), X.cpu(), lut3.dequant(idx, cb, ex), ch)
+
+
 def test_lut3_repeat_calls_identical(torch, lbq):
     """Three calls on one workspace (shared tiles, so the counters must reset)."""
     K, N, M = 14336, 264, 4
