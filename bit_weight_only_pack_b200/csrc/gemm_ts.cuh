@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
         const int rows = min(kTsBN, a.N - nt * kTsBN);
         for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const int s = it % kTsStages;
-          if (it >= kTsStages && !mbar_wait(&empty_bar[s], ((it / kTsStages) & 1) ^ 1)) { ok = false; break; }
+          if (it >= kTsStages && !mbar_wait_sleep(&empty_bar[s], ((it / kTsStages) & 1) ^ 1)) { ok = false; break; }
           uint8_t* st = ring + (size_t)s * kTsStageBytes;
           const int nxb = min(2, (a.K - kb * kTsBK + 63) / 64);  // 64-k activation boxes inside K
           if (LUT) {
@@ -230,12 +230,12 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
       TsSched sch(a);
       TsItem w;
       for (; ok && sch.next(w); ++t_iter) {
-        if (t_iter >= 1 && !mbar_wait(&d_empty, (t_iter - 1) & 1)) break;
+        if (t_iter >= 1 && !mbar_wait_sleep(&d_empty, (t_iter - 1) & 1)) break;
         tc_fence_after();
         for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const int s = it % kTsStages, b = it % kTsABufs;
-          if (!mbar_wait(&full_bar[s], (it / kTsStages) & 1)) { ok = false; break; }
-          if (!mbar_wait(&a_full[b], (it / kTsABufs) & 1)) { ok = false; break; }
+          if (!mbar_wait_sleep(&full_bar[s], (it / kTsStages) & 1)) { ok = false; break; }
+          if (!mbar_wait_sleep(&a_full[b], (it / kTsABufs) & 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t xb = smem_u32(ring + (size_t)s * kTsStageBytes);
           const int nkk = min(kTsBK, a.K - kb * kTsBK + 15) / 16;  // 16-k slices inside K (K % 32 == 0)
@@ -266,8 +266,8 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
       const bool row_ok = nt * kTsBN + r < a.N;
       for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
         const int s = it % kTsStages, b = it % kTsABufs;
-        if (ok && !mbar_wait(&full_bar[s], (it / kTsStages) & 1)) ok = false;
-        if (ok && it >= kTsABufs && !mbar_wait(&a_empty[b], ((it / kTsABufs) & 1) ^ 1)) ok = false;
+        if (ok && !mbar_wait_sleep(&full_bar[s], (it / kTsStages) & 1)) ok = false;
+        if (ok && it >= kTsABufs && !mbar_wait_sleep(&a_empty[b], ((it / kTsABufs) & 1) ^ 1)) ok = false;
         tc_fence_after();
         const uint8_t* st = ring + (size_t)s * kTsStageBytes;
         // this thread's chunks of the block (32 k, 16 pairs each)
@@ -324,8 +324,11 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
     }
   } else {
     // ------------------------------------------------------------------ epilogue
-    // every epilogue warp runs every chunk and both named barriers of it, also
-    // after a timed-out wait (then it loads and stores nothing)
+    // every epilogue warp runs every chunk and (with TMA stores) both named
+    // barriers of it, also after a timed-out wait (then it loads and stores
+    // nothing). Element stores take no barrier: each warp reads its own TMEM
+    // lanes and writes its own channels, and the accumulator is released as
+    // soon as the last chunk is in registers.
     const int q = warp & 3;
     const int r = 32 * q + lane;  // channel within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
@@ -337,7 +340,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
     TsItem w;
     for (; sch.next(w); ++t_iter) {
       const int nt = w.tile / a.m_tiles, mt = w.tile - nt * a.m_tiles;
-      if (ok && !mbar_wait(&d_full, t_iter & 1)) ok = false;
+      if (ok && !mbar_wait_sleep(&d_full, t_iter & 1)) ok = false;
       tc_fence_after();
       // an earlier part: wait for the later part's sums in slot blockIdx.x + 1
       const float* park_in = a.partials + (size_t)(blockIdx.x + 1) * (kTsBM * kTsBN) + r;
@@ -359,58 +362,73 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
         asm volatile("bar.sync 2, %0;" :: "r"(kTsEpWarps * 32) : "memory");
         ok = ok && sk_ok_sh != 0;
       }
+      // two 32-token chunks per TMEM round trip (a load's wait costs about as
+      // much as the chunk's stores)
 #pragma unroll 1
-      for (int j = 0; j < kTsBM / 32; ++j) {
-        uint32_t v[32];
+      for (int jp = 0; jp < kTsBM / 64; ++jp) {
+        uint32_t vv[2][32];
         if (ok) {
-          tmem_ld32(lane_base + kTsColD + (uint32_t)(j * 32), v);
+          tmem_ld32_nowait(lane_base + kTsColD + (uint32_t)(jp * 64), vv[0]);
+          tmem_ld32_nowait(lane_base + kTsColD + (uint32_t)(jp * 64 + 32), vv[1]);
+          tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0u;
+          for (int i = 0; i < 32; ++i) vv[0][i] = vv[1][i] = 0u;
         }
-        if (w.part == 2 && ok) {  // own sums + parked sums, in that order
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            v[i] = __float_as_uint(__uint_as_float(v[i]) + __ldcg(park_in + (j * 32 + i) * kTsBN));
-        }
-        if (j == kTsBM / 32 - 1) {  // the accumulator is in registers: the MMAs may start the next tile
+        if (jp == kTsBM / 64 - 1) {  // the accumulator is in registers: the MMAs may start the next tile
           tc_fence_before();
           __syncwarp();
           if (lane == 0 && ok) mbar_arrive(&d_empty);
         }
-        if (LUT && issuer) bulk_wait_read<1>();  // the tile written two chunks ago has been read
-        asm volatile("bar.sync 2, %0;" :: "r"(kTsEpWarps * 32) : "memory");
-        uint8_t* ot = obuf + (size_t)ob * kTsOutBytes;
-        const int m0 = mt * kTsBM + j * 32;
-        if (w.part == 1) {  // a later part: park the FP32 sums (all 256 tokens; rows past M hold zeros)
-          if (ok) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) __stcg(park_out + (j * 32 + i) * kTsBN, __uint_as_float(v[i]));
-          }
-        } else if (!a.tma_out) {  // rows of Y not 16-byte aligned: element stores
-          const int n = nt * kTsBN + r;
-          if (ok && n < a.N) {
+        for (int h = 0; h < 2; ++h) {
+          const int j = 2 * jp + h;
+          uint32_t(&v)[32] = vv[h];
+          if (w.part == 2 && ok) {  // own sums + parked sums, in that order
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              if (m0 + i < a.M) store_out(a.Y, (size_t)(m0 + i) * a.N + n, __uint_as_float(v[i]), a.y_bf16);
+              v[i] = __float_as_uint(__uint_as_float(v[i]) + __ldcg(park_in + (j * 32 + i) * kTsBN));
           }
-        }
-        if (LUT && a.tma_out && w.part != 1) {  // the staging tiles exist only in the LUT3 kernel's shared memory
+          // the shared staging tile and its barriers serve the TMA stores only:
+          // element stores and parked sums go out per warp, unordered
+          if (LUT && a.tma_out) {
+            if (issuer) bulk_wait_read<1>();  // the tile written two chunks ago has been read
+            asm volatile("bar.sync 2, %0;" :: "r"(kTsEpWarps * 32) : "memory");
+          }
+          uint8_t* ot = obuf + (size_t)ob * kTsOutBytes;
+          const int m0 = mt * kTsBM + j * 32;
+          if (w.part == 1) {  // a later part: park the FP32 sums (all 256 tokens; rows past M hold zeros)
+            if (ok) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float f = __uint_as_float(v[i]);
-            const uint16_t h =
-                a.y_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(f)) : __half_as_ushort(__float2half_rn(f));
-            *reinterpret_cast<uint16_t*>(ot + (i * kTsBN + r) * 2) = h;
+              for (int i = 0; i < 32; ++i) __stcg(park_out + (j * 32 + i) * kTsBN, __uint_as_float(v[i]));
+            }
+          } else if (!a.tma_out) {  // rows of Y not 16-byte aligned: element stores
+            const int n = nt * kTsBN + r;
+            if (ok && n < a.N) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (m0 + i < a.M) store_out(a.Y, (size_t)(m0 + i) * a.N + n, __uint_as_float(v[i]), a.y_bf16);
+            }
+          }
+          if (LUT && a.tma_out) {  // the staging tiles exist only in the LUT3 kernel's shared memory
+            if (w.part != 1) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float f = __uint_as_float(v[i]);
+                const uint16_t hb =
+                    a.y_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(f)) : __half_as_ushort(__float2half_rn(f));
+                *reinterpret_cast<uint16_t*>(ot + (i * kTsBN + r) * 2) = hb;
+              }
+            }
+            fence_proxy_async();  // the tile, to the TMA unit
+            asm volatile("bar.sync 2, %0;" :: "r"(kTsEpWarps * 32) : "memory");
+            if (issuer && ok && w.part != 1 && m0 < a.M) {
+              tma_store_2d(&ty, ot, nt * kTsBN, m0);
+              bulk_commit();
+            }
+            ob ^= 1;
           }
         }
-        fence_proxy_async();  // the tile, to the TMA unit
-        asm volatile("bar.sync 2, %0;" :: "r"(kTsEpWarps * 32) : "memory");
-        if (LUT && issuer && ok && a.tma_out && w.part != 1 && m0 < a.M) {
-          tma_store_2d(&ty, ot, nt * kTsBN, m0);
-          bulk_commit();
-        }
-        ob ^= 1;
       }
       if (w.part == 1) {  // the parked sums are visible GPU-wide before the flag
         __threadfence();

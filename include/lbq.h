@@ -180,7 +180,15 @@ lbq_status lbq_gemv_grouped(const lbq_gemv_item* items, int count, int K, int gr
  * formed exactly, the product with the scale rounded once) straight into
  * tensor memory and multiplied on the tcgen05 tensor cores with FP32
  * accumulation ("Low Bit Metal Kernels": dequantise just before the
- * multiply). Needs no workspace for M > 16. Asynchronous.
+ * multiply). For M > 16 the workspace is optional: where the 128-channel x
+ * 256-token output tiles leave the SMs' last wave part-filled,
+ * lbq_workspace_size(1, ...) is non-zero, and with a workspace of that size
+ * the last two waves' tiles are cut along K between neighbouring CTAs (one
+ * FP32 tile and one flag per CTA; the two parts are added in a fixed order,
+ * so results do not depend on timing). With ws null or smaller every tile is
+ * computed whole. A part that waits about 4 s for its partner gives up and
+ * raises LBQ_ERR_DEVICE (lbq_device_status); zero-fill the workspace again
+ * after that. Asynchronous.
  */
 lbq_status lbq_gemm(const void* X, int x_dtype, int M, int K, int N, int group, int mode,
                     const void* image, void* Y, int y_dtype, void* ws, size_t ws_bytes,
@@ -190,6 +198,9 @@ lbq_status lbq_gemm(const void* X, int x_dtype, int M, int K, int N, int group, 
  * GEMV / GEMM on LUT3 weights (image from lbq_pack_lut3), any M >= 1.
  * X must be BF16. y[m][n] = sum_k x[m][k] * w[k][n] with w the decoded
  * LUT3 value (exact in BF16 for the exponents the format's workloads use).
+ * ws: lbq_workspace_size(2, ...) bytes, zero-filled; required by the
+ * skinny kernel's split-K (M <= 16), optional for M > 16 (the prefill's
+ * cut tiles, as lbq_gemm).
  */
 lbq_status lbq_lut3_gemm(const void* X, int x_dtype, int M, int K, int N,
                          const void* image, void* Y, int y_dtype, void* ws, size_t ws_bytes,
