@@ -23,10 +23,12 @@
 //               exact packed subtract, one packed multiply); LUT3: the exact
 //               BF16 weight from the tile's table (byte permutes). 16 pairs
 //               per tcgen05.st. Four A buffers of 64 columns.
-//   warps 10-13 epilogue: tcgen05.ld the finished accumulator 32 tokens at a
-//               time (thread = one channel), round into a [32 tokens][128
-//               channels] shared-memory tile and write it with one TMA store
-//               (two tiles alternate).
+//   warps 10-17 epilogue, two per TMEM lane quarter, each taking half of the
+//               tokens: tcgen05.ld the finished accumulator 64 tokens per
+//               wait (thread = one channel) and store the elements, or (LUT3)
+//               round into a [32 tokens][128 channels] shared-memory tile per
+//               warp group and write it with one TMA store (two tiles
+//               alternate per group).
 //
 // Schedule: the CTAs (at most one per SM) take whole tiles strided over the
 // grid; when the tiles leave a part-filled last wave, the last two waves'
@@ -60,7 +62,10 @@ constexpr int kTsBK = 128;                 // k per block: 8 MMAs per pair of ba
 __host__ __device__ constexpr int ts_stages(bool lut) { return lut ? 2 : 3; }
 constexpr int kTsMaxStages = 3;
 constexpr int kTsABufs = 4;                // A (weights) buffers in tensor memory, 64 columns each
-constexpr int kTsConvWarps = 8, kTsEpWarps = 4;
+constexpr int kTsConvWarps = 8, kTsEpWarps = 8;
+// the epilogue warps of one TMEM lane quarter split the tile's tokens
+constexpr int kTsEpGroups = kTsEpWarps / 4;
+constexpr int kTsEpPairs = kTsBM / 64 / kTsEpGroups;  // 64-token pairs of chunks per epilogue warp
 // 32-k chunks per converter thread per block: the block's kTsBK / 32 chunks are
 // split over the kTsConvWarps / 4 warps that share a TMEM lane quarter
 constexpr int kTsChunksPerConv = (kTsBK / 32) / (kTsConvWarps / 4);
@@ -73,7 +78,10 @@ constexpr int kTsMBytes = 2048;                     // scales + zero points (INT
 constexpr int kTsOffC = kTsXBytes, kTsOffM = kTsOffC + kTsCBytes;
 constexpr int kTsStageBytes = kTsOffM + kTsMBytes;  // 74 KB, a multiple of 1024
 constexpr int kTsOutBytes = 32 * kTsBN * 2;          // one [32 tokens][128 channels] output tile
-__host__ __device__ constexpr int ts_smem(bool lut) { return ts_stages(lut) * kTsStageBytes + (lut ? 2 * kTsOutBytes : 0) + 1024; }
+// LUT3: two staging tiles per epilogue group
+__host__ __device__ constexpr int ts_smem(bool lut) {
+  return ts_stages(lut) * kTsStageBytes + (lut ? 2 * kTsEpGroups * kTsOutBytes : 0) + 1024;
+}
 constexpr uint32_t kTsColA = 0, kTsColD = 256;
 static_assert(kTsStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
 
@@ -153,7 +161,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
   __shared__ uint32_t tmem_base_sh;
   __shared__ int sk_ok_sh;  // the epilogue's wait for a parked part succeeded
   uint8_t* ring = dsmem + ((1024u - (smem_u32(dsmem) & 1023u)) & 1023u);
-  uint8_t* obuf = ring + (size_t)kTsStages * kTsStageBytes;  // two output tiles (LUT3)
+  uint8_t* obuf = ring + (size_t)kTsStages * kTsStageBytes;  // two output tiles per epilogue group (LUT3)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -332,7 +340,10 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
     const int q = warp & 3;
     const int r = 32 * q + lane;  // channel within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-    const bool issuer = warp == 2 + kTsConvWarps && lane == 0;
+    const int eg = (warp - 2 - kTsConvWarps) >> 2;  // epilogue group: tokens [64 kTsEpPairs eg, +64 kTsEpPairs)
+    const bool lead = warp == 2 + kTsConvWarps && lane == 0;  // flags of cut tiles
+    const bool issuer = ((warp - 2 - kTsConvWarps) & 3) == 0 && lane == 0;  // the group's TMA stores
+    const uint32_t gbar = 2u + (uint32_t)eg;  // the group's named barrier (barrier 1: all epilogue warps)
     if (issuer) tma_prefetch_desc(&ty);
     int t_iter = 0, ob = 0;
     bool ok = true;
@@ -346,7 +357,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
       const float* park_in = a.partials + (size_t)(blockIdx.x + 1) * (kTsBM * kTsBN) + r;
       float* park_out = a.partials + (size_t)blockIdx.x * (kTsBM * kTsBN) + r;
       if (w.part == 2) {
-        if (issuer) {
+        if (lead) {
           bool got = false;
           if (ok) {
             unsigned* f = a.flags + blockIdx.x + 1;
@@ -359,13 +370,13 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
           }
           sk_ok_sh = got ? 1 : 0;
         }
-        asm volatile("bar.sync 2, %0;" :: "r"(kTsEpWarps * 32) : "memory");
+        asm volatile("bar.sync 1, %0;" :: "r"(kTsEpWarps * 32) : "memory");
         ok = ok && sk_ok_sh != 0;
       }
       // two 32-token chunks per TMEM round trip (a load's wait costs about as
       // much as the chunk's stores)
 #pragma unroll 1
-      for (int jp = 0; jp < kTsBM / 64; ++jp) {
+      for (int jp = eg * kTsEpPairs; jp < (eg + 1) * kTsEpPairs; ++jp) {
         uint32_t vv[2][32];
         if (ok) {
           tmem_ld32_nowait(lane_base + kTsColD + (uint32_t)(jp * 64), vv[0]);
@@ -375,7 +386,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
 #pragma unroll
           for (int i = 0; i < 32; ++i) vv[0][i] = vv[1][i] = 0u;
         }
-        if (jp == kTsBM / 64 - 1) {  // the accumulator is in registers: the MMAs may start the next tile
+        if (jp == (eg + 1) * kTsEpPairs - 1) {  // this warp's part of the accumulator is in registers
           tc_fence_before();
           __syncwarp();
           if (lane == 0 && ok) mbar_arrive(&d_empty);
@@ -392,10 +403,10 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
           // the shared staging tile and its barriers serve the TMA stores only:
           // element stores and parked sums go out per warp, unordered
           if (LUT && a.tma_out) {
-            if (issuer) bulk_wait_read<1>();  // the tile written two chunks ago has been read
-            asm volatile("bar.sync 2, %0;" :: "r"(kTsEpWarps * 32) : "memory");
+            if (issuer) bulk_wait_read<1>();  // the group's tile written two chunks ago has been read
+            asm volatile("bar.sync %0, 128;" :: "r"(gbar) : "memory");
           }
-          uint8_t* ot = obuf + (size_t)ob * kTsOutBytes;
+          uint8_t* ot = obuf + (size_t)(2 * eg + ob) * kTsOutBytes;
           const int m0 = mt * kTsBM + j * 32;
           if (w.part == 1) {  // a later part: park the FP32 sums (all 256 tokens; rows past M hold zeros)
             if (ok) {
@@ -421,7 +432,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
               }
             }
             fence_proxy_async();  // the tile, to the TMA unit
-            asm volatile("bar.sync 2, %0;" :: "r"(kTsEpWarps * 32) : "memory");
+            asm volatile("bar.sync %0, 128;" :: "r"(gbar) : "memory");
             if (issuer && ok && w.part != 1 && m0 < a.M) {
               tma_store_2d(&ty, ot, nt * kTsBN, m0);
               bulk_commit();
@@ -432,8 +443,8 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
       }
       if (w.part == 1) {  // the parked sums are visible GPU-wide before the flag
         __threadfence();
-        asm volatile("bar.sync 2, %0;" :: "r"(kTsEpWarps * 32) : "memory");
-        if (issuer && ok && !a.debug_hold) st_release_u32(a.flags + blockIdx.x, 1u);
+        asm volatile("bar.sync 1, %0;" :: "r"(kTsEpWarps * 32) : "memory");
+        if (lead && ok && !a.debug_hold) st_release_u32(a.flags + blockIdx.x, 1u);
       }
     }
     if (LUT && issuer) bulk_wait<0>();  // every output store has landed
