@@ -25,10 +25,11 @@
 //               per tcgen05.st. Four A buffers of 64 columns.
 //   warps 10-17 epilogue, two per TMEM lane quarter, each taking half of the
 //               tokens: tcgen05.ld the finished accumulator 64 tokens per
-//               wait (thread = one channel) and store the elements, or (LUT3)
-//               round into a [32 tokens][128 channels] shared-memory tile per
-//               warp group and write it with one TMA store (two tiles
-//               alternate per group).
+//               wait (thread = one channel), round and store the elements
+//               (a warp's store of one token row is 64 contiguous bytes).
+//               The accumulator is held only while it drains, so the fewer
+//               the round trips, the less of each tile the converters (which
+//               run at most three k-blocks ahead of the stalled MMAs) lose.
 //
 // Schedule: the CTAs (at most one per SM) take whole tiles strided over the
 // grid; when the tiles leave a part-filled last wave, the last two waves'
@@ -54,13 +55,11 @@ namespace lbq {
 constexpr int kTsBN = 128;                 // channels per tile (TMEM lanes)
 constexpr int kTsBM = 256;                 // tokens per tile (MMA N)
 constexpr int kTsBK = 128;                 // k per block: 8 MMAs per pair of barrier waits
-// TMA ring depth: INT4 keeps three 74 KB stages and stores Y element by
-// element; LUT3 trades one stage for two 8 KB output tiles written by TMA
-// stores (measured on B200, K=4096 N=14336 M=2048: INT4 811 TFLOP/s with three
-// stages against 812 with two plus TMA stores, and 779 against 817 at M=8192;
-// LUT3 864 -> 907 TFLOP/s with the TMA stores)
-__host__ __device__ constexpr int ts_stages(bool lut) { return lut ? 2 : 3; }
-constexpr int kTsMaxStages = 3;
+// TMA ring depth: three 74 KB stages, Y stored element by element by eight
+// epilogue warps (measured on B200, K=4096 N=14336, LUT3 M=2048: 985-1066
+// TFLOP/s against 935-944 with two stages and the output staged through
+// shared memory for TMA stores; INT4 with two stages lost a fifth)
+constexpr int kTsStages = 3;
 constexpr int kTsABufs = 4;                // A (weights) buffers in tensor memory, 64 columns each
 constexpr int kTsConvWarps = 8, kTsEpWarps = 8;
 // the epilogue warps of one TMEM lane quarter split the tile's tokens
@@ -77,11 +76,7 @@ constexpr int kTsCBytes = kTsBN * 64;               // 8 KB codes (INT4) / 6 KB 
 constexpr int kTsMBytes = 2048;                     // scales + zero points (INT4) / tables (LUT3)
 constexpr int kTsOffC = kTsXBytes, kTsOffM = kTsOffC + kTsCBytes;
 constexpr int kTsStageBytes = kTsOffM + kTsMBytes;  // 74 KB, a multiple of 1024
-constexpr int kTsOutBytes = 32 * kTsBN * 2;          // one [32 tokens][128 channels] output tile
-// LUT3: two staging tiles per epilogue group
-__host__ __device__ constexpr int ts_smem(bool lut) {
-  return ts_stages(lut) * kTsStageBytes + (lut ? 2 * kTsEpGroups * kTsOutBytes : 0) + 1024;
-}
+constexpr int kTsSmem = kTsStages * kTsStageBytes + 1024;
 constexpr uint32_t kTsColA = 0, kTsColD = 256;
 static_assert(kTsStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
 
@@ -92,7 +87,6 @@ struct GemmTsArgs {
   int M, N, K, G, group;
   int n_tiles, m_tiles, k_blocks;  // channel tiles, token tiles, 64-k blocks
   int y_bf16;
-  int tma_out;               // 1: Y written by TMA stores (N % 8 == 0, 16-byte aligned Y); 0: element stores
   int dp_tiles;              // tiles taken whole, strided over the grid (all of them without stream-K)
   long long sk_items;        // (tile, k-block) items of the tiles after them, shared out evenly (0: none)
   float* partials;           // [grid][kTsBM tokens][kTsBN channels] parked sums of cut tiles
@@ -152,16 +146,13 @@ __device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
 template <bool BF16, bool ASYM, bool LUT>
 __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_constant__ CUtensorMap tx,
                                                                 const __grid_constant__ CUtensorMap tq,
-                                                                const __grid_constant__ CUtensorMap ty,
                                                                 const GemmTsArgs a) {
   extern __shared__ uint8_t dsmem[];
-  constexpr int kTsStages = ts_stages(LUT);
-  __shared__ __align__(8) uint64_t full_bar[kTsMaxStages], empty_bar[kTsMaxStages];
+  __shared__ __align__(8) uint64_t full_bar[kTsStages], empty_bar[kTsStages];
   __shared__ __align__(8) uint64_t a_full[kTsABufs], a_empty[kTsABufs], d_full, d_empty;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int sk_ok_sh;  // the epilogue's wait for a parked part succeeded
   uint8_t* ring = dsmem + ((1024u - (smem_u32(dsmem) & 1023u)) & 1023u);
-  uint8_t* obuf = ring + (size_t)kTsStages * kTsStageBytes;  // two output tiles per epilogue group (LUT3)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -332,20 +323,16 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
     }
   } else {
     // ------------------------------------------------------------------ epilogue
-    // every epilogue warp runs every chunk and (with TMA stores) both named
-    // barriers of it, also after a timed-out wait (then it loads and stores
-    // nothing). Element stores take no barrier: each warp reads its own TMEM
-    // lanes and writes its own channels, and the accumulator is released as
-    // soon as the last chunk is in registers.
+    // Every epilogue warp walks every item, also after a timed-out wait (then
+    // it loads and stores nothing). The stores take no barrier: each warp
+    // reads its own TMEM lanes and tokens and writes its own channels, and
+    // releases its part of the accumulator as soon as it is in registers.
     const int q = warp & 3;
     const int r = 32 * q + lane;  // channel within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
     const int eg = (warp - 2 - kTsConvWarps) >> 2;  // epilogue group: tokens [64 kTsEpPairs eg, +64 kTsEpPairs)
     const bool lead = warp == 2 + kTsConvWarps && lane == 0;  // flags of cut tiles
-    const bool issuer = ((warp - 2 - kTsConvWarps) & 3) == 0 && lane == 0;  // the group's TMA stores
-    const uint32_t gbar = 2u + (uint32_t)eg;  // the group's named barrier (barrier 1: all epilogue warps)
-    if (issuer) tma_prefetch_desc(&ty);
-    int t_iter = 0, ob = 0;
+    int t_iter = 0;
     bool ok = true;
     TsSched sch(a);
     TsItem w;
@@ -400,44 +387,19 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
             for (int i = 0; i < 32; ++i)
               v[i] = __float_as_uint(__uint_as_float(v[i]) + __ldcg(park_in + (j * 32 + i) * kTsBN));
           }
-          // the shared staging tile and its barriers serve the TMA stores only:
-          // element stores and parked sums go out per warp, unordered
-          if (LUT && a.tma_out) {
-            if (issuer) bulk_wait_read<1>();  // the group's tile written two chunks ago has been read
-            asm volatile("bar.sync %0, 128;" :: "r"(gbar) : "memory");
-          }
-          uint8_t* ot = obuf + (size_t)(2 * eg + ob) * kTsOutBytes;
           const int m0 = mt * kTsBM + j * 32;
           if (w.part == 1) {  // a later part: park the FP32 sums (all 256 tokens; rows past M hold zeros)
             if (ok) {
 #pragma unroll
               for (int i = 0; i < 32; ++i) __stcg(park_out + (j * 32 + i) * kTsBN, __uint_as_float(v[i]));
             }
-          } else if (!a.tma_out) {  // rows of Y not 16-byte aligned: element stores
+          } else {  // element stores: per warp, unordered
             const int n = nt * kTsBN + r;
             if (ok && n < a.N) {
 #pragma unroll
               for (int i = 0; i < 32; ++i)
                 if (m0 + i < a.M) store_out(a.Y, (size_t)(m0 + i) * a.N + n, __uint_as_float(v[i]), a.y_bf16);
             }
-          }
-          if (LUT && a.tma_out) {  // the staging tiles exist only in the LUT3 kernel's shared memory
-            if (w.part != 1) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float f = __uint_as_float(v[i]);
-                const uint16_t hb =
-                    a.y_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(f)) : __half_as_ushort(__float2half_rn(f));
-                *reinterpret_cast<uint16_t*>(ot + (i * kTsBN + r) * 2) = hb;
-              }
-            }
-            fence_proxy_async();  // the tile, to the TMA unit
-            asm volatile("bar.sync %0, 128;" :: "r"(gbar) : "memory");
-            if (issuer && ok && w.part != 1 && m0 < a.M) {
-              tma_store_2d(&ty, ot, nt * kTsBN, m0);
-              bulk_commit();
-            }
-            ob ^= 1;
           }
         }
       }
@@ -447,7 +409,6 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
         if (lead && ok && !a.debug_hold) st_release_u32(a.flags + blockIdx.x, 1u);
       }
     }
-    if (LUT && issuer) bulk_wait<0>();  // every output store has landed
   }
 
   tc_fence_before();

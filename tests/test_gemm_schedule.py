@@ -11,8 +11,8 @@ import pytest
 SHAPES = [
     (512, 4096, 14336),    # 224 tiles on 148 CTAs
     (2048, 4096, 14336),   # 896 tiles: 6 full waves and 8 tiles
-    (8192, 4096, 14336),   # 3584 tiles
-    (4096, 4096, 14336),   # 1792 tiles: a nearly full last wave (no stream-K)
+    (8192, 4096, 14336),   # 3584 tiles: 3% of the schedule idle (whole tiles)
+    (4096, 4096, 14336),   # 1792 tiles: 7% idle
     (300, 1056, 4000),     # ragged M, K (9 blocks, the last part-filled) and N
     (17, 64, 128),         # one tile
     (1000, 14336, 4096),   # 128 tiles: fewer than the CTAs
@@ -82,9 +82,15 @@ def test_stream_k_balances_the_last_waves(M, K, N):
             assert lbq.lbq_workspace_size(2, M, K, N, 0, lbq.MODES["lut3"]) == ws
     else:
         assert load == load_whole
-    # the shapes the bench times are cut
-    if (M, K, N) in [(512, 4096, 14336), (2048, 4096, 14336), (8192, 4096, 14336)]:
+    # the rule: cut where the last wave leaves at least 5% of the schedule's SM
+    # time idle (and 4 k-blocks per SM)
+    tiles = ((M + 255) // 256) * ((N + 127) // 128)
+    rem, waves = tiles % grid, -(-tiles // grid)
+    assert cut == (tiles > grid and rem > 0 and nkb * (grid - rem) >= 4 * grid and 20 * (grid - rem) >= grid * waves)
+    if (M, K, N) in [(512, 4096, 14336), (2048, 4096, 14336), (4096, 4096, 14336)]:
         assert cut
+    if (M, K, N) == (8192, 4096, 14336):
+        assert not cut
 
 
 def test_whole_tile_schedule_is_the_strided_order():
