@@ -29,8 +29,8 @@
 //               E4M3 weights of the block into the swizzled A tile, its scale
 //               bytes into the A scale atom, and the scale bytes of tokens r and
 //               128 + r into the B scale atoms.
-//   warps 6..9  epilogue: tcgen05.ld the finished accumulator 32 tokens at a
-//               time (thread = one channel), round into a [32 tokens][128
+//   warps 6..9  epilogue: tcgen05.ld the finished accumulator 64 tokens per
+//               wait (thread = one channel), round 32 at a time into a [32 tokens][128
 //               channels] shared-memory tile and write it with one TMA store
 //               (two tiles alternate, so the rounding of one overlaps the store
 //               of the other).
@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         const int rows = min(kMxBN, a.N - nt * kMxBN);
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % kMxStages;
-          if (it >= kMxStages && !mbar_wait(&empty_bar[s], ((it / kMxStages) & 1) ^ 1)) { ok = false; break; }
+          if (it >= kMxStages && !mbar_wait_sleep(&empty_bar[s], ((it / kMxStages) & 1) ^ 1)) { ok = false; break; }
           uint8_t* st = ring + (size_t)s * kMxStageBytes;
           const uint32_t tx_bytes =
               (uint32_t)(kMxBM * kMxBK + 2 * rows * 24 + 2 * 16 * a.cb_rows + kMxBM * 16);
@@ -252,7 +252,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       }
       // every copy this CTA issued lands before it may exit
       for (int v = max(0, it - kMxStages); v < it; ++v)
-        if (!mbar_wait(&full_bar[v % kMxStages], (v / kMxStages) & 1)) break;
+        if (!mbar_wait_sleep(&full_bar[v % kMxStages], (v / kMxStages) & 1)) break;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ scale copies + MMA issuer
@@ -260,12 +260,12 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       int it = 0, t_iter = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t_iter) {
-        if (t_iter >= 1 && !mbar_wait(&d_empty, (t_iter - 1) & 1)) break;
+        if (t_iter >= 1 && !mbar_wait_sleep(&d_empty, (t_iter - 1) & 1)) break;
         tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % kMxStages, b = it % kMxABufs;
-          if (!mbar_wait(&full_bar[s], (it / kMxStages) & 1)) { ok = false; break; }
-          if (!mbar_wait(&a_full[b], (it / kMxABufs) & 1)) { ok = false; break; }
+          if (!mbar_wait_sleep(&full_bar[s], (it / kMxStages) & 1)) { ok = false; break; }
+          if (!mbar_wait_sleep(&a_full[b], (it / kMxABufs) & 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t ab = smem_u32(abuf + (size_t)b * kMxABufBytes);
           const uint32_t xb = smem_u32(ring + (size_t)s * kMxStageBytes + kMxOffX);
@@ -296,8 +296,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       const bool row_ok = nt * kMxBN + r < a.N;
       for (int kb = 0; kb < nkb; ++kb, ++it) {
         const int s = it % kMxStages, b = it % kMxABufs;
-        if (ok && !mbar_wait(&full_bar[s], (it / kMxStages) & 1)) ok = false;
-        if (ok && it >= kMxABufs && !mbar_wait(&a_empty[b], ((it / kMxABufs) & 1) ^ 1)) ok = false;
+        if (ok && !mbar_wait_sleep(&full_bar[s], (it / kMxStages) & 1)) ok = false;
+        if (ok && it >= kMxABufs && !mbar_wait_sleep(&a_empty[b], ((it / kMxABufs) & 1) ^ 1)) ok = false;
         tc_fence_after();
         const uint8_t* st = ring + (size_t)s * kMxStageBytes;
         uint8_t* ab = abuf + (size_t)b * kMxABufBytes;
@@ -326,40 +326,48 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++t_iter) {
       const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;
-      if (ok && !mbar_wait(&d_full, t_iter & 1)) ok = false;
+      if (ok && !mbar_wait_sleep(&d_full, t_iter & 1)) ok = false;
       tc_fence_after();
+      // two 32-token chunks per TMEM round trip, each staged and stored as before
 #pragma unroll 1
-      for (int j = 0; j < kMxBM / 32; ++j) {
-        uint32_t v[32];
+      for (int jp = 0; jp < kMxBM / 64; ++jp) {
+        uint32_t vv[2][32];
         if (ok) {
-          tmem_ld32(lane_base + kMxColD + (uint32_t)(j * 32), v);
+          tmem_ld32_nowait(lane_base + kMxColD + (uint32_t)(jp * 64), vv[0]);
+          tmem_ld32_nowait(lane_base + kMxColD + (uint32_t)(jp * 64 + 32), vv[1]);
+          tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0u;
+          for (int i = 0; i < 32; ++i) vv[0][i] = vv[1][i] = 0u;
         }
-        if (j == kMxBM / 32 - 1) {  // the accumulator is in registers: the MMAs may start the next tile
+        if (jp == kMxBM / 64 - 1) {  // the accumulator is in registers: the MMAs may start the next tile
           tc_fence_before();
           __syncwarp();
           if (lane == 0 && ok) mbar_arrive(&d_empty);
         }
-        // the tile written two chunks ago has been read by its TMA store
-        if (issuer) bulk_wait_read<1>();
-        consumer_named_sync(2, kMxEpWarps * 32);
-        uint8_t* ot = obuf + (size_t)ob * kMxOutBytes;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float f = __uint_as_float(v[i]);
-          const uint16_t h = a.y_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(f)) : __half_as_ushort(__float2half_rn(f));
-          *reinterpret_cast<uint16_t*>(ot + (i * kMxBN + r) * 2) = h;
+        for (int hh = 0; hh < 2; ++hh) {
+          const int j = 2 * jp + hh;
+          uint32_t(&v)[32] = vv[hh];
+          // the tile written two chunks ago has been read by its TMA store
+          if (issuer) bulk_wait_read<1>();
+          consumer_named_sync(2, kMxEpWarps * 32);
+          uint8_t* ot = obuf + (size_t)ob * kMxOutBytes;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float f = __uint_as_float(v[i]);
+            const uint16_t h = a.y_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(f)) : __half_as_ushort(__float2half_rn(f));
+            *reinterpret_cast<uint16_t*>(ot + (i * kMxBN + r) * 2) = h;
+          }
+          fence_proxy_async();  // the tile, to the TMA unit
+          consumer_named_sync(2, kMxEpWarps * 32);
+          const int m0 = mt * kMxBM + j * 32;
+          if (issuer && ok && m0 < a.M) {
+            tma_store_2d(&ty, ot, nt * kMxBN, m0);
+            bulk_commit();
+          }
+          ob ^= 1;
         }
-        fence_proxy_async();  // the tile, to the TMA unit
-        consumer_named_sync(2, kMxEpWarps * 32);
-        const int m0 = mt * kMxBM + j * 32;
-        if (issuer && ok && m0 < a.M) {
-          tma_store_2d(&ty, ot, nt * kMxBN, m0);
-          bulk_commit();
-        }
-        ob ^= 1;
       }
     }
     if (issuer) bulk_wait<0>();  // every output store has landed

@@ -294,7 +294,10 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
               uint32_t c1, c2;
               zero_consts<BF16>(z, c1, c2);
               const uint32_t s2 = scale_pair<BF16>(sbits);
-              const uint4 wv = lds128(smem_u32(st + kTsOffC + r * 64 + kc / 2));
+              // the codes box is TMA-swizzled in 64-byte spans (16-byte chunk c of
+              // row r at chunk c ^ ((r >> 1) & 3)): a quarter-warp's loads hit
+              // eight different bank groups
+              const uint4 wv = lds128(smem_u32(st + kTsOffC + r * 64 + ((ci ^ ((r >> 1) & 3)) << 4)));
               const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
               constexpr uint32_t magic = BF16 ? 0x43004300u : 0x64006400u;
 #pragma unroll

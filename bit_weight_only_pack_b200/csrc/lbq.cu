@@ -866,7 +866,7 @@ static lbq_status run_gemm_ts(const void* X, bool xbf16, int M, const void* imag
     return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the prefill activations");
   tq = tx;
   if (!lut && !make_tmap_2d(&tq, img + L.off0, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)L.K / 2, (uint64_t)L.N,
-                            (uint64_t)L.K / 2, kTsBK / 2, kTsBN, CU_TENSOR_MAP_SWIZZLE_NONE))
+                            (uint64_t)L.K / 2, kTsBK / 2, kTsBN, CU_TENSOR_MAP_SWIZZLE_64B))
     return fail(LBQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the prefill codes");
   GemmTsArgs a{};
   a.Y = Y;
