@@ -575,9 +575,12 @@ def _secondary_measurements(torch, lbq, workloads, device, peaks, quick):
         codes_h, scales_h = workloads.mx_activations_host(60 + M, M, K)
         codes, scales = torch.from_numpy(codes_h).to(device), torch.from_numpy(scales_h).to(device)
         Ymx = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        wsmx = lbq.workspace(2, M, K, N, 0, "lut3")
 
         def mxcall(img, s):
-            lbq.lbq_lut3_mx_gemm(codes.data_ptr(), scales.data_ptr(), M, K, N, img.data_ptr(), Ymx.data_ptr(), 1, s)
+            lbq.lbq_lut3_mx_gemm(codes.data_ptr(), scales.data_ptr(), M, K, N, img.data_ptr(), Ymx.data_ptr(), 1,
+                                 wsmx.data_ptr() if wsmx is not None else None,
+                                 wsmx.numel() if wsmx is not None else 0, s)
 
         ms = rotating_ms(torch, mxcall, images, reps=3)
         tf = 2.0 * M * K * N / ms / 1e9
@@ -875,8 +878,9 @@ def run_profile_case(name):
         del idx, cb, ex
         codes_h, scales_h = workloads.mx_activations_host(7, M, K)
         codes, scales = torch.from_numpy(codes_h).to(device), torch.from_numpy(scales_h).to(device)
+        ws = lbq.workspace(2, M, K, N, 0, "lut3")
         for img in images:
-            lbq.lut3_mx_gemm(codes, scales, img, N)
+            lbq.lut3_mx_gemm(codes, scales, img, N, ws=ws)
         torch.cuda.synchronize()
         lbq.device_status()
         print(f"profile case {name}: {len(images)} launches of K={K} N={N} M={M}", flush=True)

@@ -69,7 +69,7 @@ _SIGS = {
     "lbq_gemv_noalloc": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp], _c_int),
     "lbq_gemv_grouped": ([ctypes.POINTER(lbq_gemv_item), _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp], _c_int),
     "lbq_quantize_mxfp8": ([_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp], _c_int),
-    "lbq_lut3_mx_gemm": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp], _c_int),
+    "lbq_lut3_mx_gemm": ([_vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp, _c_size, _vp], _c_int),
     "lbq_affine_packed_size": ([_c_int, _c_int, _c_int, _c_int, ctypes.POINTER(_c_size)], _c_int),
     "lbq_pack_affine": ([_vp, _c_int, _c_int, _c_int, _c_int, _vp, _c_size, _vp], _c_int),
     "lbq_affine_gemv": ([_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int, _vp], _c_int),
@@ -210,18 +210,21 @@ def quantize_mxfp8(X):
     return codes, scales
 
 
-def lbq_lut3_mx_gemm(codes, scales, M, K, N, image, Y, y_dtype, stream):
-    _check(_lib.lbq_lut3_mx_gemm(codes, scales, M, K, N, image, Y, y_dtype, stream))
+def lbq_lut3_mx_gemm(codes, scales, M, K, N, image, Y, y_dtype, ws, ws_bytes, stream):
+    _check(_lib.lbq_lut3_mx_gemm(codes, scales, M, K, N, image, Y, y_dtype, ws, ws_bytes, stream))
 
 
-def lut3_mx_gemm(codes, scales, image, N, y_dtype="bf16", Y=None):
+def lut3_mx_gemm(codes, scales, image, N, y_dtype="bf16", Y=None, ws=None):
     """Y[M, N] = MXFP8 activations (codes uint8 [M, K], scales uint8 [M, K/32]) . LUT3 weights."""
     torch = _torch()
-    _need_cuda(codes, scales, image, Y)
+    _need_cuda(codes, scales, image, Y, ws)
     M, K = codes.shape
     if Y is None:
         Y = torch.empty((M, N), dtype={"f16": torch.float16, "bf16": torch.bfloat16}[y_dtype], device=codes.device)
-    lbq_lut3_mx_gemm(codes.data_ptr(), scales.data_ptr(), M, K, N, image.data_ptr(), Y.data_ptr(), _dt(Y), _stream())
+    if ws is None and M > 16:
+        ws = workspace(2, M, K, N, 0, "lut3", codes.device)
+    lbq_lut3_mx_gemm(codes.data_ptr(), scales.data_ptr(), M, K, N, image.data_ptr(), Y.data_ptr(), _dt(Y),
+                     ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0, _stream())
     return Y
 
 

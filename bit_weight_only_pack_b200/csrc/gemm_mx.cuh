@@ -45,6 +45,7 @@
 #include "tma.cuh"
 #include "gemm_tc.cuh"
 #include "lut3_gemv.cuh"
+#include "stream_k.cuh"
 
 namespace lbq {
 
@@ -88,6 +89,7 @@ struct GemmMxArgs {
   int n_tiles, m_tiles, k_blocks;
   int cb_rows;               // rows of the codebook / exponent boxes (min(16, N/8))
   int y_bf16;
+  SkArgs sk;                 // the schedule: whole tiles, or stream-K over the last two waves (stream_k.cuh)
 };
 
 // Instruction descriptor of kind::mxf8f6f4.block_scale: A = B = E4M3, K-major,
@@ -189,13 +191,12 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   __shared__ __align__(8) uint64_t full_bar[kMxStages], empty_bar[kMxStages];
   __shared__ __align__(8) uint64_t a_full[kMxABufs], a_empty[kMxABufs], d_full, d_empty;
   __shared__ uint32_t tmem_base_sh;
+  __shared__ int sk_ok_sh;  // the epilogue's wait for a parked part succeeded
   uint8_t* ring = dsmem + ((1024u - (smem_u32(dsmem) & 1023u)) & 1023u);
   uint8_t* abuf = ring + (size_t)kMxStages * kMxStageBytes;
   uint8_t* obuf = abuf + (size_t)kMxABufs * kMxABufBytes;  // two output tiles
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int total_tiles = a.n_tiles * a.m_tiles;
-  const int nkb = a.k_blocks;
 
   if (tid == 0) {
     for (int i = 0; i < kMxStages; ++i) {
@@ -229,10 +230,12 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       tma_prefetch_desc(&te);
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;  // token tiles inner: indices reused from L2
+      SkSched sch(a.sk.dp_tiles, a.sk.sk_items, a.k_blocks, (int)blockIdx.x, (int)gridDim.x);
+      SkItem w;
+      while (ok && sch.next(w)) {
+        const int nt = w.tile / a.m_tiles, mt = w.tile - nt * a.m_tiles;  // token tiles inner: indices reused from L2
         const int rows = min(kMxBN, a.N - nt * kMxBN);
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const int s = it % kMxStages;
           if (it >= kMxStages && !mbar_wait_sleep(&empty_bar[s], ((it / kMxStages) & 1) ^ 1)) { ok = false; break; }
           uint8_t* st = ring + (size_t)s * kMxStageBytes;
@@ -259,10 +262,12 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     if (lane == 0) {
       int it = 0, t_iter = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t_iter) {
+      SkSched sch(a.sk.dp_tiles, a.sk.sk_items, a.k_blocks, (int)blockIdx.x, (int)gridDim.x);
+      SkItem w;
+      for (; ok && sch.next(w); ++t_iter) {
         if (t_iter >= 1 && !mbar_wait_sleep(&d_empty, (t_iter - 1) & 1)) break;
         tc_fence_after();
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const int s = it % kMxStages, b = it % kMxABufs;
           if (!mbar_wait_sleep(&full_bar[s], (it / kMxStages) & 1)) { ok = false; break; }
           if (!mbar_wait_sleep(&a_full[b], (it / kMxABufs) & 1)) { ok = false; break; }
@@ -278,7 +283,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             const uint64_t da = umma_desc_sw128(ab + kMxOffA) + (uint64_t)(kk * 2);
             const uint64_t db = umma_desc_sw128(xb) + (uint64_t)(kk * 2);
             umma_mx(tmem + kMxColD, da, db, umma_idesc_mx(kk), sf | (kk << 30), (sf + 4) | (kk << 30),
-                    (kb > 0 || kk > 0) ? 1u : 0u);
+                    (kb > w.kb0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&empty_bar[s]);
           umma_commit(&a_empty[b]);
@@ -291,10 +296,12 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     const int r = (warp - 2) * 32 + lane;  // channel within the tile / token within each half
     int it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      const int nt = tile / a.m_tiles;
+    SkSched sch(a.sk.dp_tiles, a.sk.sk_items, a.k_blocks, (int)blockIdx.x, (int)gridDim.x);
+    SkItem w;
+    while (sch.next(w)) {
+      const int nt = w.tile / a.m_tiles;
       const bool row_ok = nt * kMxBN + r < a.N;
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
+      for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
         const int s = it % kMxStages, b = it % kMxABufs;
         if (ok && !mbar_wait_sleep(&full_bar[s], (it / kMxStages) & 1)) ok = false;
         if (ok && it >= kMxABufs && !mbar_wait_sleep(&a_empty[b], ((it / kMxABufs) & 1) ^ 1)) ok = false;
@@ -324,10 +331,21 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     // barrier sequence stays the same in all four warps
     int t_iter = 0, ob = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++t_iter) {
-      const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;
+    SkSched sch(a.sk.dp_tiles, a.sk.sk_items, a.k_blocks, (int)blockIdx.x, (int)gridDim.x);
+    SkItem w;
+    for (; sch.next(w); ++t_iter) {
+      const int nt = w.tile / a.m_tiles, mt = w.tile - nt * a.m_tiles;
       if (ok && !mbar_wait_sleep(&d_full, t_iter & 1)) ok = false;
       tc_fence_after();
+      // cut tiles: an earlier part adds the sums parked in slot blockIdx.x + 1;
+      // a later part parks its own in slot blockIdx.x (stream_k.cuh)
+      const float* park_in = a.sk.partials + (size_t)(blockIdx.x + 1) * kSkTileFloats + r;
+      float* park_out = a.sk.partials + (size_t)blockIdx.x * kSkTileFloats + r;
+      if (w.part == 2) {
+        if (issuer) sk_ok_sh = (ok && sk_wait_parked(a.sk)) ? 1 : 0;
+        consumer_named_sync(1, kMxEpWarps * 32);
+        ok = ok && sk_ok_sh != 0;
+      }
       // two 32-token chunks per TMEM round trip, each staged and stored as before
 #pragma unroll 1
       for (int jp = 0; jp < kMxBM / 64; ++jp) {
@@ -349,25 +367,42 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         for (int hh = 0; hh < 2; ++hh) {
           const int j = 2 * jp + hh;
           uint32_t(&v)[32] = vv[hh];
+          if (w.part == 2 && ok) {  // own sums + parked sums, in that order
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              v[i] = __float_as_uint(__uint_as_float(v[i]) + __ldcg(park_in + (j * 32 + i) * kMxBN));
+          }
+          if (w.part == 1 && ok) {  // a later part: park the FP32 sums (all 256 tokens; rows past M hold zeros)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) __stcg(park_out + (j * 32 + i) * kMxBN, __uint_as_float(v[i]));
+          }
           // the tile written two chunks ago has been read by its TMA store
           if (issuer) bulk_wait_read<1>();
           consumer_named_sync(2, kMxEpWarps * 32);
           uint8_t* ot = obuf + (size_t)ob * kMxOutBytes;
+          if (w.part != 1) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float f = __uint_as_float(v[i]);
-            const uint16_t h = a.y_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(f)) : __half_as_ushort(__float2half_rn(f));
-            *reinterpret_cast<uint16_t*>(ot + (i * kMxBN + r) * 2) = h;
+            for (int i = 0; i < 32; ++i) {
+              const float f = __uint_as_float(v[i]);
+              const uint16_t h =
+                  a.y_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(f)) : __half_as_ushort(__float2half_rn(f));
+              *reinterpret_cast<uint16_t*>(ot + (i * kMxBN + r) * 2) = h;
+            }
           }
           fence_proxy_async();  // the tile, to the TMA unit
           consumer_named_sync(2, kMxEpWarps * 32);
           const int m0 = mt * kMxBM + j * 32;
-          if (issuer && ok && m0 < a.M) {
+          if (issuer && ok && w.part != 1 && m0 < a.M) {
             tma_store_2d(&ty, ot, nt * kMxBN, m0);
             bulk_commit();
           }
           ob ^= 1;
         }
+      }
+      if (w.part == 1) {  // the parked sums are visible GPU-wide before the flag
+        __threadfence();
+        consumer_named_sync(1, kMxEpWarps * 32);
+        if (issuer && ok && !a.sk.debug_hold) st_release_u32(a.sk.flags + blockIdx.x, 1u);
       }
     }
     if (issuer) bulk_wait<0>();  // every output store has landed

@@ -31,16 +31,8 @@
 //               the round trips, the less of each tile the converters (which
 //               run at most three k-blocks ahead of the stalled MMAs) lose.
 //
-// Schedule: the CTAs (at most one per SM) take whole tiles strided over the
-// grid; when the tiles leave a part-filled last wave, the last two waves'
-// tiles are instead cut into (tile, 128-k block) items shared out evenly
-// (stream-K), so every SM ends at about the same time. Each CTA's share is at
-// least one tile long, so a tile is cut at most once: its earlier part ends
-// the share of CTA c - 1 and its later part starts the share of CTA c. The
-// later part finishes first (it is its CTA's first item of the phase), parks
-// its FP32 sums in workspace slot c and raises flag c; the earlier part waits
-// for the flag (bounded), adds the parked sums to its own in a fixed order and
-// writes the tile, so results do not depend on timing.
+// Schedule: whole tiles strided over the grid, or stream-K over the last two
+// waves when the tail wave leaves SMs idle (stream_k.cuh).
 #pragma once
 
 #include "common.cuh"
@@ -49,6 +41,7 @@
 #include "gemm_tc.cuh"
 #include "tc_gemv.cuh"
 #include "lut3_gemv.cuh"
+#include "stream_k.cuh"
 
 namespace lbq {
 
@@ -78,6 +71,7 @@ constexpr int kTsOffC = kTsXBytes, kTsOffM = kTsOffC + kTsCBytes;
 constexpr int kTsStageBytes = kTsOffM + kTsMBytes;  // 74 KB, a multiple of 1024
 constexpr int kTsSmem = kTsStages * kTsStageBytes + 1024;
 constexpr uint32_t kTsColA = 0, kTsColD = 256;
+static_assert(kTsBM * kTsBN == kSkTileFloats, "a parked tile is one output tile");
 static_assert(kTsStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
 
 struct GemmTsArgs {
@@ -87,61 +81,8 @@ struct GemmTsArgs {
   int M, N, K, G, group;
   int n_tiles, m_tiles, k_blocks;  // channel tiles, token tiles, 64-k blocks
   int y_bf16;
-  int dp_tiles;              // tiles taken whole, strided over the grid (all of them without stream-K)
-  long long sk_items;        // (tile, k-block) items of the tiles after them, shared out evenly (0: none)
-  float* partials;           // [grid][kTsBM tokens][kTsBN channels] parked sums of cut tiles
-  unsigned* flags;           // [grid] 1 while slot c holds a later part's sums; reset by the reader
-  uint32_t flag_polls;       // bound on the wait for a parked part (about 1 us per poll)
-  int debug_hold;            // test hook: later parts never raise their flag
+  SkArgs sk;                 // the schedule (stream_k.cuh)
 };
-
-// One work item: k-blocks [kb0, kb1) of a tile. part 0: the whole tile;
-// 1: a later part (parks its sums in slot blockIdx.x); 2: an earlier part
-// (adds the sums parked in slot blockIdx.x + 1, then writes the tile).
-struct TsItem {
-  int tile, kb0, kb1, part;
-};
-
-// The items of CTA `cta` of `grid` in order; every role of the CTA walks the
-// same sequence (the host runs it too, for the schedule's checks).
-struct TsSched {
-  int tile, dp_tiles, step, nkb;
-  long long pos, end;
-  __host__ __device__ TsSched(int dp, long long sk_items, int k_blocks, int cta, int grid)
-      : tile(cta), dp_tiles(dp), step(grid), nkb(k_blocks) {
-    pos = sk_items * cta / grid;
-    end = sk_items * (cta + 1) / grid;
-  }
-  __device__ explicit TsSched(const GemmTsArgs& a)
-      : TsSched(a.dp_tiles, a.sk_items, a.k_blocks, (int)blockIdx.x, (int)gridDim.x) {}
-  __host__ __device__ bool next(TsItem& w) {
-    if (tile < dp_tiles) {
-      w.tile = tile;
-      w.kb0 = 0;
-      w.kb1 = nkb;
-      w.part = 0;
-      tile += step;
-      return true;
-    }
-    if (pos >= end) return false;
-    const long long t = pos / nkb;
-    w.tile = dp_tiles + (int)t;
-    w.kb0 = (int)(pos - t * nkb);
-    w.kb1 = (int)(end - pos < (long long)(nkb - w.kb0) ? w.kb0 + (end - pos) : nkb);
-    w.part = w.kb0 > 0 ? 1 : (w.kb1 < nkb ? 2 : 0);
-    pos += w.kb1 - w.kb0;
-    return true;
-  }
-};
-
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
-}
 
 template <bool BF16, bool ASYM, bool LUT>
 __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_constant__ CUtensorMap tx,
@@ -186,8 +127,8 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
       if (!LUT) tma_prefetch_desc(&tq);
       int it = 0;
       bool ok = true;
-      TsSched sch(a);
-      TsItem w;
+      SkSched sch(a.sk.dp_tiles, a.sk.sk_items, a.k_blocks, (int)blockIdx.x, (int)gridDim.x);
+      SkItem w;
       while (ok && sch.next(w)) {
         const int nt = w.tile / a.m_tiles, mt = w.tile - nt * a.m_tiles;  // token tiles inner: codes reused from L2
         const int rows = min(kTsBN, a.N - nt * kTsBN);
@@ -226,8 +167,8 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
       const uint32_t idesc = umma_idesc_m128(BF16, kTsBM);
       int it = 0, t_iter = 0;
       bool ok = true;
-      TsSched sch(a);
-      TsItem w;
+      SkSched sch(a.sk.dp_tiles, a.sk.sk_items, a.k_blocks, (int)blockIdx.x, (int)gridDim.x);
+      SkItem w;
       for (; ok && sch.next(w); ++t_iter) {
         if (t_iter >= 1 && !mbar_wait_sleep(&d_empty, (t_iter - 1) & 1)) break;
         tc_fence_after();
@@ -258,8 +199,8 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
     int it = 0;
     bool ok = true;
-    TsSched sch(a);
-    TsItem w;
+    SkSched sch(a.sk.dp_tiles, a.sk.sk_items, a.k_blocks, (int)blockIdx.x, (int)gridDim.x);
+    SkItem w;
     while (sch.next(w)) {
       const int nt = w.tile / a.m_tiles;
       const bool row_ok = nt * kTsBN + r < a.N;
@@ -337,29 +278,17 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
     const bool lead = warp == 2 + kTsConvWarps && lane == 0;  // flags of cut tiles
     int t_iter = 0;
     bool ok = true;
-    TsSched sch(a);
-    TsItem w;
+    SkSched sch(a.sk.dp_tiles, a.sk.sk_items, a.k_blocks, (int)blockIdx.x, (int)gridDim.x);
+    SkItem w;
     for (; sch.next(w); ++t_iter) {
       const int nt = w.tile / a.m_tiles, mt = w.tile - nt * a.m_tiles;
       if (ok && !mbar_wait_sleep(&d_full, t_iter & 1)) ok = false;
       tc_fence_after();
       // an earlier part: wait for the later part's sums in slot blockIdx.x + 1
-      const float* park_in = a.partials + (size_t)(blockIdx.x + 1) * (kTsBM * kTsBN) + r;
-      float* park_out = a.partials + (size_t)blockIdx.x * (kTsBM * kTsBN) + r;
+      const float* park_in = a.sk.partials + (size_t)(blockIdx.x + 1) * kSkTileFloats + r;
+      float* park_out = a.sk.partials + (size_t)blockIdx.x * kSkTileFloats + r;
       if (w.part == 2) {
-        if (lead) {
-          bool got = false;
-          if (ok) {
-            unsigned* f = a.flags + blockIdx.x + 1;
-            for (uint32_t i = 0; i < a.flag_polls && !got; ++i) {
-              got = ld_acquire_u32(f) != 0u;
-              if (!got) __nanosleep(1000);
-            }
-            if (got) atomicExch(f, 0u);  // the slot is free for the next call
-            else atomicOr(&g_device_error, kDevErrTimeout);
-          }
-          sk_ok_sh = got ? 1 : 0;
-        }
+        if (lead) sk_ok_sh = (ok && sk_wait_parked(a.sk)) ? 1 : 0;
         asm volatile("bar.sync 1, %0;" :: "r"(kTsEpWarps * 32) : "memory");
         ok = ok && sk_ok_sh != 0;
       }
@@ -409,7 +338,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
       if (w.part == 1) {  // the parked sums are visible GPU-wide before the flag
         __threadfence();
         asm volatile("bar.sync 1, %0;" :: "r"(kTsEpWarps * 32) : "memory");
-        if (lead && ok && !a.debug_hold) st_release_u32(a.flags + blockIdx.x, 1u);
+        if (lead && ok && !a.sk.debug_hold) st_release_u32(a.sk.flags + blockIdx.x, 1u);
       }
     }
   }

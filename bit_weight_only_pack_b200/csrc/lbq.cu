@@ -851,9 +851,25 @@ static TsPlan plan_gemm_ts(int M, int K, int N) {
     p.dp_tiles = (T / p.grid - 1) * p.grid;
     p.sk_items = (long long)(T - p.dp_tiles) * nkb;
     p.flags_bytes = ((size_t)p.grid * 4 + 255) / 256 * 256;
-    p.ws_bytes = p.flags_bytes + (size_t)p.grid * kTsBM * kTsBN * 4;
+    p.ws_bytes = p.flags_bytes + (size_t)p.grid * kSkTileFloats * 4;
   }
   return p;
+}
+
+// The schedule's kernel arguments: stream-K where the plan cuts tiles and the
+// caller's workspace is large enough, else whole tiles.
+static SkArgs sk_args(const TsPlan& p, int tiles, void* ws, size_t ws_bytes) {
+  SkArgs k{};
+  k.dp_tiles = tiles;
+  k.flag_polls = g_ts_polls ? g_ts_polls : (1u << 22);
+  k.debug_hold = g_ts_hold;
+  if (p.ws_bytes && g_ts_stream_k && ws && ws_bytes >= p.ws_bytes) {
+    k.dp_tiles = p.dp_tiles;
+    k.sk_items = p.sk_items;
+    k.flags = static_cast<unsigned*>(ws);
+    k.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + p.flags_bytes);
+  }
+  return k;
 }
 
 static lbq_status run_gemm_ts(const void* X, bool xbf16, int M, const void* image, const Layout& L, void* Y,
@@ -887,15 +903,7 @@ static lbq_status run_gemm_ts(const void* X, bool xbf16, int M, const void* imag
   occupancy_for((const void*)fn, kTsThreads, smem);
   const TsPlan p = plan_gemm_ts(M, L.K, L.N);
   const int grid = p.grid;
-  a.dp_tiles = a.n_tiles * a.m_tiles;
-  a.flag_polls = g_ts_polls ? g_ts_polls : (1u << 22);
-  a.debug_hold = g_ts_hold;
-  if (p.ws_bytes && g_ts_stream_k && ws && ws_bytes >= p.ws_bytes) {  // without the workspace: whole tiles
-    a.dp_tiles = p.dp_tiles;
-    a.sk_items = p.sk_items;
-    a.flags = static_cast<unsigned*>(ws);
-    a.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + p.flags_bytes);
-  }
+  a.sk = sk_args(p, a.n_tiles * a.m_tiles, ws, ws_bytes);
   void* args[] = {&tx, &tq, &a};
   return launch_kernel_ex((const void*)fn, dim3(grid), dim3(kTsThreads), smem, st, false, args,
                           "prefill GEMM launch");
@@ -1175,7 +1183,7 @@ static lbq_status run_lut3_gemm_tc(const void* X, int M, const void* image, cons
 // ----------------------------------------------------------------------------
 
 static lbq_status run_lut3_mx(const uint8_t* codes, const uint8_t* scales, int M, const void* image, const Layout& L,
-                              void* Y, bool ybf16, cudaStream_t st) {
+                              void* Y, bool ybf16, void* ws, size_t ws_bytes, cudaStream_t st) {
   const uint8_t* img = static_cast<const uint8_t*>(image);
   const int cb_rows = std::min(16, L.N / 8);
   CUtensorMap tx, ts, tc, te, ty;
@@ -1203,7 +1211,11 @@ static lbq_status run_lut3_mx(const uint8_t* codes, const uint8_t* scales, int M
   a.y_bf16 = ybf16 ? 1 : 0;
   const void* fn = (const void*)gemm_mx_lut3_kernel;
   occupancy_for(fn, kMxThreads, kMxSmem);
-  const int grid = std::min(a.n_tiles * a.m_tiles, num_sms());
+  // the tile and k-block of the BF16-decode prefill: the same schedule and workspace
+  static_assert(kMxBN == kTsBN && kMxBM == kTsBM && kMxBK == kTsBK, "one stream-K plan for both prefill GEMMs");
+  const TsPlan p = plan_gemm_ts(M, L.K, L.N);
+  const int grid = p.grid;
+  a.sk = sk_args(p, a.n_tiles * a.m_tiles, ws, ws_bytes);
   void* args[] = {&tx, &ts, &tc, &te, &ty, &a};
   return launch_kernel_ex(fn, dim3(grid), dim3(kMxThreads), kMxSmem, st, false, args, "LUT3 x MXFP8 GEMM launch");
 }
@@ -1493,9 +1505,9 @@ int lbq_debug_gemm_schedule(int M, int K, int N, int stream_k, int cta, int* gri
   *grid = p.grid;
   *k_blocks = nkb;
   const bool sk = stream_k && p.ws_bytes;
-  TsSched sch(sk ? p.dp_tiles : ((N + kTsBN - 1) / kTsBN) * ((M + kTsBM - 1) / kTsBM), sk ? p.sk_items : 0, nkb,
+  SkSched sch(sk ? p.dp_tiles : ((N + kTsBN - 1) / kTsBN) * ((M + kTsBM - 1) / kTsBM), sk ? p.sk_items : 0, nkb,
               cta, p.grid);
-  TsItem w;
+  SkItem w;
   int n = 0;
   while (sch.next(w)) {
     if (n < max_items) {
@@ -1908,7 +1920,7 @@ lbq_status lbq_gemv_noalloc(const void* X, int x_dtype, int M, int K, int N, int
 }
 
 lbq_status lbq_lut3_mx_gemm(const uint8_t* codes, const uint8_t* scales, int M, int K, int N, const void* image,
-                            void* Y, int y_dtype, void* stream) {
+                            void* Y, int y_dtype, void* ws, size_t ws_bytes, void* stream) {
   lbq_status st = check_lut3_shape(K, N);
   if (st != LBQ_OK) return st;
   if (K % 512) return fail(LBQ_ERR_UNSUPPORTED, "lbq_lut3_mx_gemm needs K %% 512 == 0 (K=%d)", K);
@@ -1918,7 +1930,7 @@ lbq_status lbq_lut3_mx_gemm(const uint8_t* codes, const uint8_t* scales, int M, 
     return fail(LBQ_ERR_INVALID_ARG, "codes, scales, image and Y must be 16-byte aligned");
   if (y_dtype != LBQ_DTYPE_F16 && y_dtype != LBQ_DTYPE_BF16) return fail(LBQ_ERR_UNSUPPORTED, "y_dtype %d", y_dtype);
   return run_lut3_mx(codes, scales, M, image, make_layout(K, N, 0, LBQ_MODE_LUT3), Y, y_dtype == LBQ_DTYPE_BF16,
-                     static_cast<cudaStream_t>(stream));
+                     ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 lbq_status lbq_moe_max_padded(int num_pairs, int num_experts, int block, int* max_padded) {

@@ -320,6 +320,10 @@ lbq_status lbq_quantize_mxfp8(const void* X, int x_dtype, int M, int K, uint8_t*
  *   scales (device) uint8 [M, K/32], UE8M0 bytes
  *   image  (device) from lbq_pack_lut3 with this K, N
  *   Y      (device) [M, N] row-major, y_dtype, fully overwritten
+ *   ws     (device) optional, lbq_workspace_size(2, M, K, N, 0, LBQ_MODE_LUT3)
+ *          bytes, zero-filled (see lbq_workspace_size): with it the tail
+ *          wave's tiles are cut along K as in lbq_gemm; null (or smaller)
+ *          computes every tile whole
  * K % 512 == 0 (the block scales are read 16 bytes, 512 k, at a time), N % 8
  * == 0, M >= 1; every pointer 16-byte aligned. NaN codes (0x7F / 0xFF) or scale
  * bytes (0xFF) give NaN outputs. Errors: LBQ_ERR_INVALID_ARG for null or
@@ -327,7 +331,7 @@ lbq_status lbq_quantize_mxfp8(const void* X, int x_dtype, int M, int K, uint8_t*
  * unknown y_dtype, before any launch. Asynchronous on `stream`.
  */
 lbq_status lbq_lut3_mx_gemm(const uint8_t* codes, const uint8_t* scales, int M, int K, int N, const void* image,
-                            void* Y, int y_dtype, void* stream);
+                            void* Y, int y_dtype, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Generic b-bit affine weights, b = 1..8 ("Low Bit ARM kernels": one GEMV

@@ -54,6 +54,64 @@ def test_mx_gemm_parity(torch, lbq, M, K, N, ydt):
     _check(Y, mxfp8.dequant(codes, scales), lut3.dequant(idx, cb, ex))
 
 
+@pytest.mark.parametrize("M,K,N", [
+    (300, 1024, 10000),  # 158 tiles: the tail wave's tiles cut along K, ragged tokens
+    (1100, 1024, 4104),  # 165 tiles, a partial channel tile
+])
+def test_mx_gemm_stream_k(torch, lbq, M, K, N):
+    """With the workspace the last waves' tiles are cut between neighbouring
+    CTAs (the parked part added in a fixed order): both schedules match the
+    oracle, repeated calls on one workspace are identical and every flag is
+    back at zero after each call."""
+    codes, scales = workloads.mx_activations_host(430 + M, M, K)
+    idx, cb, ex = workloads.lut3_host(431 + N, K, N)
+    img = lbq.pack_lut3(torch.from_numpy(idx).cuda(), torch.from_numpy(cb).cuda(), torch.from_numpy(ex).cuda())
+    cd, sd = torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda()
+    ws = lbq.workspace(2, M, K, N, 0, "lut3")
+    assert ws is not None
+    grid = lbq.lbq_debug_gemm_schedule(M, K, N, 1, 0)[0]
+    Ys = [lbq.lut3_mx_gemm(cd, sd, img, N, ws=ws) for _ in range(3)]
+    torch.cuda.synchronize()
+    lbq.device_status()
+    assert all(torch.equal(Ys[0], Y) for Y in Ys[1:])
+    assert int(ws[:grid * 4].view(torch.int32).abs().sum()) == 0
+    Xq, W = mxfp8.dequant(codes, scales), lut3.dequant(idx, cb, ex)
+    _check(Ys[0].cpu(), Xq, W)
+    lbq.lbq_debug_gemm_stream_k(0)
+    try:
+        Y0 = lbq.lut3_mx_gemm(cd, sd, img, N, ws=ws)
+        torch.cuda.synchronize()
+    finally:
+        lbq.lbq_debug_gemm_stream_k(1)
+    _check(Y0.cpu(), Xq, W)
+
+
+def test_mx_gemm_stream_k_wait_runs_out_and_is_reported(torch, lbq):
+    """A withheld flag (test hook) ends each earlier part's wait after a short
+    bound: LBQ_ERR_DEVICE is reported, and the next call on the same workspace
+    matches the oracle."""
+    M, K, N = 300, 1024, 10000
+    codes, scales = workloads.mx_activations_host(440, M, K)
+    idx, cb, ex = workloads.lut3_host(441, K, N)
+    img = lbq.pack_lut3(torch.from_numpy(idx).cuda(), torch.from_numpy(cb).cuda(), torch.from_numpy(ex).cuda())
+    cd, sd = torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda()
+    ws = lbq.workspace(2, M, K, N, 0, "lut3")
+    lbq.device_status()
+    lbq.lbq_debug_gemm_hold(2000)
+    try:
+        lbq.lut3_mx_gemm(cd, sd, img, N, ws=ws)
+        with pytest.raises(lbq.LbqError) as err:
+            lbq.device_status()
+        assert err.value.status == 4  # LBQ_ERR_DEVICE
+    finally:
+        lbq.lbq_debug_gemm_hold(0)
+    lbq.device_status()
+    Y = lbq.lut3_mx_gemm(cd, sd, img, N, ws=ws)
+    torch.cuda.synchronize()
+    lbq.device_status()
+    _check(Y.cpu(), mxfp8.dequant(codes, scales), lut3.dequant(idx, cb, ex))
+
+
 def test_mx_gemm_scale_extremes(torch, lbq):
     """Exponents and scale bytes at the ends of a wide range (weights down to
     2^-117 x E4M3, activations 2^-24..2^+8): the block scales enter the
