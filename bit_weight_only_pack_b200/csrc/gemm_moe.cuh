@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
         const uint8_t* img = a.images + (size_t)(e < 0 ? 0 : e) * a.image_stride;
         // the tile's codebook and exponent rows (16 consecutive rows of each region)
         const int mi = t_iter & 1;
-        if (t_iter >= 2 && !mbar_wait(&meta_empty[mi], ((t_iter >> 1) & 1) ^ 1)) { ok = false; break; }
+        if (t_iter >= 2 && !mbar_wait_sleep(&meta_empty[mi], ((t_iter >> 1) & 1) ^ 1)) { ok = false; break; }
         uint8_t* mt = meta + (size_t)mi * meta_bytes;
         const size_t g0 = (size_t)nt * (kMxBN / 8);
         mbar_arrive_expect_tx(&meta_full[mi], e < 0 ? 0u : (uint32_t)(groups * (a.s_stride + a.z_stride)));
@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
         }
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % kMoeStages;
-          if (it >= kMoeStages && !mbar_wait(&empty_bar[s], ((it / kMoeStages) & 1) ^ 1)) { ok = false; break; }
+          if (it >= kMoeStages && !mbar_wait_sleep(&empty_bar[s], ((it / kMoeStages) & 1) ^ 1)) { ok = false; break; }
           uint8_t* st = ring + (size_t)s * MoeStage::kBytes;
           mbar_arrive_expect_tx(&full_bar[s], e < 0 ? 0u : (uint32_t)(2 * rows * 24));
           if (e >= 0)
@@ -167,9 +167,9 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
       }
       // every copy this CTA issued lands before it may exit
       for (int v = max(0, it - kMoeStages); v < it; ++v)
-        if (!mbar_wait(&full_bar[v % kMoeStages], (v / kMoeStages) & 1)) break;
+        if (!mbar_wait_sleep(&full_bar[v % kMoeStages], (v / kMoeStages) & 1)) break;
       for (int v = max(0, t_iter - 2); v < t_iter; ++v)
-        if (!mbar_wait(&meta_full[v & 1], (v >> 1) & 1)) break;
+        if (!mbar_wait_sleep(&meta_full[v & 1], (v >> 1) & 1)) break;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ scale copies + MMA issuer
@@ -178,12 +178,12 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t_iter) {
         const int ai = t_iter & 1;  // accumulator of this tile
-        if (t_iter >= 2 && !mbar_wait(&d_empty[ai], ((t_iter >> 1) & 1) ^ 1)) break;
+        if (t_iter >= 2 && !mbar_wait_sleep(&d_empty[ai], ((t_iter >> 1) & 1) ^ 1)) break;
         tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % kMoeStages, b = it % kMoeABufs;
-          if (!mbar_wait(&full_bar[s], (it / kMoeStages) & 1)) { ok = false; break; }
-          if (!mbar_wait(&a_full[b], (it / kMoeABufs) & 1)) { ok = false; break; }
+          if (!mbar_wait_sleep(&full_bar[s], (it / kMoeStages) & 1)) { ok = false; break; }
+          if (!mbar_wait_sleep(&a_full[b], (it / kMoeABufs) & 1)) { ok = false; break; }
           fence_proxy_async();  // the gathered rows (cp.async writes), to the tensor core's proxy
           tc_fence_after();
           const uint32_t ab = smem_u32(abuf + (size_t)b * kMxABufBytes);
@@ -215,12 +215,12 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
       const int nt = tile / nblk, mb = tile - nt * nblk;
       const bool row_ok = nt * kMxBN + r < a.N && expert_of(mb) >= 0;
       const int mi = t_iter & 1;
-      if (ok && !mbar_wait(&meta_full[mi], (t_iter >> 1) & 1)) ok = false;
+      if (ok && !mbar_wait_sleep(&meta_full[mi], (t_iter >> 1) & 1)) ok = false;
       const uint8_t* mt = meta + (size_t)mi * meta_bytes;
       for (int kb = 0; kb < nkb; ++kb, ++it) {
         const int s = it % kMoeStages, b = it % kMoeABufs;
-        if (ok && !mbar_wait(&full_bar[s], (it / kMoeStages) & 1)) ok = false;
-        if (ok && it >= kMoeABufs && !mbar_wait(&a_empty[b], ((it / kMoeABufs) & 1) ^ 1)) ok = false;
+        if (ok && !mbar_wait_sleep(&full_bar[s], (it / kMoeStages) & 1)) ok = false;
+        if (ok && it >= kMoeABufs && !mbar_wait_sleep(&a_empty[b], ((it / kMoeABufs) & 1) ^ 1)) ok = false;
         tc_fence_after();
         const uint8_t* st = ring + (size_t)s * MoeStage::kBytes;
         uint8_t* ab = abuf + (size_t)b * kMxABufBytes;
@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
       const int nt = tile / nblk, mb = tile - nt * nblk;
       const int rows = min(kMxBN, a.N - nt * kMxBN);
       const int ai = t_iter & 1;
-      if (ok && !mbar_wait(&d_full[ai], (t_iter >> 1) & 1)) ok = false;
+      if (ok && !mbar_wait_sleep(&d_full[ai], (t_iter >> 1) & 1)) ok = false;
       tc_fence_after();
 #pragma unroll 1
       for (int j = 0; j < kMoeBM / 32; ++j) {
@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(kMoeThreads, 1) gemm_moe_lut3_mx_kernel(const 
       const int nb = valid ? 16 : 0;
       for (int kb = 0; kb < nkb; ++kb, ++it) {
         const int s = it % kMoeStages;
-        if (lane == 0 && it >= kMoeStages && !mbar_wait(&empty_bar[s], ((it / kMoeStages) & 1) ^ 1)) ok = false;
+        if (lane == 0 && it >= kMoeStages && !mbar_wait_sleep(&empty_bar[s], ((it / kMoeStages) & 1) ^ 1)) ok = false;
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         if (!ok) break;
         const uint32_t st = smem_u32(ring + (size_t)s * MoeStage::kBytes);
