@@ -552,6 +552,20 @@ def _secondary_measurements(torch, lbq, workloads, device, peaks, quick):
             out["c5_lut3_m4_skinny_kernel"] = {"us": ms4s * 1e3, "GBps": b / ms4s / 1e6,
                                                "frac_hbm": b / ms4s / 1e6 / hbm}
             del X4, ws4
+            # batch 16: two blocks of 8 rows on the batch kernel's columns
+            X16 = workloads.activations_device(5, 16, K, "bf16", device)
+            ws16 = lbq.workspace(2, 16, K, N, 0, "lut3")
+            ms16 = rotating_lut3_ms(torch, lbq, images, X16, N, ws16, reps=3)
+            out["c5_lut3_m16"] = {"us": ms16 * 1e3, "GBps": b / ms16 / 1e6, "frac_hbm": b / ms16 / 1e6 / hbm,
+                                  "kernel": "lut3_tmma_batch_kernel"}
+            lbq.lbq_debug_lut3_batch_off(1)
+            try:
+                ms16s = rotating_lut3_ms(torch, lbq, images, X16, N, ws16, reps=3)
+            finally:
+                lbq.lbq_debug_lut3_batch_off(0)
+            out["c5_lut3_m16_skinny_kernel"] = {"us": ms16s * 1e3, "GBps": b / ms16s / 1e6,
+                                                "frac_hbm": b / ms16s / 1e6 / hbm}
+            del X16, ws16
         else:
             tf = 2.0 * M * K * N / ms / 1e9
             out[f"c5_lut3_m{M}"] = {"us": ms * 1e3, "TFLOPs": tf, "frac_bf16_peak": tf / tc_peak,

@@ -1087,13 +1087,15 @@ static lbq_status run_lut3_tmma(const void* X, const void* image, const Layout& 
 static int g_l3b_off = 0;  // test hook: 1 = M = 2..8 on the skinny kernel instead
 
 struct L3bPlan {
-  int kj, nw, grid, stage_bytes, t_off, stages, xs_off, red_off, smem;
+  int kj, nb, nw, grid, stage_bytes, t_off, stages, xs_off, red_off, smem;
 };
 
 static L3bPlan plan_lut3_batch(int M, int K, int N) {
   L3bPlan p{};
   const int KT = K / 64;
-  if (M < 2 || M > kL3bMaxM || KT > 8 * kL3tMaxWarps || (size_t)M * K * 2 > 64 * 1024) return p;
+  // X staged whole: up to 64 KB for 8 rows, 128 KB for 16 (K <= 4096)
+  p.nb = M > 8 ? 2 : 1;
+  if (M < 2 || M > kL3bMaxM || KT > 8 * kL3tMaxWarps || (size_t)M * K * 2 > (size_t)p.nb * 64 * 1024) return L3bPlan{};
   p.nw = std::min(kL3tMaxWarps, KT);
   const int kj = (KT + p.nw - 1) / p.nw;
   p.kj = kj <= 2 ? 2 : kj <= 4 ? 4 : 8;
@@ -1103,7 +1105,7 @@ static L3bPlan plan_lut3_batch(int M, int K, int N) {
   p.t_off = (int)align_up((size_t)KT * 384, 128);
   p.stage_bytes = p.t_off + (int)align_up((size_t)KT * 32, 128);
   const int x_bytes = (int)align_up((size_t)M * K * 2, 128);
-  const int red_bytes = 2 * p.nw * 128 * (int)sizeof(float);
+  const int red_bytes = 2 * p.nw * 128 * p.nb * (int)sizeof(float);
   const int avail = max_dynamic_smem() - 2 * kL3tMaxStages * 8 - 1024 - x_bytes - red_bytes;
   const int want = g_l3t_stages ? g_l3t_stages : g_l3t_default_stages;
   p.stages = std::min(std::min(std::min(max_units, want), kL3tMaxStages), avail / p.stage_bytes);
@@ -1145,8 +1147,13 @@ static lbq_status run_lut3_batch(const void* X, int M, const void* image, const 
   a.xs_off = p.xs_off; a.red_off = p.red_off;
   a.y_bf16 = ybf16 ? 1 : 0;
   a.debug_drop = g_debug_drop;
-  const void* fn = p.kj == 2 ? (const void*)lut3_tmma_batch_kernel<2>
-                 : p.kj == 4 ? (const void*)lut3_tmma_batch_kernel<4> : (const void*)lut3_tmma_batch_kernel<8>;
+  const void* fn;
+  if (p.nb == 1)
+    fn = p.kj == 2 ? (const void*)lut3_tmma_batch_kernel<2, 1>
+       : p.kj == 4 ? (const void*)lut3_tmma_batch_kernel<4, 1> : (const void*)lut3_tmma_batch_kernel<8, 1>;
+  else
+    fn = p.kj == 2 ? (const void*)lut3_tmma_batch_kernel<2, 2>
+       : p.kj == 4 ? (const void*)lut3_tmma_batch_kernel<4, 2> : (const void*)lut3_tmma_batch_kernel<8, 2>;
   const int block = (p.nw + 1) * 32;
   occupancy_for(fn, block, p.smem);  // raises the kernel's dynamic shared-memory limit once
   void* args[] = {&mi, &mt, &a};

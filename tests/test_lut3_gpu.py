@@ -106,7 +106,7 @@ SKINNY_SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16])
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 12, 16])
 @pytest.mark.parametrize("K,N", SKINNY_SHAPES)
 # 0: library's choice (the TMA-fed warp-MMA kernel at M = 1 for K <= 8192),
 # 2: the skinny warp-MMA kernel
@@ -263,7 +263,8 @@ def test_lut3_m1_kernels(torch, lbq, K, N, path, stages):
     lbq.device_status()
 
 
-@pytest.mark.parametrize("M", [1, 4])  # the batch-1 kernel; the batch kernel (16-row units, batch on the columns)
+# the batch-1 kernel; the batch kernel (16-row units, batch on the columns) with one and two blocks of 8 rows
+@pytest.mark.parametrize("M", [1, 4, 16])
 def test_lut3_m1_bounded_wait_runs_out_and_is_reported(torch, lbq, M):
     """Failure detection without a GPU fault on the TMA-fed LUT3 kernels: with
     the producer's copies withheld (test hook) on a one-CTA launch, every
@@ -310,7 +311,7 @@ def test_tables_exact_at_the_exponent_range_ends(torch, lbq):
     lbq.device_status()
 
 
-@pytest.mark.parametrize("M", [1, 4])  # the batch-1 kernel; the batch kernel
+@pytest.mark.parametrize("M", [1, 4, 16])  # the batch-1 kernel; the batch kernel (one and two row blocks)
 def test_lut3_m1_pdl_graph(torch, lbq, M):
     """The TMA-fed LUT3 kernels with programmatic dependent launch inside a
     CUDA graph: three back-to-back launches, each reading the previous one's
@@ -349,10 +350,11 @@ def test_lut3_m1_pdl_graph(torch, lbq, M):
 
 
 @pytest.mark.parametrize("off", [0, 1])  # the TMA-fed batch kernel; the skinny kernel
-def test_lut3_batch_full_size_sampled(torch, lbq, off):
-    """The 3-bit LUT workload at batch 4 (K=4096, N=14336), sampled channel
-    groups, on the batch kernel and on the skinny kernel."""
-    K, N, M = 4096, 14336, 4
+@pytest.mark.parametrize("M", [4, 16])
+def test_lut3_batch_full_size_sampled(torch, lbq, off, M):
+    """The 3-bit LUT workload at batches 4 and 16 (K=4096, N=14336), sampled
+    channel groups, on the batch kernel and on the skinny kernel."""
+    K, N = 4096, 14336
     idx, cb, ex = workloads.lut3_host(5, K, N)
     img = _image(torch, lbq, idx, cb, ex)
     X = workloads.activations_host(344, M, K, "bf16")
