@@ -19,6 +19,6 @@ from .binding import (  # noqa: F401
     lbq_unpack_lut3_canonical, lbq_version, lbq_workspace_size, lbq_quantize_mxfp8, lbq_lut3_mx_gemm,
     affine_gemv, pack_affine, unpack_affine_canonical, lbq_affine_gemv, lbq_affine_packed_size, lbq_pack_affine,
     lbq_unpack_affine_canonical, quantize_int8, w4a8_gemv, lbq_quantize_int8, lbq_w4a8_gemv,
-    w4a8_gemv_grouped, lbq_w4a8_gemv_grouped, lbq_debug_w4a8_tiled, lbq_debug_lut3_stages, lbq_debug_lut3_batch_off, lbq_debug_gemm_stream_k, lbq_debug_gemm_hold, lbq_debug_gemm_schedule, make_w4a8_items,
+    w4a8_gemv_grouped, lbq_w4a8_gemv_grouped, lbq_debug_w4a8_tiled, lbq_debug_lut3_stages, lbq_debug_lut3_batch_off, lbq_debug_gemm_stream_k, lbq_debug_gemm_hold, lbq_debug_gemm_schedule, lbq_debug_tile_coords, make_w4a8_items,
     MOE_BLOCK, moe_align, moe_lut3_mx_gemm, pack_lut3_experts, lbq_moe_align, lbq_moe_lut3_mx_gemm, lbq_moe_max_padded,
 )

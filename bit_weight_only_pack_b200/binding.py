@@ -83,6 +83,7 @@ _SIGS = {
     "lbq_debug_lut3_batch_off": ([_c_int], None),
     "lbq_debug_gemm_stream_k": ([_c_int], None),
     "lbq_debug_gemm_hold": ([_c_int], None),
+    "lbq_debug_tile_coords": ([_c_int, _c_int, _c_int, ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)], None),
     "lbq_debug_gemm_schedule": ([_c_int, _c_int, _c_int, _c_int, _c_int, ctypes.POINTER(_c_int),
                                  ctypes.POINTER(_c_int), ctypes.POINTER(_c_int), _c_int], _c_int),
     "lbq_moe_max_padded": ([_c_int, _c_int, _c_int, ctypes.POINTER(_c_int)], _c_int),
@@ -298,6 +299,13 @@ def lbq_debug_gemm_schedule(M, K, N, stream_k, cta):
     buf = (_c_int * max(4 * n, 4))()
     _lib.lbq_debug_gemm_schedule(M, K, N, 1 if stream_k else 0, cta, ctypes.byref(grid), ctypes.byref(nkb), buf, n)
     return grid.value, nkb.value, [tuple(buf[4 * i:4 * i + 4]) for i in range(n)]
+
+
+def lbq_debug_tile_coords(tile, n_tiles, m_tiles):
+    """Test hook: (channel tile, token tile) of a prefill tile index in the kernel's banded order."""
+    nt, mt = _c_int(0), _c_int(0)
+    _lib.lbq_debug_tile_coords(tile, n_tiles, m_tiles, ctypes.byref(nt), ctypes.byref(mt))
+    return nt.value, mt.value
 
 
 def lbq_moe_max_padded(num_pairs, num_experts, block):

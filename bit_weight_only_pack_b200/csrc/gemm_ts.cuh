@@ -130,7 +130,8 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
       SkSched sch(a.sk.dp_tiles, a.sk.sk_items, a.k_blocks, (int)blockIdx.x, (int)gridDim.x);
       SkItem w;
       while (ok && sch.next(w)) {
-        const int nt = w.tile / a.m_tiles, mt = w.tile - nt * a.m_tiles;  // token tiles inner: codes reused from L2
+        int nt, mt;  // banded order: codes reused from L2 across a band's token tiles
+        sk_tile_coords(w.tile, a.n_tiles, a.m_tiles, nt, mt);
         const int rows = min(kTsBN, a.N - nt * kTsBN);
         for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const int s = it % kTsStages;
@@ -202,7 +203,8 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
     SkSched sch(a.sk.dp_tiles, a.sk.sk_items, a.k_blocks, (int)blockIdx.x, (int)gridDim.x);
     SkItem w;
     while (sch.next(w)) {
-      const int nt = w.tile / a.m_tiles;
+      int nt, mt_unused;
+      sk_tile_coords(w.tile, a.n_tiles, a.m_tiles, nt, mt_unused);
       const bool row_ok = nt * kTsBN + r < a.N;
       for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
         const int s = it % kTsStages, b = it % kTsABufs;
@@ -281,7 +283,8 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(const __grid_con
     SkSched sch(a.sk.dp_tiles, a.sk.sk_items, a.k_blocks, (int)blockIdx.x, (int)gridDim.x);
     SkItem w;
     for (; sch.next(w); ++t_iter) {
-      const int nt = w.tile / a.m_tiles, mt = w.tile - nt * a.m_tiles;
+      int nt, mt;
+      sk_tile_coords(w.tile, a.n_tiles, a.m_tiles, nt, mt);
       if (ok && !mbar_wait_sleep(&d_full, t_iter & 1)) ok = false;
       tc_fence_after();
       // an earlier part: wait for the later part's sums in slot blockIdx.x + 1

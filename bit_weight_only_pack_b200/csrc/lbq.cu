@@ -1528,6 +1528,12 @@ int lbq_debug_gemm_schedule(int M, int K, int N, int stream_k, int cta, int* gri
   return n;
 }
 
+// Test hook (not in the public header): the (channel tile, token tile) of a
+// prefill tile index in the banded order the kernel uses.
+void lbq_debug_tile_coords(int tile, int n_tiles, int m_tiles, int* nt, int* mt) {
+  sk_tile_coords(tile, n_tiles, m_tiles, *nt, *mt);
+}
+
 lbq_status lbq_set_option(int option, int value) {
   if (option == LBQ_OPT_PDL) {
     g_pdl = value ? 1 : 0;

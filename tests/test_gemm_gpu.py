@@ -31,6 +31,7 @@ GEMM_SHAPES = [
     (256, 4096, 512, 128, "asym", "bf16"),     # the prefill K, two N tiles
     (130, 96, 36, 32, "asym", "f16"),          # K < one k-block, N % 8 != 0
     (384, 2048, 768, 32, "sym", "bf16"),
+    (2500, 256, 520, 128, "asym", "bf16"),    # 10 token tiles: a full band of 8 and a ragged band of 2
 ]
 
 

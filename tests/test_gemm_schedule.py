@@ -99,3 +99,18 @@ def test_whole_tile_schedule_is_the_strided_order():
     for c, items in enumerate(per_cta):
         assert [t for (t, _, _, _) in items] == list(range(c, 896, grid))
         assert all((kb0, kb1, p) == (0, nkb, 0) for (_, kb0, kb1, p) in items)
+
+
+@pytest.mark.parametrize("n_tiles,m_tiles", [(112, 32), (112, 8), (112, 2), (33, 5), (7, 13), (10, 16), (112, 9), (1, 1)])
+def test_banded_tile_order_is_a_bijection(n_tiles, m_tiles):
+    """The kernel's tile order: bands of 8 token tiles, channel tiles outer
+    inside a band; every (channel tile, token tile) once, a partial last band
+    included, and the plain token-inner order when there are at most 8 token
+    tiles."""
+    import bit_weight_only_pack_b200 as lbq
+    got = [lbq.lbq_debug_tile_coords(t, n_tiles, m_tiles) for t in range(n_tiles * m_tiles)]
+    assert sorted(got) == [(a, b) for a in range(n_tiles) for b in range(m_tiles)]
+    if m_tiles <= 8:
+        assert got == [(t // m_tiles, t % m_tiles) for t in range(n_tiles * m_tiles)]
+    else:  # the first band: 8 token tiles of channel tile 0, then of channel tile 1, ...
+        assert got[:16] == [(0, b) for b in range(8)] + [(1, b) for b in range(8)]

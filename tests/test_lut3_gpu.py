@@ -124,7 +124,7 @@ def test_lut3_gemv_parity(torch, lbq, M, K, N, path):
     lbq.device_status()
 
 
-@pytest.mark.parametrize("M", [17, 130, 300])
+@pytest.mark.parametrize("M", [17, 130, 300, 2500])  # 2500: a band of 8 token tiles and a ragged band of 2
 @pytest.mark.parametrize("K,N", [(1024, 512), (320, 264), (4096, 1032)])
 @pytest.mark.parametrize("path", [0, 1])  # 0: weights in tensor memory, 1: weights in shared memory
 def test_lut3_gemm_parity(torch, lbq, M, K, N, path):
