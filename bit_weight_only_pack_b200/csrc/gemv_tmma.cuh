@@ -49,6 +49,7 @@ namespace lbq {
 constexpr int kTmMaxItems = 4;
 constexpr int kTmMaxSlices = 16;  // 256-k slices per K-range = consumer warps
 constexpr int kTmMaxStages = 16;
+constexpr int kTmDefaultStages = 3;  // the planner's ring depth (at most kTmMaxStages)
 constexpr int kTmRows = 16;
 constexpr int kTmSliceBytes = kTmRows * 128;  // one TMA box: 16 rows x 128 bytes of codes
 

@@ -652,7 +652,10 @@ static TmPlan plan_tmma(int K, const int* Ns, int count, int group, bool asym, b
   p.max_units = (p.row_tiles + cpk - 1) / cpk;
   const int avail = max_dynamic_smem() - 2 * kTmMaxStages * 8 - 1024;
   const int red_bytes = p.max_units * p.nsl * 16 * 4 + p.max_units * 4;
-  int S = kTmMaxStages;
+  // a short ring: the decode step (K=4096 launches, one CTA per SM) measured
+  // 1071.5 us per step with at most three stages against 1077.3 with as many
+  // as fit; copies in flight together land together and delay the decode
+  int S = kTmDefaultStages;
   while (S >= 2 && S * p.stage_bytes + red_bytes > avail) --S;
   p.stages = S;
   p.smem = 1024 + S * p.stage_bytes + red_bytes;
