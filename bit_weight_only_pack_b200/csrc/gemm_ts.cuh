@@ -31,8 +31,9 @@
 //               the round trips, the less of each tile the converters (which
 //               run at most three k-blocks ahead of the stalled MMAs) lose.
 //
-// Schedule: whole tiles strided over the grid, or stream-K over the last two
-// waves when the tail wave leaves SMs idle (stream_k.cuh).
+// Schedule: whole tiles strided over the grid in banded order (bands of 8
+// token tiles), or stream-K over the last two waves when the tail wave leaves
+// SMs idle (stream_k.cuh).
 #pragma once
 
 #include "common.cuh"
