@@ -1025,7 +1025,9 @@ struct L3tPlan {
 };
 
 static int g_l3t_stages = 0;  // test hook: ring stages of the LUT3 TMA GEMV (0 = the plan's choice)
-static int g_l3t_default_stages = 4;
+// three stages (measured on B200, K=4096 N=14336 with programmatic dependent
+// launch: 10.55 us against 10.67 with four, 10.95 with six, 12.4 with two)
+static int g_l3t_default_stages = 3;
 
 static L3tPlan plan_lut3_tmma(int K, int N) {
   L3tPlan p{};
